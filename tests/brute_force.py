@@ -1,0 +1,106 @@
+"""Brute-force OneTrans block stack in pure Python (test-only second implementation).
+
+An independent restatement used to pin the C oracle on tiny inputs: every
+candidate's tokens are one Python list of Token records, each token looks up
+its own parameter set (S shared / NS private by position), and visibility is
+decided token pair by token pair from the mask rule of the OneTrans summary
+page (an S-token sees earlier S-tokens and itself; an NS-token sees every
+S-token and the preceding NS-tokens of its candidate, and itself).  Plain
+floats and the math module only; no numpy arithmetic, no shared code with the
+C oracle.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+
+@dataclass
+class Token:
+    kind: str        # "S" or "NS"
+    index: int       # S: position in the S stream; NS: position n
+    x: list
+
+
+def _rms(x, g, eps):
+    ms = sum(v * v for v in x) / len(x)
+    inv = 1.0 / math.sqrt(ms + eps)
+    return [v * inv * gg for v, gg in zip(x, g)]
+
+
+def _mv(W, x):
+    """W given as list of output rows (out x in)."""
+    return [sum(wk * xk for wk, xk in zip(row, x)) for row in W]
+
+
+def _gelu(z):
+    return 0.5 * z * (1.0 + math.erf(z / math.sqrt(2.0)))
+
+
+def _visible(qt: Token, kt: Token) -> bool:
+    if qt.kind == "S":
+        return kt.kind == "S" and kt.index <= qt.index
+    return kt.kind == "S" or kt.index <= qt.index
+
+
+def _params(w, l, tok: Token):
+    """Nested lists for the token's parameter set at layer l."""
+    if tok.kind == "S":
+        return (w["Wqkv_s"][l], w["Wo_s"][l], w["W1_s"][l], w["W2_s"][l], w["g1_s"][l],
+                w["g2_s"][l])
+    n = tok.index
+    return (w["Wqkv_ns"][l][n], w["Wo_ns"][l][n], w["W1_ns"][l][n], w["W2_ns"][l][n],
+            w["g1_ns"][l][n], w["g2_ns"][l][n])
+
+
+def run_candidate(w, S_rows, ns_rows, q_sched, heads, eps):
+    """One candidate: S_rows [L0][d], ns_rows [N][d] (lists).
+
+    Returns (S tail rows after the last layer, NS rows, per-layer (K, V) of
+    the S tokens).  ``w`` holds nested Python lists.
+    """
+    d = len(S_rows[0])
+    hd = d // heads
+    seq = [Token("S", i, list(r)) for i, r in enumerate(S_rows)]
+    seq += [Token("NS", n, list(r)) for n, r in enumerate(ns_rows)]
+    kv_layers = []
+    for l, q in enumerate(q_sched):
+        n_s = sum(1 for t in seq if t.kind == "S")
+        proj = []
+        for t in seq:
+            Wqkv, _, _, _, g1, _ = _params(w, l, t)
+            qkv = _mv(Wqkv, _rms(t.x, g1, eps))
+            proj.append((qkv[:d], qkv[d:2 * d], qkv[2 * d:]))
+        kv_layers.append(([p[1] for t, p in zip(seq, proj) if t.kind == "S"],
+                          [p[2] for t, p in zip(seq, proj) if t.kind == "S"]))
+        new_seq = []
+        for i, t in enumerate(seq):
+            if t.kind == "S" and t.index < n_s - q:
+                continue  # not in this layer's query tail
+            a = []
+            for h in range(heads):
+                qv = proj[i][0][h * hd:(h + 1) * hd]
+                scores, vals = [], []
+                for j, kt in enumerate(seq):
+                    if not _visible(t, kt):
+                        continue
+                    kvec = proj[j][1][h * hd:(h + 1) * hd]
+                    scores.append(sum(a_ * b_ for a_, b_ in zip(qv, kvec)) / math.sqrt(hd))
+                    vals.append(proj[j][2][h * hd:(h + 1) * hd])
+                m = max(scores)
+                e = [math.exp(s - m) for s in scores]
+                z = sum(e)
+                a += [sum(e[k] / z * vals[k][c] for k in range(len(e))) for c in range(hd)]
+            _, Wo, W1, W2, _, g2 = _params(w, l, t)
+            hrow = [xv + ov for xv, ov in zip(t.x, _mv(Wo, a))]
+            f = [_gelu(v) for v in _mv(W1, _rms(hrow, g2, eps))]
+            y = [hv + fv for hv, fv in zip(hrow, _mv(W2, f))]
+            new_seq.append(Token(t.kind, t.index, y))
+        # re-index the S tail 0..q-1 so the next layer's S stream starts at 0
+        s_tail = [t for t in new_seq if t.kind == "S"]
+        for k, t in enumerate(s_tail):
+            t.index = k
+        seq = new_seq
+    return ([t.x for t in seq if t.kind == "S"], [t.x for t in seq if t.kind == "NS"],
+            kv_layers)

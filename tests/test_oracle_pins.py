@@ -1,0 +1,341 @@
+"""Pins of the CPU oracle to things other than itself (no GPU needed).
+
+* brute force: an independent pure-Python token-by-token implementation;
+* textbook reduction: with every NS parameter set equal to the S set the S/NS
+  mask is the plain causal mask over [S; NS], so each block must equal a
+  pre-norm causal Transformer layer built from torch's library routines
+  (scaled_dot_product_attention(is_causal=True), rms_norm, gelu) in fp64;
+* closed forms: uniform attention, identity blocks, single-key attention,
+  RMSNorm scale invariance;
+* the invariants the pages' design rests on: causality, pyramid
+  consistency, KV-cache equivalence, candidate independence, S-side
+  independence from NS input;
+* e4m3 rounding against torch's float8_e4m3fn cast;
+* Auto-Split and embedding gather against numpy.
+"""
+
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as Fnn
+
+from brute_force import run_candidate
+from helpers import rand_inputs, rand_weights, to_lists
+from oracle import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def cfg_of(layers, d, heads, ffn, N, L0, q, eps=1e-6, fp8=False):
+    return O.Config(layers, d, heads, ffn, N, L0, list(q), eps, fp8)
+
+
+TINY_CASES = [
+    # layers, d, heads, ffn, N, L0, q schedule, U, C
+    (1, 8, 1, 16, 1, 1, [1], 1, 1),
+    (1, 8, 2, 12, 3, 2, [2], 1, 2),
+    (2, 8, 2, 16, 3, 7, [5, 2], 2, 2),
+    (3, 12, 2, 20, 1, 33, [33, 9, 1], 1, 2),
+    (2, 16, 1, 32, 3, 33, [7, 7], 1, 1),
+]
+
+
+@pytest.mark.parametrize("case", TINY_CASES)
+def test_brute_force_matches_oracle(case):
+    layers, d, H, f, N, L0, q, U, Cn = case
+    w = rand_weights(layers, d, f, N, seed=L0 + d)
+    S, ns = rand_inputs(U, Cn, L0, N, d, seed=7 * L0 + N)
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    kv, s_out = O.encode_user(cfg, w, S)
+    ns_out = O.score_candidates(cfg, w, kv, ns)
+    js, jkv, jns = O.full_forward_joint(cfg, w, S, ns)
+    wl = to_lists(w)
+    for u in range(U):
+        for c in range(Cn):
+            bs, bns, bkv = run_candidate(wl, S[u].double().tolist(), ns[u, c].double().tolist(),
+                                         q, H, 1e-6)
+            np.testing.assert_allclose(s_out[u], np.array(bs), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(js[u, c], np.array(bs), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(ns_out[u, c], np.array(bns), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(jns[u, c], np.array(bns), rtol=0, atol=1e-12)
+            for l, (K, V) in enumerate(bkv):
+                Ko, Vo = O.kv_layer(cfg, kv[u], l)
+                np.testing.assert_allclose(Ko, np.array(K), rtol=0, atol=1e-12)
+                np.testing.assert_allclose(Vo, np.array(V), rtol=0, atol=1e-12)
+
+
+def _torch_causal_layer(x, Wqkv, Wo, W1, W2, g1, g2, H, eps):
+    """Pre-norm causal Transformer layer from torch library routines (fp64)."""
+    T, d = x.shape
+    hd = d // H
+    xn = Fnn.rms_norm(x, (d,), weight=g1, eps=eps)
+    qkv = xn @ Wqkv.T
+    q, k, v = qkv.split(d, dim=-1)
+    heads = lambda t: t.view(T, H, hd).transpose(0, 1)  # noqa: E731
+    a = Fnn.scaled_dot_product_attention(heads(q), heads(k), heads(v), is_causal=True)
+    h = x + a.transpose(0, 1).reshape(T, d) @ Wo.T
+    return h + Fnn.gelu(Fnn.rms_norm(h, (d,), weight=g2, eps=eps) @ W1.T) @ W2.T
+
+
+@pytest.mark.parametrize("pyramid", [False, True])
+def test_textbook_reduction_causal_transformer(pyramid):
+    layers, d, H, f, N, L0 = 2, 16, 2, 32, 3, 11
+    q = [7, 3] if pyramid else [L0, L0]
+    w = rand_weights(layers, d, f, N, seed=3, dtype=torch.float64)
+    for name in ("Wqkv", "Wo", "W1", "W2", "g1", "g2"):
+        w[name + "_ns"] = w[name + "_s"][:, None].expand(-1, N, *w[name + "_s"].shape[1:]).clone()
+    S, ns = rand_inputs(1, 2, L0, N, d, seed=5, dtype=torch.float64)
+    # float32-representable inputs: the oracle stores inputs as float32
+    w = {k: v.float().double() for k, v in w.items()}
+    S, ns = S.float().double(), ns.float().double()
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    kv, s_out = O.encode_user(cfg, w, S)
+    ns_out = O.score_candidates(cfg, w, kv, ns)
+    for c in range(2):
+        x = torch.cat([S[0], ns[0, c]])
+        L = L0
+        for l in range(layers):
+            y = _torch_causal_layer(x, w["Wqkv_s"][l], w["Wo_s"][l], w["W1_s"][l], w["W2_s"][l],
+                                    w["g1_s"][l], w["g2_s"][l], H, 1e-6)
+            # bottom-right alignment: keep the last q S rows, then all NS rows
+            x = torch.cat([y[L - q[l]:L], y[L:]])
+            L = q[l]
+        np.testing.assert_allclose(s_out[0], x[:L].numpy(), rtol=0, atol=1e-11)
+        np.testing.assert_allclose(ns_out[0, c], x[L:].numpy(), rtol=0, atol=1e-11)
+
+
+def _zero_rows(w, key, rows):
+    w[key] = w[key].clone()
+    w[key][..., rows, :] = 0
+
+
+def test_closed_form_uniform_attention_means():
+    """W_Q = W_K = 0: every score is 0, so attention is the mean of the visible
+    V rows.  With W_O = I and W_2 = 0 each output row is x + that mean."""
+    layers, d, H, f, N, L0 = 1, 8, 2, 16, 3, 9
+    w = rand_weights(layers, d, f, N, seed=11)
+    for key in ("Wqkv_s", "Wqkv_ns"):
+        _zero_rows(w, key, slice(0, 2 * d))
+    w["Wo_s"] = torch.eye(d).expand(layers, d, d).clone()
+    w["Wo_ns"] = torch.eye(d).expand(layers, N, d, d).clone()
+    w["W2_s"] = torch.zeros_like(w["W2_s"])
+    w["W2_ns"] = torch.zeros_like(w["W2_ns"])
+    S, ns = rand_inputs(1, 1, L0, N, d, seed=12)
+    cfg = cfg_of(layers, d, H, f, N, L0, [L0])
+    kv, s_out = O.encode_user(cfg, w, S)
+    ns_out = O.score_candidates(cfg, w, kv, ns)
+    K, V = O.kv_layer(cfg, kv[0], 0)
+    assert np.all(K == 0.0)
+    Sd = S[0].double().numpy()
+    for t in range(L0):
+        np.testing.assert_allclose(s_out[0, t], Sd[t] + V[: t + 1].mean(0), atol=1e-13)
+    # NS: V_N rows from the private V projection of the normalised NS rows
+    x = ns[0, 0].double().numpy()
+    VN = []
+    for n in range(N):
+        xn = x[n] / np.sqrt((x[n] ** 2).mean() + 1e-6) * w["g1_ns"][0, n].double().numpy()
+        VN.append(w["Wqkv_ns"][0, n, 2 * d:].double().numpy() @ xn)
+    VN = np.array(VN)
+    for n in range(N):
+        mean = (V.sum(0) + VN[: n + 1].sum(0)) / (L0 + n + 1)
+        np.testing.assert_allclose(ns_out[0, 0, n], x[n] + mean, atol=1e-13)
+
+
+def test_closed_form_identity_blocks_pyramid():
+    """W_O = W_2 = 0: every block is the identity on the rows it keeps, so the
+    stack returns input rows L0-q_last .. L0-1 exactly and the NS rows
+    unchanged."""
+    layers, d, H, f, N, L0 = 3, 8, 2, 16, 2, 20
+    q = [14, 6, 4]
+    w = rand_weights(layers, d, f, N, seed=21)
+    for k in ("Wo_s", "Wo_ns", "W2_s", "W2_ns"):
+        w[k] = torch.zeros_like(w[k])
+    S, ns = rand_inputs(2, 3, L0, N, d, seed=22)
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    kv, s_out = O.encode_user(cfg, w, S)
+    ns_out = O.score_candidates(cfg, w, kv, ns)
+    assert np.array_equal(s_out, S[:, L0 - q[-1]:].double().numpy())
+    assert np.array_equal(ns_out, ns.double().numpy())
+
+
+def test_closed_form_first_query_returns_v0():
+    """An S query at t = 0 sees only key 0: its attention output is v_0."""
+    layers, d, H, f, N, L0 = 1, 8, 2, 16, 1, 5
+    w = rand_weights(layers, d, f, N, seed=31)
+    w["Wo_s"] = torch.eye(d).expand(layers, d, d).clone()
+    w["W2_s"] = torch.zeros_like(w["W2_s"])
+    S, ns = rand_inputs(1, 1, L0, N, d, seed=32)
+    cfg = cfg_of(layers, d, H, f, N, L0, [L0])
+    kv, s_out = O.encode_user(cfg, w, S)
+    K, V = O.kv_layer(cfg, kv[0], 0)
+    np.testing.assert_allclose(s_out[0, 0], S[0, 0].double().numpy() + V[0], atol=1e-14)
+
+
+def test_closed_form_rmsnorm_scale_invariance():
+    """K/V of layer 0 are projections of RMSNorm(x), which ignores a positive
+    scale of x up to eps."""
+    layers, d, H, f, N, L0 = 1, 16, 2, 32, 1, 6
+    w = rand_weights(layers, d, f, N, seed=41)
+    S, _ = rand_inputs(1, 1, L0, N, d, seed=42)
+    cfg = cfg_of(layers, d, H, f, N, L0, [L0], eps=1e-30)
+    kv1, _ = O.encode_user(cfg, w, S)
+    kv2, _ = O.encode_user(cfg, w, S * 4.0)
+    np.testing.assert_allclose(kv1, kv2, rtol=1e-13, atol=1e-14)
+
+
+def _small():
+    layers, d, H, f, N, L0 = 2, 16, 2, 32, 3, 13
+    return layers, d, H, f, N, L0, [9, 4]
+
+
+def test_invariant_causal():
+    """Perturbing S row j leaves S K/V rows < j of layer 0 and the S outputs
+    of rows < j (no pyramid) unchanged; rows >= j do change."""
+    layers, d, H, f, N, L0, _ = _small()
+    q = [L0, L0]
+    w = rand_weights(layers, d, f, N, seed=51)
+    S, _ = rand_inputs(1, 1, L0, N, d, seed=52)
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    kv, s_out = O.encode_user(cfg, w, S)
+    j = 6
+    S2 = S.clone()
+    S2[0, j] += 1.0
+    kv2, s_out2 = O.encode_user(cfg, w, S2)
+    assert np.array_equal(s_out[0, :j], s_out2[0, :j])
+    assert not np.allclose(s_out[0, j:], s_out2[0, j:])
+    for l in range(layers):
+        K1, V1 = O.kv_layer(cfg, kv[0], l)
+        K2, V2 = O.kv_layer(cfg, kv2[0], l)
+        assert np.array_equal(K1[:j], K2[:j]) and np.array_equal(V1[:j], V2[:j])
+
+
+def test_invariant_pyramid_consistency():
+    """A layer with query tail q equals the matching rows of the same layer
+    with every row as a query, on the same input."""
+    layers, d, H, f, N, L0, _ = _small()
+    w = rand_weights(1, d, f, N, seed=61)
+    S, ns = rand_inputs(1, 2, L0, N, d, seed=62)
+    full = cfg_of(1, d, H, f, N, L0, [L0])
+    kvf, sf = O.encode_user(full, w, S)
+    nsf = O.score_candidates(full, w, kvf, ns)
+    for q in (1, 5, L0 - 1):
+        part = cfg_of(1, d, H, f, N, L0, [q])
+        kvp, sp = O.encode_user(part, w, S)
+        nsp = O.score_candidates(part, w, kvp, ns)
+        assert np.array_equal(sp[0], sf[0, L0 - q:])
+        assert np.array_equal(kvp, kvf)
+        assert np.array_equal(nsp, nsf)
+
+
+def test_invariant_kv_cache_equivalence_and_s_independence():
+    """Encode-once + score-per-candidate equals the no-cache joint run of each
+    candidate; the joint run's S outputs and K/V are the same for every
+    candidate (S never sees NS)."""
+    layers, d, H, f, N, L0, q = _small()
+    w = rand_weights(layers, d, f, N, seed=71)
+    S, ns = rand_inputs(2, 3, L0, N, d, seed=72)
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    kv, s_out = O.encode_user(cfg, w, S)
+    ns_out = O.score_candidates(cfg, w, kv, ns)
+    js, jkv, jns = O.full_forward_joint(cfg, w, S, ns)
+    np.testing.assert_allclose(jns, ns_out, rtol=0, atol=1e-12)
+    for c in range(3):
+        np.testing.assert_allclose(js[:, c], s_out, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(jkv[:, c], kv, rtol=0, atol=1e-12)
+
+
+def test_invariant_candidate_independence():
+    layers, d, H, f, N, L0, q = _small()
+    w = rand_weights(layers, d, f, N, seed=81)
+    S, ns = rand_inputs(1, 5, L0, N, d, seed=82)
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    kv, _ = O.encode_user(cfg, w, S)
+    batch = O.score_candidates(cfg, w, kv, ns)
+    for c in range(5):
+        alone = O.score_candidates(cfg, w, kv, ns[:, c:c + 1])
+        assert np.array_equal(alone[:, 0], batch[:, c])
+
+
+def test_ns_mask_excludes_later_ns_and_other_candidates():
+    """Changing NS token m of a candidate leaves NS outputs n < m of that
+    candidate unchanged and changes n >= m."""
+    layers, d, H, f, N, L0, q = _small()
+    w = rand_weights(layers, d, f, N, seed=91)
+    S, ns = rand_inputs(1, 2, L0, N, d, seed=92)
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    kv, _ = O.encode_user(cfg, w, S)
+    a = O.score_candidates(cfg, w, kv, ns)
+    ns2 = ns.clone()
+    ns2[0, 0, 1] += 1.0
+    b = O.score_candidates(cfg, w, kv, ns2)
+    assert np.array_equal(a[0, 0, :1], b[0, 0, :1])
+    assert not np.allclose(a[0, 0, 1:], b[0, 0, 1:])
+    assert np.array_equal(a[0, 1], b[0, 1])
+
+
+def test_pyramid_schedule_golden():
+    with open(os.path.join(GOLDEN, "pyramid_schedules.json")) as fh:
+        gold = json.load(fh)
+    for case in gold["cases"]:
+        assert O.pyramid_schedule(case["L0"], case["q_end"], case["layers"]) == case["q"]
+
+
+def test_e4m3_round_matches_torch_cast():
+    """Every in-range value rounds like torch's float8_e4m3fn cast (RNE)."""
+    fp8 = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float()
+    finite = fp8[torch.isfinite(fp8)]
+    for v in finite.tolist():
+        assert O.e4m3_round(v) == v
+    g = torch.Generator().manual_seed(5)
+    xs = torch.cat([torch.randn(4000, generator=g) * s for s in (1e-3, 0.05, 1, 30, 150)])
+    xs = xs[xs.abs() < 440]
+    # midpoints between neighbours are ties: they must go to the even code
+    pos = finite[finite > 0].sort().values
+    mids = (pos[:-1].double() + pos[1:].double()) / 2
+    xs = torch.cat([xs.double(), mids, -mids])
+    want = xs.float().to(torch.float8_e4m3fn).double()
+    got = torch.tensor([O.e4m3_round(v) for v in xs.tolist()], dtype=torch.float64)
+    assert torch.equal(got, want)
+    assert O.e4m3_round(1e6) == 448.0 and O.e4m3_round(-500.0) == -448.0
+
+
+def test_fp8_mode_quantises_and_stays_close():
+    """FP8 mode really quantises (results move) and stays inside the format's
+    bound: e4m3 keeps 3 mantissa bits, so each operand carries at most 2^-4
+    relative rounding error and a product of two at most about 2 * 2^-4."""
+    layers, d, H, f, N, L0, q = _small()
+    w = rand_weights(layers, d, f, N, seed=95)
+    S, ns = rand_inputs(1, 2, L0, N, d, seed=96)
+    c64 = cfg_of(layers, d, H, f, N, L0, q)
+    c8 = cfg_of(layers, d, H, f, N, L0, q, fp8=True)
+    kv, s = O.encode_user(c64, w, S)
+    kv8, s8 = O.encode_user(c8, w, S)
+    n64 = O.score_candidates(c64, w, kv, ns)
+    n8 = O.score_candidates(c8, w, kv8, ns)
+    for a, b in ((s8, s), (kv8, kv), (n8, n64)):
+        err = O.rel_l2(a, b)
+        assert 1e-4 < err < 2 * 2.0 ** -4, err
+
+
+def test_auto_split_matches_numpy():
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn(5, 32, generator=g)
+    Wsp = torch.randn(4 * 8, 32, generator=g)
+    ns = O.auto_split(x, Wsp, 4, 8)
+    ref = (x.double().numpy() @ Wsp.double().numpy().T).reshape(5, 4, 8)
+    np.testing.assert_allclose(ns, ref, rtol=1e-13, atol=1e-13)
+
+
+def test_embed_gather_matches_numpy():
+    g = torch.Generator().manual_seed(4)
+    table = torch.randn(50, 8, generator=g)
+    ids = torch.randint(0, 50, (3, 7), generator=g)
+    out = O.embed_gather(table, ids)
+    assert np.array_equal(out, table.double().numpy()[ids.numpy()])
+    with pytest.raises(IndexError):
+        O.embed_gather(table, np.array([50]))
