@@ -1,0 +1,364 @@
+"""Throughput of the OneTrans block-stack forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload onetrans_s_full]
+
+One step = one pass of the whole hot path over one batch: Auto-Split of the
+static features into NS tokens, then the full forward (every layer's S QKV
+GEMM with the KV-cache store, pyramid-tail S attention, O / FFN GEMMs, and the
+NS side: grouped private-weight GEMMs and NS attention against the cache).
+Default workload: OneTransS-shaped full forward, 6 layers, d=256, 4 heads,
+16 NS tokens, 1190 S tokens (1190 -> 12 pyramid), 64 users x 1 candidate.
+Metric: S-tokens/s = users * L0 / step time.
+
+N > 1 (one process per GPU, launched by torch.distributed.run): every rank runs
+its own replica on its own 64 users (weak scaling, no data-path collective);
+timing is the max over ranks of the device time.
+
+--impl reference times the CPU fp64 oracle on this machine's cores on a
+bounded sample of the same workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback"
+    return d
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        sm.sort()
+        med = sm[len(sm) // 2] if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ---------------------------------------------------------------- oracle (CPU)
+def oracle_sample(wl, users=1, threads=0):
+    """Time the oracle's full forward on `users` users of the workload (full
+    sequence length, all candidates of those users).  Returns (seconds,
+    S tokens processed, threads used)."""
+    import torch  # noqa: F401
+
+    from oracle import oracle as O
+    from synth import gen_auto_split_features, gen_s_tokens, gen_weights
+
+    wl1 = wl.with_(users=users)
+    w = gen_weights(wl1)
+    S = gen_s_tokens(wl1, weights=w)
+    x = gen_auto_split_features(wl1)
+    nthreads = O.set_threads(threads)
+    cfg = O.Config.of(wl1)
+    W = O.Weights(w)
+    t0 = time.perf_counter()
+    ns = O.auto_split(x, w["W_split"], wl.n_ns, wl.d)
+    O.full_forward(cfg, W, S, ns)
+    dt = time.perf_counter() - t0
+    return dt, users * wl.L0, nthreads
+
+
+def run_reference(args, wl):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    # bounded sample: one user of the workload per step (about 10-30 s each)
+    per = []
+    for _ in range(args.warmup_ref):
+        oracle_sample(wl, users=1)
+    cores = 0
+    for _ in range(args.steps_ref):
+        dt, toks, cores = oracle_sample(wl, users=1)
+        per.append(dt / toks)
+    sec_per_tok = sum(per) / len(per)
+    value = 1.0 / sec_per_tok
+    line = {
+        "impl": "reference", "metric": "S-tokens/s (full forward)", "value": value,
+        "unit": "S-tokens/s", "n_gpus": ws, "steps": args.steps_ref, "warmup": args.warmup_ref,
+        "ms_per_step": 1e3 * sec_per_tok * wl.L0, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "users": wl.users, "cands": wl.cands, "L0": wl.L0,
+                   "layers": wl.layers, "d": wl.d},
+        "cpu_baseline": {"value": value, "unit": "S-tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"1 user x {wl.cands} candidate(s) of {wl.name} at full "
+                                   f"length per step, C fp64 oracle, OpenMP"},
+        "e2e": {"value": value, "unit": "S-tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    import unified_transformer_recommender_onetrans_b200 as ot
+    from synth import gen_auto_split_features, gen_s_tokens, gen_weights
+    from unified_transformer_recommender_onetrans_b200.binding import WEIGHT_NAMES
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    ot.lib()
+    dev = torch.device("cuda", local)
+
+    w = gen_weights(wl)
+    S_cpu = gen_s_tokens(wl, weights=w)
+    x_cpu = gen_auto_split_features(wl)
+    q = ot.pyramid_schedule(wl.L0, wl.q_end, wl.layers)
+    m = ot.Model(layers=wl.layers, d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns, L0=wl.L0,
+                 q=q, F=wl.F, eps=wl.eps, dtype=wl.dtype,
+                 weights={k: w[k].to(dev) for k in WEIGHT_NAMES})
+    U, C = wl.users, wl.cands
+    S = S_cpu.to(dev)
+    x = x_cpu.to(dev)
+    ns = torch.empty(U, C, wl.n_ns, wl.d, dtype=m.storage, device=dev)
+    out_ns = torch.empty_like(ns)
+    s_tail = torch.empty(U, q[-1], wl.d, dtype=m.storage, device=dev)
+    kv = m.new_kv_cache(U)
+    ws = torch.empty(m.workspace_bytes(U, C), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def step():
+        m.auto_split(x, ns)
+        m.full_forward(S, ns, kv=kv, out_s_tail=s_tail, out_ns=out_ns, ws=ws)
+
+    for _ in range(args.warmup):
+        step()
+        flush.zero_()
+    m.poll()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- device-timed steps, inputs resident in HBM, L2 flushed between steps
+    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
+                          if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit()
+                          else local)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    launches0 = m.launch_count()
+    m.profile(True)
+    barrier()
+    clocks.start()
+    for e0, e1 in ev:
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        flush.zero_()
+    barrier()
+    clk = clocks.stop()
+    launches = m.launch_count() - launches0
+    recs = m.profile_read()
+    m.profile(False)
+    m.poll()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens_per_step = U * wl.L0 * world
+    value = tokens_per_step / (ms_per_step / 1e3)
+
+    # ---- end to end through the public API: pinned host inputs -> device -> host outputs
+    S_h = S_cpu.pin_memory()
+    x_h = x_cpu.pin_memory()
+    s_tail_h = torch.empty(s_tail.shape, dtype=s_tail.dtype).pin_memory()
+    out_ns_h = torch.empty(out_ns.shape, dtype=out_ns.dtype).pin_memory()
+    S_e2e = torch.empty_like(S)
+    x_e2e = torch.empty_like(x)
+
+    def step_e2e():
+        S_e2e.copy_(S_h, non_blocking=True)
+        x_e2e.copy_(x_h, non_blocking=True)
+        m.auto_split(x_e2e, ns)
+        m.full_forward(S_e2e, ns, kv=kv, out_s_tail=s_tail, out_ns=out_ns, ws=ws)
+        s_tail_h.copy_(s_tail, non_blocking=True)
+        out_ns_h.copy_(out_ns, non_blocking=True)
+
+    for _ in range(2):
+        step_e2e()
+    barrier()
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for e0, e1 in ev2:
+        e0.record(stream)
+        step_e2e()
+        e1.record(stream)
+        flush.zero_()
+    barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = S_h.numel() * S_h.element_size() + x_h.numel() * x_h.element_size()
+    d2h = s_tail_h.numel() * s_tail_h.element_size() + out_ns_h.numel() * out_ns_h.element_size()
+
+    # ---- roofline of the dominant kernel (from the live per-launch events)
+    peaks = load_peaks()
+    by_kind, by_role = {}, {}
+    for r in recs:
+        for key, tab in ((r["kind"], by_kind), (r["role"], by_role)):
+            t = tab.setdefault(key, {"ms": 0.0, "flops": 0.0, "bytes": 0.0, "launches": 0})
+            t["ms"] += r["ms"]
+            t["flops"] += r["flops"]
+            t["bytes"] += r["bytes"]
+            t["launches"] += 1
+    dom = max(by_kind, key=lambda k: by_kind[k]["ms"])
+    dk = by_kind[dom]
+    tf = dk["flops"] / (dk["ms"] / 1e3) / 1e12
+    peak_tf = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": tf, "peak": peak_tf,
+                "unit": "TFLOP/s", "frac": tf / peak_tf, "traffic": None,
+                "peak_source": f"{peaks['_source']} bf16 dense sustained",
+                "launches_per_step": dk["launches"] / args.steps,
+                "algorithmic_tflop_per_step": dk["flops"] / args.steps / 1e12}
+    step_flops = sum(v["flops"] for v in by_kind.values()) / args.steps
+    kernels = {k: {"ms_per_step": v["ms"] / args.steps,
+                   "share": v["ms"] / max(sum(x["ms"] for x in by_kind.values()), 1e-9),
+                   "tflops": v["flops"] / max(v["ms"], 1e-9) / 1e9,
+                   "gbs": v["bytes"] / max(v["ms"], 1e-9) / 1e6}
+               for k, v in by_kind.items()}
+    roles = {k: {"ms_per_step": v["ms"] / args.steps,
+                 "tflops": v["flops"] / max(v["ms"], 1e-9) / 1e9}
+             for k, v in by_role.items()}
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            dt, toks, cores = oracle_sample(wl, users=args.cpu_users)
+            cpu = {"value": toks / dt, "unit": "S-tokens/s", "cores": cores, "kind": "oracle",
+                   "sample": f"{args.cpu_users} users of {wl.name} (full length, {wl.cands} "
+                             f"candidate each), "
+                             f"Auto-Split + encode + score, C fp64 oracle, OpenMP"}
+        line = {
+            "metric": "S-tokens/s (OneTransS full forward)", "value": value, "unit": "S-tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "users_per_gpu": U, "cands": C, "L0": wl.L0,
+                       "pyramid": q, "layers": wl.layers, "d": wl.d, "heads": wl.heads,
+                       "ffn": wl.ffn, "n_ns": wl.n_ns, "parallelism": f"replicas{world}",
+                       "l2": "flushed between steps (256 MB write)"},
+            "step_tflops": step_flops / (ms_per_step / 1e3) / 1e12,
+            "roofline": roofline,
+            "kernels": kernels, "roles": roles,
+            "cpu_baseline": cpu,
+            "e2e": {"value": tokens_per_step / (e2e_ms / 1e3), "unit": "S-tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="onetrans_s_full")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-users", type=int, default=8)
+    args = ap.parse_args()
+    args.steps_ref = max(1, min(args.steps, 3))
+    args.warmup_ref = 0
+    from synth import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,205 @@
+/*
+ * onetrans.h - C ABI of the B200 (sm_100a) OneTrans block-stack forward.
+ *
+ * The method: OneTrans ("OneTrans: Unified Feature Interaction and Sequence
+ * Modeling with One Transformer in Industrial Recommender", WWW 2026).  The
+ * summary page's tokenizer, block, pyramid and KV-cache paragraphs define what
+ * is computed; the blog page's "Mixed Parameterization" and "Cross-Request KV
+ * Caching" designs restate the private-NS-weights and encode-once rules.
+ *
+ *   - S-tokens (behaviour rows) come first, N NS-tokens per candidate follow.
+ *   - Each block: pre-norm RMSNorm, attention, residual, RMSNorm, GELU FFN,
+ *     residual.  All S-tokens share one QKV / O / FFN set; NS position n has
+ *     its own private set.
+ *   - Mask: S-token t sees S-tokens 0..t; NS-token n sees every S-token of the
+ *     layer and NS-tokens 0..n of its own candidate.
+ *   - Pyramid: layer l reads L_l S rows (L_0 = L0), computes K/V for all of
+ *     them, queries for the last q_l only; its S output is those q_l rows,
+ *     so L_{l+1} = q_l.
+ *   - Cross-request KV cache: the S-side runs once per user (encode) and
+ *     stores every layer's S K/V; each candidate's NS-side runs against it.
+ *
+ * Conventions for every call below:
+ *   - Pointers marked "device" are CUDA device pointers owned by the caller,
+ *     contiguous, row-major, 16-byte aligned.  "host" pointers are read only
+ *     during the call.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous on it; nothing synchronises except
+ *     ot_model_create, ot_model_destroy and ot_poll_device_error.
+ *   - Arguments are checked on the host before anything is launched; a
+ *     failed check returns its status and launches nothing.
+ *   - Device-side failures (a bounded wait that expired, a failed index
+ *     check) set the model's device error word instead of trapping; read it
+ *     with ot_poll_device_error.
+ *   - No C++ exception crosses this ABI.  The only allocations are made by
+ *     ot_model_create (weights and the error word); hot calls never allocate.
+ *   - A model may be used from several streams at once if every concurrent
+ *     call has its own workspace and output buffers.
+ *
+ * Storage dtypes: OT_DTYPE_F32 = float32 everywhere (SIMT fp32 arithmetic,
+ * no TF32); OT_DTYPE_BF16 = bfloat16 activations, weights, cache (fp32
+ * accumulation on tcgen05 tensor cores); OT_DTYPE_FP8 = bfloat16 storage with
+ * every QKV / O / FFN projection run on e4m3 operands (per-row activation
+ * scales, one scale per weight matrix), attention and cache in bf16.
+ */
+#ifndef ONETRANS_H
+#define ONETRANS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define OT_MAX_LAYERS 32
+
+typedef enum {
+    OT_OK = 0,
+    OT_ERR_ARG = 1,              /* null pointer, negative or zero count */
+    OT_ERR_SHAPE = 2,            /* config or call shape outside what the kernels support */
+    OT_ERR_DTYPE = 3,            /* dtype not supported by this call */
+    OT_ERR_ALIGN = 4,            /* a pointer is not 16-byte aligned */
+    OT_ERR_CACHE_TOO_SMALL = 5,  /* reserved: cache sizing is by ot_kv_cache_bytes */
+    OT_ERR_WORKSPACE_TOO_SMALL = 6,
+    OT_ERR_CUDA = 7,             /* a CUDA runtime / driver call failed */
+    OT_ERR_DEVICE_TIMEOUT = 8,   /* a device wait hit its iteration bound */
+    OT_ERR_DEVICE_BOUNDS = 9,    /* a device index check failed (e.g. embedding id) */
+    OT_ERR_UNSUPPORTED = 10      /* no kernel for this combination */
+} ot_status;
+
+typedef enum { OT_DTYPE_F32 = 0, OT_DTYPE_BF16 = 1, OT_DTYPE_FP8 = 2 } ot_dtype;
+
+/* Model shape.  q[l] is the S query tail of layer l (1 <= q[l] <= L_l,
+ * L_0 = L0, L_{l+1} = q[l]).  F is the Auto-Split input width (0: no
+ * Auto-Split weights).  heads must divide d and d / heads must be 64 for the
+ * bf16 / fp8 kernels (any value for fp32); d a multiple of 64 (bf16 / fp8),
+ * ffn a multiple of 64. */
+typedef struct {
+    int layers, d, heads, ffn, n_ns, L0;
+    int q[OT_MAX_LAYERS];
+    int F;
+    float eps;
+    int dtype; /* ot_dtype */
+} ot_config;
+
+/* Weights, device pointers in the storage dtype (float32 for OT_DTYPE_F32,
+ * bfloat16 otherwise), "out x in" row-major like a linear layer's weight:
+ *   Wqkv_s [layers][3d][d] (rows: Q | K | V), Wo_s [layers][d][d],
+ *   W1_s [layers][ffn][d], W2_s [layers][d][ffn], g1_s, g2_s [layers][d];
+ *   Wqkv_ns [layers][N][3d][d], Wo_ns [layers][N][d][d],
+ *   W1_ns [layers][N][ffn][d], W2_ns [layers][N][d][ffn],
+ *   g1_ns, g2_ns [layers][N][d];  W_split [N*d][F] (may be NULL if F == 0).
+ * g1 / g2 are the RMSNorm gains before attention and before the FFN. */
+typedef struct {
+    const void *Wqkv_s, *Wo_s, *W1_s, *W2_s, *g1_s, *g2_s;
+    const void *Wqkv_ns, *Wo_ns, *W1_ns, *W2_ns, *g1_ns, *g2_ns;
+    const void *W_split;
+} ot_weights;
+
+typedef struct ot_model ot_model;
+
+/* Validate the config, copy the weights into library-owned device memory in
+ * the layout the kernels read (gains folded into the following projection;
+ * e4m3 copies with per-matrix scales for OT_DTYPE_FP8), and allocate the
+ * device error word.  Runs on the current device; synchronous.
+ * Errors: OT_ERR_ARG / OT_ERR_SHAPE / OT_ERR_DTYPE on a bad config,
+ * OT_ERR_CUDA if an allocation or copy fails (nothing is leaked). */
+ot_status ot_model_create(const ot_config *cfg, const ot_weights *w, ot_model **out);
+void ot_model_destroy(ot_model *m);
+
+/* Bytes of the KV cache for `users` users:
+ * users * sum_l 2 * L_l * d * sizeof(storage).  Layout per user: layers in
+ * order; layer l = K [L_l][d] then V [L_l][d] (heads side by side along d). */
+size_t ot_kv_cache_bytes(const ot_model *m, int users);
+
+/* Workspace bytes a call with `users` users and `cands` candidates per user
+ * needs (encode: cands = 0; score / full forward: cands >= 1).  Includes
+ * room for the KV cache when ot_full_forward is given kv_cache = NULL. */
+size_t ot_workspace_bytes(const ot_model *m, int users, int cands);
+
+/* Auto-Split (summary page, tokenizer paragraph: one projection of the
+ * concatenated static features, then sliced): ns[r][n][:] =
+ * (x[r][:] . W_split^T)[n*d .. n*d+d-1].  x: device [M][F], ns: device
+ * [M][N][d], storage dtype.  Errors: OT_ERR_ARG, OT_ERR_SHAPE (F == 0). */
+ot_status ot_auto_split(ot_model *m, const void *x, long M, void *ns, void *stream);
+
+/* Embedding gather for S-token assembly: out[i][:] = table[ids[i]][:].
+ * table: device bf16 [rows][d]; ids: device int64 [n]; out: device bf16
+ * [n][d].  d must be a multiple of 8.  An id outside [0, rows) writes a zero
+ * row and sets OT_ERR_DEVICE_BOUNDS in `err_word` if err_word != NULL
+ * (device int32, caller-owned). */
+ot_status ot_embed_gather(const void *table, long rows, int d, const int64_t *ids, long n,
+                          void *out, int32_t *err_word, void *stream);
+
+/* Encode U users (S-side, once per user): S device [U][L0][d] ->
+ * kv_cache device (ot_kv_cache_bytes(m, U) bytes) and, if out_s_tail is not
+ * NULL, the last layer's S rows device [U][q_last][d].
+ * ws: device workspace of ws_bytes >= ot_workspace_bytes(m, U, 0). */
+ot_status ot_encode_user(ot_model *m, const void *S, int U, void *kv_cache, void *out_s_tail,
+                         void *ws, size_t ws_bytes, void *stream);
+
+/* Score C candidates per user against the users' cached S K/V (NS-side):
+ * ns device [U][C][N][d] -> out_ns device [U][C][N][d].  kv_cache as written
+ * by ot_encode_user for the same U users.  ws >= ot_workspace_bytes(m, U, C).
+ * A candidate's result does not depend on the other candidates in the call. */
+ot_status ot_score_candidates(ot_model *m, const void *kv_cache, int U, const void *ns, int C,
+                              void *out_ns, void *ws, size_t ws_bytes, void *stream);
+
+/* Training-style batch: B users with C candidates each, S and NS in one
+ * call.  S device [B][L0][d], ns device [B][C][N][d] -> out_s_tail device
+ * [B][q_last][d], out_ns device [B][C][N][d]; the S K/V go to kv_cache if
+ * not NULL (ot_kv_cache_bytes(m, B) bytes), else to the workspace.
+ * ws >= ot_workspace_bytes(m, B, C). */
+ot_status ot_full_forward(ot_model *m, const void *S, const void *ns, int B, int C,
+                          void *out_s_tail, void *out_ns, void *kv_cache, void *ws,
+                          size_t ws_bytes, void *stream);
+
+/* Synchronise `stream`, then read and clear the model's device error word.
+ * Returns OT_OK, OT_ERR_DEVICE_TIMEOUT, OT_ERR_DEVICE_BOUNDS or OT_ERR_CUDA. */
+ot_status ot_poll_device_error(ot_model *m, void *stream);
+
+/* Iteration bound of every device-side wait (mbarrier / flag spin), default
+ * 1 << 26 polls.  A wait that reaches it sets OT_ERR_DEVICE_TIMEOUT and the
+ * kernel returns early.  Test hook: values < 1 are rejected. */
+ot_status ot_set_wait_limit(ot_model *m, long long polls);
+
+/* Kernel family for the bf16 / fp8 projections and attention: 0 = tcgen05
+ * tensor-core kernels (default), 1 = the CUDA-core kernels the fp32 path
+ * uses (slow; a second GPU implementation for cross-checks).  fp32 models
+ * always use the CUDA-core kernels.  Errors: OT_ERR_ARG. */
+ot_status ot_set_kernel_path(ot_model *m, int path);
+
+/* Per-launch timing for roofline reports.  While enabled, every kernel the
+ * model launches is bracketed by two CUDA events on its stream and logged
+ * with its kind and its algorithmic work (FLOPs of the computed outputs only;
+ * bytes = each operand read once plus each output written once).
+ * ot_profile_read synchronises the device, copies up to `max` records
+ * (oldest first) into `out`, clears the log and returns the number copied
+ * (negative on error).  Records beyond an internal 1 << 16 are dropped. */
+typedef enum {
+    OT_KIND_GEMM_TC = 0, OT_KIND_GEMM_SIMT = 1, OT_KIND_ATTN_TC = 2, OT_KIND_ATTN_SIMT = 3,
+    OT_KIND_GATHER = 4, OT_KIND_QUANT = 5
+} ot_kernel_kind;
+
+typedef struct {
+    int kind;      /* ot_kernel_kind */
+    int role;      /* 0 S-QKV, 1 S-attn, 2 S-O, 3 S-FFN1, 4 S-FFN2, 5..9 the NS ones, 10 Auto-Split, 11 other */
+    float ms;      /* device time between the two events */
+    double flops;  /* algorithmic floating-point operations */
+    double bytes;  /* algorithmic HBM bytes */
+} ot_launch_record;
+
+ot_status ot_profile_enable(ot_model *m, int enable);
+int ot_profile_read(ot_model *m, ot_launch_record *out, int max);
+
+/* Static string for a status code. */
+const char *ot_status_str(ot_status s);
+
+/* Kernel launches issued by this model since creation (host-side count). */
+long long ot_launch_count(const ot_model *m);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ONETRANS_H */

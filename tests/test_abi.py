@@ -1,0 +1,109 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/onetrans.h declares, and rejects bad arguments on the host before
+touching the device."""
+
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import unified_transformer_recommender_onetrans_b200 as ot
+from unified_transformer_recommender_onetrans_b200 import binding as B
+from unified_transformer_recommender_onetrans_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return B.lib()
+
+
+def header_functions():
+    txt = open(os.path.join(ROOT, "include", "onetrans.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(ot_[a-z_0-9]+)\s*\(", txt)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = header_functions()
+    assert len(names) >= 14, names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(B.SIGNATURES), set(names) ^ set(B.SIGNATURES)
+
+
+def test_status_strings(lib):
+    for code in range(11):
+        assert lib.ot_status_str(code)
+    assert lib.ot_status_str(0) == b"ok"
+
+
+def _cfg(**kw):
+    c = B.OtConfig()
+    base = dict(layers=2, d=128, heads=2, ffn=256, n_ns=3, L0=40, F=64, eps=1e-6, dtype=1)
+    base.update(kw)
+    q = base.pop("q", [40, 10])
+    for k, v in base.items():
+        setattr(c, k, v)
+    for i, v in enumerate(q):
+        c.q[i] = v
+    return c
+
+
+def _create(lib, cfg, weights=None):
+    w = weights or B.OtWeights(**{n: 16 * (i + 1) for i, n in enumerate(B.WEIGHT_NAMES)})
+    h = C.c_void_p()
+    return lib.ot_model_create(C.byref(cfg), C.byref(w), C.byref(h))
+
+
+def test_create_rejects_bad_config_on_host(lib):
+    assert lib.ot_model_create(None, None, None) == 1
+    assert _create(lib, _cfg(q=[41, 10])) == 2          # q_0 > L0
+    assert _create(lib, _cfg(q=[40, 41])) == 2          # q_1 > L_1
+    assert _create(lib, _cfg(q=[40, 0])) == 2
+    assert _create(lib, _cfg(heads=4)) == 2             # head_dim 32 on the bf16 path
+    assert _create(lib, _cfg(d=96, heads=1, q=[40, 10])) == 2
+    assert _create(lib, _cfg(dtype=7)) == 3
+    assert _create(lib, _cfg(layers=0)) == 1
+    w = B.OtWeights(**{n: 16 * (i + 1) for i, n in enumerate(B.WEIGHT_NAMES)})
+    w.Wo_s = 18                                          # misaligned
+    assert _create(lib, _cfg(), w) == 4
+    w.Wo_s = None
+    assert _create(lib, _cfg(), w) == 1
+
+
+def test_calls_reject_null_model(lib):
+    assert lib.ot_encode_user(None, None, 1, None, None, None, 0, None) == 1
+    assert lib.ot_score_candidates(None, None, 1, None, 1, None, None, 0, None) == 1
+    assert lib.ot_full_forward(None, None, None, 1, 1, None, None, None, None, 0, None) == 1
+    assert lib.ot_auto_split(None, None, 1, None, None) == 1
+    assert lib.ot_embed_gather(None, 1, 8, None, 1, None, None, None) == 1
+    assert lib.ot_embed_gather(16, 1, 12, 16, 1, 16, None, None) == 2
+    assert lib.ot_embed_gather(16, 1, 8, 16, 1, 24, None, None) == 4
+    assert lib.ot_kv_cache_bytes(None, 1) == 0
+    assert lib.ot_set_wait_limit(None, 5) == 1
+    assert lib.ot_launch_count(None) == -1
+
+
+def test_product_pyramid_schedule_matches_golden():
+    import json
+    gold = json.load(open(os.path.join(ROOT, "tests", "golden", "pyramid_schedules.json")))
+    for case in gold["cases"]:
+        assert ot.pyramid_schedule(case["L0"], case["q_end"], case["layers"]) == case["q"]
+    # ties go to even: L0=10, q_end=1, 3 layers -> 10, 5.5 -> 6? (5.5 ties to 6), 1
+    assert ot.pyramid_schedule(10, 1, 3) == [10, 6, 1]
+    assert ot.pyramid_schedule(9, 2, 3) == [9, 6, 2]     # 5.5 -> 6
+    assert ot.pyramid_schedule(11, 2, 3) == [11, 6, 2]   # 6.5 -> 6
+
+
+def test_product_path_does_not_import_oracle():
+    """The product package never reaches the oracle (no CPU fallback)."""
+    pkg = os.path.join(ROOT, "unified_transformer_recommender_onetrans_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in src.replace("oracle-free", ""), f

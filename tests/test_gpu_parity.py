@@ -1,0 +1,273 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU fp64 oracle.
+
+Tolerances are the stated maximum relative L2 error per output tensor: 1e-5
+(fp32 path), 2e-2 (bf16), 6e-2 (fp8); the mask and the pyramid indexing are
+checked bit-exactly.  Output tensors: the final S tail rows, the NS outputs,
+and every layer's K and V in the cache.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import unified_transformer_recommender_onetrans_b200 as ot
+from gpu_common import TOL, assert_within, kv_errors, make_model, model_of, oracle_cfg
+from helpers import rand_inputs, rand_weights
+from oracle import oracle as O
+from synth import WORKLOADS, gen_auto_split_features, gen_s_tokens, gen_weights
+
+pytestmark = pytest.mark.gpu
+
+TEST_WAIT = 1 << 22
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    from unified_transformer_recommender_onetrans_b200.build import build
+    build()
+    assert torch.cuda.is_available()
+
+
+def _run_full(m, S, ns):
+    kv = m.new_kv_cache(S.shape[0])
+    s_tail, ns_out = m.full_forward(S, ns, kv=kv)
+    m.poll()
+    return s_tail, ns_out, kv
+
+
+def _errors_vs_oracle(m, w, S_cpu, ns_cpu, s_tail, ns_out, kv, users):
+    cfg = oracle_cfg(m)
+    kv_o, s_o = O.encode_user(cfg, w, S_cpu[users])
+    ns_o = O.score_candidates(cfg, w, kv_o, ns_cpu[users])
+    errs = {"s_tail": O.rel_l2(s_tail[users].double().cpu().numpy(), s_o),
+            "ns_out": O.rel_l2(ns_out[users].double().cpu().numpy(), ns_o)}
+    errs.update(kv_errors(m, kv[users], kv_o, cfg))
+    return errs
+
+
+# ----------------------------------------------------------------- fp32 path
+def test_tiny_fp32_block_parity():
+    wl = WORKLOADS["tiny_fp32"]
+    w = gen_weights(wl)
+    S = gen_s_tokens(wl, weights=w)
+    x = gen_auto_split_features(wl)                       # [1, 4, 256]
+    m = model_of(wl, w)
+    m.set_wait_limit(TEST_WAIT)
+    ns = m.auto_split(x.cuda())                           # [1, 4, 8, 64]
+    ns_o = O.auto_split(x, w["W_split"], wl.n_ns, wl.d)
+    assert O.rel_l2(ns.double().cpu().numpy(), ns_o) <= TOL["f32"]
+    s_tail, ns_out, kv = _run_full(m, S.cuda(), ns)
+    # the oracle starts from its own fp64 Auto-Split output
+    cfg = oracle_cfg(m)
+    kv_o, s_o = O.encode_user(cfg, w, S)
+    nso = O.score_candidates(cfg, w, kv_o, ns_o)
+    errs = {"s_tail": O.rel_l2(s_tail.double().cpu().numpy(), s_o),
+            "ns_out": O.rel_l2(ns_out.double().cpu().numpy(), nso)}
+    errs.update(kv_errors(m, kv, kv_o, cfg))
+    assert_within(errs, TOL["f32"])
+
+
+# ----------------------------------------------------------------- bf16, small
+SMALL = dict(layers=3, d=128, heads=2, ffn=256, n_ns=5, L0=300, q=[300, 170, 37])
+
+
+@pytest.fixture(scope="module")
+def small_case():
+    w = rand_weights(3, 128, 256, 5, seed=101, dtype=torch.bfloat16)
+    S, ns = rand_inputs(3, 7, 300, 5, 128, seed=102, dtype=torch.bfloat16)
+    return w, S, ns
+
+
+@pytest.mark.parametrize("path", [0, 1], ids=["tcgen05", "cuda_core"])
+def test_bf16_small_parity(small_case, path):
+    w, S, ns = small_case
+    m = make_model(w, **SMALL)
+    m.set_wait_limit(TEST_WAIT)
+    m.set_kernel_path(path)
+    s_tail, ns_out, kv = _run_full(m, S.cuda(), ns.cuda())
+    errs = _errors_vs_oracle(m, w, S, ns, s_tail, ns_out, kv, [0, 1, 2])
+    assert_within(errs, TOL["bf16"])
+
+
+def test_bf16_tcgen05_matches_cuda_core_path(small_case):
+    w, S, ns = small_case
+    m = make_model(w, **SMALL)
+    m.set_wait_limit(TEST_WAIT)
+    a = _run_full(m, S.cuda(), ns.cuda())
+    m.set_kernel_path(1)
+    b = _run_full(m, S.cuda(), ns.cuda())
+    for x, y in zip(a, b):
+        assert O.rel_l2(x.double().cpu().numpy(), y.double().cpu().numpy()) < 1e-2
+
+
+def test_bf16_deterministic(small_case):
+    w, S, ns = small_case
+    m = make_model(w, **SMALL)
+    a = _run_full(m, S.cuda(), ns.cuda())
+    b = _run_full(m, S.cuda(), ns.cuda())
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_kv_cache_equivalence_and_candidate_independence(small_case):
+    w, S, ns = small_case
+    m = make_model(w, **SMALL)
+    Sd, nsd = S.cuda(), ns.cuda()
+    s_tail, ns_out, kv = _run_full(m, Sd, nsd)
+    kv2, s2 = m.encode_user(Sd)
+    sc = m.score_candidates(kv2, nsd)
+    m.poll()
+    assert torch.equal(kv2, kv) and torch.equal(s2, s_tail) and torch.equal(sc, ns_out)
+    # a candidate scored alone matches the same candidate inside the batch
+    for c in (0, 3, 6):
+        alone = m.score_candidates(kv2, nsd[:, c:c + 1].contiguous())
+        m.poll()
+        err = O.rel_l2(alone[:, 0].double().cpu().numpy(), ns_out[:, c].double().cpu().numpy())
+        assert err < 1e-3, (c, err)
+
+
+def test_encode_without_tail_writes_same_cache(small_case):
+    w, S, ns = small_case
+    m = make_model(w, **SMALL)
+    kv_a, _ = m.encode_user(S.cuda())
+    kv_b, none = m.encode_user(S.cuda(), want_s_tail=False)
+    m.poll()
+    assert none is None and torch.equal(kv_a, kv_b)
+
+
+# ----------------------------------------------------------------- bit-exact probes
+def test_mask_probe_bitexact():
+    """W_Q = W_K = 0 makes every score 0; with one-hot S / NS rows, gain 1,
+    W_V = I, W_O = I and W_2 = 0, output row i has a non-zero in column j
+    exactly when key j is visible to query i (plus its own one-hot)."""
+    L0, N, d, q = 100, 8, 128, 60
+    w = rand_weights(1, d, 256, N, seed=5, dtype=torch.bfloat16)
+    eye = torch.eye(d, dtype=torch.bfloat16)
+    for k, shape in (("Wqkv_s", (1, 3 * d, d)), ("Wqkv_ns", (1, N, 3 * d, d))):
+        t = torch.zeros(shape, dtype=torch.bfloat16)
+        t[..., 2 * d:, :] = eye
+        w[k] = t
+    w["g1_s"] = torch.ones_like(w["g1_s"])
+    w["g1_ns"] = torch.ones_like(w["g1_ns"])
+    w["Wo_s"] = eye.expand(1, d, d).clone()
+    w["Wo_ns"] = eye.expand(1, N, d, d).clone()
+    w["W2_s"] = torch.zeros_like(w["W2_s"])
+    w["W2_ns"] = torch.zeros_like(w["W2_ns"])
+    S = torch.zeros(1, L0, d, dtype=torch.bfloat16)
+    S[0, torch.arange(L0), torch.arange(L0)] = 1
+    ns = torch.zeros(1, 2, N, d, dtype=torch.bfloat16)
+    for c in range(2):
+        ns[0, c, torch.arange(N), L0 + torch.arange(N)] = 1
+    for path in (0, 1):
+        m = make_model(w, layers=1, d=d, heads=2, ffn=256, n_ns=N, L0=L0, q=[q])
+        m.set_kernel_path(path)
+        s_tail, ns_out, _ = _run_full(m, S.cuda(), ns.cuda())
+        nz_s = (s_tail[0].float().cpu() != 0)
+        want = torch.zeros(q, d, dtype=torch.bool)
+        for i in range(q):
+            t = L0 - q + i
+            want[i, : t + 1] = True
+        assert torch.equal(nz_s, want), path
+        for c in range(2):
+            nz = ns_out[0, c].float().cpu() != 0
+            want = torch.zeros(N, d, dtype=torch.bool)
+            for n in range(N):
+                want[n, :L0] = True
+                want[n, L0: L0 + n + 1] = True
+            assert torch.equal(nz, want), (path, c)
+
+
+def test_pyramid_identity_bitexact():
+    """W_O = W_2 = 0: every block is the identity on its kept rows, so the
+    final S rows are exactly input rows L0 - q_last .. L0 - 1."""
+    w = rand_weights(4, 128, 256, 3, seed=9, dtype=torch.bfloat16)
+    for k in ("Wo_s", "Wo_ns", "W2_s", "W2_ns"):
+        w[k] = torch.zeros_like(w[k])
+    q = [250, 131, 60, 7]
+    S, ns = rand_inputs(3, 2, 250, 3, 128, seed=10, dtype=torch.bfloat16)
+    m = make_model(w, layers=4, d=128, heads=2, ffn=256, n_ns=3, L0=250, q=q)
+    s_tail, ns_out, _ = _run_full(m, S.cuda(), ns.cuda())
+    assert torch.equal(s_tail.cpu(), S[:, 250 - 7:])
+    assert torch.equal(ns_out.cpu(), ns)
+
+
+# ----------------------------------------------------------------- errors on the device
+def test_device_wait_timeout_is_reported_and_context_survives(small_case):
+    w, S, ns = small_case
+    m = make_model(w, **SMALL)
+    m.set_wait_limit(1)  # a wait that runs out: kernels record it and return
+    m.full_forward(S.cuda(), ns.cuda())
+    with pytest.raises(ot.OtError) as e:
+        m.poll()
+    assert e.value.code == 8
+    m.set_wait_limit(TEST_WAIT)
+    s_tail, ns_out, kv = _run_full(m, S.cuda(), ns.cuda())
+    errs = _errors_vs_oracle(m, w, S, ns, s_tail, ns_out, kv, [1])
+    assert_within(errs, TOL["bf16"])
+
+
+def test_embed_gather_and_bounds_flag():
+    g = torch.Generator().manual_seed(0)
+    table = torch.randn(1000, 384, generator=g).to(torch.bfloat16).cuda()
+    ids = torch.randint(0, 1000, (3, 77), generator=g).cuda()
+    out = ot.embed_gather(table, ids)
+    torch.cuda.synchronize()
+    assert torch.equal(out, table[ids])
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bad = ids.clone()
+    bad[1, 5] = 1000
+    out = ot.embed_gather(table, bad, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 9
+    assert torch.all(out[1, 5] == 0) and torch.equal(out[0], table[ids[0]])
+
+
+# ----------------------------------------------------------------- full-size workloads
+def _full_size(name, users_checked):
+    wl = WORKLOADS[name]
+    w = gen_weights(wl)
+    S = gen_s_tokens(wl, weights=w)
+    x = gen_auto_split_features(wl)
+    m = model_of(wl, w)
+    m.set_wait_limit(TEST_WAIT)
+    ns = m.auto_split(x.cuda())
+    s_tail, ns_out, kv = _run_full(m, S.cuda(), ns)
+    cfg = oracle_cfg(m)
+    ns_o = O.auto_split(x[users_checked], w["W_split"], wl.n_ns, wl.d)
+    kv_o, s_o = O.encode_user(cfg, w, S[users_checked])
+    nso = O.score_candidates(cfg, w, kv_o, ns_o)
+    errs = {"s_tail": O.rel_l2(s_tail[users_checked].double().cpu().numpy(), s_o),
+            "ns_out": O.rel_l2(ns_out[users_checked].double().cpu().numpy(), nso)}
+    errs.update(kv_errors(m, kv[users_checked], kv_o, cfg))
+    return errs
+
+
+def test_onetrans_s_full_forward_sampled_users():
+    assert_within(_full_size("onetrans_s_full", [0, 37]), TOL["bf16"])
+
+
+def test_onetrans_l_full_forward_sampled_users():
+    assert_within(_full_size("onetrans_l_full", [5]), TOL["bf16"])
+
+
+def test_onetrans_s_serving_sampled():
+    wl = WORKLOADS["onetrans_s_serve"]
+    w = gen_weights(wl)
+    S = gen_s_tokens(wl, weights=w)
+    x = gen_auto_split_features(wl)                    # [16, 512, 1024]
+    m = model_of(wl, w)
+    m.set_wait_limit(TEST_WAIT)
+    kv, _ = m.encode_user(S.cuda(), want_s_tail=False)
+    ns = m.auto_split(x.cuda())
+    out = m.score_candidates(kv, ns)
+    m.poll()
+    users, cands = [3, 11], [0, 1, 100, 255, 256, 300, 510, 511]
+    cfg = oracle_cfg(m)
+    kv_o, _ = O.encode_user(cfg, w, S[users])
+    ns_o = O.auto_split(x[users][:, cands], w["W_split"], wl.n_ns, wl.d)
+    out_o = O.score_candidates(cfg, w, kv_o, ns_o)
+    errs = {"ns_out": O.rel_l2(out[users][:, cands].double().cpu().numpy(), out_o)}
+    errs.update(kv_errors(m, kv[users], kv_o, cfg))
+    assert_within(errs, TOL["bf16"])

@@ -1,0 +1,290 @@
+"""ctypes binding of libonetrans.so (argument marshalling only).
+
+The functions keep the C names (``ot_model_create``, ``ot_encode_user``, ...)
+and take plain integers / pointers; :class:`Model` wraps them for torch CUDA
+tensors.  Every step of the forward runs in the library's CUDA kernels: there
+is no CPU or PyTorch fallback, and a missing or unloadable library raises.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "_lib", "libonetrans.so")
+MAX_LAYERS = 32
+
+OT_OK = 0
+STATUS = {0: "OT_OK", 1: "OT_ERR_ARG", 2: "OT_ERR_SHAPE", 3: "OT_ERR_DTYPE", 4: "OT_ERR_ALIGN",
+          5: "OT_ERR_CACHE_TOO_SMALL", 6: "OT_ERR_WORKSPACE_TOO_SMALL", 7: "OT_ERR_CUDA",
+          8: "OT_ERR_DEVICE_TIMEOUT", 9: "OT_ERR_DEVICE_BOUNDS", 10: "OT_ERR_UNSUPPORTED"}
+DTYPES = {"f32": 0, "bf16": 1, "fp8": 2}
+
+# Every function the header declares, with (restype, argtypes).
+_vp, _i, _l, _ll, _sz = C.c_void_p, C.c_int, C.c_long, C.c_longlong, C.c_size_t
+
+
+class OtConfig(C.Structure):
+    _fields_ = [("layers", C.c_int), ("d", C.c_int), ("heads", C.c_int), ("ffn", C.c_int),
+                ("n_ns", C.c_int), ("L0", C.c_int), ("q", C.c_int * MAX_LAYERS), ("F", C.c_int),
+                ("eps", C.c_float), ("dtype", C.c_int)]
+
+
+WEIGHT_NAMES = ("Wqkv_s", "Wo_s", "W1_s", "W2_s", "g1_s", "g2_s", "Wqkv_ns", "Wo_ns", "W1_ns",
+                "W2_ns", "g1_ns", "g2_ns", "W_split")
+
+
+class OtWeights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in WEIGHT_NAMES]
+
+
+class OtLaunchRecord(C.Structure):
+    _fields_ = [("kind", C.c_int), ("role", C.c_int), ("ms", C.c_float), ("flops", C.c_double),
+                ("bytes", C.c_double)]
+
+
+KINDS = {0: "gemm_tc", 1: "gemm_simt", 2: "attn_tc", 3: "attn_simt", 4: "gather", 5: "quant"}
+ROLES = {0: "S_QKV", 1: "S_attn", 2: "S_O", 3: "S_FFN1", 4: "S_FFN2", 5: "NS_QKV", 6: "NS_attn",
+         7: "NS_O", 8: "NS_FFN1", 9: "NS_FFN2", 10: "auto_split", 11: "other"}
+
+SIGNATURES = {
+    "ot_model_create": (_i, [C.POINTER(OtConfig), C.POINTER(OtWeights), C.POINTER(_vp)]),
+    "ot_model_destroy": (None, [_vp]),
+    "ot_kv_cache_bytes": (_sz, [_vp, _i]),
+    "ot_workspace_bytes": (_sz, [_vp, _i, _i]),
+    "ot_auto_split": (_i, [_vp, _vp, _l, _vp, _vp]),
+    "ot_embed_gather": (_i, [_vp, _l, _i, _vp, _l, _vp, _vp, _vp]),
+    "ot_encode_user": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
+    "ot_score_candidates": (_i, [_vp, _vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
+    "ot_full_forward": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "ot_poll_device_error": (_i, [_vp, _vp]),
+    "ot_set_wait_limit": (_i, [_vp, _ll]),
+    "ot_set_kernel_path": (_i, [_vp, _i]),
+    "ot_status_str": (C.c_char_p, [_i]),
+    "ot_launch_count": (_ll, [_vp]),
+    "ot_profile_enable": (_i, [_vp, _i]),
+    "ot_profile_read": (_i, [_vp, C.POINTER(OtLaunchRecord), _i]),
+}
+
+_lib = None
+
+
+def lib():
+    """Load libonetrans.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libonetrans.so not built ({LIB_PATH}); run "
+                              "python -m unified_transformer_recommender_onetrans_b200.build")
+        L = C.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+class OtError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+
+
+def check(code: int, where: str) -> None:
+    if code != OT_OK:
+        raise OtError(code, where)
+
+
+def pyramid_schedule(L0: int, q_end: int | None, layers: int) -> list[int]:
+    """S query tail per layer, linear from L0 to q_end (ties to even).
+
+    Integer form of q_l = L0 - (L0 - q_end) * l / (layers - 1): numerator
+    num = L0 * (layers - 1) - (L0 - q_end) * l over den = layers - 1."""
+    if q_end is None or layers == 1:
+        return [L0] * layers
+    den = layers - 1
+    out = []
+    for l in range(layers):
+        num = L0 * den - (L0 - q_end) * l
+        qd, rem = divmod(num, den)
+        if 2 * rem > den or (2 * rem == den and qd % 2 == 1):
+            qd += 1
+        out.append(qd)
+    return out
+
+
+# ------------------------------------------------------------------ torch face
+def _ptr(t) -> int:
+    if t is None:
+        return 0
+    if not t.is_cuda:
+        raise ValueError("tensors passed to the library must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+class Model:
+    """A OneTrans block stack living on the current CUDA device.
+
+    ``weights``: dict of CUDA tensors in the storage dtype (see
+    include/onetrans.h for layouts).  ``q``: S query tail per layer.
+    """
+
+    def __init__(self, *, layers, d, heads, ffn, n_ns, L0, q, F=0, eps=1e-6, dtype="bf16",
+                 weights: dict):
+        import torch
+        if not torch.cuda.is_available():
+            raise RuntimeError("the OneTrans library needs a CUDA GPU")
+        self.layers, self.d, self.heads, self.ffn, self.n_ns, self.L0 = (layers, d, heads, ffn,
+                                                                         n_ns, L0)
+        self.q, self.F, self.eps, self.dtype = list(q), F, eps, dtype
+        self.storage = torch.float32 if dtype == "f32" else torch.bfloat16
+        cfg = OtConfig()
+        cfg.layers, cfg.d, cfg.heads, cfg.ffn, cfg.n_ns, cfg.L0 = layers, d, heads, ffn, n_ns, L0
+        for i, v in enumerate(self.q):
+            cfg.q[i] = int(v)
+        cfg.F, cfg.eps, cfg.dtype = F, eps, DTYPES[dtype]
+        self._cfg = cfg
+        self._w = {k: weights[k].contiguous() for k in WEIGHT_NAMES if weights.get(k) is not None}
+        for k, t in self._w.items():
+            if t.dtype != self.storage:
+                raise ValueError(f"weight {k} must be {self.storage}")
+        w = OtWeights(**{k: _ptr(self._w.get(k)) for k in WEIGHT_NAMES})
+        h = C.c_void_p()
+        check(lib().ot_model_create(C.byref(cfg), C.byref(w), C.byref(h)), "ot_model_create")
+        self.handle = h
+        self._w = None  # the library holds its own copies
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib().ot_model_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # sizes
+    def kv_cache_bytes(self, users: int) -> int:
+        return int(lib().ot_kv_cache_bytes(self.handle, users))
+
+    def workspace_bytes(self, users: int, cands: int = 0) -> int:
+        return int(lib().ot_workspace_bytes(self.handle, users, cands))
+
+    def rows_at(self, l: int) -> int:
+        return self.L0 if l == 0 else self.q[l - 1]
+
+    def kv_layer_offset(self, l: int) -> int:
+        return sum(2 * self.d * self.rows_at(j) for j in range(l))
+
+    def kv_layer(self, kv_user, l: int):
+        """(K, V) views [L_l, d] of layer l from one user's cache row."""
+        off, L, d = self.kv_layer_offset(l), self.rows_at(l), self.d
+        return (kv_user[off: off + L * d].view(L, d), kv_user[off + L * d: off + 2 * L * d].view(L, d))
+
+    def _ws(self, ws, nbytes):
+        import torch
+        if ws is None:
+            ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device="cuda")
+        return ws
+
+    def set_kernel_path(self, path: int):
+        check(lib().ot_set_kernel_path(self.handle, path), "ot_set_kernel_path")
+
+    def set_wait_limit(self, polls: int):
+        check(lib().ot_set_wait_limit(self.handle, polls), "ot_set_wait_limit")
+
+    def profile(self, enable: bool = True):
+        check(lib().ot_profile_enable(self.handle, int(enable)), "ot_profile_enable")
+
+    def profile_read(self, max_records: int = 1 << 16):
+        """List of dicts (kind, role, ms, flops, bytes) since the last read."""
+        buf = (OtLaunchRecord * max_records)()
+        n = lib().ot_profile_read(self.handle, buf, max_records)
+        if n < 0:
+            raise OtError(-n, "ot_profile_read")
+        return [dict(kind=KINDS.get(r.kind, r.kind), role=ROLES.get(r.role, r.role), ms=r.ms,
+                     flops=r.flops, bytes=r.bytes) for r in buf[:n]]
+
+    def launch_count(self) -> int:
+        return int(lib().ot_launch_count(self.handle))
+
+    def poll(self, stream=None):
+        check(lib().ot_poll_device_error(self.handle, _stream(stream)), "device")
+
+    # calls
+    def new_kv_cache(self, users: int):
+        import torch
+        elems = self.kv_cache_bytes(users) // (4 if self.dtype == "f32" else 2)
+        return torch.empty((users, elems // max(users, 1)), dtype=self.storage, device="cuda")
+
+    def auto_split(self, x, ns=None, stream=None):
+        import torch
+        lead = x.shape[:-1]
+        M = x.numel() // x.shape[-1]
+        if ns is None:
+            ns = torch.empty(*lead, self.n_ns, self.d, dtype=self.storage, device=x.device)
+        check(lib().ot_auto_split(self.handle, _ptr(x), M, _ptr(ns), _stream(stream)),
+              "ot_auto_split")
+        return ns
+
+    def encode_user(self, S, kv=None, out_s_tail=None, ws=None, want_s_tail=True, stream=None):
+        import torch
+        U = S.shape[0]
+        if kv is None:
+            kv = self.new_kv_cache(U)
+        if out_s_tail is None and want_s_tail:
+            out_s_tail = torch.empty(U, self.q[-1], self.d, dtype=self.storage, device=S.device)
+        nb = self.workspace_bytes(U, 0)
+        ws = self._ws(ws, nb)
+        check(lib().ot_encode_user(self.handle, _ptr(S), U, _ptr(kv), _ptr(out_s_tail), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)),
+              "ot_encode_user")
+        return kv, out_s_tail
+
+    def score_candidates(self, kv, ns, out=None, ws=None, stream=None):
+        import torch
+        U, Cn = ns.shape[0], ns.shape[1]
+        if out is None:
+            out = torch.empty_like(ns)
+        ws = self._ws(ws, self.workspace_bytes(U, Cn))
+        check(lib().ot_score_candidates(self.handle, _ptr(kv), U, _ptr(ns), Cn, _ptr(out),
+                                        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+              "ot_score_candidates")
+        return out
+
+    def full_forward(self, S, ns, kv=None, out_s_tail=None, out_ns=None, ws=None, stream=None):
+        import torch
+        B, Cn = ns.shape[0], ns.shape[1]
+        if out_s_tail is None:
+            out_s_tail = torch.empty(B, self.q[-1], self.d, dtype=self.storage, device=S.device)
+        if out_ns is None:
+            out_ns = torch.empty_like(ns)
+        ws = self._ws(ws, self.workspace_bytes(B, Cn))
+        check(lib().ot_full_forward(self.handle, _ptr(S), _ptr(ns), B, Cn, _ptr(out_s_tail),
+                                    _ptr(out_ns), _ptr(kv), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream)),
+              "ot_full_forward")
+        return out_s_tail, out_ns
+
+
+def embed_gather(table, ids, out=None, err=None, stream=None):
+    import torch
+    n = ids.numel()
+    d = table.shape[1]
+    if out is None:
+        out = torch.empty(*ids.shape, d, dtype=table.dtype, device=table.device)
+    check(lib().ot_embed_gather(_ptr(table), table.shape[0], d, _ptr(ids), n, _ptr(out),
+                                _ptr(err), _stream(stream)), "ot_embed_gather")
+    return out

@@ -1,0 +1,727 @@
+// Host entry points of the C ABI declared in include/onetrans.h: argument
+// checks, weight preparation, workspace layout and the per-layer launch
+// sequence of the OneTrans block stack.
+//
+// Per layer l of the S-side (encode, U users, L = L_l rows per user, q = q_l):
+//   1. S QKV GEMM over all U*L rows (RMSNorm row scale in the epilogue, gain
+//      folded into W): K, V -> KV cache rows of layer l; Q -> only the tail
+//      rows t >= L - q, packed [U][q][d].
+//   2. S attention (bottom-right causal over the tail) -> A [U][q][d].
+//   3. O GEMM + residual from the tail rows of the layer input -> H.
+//   4. FFN1 GEMM (norm, GELU) -> hidden; FFN2 GEMM + residual H -> next X.
+// Per layer of the NS-side (score, U users x C candidates x N tokens):
+//   the same four steps with grouped GEMMs (group = NS position n, its own
+//   weights), and NS attention against layer l of the cache.
+#include <cudaTypedefs.h>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "ot_internal.h"
+
+struct ot_model {
+    ot_config cfg;
+    int device;
+    int esz;            // storage bytes per element
+    int path;           // 0 = tensor-core kernels (bf16 / fp8), 1 = CUDA-core kernels
+    void *Wqkv_s, *Wo_s, *W1_s, *W2_s;
+    void *Wqkv_ns, *Wo_ns, *W1_ns, *W2_ns;
+    void *W_split;
+    int *err;
+    long long wait_limit;
+    long long launches;
+    std::vector<void *> allocs;
+    // per-launch profiling
+    struct Rec {
+        int kind, role;
+        double flops, bytes;
+        cudaEvent_t e0, e1;
+    };
+    int profiling = 0;
+    std::vector<Rec> recs;
+    std::vector<cudaEvent_t> event_pool;
+};
+
+namespace ot {
+
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int encode_tmap_3d(void *map, int esz, const void *base, const uint64_t dims[3],
+                   const uint64_t strides_bytes[2], const uint32_t box[3])
+{
+    if (!g_encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return 1;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if ((reinterpret_cast<uintptr_t>(base) & 15) || (strides_bytes[0] & 15) ||
+        (strides_bytes[1] & 15))
+        return 1;
+    CUtensorMapDataType dt = esz == 2   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                             : esz == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    cuuint64_t gd[3] = {dims[0], dims[1], dims[2]};
+    cuuint64_t gs[2] = {strides_bytes[0], strides_bytes[1]};
+    cuuint32_t bx[3] = {box[0], box[1], box[2]};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = g_encode(reinterpret_cast<CUtensorMap *>(map), dt, 3, const_cast<void *>(base),
+                          gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r != CUDA_SUCCESS;
+}
+
+} // namespace ot
+
+using namespace ot;
+
+namespace {
+
+inline int rows_at(const ot_config &c, int l) { return l == 0 ? c.L0 : c.q[l - 1]; }
+
+inline long long kv_layer_off(const ot_config &c, int l)
+{
+    long long off = 0;
+    for (int j = 0; j < l; ++j) off += 2LL * c.d * rows_at(c, j);
+    return off;
+}
+
+inline long long kv_user_elems(const ot_config &c) { return kv_layer_off(c, c.layers); }
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+inline char *at(const void *base, long long elems, int esz)
+{
+    return const_cast<char *>(static_cast<const char *>(base)) + elems * esz;
+}
+
+ot_status check_config(const ot_config &c)
+{
+    if (c.layers < 1 || c.layers > OT_MAX_LAYERS || c.d < 1 || c.heads < 1 || c.ffn < 1 ||
+        c.n_ns < 1 || c.L0 < 1 || c.F < 0 || !(c.eps >= 0.f))
+        return OT_ERR_ARG;
+    if (c.dtype != OT_DTYPE_F32 && c.dtype != OT_DTYPE_BF16 && c.dtype != OT_DTYPE_FP8)
+        return OT_ERR_DTYPE;
+    if (c.d % c.heads) return OT_ERR_SHAPE;
+    int L = c.L0;
+    for (int l = 0; l < c.layers; ++l) {
+        if (c.q[l] < 1 || c.q[l] > L) return OT_ERR_SHAPE;
+        L = c.q[l];
+    }
+    const int hd = c.d / c.heads;
+    if (c.dtype == OT_DTYPE_F32) {
+        if (hd != 16 && hd != 32 && hd != 64) return OT_ERR_SHAPE;
+    } else {
+        if (hd != 64 || c.d % 64 || c.ffn % 64 || c.F % 64) return OT_ERR_SHAPE;
+        if (c.dtype == OT_DTYPE_FP8 && (c.d % 128 || c.ffn % 128)) return OT_ERR_SHAPE;
+    }
+    if (static_cast<long long>(c.n_ns) > 4096) return OT_ERR_SHAPE;
+    return OT_OK;
+}
+
+struct Ws {
+    char *p;
+    size_t left;
+    int esz;
+    void *take(long long elems)
+    {
+        size_t b = (static_cast<size_t>(elems) * esz + 255) & ~static_cast<size_t>(255);
+        if (b > left) return nullptr;
+        void *r = p;
+        p += b;
+        left -= b;
+        return r;
+    }
+};
+
+size_t bytes_of(long long elems, int esz)
+{
+    return (static_cast<size_t>(elems) * esz + 255) & ~static_cast<size_t>(255);
+}
+
+size_t encode_ws_bytes(const ot_config &c, int U, int esz)
+{
+    long long rows = static_cast<long long>(U) * c.L0;
+    return 5 * bytes_of(rows * c.d, esz) + bytes_of(rows * c.ffn, esz);
+}
+
+size_t score_ws_bytes(const ot_config &c, int U, int C, int esz)
+{
+    long long rows = static_cast<long long>(U) * C * c.n_ns;
+    return 7 * bytes_of(rows * c.d, esz) + bytes_of(rows * c.ffn, esz);
+}
+
+enum { ROLE_S_QKV = 0, ROLE_S_ATTN, ROLE_S_O, ROLE_S_FFN1, ROLE_S_FFN2, ROLE_NS_QKV, ROLE_NS_ATTN,
+       ROLE_NS_O, ROLE_NS_FFN1, ROLE_NS_FFN2, ROLE_AUTO_SPLIT, ROLE_OTHER };
+
+cudaEvent_t pooled_event(ot_model *m)
+{
+    if (!m->event_pool.empty()) {
+        cudaEvent_t e = m->event_pool.back();
+        m->event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// Launch `fn` bracketed by profiling events when profiling is on.
+template <typename F>
+ot_status profiled(ot_model *m, cudaStream_t s, int kind, int role, double flops, double bytes,
+                   F fn)
+{
+    cudaEvent_t e0 = nullptr, e1 = nullptr;
+    const bool prof = m->profiling && m->recs.size() < (1u << 16);
+    if (prof) {
+        e0 = pooled_event(m);
+        e1 = pooled_event(m);
+        if (e0) cudaEventRecord(e0, s);
+    }
+    cudaError_t e = fn();
+    m->launches++;
+    if (prof && e0 && e1) {
+        cudaEventRecord(e1, s);
+        m->recs.push_back(ot_model::Rec{kind, role, flops, bytes, e0, e1});
+    }
+    return e == cudaSuccess ? OT_OK : OT_ERR_CUDA;
+}
+
+long long kept_rows(const RowMap &mp, long long M)
+{
+    long long full = (M / mp.P) * (mp.P - mp.min_t);
+    long long rem = M % mp.P - mp.min_t;
+    return full + (rem > 0 ? rem : 0);
+}
+
+ot_status gemm(ot_model *m, GemmArgs &a, cudaStream_t s, int role)
+{
+    a.wait = WaitCtl{m->err, m->wait_limit};
+    a.in_dtype = m->cfg.dtype;
+    a.store = m->cfg.dtype == OT_DTYPE_F32 ? OT_STORE_F32 : OT_STORE_BF16;
+    const bool simt = m->cfg.dtype == OT_DTYPE_F32 || m->path == 1;
+    double flops = 0, bytes = 0;
+    if (m->profiling) {
+        const double esz = m->esz, G = a.G;
+        double out_elems = 0;
+        for (int i = 0; i < a.nseg; ++i)
+            out_elems += static_cast<double>(kept_rows(a.seg[i].map, a.M)) *
+                         (a.seg[i].c_hi - a.seg[i].c_lo);
+        flops = 2.0 * a.K * out_elems * G;
+        bytes = esz * G * (static_cast<double>(a.M) * a.K + static_cast<double>(a.N) * a.K +
+                           out_elems + (a.res ? static_cast<double>(a.M) * a.N : 0.0));
+    }
+    return profiled(m, s, simt ? OT_KIND_GEMM_SIMT : OT_KIND_GEMM_TC, role, flops, bytes, [&] {
+        return simt ? launch_gemm_simt(a, s) : launch_gemm_tc(a, s);
+    });
+}
+
+ot_status attn(ot_model *m, AttnArgs &a, cudaStream_t s)
+{
+    a.wait = WaitCtl{m->err, m->wait_limit};
+    a.dtype = m->cfg.dtype;
+    const bool simt = m->cfg.dtype == OT_DTYPE_F32 || m->path == 1;
+    double flops = 0, bytes = 0;
+    if (m->profiling) {
+        const double L = a.L, nq = a.nq, N = a.N, U = a.U, esz = m->esz;
+        double pairs; // visible (query, key) pairs per user and head
+        if (a.mode == 0)
+            pairs = nq * (L - nq) + nq * (nq + 1) / 2;
+        else
+            pairs = (nq / N) * (N * L + N * (N + 1) / 2);
+        flops = 4.0 * a.hd * pairs * a.H * U;
+        bytes = esz * U * a.d * (2 * nq + 2 * L + (a.mode == 1 ? 2 * nq : 0));
+    }
+    return profiled(m, s, simt ? OT_KIND_ATTN_SIMT : OT_KIND_ATTN_TC,
+                    a.mode == 0 ? ROLE_S_ATTN : ROLE_NS_ATTN, flops, bytes, [&] {
+                        return simt ? launch_attn_simt(a, s) : launch_attn_tc(a, s);
+                    });
+}
+
+GemmArgs gemm_base(const ot_config &c, int M, int N, int K, int G)
+{
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.G = G;
+    a.a_map = rowmap_identity();
+    a.res_map = rowmap_identity();
+    a.eps = c.eps;
+    return a;
+}
+
+EpiSeg seg_of(void *out, long long ld, int lo, int hi, RowMap map)
+{
+    EpiSeg s;
+    s.out = out;
+    s.ld = ld;
+    s.c_lo = lo;
+    s.c_hi = hi;
+    s.map = map;
+    return s;
+}
+
+// S-side of every layer for U users.  X0: [U][L0][d].  s_out may be null.
+ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, Ws ws,
+                     cudaStream_t st)
+{
+    const ot_config &c = m->cfg;
+    const int d = c.d, f = c.ffn, esz = m->esz;
+    const long long rows0 = static_cast<long long>(U) * c.L0;
+    void *Xb[2] = {ws.take(rows0 * d), ws.take(rows0 * d)};
+    void *Qb = ws.take(rows0 * d), *Ab = ws.take(rows0 * d), *Hb = ws.take(rows0 * d);
+    void *hid = ws.take(rows0 * f);
+    if (!Xb[0] || !Xb[1] || !Qb || !Ab || !Hb || !hid) return OT_ERR_WORKSPACE_TOO_SMALL;
+    const long long ustride = kv_user_elems(c);
+    const void *X = X0;
+    ot_status r;
+    for (int l = 0; l < c.layers; ++l) {
+        const int L = rows_at(c, l), q = c.q[l];
+        const bool last = l == c.layers - 1;
+        const bool kv_only = last && s_out == nullptr; // the S tail of the last layer is unused
+        char *K = at(kv, kv_layer_off(c, l), esz);
+        char *V = K + static_cast<long long>(L) * d * esz;
+        const RowMap cache_map{L, ustride / d, 0, 0, 0};
+        // 1. QKV (or KV only)
+        GemmArgs g = gemm_base(c, U * L, kv_only ? 2 * d : 3 * d, d, 1);
+        g.A = X;
+        g.lda = d;
+        g.B = at(m->Wqkv_s, static_cast<long long>(l) * 3 * d * d + (kv_only ? d * d : 0), esz);
+        g.b_gstride = 3LL * d * d;
+        g.norm = 1;
+        if (kv_only) {
+            g.nseg = 2;
+            g.seg[0] = seg_of(K, d, 0, d, cache_map);
+            g.seg[1] = seg_of(V, d, d, 2 * d, cache_map);
+        } else {
+            g.nseg = 3;
+            g.seg[0] = seg_of(Qb, d, 0, d, RowMap{L, q, -(L - q), 0, L - q});
+            g.seg[1] = seg_of(K, d, d, 2 * d, cache_map);
+            g.seg[2] = seg_of(V, d, 2 * d, 3 * d, cache_map);
+        }
+        if ((r = gemm(m, g, st, ROLE_S_QKV)) != OT_OK) return r;
+        if (kv_only) break;
+        // 2. attention over the tail
+        AttnArgs at_;
+        memset(&at_, 0, sizeof(at_));
+        at_.mode = 0;
+        at_.U = U;
+        at_.H = c.heads;
+        at_.hd = d / c.heads;
+        at_.d = d;
+        at_.L = L;
+        at_.nq = q;
+        at_.N = c.n_ns;
+        at_.Q = Qb;
+        at_.KS = K;
+        at_.VS = V;
+        at_.s_ustride = ustride;
+        at_.O = Ab;
+        at_.scale = 1.0f / sqrtf(static_cast<float>(at_.hd));
+        if ((r = attn(m, at_, st)) != OT_OK) return r;
+        // 3. O projection + residual from the tail rows of the layer input
+        g = gemm_base(c, U * q, d, d, 1);
+        g.A = Ab;
+        g.lda = d;
+        g.B = at(m->Wo_s, static_cast<long long>(l) * d * d, esz);
+        g.b_gstride = static_cast<long long>(d) * d;
+        g.res = X;
+        g.res_ld = d;
+        g.res_map = RowMap{q, L, L - q, 0, 0};
+        g.nseg = 1;
+        g.seg[0] = seg_of(Hb, d, 0, d, rowmap_identity());
+        if ((r = gemm(m, g, st, ROLE_S_O)) != OT_OK) return r;
+        // 4. FFN
+        g = gemm_base(c, U * q, f, d, 1);
+        g.A = Hb;
+        g.lda = d;
+        g.B = at(m->W1_s, static_cast<long long>(l) * f * d, esz);
+        g.b_gstride = static_cast<long long>(f) * d;
+        g.norm = 1;
+        g.gelu = 1;
+        g.nseg = 1;
+        g.seg[0] = seg_of(hid, f, 0, f, rowmap_identity());
+        if ((r = gemm(m, g, st, ROLE_S_FFN1)) != OT_OK) return r;
+        void *Xn = (last && s_out) ? s_out : Xb[l & 1];
+        g = gemm_base(c, U * q, d, f, 1);
+        g.A = hid;
+        g.lda = f;
+        g.B = at(m->W2_s, static_cast<long long>(l) * d * f, esz);
+        g.b_gstride = static_cast<long long>(d) * f;
+        g.res = Hb;
+        g.res_ld = d;
+        g.nseg = 1;
+        g.seg[0] = seg_of(Xn, d, 0, d, rowmap_identity());
+        if ((r = gemm(m, g, st, ROLE_S_FFN2)) != OT_OK) return r;
+        X = Xn;
+    }
+    return OT_OK;
+}
+
+// NS-side of every layer: U users x C candidates, N tokens each, against kv.
+ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, void *out, Ws ws,
+                    cudaStream_t st)
+{
+    const ot_config &c = m->cfg;
+    const int d = c.d, f = c.ffn, N = c.n_ns, esz = m->esz;
+    const int Mc = U * C;
+    const long long R = static_cast<long long>(Mc) * N;
+    void *Xb[2] = {ws.take(R * d), ws.take(R * d)};
+    void *Qn = ws.take(R * d), *Kn = ws.take(R * d), *Vn = ws.take(R * d);
+    void *An = ws.take(R * d), *Hn = ws.take(R * d), *hid = ws.take(R * f);
+    if (!Xb[0] || !Xb[1] || !Qn || !Kn || !Vn || !An || !Hn || !hid)
+        return OT_ERR_WORKSPACE_TOO_SMALL;
+    const long long ustride = kv_user_elems(c);
+    const RowMap grp{1, N, 0, 1, 0}; // candidate m, position g -> row m*N + g
+    const void *X = ns;
+    ot_status r;
+    for (int l = 0; l < c.layers; ++l) {
+        const int L = rows_at(c, l);
+        const bool last = l == c.layers - 1;
+        const char *K = at(kv, kv_layer_off(c, l), esz);
+        const char *V = K + static_cast<long long>(L) * d * esz;
+        const long long lN = static_cast<long long>(l) * N;
+        GemmArgs g = gemm_base(c, Mc, 3 * d, d, N);
+        g.A = X;
+        g.lda = d;
+        g.a_map = grp;
+        g.B = at(m->Wqkv_ns, lN * 3 * d * d, esz);
+        g.b_gstride = 3LL * d * d;
+        g.norm = 1;
+        g.nseg = 3;
+        g.seg[0] = seg_of(Qn, d, 0, d, grp);
+        g.seg[1] = seg_of(Kn, d, d, 2 * d, grp);
+        g.seg[2] = seg_of(Vn, d, 2 * d, 3 * d, grp);
+        if ((r = gemm(m, g, st, ROLE_NS_QKV)) != OT_OK) return r;
+        AttnArgs at_;
+        memset(&at_, 0, sizeof(at_));
+        at_.mode = 1;
+        at_.U = U;
+        at_.H = c.heads;
+        at_.hd = d / c.heads;
+        at_.d = d;
+        at_.L = L;
+        at_.nq = C * N;
+        at_.N = N;
+        at_.Q = Qn;
+        at_.KS = K;
+        at_.VS = V;
+        at_.s_ustride = ustride;
+        at_.KN = Kn;
+        at_.VN = Vn;
+        at_.O = An;
+        at_.scale = 1.0f / sqrtf(static_cast<float>(at_.hd));
+        if ((r = attn(m, at_, st)) != OT_OK) return r;
+        g = gemm_base(c, Mc, d, d, N);
+        g.A = An;
+        g.lda = d;
+        g.a_map = grp;
+        g.B = at(m->Wo_ns, lN * d * d, esz);
+        g.b_gstride = static_cast<long long>(d) * d;
+        g.res = X;
+        g.res_ld = d;
+        g.res_map = grp;
+        g.nseg = 1;
+        g.seg[0] = seg_of(Hn, d, 0, d, grp);
+        if ((r = gemm(m, g, st, ROLE_NS_O)) != OT_OK) return r;
+        g = gemm_base(c, Mc, f, d, N);
+        g.A = Hn;
+        g.lda = d;
+        g.a_map = grp;
+        g.B = at(m->W1_ns, lN * f * d, esz);
+        g.b_gstride = static_cast<long long>(f) * d;
+        g.norm = 1;
+        g.gelu = 1;
+        g.nseg = 1;
+        g.seg[0] = seg_of(hid, f, 0, f, grp);
+        if ((r = gemm(m, g, st, ROLE_NS_FFN1)) != OT_OK) return r;
+        void *Xn = last ? out : Xb[l & 1];
+        g = gemm_base(c, Mc, d, f, N);
+        g.A = hid;
+        g.lda = f;
+        g.a_map = grp;
+        g.B = at(m->W2_ns, lN * d * f, esz);
+        g.b_gstride = static_cast<long long>(d) * f;
+        g.res = Hn;
+        g.res_ld = d;
+        g.res_map = grp;
+        g.nseg = 1;
+        g.seg[0] = seg_of(Xn, d, 0, d, grp);
+        if ((r = gemm(m, g, st, ROLE_NS_FFN2)) != OT_OK) return r;
+        X = Xn;
+    }
+    return OT_OK;
+}
+
+ot_status device_copy(ot_model *m, void **dst, const void *src, size_t bytes)
+{
+    if (cudaMalloc(dst, bytes) != cudaSuccess) return OT_ERR_CUDA;
+    m->allocs.push_back(*dst);
+    if (cudaMemcpy(*dst, src, bytes, cudaMemcpyDeviceToDevice) != cudaSuccess) return OT_ERR_CUDA;
+    return OT_OK;
+}
+
+ot_status device_fold(ot_model *m, void **dst, const void *W, const void *gain, long long rows,
+                      int cols, long long groups)
+{
+    size_t bytes = static_cast<size_t>(groups * rows * cols) * m->esz;
+    if (cudaMalloc(dst, bytes) != cudaSuccess) return OT_ERR_CUDA;
+    m->allocs.push_back(*dst);
+    if (launch_fold_gain(W, gain, *dst, rows, cols, groups, cols, m->cfg.dtype == OT_DTYPE_F32
+                                                                      ? OT_DTYPE_F32
+                                                                      : OT_DTYPE_BF16,
+                         0) != cudaSuccess)
+        return OT_ERR_CUDA;
+    return OT_OK;
+}
+
+} // namespace
+
+extern "C" {
+
+const char *ot_status_str(ot_status s)
+{
+    switch (s) {
+    case OT_OK: return "ok";
+    case OT_ERR_ARG: return "invalid argument";
+    case OT_ERR_SHAPE: return "unsupported shape";
+    case OT_ERR_DTYPE: return "unsupported dtype";
+    case OT_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case OT_ERR_CACHE_TOO_SMALL: return "kv cache too small";
+    case OT_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case OT_ERR_CUDA: return "CUDA error";
+    case OT_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case OT_ERR_DEVICE_BOUNDS: return "device index out of bounds";
+    case OT_ERR_UNSUPPORTED: return "unsupported";
+    }
+    return "unknown status";
+}
+
+ot_status ot_model_create(const ot_config *cfg, const ot_weights *w, ot_model **out)
+{
+    if (!cfg || !w || !out) return OT_ERR_ARG;
+    *out = nullptr;
+    ot_status r = check_config(*cfg);
+    if (r != OT_OK) return r;
+    const void *need[] = {w->Wqkv_s, w->Wo_s, w->W1_s, w->W2_s, w->g1_s, w->g2_s,
+                          w->Wqkv_ns, w->Wo_ns, w->W1_ns, w->W2_ns, w->g1_ns, w->g2_ns};
+    for (const void *p : need) {
+        if (!p) return OT_ERR_ARG;
+        if (!aligned16(p)) return OT_ERR_ALIGN;
+    }
+    if (cfg->F > 0 && !w->W_split) return OT_ERR_ARG;
+    if (cfg->dtype == OT_DTYPE_FP8) return OT_ERR_UNSUPPORTED;
+    ot_model *m = new (std::nothrow) ot_model();
+    if (!m) return OT_ERR_CUDA;
+    m->cfg = *cfg;
+    m->esz = cfg->dtype == OT_DTYPE_F32 ? 4 : 2;
+    m->path = 0;
+    m->wait_limit = 1LL << 26;
+    m->launches = 0;
+    cudaGetDevice(&m->device);
+    const long long L = cfg->layers, d = cfg->d, f = cfg->ffn, N = cfg->n_ns;
+    const int esz = m->esz;
+    r = OT_OK;
+    do {
+        if (cudaMalloc(reinterpret_cast<void **>(&m->err), sizeof(int)) != cudaSuccess) {
+            r = OT_ERR_CUDA;
+            break;
+        }
+        m->allocs.push_back(m->err);
+        if (cudaMemset(m->err, 0, sizeof(int)) != cudaSuccess) { r = OT_ERR_CUDA; break; }
+        // gains folded into the projection that follows each norm
+        if ((r = device_fold(m, &m->Wqkv_s, w->Wqkv_s, w->g1_s, 3 * d, d, L)) != OT_OK) break;
+        if ((r = device_fold(m, &m->W1_s, w->W1_s, w->g2_s, f, d, L)) != OT_OK) break;
+        if ((r = device_fold(m, &m->Wqkv_ns, w->Wqkv_ns, w->g1_ns, 3 * d, d, L * N)) != OT_OK)
+            break;
+        if ((r = device_fold(m, &m->W1_ns, w->W1_ns, w->g2_ns, f, d, L * N)) != OT_OK) break;
+        if ((r = device_copy(m, &m->Wo_s, w->Wo_s, L * d * d * esz)) != OT_OK) break;
+        if ((r = device_copy(m, &m->W2_s, w->W2_s, L * d * f * esz)) != OT_OK) break;
+        if ((r = device_copy(m, &m->Wo_ns, w->Wo_ns, L * N * d * d * esz)) != OT_OK) break;
+        if ((r = device_copy(m, &m->W2_ns, w->W2_ns, L * N * d * f * esz)) != OT_OK) break;
+        if (cfg->F > 0 &&
+            (r = device_copy(m, &m->W_split, w->W_split, N * d * cfg->F * esz)) != OT_OK)
+            break;
+        if (cudaDeviceSynchronize() != cudaSuccess) { r = OT_ERR_CUDA; break; }
+    } while (0);
+    if (r != OT_OK) {
+        ot_model_destroy(m);
+        return r;
+    }
+    *out = m;
+    return OT_OK;
+}
+
+void ot_model_destroy(ot_model *m)
+{
+    if (!m) return;
+    cudaDeviceSynchronize();
+    for (void *p : m->allocs) cudaFree(p);
+    for (auto &r : m->recs) {
+        cudaEventDestroy(r.e0);
+        cudaEventDestroy(r.e1);
+    }
+    for (cudaEvent_t e : m->event_pool) cudaEventDestroy(e);
+    delete m;
+}
+
+ot_status ot_profile_enable(ot_model *m, int enable)
+{
+    if (!m) return OT_ERR_ARG;
+    m->profiling = enable != 0;
+    return OT_OK;
+}
+
+int ot_profile_read(ot_model *m, ot_launch_record *out, int max)
+{
+    if (!m || (!out && max > 0) || max < 0) return -OT_ERR_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return -OT_ERR_CUDA;
+    int n = 0;
+    for (auto &r : m->recs) {
+        if (n < max) {
+            float ms = 0.f;
+            cudaEventElapsedTime(&ms, r.e0, r.e1);
+            out[n] = ot_launch_record{r.kind, r.role, ms, r.flops, r.bytes};
+            ++n;
+        }
+        m->event_pool.push_back(r.e0);
+        m->event_pool.push_back(r.e1);
+    }
+    m->recs.clear();
+    return n;
+}
+
+size_t ot_kv_cache_bytes(const ot_model *m, int users)
+{
+    if (!m || users < 0) return 0;
+    return static_cast<size_t>(users) * kv_user_elems(m->cfg) * m->esz;
+}
+
+size_t ot_workspace_bytes(const ot_model *m, int users, int cands)
+{
+    if (!m || users < 0 || cands < 0) return 0;
+    size_t enc = encode_ws_bytes(m->cfg, users, m->esz);
+    if (cands == 0) return enc;
+    size_t sc = score_ws_bytes(m->cfg, users, cands, m->esz);
+    size_t kv = bytes_of(static_cast<long long>(users) * kv_user_elems(m->cfg), m->esz);
+    return (enc > sc ? enc : sc) + kv;
+}
+
+ot_status ot_set_wait_limit(ot_model *m, long long polls)
+{
+    if (!m || polls < 1) return OT_ERR_ARG;
+    m->wait_limit = polls;
+    return OT_OK;
+}
+
+ot_status ot_set_kernel_path(ot_model *m, int path)
+{
+    if (!m || (path != 0 && path != 1)) return OT_ERR_ARG;
+    m->path = path;
+    return OT_OK;
+}
+
+long long ot_launch_count(const ot_model *m) { return m ? m->launches : -1; }
+
+ot_status ot_poll_device_error(ot_model *m, void *stream)
+{
+    if (!m) return OT_ERR_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return OT_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpy(&h, m->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return OT_ERR_CUDA;
+    if (h != 0 && cudaMemset(m->err, 0, sizeof(int)) != cudaSuccess) return OT_ERR_CUDA;
+    return static_cast<ot_status>(h);
+}
+
+ot_status ot_auto_split(ot_model *m, const void *x, long M, void *ns, void *stream)
+{
+    if (!m || !x || !ns || M < 1) return OT_ERR_ARG;
+    if (m->cfg.F <= 0) return OT_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(ns)) return OT_ERR_ALIGN;
+    if (M > (1L << 30)) return OT_ERR_SHAPE;
+    const ot_config &c = m->cfg;
+    const int Nd = c.n_ns * c.d;
+    GemmArgs g = gemm_base(c, static_cast<int>(M), Nd, c.F, 1);
+    g.A = x;
+    g.lda = c.F;
+    g.B = m->W_split;
+    g.b_gstride = static_cast<long long>(Nd) * c.F;
+    g.nseg = 1;
+    g.seg[0] = seg_of(ns, Nd, 0, Nd, rowmap_identity());
+    return gemm(m, g, static_cast<cudaStream_t>(stream), ROLE_AUTO_SPLIT);
+}
+
+ot_status ot_embed_gather(const void *table, long rows, int d, const int64_t *ids, long n,
+                          void *out, int32_t *err_word, void *stream)
+{
+    if (!table || !ids || !out || rows < 1 || d < 8 || n < 0) return OT_ERR_ARG;
+    if (d % 8) return OT_ERR_SHAPE;
+    if (!aligned16(table) || !aligned16(out) || (reinterpret_cast<uintptr_t>(ids) & 7))
+        return OT_ERR_ALIGN;
+    cudaError_t e = launch_embed_gather(table, rows, d, ids, n, out, err_word,
+                                        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? OT_OK : OT_ERR_CUDA;
+}
+
+ot_status ot_encode_user(ot_model *m, const void *S, int U, void *kv_cache, void *out_s_tail,
+                         void *ws, size_t ws_bytes, void *stream)
+{
+    if (!m || !S || !kv_cache || !ws || U < 1) return OT_ERR_ARG;
+    if (!aligned16(S) || !aligned16(kv_cache) || !aligned16(ws) ||
+        (out_s_tail && !aligned16(out_s_tail)))
+        return OT_ERR_ALIGN;
+    if (static_cast<long long>(U) * m->cfg.L0 > (1LL << 31) - 1) return OT_ERR_SHAPE;
+    if (ws_bytes < ot_workspace_bytes(m, U, 0)) return OT_ERR_WORKSPACE_TOO_SMALL;
+    Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
+    return run_encode(m, S, U, kv_cache, out_s_tail, w, static_cast<cudaStream_t>(stream));
+}
+
+ot_status ot_score_candidates(ot_model *m, const void *kv_cache, int U, const void *ns, int C,
+                              void *out_ns, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!m || !kv_cache || !ns || !out_ns || !ws || U < 1 || C < 1) return OT_ERR_ARG;
+    if (!aligned16(kv_cache) || !aligned16(ns) || !aligned16(out_ns) || !aligned16(ws))
+        return OT_ERR_ALIGN;
+    if (static_cast<long long>(U) * C * m->cfg.n_ns > (1LL << 31) - 1) return OT_ERR_SHAPE;
+    if (static_cast<long long>(C) * m->cfg.n_ns > (1LL << 30)) return OT_ERR_SHAPE;
+    if (ws_bytes < score_ws_bytes(m->cfg, U, C, m->esz)) return OT_ERR_WORKSPACE_TOO_SMALL;
+    Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
+    return run_score(m, kv_cache, U, ns, C, out_ns, w, static_cast<cudaStream_t>(stream));
+}
+
+ot_status ot_full_forward(ot_model *m, const void *S, const void *ns, int B, int C,
+                          void *out_s_tail, void *out_ns, void *kv_cache, void *ws,
+                          size_t ws_bytes, void *stream)
+{
+    if (!m || !S || !ns || !out_s_tail || !out_ns || !ws || B < 1 || C < 1) return OT_ERR_ARG;
+    if (!aligned16(S) || !aligned16(ns) || !aligned16(out_s_tail) || !aligned16(out_ns) ||
+        !aligned16(ws) || (kv_cache && !aligned16(kv_cache)))
+        return OT_ERR_ALIGN;
+    if (static_cast<long long>(B) * m->cfg.L0 > (1LL << 31) - 1 ||
+        static_cast<long long>(B) * C * m->cfg.n_ns > (1LL << 31) - 1)
+        return OT_ERR_SHAPE;
+    if (ws_bytes < ot_workspace_bytes(m, B, C)) return OT_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
+    void *kv = kv_cache;
+    if (!kv) {
+        kv = w.take(static_cast<long long>(B) * kv_user_elems(m->cfg));
+        if (!kv) return OT_ERR_WORKSPACE_TOO_SMALL;
+    }
+    ot_status r = run_encode(m, S, B, kv, out_s_tail, w, st);
+    if (r != OT_OK) return r;
+    return run_score(m, kv, B, ns, C, out_ns, w, st);
+}
+
+} // extern "C"

@@ -1,0 +1,120 @@
+// Internal types shared by the host entry points and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/onetrans.h"
+
+namespace ot {
+
+// Bounded-wait control passed to every kernel that waits on device state.
+struct WaitCtl {
+    int *err;         // model error word (device)
+    long long limit;  // polls before giving up
+};
+
+// Row mapping from a GEMM row r (in group g) to a row of some buffer:
+//   row = (r / P) * A + (r % P) + B + g * Gs,   skipped when (r % P) < min_t.
+// It expresses every layout the block needs: flat rows, per-user tails of a
+// pyramid layer, per-user strides of the KV cache, and NS position-major
+// groups over candidate-major storage.
+struct RowMap {
+    long long P, A, B, Gs, min_t;
+};
+
+__host__ __device__ inline RowMap rowmap_identity()
+{
+    return RowMap{1, 1, 0, 0, 0};
+}
+
+__host__ __device__ inline long long rowmap_apply(const RowMap &m, long long r, long long g)
+{
+    long long t = r % m.P;
+    return (r / m.P) * m.A + t + m.B + g * m.Gs;
+}
+
+__host__ __device__ inline bool rowmap_keep(const RowMap &m, long long r)
+{
+    return (r % m.P) >= m.min_t;
+}
+
+// One output column segment [c_lo, c_hi) of a GEMM: written to
+// out + row(r, g) * ld + (c - c_lo).
+struct EpiSeg {
+    void *out;
+    long long ld;
+    int c_lo, c_hi;
+    RowMap map;
+};
+
+enum { OT_STORE_F32 = 0, OT_STORE_BF16 = 1 };
+
+// C[r, c] (group g) = epilogue( sum_k A[row_a(r,g), k] * B[g][c][k] ).
+// Epilogue, in order: * rsqrt(mean_k A^2 + eps) if norm; * row_scale[row_a]
+// if given; * g_scale[g] if given; GELU if gelu; + residual[row_res] if given.
+struct GemmArgs {
+    int M, N, K, G;
+    const void *A;
+    long long lda;
+    RowMap a_map;
+    const void *B;          // [G][N][K]
+    long long b_gstride;    // elements between groups of B
+    int in_dtype;           // OT_DTYPE_F32 / BF16 / FP8 (operand dtype)
+    int store;              // OT_STORE_F32 / BF16
+    int nseg;
+    EpiSeg seg[3];
+    int norm;
+    float eps;
+    const float *row_scale; // indexed by row_a(r, g)
+    const float *g_scale;   // indexed by g
+    int gelu;
+    const void *res;
+    long long res_ld;
+    RowMap res_map;
+    WaitCtl wait;
+};
+
+// Attention over one layer.  Query rows come from Q [U][nq][d] (head h at
+// columns h*hd); S keys / values from the per-user cache rows
+// [U][L][d] (user stride s_ustride elements); NS keys / values (NS mode)
+// from KN / VN [U][nq][d].
+//   S mode  : query i is S row t = L - nq + i; it sees S keys 0..t.
+//   NS mode : query i is NS token n = i % N of candidate c = i / N; it sees
+//             all L S keys and NS keys m <= n of candidate c.
+struct AttnArgs {
+    int mode;           // 0 = S, 1 = NS
+    int U, H, hd, d;
+    int L;              // S keys
+    int nq;             // query rows per user
+    int N;              // NS tokens per candidate (NS mode)
+    const void *Q;
+    const void *KS, *VS;
+    long long s_ustride; // elements between users in KS / VS
+    const void *KN, *VN;
+    void *O;            // [U][nq][d]
+    float scale;        // 1/sqrt(hd)
+    int dtype;
+    WaitCtl wait;
+};
+
+// Launchers (return cudaGetLastError() after the launch).
+cudaError_t launch_gemm_simt(const GemmArgs &a, cudaStream_t s);
+cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s);
+cudaError_t launch_attn_simt(const AttnArgs &a, cudaStream_t s);
+cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s);
+cudaError_t launch_fold_gain(const void *W, const void *g, void *out, long long rows, int cols,
+                             long long groups, long long g_gstride, int dtype, cudaStream_t s);
+cudaError_t launch_embed_gather(const void *table, long long rows, int d, const int64_t *ids,
+                                long long n, void *out, int *err, cudaStream_t s);
+cudaError_t launch_quant_rows(const void *X, long long lda, RowMap map, long long M, int G, int K,
+                              const void *gain, long long gain_gstride, int norm, float eps,
+                              uint8_t *q_out, float *scale_out, cudaStream_t s);
+cudaError_t launch_quant_weights(const void *W, long long per_mat, long long mats, uint8_t *q_out,
+                                 float *scale_out, float *amax_scratch, cudaStream_t s);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+int encode_tmap_3d(void *map, int dtype_bytes, const void *base, const uint64_t dims[3],
+                   const uint64_t strides_bytes[2], const uint32_t box[3]);
+
+} // namespace ot
