@@ -154,6 +154,9 @@ __global__ void __launch_bounds__(192, 1)
                         ss = fmaf(hi, hi, ss);
                     }
                 }
+                // the stage is refilled by TMA (async proxy) once released: order
+                // these generic-proxy reads before that write
+                fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
             }
