@@ -39,8 +39,14 @@
  * Storage dtypes: OT_DTYPE_F32 = float32 everywhere (SIMT fp32 arithmetic,
  * no TF32); OT_DTYPE_BF16 = bfloat16 activations, weights, cache (fp32
  * accumulation on tcgen05 tensor cores); OT_DTYPE_FP8 = bfloat16 storage with
- * every QKV / O / FFN projection run on e4m3 operands (per-row activation
- * scales, one scale per weight matrix), attention and cache in bf16.
+ * every QKV / O / FFN projection run on e4m3 operands, attention and cache in
+ * bf16.  FP8 rule (the V2 podcast page names "kernel fusion + FP8" without a
+ * recipe; this is the library's reading): each projection input row, after
+ * its RMSNorm and gain where the block has one, is quantised with its own
+ * scale s = amax(row) / 448 (s = 1 for an all-zero row), round to nearest
+ * even, saturating; each weight matrix (one layer's Wqkv, Wo, W1 or W2, per
+ * NS position for the private sets) has one scale; the fp32 product is
+ * multiplied by both scales.  Auto-Split stays bf16.
  */
 #ifndef ONETRANS_H
 #define ONETRANS_H
@@ -72,9 +78,9 @@ typedef enum { OT_DTYPE_F32 = 0, OT_DTYPE_BF16 = 1, OT_DTYPE_FP8 = 2 } ot_dtype;
 
 /* Model shape.  q[l] is the S query tail of layer l (1 <= q[l] <= L_l,
  * L_0 = L0, L_{l+1} = q[l]).  F is the Auto-Split input width (0: no
- * Auto-Split weights).  heads must divide d and d / heads must be 64 for the
- * bf16 / fp8 kernels (any value for fp32); d a multiple of 64 (bf16 / fp8),
- * ffn a multiple of 64. */
+ * Auto-Split weights).  heads must divide d; d / heads must be 64 for the
+ * bf16 / fp8 kernels (16, 32 or 64 for fp32); bf16: d, ffn and F multiples
+ * of 64; fp8: d and ffn multiples of 128 (ffn <= 1536). */
 typedef struct {
     int layers, d, heads, ffn, n_ns, L0;
     int q[OT_MAX_LAYERS];
@@ -164,10 +170,11 @@ ot_status ot_poll_device_error(ot_model *m, void *stream);
  * kernel returns early.  Test hook: values < 1 are rejected. */
 ot_status ot_set_wait_limit(ot_model *m, long long polls);
 
-/* Kernel family for the bf16 / fp8 projections and attention: 0 = tcgen05
+/* Kernel family for the bf16 projections and attention: 0 = tcgen05
  * tensor-core kernels (default), 1 = the CUDA-core kernels the fp32 path
  * uses (slow; a second GPU implementation for cross-checks).  fp32 models
- * always use the CUDA-core kernels.  Errors: OT_ERR_ARG. */
+ * always use the CUDA-core kernels.  Errors: OT_ERR_ARG; OT_ERR_UNSUPPORTED
+ * for path 1 on an fp8 model (the CUDA-core kernels read no e4m3). */
 ot_status ot_set_kernel_path(ot_model *m, int path);
 
 /* Per-launch timing for roofline reports.  While enabled, every kernel the

@@ -1,0 +1,162 @@
+// FP8 (e4m3) operand preparation for the projections of the block.
+//
+// Activations: one warp per projection input row.  The row is read once
+// (bf16), optionally RMSNorm-ed with its gain (y = x * rsqrt(mean(x^2) + eps)
+// * gain), its amax taken, scale s = amax / 448 (1 for an all-zero row), and
+// y / s converted to e4m3 with round-to-nearest-even and saturation.  The
+// GEMM epilogue multiplies the fp32 accumulator by s (per row) and by the
+// weight matrix's own scale.  Per-row scales keep each token's projection
+// independent of every other row in the call, so a candidate's result does
+// not depend on which other candidates share the batch.
+//
+// Weights: one CTA per matrix computes its amax, then writes e4m3(w / s_w).
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <math.h>
+
+#include "ot_internal.h"
+
+namespace ot {
+
+constexpr int QR_MAX_CHUNKS = 6; // per lane: 6 x 8 elements -> rows up to 1536
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16 *X, long long lda,
+                                                         RowMap map, long long M, int G, int K,
+                                                         const __nv_bfloat16 *gain,
+                                                         long long gain_gstride, int norm,
+                                                         float eps, uint8_t *q, float *scale)
+{
+    const int lane = threadIdx.x & 31;
+    const long long warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+    const int chunks = K >> 3;
+    for (long long w = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
+         w < M * G; w += warps) {
+        const long long r = w / G;
+        const int g = static_cast<int>(w % G);
+        const long long arow = rowmap_apply(map, r, g);
+        const uint4 *src = reinterpret_cast<const uint4 *>(X + arow * lda);
+        float v[QR_MAX_CHUNKS][8];
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < QR_MAX_CHUNKS; ++i) {
+            const int c = lane + 32 * i;
+            uint4 u = make_uint4(0, 0, 0, 0);
+            if (c < chunks) u = src[c];
+            const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                v[i][2 * e] = __uint_as_float(wd[e] << 16);
+                v[i][2 * e + 1] = __uint_as_float(wd[e] & 0xFFFF0000u);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(v[i][e], v[i][e], ss);
+        }
+        float amax = 0.f;
+        if (norm) {
+            const float rs = 1.0f / sqrtf(warp_sum(ss) / static_cast<float>(K) + eps);
+            const __nv_bfloat16 *gp = gain + g * gain_gstride;
+#pragma unroll
+            for (int i = 0; i < QR_MAX_CHUNKS; ++i) {
+                const int c = lane + 32 * i;
+                if (c >= chunks) continue;
+                const uint4 u = reinterpret_cast<const uint4 *>(gp)[c];
+                const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    v[i][2 * e] *= rs * __uint_as_float(wd[e] << 16);
+                    v[i][2 * e + 1] *= rs * __uint_as_float(wd[e] & 0xFFFF0000u);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < QR_MAX_CHUNKS; ++i)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
+        amax = warp_max(amax);
+        const float s = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        uint2 *dst = reinterpret_cast<uint2 *>(q + arow * K);
+#pragma unroll
+        for (int i = 0; i < QR_MAX_CHUNKS; ++i) {
+            const int c = lane + 32 * i;
+            if (c >= chunks) continue;
+            uint32_t packed[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+                    make_float2(__fdiv_rn(v[i][4 * h], s), __fdiv_rn(v[i][4 * h + 1], s)),
+                    __NV_SATFINITE, __NV_E4M3);
+                __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+                    make_float2(__fdiv_rn(v[i][4 * h + 2], s), __fdiv_rn(v[i][4 * h + 3], s)),
+                    __NV_SATFINITE, __NV_E4M3);
+                packed[h] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+            }
+            dst[c] = make_uint2(packed[0], packed[1]);
+        }
+        if (lane == 0) scale[arow] = s;
+    }
+}
+
+cudaError_t launch_quant_rows(const void *X, long long lda, RowMap map, long long M, int G, int K,
+                              const void *gain, long long gain_gstride, int norm, float eps,
+                              uint8_t *q_out, float *scale_out, cudaStream_t s)
+{
+    if (K % 8 || K > QR_MAX_CHUNKS * 8 * 32) return cudaErrorInvalidValue;
+    const long long rows = M * G;
+    long long blocks = (rows * 32 + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    quant_rows_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16 *>(X), lda, map, M, G, K,
+        static_cast<const __nv_bfloat16 *>(gain), gain_gstride, norm, eps, q_out, scale_out);
+    return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(1024) quant_weights_kernel(const __nv_bfloat16 *W,
+                                                             long long per_mat, uint8_t *q,
+                                                             float *scale)
+{
+    __shared__ float red[32];
+    const long long base = static_cast<long long>(blockIdx.x) * per_mat;
+    float amax = 0.f;
+    for (long long e = threadIdx.x; e < per_mat; e += blockDim.x)
+        amax = fmaxf(amax, fabsf(__bfloat162float(W[base + e])));
+    amax = warp_max(amax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+        v = warp_max(v);
+        if (threadIdx.x == 0) red[0] = v;
+    }
+    __syncthreads();
+    const float s = red[0] > 0.f ? __fdiv_rn(red[0], 448.0f) : 1.0f;
+    for (long long e = threadIdx.x; e < per_mat; e += blockDim.x)
+        q[base + e] = static_cast<uint8_t>(
+            __nv_cvt_float_to_fp8(__fdiv_rn(__bfloat162float(W[base + e]), s), __NV_SATFINITE,
+                                  __NV_E4M3));
+    if (threadIdx.x == 0) scale[blockIdx.x] = s;
+}
+
+cudaError_t launch_quant_weights(const void *W, long long per_mat, long long mats, uint8_t *q_out,
+                                 float *scale_out, float *, cudaStream_t s)
+{
+    quant_weights_kernel<<<static_cast<int>(mats), 1024, 0, s>>>(
+        static_cast<const __nv_bfloat16 *>(W), per_mat, q_out, scale_out);
+    return cudaGetLastError();
+}
+
+} // namespace ot
