@@ -219,7 +219,6 @@ def run_ours(args, wl):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     launches0 = m.launch_count()
-    m.profile(True)
     barrier()
     clocks.start()
     for e0, e1 in ev:
@@ -230,8 +229,6 @@ def run_ours(args, wl):
     barrier()
     clk = clocks.stop()
     launches = m.launch_count() - launches0
-    recs = m.profile_read()
-    m.profile(False)
     m.poll()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = sum(step_ms)
@@ -277,6 +274,18 @@ def run_ours(args, wl):
         e2e_ms = float(t.item())
     h2d = S_h.numel() * S_h.element_size() + x_h.numel() * x_h.element_size()
     d2h = s_tail_h.numel() * s_tail_h.element_size() + out_ns_h.numel() * out_ns_h.element_size()
+
+    # ---- per-kernel times: the same steps again with per-launch events on the
+    # launching streams; profiling runs every kernel alone (no S/NS overlap),
+    # so each event pair brackets exactly one kernel
+    m.profile(True)
+    barrier()
+    for _ in range(args.steps):
+        step()
+        flush.zero_()
+    barrier()
+    recs = m.profile_read()
+    m.profile(False)
 
     # ---- roofline of the dominant kernel (from the live per-launch events)
     peaks = load_peaks()

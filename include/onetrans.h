@@ -79,8 +79,8 @@ typedef enum { OT_DTYPE_F32 = 0, OT_DTYPE_BF16 = 1, OT_DTYPE_FP8 = 2 } ot_dtype;
 /* Model shape.  q[l] is the S query tail of layer l (1 <= q[l] <= L_l,
  * L_0 = L0, L_{l+1} = q[l]).  F is the Auto-Split input width (0: no
  * Auto-Split weights).  heads must divide d; d / heads must be 64 for the
- * bf16 / fp8 kernels (16, 32 or 64 for fp32); bf16: d, ffn and F multiples
- * of 64; fp8: d and ffn multiples of 128 (ffn <= 1536). */
+ * bf16 / fp8 kernels (16, 32 or 64 for fp32); bf16 / fp8: d and ffn
+ * multiples of 128 and F a multiple of 64; fp8: d, ffn <= 1536. */
 typedef struct {
     int layers, d, heads, ffn, n_ns, L0;
     int q[OT_MAX_LAYERS];

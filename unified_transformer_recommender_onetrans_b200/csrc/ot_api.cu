@@ -131,7 +131,7 @@ ot_status check_config(const ot_config &c)
     if (c.dtype == OT_DTYPE_F32) {
         if (hd != 16 && hd != 32 && hd != 64) return OT_ERR_SHAPE;
     } else {
-        if (hd != 64 || c.d % 64 || c.ffn % 64 || c.F % 64) return OT_ERR_SHAPE;
+        if (hd != 64 || c.d % 128 || c.ffn % 128 || c.F % 64) return OT_ERR_SHAPE;
         if (c.dtype == OT_DTYPE_FP8 && (c.d % 128 || c.ffn % 128 || c.d > 1536 || c.ffn > 1536))
             return OT_ERR_SHAPE;
     }

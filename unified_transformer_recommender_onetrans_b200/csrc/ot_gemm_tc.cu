@@ -2,85 +2,145 @@
 // grouped private NS QKV / O / FFN with one weight matrix per NS position,
 // Auto-Split), bf16 or e4m3 operands, fp32 accumulation in TMEM.
 //
-// One CTA computes a 128 x BN tile of one group:
-//   warp 0      TMA producer: A tile [128 rows][128 B] and B tile [BN][128 B]
-//               per stage, 128-byte swizzle, STAGES-deep ring.
-//   warp 1      allocates TMEM (BN columns); lane 0 issues 4 MMAs per stage
-//               (K = 16 bf16 / 32 e4m3 each) and commits stage releases.
-//   warps 2-5   epilogue.  While the main loop runs they also read their row
-//               of every A stage from shared memory and accumulate sum(x^2),
-//               which gives the RMSNorm row scale rsqrt(mean(x^2) + eps) for
-//               the projections that follow a norm (the gain is folded into
-//               the weights on the host).  After the last MMA they load the
-//               accumulator from TMEM (thread = row), apply row scale /
-//               per-row and per-group fp8 scales / GELU / residual, and store
-//               bf16 rows through the row maps.
-//
-// A stage is released when both the MMAs that read it have completed
-// (tcgen05.commit) and, for norm GEMMs, the four epilogue warps have read it.
+// Persistent: one CTA per SM walks a static list of 128 x 128 output tiles
+// (group-major, then M, then N fastest, so CTAs running together share their
+// A tiles in L2).  Warp roles:
+//   warp 0      TMA producer: per k-block an A tile [128 rows][128 B] and a
+//               B tile [128][128 B], 128-byte swizzle, 6-stage ring.
+//   warp 1      TMEM owner (256 columns = two 128-column accumulators); lane 0
+//               issues 4 MMAs per k-block (K = 16 bf16 / 32 e4m3 each) into
+//               accumulator t % 2, so the MMAs of tile t+1 run while the
+//               epilogue drains tile t.
+//   warps 2-9   epilogue, two per TMEM lane quarter (32 rows x 64 columns
+//               each): residual rows prefetched into a swizzled staging buffer
+//               before the accumulator is ready, then per 32 columns: TMEM ->
+//               registers, row scale (RMSNorm, fp8 scales), GELU, + residual,
+//               bf16 into the staging buffer; finally 128-byte coalesced row
+//               stores through the row maps (Q tail, KV cache rows, NS groups),
+//               each row's address computed once per tile by its own lane.
+//   warps 10-13 RMSNorm warps (projections that follow a norm): read their row
+//               of every A stage of the tile in flight and hand
+//               sum(x^2) to the epilogue through shared memory; the gain is
+//               folded into the weights on the host.
+// A stage returns to the producer when its MMAs completed (tcgen05.commit)
+// and, for norm GEMMs, the four norm warps read it (their generic-proxy reads
+// are ordered before the next TMA write by fence.proxy.async).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include "ot_gelu_poly.h"
 #include "ot_internal.h"
 #include "ot_ptx.cuh"
 
 namespace ot {
 
-constexpr int TC_BM = 128;
-constexpr int TC_ROW_BYTES = 128; // one swizzle row of K per stage
+constexpr int G_BM = 128, G_BN = 128, G_STAGES = 6;
+constexpr int G_EPI_WARPS = 8, G_NORM_WARPS = 4;
+constexpr int G_THREADS = 32 * (2 + G_EPI_WARPS + G_NORM_WARPS);
+constexpr uint32_t G_TILE = 128 * 128;          // one stage operand: 128 rows x 128 bytes
+constexpr uint32_t G_EPI_COLS = G_BN / 2;       // each epilogue warp: 32 rows x 64 columns
+constexpr uint32_t G_STAGING = 32 * G_EPI_COLS * 2;
+constexpr size_t G_SMEM = 1024 + 2 * G_STAGES * G_TILE + G_EPI_WARPS * G_STAGING +
+                          2 * G_BM * sizeof(float) + 256;
 
 struct TcGemmParams {
     GemmArgs a;
     int a_grouped; // A tensor map is (K, G, M) instead of (K, M, 1)
+    int m_tiles, n_tiles;
+    long long tiles;
 };
 
-__device__ __forceinline__ float gelu_erf_tc(float z)
+// exact-erf GELU, z * Phi(z), with Phi from the fitted odd polynomial
+__device__ __forceinline__ float gelu_poly(float z)
 {
-    return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+    const float zc = fminf(fmaxf(z, -OT_GELU_ZC), OT_GELU_ZC);
+    const float v = zc * zc * (1.0f / (OT_GELU_ZC * OT_GELU_ZC));
+    float p = kGeluPoly[OT_GELU_DEG];
+#pragma unroll
+    for (int k = OT_GELU_DEG - 1; k >= 0; --k) p = fmaf(p, v, kGeluPoly[k]);
+    return z * fmaf(zc, p, 0.5f);
 }
 
-template <int BN, int STAGES, bool FP8>
-__global__ void __launch_bounds__(192, 1)
+__device__ __forceinline__ void decode_tile(const TcGemmParams &P, long long tile, int &g, int &m0,
+                                            int &n0)
+{
+    const int nt = static_cast<int>(tile % P.n_tiles);
+    const long long rest = tile / P.n_tiles;
+    m0 = static_cast<int>(rest % P.m_tiles) * G_BM;
+    g = static_cast<int>(rest / P.m_tiles);
+    n0 = nt * G_BN;
+}
+
+// staging layout: row r (0..31) is 128 bytes, 16-byte chunk c stored at c ^ (r & 7)
+__device__ __forceinline__ uint4 *stage_chunk(uint8_t *stage, int r, int c)
+{
+    return reinterpret_cast<uint4 *>(stage + r * (G_EPI_COLS * 2) + ((c ^ (r & 7)) << 4));
+}
+
+// Row map with 32-bit quotient / remainder (rows and periods fit in 31 bits).
+__device__ __forceinline__ long long rowmap_dev(const RowMap &m, int r, int g)
+{
+    const unsigned P = static_cast<unsigned>(m.P);
+    const unsigned ur = static_cast<unsigned>(r);
+    const unsigned qt = ur / P, t = ur - qt * P;
+    return static_cast<long long>(qt) * m.A + t + m.B + static_cast<long long>(g) * m.Gs;
+}
+
+__device__ __forceinline__ bool rowmap_keep_dev(const RowMap &m, int r)
+{
+    const unsigned P = static_cast<unsigned>(m.P);
+    return static_cast<long long>(static_cast<unsigned>(r) % P) >= m.min_t;
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(G_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ TcGemmParams P)
 {
-    constexpr uint32_t A_BYTES = TC_BM * TC_ROW_BYTES;
-    constexpr uint32_t B_BYTES = BN * TC_ROW_BYTES;
-    constexpr uint32_t IDESC = make_idesc(TC_BM, BN, FP8 ? 0 : 1, 0, 0);
+    constexpr uint32_t IDESC = make_idesc(G_BM, G_BN, FP8 ? 0 : 1, 0, 0);
     const GemmArgs &a = P.a;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     uint8_t *sA = smem;
-    uint8_t *sB = smem + STAGES * A_BYTES;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sB + STAGES * B_BYTES);
-    uint64_t *empty = full + STAGES;
-    uint64_t *acc_full = empty + STAGES;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    uint8_t *sB = sA + G_STAGES * G_TILE;
+    uint8_t *sOut = sB + G_STAGES * G_TILE;
+    float *ssbuf = reinterpret_cast<float *>(sOut + G_EPI_WARPS * G_STAGING); // [2][128]
+    uint64_t *full = reinterpret_cast<uint64_t *>(ssbuf + 2 * G_BM);
+    uint64_t *empty = full + G_STAGES;
+    uint64_t *tfull = empty + G_STAGES;   // [2]
+    uint64_t *tempty = tfull + 2;         // [2]
+    uint64_t *nfull = tempty + 2;         // [2]
+    uint64_t *nempty = nfull + 2;         // [2]
+    uint64_t *mma_done = nempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN;
-    const int m0 = blockIdx.y * TC_BM;
-    const int g = blockIdx.z;
     const int num_kb = a.K / (FP8 ? 128 : 64);
-    const bool norm = a.norm != 0;
+    const bool norm = a.norm != 0 && !FP8;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < G_STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], norm ? 5 : 1);
+            mbar_init(&empty[s], norm ? 1 + G_NORM_WARPS : 1);
         }
-        mbar_init(acc_full, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], G_EPI_WARPS);
+            mbar_init(&nfull[b], G_NORM_WARPS);
+            mbar_init(&nempty[b], G_EPI_WARPS);
+        }
+        mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch(&tmA);
         tma_prefetch(&tmB);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, BN < 32 ? 32 : BN);
+        tmem_alloc(tmem_slot, 2 * G_BN);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -92,64 +152,188 @@ __global__ void __launch_bounds__(192, 1)
     volatile int no_abort = 0;
 
     if (warp == 0) {
+        // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            int issued = 0;
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const int s = kb % STAGES;
-                const uint32_t ph = (kb / STAGES) & 1;
-                if (!mbar_wait(&empty[s], ph ^ 1, a.wait, abort_flag)) break;
-                mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
-                const int kx = kb * (FP8 ? 128 : 64);
-                if (P.a_grouped)
-                    tma_load_3d(sA + s * A_BYTES, &tmA, &full[s], kx, g, m0);
-                else
-                    tma_load_3d(sA + s * A_BYTES, &tmA, &full[s], kx, m0, 0);
-                tma_load_3d(sB + s * B_BYTES, &tmB, &full[s], kx, n0, g);
-                issued = kb + 1;
+            long long it = 0;
+            bool ok = true;
+            for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x) {
+                int g, m0, n0;
+                decode_tile(P, tile, g, m0, n0);
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = static_cast<int>(it % G_STAGES);
+                    const uint32_t ph = static_cast<uint32_t>((it / G_STAGES) & 1);
+                    if (!mbar_wait(&empty[s], ph ^ 1, a.wait, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&full[s], 2 * G_TILE);
+                    const int kx = kb * (FP8 ? 128 : 64);
+                    if (P.a_grouped)
+                        tma_load_3d(sA + s * G_TILE, &tmA, &full[s], kx, g, m0);
+                    else
+                        tma_load_3d(sA + s * G_TILE, &tmA, &full[s], kx, m0, 0);
+                    tma_load_3d(sB + s * G_TILE, &tmB, &full[s], kx, n0, g);
+                }
             }
-            // never leave a load in flight: wait for the last STAGES issued
-            for (int kb = issued > STAGES ? issued - STAGES : 0; kb < issued; ++kb)
-                mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, final_wait, &no_abort);
+            // never leave a load in flight
+            for (long long j = it > G_STAGES ? it - G_STAGES : 0; j < it; ++j)
+                mbar_wait(&full[j % G_STAGES], static_cast<uint32_t>((j / G_STAGES) & 1),
+                          final_wait, &no_abort);
         }
     } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const int s = kb % STAGES;
-                if (!mbar_wait(&full[s], (kb / STAGES) & 1, a.wait, abort_flag)) break;
+            long long it = 0;
+            int t = 0;
+            bool ok = true;
+            for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x, ++t) {
+                const int b = t & 1;
+                if (!mbar_wait(&tempty[b], ((t >> 1) & 1) ^ 1, a.wait, abort_flag)) break;
                 tc_fence_after();
-                const uint32_t a_addr = smem_u32(sA + s * A_BYTES);
-                const uint32_t b_addr = smem_u32(sB + s * B_BYTES);
+                const uint32_t acc = tmem + b * G_BN;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = static_cast<int>(it % G_STAGES);
+                    if (!mbar_wait(&full[s], static_cast<uint32_t>((it / G_STAGES) & 1), a.wait,
+                                   abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(sA + s * G_TILE);
+                    const uint32_t b_addr = smem_u32(sB + s * G_TILE);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint64_t ad = sw128_desc(a_addr + k * 32, 16);
-                    const uint64_t bd = sw128_desc(b_addr + k * 32, 16);
-                    if (FP8)
-                        mma_f8(tmem, ad, bd, IDESC, (kb | k) != 0);
-                    else
-                        mma_f16(tmem, ad, bd, IDESC, (kb | k) != 0);
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t ad = sw128_desc(a_addr + k * 32, 16);
+                        const uint64_t bd = sw128_desc(b_addr + k * 32, 16);
+                        if (FP8)
+                            mma_f8(acc, ad, bd, IDESC, (kb | k) != 0);
+                        else
+                            mma_f16(acc, ad, bd, IDESC, (kb | k) != 0);
+                    }
+                    mma_commit(&empty[s]);
                 }
-                mma_commit(&empty[s]);
+                if (!ok) break;
+                mma_commit(&tfull[b]);
             }
-            mma_commit(acc_full); // always: completes once every issued MMA is done
+            // every issued MMA must be complete before TMEM is released
+            mma_commit(mma_done);
+            mbar_wait(mma_done, 0, final_wait, &no_abort);
         }
-    } else {
-        // ---------------- epilogue warps
-        const int quarter = warp & 3;
-        const int row = quarter * 32 + lane;
-        float ss = 0.f;
-        if (norm) {
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const int s = kb % STAGES;
-                if (!mbar_wait(&full[s], (kb / STAGES) & 1, a.wait, abort_flag)) break;
-                const uint4 *src = reinterpret_cast<const uint4 *>(sA + s * A_BYTES + row * TC_ROW_BYTES);
+    } else if (warp < 2 + G_EPI_WARPS) {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;              // TMEM lane quarter = rows 32q .. 32q+31
+        const int half = (warp - 2) >> 2;    // columns 64*half .. 64*half+63 of the tile
+        uint8_t *stage = sOut + (warp - 2) * G_STAGING;
+        const __nv_bfloat16 *res = static_cast<const __nv_bfloat16 *>(a.res);
+        int t = 0;
+        for (long long tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++t) {
+            int g, m0, n0;
+            decode_tile(P, tile, g, m0, n0);
+            const int b = t & 1;
+            const int c0 = n0 + half * G_EPI_COLS; // first output column of this warp
+            const int r = m0 + 32 * q + lane;      // this lane's row
+            const bool live = r < a.M;
+            // per-row addresses, computed once by the lane that owns the row
+            int sidx = 0;
+            while (sidx + 1 < a.nseg && !(n0 >= a.seg[sidx].c_lo && n0 < a.seg[sidx].c_hi)) ++sidx;
+            const EpiSeg &sg = a.seg[sidx];
+            long long out_off = -1, res_off = 0;
+            if (live && rowmap_keep_dev(sg.map, r))
+                out_off = rowmap_dev(sg.map, r, g) * sg.ld + (c0 - sg.c_lo);
+            if (live && res) res_off = rowmap_dev(a.res_map, r, g) * a.res_ld + c0;
+            if (res) { // coalesced residual prefetch: 4 rows x 128 B per instruction
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int rl = 4 * i + (lane >> 3), ch = lane & 7;
+                    const long long ro = __shfl_sync(0xffffffffu, res_off, rl);
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (m0 + 32 * q + rl < a.M)
+                        v = *reinterpret_cast<const uint4 *>(res + ro + ch * 8);
+                    *stage_chunk(stage, rl, ch) = v;
+                }
+            }
+            if (!mbar_wait(&tfull[b], (t >> 1) & 1, a.wait, abort_flag)) break;
+            tc_fence_after();
+            float rs = 1.f;
+            if (norm) {
+                if (!mbar_wait(&nfull[b], (t >> 1) & 1, a.wait, abort_flag)) break;
+                rs = rsqrtf(ssbuf[b * G_BM + 32 * q + lane] / static_cast<float>(a.K) + a.eps);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&nempty[b]);
+            }
+            if (live && a.row_scale) rs *= a.row_scale[rowmap_dev(a.a_map, r, g)];
+            if (a.g_scale) rs *= a.g_scale[g];
+            __syncwarp(); // residual staging complete before rows are read back
+#pragma unroll 1
+            for (int c = 0; c < G_EPI_COLS / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tmem + b * G_BN + (static_cast<uint32_t>(q * 32) << 16) +
+                              half * G_EPI_COLS + c * 32,
+                          v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint4 *p = stage_chunk(stage, lane, 4 * c + j);
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        f[e] = __uint_as_float(v[8 * j + e]) * rs;
+                        if (a.gelu) f[e] = gelu_poly(f[e]);
+                    }
+                    if (res) {
+                        const uint4 x = *p;
+                        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            f[2 * e] += __uint_as_float(w[e] << 16);
+                            f[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+                        }
+                    }
+                    uint4 o;
+                    o.x = pack_bf16x2(f[0], f[1]);
+                    o.y = pack_bf16x2(f[2], f[3]);
+                    o.z = pack_bf16x2(f[4], f[5]);
+                    o.w = pack_bf16x2(f[6], f[7]);
+                    *p = o;
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[b]); // accumulator b may be overwritten
+            // coalesced stores: 8 lanes per row, 128 contiguous bytes
+            __nv_bfloat16 *obase = static_cast<__nv_bfloat16 *>(sg.out);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int rl = 4 * i + (lane >> 3), ch = lane & 7;
+                const long long oo = __shfl_sync(0xffffffffu, out_off, rl);
+                if (oo < 0) continue;
+                *reinterpret_cast<uint4 *>(obase + oo + ch * 8) = *stage_chunk(stage, rl, ch);
+            }
+            __syncwarp(); // staging free for the next tile
+        }
+    } else if (norm) {
+        // ------------------------------------------------ RMSNorm row sums
+        const int row = 32 * (warp - 2 - G_EPI_WARPS) + lane; // warps 10-13: rows 0..127
+        long long it = 0;
+        int t = 0;
+        bool ok = true;
+        for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x, ++t) {
+            const int b = t & 1;
+            if (!mbar_wait(&nempty[b], ((t >> 1) & 1) ^ 1, a.wait, abort_flag)) break;
+            float ss = 0.f;
+            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                const int s = static_cast<int>(it % G_STAGES);
+                if (!mbar_wait(&full[s], static_cast<uint32_t>((it / G_STAGES) & 1), a.wait,
+                               abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint4 *src = reinterpret_cast<const uint4 *>(sA + s * G_TILE + row * 128);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    uint4 v = src[c];
+                    const uint4 v = src[c];
                     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        float lo = __uint_as_float(w[e] << 16);
-                        float hi = __uint_as_float(w[e] & 0xFFFF0000u);
+                        const float lo = __uint_as_float(w[e] << 16);
+                        const float hi = __uint_as_float(w[e] & 0xFFFF0000u);
                         ss = fmaf(lo, lo, ss);
                         ss = fmaf(hi, hi, ss);
                     }
@@ -160,74 +344,23 @@ __global__ void __launch_bounds__(192, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
             }
-        }
-        const bool ok = mbar_wait(acc_full, 0, final_wait, &no_abort) && !*abort_flag;
-        tc_fence_after();
-        const long long r = static_cast<long long>(m0) + row;
-        const bool live = ok && r < a.M;
-        float rs = 1.f;
-        long long arow = 0;
-        if (live) {
-            arow = rowmap_apply(a.a_map, r, g);
-            if (norm) rs = rsqrtf(ss / static_cast<float>(a.K) + a.eps);
-            if (a.row_scale) rs *= a.row_scale[arow];
-            if (a.g_scale) rs *= a.g_scale[g];
-        }
-        const __nv_bfloat16 *res = static_cast<const __nv_bfloat16 *>(a.res);
-        const long long res_row = (live && res) ? rowmap_apply(a.res_map, r, g) : 0;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-            uint32_t v[32];
-            tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + c, v);
-            tmem_ld_wait();
-            if (!live) continue;
-            const int col = n0 + c;
-            float f[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                f[e] = __uint_as_float(v[e]) * rs;
-                if (a.gelu) f[e] = gelu_erf_tc(f[e]);
-            }
-            if (res) {
-                const uint4 *rp = reinterpret_cast<const uint4 *>(res + res_row * a.res_ld + col);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint4 x = rp[q];
-                    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        f[q * 8 + 2 * e] += __uint_as_float(w[e] << 16);
-                        f[q * 8 + 2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
-                    }
-                }
-            }
-            for (int sidx = 0; sidx < a.nseg; ++sidx) {
-                const EpiSeg &sg = a.seg[sidx];
-                if (col < sg.c_lo || col >= sg.c_hi || !rowmap_keep(sg.map, r)) continue;
-                __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(sg.out) +
-                                     rowmap_apply(sg.map, r, g) * sg.ld + (col - sg.c_lo);
-                uint4 *dp = reinterpret_cast<uint4 *>(dst);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint4 o;
-                    o.x = pack_bf16x2(f[q * 8 + 0], f[q * 8 + 1]);
-                    o.y = pack_bf16x2(f[q * 8 + 2], f[q * 8 + 3]);
-                    o.z = pack_bf16x2(f[q * 8 + 4], f[q * 8 + 5]);
-                    o.w = pack_bf16x2(f[q * 8 + 6], f[q * 8 + 7]);
-                    dp[q] = o;
-                }
-            }
+            if (!ok) break;
+            ssbuf[b * G_BM + row] = ss;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&nfull[b]);
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, BN < 32 ? 32 : BN);
+        tmem_dealloc(tmem, 2 * G_BN);
     }
 }
 
-template <int BN, int STAGES, bool FP8>
+static int g_num_sms = 0;
+
+template <bool FP8>
 static cudaError_t launch_tc_cfg(const GemmArgs &a, cudaStream_t s)
 {
     const int esz = FP8 ? 1 : 2;
@@ -236,19 +369,22 @@ static cudaError_t launch_tc_cfg(const GemmArgs &a, cudaStream_t s)
     TcGemmParams p;
     p.a = a;
     p.a_grouped = a.G > 1 && a.a_map.Gs != 0;
+    p.m_tiles = (a.M + G_BM - 1) / G_BM;
+    p.n_tiles = a.N / G_BN;
+    p.tiles = static_cast<long long>(p.m_tiles) * p.n_tiles * a.G;
     const char *Abase = static_cast<const char *>(a.A) + a.a_map.B * a.lda * esz;
     if (p.a_grouped) {
         uint64_t dims[3] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.G),
                             static_cast<uint64_t>(a.M)};
         uint64_t str[2] = {static_cast<uint64_t>(a.a_map.Gs * a.lda * esz),
                            static_cast<uint64_t>(a.a_map.A * a.lda * esz)};
-        uint32_t box[3] = {static_cast<uint32_t>(kbox), 1, TC_BM};
+        uint32_t box[3] = {static_cast<uint32_t>(kbox), 1, G_BM};
         if (encode_tmap_3d(&tmA, esz, Abase, dims, str, box)) return cudaErrorInvalidValue;
     } else {
         uint64_t dims[3] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M), 1};
         uint64_t rs = static_cast<uint64_t>(a.a_map.A * a.lda * esz);
         uint64_t str[2] = {rs, rs * static_cast<uint64_t>(a.M)};
-        uint32_t box[3] = {static_cast<uint32_t>(kbox), TC_BM, 1};
+        uint32_t box[3] = {static_cast<uint32_t>(kbox), G_BM, 1};
         if (encode_tmap_3d(&tmA, esz, Abase, dims, str, box)) return cudaErrorInvalidValue;
     }
     {
@@ -258,16 +394,22 @@ static cudaError_t launch_tc_cfg(const GemmArgs &a, cudaStream_t s)
                            static_cast<uint64_t>(a.b_gstride > 0 ? a.b_gstride
                                                                  : static_cast<long long>(a.N) * a.K) *
                                esz};
-        uint32_t box[3] = {static_cast<uint32_t>(kbox), static_cast<uint32_t>(BN), 1};
+        uint32_t box[3] = {static_cast<uint32_t>(kbox), G_BN, 1};
         if (encode_tmap_3d(&tmB, esz, a.B, dims, str, box)) return cudaErrorInvalidValue;
     }
-    const size_t smem = 1024 + STAGES * (TC_BM + BN) * TC_ROW_BYTES + 256;
-    auto kern = gemm_tc_kernel<BN, STAGES, FP8>;
+    if (g_num_sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            g_num_sms < 1)
+            g_num_sms = 148;
+    }
+    auto kern = gemm_tc_kernel<FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+                                         static_cast<int>(G_SMEM));
     if (e != cudaSuccess) return e;
-    dim3 grid(a.N / BN, (a.M + TC_BM - 1) / TC_BM, a.G);
-    kern<<<grid, 192, smem, s>>>(tmA, tmB, p);
+    const long long grid = p.tiles < g_num_sms ? p.tiles : g_num_sms;
+    kern<<<static_cast<int>(grid), G_THREADS, G_SMEM, s>>>(tmA, tmB, p);
     return cudaGetLastError();
 }
 
@@ -275,14 +417,11 @@ cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s)
 {
     const bool fp8 = a.in_dtype == OT_DTYPE_FP8;
     if (a.store != OT_STORE_BF16) return cudaErrorInvalidValue;
-    if (a.K % (fp8 ? 128 : 64) != 0 || a.a_map.P != 1) return cudaErrorInvalidValue;
-    if (a.N % 128 == 0) {
-        return fp8 ? launch_tc_cfg<128, 4, true>(a, s) : launch_tc_cfg<128, 3, false>(a, s);
-    }
-    if (a.N % 64 == 0) {
-        return fp8 ? launch_tc_cfg<64, 4, true>(a, s) : launch_tc_cfg<64, 4, false>(a, s);
-    }
-    return cudaErrorInvalidValue;
+    if (a.K % (fp8 ? 128 : 64) != 0 || a.a_map.P != 1 || a.N % G_BN != 0 || a.M < 1)
+        return cudaErrorInvalidValue;
+    for (int i = 0; i < a.nseg; ++i)
+        if (a.seg[i].c_lo % G_BN || a.seg[i].c_hi % G_BN) return cudaErrorInvalidValue;
+    return fp8 ? launch_tc_cfg<true>(a, s) : launch_tc_cfg<false>(a, s);
 }
 
 } // namespace ot
