@@ -152,6 +152,33 @@ ot_status ot_encode_user(ot_model *m, const void *S, int U, void *kv_cache, void
 ot_status ot_score_candidates(ot_model *m, const void *kv_cache, int U, const void *ns, int C,
                               void *out_ns, void *ws, size_t ws_bytes, void *stream);
 
+/* Capacity of the scratch array used by ot_score_candidates_noalloc (bytes). */
+#define OT_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* ot_score_candidates for callers that cannot allocate device memory (a
+ * serving runtime that forbids allocation on its request path, a caller in
+ * the middle of stream capture, a host that owns all GPU memory through its
+ * own pool).  The pages have no counterpart: this is a deployment variant of
+ * the NS-side call, computing exactly what ot_score_candidates computes.
+ * Same arguments minus the workspace: the scratch is a fixed device array of
+ * OT_NOALLOC_SCRATCH_BYTES inside the library's device image, present on
+ * every GPU that loads the library until the process exits.  The call makes
+ * no cudaMalloc / cudaFree or other allocating call.
+ *   - The model's device must be current.  The first call on a device looks
+ *     up the array's address there (cudaGetSymbolAddress); make that first
+ *     call before any stream capture.
+ *   - All calls on a device share the array; concurrent calls (other
+ *     streams or threads) race on it and must be serialised by the caller.
+ *     Contents persist between calls; the path never reads scratch it has
+ *     not written in the same call.
+ * Errors: OT_ERR_WORKSPACE_TOO_SMALL when U * C * N rows need more scratch
+ * than OT_NOALLOC_SCRATCH_BYTES (the bytes ot_score_candidates would need
+ * are 7 * rows * d + rows * ffn storage elements, fp8 adds rows * max(d, ffn)
+ * + 4 * rows); OT_ERR_UNSUPPORTED while per-launch profiling is enabled;
+ * OT_ERR_ARG if another device is current; otherwise as ot_score_candidates. */
+ot_status ot_score_candidates_noalloc(ot_model *m, const void *kv_cache, int U, const void *ns,
+                                      int C, void *out_ns, void *stream);
+
 /* Training-style batch: B users with C candidates each, S and NS in one
  * call.  S device [B][L0][d], ns device [B][C][N][d] -> out_s_tail device
  * [B][q_last][d], out_ns device [B][C][N][d]; the S K/V go to kv_cache if

@@ -65,6 +65,7 @@ SIGNATURES = {
     "ot_launch_count": (_ll, [_vp]),
     "ot_profile_enable": (_i, [_vp, _i]),
     "ot_profile_read": (_i, [_vp, C.POINTER(OtLaunchRecord), _i]),
+    "ot_score_candidates_noalloc": (_i, [_vp, _vp, _i, _vp, _i, _vp, _vp]),
 }
 
 _lib = None
@@ -262,6 +263,18 @@ class Model:
         check(lib().ot_score_candidates(self.handle, _ptr(kv), U, _ptr(ns), Cn, _ptr(out),
                                         _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
               "ot_score_candidates")
+        return out
+
+    def score_candidates_noalloc(self, kv, ns, out=None, stream=None):
+        """score_candidates into the library's fixed device scratch (no
+        workspace, no allocation inside the call); see the header for the
+        size limit and the sharing rules."""
+        import torch
+        U, Cn = ns.shape[0], ns.shape[1]
+        if out is None:
+            out = torch.empty_like(ns)
+        check(lib().ot_score_candidates_noalloc(self.handle, _ptr(kv), U, _ptr(ns), Cn, _ptr(out),
+                                                _stream(stream)), "ot_score_candidates_noalloc")
         return out
 
     def full_forward(self, S, ns, kv=None, out_s_tail=None, out_ns=None, ws=None, stream=None):

@@ -90,6 +90,10 @@ int encode_tmap_3d(void *map, int esz, const void *base, const uint64_t dims[3],
     return r != CUDA_SUCCESS;
 }
 
+int internal_profiling(const ot_model *m) { return m->profiling; }
+
+int internal_device(const ot_model *m) { return m->device; }
+
 } // namespace ot
 
 using namespace ot;
@@ -586,6 +590,14 @@ ot_status device_quant(ot_model *m, void **dst, float **scales, const void *W, l
 }
 
 } // namespace
+
+namespace ot {
+size_t internal_score_ws_bytes(const ot_model *m, int users, int cands)
+{
+    if (!m || users < 1 || cands < 1) return 0;
+    return score_ws_bytes(m->cfg, users, cands, m->esz);
+}
+} // namespace ot
 
 extern "C" {
 

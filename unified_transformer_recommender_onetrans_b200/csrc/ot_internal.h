@@ -113,6 +113,11 @@ cudaError_t launch_quant_rows(const void *X, long long lda, RowMap map, long lon
 cudaError_t launch_quant_weights(const void *W, long long per_mat, long long mats, uint8_t *q_out,
                                  float *scale_out, float *amax_scratch, cudaStream_t s);
 
+// Read-only model queries for entry points defined outside ot_api.cu.
+int internal_profiling(const ot_model *m);
+int internal_device(const ot_model *m);
+size_t internal_score_ws_bytes(const ot_model *m, int users, int cands);
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point.
 int encode_tmap_3d(void *map, int dtype_bytes, const void *base, const uint64_t dims[3],
                    const uint64_t strides_bytes[2], const uint32_t box[3]);
