@@ -120,12 +120,14 @@ def test_kv_cache_equivalence_and_candidate_independence(small_case):
     sc = m.score_candidates(kv2, nsd)
     m.poll()
     assert torch.equal(kv2, kv) and torch.equal(s2, s_tail) and torch.equal(sc, ns_out)
-    # a candidate scored alone matches the same candidate inside the batch
+    # a candidate scored alone matches the same candidate inside the batch, up
+    # to the bf16 rounding of values whose summation order depends on how the
+    # candidate's NS keys fall into key blocks (two bf16 ulps, 2 * 2^-8)
     for c in (0, 3, 6):
         alone = m.score_candidates(kv2, nsd[:, c:c + 1].contiguous())
         m.poll()
         err = O.rel_l2(alone[:, 0].double().cpu().numpy(), ns_out[:, c].double().cpu().numpy())
-        assert err < 1e-3, (c, err)
+        assert err < 2 * 2.0 ** -8, (c, err)
 
 
 def test_encode_without_tail_writes_same_cache(small_case):

@@ -35,14 +35,23 @@
 
 namespace ot {
 
-constexpr int G_BM = 128, G_BN = 128, G_STAGES = 6;
+constexpr int G_BM = 128;
 constexpr int G_EPI_WARPS = 8, G_NORM_WARPS = 4;
 constexpr int G_THREADS = 32 * (2 + G_EPI_WARPS + G_NORM_WARPS);
-constexpr uint32_t G_TILE = 128 * 128;          // one stage operand: 128 rows x 128 bytes
-constexpr uint32_t G_EPI_COLS = G_BN / 2;       // each epilogue warp: 32 rows x 64 columns
-constexpr uint32_t G_STAGING = 32 * G_EPI_COLS * 2;
-constexpr size_t G_SMEM = 1024 + 2 * G_STAGES * G_TILE + G_EPI_WARPS * G_STAGING +
-                          2 * G_BM * sizeof(float) + 256;
+constexpr uint32_t G_ROWB = 128;                // bytes of K per operand row per stage
+
+// Tile shapes: 128 x BN.  BN = 256 reads 96 B of operands from shared memory
+// per MMA clock instead of 128 B for BN = 128 (the A tile is reused across
+// twice the columns), leaving bandwidth for the TMA fills and the epilogue.
+template <int BN> struct GemmShape {
+    static constexpr int STAGES = BN == 256 ? 3 : 6;
+    static constexpr uint32_t A_BYTES = G_BM * G_ROWB;
+    static constexpr uint32_t B_BYTES = BN * G_ROWB;
+    static constexpr int EPI_COLS = BN / 2;                    // per epilogue warp
+    static constexpr uint32_t STAGING = 32 * EPI_COLS * 2;     // 32 rows x EPI_COLS bf16
+    static constexpr size_t SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + G_EPI_WARPS * STAGING +
+                                   2 * G_BM * sizeof(float) + 256;
+};
 
 struct TcGemmParams {
     GemmArgs a;
@@ -62,20 +71,22 @@ __device__ __forceinline__ float gelu_poly(float z)
     return z * fmaf(zc, p, 0.5f);
 }
 
-__device__ __forceinline__ void decode_tile(const TcGemmParams &P, long long tile, int &g, int &m0,
-                                            int &n0)
+__device__ __forceinline__ void decode_tile(const TcGemmParams &P, long long tile, int bn, int &g,
+                                            int &m0, int &n0)
 {
     const int nt = static_cast<int>(tile % P.n_tiles);
     const long long rest = tile / P.n_tiles;
     m0 = static_cast<int>(rest % P.m_tiles) * G_BM;
     g = static_cast<int>(rest / P.m_tiles);
-    n0 = nt * G_BN;
+    n0 = nt * bn;
 }
 
-// staging layout: row r (0..31) is 128 bytes, 16-byte chunk c stored at c ^ (r & 7)
+// staging layout: row r (0..31) is ROWB bytes, 16-byte chunk c stored at
+// (c & ~7) | ((c ^ r) & 7), so 8 consecutive rows hit 8 different bank groups
+template <int ROWB>
 __device__ __forceinline__ uint4 *stage_chunk(uint8_t *stage, int r, int c)
 {
-    return reinterpret_cast<uint4 *>(stage + r * (G_EPI_COLS * 2) + ((c ^ (r & 7)) << 4));
+    return reinterpret_cast<uint4 *>(stage + r * ROWB + (((c & ~7) | ((c ^ r) & 7)) << 4));
 }
 
 // Row map with 32-bit quotient / remainder (rows and periods fit in 31 bits).
@@ -93,11 +104,17 @@ __device__ __forceinline__ bool rowmap_keep_dev(const RowMap &m, int r)
     return static_cast<long long>(static_cast<unsigned>(r) % P) >= m.min_t;
 }
 
-template <bool FP8>
+template <int BN, bool FP8>
 __global__ void __launch_bounds__(G_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ TcGemmParams P)
 {
+    using Sh = GemmShape<BN>;
+    constexpr int G_STAGES = Sh::STAGES;
+    constexpr int G_BN = BN;
+    constexpr int G_EPI_COLS = Sh::EPI_COLS;
+    constexpr uint32_t G_STAGING = Sh::STAGING;
+    constexpr int ROWB = G_EPI_COLS * 2; // staging row bytes
     constexpr uint32_t IDESC = make_idesc(G_BM, G_BN, FP8 ? 0 : 1, 0, 0);
     const GemmArgs &a = P.a;
 
@@ -105,8 +122,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     uint8_t *sA = smem;
-    uint8_t *sB = sA + G_STAGES * G_TILE;
-    uint8_t *sOut = sB + G_STAGES * G_TILE;
+    uint8_t *sB = sA + G_STAGES * Sh::A_BYTES;
+    uint8_t *sOut = sB + G_STAGES * Sh::B_BYTES;
     float *ssbuf = reinterpret_cast<float *>(sOut + G_EPI_WARPS * G_STAGING); // [2][128]
     uint64_t *full = reinterpret_cast<uint64_t *>(ssbuf + 2 * G_BM);
     uint64_t *empty = full + G_STAGES;
@@ -121,6 +138,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_kb = a.K / (FP8 ? 128 : 64);
     const bool norm = a.norm != 0 && !FP8;
+    pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < G_STAGES; ++s) {
@@ -150,6 +168,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     // waits at the end ignore the abort flag and never use a test-lowered limit
     const WaitCtl final_wait{a.wait.err, a.wait.limit > (1LL << 24) ? a.wait.limit : (1LL << 24)};
     volatile int no_abort = 0;
+    pdl_wait(); // prologue done; from here on the previous kernel's memory is read / written
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -158,18 +177,18 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             bool ok = true;
             for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x) {
                 int g, m0, n0;
-                decode_tile(P, tile, g, m0, n0);
+                decode_tile(P, tile, G_BN, g, m0, n0);
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const int s = static_cast<int>(it % G_STAGES);
                     const uint32_t ph = static_cast<uint32_t>((it / G_STAGES) & 1);
                     if (!mbar_wait(&empty[s], ph ^ 1, a.wait, abort_flag)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&full[s], 2 * G_TILE);
+                    mbar_arrive_expect_tx(&full[s], Sh::A_BYTES + Sh::B_BYTES);
                     const int kx = kb * (FP8 ? 128 : 64);
                     if (P.a_grouped)
-                        tma_load_3d(sA + s * G_TILE, &tmA, &full[s], kx, g, m0);
+                        tma_load_3d(sA + s * Sh::A_BYTES, &tmA, &full[s], kx, g, m0);
                     else
-                        tma_load_3d(sA + s * G_TILE, &tmA, &full[s], kx, m0, 0);
-                    tma_load_3d(sB + s * G_TILE, &tmB, &full[s], kx, n0, g);
+                        tma_load_3d(sA + s * Sh::A_BYTES, &tmA, &full[s], kx, m0, 0);
+                    tma_load_3d(sB + s * Sh::B_BYTES, &tmB, &full[s], kx, n0, g);
                 }
             }
             // never leave a load in flight
@@ -196,8 +215,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(sA + s * G_TILE);
-                    const uint32_t b_addr = smem_u32(sB + s * G_TILE);
+                    const uint32_t a_addr = smem_u32(sA + s * Sh::A_BYTES);
+                    const uint32_t b_addr = smem_u32(sB + s * Sh::B_BYTES);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const uint64_t ad = sw128_desc(a_addr + k * 32, 16);
@@ -225,7 +244,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         int t = 0;
         for (long long tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++t) {
             int g, m0, n0;
-            decode_tile(P, tile, g, m0, n0);
+            decode_tile(P, tile, G_BN, g, m0, n0);
             const int b = t & 1;
             const int c0 = n0 + half * G_EPI_COLS; // first output column of this warp
             const int r = m0 + 32 * q + lane;      // this lane's row
@@ -238,16 +257,24 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             if (live && rowmap_keep_dev(sg.map, r))
                 out_off = rowmap_dev(sg.map, r, g) * sg.ld + (c0 - sg.c_lo);
             if (live && res) res_off = rowmap_dev(a.res_map, r, g) * a.res_ld + c0;
-            if (res) { // coalesced residual prefetch: 4 rows x 128 B per instruction
+            constexpr int LPR = ROWB / 16;       // lanes per staged row
+            constexpr int RPI = 32 / LPR;        // rows per warp instruction
+            if (res) {
+                // coalesced residual prefetch, RPI rows x ROWB bytes per instruction:
+                // every load is issued before the first shared-memory store, so
+                // the loads overlap instead of each waiting out the latency
+                uint4 rv[32 / RPI];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int rl = 4 * i + (lane >> 3), ch = lane & 7;
+                for (int i = 0; i < 32 / RPI; ++i) {
+                    const int rl = RPI * i + lane / LPR, ch = lane % LPR;
                     const long long ro = __shfl_sync(0xffffffffu, res_off, rl);
-                    uint4 v = make_uint4(0, 0, 0, 0);
+                    rv[i] = make_uint4(0, 0, 0, 0);
                     if (m0 + 32 * q + rl < a.M)
-                        v = *reinterpret_cast<const uint4 *>(res + ro + ch * 8);
-                    *stage_chunk(stage, rl, ch) = v;
+                        rv[i] = __ldg(reinterpret_cast<const uint4 *>(res + ro + ch * 8));
                 }
+#pragma unroll
+                for (int i = 0; i < 32 / RPI; ++i)
+                    *stage_chunk<ROWB>(stage, RPI * i + lane / LPR, lane % LPR) = rv[i];
             }
             if (!mbar_wait(&tfull[b], (t >> 1) & 1, a.wait, abort_flag)) break;
             tc_fence_after();
@@ -270,7 +297,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                 tmem_ld_wait();
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    uint4 *p = stage_chunk(stage, lane, 4 * c + j);
+                    uint4 *p = stage_chunk<ROWB>(stage, lane, 4 * c + j);
                     float f[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
@@ -297,14 +324,14 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[b]); // accumulator b may be overwritten
-            // coalesced stores: 8 lanes per row, 128 contiguous bytes
+            // coalesced stores: LPR lanes per row, ROWB contiguous bytes
             __nv_bfloat16 *obase = static_cast<__nv_bfloat16 *>(sg.out);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int rl = 4 * i + (lane >> 3), ch = lane & 7;
+            for (int i = 0; i < 32 / RPI; ++i) {
+                const int rl = RPI * i + lane / LPR, ch = lane % LPR;
                 const long long oo = __shfl_sync(0xffffffffu, out_off, rl);
                 if (oo < 0) continue;
-                *reinterpret_cast<uint4 *>(obase + oo + ch * 8) = *stage_chunk(stage, rl, ch);
+                *reinterpret_cast<uint4 *>(obase + oo + ch * 8) = *stage_chunk<ROWB>(stage, rl, ch);
             }
             __syncwarp(); // staging free for the next tile
         }
@@ -325,10 +352,12 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                     ok = false;
                     break;
                 }
-                const uint4 *src = reinterpret_cast<const uint4 *>(sA + s * G_TILE + row * 128);
+                const uint4 *src = reinterpret_cast<const uint4 *>(sA + s * Sh::A_BYTES + row * 128);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const uint4 v = src[c];
+                    // rotate the chunk order by lane: 8 neighbouring rows then read
+                    // 8 different bank groups (the row sum ignores the order)
+                    const uint4 v = src[(c + lane) & 7];
                     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -360,9 +389,11 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 
 static int g_num_sms = 0;
 
-template <bool FP8>
+template <int BN, bool FP8>
 static cudaError_t launch_tc_cfg(const GemmArgs &a, cudaStream_t s)
 {
+    constexpr int G_BN = BN;
+    using Sh = GemmShape<BN>;
     const int esz = FP8 ? 1 : 2;
     const int kbox = FP8 ? 128 : 64;
     alignas(64) CUtensorMap tmA, tmB;
@@ -404,24 +435,28 @@ static cudaError_t launch_tc_cfg(const GemmArgs &a, cudaStream_t s)
             g_num_sms < 1)
             g_num_sms = 148;
     }
-    auto kern = gemm_tc_kernel<FP8>;
+    auto kern = gemm_tc_kernel<BN, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(G_SMEM));
+                                         static_cast<int>(Sh::SMEM));
     if (e != cudaSuccess) return e;
     const long long grid = p.tiles < g_num_sms ? p.tiles : g_num_sms;
-    kern<<<static_cast<int>(grid), G_THREADS, G_SMEM, s>>>(tmA, tmB, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(G_THREADS), Sh::SMEM, s, tmA,
+                      tmB, p);
 }
 
 cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s)
 {
     const bool fp8 = a.in_dtype == OT_DTYPE_FP8;
     if (a.store != OT_STORE_BF16) return cudaErrorInvalidValue;
-    if (a.K % (fp8 ? 128 : 64) != 0 || a.a_map.P != 1 || a.N % G_BN != 0 || a.M < 1)
+    if (a.K % (fp8 ? 128 : 64) != 0 || a.a_map.P != 1 || a.N % 128 != 0 || a.M < 1)
         return cudaErrorInvalidValue;
-    for (int i = 0; i < a.nseg; ++i)
-        if (a.seg[i].c_lo % G_BN || a.seg[i].c_hi % G_BN) return cudaErrorInvalidValue;
-    return fp8 ? launch_tc_cfg<true>(a, s) : launch_tc_cfg<false>(a, s);
+    bool wide = a.N % 256 == 0;
+    for (int i = 0; i < a.nseg; ++i) {
+        if (a.seg[i].c_lo % 128 || a.seg[i].c_hi % 128) return cudaErrorInvalidValue;
+        if (a.seg[i].c_lo % 256 || a.seg[i].c_hi % 256) wide = false;
+    }
+    if (wide) return fp8 ? launch_tc_cfg<256, true>(a, s) : launch_tc_cfg<256, false>(a, s);
+    return fp8 ? launch_tc_cfg<128, true>(a, s) : launch_tc_cfg<128, false>(a, s);
 }
 
 } // namespace ot

@@ -98,6 +98,26 @@ struct AttnArgs {
     WaitCtl wait;
 };
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel in the stream finishes; it must call pdl_wait() before
+// touching global memory.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Launchers (return cudaGetLastError() after the launch).
 cudaError_t launch_gemm_simt(const GemmArgs &a, cudaStream_t s);
 cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s);
