@@ -163,6 +163,113 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- serving arms
+def _time_device(fn, steps, flush, world, dist, dev):
+    """Mean device ms of `fn` over `steps` calls (CUDA events on the current
+    stream, L2 flushed between calls), max over ranks."""
+    import torch
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for e0, e1 in ev:
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        flush.zero_()
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+def run_serving(name, steps, flush, world, dist, dev, peaks, cands=None):
+    """Encode once per user, then score every candidate against the cache
+    (Auto-Split of the candidates' features included in scoring)."""
+    import torch
+
+    import unified_transformer_recommender_onetrans_b200 as ot
+    from synth import (WORKLOADS, gen_auto_split_features, gen_embedding_table, gen_s_tokens,
+                       gen_weights, gen_zipf_ids)
+    from unified_transformer_recommender_onetrans_b200.binding import WEIGHT_NAMES
+
+    wl = WORKLOADS[name]
+    if cands is not None:
+        wl = wl.with_(cands=cands)
+    w = gen_weights(wl)
+    q = ot.pyramid_schedule(wl.L0, wl.q_end, wl.layers)
+    m = ot.Model(layers=wl.layers, d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns, L0=wl.L0,
+                 q=q, F=wl.F, eps=wl.eps, dtype=wl.dtype,
+                 weights={k: w[k].to(dev) for k in WEIGHT_NAMES})
+    U, C = wl.users, wl.cands
+    out = {"workload": name, "users": U, "cands": C, "dtype": wl.dtype}
+    if wl.zipf_s is not None:
+        table = gen_embedding_table(wl).to(dev)
+        ids = gen_zipf_ids(wl).to(dev)
+        S = torch.empty(U, wl.L0, wl.d, dtype=torch.bfloat16, device=dev)
+        gather = lambda: ot.embed_gather(table, ids, out=S)  # noqa: E731
+        del w
+    else:
+        S = gen_s_tokens(wl, weights=w).to(dev)
+        gather = None
+    x = gen_auto_split_features(wl).to(dev)
+    kv = m.new_kv_cache(U)
+    ws = torch.empty(max(m.workspace_bytes(U, 0), m.workspace_bytes(U, C)), dtype=torch.uint8,
+                     device=dev)
+    ns = torch.empty(U, C, wl.n_ns, wl.d, dtype=m.storage, device=dev)
+    out_ns = torch.empty_like(ns)
+
+    def encode():
+        if gather:
+            gather()
+        m.encode_user(S, kv=kv, ws=ws, want_s_tail=False)
+
+    def score():
+        m.auto_split(x, ns)
+        m.score_candidates(kv, ns, out=out_ns, ws=ws)
+
+    for _ in range(3):
+        encode()
+        score()
+    m.poll()
+    enc_ms = _time_device(encode, steps, flush, world, dist, dev)
+    sc_ms = _time_device(score, steps, flush, world, dist, dev)
+    m.poll()
+    # algorithmic work from the library's own per-launch accounting
+    m.profile(True)
+    encode()
+    enc_recs = m.profile_read()
+    score()
+    sc_recs = m.profile_read()
+    m.profile(False)
+    enc_flops = sum(r["flops"] for r in enc_recs)
+    sc_flops = sum(r["flops"] for r in sc_recs)
+    sc_bytes = sum(r["bytes"] for r in sc_recs)
+    # bytes a score call must move at least once: every NS weight, the users'
+    # cache, the candidates' features in and NS tokens out
+    d, f, N, L = wl.d, wl.ffn, wl.n_ns, wl.layers
+    wbytes = (1 if wl.dtype == "fp8" else 2) * L * N * (3 * d * d + d * d + 2 * d * f)
+    min_bytes = wbytes + m.kv_cache_bytes(U) + x.numel() * 2 + out_ns.numel() * 2 + \
+        N * d * wl.F * 2
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    out.update({
+        "encode_s_tokens_per_s": world * U * wl.L0 / (enc_ms / 1e3),
+        "encode_ms": enc_ms,
+        "encode_tflops": enc_flops / (enc_ms / 1e3) / 1e12,
+        "score_candidates_per_s": world * U * C / (sc_ms / 1e3),
+        "score_ms": sc_ms,
+        "score_tflops": sc_flops / (sc_ms / 1e3) / 1e12,
+        "score_min_hbm_bytes": min_bytes,
+        "score_hbm_gbs_min_bytes": min_bytes / (sc_ms / 1e3) / 1e9,
+        "score_hbm_frac": min_bytes / (sc_ms / 1e3) / 1e9 / hbm,
+        "score_launch_bytes_gbs": sc_bytes / (sc_ms / 1e3) / 1e9,
+    })
+    m.close()
+    return out
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, wl):
     import torch
@@ -287,8 +394,17 @@ def run_ours(args, wl):
     recs = m.profile_read()
     m.profile(False)
 
-    # ---- roofline of the dominant kernel (from the live per-launch events)
     peaks = load_peaks()
+    serving = []
+    if not args.no_serving:
+        del ws, kv
+        torch.cuda.empty_cache()
+        for name, cands in (("onetrans_s_serve", None), ("onetrans_l_full", 8), ("long_fp8", None)):
+            serving.append(run_serving(name, min(args.steps, 10), flush, world, dist, dev, peaks,
+                                       cands))
+            torch.cuda.empty_cache()
+
+    # ---- roofline of the dominant kernel (from the live per-launch events)
     by_kind, by_role = {}, {}
     for r in recs:
         for key, tab in ((r["kind"], by_kind), (r["role"], by_role)):
@@ -342,6 +458,7 @@ def run_ours(args, wl):
                     "ms_per_step": e2e_ms},
             "gpu_launches": launches,
             "clocks": clk,
+            "serving": serving,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -358,6 +475,7 @@ def main():
     ap.add_argument("--workload", default="onetrans_s_full")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-users", type=int, default=8)
+    ap.add_argument("--no-serving", action="store_true")
     args = ap.parse_args()
     args.steps_ref = max(1, min(args.steps, 3))
     args.warmup_ref = 0
