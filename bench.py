@@ -48,18 +48,57 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+    """SM clocks and clock-event (throttle) reasons sampled while active: the
+    nvidia-smi query loop (every 200 ms) plus an NVML poll every 10 ms, so a
+    timed region of a few tens of milliseconds still holds samples."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, uuid: str | None = None):
         self.gpu = gpu_index
+        self.uuid = uuid
         self.proc = None
-        self.lines = []
+        self.lines = []     # (host time, nvidia-smi csv line)
+        self.nvml = []      # (host time, sm MHz, max MHz, reason names)
+        self.t0, self.t1 = float("-inf"), float("inf")
+        self._stop = threading.Event()
+        self._poll = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.uuid:
+            try:
+                return pynvml, pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            except pynvml.NVMLError:
+                pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _poll_nvml(self):
+        try:
+            nv, h = self._nvml_handle()
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            while not self._stop.is_set():
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.nvml.append((time.monotonic(), sm, mx,
+                                  [k for k, v in bits.items() if r & v]))
+                self._stop.wait(0.01)
+        except Exception:  # NVML missing or refused: nvidia-smi samples remain
+            return
 
     def start(self):
+        """Start both samplers and wait (up to 10 s) for nvidia-smi's first
+        line, so sampling is running when the timed region opens."""
+        self._poll = threading.Thread(target=self._poll_nvml, daemon=True)
+        self._poll.start()
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
@@ -69,23 +108,34 @@ class ClockSampler:
             self.t.start()
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        t_end = time.monotonic() + 10.0
+        while not self.lines and time.monotonic() < t_end and self.proc.poll() is None:
+            time.sleep(0.02)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def window(self, t0: float, t1: float):
+        """Restrict the summary to samples taken between host times t0 and t1."""
+        self.t0, self.t1 = t0, t1
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.t.join(timeout=2)
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        self._stop.set()
+        if self._poll is not None:
+            self._poll.join(timeout=2)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+        sm, mx, reasons, n_smi = [], None, set(), 0
+        for ts, ln in self.lines:
+            if not self.t0 <= ts <= self.t1:
+                continue
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -94,12 +144,33 @@ class ClockSampler:
                 mx = float(parts[2])
             except ValueError:
                 continue
-            for nm, v in zip(names, parts[5:9]):
+            n_smi += 1
+            for nm, v in zip(self.NAMES, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(nm)
+        n_nvml = 0
+        for ts, f, m, rs in self.nvml:
+            if self.t0 <= ts <= self.t1:
+                sm.append(f)
+                mx = m
+                reasons.update(rs)
+                n_nvml += 1
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
         sm.sort()
-        med = sm[len(sm) // 2] if sm else None
-        return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "samples_nvidia_smi": n_smi, "samples_nvml": n_nvml,
+                "sm_mhz_min": sm[0]}
+
+
+def device_uuid(local: int):
+    """NVML-style UUID of the CUDA device `local`, or None."""
+    try:
+        import torch
+        u = str(torch.cuda.get_device_properties(local).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
 
 
 def dist_env():
@@ -137,19 +208,24 @@ def run_reference(args, wl):
     ws, rank, _ = dist_env()
     if rank != 0:
         return
-    # bounded sample: one user of the workload per step (about 10-30 s each)
+    # bounded sample: one user of the workload per step (under a second on a
+    # many-core host); the timed steps stop early after 150 s of oracle time
     per = []
     for _ in range(args.warmup_ref):
         oracle_sample(wl, users=1)
     cores = 0
+    spent = 0.0
     for _ in range(args.steps_ref):
         dt, toks, cores = oracle_sample(wl, users=1)
         per.append(dt / toks)
+        spent += dt
+        if spent > 150.0:
+            break
     sec_per_tok = sum(per) / len(per)
     value = 1.0 / sec_per_tok
     line = {
         "impl": "reference", "metric": "S-tokens/s (full forward)", "value": value,
-        "unit": "S-tokens/s", "n_gpus": ws, "steps": args.steps_ref, "warmup": args.warmup_ref,
+        "unit": "S-tokens/s", "n_gpus": ws, "steps": len(per), "warmup": args.warmup_ref,
         "ms_per_step": 1e3 * sec_per_tok * wl.L0, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "users": wl.users, "cands": wl.cands, "L0": wl.L0,
@@ -322,18 +398,20 @@ def run_ours(args, wl):
     # ---- device-timed steps, inputs resident in HBM, L2 flushed between steps
     clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
                           if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit()
-                          else local)
+                          else local, device_uuid(local))
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     launches0 = m.launch_count()
-    barrier()
     clocks.start()
+    barrier()
+    t_host0 = time.monotonic()
     for e0, e1 in ev:
         e0.record(stream)
         step()
         e1.record(stream)
         flush.zero_()
     barrier()
+    clocks.window(t_host0, time.monotonic())
     clk = clocks.stop()
     launches = m.launch_count() - launches0
     m.poll()
@@ -385,9 +463,10 @@ def run_ours(args, wl):
     # ---- per-kernel times: the same steps again with per-launch events on the
     # launching streams; profiling runs every kernel alone (no S/NS overlap),
     # so each event pair brackets exactly one kernel
+    prof_steps = min(args.steps, 20)
     m.profile(True)
     barrier()
-    for _ in range(args.steps):
+    for _ in range(prof_steps):
         step()
         flush.zero_()
     barrier()
@@ -420,15 +499,15 @@ def run_ours(args, wl):
     roofline = {"kernel": dom, "bound": "tensor", "achieved": tf, "peak": peak_tf,
                 "unit": "TFLOP/s", "frac": tf / peak_tf, "traffic": None,
                 "peak_source": f"{peaks['_source']} bf16 dense sustained",
-                "launches_per_step": dk["launches"] / args.steps,
-                "algorithmic_tflop_per_step": dk["flops"] / args.steps / 1e12}
-    step_flops = sum(v["flops"] for v in by_kind.values()) / args.steps
-    kernels = {k: {"ms_per_step": v["ms"] / args.steps,
+                "launches_per_step": dk["launches"] / prof_steps,
+                "algorithmic_tflop_per_step": dk["flops"] / prof_steps / 1e12}
+    step_flops = sum(v["flops"] for v in by_kind.values()) / prof_steps
+    kernels = {k: {"ms_per_step": v["ms"] / prof_steps,
                    "share": v["ms"] / max(sum(x["ms"] for x in by_kind.values()), 1e-9),
                    "tflops": v["flops"] / max(v["ms"], 1e-9) / 1e9,
                    "gbs": v["bytes"] / max(v["ms"], 1e-9) / 1e6}
                for k, v in by_kind.items()}
-    roles = {k: {"ms_per_step": v["ms"] / args.steps,
+    roles = {k: {"ms_per_step": v["ms"] / prof_steps,
                  "tflops": v["flops"] / max(v["ms"], 1e-9) / 1e9}
              for k, v in by_role.items()}
 
@@ -469,7 +548,7 @@ def run_ours(args, wl):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="onetrans_s_full")
@@ -477,8 +556,8 @@ def main():
     ap.add_argument("--cpu-users", type=int, default=8)
     ap.add_argument("--no-serving", action="store_true")
     args = ap.parse_args()
-    args.steps_ref = max(1, min(args.steps, 3))
-    args.warmup_ref = 0
+    args.steps_ref = max(1, args.steps)
+    args.warmup_ref = min(args.warmup, 3)
     from synth import WORKLOADS
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":
