@@ -90,6 +90,8 @@ __device__ __forceinline__ void softmax_pass(uint32_t tS_row, uint32_t tP_row, f
         tmem_ld32(tS_row + c, v[0]);
         tmem_ld32(tS_row + c + 32, v[1]);
         tmem_ld_wait();
+        tmem_reg_fence(v[0]);
+        tmem_reg_fence(v[1]);
         uint32_t pk[32]; // 64 keys as bf16 pairs: column c/2 + j holds keys c + 2j, c + 2j + 1
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
@@ -326,6 +328,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                         uint32_t v[32];
                         tmem_ld32(tS + lane_off + c, v);
                         tmem_ld_wait();
+                        tmem_reg_fence(v);
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
                             if (c + e >= klo && c + e <= khi) mraw = fmaxf(mraw, __uint_as_float(v[e]));
@@ -350,6 +353,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                             uint32_t v[32];
                             tmem_ld32(tO + lane_off + c, v);
                             tmem_ld_wait();
+                            tmem_reg_fence(v);
 #pragma unroll
                             for (int e = 0; e < 32; ++e)
                                 v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
@@ -377,6 +381,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             uint32_t v[32];
             tmem_ld32(tO + lane_off + c, v);
             tmem_ld_wait();
+            tmem_reg_fence(v);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[c + e] = __uint_as_float(v[e]);
         }

@@ -293,6 +293,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                               half * G_EPI_COLS + c * 32,
                           v);
                 tmem_ld_wait();
+                tmem_reg_fence(v);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     uint4 *p = stage_chunk<ROWB>(stage, lane, 4 * c + j);

@@ -229,6 +229,20 @@ __device__ __forceinline__ void tmem_ld_wait()
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Ties registers filled by tcgen05.ld to a point after tcgen05.wait::ld: an
+// empty statement that "modifies" them, so no use of them can be scheduled
+// before the wait (asm volatile statements keep their order).
+__device__ __forceinline__ void tmem_reg_fence(uint32_t (&r)[32])
+{
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                   "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                   "+r"(r[30]), "+r"(r[31]));
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled tile whose rows are
 // 128 bytes apart (8-row swizzle atoms of 1024 bytes, atom-aligned base).
 //   K-major operand: rows = M or N index, 128 bytes of K per row; SBO = 1024
