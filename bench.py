@@ -241,7 +241,7 @@ def run_reference(args, wl):
 
 # ---------------------------------------------------------------- serving arms
 def _time_device(fn, steps, flush, world, dist, dev):
-    """Mean device ms of `fn` over `steps` calls (CUDA events on the current
+    """Median device ms of `fn` over `steps` calls (CUDA events on the current
     stream, L2 flushed between calls), max over ranks."""
     import torch
     stream = torch.cuda.current_stream()
@@ -253,7 +253,8 @@ def _time_device(fn, steps, flush, world, dist, dev):
         e1.record(stream)
         flush.zero_()
     torch.cuda.synchronize()
-    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    t = sorted(a.elapsed_time(b) for a, b in ev)
+    ms = t[len(t) // 2]
     if world > 1:
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -261,9 +262,98 @@ def _time_device(fn, steps, flush, world, dist, dev):
     return ms
 
 
-def run_serving(name, steps, flush, world, dist, dev, peaks, cands=None):
+def _score_point(m, wl, U, C, x, kv, steps, flush, world, dist, dev, peaks, tensor_peak):
+    """Time score_candidates (with the candidates' Auto-Split) at C candidates
+    per user against an encoded cache; its roofline is the slower of the
+    bytes the call must move once over HBM and its FLOPs on the tensor cores."""
+    import torch
+
+    ns = torch.empty(U, C, wl.n_ns, wl.d, dtype=m.storage, device=dev)
+    out_ns = torch.empty_like(ns)
+    ws = torch.empty(m.workspace_bytes(U, C), dtype=torch.uint8, device=dev)
+
+    def score():
+        m.auto_split(x, ns)
+        m.score_candidates(kv, ns, out=out_ns, ws=ws)
+
+    for _ in range(10):
+        score()
+    m.poll()
+    ms = _time_device(score, steps, flush, world, dist, dev)
+    m.poll()
+    m.profile(True)
+    score()
+    recs = m.profile_read()
+    m.profile(False)
+    flops = sum(r["flops"] for r in recs)
+    gemm_flops = sum(r["flops"] for r in recs if r["kind"] != "attn_tc")
+    # bytes a score call must move at least once: every NS weight, the users'
+    # cache, the candidates' features in, NS tokens out and W_split
+    d, f, N, L = wl.d, wl.ffn, wl.n_ns, wl.layers
+    wbytes = (1 if wl.dtype == "fp8" else 2) * L * N * (3 * d * d + d * d + 2 * d * f)
+    min_bytes = wbytes + m.kv_cache_bytes(U) + x.numel() * 2 + out_ns.numel() * 2 + \
+        N * d * wl.F * 2
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    t_hbm = min_bytes / (hbm * 1e9)
+    # GEMMs at the GEMM dtype's peak, attention (always bf16) at the bf16 peak
+    t_tc = gemm_flops / (tensor_peak["gemm"] * 1e12) + \
+        (flops - gemm_flops) / (tensor_peak["attn"] * 1e12)
+    return {
+        "cands": C,
+        "candidates_per_s": world * U * C / (ms / 1e3),
+        "ms": ms,
+        "tflops": flops / (ms / 1e3) / 1e12,
+        "min_hbm_bytes": min_bytes,
+        "hbm_gbs_min_bytes": min_bytes / (ms / 1e3) / 1e9,
+        "hbm_frac": min_bytes / (ms / 1e3) / 1e9 / hbm,
+        "tensor_frac": t_tc / (ms / 1e3),
+        "bound": "hbm" if t_hbm >= t_tc else "tensor",
+        "roofline_ms": 1e3 * max(t_hbm, t_tc),
+        "roofline_frac": 1e3 * max(t_hbm, t_tc) / ms,
+    }
+
+
+def measure_fp8_peak(dev, n=8192, seconds=2.0):
+    """Dense e4m3 x e4m3 -> bf16 GEMM throughput of the library GEMM
+    (torch._scaled_mm, cuBLASLt), n^3: best of 10 (burst) and back to back
+    for `seconds` (sustained).  The denominator for the e4m3 GEMMs."""
+    import torch
+    try:
+        a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev)
+        mm = lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one,  # noqa: E731
+                                      out_dtype=torch.bfloat16)
+        for _ in range(3):
+            mm()
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            mm()
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(1, int(seconds * 1e3 / best))
+        e0.record()
+        for _ in range(reps):
+            mm()
+        e1.record()
+        torch.cuda.synchronize()
+        sus = e0.elapsed_time(e1) / reps
+        fl = 2.0 * n ** 3
+        return {"tflops_burst": fl / (best / 1e3) / 1e12, "tflops_sustained": fl / (sus / 1e3) / 1e12,
+                "how": f"torch._scaled_mm e4m3 {n}^3, best of 10 / {reps} back to back"}
+    except Exception as e:  # no fp8 GEMM in this torch build
+        return {"error": str(e).splitlines()[0][:200]}
+
+
+def run_serving(name, steps, flush, world, dist, dev, peaks, cands=None, sweep=None):
     """Encode once per user, then score every candidate against the cache
-    (Auto-Split of the candidates' features included in scoring)."""
+    (Auto-Split of the candidates' features included in scoring); with
+    `sweep`, score the same cache again at each candidate count in it."""
     import torch
 
     import unified_transformer_recommender_onetrans_b200 as ot
@@ -292,56 +382,50 @@ def run_serving(name, steps, flush, world, dist, dev, peaks, cands=None):
         gather = None
     x = gen_auto_split_features(wl).to(dev)
     kv = m.new_kv_cache(U)
-    ws = torch.empty(max(m.workspace_bytes(U, 0), m.workspace_bytes(U, C)), dtype=torch.uint8,
-                     device=dev)
-    ns = torch.empty(U, C, wl.n_ns, wl.d, dtype=m.storage, device=dev)
-    out_ns = torch.empty_like(ns)
+    ws = torch.empty(m.workspace_bytes(U, 0), dtype=torch.uint8, device=dev)
 
     def encode():
         if gather:
             gather()
         m.encode_user(S, kv=kv, ws=ws, want_s_tail=False)
 
-    def score():
-        m.auto_split(x, ns)
-        m.score_candidates(kv, ns, out=out_ns, ws=ws)
-
-    for _ in range(3):
+    for _ in range(10):
         encode()
-        score()
     m.poll()
     enc_ms = _time_device(encode, steps, flush, world, dist, dev)
-    sc_ms = _time_device(score, steps, flush, world, dist, dev)
     m.poll()
-    # algorithmic work from the library's own per-launch accounting
     m.profile(True)
     encode()
-    enc_recs = m.profile_read()
-    score()
-    sc_recs = m.profile_read()
+    enc_flops = sum(r["flops"] for r in m.profile_read())
     m.profile(False)
-    enc_flops = sum(r["flops"] for r in enc_recs)
-    sc_flops = sum(r["flops"] for r in sc_recs)
-    sc_bytes = sum(r["bytes"] for r in sc_recs)
-    # bytes a score call must move at least once: every NS weight, the users'
-    # cache, the candidates' features in and NS tokens out
-    d, f, N, L = wl.d, wl.ffn, wl.n_ns, wl.layers
-    wbytes = (1 if wl.dtype == "fp8" else 2) * L * N * (3 * d * d + d * d + 2 * d * f)
-    min_bytes = wbytes + m.kv_cache_bytes(U) + x.numel() * 2 + out_ns.numel() * 2 + \
-        N * d * wl.F * 2
-    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     out.update({
         "encode_s_tokens_per_s": world * U * wl.L0 / (enc_ms / 1e3),
         "encode_ms": enc_ms,
         "encode_tflops": enc_flops / (enc_ms / 1e3) / 1e12,
-        "score_candidates_per_s": world * U * C / (sc_ms / 1e3),
-        "score_ms": sc_ms,
-        "score_tflops": sc_flops / (sc_ms / 1e3) / 1e12,
-        "score_min_hbm_bytes": min_bytes,
-        "score_hbm_gbs_min_bytes": min_bytes / (sc_ms / 1e3) / 1e9,
-        "score_hbm_frac": min_bytes / (sc_ms / 1e3) / 1e9 / hbm,
-        "score_launch_bytes_gbs": sc_bytes / (sc_ms / 1e3) / 1e9,
     })
+    bf16_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    tensor_peak = {"gemm": bf16_peak, "attn": bf16_peak}
+    peak_note = f"{peaks['_source']} bf16 dense sustained"
+    if wl.dtype == "fp8":
+        fp8 = measure_fp8_peak(dev)
+        out["fp8_peak"] = fp8
+        if fp8.get("tflops_sustained"):
+            tensor_peak["gemm"] = fp8["tflops_sustained"]
+            peak_note += "; GEMMs: e4m3 measured here (cuBLASLt, sustained)"
+    del ws
+    pt = _score_point(m, wl, U, C, x, kv, steps, flush, world, dist, dev, peaks, tensor_peak)
+    out.update({"score_" + k: v for k, v in pt.items()})
+    out["score_peak_source"] = peak_note
+    if sweep:
+        out["score_c_sweep"] = []
+        for c in sweep:
+            wc = wl.with_(cands=c)
+            xc = gen_auto_split_features(wc).to(dev)
+            out["score_c_sweep"].append(
+                _score_point(m, wc, U, c, xc, kv, steps, flush, world, dist, dev, peaks,
+                             tensor_peak))
+            del xc
+            torch.cuda.empty_cache()
     m.close()
     return out
 
@@ -478,9 +562,11 @@ def run_ours(args, wl):
     if not args.no_serving:
         del ws, kv
         torch.cuda.empty_cache()
-        for name, cands in (("onetrans_s_serve", None), ("onetrans_l_full", 8), ("long_fp8", None)):
-            serving.append(run_serving(name, min(args.steps, 10), flush, world, dist, dev, peaks,
-                                       cands))
+        sweep = [1, 2, 4, 8, 16, 64, 512] if args.c_sweep else None
+        for name, cands, sw in (("onetrans_s_serve", None, sweep), ("onetrans_l_full", 8, sweep),
+                                ("long_fp8", None, None)):
+            # 10 warm-up calls, median of 50 per call
+            serving.append(run_serving(name, 50, flush, world, dist, dev, peaks, cands, sw))
             torch.cuda.empty_cache()
 
     # ---- roofline of the dominant kernel (from the live per-launch events)
@@ -555,6 +641,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-users", type=int, default=8)
     ap.add_argument("--no-serving", action="store_true")
+    ap.add_argument("--c-sweep", action="store_true",
+                    help="also score the serving caches at C = 1, 2, 4, 8, 16, 64, 512")
     args = ap.parse_args()
     args.steps_ref = max(1, args.steps)
     args.warmup_ref = min(args.warmup, 3)
