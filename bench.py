@@ -173,6 +173,26 @@ def device_uuid(local: int):
         return None
 
 
+def user_shard(world: int, rank: int, users_per_rank: int) -> range:
+    """The users rank `rank` of `world` works on: a disjoint block of
+    `users_per_rank` user indices (inputs are seeded per user, so a rank's
+    block is generated exactly as that slice of one big batch would be)."""
+    if not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside world of {world}")
+    return range(rank * users_per_rank, (rank + 1) * users_per_rank)
+
+
+def max_over_ranks(value: float, world: int, dist, device) -> float:
+    """The largest `value` over all ranks (every rank calls it, in the same
+    order); the step time of a weak-scaling job is the slowest rank's."""
+    if world == 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -254,12 +274,7 @@ def _time_device(fn, steps, flush, world, dist, dev):
         flush.zero_()
     torch.cuda.synchronize()
     t = sorted(a.elapsed_time(b) for a, b in ev)
-    ms = t[len(t) // 2]
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    return max_over_ranks(t[len(t) // 2], world, dist, dev)
 
 
 def _score_point(m, wl, U, C, x, kv, steps, flush, world, dist, dev, peaks, tensor_peak):
@@ -448,8 +463,9 @@ def run_ours(args, wl):
     dev = torch.device("cuda", local)
 
     w = gen_weights(wl)
-    S_cpu = gen_s_tokens(wl, weights=w)
-    x_cpu = gen_auto_split_features(wl)
+    shard = user_shard(world, rank, wl.users)
+    S_cpu = gen_s_tokens(wl, users=shard, weights=w)
+    x_cpu = gen_auto_split_features(wl, users=shard)
     q = ot.pyramid_schedule(wl.L0, wl.q_end, wl.layers)
     m = ot.Model(layers=wl.layers, d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns, L0=wl.L0,
                  q=q, F=wl.F, eps=wl.eps, dtype=wl.dtype,
@@ -500,11 +516,7 @@ def run_ours(args, wl):
     launches = m.launch_count() - launches0
     m.poll()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dist, dev)
     ms_per_step = total_ms / args.steps
     tokens_per_step = U * wl.L0 * world
     value = tokens_per_step / (ms_per_step / 1e3)
@@ -536,11 +548,8 @@ def run_ours(args, wl):
         e1.record(stream)
         flush.zero_()
     barrier()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2) / args.steps, world, dist,
+                            dev)
     h2d = S_h.numel() * S_h.element_size() + x_h.numel() * x_h.element_size()
     d2h = s_tail_h.numel() * s_tail_h.element_size() + out_ns_h.numel() * out_ns_h.element_size()
 
