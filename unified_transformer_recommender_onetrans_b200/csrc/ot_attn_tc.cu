@@ -56,18 +56,20 @@ constexpr int AT_STAGES = 6;              // K/V ring depth
 constexpr size_t AT_SMEM = (2 + 2 * AT_STAGES) * AT_TILE + 256;
 constexpr int AT_THREADS = 32 * (2 + 4 * AT_TILES);
 
-// 2^x on the FMA pipe: 2^floor(x) applied to the exponent field times a fitted
-// cubic for 2^f, f in [0, 1) (relative error < 1e-4).  Arguments below -126
-// are clamped (the result is then ~1e-38 instead of smaller).
+// 2^x on the FMA pipe: x = n + f with n the nearest integer (found by adding
+// and subtracting 1.5 * 2^23, which leaves n in the low mantissa bits), a
+// fitted cubic for 2^f on [-1/2, 1/2] (relative error < 7.5e-5), and n added
+// to the exponent field.  Arguments below -126 are clamped (the result is then
+// ~1e-38 instead of smaller); the softmax never passes more than 2^8.
 __device__ __forceinline__ float poly_exp2(float x)
 {
     x = fmaxf(x, -126.0f);
-    const float fl = floorf(x);
-    const float f = x - fl;
+    const float t = x + 12582912.0f;
+    const float f = x - (t - 12582912.0f);
     float p = fmaf(f, OT_EXP2_C3, OT_EXP2_C2);
     p = fmaf(f, p, OT_EXP2_C1);
-    p = fmaf(f, p, 1.0f);
-    return __int_as_float(__float_as_int(p) + (static_cast<int>(fl) << 23));
+    p = fmaf(f, p, OT_EXP2_C0);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 // Lazy rescale threshold (base-2): the running max moves only when it would
