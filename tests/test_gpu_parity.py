@@ -273,3 +273,25 @@ def test_onetrans_s_serving_sampled():
     errs = {"ns_out": O.rel_l2(out[users][:, cands].double().cpu().numpy(), out_o)}
     errs.update(kv_errors(m, kv[users], kv_o, cfg))
     assert_within(errs, TOL["bf16"])
+
+
+# ----------------------------------------------------------------- many items per CTA
+def test_bf16_many_items_per_cta():
+    """More (user, head, query pair) items than SMs in both attention modes, a
+    ragged last pair and a pyramid layer whose second query tile is empty:
+    every user against the CUDA-core path, sampled users against the oracle."""
+    layers, d, H, f, N, L0 = 3, 128, 2, 256, 5, 520
+    q = [520, 300, 45]
+    U, C = 90, 60                      # NS rows per user: 300 (two pairs)
+    w = rand_weights(layers, d, f, N, seed=31, dtype=torch.bfloat16)
+    S, ns = rand_inputs(U, C, L0, N, d, seed=32, dtype=torch.bfloat16)
+    m = make_model(w, layers=layers, d=d, heads=H, ffn=f, n_ns=N, L0=L0, q=q)
+    m.set_wait_limit(TEST_WAIT)
+    a = _run_full(m, S.cuda(), ns.cuda())
+    users = [0, 47, 89]
+    errs = _errors_vs_oracle(m, w, S, ns, *a, users)
+    assert_within(errs, TOL["bf16"])
+    m.set_kernel_path(1)
+    b = _run_full(m, S.cuda(), ns.cuda())
+    for x, y in zip(a, b):
+        assert O.rel_l2(x.double().cpu().numpy(), y.double().cpu().numpy()) < 1e-2

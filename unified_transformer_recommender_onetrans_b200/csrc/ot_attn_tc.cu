@@ -1,46 +1,49 @@
 // tcgen05 attention for one layer of the block (head_dim 64, bf16 operands,
-// fp32 scores and softmax).  One CTA = one (user, head) and two 128-query
-// tiles (256 consecutive query rows), one CTA per SM.
+// fp32 scores and softmax).  Persistent: one CTA per SM walks a list of work
+// items, each a (user, head) and two 128-query tiles (256 consecutive query
+// rows); the next item's Q and K/V loads and its first scores overlap the
+// current item's last blocks and output read-out.
 //
 // Key blocks of 128 rows are visited in order: first the user's S keys (from
-// the KV cache), then, in NS mode, the NS keys of the candidates the CTA's
+// the KV cache), then, in NS mode, the NS keys of the candidates the item's
 // rows belong to.  Visibility (the OneTrans mask):
 //   S mode  : query i is S row t = L - nq + i (the pyramid tail, bottom-right
-//             aligned); it sees S keys 0..t.  Blocks past the CTA's last row
+//             aligned); it sees S keys 0..t.  Blocks past the item's last row
 //             are never loaded.
 //   NS mode : query i is NS token n = i % N of candidate c = i / N; it sees
 //             every S key 0..L-1 and NS keys m <= n of candidate c.  Each
-//             cached S K/V tile is read once per CTA and shared by all the
-//             CTA's candidates (256 / N of them).
+//             cached S K/V tile is read once per item and shared by all the
+//             item's candidates (256 / N of them).
 //
-//   warp 0      TMA: both Q tiles once, K/V blocks through a 6-deep ring
-//               (shared memory holds only Q and K/V, so most of a CTA's keys
-//               are in flight at once).
-//   warp 1      TMEM (512 cols: S_0, S_1 at 0 / 128, O_0, O_1 at 256 / 320,
-//               P_0, P_1 at 384 / 448); lane 0 issues S_w = Q_w K^T (4 MMAs,
-//               both operands in shared memory) and O_w += P_w V (8 MMAs, P
-//               read from TMEM, V MN-major from its row-major tile).  After
-//               P_w(b) is ready it issues S_w(b+1) and then O_w(b), so the
-//               tensor core works for one warpgroup while the other runs its
-//               softmax.
-//   warps 2-5   softmax warpgroup of tile 0, warps 6-9 of tile 1: one query
-//               row per thread; scores from TMEM, running max / sum (base-2
-//               exponent with 1/sqrt(hd) folded in), P as packed bf16 into
-//               TMEM (tcgen05.st).  O accumulates in TMEM across key
-//               blocks.  Each block is one pass against the current running
-//               max, which is raised (O and l rescaled in place, the pass
-//               redone) only when a row's max grows by more than 2^8 -- after
-//               the first block that is rare, so most blocks read their scores
-//               once and touch no O.  Every fourth exponential is a
-//               polynomial on the FMA pipe, the rest use the special-function
-//               unit.  Warp-uniform fast paths: no mask arithmetic on blocks
-//               every row of the warp fully sees, no exponentials on blocks no
-//               row of the warp sees.
+// A tcgen05.mma issued from one thread takes about 100-130 cycles whatever
+// its N up to 128, so at head_dim 64 (12 MMAs per tile and key block) the
+// kernel is bound by MMA issue unless both tiles have their own issuer.
+//   warp 0      TMA: Q of both tiles into one of two Q buffers (item parity),
+//               K/V blocks through a 5-deep ring that runs on across items.
+//   warps 1, 2  MMA issuers of tiles 0 and 1 (warp 1 also owns the 512 TMEM
+//               columns: tile w uses S at 256 w, P at 256 w + 128, O at
+//               256 w + 192).  Per key block b: once the softmax holds S(b) in
+//               registers, S(b+1) = Q K^T (4 MMAs, operands in shared memory)
+//               goes into the S columns, overlapping the exponentials; once
+//               P(b) is stored, O += P(b) V (8 MMAs, P from TMEM, V MN-major
+//               from its row-major tile).  A tile with no live query row gets
+//               no MMAs, only the signals.
+//   warp 3      idle (it completes the producer warpgroup, whose registers
+//               go to the softmax warpgroups through setmaxnreg).
+//   warps 4-7   softmax warpgroup of tile 0, warps 8-11 of tile 1: one query
+//               row per thread, its 128 scores read from TMEM in one round
+//               trip; block max, lazy running max (O and l rescaled only when
+//               the max grows by more than 2^8), p = 2^(s c2 - m) on the
+//               special-function unit, P packed to bf16 into TMEM.  Warp-
+//               uniform fast paths: no mask arithmetic on blocks every row of
+//               the warp fully sees, no exponentials on blocks no row of the
+//               warp sees (or whose rows are all past nq).  At the end of an
+//               item the warpgroup reads O out of TMEM, frees it for the next
+//               item's first PV, and stores O / l.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
 
-#include "ot_exp2_poly.h"
 #include "ot_internal.h"
 #include "ot_ptx.cuh"
 
@@ -51,77 +54,157 @@ constexpr int AT_TILES = 2; // tiles per CTA
 constexpr int AT_BK = 128;  // keys per block
 constexpr int AT_HD = 64;
 constexpr uint32_t AT_TILE = AT_BM * 128; // 16 KB: 128 rows x 128 bytes
-constexpr int AT_STAGES = 6;              // K/V ring depth
-// Q[2], then per stage K and V, then barriers
-constexpr size_t AT_SMEM = (2 + 2 * AT_STAGES) * AT_TILE + 256;
-constexpr int AT_THREADS = 32 * (2 + 4 * AT_TILES);
-
-// 2^x on the FMA pipe: x = n + f with n the nearest integer (found by adding
-// and subtracting 1.5 * 2^23, which leaves n in the low mantissa bits), a
-// fitted cubic for 2^f on [-1/2, 1/2] (relative error < 7.5e-5), and n added
-// to the exponent field.  Arguments below -126 are clamped (the result is then
-// ~1e-38 instead of smaller); the softmax never passes more than 2^8.
-__device__ __forceinline__ float poly_exp2(float x)
-{
-    x = fmaxf(x, -126.0f);
-    const float t = x + 12582912.0f;
-    const float f = x - (t - 12582912.0f);
-    float p = fmaf(f, OT_EXP2_C3, OT_EXP2_C2);
-    p = fmaf(f, p, OT_EXP2_C1);
-    p = fmaf(f, p, OT_EXP2_C0);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
+constexpr int AT_STAGES = 5;              // K/V ring depth
+constexpr int AT_QBUF = 2;                // Q buffers (items in flight)
+// Q[AT_QBUF][AT_TILES], then per stage K and V, then barriers
+constexpr size_t AT_SMEM = (AT_QBUF * AT_TILES + 2 * AT_STAGES) * AT_TILE + 256;
+constexpr int AT_THREADS = 128 * (1 + AT_TILES); // producer warpgroup + one softmax warpgroup per tile
+// Register split (setmaxnreg): the producer warpgroup (TMA warp, MMA warp, two
+// idle warps) drops to AT_REG_PRODUCER per thread and the softmax warpgroups
+// rise to AT_REG_SOFTMAX, which holds a row's 128 scores at once.  The sum
+// must stay within what the launch allocated (registers per thread x
+// AT_THREADS); the launcher checks it against the compiled kernel.
+constexpr int AT_REG_PRODUCER = 64;
+constexpr int AT_REG_SOFTMAX = 216;
 
 // Lazy rescale threshold (base-2): the running max moves only when it would
 // grow by more than 2^8; until then p <= 2^8, well inside fp32 / bf16 range.
 constexpr float AT_RESCALE_LOG2 = 8.0f;
 
-// One pass over a row's 128 scores of a key block: p = 2^(s * c2 - m) for
-// visible keys (0 elsewhere), bf16 P into the row's 128-byte-swizzled slot,
-// sum of p and the max raw score seen.  FULL: every key of the block is
-// visible, so no mask arithmetic.  Every fourth exponential is the FMA-pipe
-// polynomial, the rest use the special-function unit.
-template <bool FULL, typename BeforeStore>
-__device__ __forceinline__ void softmax_pass(uint32_t tS_row, uint32_t tP_row, float c2, float m,
-                                             int klo, int khi, float &rsum, float &mraw,
-                                             BeforeStore &&before_store)
+// Softmax of one row of one key block against the running max m (base-2
+// units).  The row's 128 scores are read from TMEM in one round trip, after
+// which released() lets the MMA warp reuse the S columns; then
+//   1. the block's max over all 128 scores (keys the row cannot see included:
+//      a larger reference max leaves the softmax unchanged); m takes it on
+//      the row's first block and is raised later only when the block's max
+//      exceeds it by more than 2^8 (so p <= 2^8); alpha is the factor O and
+//      l must then be rescaled by, 1 otherwise;
+//   2. p = 2^(s c2 - m) for the visible keys [klo, khi], 0 elsewhere, packed
+//      to bf16 pairs (pk[q][j] holds keys 32 q + 2j, 32 q + 2j + 1) and
+//      summed into rsum.  FULL: every key of the block is visible (no mask).
+template <bool FULL, typename Released>
+__device__ __forceinline__ void softmax_unit(uint32_t tS_row, float c2, int klo, int khi, float &m,
+                                             uint32_t (&pk)[4][16], float &alpha, float &rsum,
+                                             Released &&released)
 {
-#pragma unroll 1
-    for (int c = 0; c < AT_BK; c += 64) {
-        uint32_t v[2][32];
-        tmem_ld32(tS_row + c, v[0]);
-        tmem_ld32(tS_row + c + 32, v[1]);
-        tmem_ld_wait();
-        tmem_reg_fence(v[0]);
-        tmem_reg_fence(v[1]);
-        uint32_t pk[32]; // 64 keys as bf16 pairs: column c/2 + j holds keys c + 2j, c + 2j + 1
+    uint32_t v[4][32];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int cc = c + 32 * hh;
-            float p[32];
+    for (int q = 0; q < 4; ++q) tmem_ld32(tS_row + 32 * q, v[q]);
+    tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const float sc = __uint_as_float(v[hh][e]);
-                const float x = fmaf(sc, c2, -m);
-                const float ex = (e & 3) == 3 ? poly_exp2(x) : fast_exp2(x);
-                if (FULL) {
-                    p[e] = ex;
-                    mraw = fmaxf(mraw, sc);
-                } else {
-                    const bool vis = cc + e >= klo && cc + e <= khi;
-                    p[e] = vis ? ex : 0.f;
-                    mraw = vis ? fmaxf(mraw, sc) : mraw;
-                }
-                rsum += p[e];
-            }
+    for (int q = 0; q < 4; ++q) tmem_reg_fence(v[q]);
+    released();
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int j = 0; j < 16; ++j) pk[16 * hh + j] = pack_bf16x2(p[2 * j], p[2 * j + 1]);
-        }
-        if (c == 0) before_store(); // P may be overwritten once the previous PV is done
-        tmem_st32(tP_row + c / 2, pk);
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[q][e]));
+    const float mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c2;
+    alpha = 1.f;
+    if (m == -INFINITY) {
+        m = mb; // the row's first block: l is 0 and O holds nothing for it
+    } else if (mb > m + AT_RESCALE_LOG2) {
+        alpha = fast_exp2(m - mb);
+        m = mb;
     }
-    tmem_st_wait();
+    const float mneg = -m;
+    float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            float p2[2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int k = 32 * q + 2 * j + t;
+                const float ex = fast_exp2(fmaf(__uint_as_float(v[q][2 * j + t]), c2, mneg));
+                p2[t] = (FULL || (k >= klo && k <= khi)) ? ex : 0.f;
+                rs[t + 2 * (j & 1)] += p2[t];
+            }
+            pk[q][j] = pack_bf16x2(p2[0], p2[1]);
+        }
+    rsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
 }
+
+// One work item of the persistent kernel: a (user, head, query pair) and its
+// key-block schedule, shared by every role of the CTA.
+struct AtItem {
+    int u, h, i0;     // user, head, first query row of the pair
+    int n_s_blocks;   // S key blocks
+    int k_begin;      // NS mode: first NS key row of the pair's candidates
+    int n_blocks;     // S blocks + NS blocks
+};
+
+// Item k.  S mode orders the pairs longest first (pairs later in the tail see
+// more keys), so the snake assignment below balances the CTAs; NS mode keeps
+// the pairs of one (user, head) together so they share K/V tiles in L2.
+template <bool NS>
+__device__ __forceinline__ AtItem at_item(const AttnArgs &a, int n_pairs, int k)
+{
+    AtItem it;
+    int pair, uh;
+    if (!NS) {
+        const int UH = a.U * a.H;
+        pair = n_pairs - 1 - k / UH;
+        uh = k % UH;
+    } else {
+        pair = k % n_pairs;
+        uh = k / n_pairs;
+    }
+    it.u = uh / a.H;
+    it.h = uh % a.H;
+    it.i0 = pair * (AT_BM * AT_TILES);
+    const int i_last = min(it.i0 + AT_BM * AT_TILES, a.nq) - 1;
+    it.k_begin = 0;
+    if (!NS) {
+        const int t_last = a.L - a.nq + i_last;
+        it.n_s_blocks = (t_last + AT_BK) / AT_BK;
+        it.n_blocks = it.n_s_blocks;
+    } else {
+        it.n_s_blocks = (a.L + AT_BK - 1) / AT_BK;
+        it.k_begin = (it.i0 / a.N) * a.N;
+        const int k_end = (i_last / a.N + 1) * a.N;
+        it.n_blocks = it.n_s_blocks + (k_end - it.k_begin + AT_BK - 1) / AT_BK;
+    }
+    return it;
+}
+
+// The r-th item of this CTA, or -1: rounds of gridDim.x items, walked
+// forwards in even rounds and backwards in odd ones (with longest-first items
+// every CTA then gets a similar total).
+__device__ __forceinline__ int at_item_of(int r, int n_items)
+{
+    const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+    const long long k = static_cast<long long>(r) * G + ((r & 1) ? G - 1 - c : c);
+    return k < n_items ? static_cast<int>(k) : -1;
+}
+
+// This CTA's key blocks in order, across its items.
+template <bool NS>
+struct BlockCursor {
+    int r, k;      // item ordinal within the CTA, item index (k < 0: past the end)
+    AtItem it;
+    int b;         // block within the item
+    long long gb;  // global block counter of the CTA
+    __device__ __forceinline__ void init(const AttnArgs &a, int n_pairs, int n_items)
+    {
+        r = 0;
+        b = 0;
+        gb = 0;
+        k = at_item_of(0, n_items);
+        if (k >= 0) it = at_item<NS>(a, n_pairs, k);
+    }
+    __device__ __forceinline__ void next(const AttnArgs &a, int n_pairs, int n_items)
+    {
+        ++gb;
+        if (++b < it.n_blocks) return;
+        b = 0;
+        k = at_item_of(++r, n_items);
+        if (k >= 0) it = at_item<NS>(a, n_pairs, k);
+    }
+    __device__ __forceinline__ bool valid() const { return k >= 0; }
+    __device__ __forceinline__ bool last_in_item() const { return b == it.n_blocks - 1; }
+};
 
 template <bool NS>
 __global__ void __launch_bounds__(AT_THREADS, 1)
@@ -133,49 +216,44 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     constexpr uint32_t IDESC_O = make_idesc(128, 64, 1, 0, 1);
 
     extern __shared__ __align__(1024) uint8_t smem[];
-    uint8_t *sQ = smem;                    // [2 tiles]
-    uint8_t *sKV = smem + 2 * AT_TILE;     // [stage][K | V]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (2 + 2 * AT_STAGES) * AT_TILE);
-    uint64_t *q_full = bars + 0;
-    uint64_t *kv_full = bars + 1;                  // [AT_STAGES]
-    uint64_t *kv_empty = kv_full + AT_STAGES;      // [AT_STAGES]
-    uint64_t *s_full = kv_empty + AT_STAGES;       // [2 tiles]
-    uint64_t *p_full = s_full + 2;                 // [2 tiles]
-    uint64_t *o_full = p_full + 2;                 // [2 tiles]
-    uint64_t *mma_done = o_full + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    uint8_t *sQ = smem;                                  // [AT_QBUF][AT_TILES]
+    uint8_t *sKV = smem + AT_QBUF * AT_TILES * AT_TILE;  // [stage][K | V]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sKV + 2 * AT_STAGES * AT_TILE);
+    uint64_t *q_full = bars;                       // [AT_QBUF]
+    uint64_t *q_empty = q_full + AT_QBUF;          // [AT_QBUF]   both MMA warps release
+    uint64_t *kv_full = q_empty + AT_QBUF;         // [AT_STAGES]
+    uint64_t *kv_empty = kv_full + AT_STAGES;      // [AT_STAGES] both MMA warps release
+    uint64_t *s_full = kv_empty + AT_STAGES;       // [tile] S computed
+    uint64_t *s_free = s_full + AT_TILES;          // [tile] S read into registers
+    uint64_t *p_full = s_free + AT_TILES;          // [tile] P stored
+    uint64_t *o_full = p_full + AT_TILES;          // [tile] PV completed
+    uint64_t *o_free = o_full + AT_TILES;          // [tile] O read out (end of an item)
+    uint64_t *mma_done = o_free + AT_TILES;        // [tile]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + AT_TILES);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int i0 = blockIdx.x * (AT_BM * AT_TILES), h = blockIdx.y, u = blockIdx.z;
+    const int n_pairs = (a.nq + AT_BM * AT_TILES - 1) / (AT_BM * AT_TILES);
+    const int n_items = n_pairs * a.U * a.H;
     pdl_launch_dependents();
-    const int i_last = min(i0 + AT_BM * AT_TILES, a.nq) - 1;
-
-    // key-block schedule, shared by both tiles
-    int n_s_blocks, k_begin = 0, n_blocks;
-    if (!NS) {
-        const int t_last = a.L - a.nq + i_last;
-        n_s_blocks = (t_last + AT_BK) / AT_BK;
-        n_blocks = n_s_blocks;
-    } else {
-        n_s_blocks = (a.L + AT_BK - 1) / AT_BK;
-        k_begin = (i0 / a.N) * a.N;
-        const int k_end = (i_last / a.N + 1) * a.N;
-        n_blocks = n_s_blocks + (k_end - k_begin + AT_BK - 1) / AT_BK;
-    }
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
+        for (int i = 0; i < AT_QBUF; ++i) {
+            mbar_init(&q_full[i], 1);
+            mbar_init(&q_empty[i], AT_TILES);
+        }
         for (int i = 0; i < AT_STAGES; ++i) {
             mbar_init(&kv_full[i], 1);
-            mbar_init(&kv_empty[i], 1);
+            mbar_init(&kv_empty[i], AT_TILES);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < AT_TILES; ++i) {
             mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], 4);
             mbar_init(&p_full[i], 4);
             mbar_init(&o_full[i], 1);
+            mbar_init(&o_free[i], 4);
+            mbar_init(&mma_done[i], 1);
         }
-        mbar_init(mma_done, 1);
         *abort_flag = 0;
         if (smem_u32(smem) & 1023) { // swizzle atoms need a 1024-byte aligned base
             *abort_flag = 1;
@@ -197,209 +275,260 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     const bool aborted_at_start = *abort_flag != 0;
     pdl_wait(); // prologue done; from here on the previous kernel's memory is read / written
 
+    if (warp < 4) {
+        // producer warpgroup: hand registers to the softmax warpgroups
+        setmaxnreg_dec<AT_REG_PRODUCER>();
+    }
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0 && !aborted_at_start) {
             tma_prefetch(&tmQ);
-            mbar_arrive_expect_tx(q_full, AT_TILES * AT_TILE);
-            for (int w = 0; w < AT_TILES; ++w)
-                tma_load_3d(sQ + w * AT_TILE, &tmQ, q_full, h * AT_HD, i0 + w * AT_BM, u);
-            int issued = 0;
-            for (int b = 0; b < n_blocks; ++b) {
-                const int st = b % AT_STAGES;
-                if (!mbar_wait(&kv_empty[st], ((b / AT_STAGES) & 1) ^ 1, a.wait, abort_flag)) break;
-                mbar_arrive_expect_tx(&kv_full[st], 2 * AT_TILE);
-                uint8_t *k_dst = sKV + 2 * st * AT_TILE, *v_dst = k_dst + AT_TILE;
-                if (b < n_s_blocks) {
-                    tma_load_3d(k_dst, &tmKS, &kv_full[st], h * AT_HD, b * AT_BK, u);
-                    tma_load_3d(v_dst, &tmVS, &kv_full[st], h * AT_HD, b * AT_BK, u);
-                } else {
-                    const int j0 = k_begin + (b - n_s_blocks) * AT_BK;
-                    tma_load_3d(k_dst, &tmKN, &kv_full[st], h * AT_HD, j0, u);
-                    tma_load_3d(v_dst, &tmVN, &kv_full[st], h * AT_HD, j0, u);
-                }
-                issued = b + 1;
+            tma_prefetch(&tmKS);
+            tma_prefetch(&tmVS);
+            if (NS) {
+                tma_prefetch(&tmKN);
+                tma_prefetch(&tmVN);
             }
-            mbar_wait(q_full, 0, final_wait, &no_abort);
-            for (int b = issued > AT_STAGES ? issued - AT_STAGES : 0; b < issued; ++b)
-                mbar_wait(&kv_full[b % AT_STAGES], (b / AT_STAGES) & 1, final_wait, &no_abort);
+            long long gb = 0; // global key-block counter of this CTA
+            int r = 0;        // items whose Q load was issued
+            bool ok = true;
+            for (; ok; ++r) {
+                const int k = at_item_of(r, n_items);
+                if (k < 0) break;
+                const AtItem it = at_item<NS>(a, n_pairs, k);
+                const int qb = r & 1;
+                // the Q buffer of item r - 2 is free once all its S MMAs completed
+                if (!mbar_wait(&q_empty[qb], ((r >> 1) & 1) ^ 1, a.wait, abort_flag)) break;
+                mbar_arrive_expect_tx(&q_full[qb], AT_TILES * AT_TILE);
+                for (int w = 0; w < AT_TILES; ++w)
+                    tma_load_3d(sQ + (qb * AT_TILES + w) * AT_TILE, &tmQ, &q_full[qb],
+                                it.h * AT_HD, it.i0 + w * AT_BM, it.u);
+                for (int b = 0; b < it.n_blocks; ++b, ++gb) {
+                    const int st = static_cast<int>(gb % AT_STAGES);
+                    if (!mbar_wait(&kv_empty[st], static_cast<uint32_t>((gb / AT_STAGES) & 1) ^ 1,
+                                   a.wait, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&kv_full[st], 2 * AT_TILE);
+                    uint8_t *k_dst = sKV + 2 * st * AT_TILE, *v_dst = k_dst + AT_TILE;
+                    if (b < it.n_s_blocks) {
+                        tma_load_3d(k_dst, &tmKS, &kv_full[st], it.h * AT_HD, b * AT_BK, it.u);
+                        tma_load_3d(v_dst, &tmVS, &kv_full[st], it.h * AT_HD, b * AT_BK, it.u);
+                    } else {
+                        const int j0 = it.k_begin + (b - it.n_s_blocks) * AT_BK;
+                        tma_load_3d(k_dst, &tmKN, &kv_full[st], it.h * AT_HD, j0, it.u);
+                        tma_load_3d(v_dst, &tmVN, &kv_full[st], it.h * AT_HD, j0, it.u);
+                    }
+                }
+                if (!ok) {
+                    ++r; // its Q load was issued
+                    break;
+                }
+            }
+            // never leave a load in flight: the last two Q loads, the last ring's K/V
+            for (int rr = r > AT_QBUF ? r - AT_QBUF : 0; rr < r; ++rr)
+                mbar_wait(&q_full[rr & 1], (rr >> 1) & 1, final_wait, &no_abort);
+            for (long long j = gb > AT_STAGES ? gb - AT_STAGES : 0; j < gb; ++j)
+                mbar_wait(&kv_full[j % AT_STAGES], static_cast<uint32_t>((j / AT_STAGES) & 1),
+                          final_wait, &no_abort);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer (ping-pong)
+    } else if (warp == 1 || warp == 2) {
+        // ------------------------------------------------ MMA issuer of tile w
+        // Issued from one thread, a short tcgen05.mma takes about 100 cycles:
+        // one issuer per tile keeps both tiles' MMAs flowing.  Per key block:
+        // once the softmax has S(b) in registers (s_free), S(b+1) = Q K^T goes
+        // into the S columns, so it runs while P(b) is being computed; then,
+        // once P(b) is stored (p_full), O += P(b) V.
+        const int w = warp - 1;
         if (lane == 0 && !aborted_at_start) {
-            const uint32_t q_addr = smem_u32(sQ);
-            auto issue_s = [&](int w, int b) {
-                const uint32_t k_addr = smem_u32(sKV + 2 * (b % AT_STAGES) * AT_TILE);
+            const uint32_t tS = tmem + w * 256, tP = tS + 128, tO = tS + 192;
+            auto live = [&](const AtItem &it) { return it.i0 + w * AT_BM < a.nq; };
+            auto issue_s = [&](const BlockCursor<NS> &c) {
+                if (live(c.it)) {
+                    const uint32_t q_addr = smem_u32(sQ + ((c.r & 1) * AT_TILES + w) * AT_TILE);
+                    const uint32_t k_addr = smem_u32(sKV + 2 * (c.gb % AT_STAGES) * AT_TILE);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_f16(tmem + w * 128, sw128_desc(q_addr + w * AT_TILE + k * 32, 16),
-                            sw128_desc(k_addr + k * 32, 16), IDESC_S, k != 0);
+                    for (int k = 0; k < 4; ++k)
+                        mma_f16(tS, sw128_desc(q_addr + k * 32, 16), sw128_desc(k_addr + k * 32, 16),
+                                IDESC_S, k != 0);
+                }
                 mma_commit(&s_full[w]);
+                // the item's last S of this tile: its Q buffer is free once they completed
+                if (c.last_in_item()) mma_commit(&q_empty[c.r & 1]);
             };
-            bool run = mbar_wait(q_full, 0, a.wait, abort_flag) &&
-                       mbar_wait(&kv_full[0], 0, a.wait, abort_flag);
+            auto ready_s = [&](const BlockCursor<NS> &c) {
+                return mbar_wait(&kv_full[c.gb % AT_STAGES], static_cast<uint32_t>((c.gb / AT_STAGES) & 1),
+                                 a.wait, abort_flag) &&
+                       mbar_wait(&q_full[c.r & 1], (c.r >> 1) & 1, a.wait, abort_flag);
+            };
+            BlockCursor<NS> cur;
+            cur.init(a, n_pairs, n_items);
+            bool run = cur.valid() && ready_s(cur);
             if (run) {
                 tc_fence_after();
-                issue_s(0, 0);
-                issue_s(1, 0);
+                issue_s(cur);
             }
-            for (int b = 0; run && b < n_blocks; ++b) {
-                const int st = b % AT_STAGES;
-                const uint32_t v_addr = smem_u32(sKV + (2 * st + 1) * AT_TILE);
-                for (int w = 0; run && w < AT_TILES; ++w) {
-                    if (!mbar_wait(&p_full[w], b & 1, a.wait, abort_flag)) { run = false; break; }
+            while (run) {
+                BlockCursor<NS> nxt = cur;
+                nxt.next(a, n_pairs, n_items);
+                if (nxt.valid()) {
+                    if (!mbar_wait(&s_free[w], static_cast<uint32_t>(cur.gb & 1), a.wait, abort_flag) ||
+                        !ready_s(nxt))
+                        break;
                     tc_fence_after();
-                    // the next scores first: the warpgroup can start block b+1
-                    // while O(b) is being accumulated
-                    if (b + 1 < n_blocks) {
-                        if (w == 0 && !mbar_wait(&kv_full[(b + 1) % AT_STAGES],
-                                                 ((b + 1) / AT_STAGES) & 1, a.wait, abort_flag)) {
-                            run = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        issue_s(w, b + 1);
-                    }
+                    issue_s(nxt);
+                }
+                if (!mbar_wait(&p_full[w], static_cast<uint32_t>(cur.gb & 1), a.wait, abort_flag)) break;
+                tc_fence_after();
+                // the first PV of an item overwrites O: the previous item's
+                // output has been read out by then (the warpgroup did that
+                // before computing P of this block)
+                if (cur.b == 0 && cur.r > 0) {
+                    if (!mbar_wait(&o_free[w], (cur.r - 1) & 1, a.wait, abort_flag)) break;
+                    tc_fence_after();
+                }
+                if (live(cur.it)) {
+                    const uint32_t v_addr = smem_u32(sKV + (2 * (cur.gb % AT_STAGES) + 1) * AT_TILE);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) // P from TMEM: 8 columns per 16 keys
-                        mma_f16_ts(tmem + 256 + w * 64, tmem + 384 + w * 64 + kk * 8,
-                                   sw128_desc(v_addr + kk * 2048, AT_TILE), IDESC_O, (b | kk) != 0);
-                    mma_commit(&o_full[w]);
-                    if (w == AT_TILES - 1) mma_commit(&kv_empty[st]);
+                        mma_f16_ts(tO, tP + kk * 8, sw128_desc(v_addr + kk * 2048, AT_TILE), IDESC_O,
+                                   (cur.b | kk) != 0);
                 }
+                mma_commit(&o_full[w]);
+                mma_commit(&kv_empty[cur.gb % AT_STAGES]);
+                if (!nxt.valid()) break;
+                cur = nxt;
             }
             // every issued MMA must be complete before TMEM is released
-            mma_commit(mma_done);
-            mbar_wait(mma_done, 0, final_wait, &no_abort);
+            mma_commit(&mma_done[w]);
+            mbar_wait(&mma_done[w], 0, final_wait, &no_abort);
         }
-    } else {
+    } else if (warp >= 4) {
         // ------------------------------------------------ softmax warpgroups
-        const int w = (warp - 2) >> 2;         // tile of this warpgroup
+        setmaxnreg_inc<AT_REG_SOFTMAX>();
+        const int w = (warp - 4) >> 2;         // tile of this warpgroup
         const int quarter = warp & 3;          // TMEM lane quarter
         const int row = quarter * 32 + lane;   // row within the tile
-        const int i = i0 + w * AT_BM + row;    // query row within the user
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        const uint32_t tS = tmem + w * 128, tO = tmem + 256 + w * 64, tP = tmem + 384 + w * 64;
+        const uint32_t tS = tmem + w * 256 + lane_off, tP = tS + 128, tO = tS + 192;
         const float c2 = a.scale * 1.4426950408889634f; // scores -> base-2 exponent
-        const int t_self = a.L - a.nq + i;              // S mode
-        const int my_c = NS ? i / a.N : 0, my_n = NS ? i % a.N : 0;
-        float m = -INFINITY, l = 0.f;
         bool ok = !aborted_at_start;
-        // wait for the PV of block j (completion j of this tile's o_full);
-        // PV(j + 1) cannot be issued before this warpgroup releases P(j + 1),
-        // so the wait never falls two phases behind
-        auto wait_o = [&](int j) {
-            if (ok && !mbar_wait(&o_full[w], j & 1, a.wait, abort_flag)) ok = false;
+        long long gb = 0;
+        // wait for the PV of this tile's global block jb (completion jb of
+        // o_full[w]).  Waiting twice for the same block is harmless: PV(jb + 1)
+        // is not issued before this warpgroup releases P(jb + 1), which it
+        // does only after observing PV(jb), so o_full is at most one phase
+        // ahead of every wait
+        auto wait_o = [&](long long jb) {
+            if (ok && !mbar_wait(&o_full[w], static_cast<uint32_t>(jb & 1), a.wait, abort_flag)) ok = false;
             tc_fence_after();
         };
-        for (int b = 0; ok && b < n_blocks; ++b) {
-            const bool s_block = b < n_s_blocks;
-            const int j0 = s_block ? b * AT_BK : k_begin + (b - n_s_blocks) * AT_BK;
-            // visible key range [klo, khi] of this row inside the block
-            int klo = 0, khi;
-            if (s_block) {
-                khi = NS ? min(a.L - 1 - j0, AT_BK - 1) : min(t_self - j0, AT_BK - 1);
-            } else {
-                const int first = my_c * a.N - j0; // key index of (my_c, 0)
-                klo = max(first, 0);
-                khi = min(first + my_n, AT_BK - 1);
-            }
-            const bool warp_full = __all_sync(0xffffffffu, klo <= 0 && khi >= AT_BK - 1);
-            const bool warp_none = __all_sync(0xffffffffu, khi < klo);
-            // P in TMEM was last read by O(b-1): wait for it just before overwriting
-            auto before_store = [&] {
-                if (b >= 1) wait_o(b - 1);
-            };
-            if (!mbar_wait(&s_full[w], b & 1, a.wait, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            if (warp_none) {
-                // no row of this warp sees the block: P = 0, state unchanged
-                uint32_t z[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) z[j] = 0u;
-                before_store();
-                tmem_st32(tP + lane_off, z);
-                tmem_st32(tP + lane_off + 32, z);
-                tmem_st_wait();
-            } else {
-                // a row with no max yet (its first visible block) needs one first
-                if (__any_sync(0xffffffffu, m == -INFINITY)) {
-                    float mraw = -INFINITY;
-#pragma unroll 1
-                    for (int c = 0; c < AT_BK; c += 32) {
-                        uint32_t v[32];
-                        tmem_ld32(tS + lane_off + c, v);
-                        tmem_ld_wait();
-                        tmem_reg_fence(v);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (c + e >= klo && c + e <= khi) mraw = fmaxf(mraw, __uint_as_float(v[e]));
-                    }
-                    if (m == -INFINITY) m = mraw * c2; // l is 0 and O holds nothing for this row
+        auto release = [&](uint64_t *bar) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
+        };
+        for (int r = 0; ok; ++r) {
+            const int k = at_item_of(r, n_items);
+            if (k < 0) break;
+            const AtItem it = at_item<NS>(a, n_pairs, k);
+            const int i = it.i0 + w * AT_BM + row;  // query row within the user
+            const bool warp_dead = __all_sync(0xffffffffu, i >= a.nq);
+            const int t_self = a.L - a.nq + i;      // S mode
+            const int my_c = NS ? i / a.N : 0, my_n = NS ? i % a.N : 0;
+            float m = -INFINITY, l = 0.f;
+            for (int b = 0; ok && b < it.n_blocks; ++b, ++gb) {
+                const bool s_block = b < it.n_s_blocks;
+                const int j0 = s_block ? b * AT_BK : it.k_begin + (b - it.n_s_blocks) * AT_BK;
+                // visible key range [klo, khi] of this row inside the block
+                int klo = 0, khi;
+                if (s_block) {
+                    khi = NS ? min(a.L - 1 - j0, AT_BK - 1) : min(t_self - j0, AT_BK - 1);
+                } else {
+                    const int first = my_c * a.N - j0; // key index of (my_c, 0)
+                    klo = max(first, 0);
+                    khi = min(first + my_n, AT_BK - 1);
                 }
-                // one pass against the current max; also track the raw max
-                float rsum = 0.f, mraw = -INFINITY;
-                if (warp_full)
-                    softmax_pass<true>(tS + lane_off, tP + lane_off, c2, m, 0, AT_BK - 1, rsum, mraw, before_store);
-                else
-                    softmax_pass<false>(tS + lane_off, tP + lane_off, c2, m, klo, khi, rsum, mraw, before_store);
-                const float m_cand = fmaxf(m, mraw * c2);
-                const bool raise = m_cand > m + AT_RESCALE_LOG2;
-                if (__any_sync(0xffffffffu, raise)) {
-                    // some row's max grew by more than 2^8: rescale O and l, redo P
-                    const float alpha = raise ? fast_exp2(m - m_cand) : 1.f;
-                    if (raise) m = m_cand;
-                    if (b > 0) { // O holds the blocks before b: the pass above waited for them
+                const bool warp_full = __all_sync(0xffffffffu, klo <= 0 && khi >= AT_BK - 1);
+                const bool warp_none = __all_sync(0xffffffffu, khi < klo);
+                if (!mbar_wait(&s_full[w], static_cast<uint32_t>(gb & 1), a.wait, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (warp_dead || warp_none) {
+                    // nothing of this warp's rows is visible (or no live row):
+                    // the scores are not read; a live warp stores P = 0
+                    release(&s_free[w]);
+                    if (b >= 1) wait_o(gb - 1);
+                    if (!warp_dead) {
+                        uint32_t z[32];
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) z[q] = 0u;
+                        tmem_st32(tP, z);
+                        tmem_st32(tP + 32, z);
+                        tmem_st_wait();
+                    }
+                } else {
+                    uint32_t pk[4][16];
+                    float alpha, rsum;
+                    if (warp_full)
+                        softmax_unit<true>(tS, c2, 0, AT_BK - 1, m, pk, alpha, rsum, [&] { release(&s_free[w]); });
+                    else
+                        softmax_unit<false>(tS, c2, klo, khi, m, pk, alpha, rsum, [&] { release(&s_free[w]); });
+                    // P(b) goes where PV(b - 1) read P(b - 1) from
+                    if (b >= 1) wait_o(gb - 1);
+                    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                        // some row raised its max: O holds this item's blocks before
+                        // b relative to the old max (their PV has completed)
 #pragma unroll
                         for (int c = 0; c < AT_HD; c += 32) {
                             uint32_t v[32];
-                            tmem_ld32(tO + lane_off + c, v);
+                            tmem_ld32(tO + c, v);
                             tmem_ld_wait();
                             tmem_reg_fence(v);
 #pragma unroll
                             for (int e = 0; e < 32; ++e)
                                 v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                            tmem_st32(tO + lane_off + c, v);
+                            tmem_st32(tO + c, v);
                         }
-                        tmem_st_wait();
                     }
-                    l *= alpha;
-                    rsum = 0.f;
-                    if (warp_full)
-                        softmax_pass<true>(tS + lane_off, tP + lane_off, c2, m, 0, AT_BK - 1, rsum, mraw, before_store);
-                    else
-                        softmax_pass<false>(tS + lane_off, tP + lane_off, c2, m, klo, khi, rsum, mraw, before_store);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) tmem_st16(tP + 16 * q, pk[q]);
+                    tmem_st_wait();
+                    l = l * alpha + rsum;
                 }
-                l += rsum;
+                release(&p_full[w]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[w]);
-        }
-        wait_o(n_blocks - 1); // the last PV
-        float o[AT_HD];
+            if (!ok) break;
+            wait_o(gb - 1); // the item's last PV
+            if (!ok) break;
+            // O / l as bf16 pairs, read 32 columns at a time
+            uint32_t ob[AT_HD / 2];
+            if (!warp_dead) {
+                const float inv = 1.f / l;
 #pragma unroll
-        for (int c = 0; c < AT_HD; c += 32) {
-            uint32_t v[32];
-            tmem_ld32(tO + lane_off + c, v);
-            tmem_ld_wait();
-            tmem_reg_fence(v);
+                for (int c = 0; c < AT_HD; c += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(tO + c, v);
+                    tmem_ld_wait();
+                    tmem_reg_fence(v);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[c + e] = __uint_as_float(v[e]);
-        }
-        if (ok && i < a.nq) {
-            const float inv = 1.f / l;
-            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.O) +
-                                 (static_cast<long long>(u) * a.nq + i) * a.d + h * AT_HD;
-            uint4 *dp = reinterpret_cast<uint4 *>(dst);
+                    for (int e = 0; e < 16; ++e)
+                        ob[c / 2 + e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv,
+                                                    __uint_as_float(v[2 * e + 1]) * inv);
+                }
+            }
+            // O may now be overwritten by the next item's first PV
+            release(&o_free[w]);
+            if (i < a.nq) {
+                uint4 *dp = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.O) +
+                                                      (static_cast<long long>(it.u) * a.nq + i) * a.d +
+                                                      it.h * AT_HD);
 #pragma unroll
-            for (int qd = 0; qd < 8; ++qd) {
-                uint4 wv;
-                wv.x = pack_bf16x2(o[qd * 8 + 0] * inv, o[qd * 8 + 1] * inv);
-                wv.y = pack_bf16x2(o[qd * 8 + 2] * inv, o[qd * 8 + 3] * inv);
-                wv.z = pack_bf16x2(o[qd * 8 + 4] * inv, o[qd * 8 + 5] * inv);
-                wv.w = pack_bf16x2(o[qd * 8 + 6] * inv, o[qd * 8 + 7] * inv);
-                dp[qd] = wv;
+                for (int qd = 0; qd < 8; ++qd)
+                    dp[qd] = make_uint4(ob[4 * qd], ob[4 * qd + 1], ob[4 * qd + 2], ob[4 * qd + 3]);
             }
         }
     }
@@ -437,8 +566,29 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
         tkn = tks;
         tvn = tvs;
     }
-    dim3 grid((a.nq + AT_BM * AT_TILES - 1) / (AT_BM * AT_TILES), a.H, a.U);
+    static int num_sms = 0;
+    if (num_sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            num_sms < 1)
+            num_sms = 148;
+    }
+    const long long items = static_cast<long long>((a.nq + AT_BM * AT_TILES - 1) / (AT_BM * AT_TILES)) *
+                            a.H * a.U;
+    if (items < 1 || items > (1LL << 30)) return cudaErrorInvalidValue;
+    dim3 grid(static_cast<unsigned>(items < num_sms ? items : num_sms));
     cudaError_t e;
+    // the setmaxnreg split must fit the registers the launch allocates, or the
+    // softmax warpgroups' increase would wait forever
+    {
+        cudaFuncAttributes fa;
+        e = a.mode == 1 ? cudaFuncGetAttributes(&fa, attn_tc_kernel<true>)
+                        : cudaFuncGetAttributes(&fa, attn_tc_kernel<false>);
+        if (e != cudaSuccess) return e;
+        if (128 * AT_REG_PRODUCER + 128 * AT_TILES * AT_REG_SOFTMAX > fa.numRegs * AT_THREADS)
+            return cudaErrorInvalidConfiguration;
+    }
     if (a.mode == 1) {
         e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(AT_SMEM));
