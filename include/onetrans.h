@@ -198,10 +198,13 @@ ot_status ot_poll_device_error(ot_model *m, void *stream);
 ot_status ot_set_wait_limit(ot_model *m, long long polls);
 
 /* Kernel family for the bf16 projections and attention: 0 = tcgen05
- * tensor-core kernels (default), 1 = the CUDA-core kernels the fp32 path
- * uses (slow; a second GPU implementation for cross-checks).  fp32 models
- * always use the CUDA-core kernels.  Errors: OT_ERR_ARG; OT_ERR_UNSUPPORTED
- * for path 1 on an fp8 model (the CUDA-core kernels read no e4m3). */
+ * tensor-core kernels (default; the feed-forward runs as one fused kernel
+ * where the width allows), 1 = the CUDA-core kernels the fp32 path uses
+ * (slow; a second GPU implementation for cross-checks), 2 = tensor-core
+ * kernels with the feed-forward as two separate GEMMs (cross-check of the
+ * fused kernel).  fp32 models always use the CUDA-core kernels.  Errors:
+ * OT_ERR_ARG; OT_ERR_UNSUPPORTED for path 1 on an fp8 model (the CUDA-core
+ * kernels read no e4m3). */
 ot_status ot_set_kernel_path(ot_model *m, int path);
 
 /* Per-launch timing for roofline reports.  While enabled, every kernel the
@@ -213,12 +216,13 @@ ot_status ot_set_kernel_path(ot_model *m, int path);
  * (negative on error).  Records beyond an internal 1 << 16 are dropped. */
 typedef enum {
     OT_KIND_GEMM_TC = 0, OT_KIND_GEMM_SIMT = 1, OT_KIND_ATTN_TC = 2, OT_KIND_ATTN_SIMT = 3,
-    OT_KIND_GATHER = 4, OT_KIND_QUANT = 5
+    OT_KIND_GATHER = 4, OT_KIND_QUANT = 5, OT_KIND_FFN_TC = 6 /* fused FFN1 + GELU + FFN2 */
 } ot_kernel_kind;
 
 typedef struct {
     int kind;      /* ot_kernel_kind */
-    int role;      /* 0 S-QKV, 1 S-attn, 2 S-O, 3 S-FFN1, 4 S-FFN2, 5..9 the NS ones, 10 Auto-Split, 11 other */
+    int role;      /* 0 S-QKV, 1 S-attn, 2 S-O, 3 S-FFN1, 4 S-FFN2, 5..9 the NS ones, 10 Auto-Split,
+                      11 other, 12 S-FFN (fused), 13 NS-FFN (fused) */
     float ms;      /* device time between the two events */
     double flops;  /* algorithmic floating-point operations */
     double bytes;  /* algorithmic HBM bytes */

@@ -295,3 +295,31 @@ def test_bf16_many_items_per_cta():
     b = _run_full(m, S.cuda(), ns.cuda())
     for x, y in zip(a, b):
         assert O.rel_l2(x.double().cpu().numpy(), y.double().cpu().numpy()) < 1e-2
+
+
+# ----------------------------------------------------------------- fused feed-forward
+@pytest.mark.parametrize("shape", ["small_d128", "onetrans_s_d256"])
+def test_fused_ffn_matches_two_gemm_path(shape):
+    """The fused FFN kernel (hidden kept on chip) against the two tensor-core
+    GEMMs it replaces (kernel path 2), on the S side and the grouped NS side:
+    same bf16 roundings of the hidden and the output, so they agree to within
+    the odd bf16 ulp from a different RMSNorm summation order."""
+    if shape == "small_d128":
+        w = rand_weights(3, 128, 256, 5, seed=41, dtype=torch.bfloat16)
+        S, ns = rand_inputs(5, 40, 300, 5, 128, seed=42, dtype=torch.bfloat16)
+        kw = SMALL
+    else:
+        wl = WORKLOADS["onetrans_s_full"]
+        kw = dict(layers=2, d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns, L0=600,
+                  q=[600, 300])
+        w = rand_weights(2, wl.d, wl.ffn, wl.n_ns, seed=43, dtype=torch.bfloat16)
+        S, ns = rand_inputs(6, 3, 600, wl.n_ns, wl.d, seed=44, dtype=torch.bfloat16)
+    m = make_model(w, **kw)
+    m.set_wait_limit(TEST_WAIT)
+    a = _run_full(m, S.cuda(), ns.cuda())
+    m.set_kernel_path(2)
+    b = _run_full(m, S.cuda(), ns.cuda())
+    for x, y in zip(a, b):
+        assert O.rel_l2(x.double().cpu().numpy(), y.double().cpu().numpy()) < 2e-3
+    errs = _errors_vs_oracle(m, w, S, ns, *a, [0, S.shape[0] - 1])
+    assert_within(errs, TOL["bf16"])

@@ -182,7 +182,7 @@ size_t score_ws_bytes(const ot_config &c, int U, int C, int esz)
 }
 
 enum { ROLE_S_QKV = 0, ROLE_S_ATTN, ROLE_S_O, ROLE_S_FFN1, ROLE_S_FFN2, ROLE_NS_QKV, ROLE_NS_ATTN,
-       ROLE_NS_O, ROLE_NS_FFN1, ROLE_NS_FFN2, ROLE_AUTO_SPLIT, ROLE_OTHER };
+       ROLE_NS_O, ROLE_NS_FFN1, ROLE_NS_FFN2, ROLE_AUTO_SPLIT, ROLE_OTHER, ROLE_S_FFN, ROLE_NS_FFN };
 
 cudaEvent_t pooled_event(ot_model *m)
 {
@@ -270,6 +270,43 @@ ot_status attn(ot_model *m, AttnArgs &a, cudaStream_t s)
                     a.mode == 0 ? ROLE_S_ATTN : ROLE_NS_ATTN, flops, bytes, [&] {
                         return simt ? launch_attn_simt(a, s) : launch_attn_tc(a, s);
                     });
+}
+
+// The fused FFN kernel runs for bf16 models on the tensor-core path (not for
+// path 2, which keeps the two FFN GEMMs for cross-checks) at supported widths.
+bool use_fused_ffn(const ot_model *m)
+{
+    return m->cfg.dtype == OT_DTYPE_BF16 && m->path == 0 && ffn_tc_supported(m->cfg.d, m->cfg.ffn);
+}
+
+// Y = H + GELU(n(H) W1^T) W2^T over G groups of M rows (gain folded into W1).
+ot_status ffn(ot_model *m, int M, int G, const void *H, RowMap h_map, const void *W1,
+              const void *W2, void *Y, RowMap y_map, cudaStream_t s, int role)
+{
+    const ot_config &c = m->cfg;
+    FfnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.M = M;
+    a.G = G;
+    a.D = c.d;
+    a.F = c.ffn;
+    a.H = H;
+    a.h_map = h_map;
+    a.W1 = W1;
+    a.w1_gstride = static_cast<long long>(c.ffn) * c.d;
+    a.W2 = W2;
+    a.w2_gstride = static_cast<long long>(c.d) * c.ffn;
+    a.Y = Y;
+    a.y_map = y_map;
+    a.eps = c.eps;
+    a.wait = WaitCtl{m->err, m->wait_limit};
+    double flops = 0, bytes = 0;
+    if (m->profiling) {
+        const double rows = static_cast<double>(M) * G, d = c.d, f = c.ffn;
+        flops = 4.0 * rows * d * f;
+        bytes = 2.0 * (2.0 * rows * d + 2.0 * G * d * f); // H in, Y out, W1 + W2 once
+    }
+    return profiled(m, s, OT_KIND_FFN_TC, role, flops, bytes, [&] { return launch_ffn_tc(a, s); });
 }
 
 GemmArgs gemm_base(const ot_config &c, int M, int N, int K, int G)
@@ -425,6 +462,15 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
         g.seg[0] = seg_of(Hb, d, 0, d, rowmap_identity());
         if ((r = gemm(m, g, st, ROLE_S_O)) != OT_OK) return r;
         // 4. FFN: RMSNorm2 + W1 + GELU, then W2 + residual
+        void *Xn = (last && s_out) ? s_out : Xb[l & 1];
+        if (use_fused_ffn(m)) {
+            if ((r = ffn(m, U * q, 1, Hb, rowmap_identity(), at(m->W1_s, static_cast<long long>(l) * f * d, esz),
+                         at(m->W2_s, static_cast<long long>(l) * d * f, esz), Xn, rowmap_identity(), st,
+                         ROLE_S_FFN)) != OT_OK)
+                return r;
+            X = Xn;
+            continue;
+        }
         g = gemm_base(c, U * q, f, d, 1);
         if ((r = projection(m, g, Hb, d, rowmap_identity(),
                             at(m->W1_s, static_cast<long long>(l) * f * d, wesz),
@@ -435,7 +481,6 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
         g.nseg = 1;
         g.seg[0] = seg_of(hid, f, 0, f, rowmap_identity());
         if ((r = gemm(m, g, st, ROLE_S_FFN1)) != OT_OK) return r;
-        void *Xn = (last && s_out) ? s_out : Xb[l & 1];
         g = gemm_base(c, U * q, d, f, 1);
         if ((r = projection(m, g, hid, f, rowmap_identity(),
                             at(m->W2_s, static_cast<long long>(l) * d * f, wesz),
@@ -527,6 +572,14 @@ ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, v
         g.nseg = 1;
         g.seg[0] = seg_of(Hn, d, 0, d, grp);
         if ((r = gemm(m, g, st, ROLE_NS_O)) != OT_OK) return r;
+        void *Xn = last ? out : Xb[l & 1];
+        if (use_fused_ffn(m)) {
+            if ((r = ffn(m, Mc, N, Hn, grp, at(m->W1_ns, lN * f * d, esz), at(m->W2_ns, lN * d * f, esz), Xn,
+                         grp, st, ROLE_NS_FFN)) != OT_OK)
+                return r;
+            X = Xn;
+            continue;
+        }
         g = gemm_base(c, Mc, f, d, N);
         if ((r = projection(m, g, Hn, d, grp, at(m->W1_ns, lN * f * d, wesz),
                             static_cast<long long>(f) * d, fp8 ? m->sc_1_ns + lN : nullptr, g2, d,
@@ -536,7 +589,6 @@ ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, v
         g.nseg = 1;
         g.seg[0] = seg_of(hid, f, 0, f, grp);
         if ((r = gemm(m, g, st, ROLE_NS_FFN1)) != OT_OK) return r;
-        void *Xn = last ? out : Xb[l & 1];
         g = gemm_base(c, Mc, d, f, N);
         if ((r = projection(m, g, hid, f, grp, at(m->W2_ns, lN * d * f, wesz),
                             static_cast<long long>(d) * f, fp8 ? m->sc_2_ns + lN : nullptr, nullptr,
@@ -773,7 +825,7 @@ ot_status ot_set_wait_limit(ot_model *m, long long polls)
 
 ot_status ot_set_kernel_path(ot_model *m, int path)
 {
-    if (!m || (path != 0 && path != 1)) return OT_ERR_ARG;
+    if (!m || path < 0 || path > 2) return OT_ERR_ARG;
     if (path == 1 && m->cfg.dtype == OT_DTYPE_FP8) return OT_ERR_UNSUPPORTED;
     m->path = path;
     return OT_OK;

@@ -98,6 +98,24 @@ struct AttnArgs {
     WaitCtl wait;
 };
 
+// Fused feed-forward over G groups of M rows:
+//   Y[row_y(r, g)] = H[row_h(r, g)] + GELU(n(H) W1[g]^T) W2[g]^T,
+// n(H) = H * rsqrt(mean(H^2) + eps) (the RMSNorm gain folded into W1).
+// H / Y rows are D wide; W1 is [G][F][D], W2 is [G][D][F] (bf16).
+struct FfnArgs {
+    int M, G, D, F;
+    const void *H;
+    RowMap h_map;
+    const void *W1;
+    long long w1_gstride;   // elements between groups of W1
+    const void *W2;
+    long long w2_gstride;   // elements between groups of W2
+    void *Y;
+    RowMap y_map;
+    float eps;
+    WaitCtl wait;
+};
+
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel in the stream finishes; it must call pdl_wait() before
 // touching global memory.
@@ -123,6 +141,8 @@ cudaError_t launch_gemm_simt(const GemmArgs &a, cudaStream_t s);
 cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s);
+bool ffn_tc_supported(int D, int F);
+cudaError_t launch_ffn_tc(const FfnArgs &a, cudaStream_t s);
 cudaError_t launch_fold_gain(const void *W, const void *g, void *out, long long rows, int cols,
                              long long groups, long long g_gstride, int dtype, cudaStream_t s);
 cudaError_t launch_embed_gather(const void *table, long long rows, int d, const int64_t *ids,
