@@ -300,26 +300,34 @@ def test_bf16_many_items_per_cta():
 # ----------------------------------------------------------------- fused feed-forward
 @pytest.mark.parametrize("shape", ["small_d128", "onetrans_s_d256"])
 def test_fused_ffn_matches_two_gemm_path(shape):
-    """The fused FFN kernel (hidden kept on chip) against the two tensor-core
-    GEMMs it replaces (kernel path 2), on the S side and the grouped NS side:
-    same bf16 roundings of the hidden and the output, so they agree to within
-    the odd bf16 ulp from a different RMSNorm summation order."""
+    """The fused FFN kernel (hidden kept on chip, residual seeded into the
+    fp32 accumulator) against the two tensor-core GEMMs it replaces (kernel
+    path 2), on the S side and the grouped NS side.  After one layer they
+    differ only in fp32 summation order (below 1e-3); through a pyramid of
+    layers the occasional different bf16 rounding of an intermediate
+    compounds, so the stack is held to two bf16 ulps (2 * 2^-8), and both to
+    the oracle tolerance."""
     if shape == "small_d128":
+        w1 = rand_weights(1, 128, 256, 5, seed=40, dtype=torch.bfloat16)
         w = rand_weights(3, 128, 256, 5, seed=41, dtype=torch.bfloat16)
         S, ns = rand_inputs(5, 40, 300, 5, 128, seed=42, dtype=torch.bfloat16)
+        kw1 = dict(SMALL, layers=1, q=[300])
         kw = SMALL
     else:
         wl = WORKLOADS["onetrans_s_full"]
-        kw = dict(layers=2, d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns, L0=600,
-                  q=[600, 300])
+        base = dict(d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns, L0=600)
+        w1 = rand_weights(1, wl.d, wl.ffn, wl.n_ns, seed=45, dtype=torch.bfloat16)
         w = rand_weights(2, wl.d, wl.ffn, wl.n_ns, seed=43, dtype=torch.bfloat16)
         S, ns = rand_inputs(6, 3, 600, wl.n_ns, wl.d, seed=44, dtype=torch.bfloat16)
-    m = make_model(w, **kw)
-    m.set_wait_limit(TEST_WAIT)
-    a = _run_full(m, S.cuda(), ns.cuda())
-    m.set_kernel_path(2)
-    b = _run_full(m, S.cuda(), ns.cuda())
-    for x, y in zip(a, b):
-        assert O.rel_l2(x.double().cpu().numpy(), y.double().cpu().numpy()) < 2e-3
-    errs = _errors_vs_oracle(m, w, S, ns, *a, [0, S.shape[0] - 1])
-    assert_within(errs, TOL["bf16"])
+        kw1 = dict(base, layers=1, q=[600])
+        kw = dict(base, layers=2, q=[600, 300])
+    for weights, shapes, tol in ((w1, kw1, 1e-3), (w, kw, 2 * 2.0 ** -8)):
+        m = make_model(weights, **shapes)
+        m.set_wait_limit(TEST_WAIT)
+        a = _run_full(m, S.cuda(), ns.cuda())
+        m.set_kernel_path(2)
+        b = _run_full(m, S.cuda(), ns.cuda())
+        for x, y in zip(a, b):
+            assert O.rel_l2(x.double().cpu().numpy(), y.double().cpu().numpy()) < tol
+        errs = _errors_vs_oracle(m, weights, S, ns, *a, [0, S.shape[0] - 1])
+        assert_within(errs, TOL["bf16"])

@@ -26,10 +26,12 @@
 //               memory at the start of a tile (each warp sums half the row,
 //               partials combined in shared memory); per chunk acc1 -> row
 //               scale -> GELU -> bf16 into G (the 128-byte-swizzled K-major
-//               layout the FFN2 MMA reads); at the end of the tile acc2 +
-//               residual H (the tile still in shared memory) -> bf16 written
-//               over H in place -> one TMA store of the tile to Y, after
-//               which the H buffer takes the next tile.
+//               layout the FFN2 MMA reads).  The residual is free: at the
+//               start of a tile the same pass that sums squares for the norm
+//               stores H in fp32 into acc2, and FFN2 accumulates onto it, so
+//               the H buffer is released once FFN1 has read it and the next
+//               tile's H loads while this tile finishes; at the end acc2 ->
+//               bf16, staged in the W2 stages, one TMA store to Y.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -100,7 +102,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
     float *s_ss = reinterpret_cast<float *>(sG);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sW2 + 2 * Sh::W2_BYTES);
     uint64_t *h_full = bars;
-    uint64_t *h_free = h_full + 1;     // the tile's output has left the H buffer
+    uint64_t *h_free = h_full + 1;     // FFN1's last MMAs and the epilogue's reads of H
     uint64_t *w1_full = h_free + 1;    // [K-half]
     uint64_t *w1_empty = w1_full + 2;  // [K-half]
     uint64_t *w2_full = w1_empty + 2;  // [2]
@@ -110,8 +112,9 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
     uint64_t *g_full = a1_free + 4;    // [2]
     uint64_t *g_free = g_full + 2;     // [2]
     uint64_t *a2_full = g_free + 2;
-    uint64_t *a2_free = a2_full + 1;
-    uint64_t *mma_done = a2_free + 1;  // [2] one per issuer
+    uint64_t *a2_init = a2_full + 1;   // acc2 holds the tile's H (the residual) in fp32
+    uint64_t *stg_free = a2_init + 1;  // the W2 stages no longer hold the previous output
+    uint64_t *mma_done = stg_free + 1; // [2] one per issuer
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
     pdl_launch_dependents();
     if (threadIdx.x == 0) {
         mbar_init(h_full, 1);
-        mbar_init(h_free, 1);
+        mbar_init(h_free, 1 + FF_EPI_WARPS);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&w1_full[b], 1);
             mbar_init(&w1_empty[b], 1);
@@ -134,7 +137,8 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             mbar_init(&mma_done[b], 1);
         }
         mbar_init(a2_full, 1);
-        mbar_init(a2_free, FF_EPI_WARPS);
+        mbar_init(a2_init, FF_EPI_WARPS);
+        mbar_init(stg_free, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -176,6 +180,8 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                             tma_load_3d(sH + k * FF_SLAB, &tmH, h_full, k * 64, m0, 0);
                     }
                     ++n_h;
+                } else if (tl > 0 && !mbar_wait(stg_free, (tl - 1) & 1, a.wait, abort_flag)) {
+                    break; // the W2 stages staged the previous tile's output
                 }
                 for (int c = 0; c < NC; ++c, ++gc) {
                     const int st = static_cast<int>(gc & 1);
@@ -243,6 +249,8 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                     }
                     if (ok) mma_commit(&a1_full[b]);
                 }
+                // every FFN1 MMA of the tile has read H
+                if (ok) mma_commit(h_free);
             }
             mma_commit(&mma_done[0]);
             mbar_wait(&mma_done[0], 0, final_wait, &no_abort);
@@ -262,9 +270,9 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                         ok = false;
                         break;
                     }
-                    // the tile's first chunk overwrites acc2: the previous tile's
-                    // output must have been read out
-                    if (c == 0 && !mbar_wait(a2_free, (tl & 1) ^ 1, a.wait, abort_flag)) {
+                    // the tile's first chunk accumulates onto H, which the
+                    // epilogue has stored into acc2
+                    if (c == 0 && !mbar_wait(a2_init, tl & 1, a.wait, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -273,8 +281,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                     const uint32_t w_addr = smem_u32(sW2 + st * Sh::W2_BYTES);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        mma_f16(t_acc2, sw128_desc(g_addr + k * 32, 16), sw128_desc(w_addr + k * 32, 16), IDESC2,
-                                (c | k) != 0);
+                        mma_f16(t_acc2, sw128_desc(g_addr + k * 32, 16), sw128_desc(w_addr + k * 32, 16), IDESC2, 1);
                     mma_commit(&w2_empty[st]);
                     mma_commit(&g_free[st]);
                 }
@@ -297,23 +304,42 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             const int g = static_cast<int>(tile / P.m_tiles);
             const int m0 = static_cast<int>(tile % P.m_tiles) * FF_BM;
             if (!mbar_wait(h_full, tl & 1, a.wait, abort_flag)) break;
-            // RMSNorm row scale from the tile in shared memory: this warp sums
-            // columns hf*HALF .. hf*HALF+HALF-1 of its rows (chunk j of a slab
-            // sits at 16-byte position j ^ (r & 7))
+            // This warp's half of its rows of H (columns hf*HALF ..): the
+            // RMSNorm partial sum of squares, and the values in fp32 into
+            // acc2, onto which the second projection accumulates (so the
+            // residual needs no read at the end).  acc2 is free: the previous
+            // tile's output was read out of it by these warps.  Chunk j of a
+            // slab row sits at 16-byte position j ^ (r & 7).
             float ss = 0.f;
-#pragma unroll
-            for (int j8 = 0; j8 < HALF / 8; ++j8) {
-                const int col = hf * HALF + 8 * j8;
+#pragma unroll 1
+            for (int c32 = 0; c32 < HALF / 32; ++c32) {
+                const int col = hf * HALF + 32 * c32;
                 const uint8_t *row = sH + (col / 64) * FF_SLAB + r * 128;
-                const uint4 v = *reinterpret_cast<const uint4 *>(row + ((((col % 64) / 8) ^ (r & 7)) << 4));
-                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                uint32_t hv[32];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float lo = __uint_as_float(w4[e] << 16);
-                    const float hi = __uint_as_float(w4[e] & 0xFFFF0000u);
-                    ss = fmaf(lo, lo, ss);
-                    ss = fmaf(hi, hi, ss);
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(row + ((((col % 64) / 8 + i) ^ (r & 7)) << 4));
+                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float lo = __uint_as_float(w4[e] << 16);
+                        const float hi = __uint_as_float(w4[e] & 0xFFFF0000u);
+                        ss = fmaf(lo, lo, ss);
+                        ss = fmaf(hi, hi, ss);
+                        hv[8 * i + 2 * e] = __float_as_uint(lo);
+                        hv[8 * i + 2 * e + 1] = __float_as_uint(hi);
+                    }
                 }
+                tmem_st32(t_acc2 + lane_off + col, hv);
+            }
+            tmem_st_wait();
+            // H read (generic proxy) before its buffer is refilled by TMA
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(a2_init);
+                mbar_arrive(h_free);
             }
             s_ss[hf * FF_BM + r] = ss;
             named_bar_sync(1, 32 * FF_EPI_WARPS);
@@ -361,9 +387,11 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             if (!ok) break;
             if (!mbar_wait(a2_full, tl & 1, a.wait, abort_flag)) break;
             tc_fence_after();
-            // Y = acc2 + H: the residual is the H tile still in shared memory;
-            // the output replaces it in place (same swizzled layout) and
-            // leaves through one TMA store
+            // Y = acc2 (= H + GELU(..) W2^T) as bf16, staged in the W2 stages
+            // (the second projection has read its last weights; the next
+            // tile's W2 loads wait for stg_free) in the 128-byte-swizzled
+            // layout of the Y tensor map, then one TMA store
+            uint8_t *stg = sW2;
 #pragma unroll 1
             for (int c32 = 0; c32 < HALF / 32; ++c32) {
                 const int col = hf * HALF + 32 * c32;
@@ -371,40 +399,35 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                 tmem_ld32(t_acc2 + lane_off + col, v);
                 tmem_ld_wait();
                 tmem_reg_fence(v);
-                uint8_t *row = sH + (col / 64) * FF_SLAB + r * 128;
+                uint8_t *row = stg + (col / 64) * FF_SLAB + r * 128;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    uint4 *p = reinterpret_cast<uint4 *>(row + ((((col % 64) / 8 + i) ^ (r & 7)) << 4));
-                    const uint4 x = *p;
-                    const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
                     uint32_t ow[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        ow[e] = pack_bf16x2(__uint_as_float(v[8 * i + 2 * e]) + __uint_as_float(w4[e] << 16),
-                                            __uint_as_float(v[8 * i + 2 * e + 1]) +
-                                                __uint_as_float(w4[e] & 0xFFFF0000u));
-                    *p = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                        ow[e] = pack_bf16x2(__uint_as_float(v[8 * i + 2 * e]), __uint_as_float(v[8 * i + 2 * e + 1]));
+                    *reinterpret_cast<uint4 *>(row + ((((col % 64) / 8 + i) ^ (r & 7)) << 4)) =
+                        make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 }
             }
-            // acc2 read out: the next tile's second projection may start
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(a2_free);
+            tc_fence_before(); // acc2 read before the next tile's H is stored into it
             // generic writes, read next by the TMA store (async proxy)
             fence_proxy_async_smem();
             named_bar_sync(1, 32 * FF_EPI_WARPS);
             if (warp == FF_EPI0 && lane == 0) {
                 for (int k = 0; k < KS; ++k) {
                     if (P.grouped)
-                        tma_store_3d(&tmY, sH + k * FF_SLAB, k * 64, g, m0);
+                        tma_store_3d(&tmY, stg + k * FF_SLAB, k * 64, g, m0);
                     else
-                        tma_store_3d(&tmY, sH + k * FF_SLAB, k * 64, m0, 0);
+                        tma_store_3d(&tmY, stg + k * FF_SLAB, k * 64, m0, 0);
                 }
                 bulk_commit_group();
                 bulk_wait_group_read0();
-                mbar_arrive(h_free); // the H buffer may take the next tile
+                mbar_arrive(stg_free); // the W2 stages may take the next tile's weights
             }
         }
+        // the output's global writes complete before the kernel ends
+        if (warp == FF_EPI0 && lane == 0) bulk_wait_group0();
     }
     tc_fence_before();
     __syncthreads();
