@@ -297,6 +297,32 @@ def test_bf16_many_items_per_cta():
         assert O.rel_l2(x.double().cpu().numpy(), y.double().cpu().numpy()) < 1e-2
 
 
+# ----------------------------------------------------------------- split-key NS attention
+@pytest.mark.parametrize("shape", ["nq128_odd_even_blocks", "nq1_two_blocks"])
+def test_split_key_ns_attention(shape):
+    """NS attention with every query row of a (user, head) in one tile: the
+    two tiles of a CTA take alternate key blocks and merge their softmax
+    states.  Layers with an even (4) and an odd (3) number of key blocks and
+    with exactly two (one S block, one NS block), a full tile of NS rows
+    (C N = 128) and a single NS row; every user against the oracle and the
+    CUDA-core path."""
+    if shape == "nq128_odd_even_blocks":
+        layers, d, H, f, N, U, C, L0, q = 3, 128, 2, 256, 16, 4, 8, 260, [260, 200, 60]
+    else:
+        layers, d, H, f, N, U, C, L0, q = 3, 128, 2, 256, 1, 5, 1, 100, [100, 64, 1]
+    w = rand_weights(layers, d, f, N, seed=51, dtype=torch.bfloat16)
+    S, ns = rand_inputs(U, C, L0, N, d, seed=52, dtype=torch.bfloat16)
+    m = make_model(w, layers=layers, d=d, heads=H, ffn=f, n_ns=N, L0=L0, q=q)
+    m.set_wait_limit(TEST_WAIT)
+    a = _run_full(m, S.cuda(), ns.cuda())
+    errs = _errors_vs_oracle(m, w, S, ns, *a, list(range(U)))
+    assert_within(errs, TOL["bf16"])
+    m.set_kernel_path(1)
+    b = _run_full(m, S.cuda(), ns.cuda())
+    for x, y in zip(a, b):
+        assert O.rel_l2(x.double().cpu().numpy(), y.double().cpu().numpy()) < 1e-2
+
+
 # ----------------------------------------------------------------- fused feed-forward
 @pytest.mark.parametrize("shape", ["small_d128", "onetrans_s_d256"])
 def test_fused_ffn_matches_two_gemm_path(shape):

@@ -56,8 +56,13 @@ constexpr int AT_HD = 64;
 constexpr uint32_t AT_TILE = AT_BM * 128; // 16 KB: 128 rows x 128 bytes
 constexpr int AT_STAGES = 5;              // K/V ring depth
 constexpr int AT_QBUF = 2;                // Q buffers (items in flight)
-// Q[AT_QBUF][AT_TILES], then per stage K and V, then barriers
-constexpr size_t AT_SMEM = (AT_QBUF * AT_TILES + 2 * AT_STAGES) * AT_TILE + 256;
+// Q[AT_QBUF][AT_TILES], then per stage K and V, then barriers, then the
+// split-key exchange (tile 1's running max and sum per row)
+constexpr size_t AT_BAR_BYTES = 256;
+constexpr size_t AT_XCH_BYTES = AT_BM * 2 * sizeof(float);
+constexpr size_t AT_SMEM = (AT_QBUF * AT_TILES + 2 * AT_STAGES) * AT_TILE + AT_BAR_BYTES + AT_XCH_BYTES;
+static_assert((2 * AT_QBUF + 2 * AT_STAGES + 6 * AT_TILES + 1) * 8 + 8 <= AT_BAR_BYTES, "barrier area");
+static_assert(AT_SMEM <= 227 * 1024, "shared memory per CTA");
 constexpr int AT_THREADS = 128 * (1 + AT_TILES); // producer warpgroup + one softmax warpgroup per tile
 // Register split (setmaxnreg): the producer warpgroup (TMA warp, MMA warp, two
 // idle warps) drops to AT_REG_PRODUCER per thread and the softmax warpgroups
@@ -179,22 +184,21 @@ __device__ __forceinline__ int at_item_of(int r, int n_items)
     return k < n_items ? static_cast<int>(k) : -1;
 }
 
-// This CTA's key blocks in order, across its items.
-template <bool NS>
+// The key blocks tile w works on, in order, across this CTA's items.  Every
+// tile takes every block, except in split-key mode (SPLIT: NS mode with all
+// query rows in one tile), where tile w takes the blocks b = w (mod 2) of an
+// item and the two tiles' partial softmax states are merged at its end.
+// gb counts all blocks of the CTA (the K/V ring position), lb this tile's.
+template <bool NS, bool SPLIT>
 struct BlockCursor {
     int r, k;      // item ordinal within the CTA, item index (k < 0: past the end)
     AtItem it;
     int b;         // block within the item
+    int w;         // tile
     long long gb;  // global block counter of the CTA
-    __device__ __forceinline__ void init(const AttnArgs &a, int n_pairs, int n_items)
-    {
-        r = 0;
-        b = 0;
-        gb = 0;
-        k = at_item_of(0, n_items);
-        if (k >= 0) it = at_item<NS>(a, n_pairs, k);
-    }
-    __device__ __forceinline__ void next(const AttnArgs &a, int n_pairs, int n_items)
+    long long lb;  // blocks of this tile before this one
+    __device__ __forceinline__ bool owned() const { return !SPLIT || (b & 1) == w; }
+    __device__ __forceinline__ void step(const AttnArgs &a, int n_pairs, int n_items)
     {
         ++gb;
         if (++b < it.n_blocks) return;
@@ -202,11 +206,32 @@ struct BlockCursor {
         k = at_item_of(++r, n_items);
         if (k >= 0) it = at_item<NS>(a, n_pairs, k);
     }
+    __device__ __forceinline__ void init(const AttnArgs &a, int n_pairs, int n_items, int tile)
+    {
+        w = tile;
+        r = 0;
+        b = 0;
+        gb = 0;
+        lb = 0;
+        k = at_item_of(0, n_items);
+        if (k >= 0) it = at_item<NS>(a, n_pairs, k);
+        while (valid() && !owned()) step(a, n_pairs, n_items);
+    }
+    __device__ __forceinline__ void next(const AttnArgs &a, int n_pairs, int n_items)
+    {
+        ++lb;
+        do step(a, n_pairs, n_items);
+        while (valid() && !owned());
+    }
     __device__ __forceinline__ bool valid() const { return k >= 0; }
-    __device__ __forceinline__ bool last_in_item() const { return b == it.n_blocks - 1; }
+    __device__ __forceinline__ bool first_in_item() const { return b == (SPLIT ? w : 0); }
+    __device__ __forceinline__ bool last_in_item() const
+    {
+        return SPLIT ? b + 2 >= it.n_blocks : b == it.n_blocks - 1;
+    }
 };
 
-template <bool NS>
+template <bool NS, bool SPLIT>
 __global__ void __launch_bounds__(AT_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKS,
                    const __grid_constant__ CUtensorMap tmVS, const __grid_constant__ CUtensorMap tmKN,
@@ -229,8 +254,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     uint64_t *o_full = p_full + AT_TILES;          // [tile] PV completed
     uint64_t *o_free = o_full + AT_TILES;          // [tile] O read out (end of an item)
     uint64_t *mma_done = o_free + AT_TILES;        // [tile]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + AT_TILES);
+    uint64_t *x_full = mma_done + AT_TILES;        // split-key: tile 1's state is in xch
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(x_full + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    float *xch = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + AT_BAR_BYTES); // [2][AT_BM]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_pairs = (a.nq + AT_BM * AT_TILES - 1) / (AT_BM * AT_TILES);
@@ -254,6 +281,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             mbar_init(&o_free[i], 4);
             mbar_init(&mma_done[i], 1);
         }
+        mbar_init(x_full, AT_BM);
         *abort_flag = 0;
         if (smem_u32(smem) & 1023) { // swizzle atoms need a 1024-byte aligned base
             *abort_flag = 1;
@@ -299,8 +327,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 const int qb = r & 1;
                 // the Q buffer of item r - 2 is free once all its S MMAs completed
                 if (!mbar_wait(&q_empty[qb], ((r >> 1) & 1) ^ 1, a.wait, abort_flag)) break;
-                mbar_arrive_expect_tx(&q_full[qb], AT_TILES * AT_TILE);
-                for (int w = 0; w < AT_TILES; ++w)
+                // split-key: both tiles read the one Q tile of the item
+                constexpr int q_tiles = SPLIT ? 1 : AT_TILES;
+                mbar_arrive_expect_tx(&q_full[qb], q_tiles * AT_TILE);
+                for (int w = 0; w < q_tiles; ++w)
                     tma_load_3d(sQ + (qb * AT_TILES + w) * AT_TILE, &tmQ, &q_full[qb],
                                 it.h * AT_HD, it.i0 + w * AT_BM, it.u);
                 for (int b = 0; b < it.n_blocks; ++b, ++gb) {
@@ -343,10 +373,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         const int w = warp - 1;
         if (lane == 0 && !aborted_at_start) {
             const uint32_t tS = tmem + w * 256, tP = tS + 128, tO = tS + 192;
-            auto live = [&](const AtItem &it) { return it.i0 + w * AT_BM < a.nq; };
-            auto issue_s = [&](const BlockCursor<NS> &c) {
+            auto live = [&](const AtItem &it) { return SPLIT || it.i0 + w * AT_BM < a.nq; };
+            auto issue_s = [&](const BlockCursor<NS, SPLIT> &c) {
                 if (live(c.it)) {
-                    const uint32_t q_addr = smem_u32(sQ + ((c.r & 1) * AT_TILES + w) * AT_TILE);
+                    const uint32_t q_addr = smem_u32(sQ + ((c.r & 1) * AT_TILES + (SPLIT ? 0 : w)) * AT_TILE);
                     const uint32_t k_addr = smem_u32(sKV + 2 * (c.gb % AT_STAGES) * AT_TILE);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
@@ -357,34 +387,36 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 // the item's last S of this tile: its Q buffer is free once they completed
                 if (c.last_in_item()) mma_commit(&q_empty[c.r & 1]);
             };
-            auto ready_s = [&](const BlockCursor<NS> &c) {
+            auto ready_s = [&](const BlockCursor<NS, SPLIT> &c) {
                 return mbar_wait(&kv_full[c.gb % AT_STAGES], static_cast<uint32_t>((c.gb / AT_STAGES) & 1),
                                  a.wait, abort_flag) &&
                        mbar_wait(&q_full[c.r & 1], (c.r >> 1) & 1, a.wait, abort_flag);
             };
-            BlockCursor<NS> cur;
-            cur.init(a, n_pairs, n_items);
+            BlockCursor<NS, SPLIT> cur;
+            cur.init(a, n_pairs, n_items, w);
             bool run = cur.valid() && ready_s(cur);
             if (run) {
                 tc_fence_after();
                 issue_s(cur);
             }
             while (run) {
-                BlockCursor<NS> nxt = cur;
+                BlockCursor<NS, SPLIT> nxt = cur;
                 nxt.next(a, n_pairs, n_items);
                 if (nxt.valid()) {
-                    if (!mbar_wait(&s_free[w], static_cast<uint32_t>(cur.gb & 1), a.wait, abort_flag) ||
+                    if (!mbar_wait(&s_free[w], static_cast<uint32_t>(cur.lb & 1), a.wait, abort_flag) ||
                         !ready_s(nxt))
                         break;
                     tc_fence_after();
                     issue_s(nxt);
                 }
-                if (!mbar_wait(&p_full[w], static_cast<uint32_t>(cur.gb & 1), a.wait, abort_flag)) break;
+                if (!mbar_wait(&p_full[w], static_cast<uint32_t>(cur.lb & 1), a.wait, abort_flag)) break;
                 tc_fence_after();
                 // the first PV of an item overwrites O: the previous item's
                 // output has been read out by then (the warpgroup did that
-                // before computing P of this block)
-                if (cur.b == 0 && cur.r > 0) {
+                // before computing P of this block; in split-key mode tile 0
+                // reads both tiles' O)
+                const bool first = cur.first_in_item();
+                if (first && cur.r > 0) {
                     if (!mbar_wait(&o_free[w], (cur.r - 1) & 1, a.wait, abort_flag)) break;
                     tc_fence_after();
                 }
@@ -393,10 +425,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) // P from TMEM: 8 columns per 16 keys
                         mma_f16_ts(tO, tP + kk * 8, sw128_desc(v_addr + kk * 2048, AT_TILE), IDESC_O,
-                                   (cur.b | kk) != 0);
+                                   !first || kk != 0);
                 }
                 mma_commit(&o_full[w]);
+                // both arrivals the stage waits for: split-key stages have one reader
                 mma_commit(&kv_empty[cur.gb % AT_STAGES]);
+                if (SPLIT) mma_commit(&kv_empty[cur.gb % AT_STAGES]);
                 if (!nxt.valid()) break;
                 cur = nxt;
             }
@@ -414,8 +448,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         const uint32_t tS = tmem + w * 256 + lane_off, tP = tS + 128, tO = tS + 192;
         const float c2 = a.scale * 1.4426950408889634f; // scores -> base-2 exponent
         bool ok = !aborted_at_start;
-        long long gb = 0;
-        // wait for the PV of this tile's global block jb (completion jb of
+        long long lb = 0; // blocks of this tile so far
+        int xr = 0;       // split-key hand-overs so far
+        // wait for the PV of this tile's block jb (completion jb of
         // o_full[w]).  Waiting twice for the same block is harmless: PV(jb + 1)
         // is not issued before this warpgroup releases P(jb + 1), which it
         // does only after observing PV(jb), so o_full is at most one phase
@@ -433,12 +468,13 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             const int k = at_item_of(r, n_items);
             if (k < 0) break;
             const AtItem it = at_item<NS>(a, n_pairs, k);
-            const int i = it.i0 + w * AT_BM + row;  // query row within the user
+            const int i = it.i0 + (SPLIT ? 0 : w * AT_BM) + row; // query row within the user
             const bool warp_dead = __all_sync(0xffffffffu, i >= a.nq);
             const int t_self = a.L - a.nq + i;      // S mode
             const int my_c = NS ? i / a.N : 0, my_n = NS ? i % a.N : 0;
             float m = -INFINITY, l = 0.f;
-            for (int b = 0; ok && b < it.n_blocks; ++b, ++gb) {
+            const int b0 = SPLIT ? w : 0; // this tile's first block of the item
+            for (int b = b0; ok && b < it.n_blocks; b += SPLIT ? 2 : 1, ++lb) {
                 const bool s_block = b < it.n_s_blocks;
                 const int j0 = s_block ? b * AT_BK : it.k_begin + (b - it.n_s_blocks) * AT_BK;
                 // visible key range [klo, khi] of this row inside the block
@@ -452,7 +488,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 }
                 const bool warp_full = __all_sync(0xffffffffu, klo <= 0 && khi >= AT_BK - 1);
                 const bool warp_none = __all_sync(0xffffffffu, khi < klo);
-                if (!mbar_wait(&s_full[w], static_cast<uint32_t>(gb & 1), a.wait, abort_flag)) {
+                if (!mbar_wait(&s_full[w], static_cast<uint32_t>(lb & 1), a.wait, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -461,7 +497,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                     // nothing of this warp's rows is visible (or no live row):
                     // the scores are not read; a live warp stores P = 0
                     release(&s_free[w]);
-                    if (b >= 1) wait_o(gb - 1);
+                    if (b > b0) wait_o(lb - 1);
                     if (!warp_dead) {
                         uint32_t z[32];
 #pragma unroll
@@ -477,8 +513,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                         softmax_unit<true>(tS, c2, 0, AT_BK - 1, m, pk, alpha, rsum, [&] { release(&s_free[w]); });
                     else
                         softmax_unit<false>(tS, c2, klo, khi, m, pk, alpha, rsum, [&] { release(&s_free[w]); });
-                    // P(b) goes where PV(b - 1) read P(b - 1) from
-                    if (b >= 1) wait_o(gb - 1);
+                    // P(b) goes where the previous PV read its P from
+                    if (b > b0) wait_o(lb - 1);
                     if (__any_sync(0xffffffffu, alpha != 1.f)) {
                         // some row raised its max: O holds this item's blocks before
                         // b relative to the old max (their PV has completed)
@@ -502,18 +538,55 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 release(&p_full[w]);
             }
             if (!ok) break;
-            wait_o(gb - 1); // the item's last PV
+            wait_o(lb - 1); // the item's last PV
             if (!ok) break;
+            if (SPLIT && w == 1) {
+                // hand the row's state to tile 0, which merges it with its own
+                // and reads this tile's O straight from TMEM (its lanes are the
+                // same rows); tile 0 also frees this O for the next item
+                xch[row] = m;
+                xch[AT_BM + row] = l;
+                tc_fence_before();
+                mbar_arrive(x_full);
+                ++xr;
+                continue;
+            }
             // O / l as bf16 pairs, read 32 columns at a time
             uint32_t ob[AT_HD / 2];
+            float a0 = 1.f, a1 = 0.f, inv = 0.f;
+            if (SPLIT) {
+                // merge with tile 1: O = O0 2^(m0 - m) + O1 2^(m1 - m), same for l
+                if (!mbar_wait(x_full, static_cast<uint32_t>(xr & 1), a.wait, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                ++xr;
+                const float m1 = xch[row], l1 = xch[AT_BM + row];
+                const float mm = fmaxf(m, m1);
+                a0 = fast_exp2(m - mm);
+                a1 = fast_exp2(m1 - mm);
+                l = l * a0 + l1 * a1;
+            }
             if (!warp_dead) {
-                const float inv = 1.f / l;
+                inv = 1.f / l;
 #pragma unroll
                 for (int c = 0; c < AT_HD; c += 32) {
                     uint32_t v[32];
                     tmem_ld32(tO + c, v);
-                    tmem_ld_wait();
-                    tmem_reg_fence(v);
+                    if (SPLIT) {
+                        uint32_t v1[32];
+                        tmem_ld32(tO + 256 + c, v1); // tile 1's O, same lanes
+                        tmem_ld_wait();
+                        tmem_reg_fence(v);
+                        tmem_reg_fence(v1);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            v[e] = __float_as_uint(fmaf(__uint_as_float(v[e]), a0, __uint_as_float(v1[e]) * a1));
+                    } else {
+                        tmem_ld_wait();
+                        tmem_reg_fence(v);
+                    }
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         ob[c / 2 + e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv,
@@ -522,6 +595,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             }
             // O may now be overwritten by the next item's first PV
             release(&o_free[w]);
+            if (SPLIT) release(&o_free[1]);
             if (i < a.nq) {
                 uint4 *dp = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.O) +
                                                       (static_cast<long long>(it.u) * a.nq + i) * a.d +
@@ -578,29 +652,24 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
                             a.H * a.U;
     if (items < 1 || items > (1LL << 30)) return cudaErrorInvalidValue;
     dim3 grid(static_cast<unsigned>(items < num_sms ? items : num_sms));
-    cudaError_t e;
-    // the setmaxnreg split must fit the registers the launch allocates, or the
-    // softmax warpgroups' increase would wait forever
-    {
+    // split-key mode: every query row in one tile and at least one S block,
+    // so each item has two or more key blocks and each tile gets one
+    const bool split = a.mode == 1 && a.nq <= AT_BM && a.L >= 1;
+    auto run = [&](auto kernel) -> cudaError_t {
+        // the setmaxnreg split must fit the registers the launch allocates,
+        // or the softmax warpgroups' increase would wait forever
         cudaFuncAttributes fa;
-        e = a.mode == 1 ? cudaFuncGetAttributes(&fa, attn_tc_kernel<true>)
-                        : cudaFuncGetAttributes(&fa, attn_tc_kernel<false>);
-        if (e != cudaSuccess) return e;
+        cudaError_t err = cudaFuncGetAttributes(&fa, kernel);
+        if (err != cudaSuccess) return err;
         if (128 * AT_REG_PRODUCER + 128 * AT_TILES * AT_REG_SOFTMAX > fa.numRegs * AT_THREADS)
             return cudaErrorInvalidConfiguration;
-    }
-    if (a.mode == 1) {
-        e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(AT_SMEM));
-        if (e != cudaSuccess) return e;
-        return launch_pdl(attn_tc_kernel<true>, grid, dim3(AT_THREADS), AT_SMEM, s, tq, tks, tvs,
-                          tkn, tvn, a);
-    }
-    e = cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(AT_SMEM));
-    if (e != cudaSuccess) return e;
-    return launch_pdl(attn_tc_kernel<false>, grid, dim3(AT_THREADS), AT_SMEM, s, tq, tks, tvs, tkn,
-                      tvn, a);
+        err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(AT_SMEM));
+        if (err != cudaSuccess) return err;
+        return launch_pdl(kernel, grid, dim3(AT_THREADS), AT_SMEM, s, tq, tks, tvs, tkn, tvn, a);
+    };
+    if (a.mode != 1) return run(attn_tc_kernel<false, false>);
+    return split ? run(attn_tc_kernel<true, true>) : run(attn_tc_kernel<true, false>);
 }
 
 } // namespace ot
