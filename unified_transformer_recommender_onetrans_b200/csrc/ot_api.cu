@@ -12,6 +12,9 @@
 // Per layer of the NS-side (score, U users x C candidates x N tokens):
 //   the same four steps with grouped GEMMs (group = NS position n, its own
 //   weights), and NS attention against layer l of the cache.
+// Full forward (both sides): steps 3 and 4 of the two sides share one launch
+// each (the NS tiles fill the S launch's last partial wave); the NS QKV and
+// attention run on a second stream beside the S attention.
 #include <cudaTypedefs.h>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -53,6 +56,7 @@ struct ot_model {
     // kv_ready[l] (recorded after the S QKV GEMM of layer l) has fired.
     cudaStream_t side = nullptr;
     cudaEvent_t kv_ready[OT_MAX_LAYERS];
+    cudaEvent_t ns_attn_done[OT_MAX_LAYERS]; // merged full forward: NS attention of layer l
     cudaEvent_t fork_ev = nullptr, join_ev = nullptr;
     std::mutex enqueue_mu; // event re-recording must not interleave between calls
 };
@@ -182,7 +186,9 @@ size_t score_ws_bytes(const ot_config &c, int U, int C, int esz)
 }
 
 enum { ROLE_S_QKV = 0, ROLE_S_ATTN, ROLE_S_O, ROLE_S_FFN1, ROLE_S_FFN2, ROLE_NS_QKV, ROLE_NS_ATTN,
-       ROLE_NS_O, ROLE_NS_FFN1, ROLE_NS_FFN2, ROLE_AUTO_SPLIT, ROLE_OTHER, ROLE_S_FFN, ROLE_NS_FFN };
+       ROLE_NS_O, ROLE_NS_FFN1, ROLE_NS_FFN2, ROLE_AUTO_SPLIT, ROLE_OTHER, ROLE_S_FFN, ROLE_NS_FFN,
+       // one launch for the S and NS sides of a layer (full forward)
+       ROLE_O, ROLE_FFN };
 
 cudaEvent_t pooled_event(ot_model *m)
 {
@@ -224,7 +230,19 @@ long long kept_rows(const RowMap &mp, long long M)
     return full + (rem > 0 ? rem : 0);
 }
 
-ot_status gemm(ot_model *m, GemmArgs &a, cudaStream_t s, int role)
+// algorithmic flops and bytes of one GEMM problem (per-launch profiling)
+void gemm_cost(const ot_model *m, const GemmArgs &a, double &flops, double &bytes)
+{
+    const double esz = a.in_dtype == OT_DTYPE_FP8 ? 1 : m->esz, G = a.G;
+    double out_elems = 0;
+    for (int i = 0; i < a.nseg; ++i)
+        out_elems += static_cast<double>(kept_rows(a.seg[i].map, a.M)) * (a.seg[i].c_hi - a.seg[i].c_lo);
+    flops += 2.0 * a.K * out_elems * G;
+    bytes += esz * G * (static_cast<double>(a.M) * a.K + static_cast<double>(a.N) * a.K + out_elems +
+                        (a.res ? static_cast<double>(a.M) * a.N : 0.0));
+}
+
+void gemm_prepare(const ot_model *m, GemmArgs &a)
 {
     a.wait = WaitCtl{m->err, m->wait_limit};
     // operand dtype: e4m3 only where the caller prepared quantised operands
@@ -232,22 +250,31 @@ ot_status gemm(ot_model *m, GemmArgs &a, cudaStream_t s, int role)
                  : a.in_dtype == OT_DTYPE_FP8 ? OT_DTYPE_FP8
                                               : OT_DTYPE_BF16;
     a.store = m->cfg.dtype == OT_DTYPE_F32 ? OT_STORE_F32 : OT_STORE_BF16;
+}
+
+ot_status gemm(ot_model *m, GemmArgs &a, cudaStream_t s, int role)
+{
+    gemm_prepare(m, a);
     const bool simt = m->cfg.dtype == OT_DTYPE_F32 || m->path == 1;
     if (simt && a.in_dtype == OT_DTYPE_FP8) return OT_ERR_UNSUPPORTED;
     double flops = 0, bytes = 0;
-    if (m->profiling) {
-        const double esz = a.in_dtype == OT_DTYPE_FP8 ? 1 : m->esz, G = a.G;
-        double out_elems = 0;
-        for (int i = 0; i < a.nseg; ++i)
-            out_elems += static_cast<double>(kept_rows(a.seg[i].map, a.M)) *
-                         (a.seg[i].c_hi - a.seg[i].c_lo);
-        flops = 2.0 * a.K * out_elems * G;
-        bytes = esz * G * (static_cast<double>(a.M) * a.K + static_cast<double>(a.N) * a.K +
-                           out_elems + (a.res ? static_cast<double>(a.M) * a.N : 0.0));
-    }
+    if (m->profiling) gemm_cost(m, a, flops, bytes);
     return profiled(m, s, simt ? OT_KIND_GEMM_SIMT : OT_KIND_GEMM_TC, role, flops, bytes, [&] {
         return simt ? launch_gemm_simt(a, s) : launch_gemm_tc(a, s);
     });
+}
+
+// algorithmic flops (visible query-key pairs) and bytes of one attention problem
+void attn_cost(const ot_model *m, const AttnArgs &a, double &flops, double &bytes)
+{
+    const double L = a.L, nq = a.nq, N = a.N, U = a.U, esz = m->esz;
+    double pairs; // visible (query, key) pairs per user and head
+    if (a.mode == 0)
+        pairs = nq * (L - nq) + nq * (nq + 1) / 2;
+    else
+        pairs = (nq / N) * (N * L + N * (N + 1) / 2);
+    flops += 4.0 * a.hd * pairs * a.H * U;
+    bytes += esz * U * a.d * (2 * nq + 2 * L + (a.mode == 1 ? 2 * nq : 0));
 }
 
 ot_status attn(ot_model *m, AttnArgs &a, cudaStream_t s)
@@ -256,16 +283,7 @@ ot_status attn(ot_model *m, AttnArgs &a, cudaStream_t s)
     a.dtype = m->cfg.dtype;
     const bool simt = m->cfg.dtype == OT_DTYPE_F32 || m->path == 1;
     double flops = 0, bytes = 0;
-    if (m->profiling) {
-        const double L = a.L, nq = a.nq, N = a.N, U = a.U, esz = m->esz;
-        double pairs; // visible (query, key) pairs per user and head
-        if (a.mode == 0)
-            pairs = nq * (L - nq) + nq * (nq + 1) / 2;
-        else
-            pairs = (nq / N) * (N * L + N * (N + 1) / 2);
-        flops = 4.0 * a.hd * pairs * a.H * U;
-        bytes = esz * U * a.d * (2 * nq + 2 * L + (a.mode == 1 ? 2 * nq : 0));
-    }
+    if (m->profiling) attn_cost(m, a, flops, bytes);
     return profiled(m, s, simt ? OT_KIND_ATTN_SIMT : OT_KIND_ATTN_TC,
                     a.mode == 0 ? ROLE_S_ATTN : ROLE_NS_ATTN, flops, bytes, [&] {
                         return simt ? launch_attn_simt(a, s) : launch_attn_tc(a, s);
@@ -280,8 +298,8 @@ bool use_fused_ffn(const ot_model *m)
 }
 
 // Y = H + GELU(n(H) W1^T) W2^T over G groups of M rows (gain folded into W1).
-ot_status ffn(ot_model *m, int M, int G, const void *H, RowMap h_map, const void *W1,
-              const void *W2, void *Y, RowMap y_map, cudaStream_t s, int role)
+FfnArgs ffn_args(const ot_model *m, int M, int G, const void *H, RowMap h_map, const void *W1,
+                 const void *W2, void *Y, RowMap y_map)
 {
     const ot_config &c = m->cfg;
     FfnArgs a;
@@ -300,13 +318,51 @@ ot_status ffn(ot_model *m, int M, int G, const void *H, RowMap h_map, const void
     a.y_map = y_map;
     a.eps = c.eps;
     a.wait = WaitCtl{m->err, m->wait_limit};
+    return a;
+}
+
+void ffn_cost(const FfnArgs &a, double &flops, double &bytes)
+{
+    const double rows = static_cast<double>(a.M) * a.G, d = a.D, f = a.F;
+    flops += 4.0 * rows * d * f;
+    bytes += 2.0 * (2.0 * rows * d + 2.0 * a.G * d * f); // H in, Y out, W1 + W2 once
+}
+
+ot_status ffn(ot_model *m, int M, int G, const void *H, RowMap h_map, const void *W1,
+              const void *W2, void *Y, RowMap y_map, cudaStream_t s, int role)
+{
+    FfnArgs a = ffn_args(m, M, G, H, h_map, W1, W2, Y, y_map);
+    double flops = 0, bytes = 0;
+    if (m->profiling) ffn_cost(a, flops, bytes);
+    return profiled(m, s, OT_KIND_FFN_TC, role, flops, bytes, [&] { return launch_ffn_tc(a, s); });
+}
+
+// One launch for the S and NS problems of a layer step (either may be absent).
+ot_status gemm2(ot_model *m, GemmArgs *a, GemmArgs *b, cudaStream_t s, int role)
+{
+    if (!a) a = b, b = nullptr;
+    if (!a) return OT_ERR_ARG;
+    double flops = 0, bytes = 0;
+    for (GemmArgs *g : {a, b})
+        if (g) {
+            gemm_prepare(m, *g);
+            if (m->profiling) gemm_cost(m, *g, flops, bytes);
+        }
+    return profiled(m, s, OT_KIND_GEMM_TC, role, flops, bytes,
+                    [&] { return launch_gemm_tc_multi(*a, b, s); });
+}
+
+ot_status ffn2(ot_model *m, FfnArgs *a, FfnArgs *b, cudaStream_t s)
+{
+    if (!a) a = b, b = nullptr;
+    if (!a) return OT_ERR_ARG;
     double flops = 0, bytes = 0;
     if (m->profiling) {
-        const double rows = static_cast<double>(M) * G, d = c.d, f = c.ffn;
-        flops = 4.0 * rows * d * f;
-        bytes = 2.0 * (2.0 * rows * d + 2.0 * G * d * f); // H in, Y out, W1 + W2 once
+        ffn_cost(*a, flops, bytes);
+        if (b) ffn_cost(*b, flops, bytes);
     }
-    return profiled(m, s, OT_KIND_FFN_TC, role, flops, bytes, [&] { return launch_ffn_tc(a, s); });
+    return profiled(m, s, OT_KIND_FFN_TC, ROLE_FFN, flops, bytes,
+                    [&] { return launch_ffn_tc_multi(*a, b, s); });
 }
 
 GemmArgs gemm_base(const ot_config &c, int M, int N, int K, int G)
@@ -605,6 +661,140 @@ ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, v
     return OT_OK;
 }
 
+// The S and NS sides can share launches: bf16 tensor-core path with the
+// fused FFN and head_dim 64 attention.
+bool merged_supported(const ot_model *m)
+{
+    return use_fused_ffn(m) && m->cfg.d / m->cfg.heads == 64;
+}
+
+// Full forward with the S and NS sides sharing the O-projection and FFN
+// launches of each layer: the NS work units come after the S ones and fill
+// the S launches' last partial waves (at small C a whole NS step costs
+// almost nothing there).  The NS QKV projection and attention of layer l run
+// on the side stream once layer l's S K/V are cached, beside the S attention;
+// the merged O launch waits for them.  Same arithmetic, buffers and workspace
+// layouts as run_encode + run_score.
+ot_status run_full_merged(ot_model *m, const void *X0, int U, const void *ns, int C, void *kv,
+                          void *s_out, void *out, Ws ws_enc, Ws ws_sc, cudaStream_t st)
+{
+    const ot_config &c = m->cfg;
+    const int d = c.d, f = c.ffn, N = c.n_ns;
+    // S-side buffers (as run_encode)
+    const long long rows0 = static_cast<long long>(U) * c.L0;
+    void *Xb[2] = {ws_enc.take(rows0 * d), ws_enc.take(rows0 * d)};
+    void *Qb = ws_enc.take(rows0 * d), *Ab = ws_enc.take(rows0 * d), *Hb = ws_enc.take(rows0 * d);
+    if (!Xb[0] || !Xb[1] || !Qb || !Ab || !Hb) return OT_ERR_WORKSPACE_TOO_SMALL;
+    // NS-side buffers (as run_score)
+    const int Mc = U * C;
+    const long long R = static_cast<long long>(Mc) * N;
+    void *Yb[2] = {ws_sc.take(R * d), ws_sc.take(R * d)};
+    void *Qn = ws_sc.take(R * d), *Kn = ws_sc.take(R * d), *Vn = ws_sc.take(R * d);
+    void *An = ws_sc.take(R * d), *Hn = ws_sc.take(R * d);
+    if (!Yb[0] || !Yb[1] || !Qn || !Kn || !Vn || !An || !Hn) return OT_ERR_WORKSPACE_TOO_SMALL;
+    const long long ustride = kv_user_elems(c);
+    const RowMap grp{1, N, 0, 1, 0}; // candidate m, position g -> row m*N + g
+    const Fp8Scratch no_f8{nullptr, nullptr};
+    const float scale = 1.0f / sqrtf(static_cast<float>(d / c.heads));
+    // per-launch profiling times each kernel alone: everything on one stream
+    cudaStream_t side = m->profiling ? st : m->side;
+    const bool two = side != st;
+    const void *X = X0, *Y = ns;
+    ot_status r;
+    for (int l = 0; l < c.layers; ++l) {
+        const int L = rows_at(c, l), q = c.q[l];
+        const bool last = l == c.layers - 1;
+        char *K = at(kv, kv_layer_off(c, l), m->esz);
+        char *V = K + static_cast<long long>(L) * d * m->esz;
+        const RowMap cache_map{L, ustride / d, 0, 0, 0};
+        const long long lN = static_cast<long long>(l) * N;
+        // 1. S QKV: K / V into the cache, Q of the tail rows
+        GemmArgs gs = gemm_base(c, U * L, 3 * d, d, 1);
+        if ((r = projection(m, gs, X, d, rowmap_identity(),
+                            at(m->Wqkv_s, static_cast<long long>(l) * 3 * d * d, m->esz), 3LL * d * d, nullptr,
+                            nullptr, d, true, no_f8, st)) != OT_OK)
+            return r;
+        gs.nseg = 3;
+        gs.seg[0] = seg_of(Qb, d, 0, d, RowMap{L, q, -(L - q), 0, L - q});
+        gs.seg[1] = seg_of(K, d, d, 2 * d, cache_map);
+        gs.seg[2] = seg_of(V, d, 2 * d, 3 * d, cache_map);
+        if ((r = gemm(m, gs, st, ROLE_S_QKV)) != OT_OK) return r;
+        // the NS side of this layer needs these K/V and the previous layer's NS output
+        if (two && (cudaEventRecord(m->kv_ready[l], st) != cudaSuccess ||
+                    cudaStreamWaitEvent(side, m->kv_ready[l], 0) != cudaSuccess))
+            return OT_ERR_CUDA;
+        // 2. NS QKV + NS attention (side stream)
+        GemmArgs gn = gemm_base(c, Mc, 3 * d, d, N);
+        if ((r = projection(m, gn, Y, d, grp, at(m->Wqkv_ns, lN * 3 * d * d, m->esz), 3LL * d * d, nullptr,
+                            nullptr, d, true, no_f8, side)) != OT_OK)
+            return r;
+        gn.nseg = 3;
+        gn.seg[0] = seg_of(Qn, d, 0, d, grp);
+        gn.seg[1] = seg_of(Kn, d, d, 2 * d, grp);
+        gn.seg[2] = seg_of(Vn, d, 2 * d, 3 * d, grp);
+        if ((r = gemm(m, gn, side, ROLE_NS_QKV)) != OT_OK) return r;
+        AttnArgs as_, an_;
+        memset(&as_, 0, sizeof(as_));
+        as_.mode = 0;
+        as_.U = U;
+        as_.H = c.heads;
+        as_.hd = d / c.heads;
+        as_.d = d;
+        as_.L = L;
+        as_.nq = q;
+        as_.N = N;
+        as_.Q = Qb;
+        as_.KS = K;
+        as_.VS = V;
+        as_.s_ustride = ustride;
+        as_.O = Ab;
+        as_.scale = scale;
+        an_ = as_;
+        an_.mode = 1;
+        an_.nq = C * N;
+        an_.Q = Qn;
+        an_.KN = Kn;
+        an_.VN = Vn;
+        an_.O = An;
+        if ((r = attn(m, an_, side)) != OT_OK) return r;
+        if (two && cudaEventRecord(m->ns_attn_done[l], side) != cudaSuccess) return OT_ERR_CUDA;
+        // 3. S attention (main stream)
+        if ((r = attn(m, as_, st)) != OT_OK) return r;
+        if (two && cudaStreamWaitEvent(st, m->ns_attn_done[l], 0) != cudaSuccess) return OT_ERR_CUDA;
+        // 4. O projection + residual, both sides in one launch
+        GemmArgs os_ = gemm_base(c, U * q, d, d, 1);
+        if ((r = projection(m, os_, Ab, d, rowmap_identity(), at(m->Wo_s, static_cast<long long>(l) * d * d, m->esz),
+                            static_cast<long long>(d) * d, nullptr, nullptr, 0, false, no_f8, st)) != OT_OK)
+            return r;
+        os_.res = X;
+        os_.res_ld = d;
+        os_.res_map = RowMap{q, L, L - q, 0, 0};
+        os_.nseg = 1;
+        os_.seg[0] = seg_of(Hb, d, 0, d, rowmap_identity());
+        GemmArgs on_ = gemm_base(c, Mc, d, d, N);
+        if ((r = projection(m, on_, An, d, grp, at(m->Wo_ns, lN * d * d, m->esz), static_cast<long long>(d) * d,
+                            nullptr, nullptr, 0, false, no_f8, st)) != OT_OK)
+            return r;
+        on_.res = Y;
+        on_.res_ld = d;
+        on_.res_map = grp;
+        on_.nseg = 1;
+        on_.seg[0] = seg_of(Hn, d, 0, d, grp);
+        if ((r = gemm2(m, &os_, &on_, st, ROLE_O)) != OT_OK) return r;
+        // 5. FFN (RMSNorm, W1, GELU, W2, residual), both sides in one launch
+        void *Xn = (last && s_out) ? s_out : Xb[l & 1];
+        void *Yn = last ? out : Yb[l & 1];
+        FfnArgs fs = ffn_args(m, U * q, 1, Hb, rowmap_identity(), at(m->W1_s, static_cast<long long>(l) * f * d, m->esz),
+                              at(m->W2_s, static_cast<long long>(l) * d * f, m->esz), Xn, rowmap_identity());
+        FfnArgs fn = ffn_args(m, Mc, N, Hn, grp, at(m->W1_ns, lN * f * d, m->esz), at(m->W2_ns, lN * d * f, m->esz),
+                              Yn, grp);
+        if ((r = ffn2(m, &fs, &fn, st)) != OT_OK) return r;
+        X = Xn;
+        Y = Yn;
+    }
+    return OT_OK;
+}
+
 ot_status device_copy(ot_model *m, void **dst, const void *src, size_t bytes)
 {
     if (cudaMalloc(dst, bytes) != cudaSuccess) return OT_ERR_CUDA;
@@ -709,7 +899,8 @@ ot_status ot_model_create(const ot_config *cfg, const ot_weights *w, ot_model **
             break;
         }
         for (int l = 0; l < cfg->layers && r == OT_OK; ++l)
-            if (cudaEventCreateWithFlags(&m->kv_ready[l], cudaEventDisableTiming) != cudaSuccess)
+            if (cudaEventCreateWithFlags(&m->kv_ready[l], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&m->ns_attn_done[l], cudaEventDisableTiming) != cudaSuccess)
                 r = OT_ERR_CUDA;
         if (r != OT_OK) break;
         if (cfg->dtype == OT_DTYPE_FP8) {
@@ -766,8 +957,10 @@ void ot_model_destroy(ot_model *m)
         cudaEventDestroy(r.e1);
     }
     for (cudaEvent_t e : m->event_pool) cudaEventDestroy(e);
-    for (int l = 0; l < m->cfg.layers && l < OT_MAX_LAYERS; ++l)
+    for (int l = 0; l < m->cfg.layers && l < OT_MAX_LAYERS; ++l) {
         if (m->kv_ready[l]) cudaEventDestroy(m->kv_ready[l]);
+        if (m->ns_attn_done[l]) cudaEventDestroy(m->ns_attn_done[l]);
+    }
     if (m->fork_ev) cudaEventDestroy(m->fork_ev);
     if (m->join_ev) cudaEventDestroy(m->join_ev);
     if (m->side) cudaStreamDestroy(m->side);
@@ -923,9 +1116,16 @@ ot_status ot_full_forward(ot_model *m, const void *S, const void *ns, int B, int
         kv = w.take(static_cast<long long>(B) * kv_user_elems(c));
         if (!kv) return OT_ERR_WORKSPACE_TOO_SMALL;
     }
-    // Overlapped when the workspace holds both sides and per-launch profiling
-    // (which times each kernel alone) is off: the NS side of layer l waits
-    // only for layer l's cached S K/V, so it runs beside S layers l+1...
+    // Shared O / FFN launches for both sides where the kernels allow it
+    if (merged_supported(m) && m->side && w.left >= enc + sc) {
+        std::lock_guard<std::mutex> lock(m->enqueue_mu);
+        Ws w_enc = w;
+        Ws w_sc{w.p + enc, w.left - enc, m->esz};
+        return run_full_merged(m, S, B, ns, C, kv, out_s_tail, out_ns, w_enc, w_sc, st);
+    }
+    // Otherwise overlapped when the workspace holds both sides and per-launch
+    // profiling (which times each kernel alone) is off: the NS side of layer
+    // l waits only for layer l's cached S K/V, so it runs beside S layers l+1...
     const bool overlap = !m->profiling && m->side && w.left >= enc + sc;
     if (!overlap) {
         ot_status r = run_encode(m, S, B, kv, out_s_tail, w, st);

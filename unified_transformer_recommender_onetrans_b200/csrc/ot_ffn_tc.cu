@@ -32,6 +32,8 @@
 //               the H buffer is released once FFN1 has read it and the next
 //               tile's H loads while this tile finishes; at the end acc2 ->
 //               bf16, staged in the W2 stages, one TMA store to Y.
+#include <cstring>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -67,6 +69,25 @@ struct FfnParams {
     long long tiles;
 };
 
+// One launch over one or two problems with the same D, F and eps (the S and
+// NS feed-forwards of a layer): problem 0's tiles, then problem 1's.
+struct FfnMulti {
+    FfnParams q[2];
+    long long split; // first tile of problem 1
+    long long tiles;
+};
+
+// problem, group and first row of tile `tile` of the launch
+__device__ __forceinline__ int ffn_tile(const FfnMulti &P, long long tile, int &g, int &m0)
+{
+    const int pi = tile >= P.split ? 1 : 0;
+    const long long lt = tile - (pi ? P.split : 0);
+    const FfnParams &Q = P.q[pi];
+    g = static_cast<int>(lt / Q.m_tiles);
+    m0 = static_cast<int>(lt % Q.m_tiles) * FF_BM;
+    return pi;
+}
+
 // exact-erf GELU, z * Phi(z), with Phi(z) ~ 1/2 + 1/2 tanh(z (A + B z^2)):
 // the same fitted form as the GEMM epilogue
 __device__ __forceinline__ float ffn_gelu(float z)
@@ -78,16 +99,19 @@ __device__ __forceinline__ float ffn_gelu(float z)
 
 template <int D>
 __global__ void __launch_bounds__(FF_THREADS, 1)
-    ffn_tc_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW1,
-                  const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmY,
-                  const __grid_constant__ FfnParams P)
+    ffn_tc_kernel(const __grid_constant__ CUtensorMap tmH0, const __grid_constant__ CUtensorMap tmW10,
+                  const __grid_constant__ CUtensorMap tmW20, const __grid_constant__ CUtensorMap tmY0,
+                  const __grid_constant__ CUtensorMap tmH1, const __grid_constant__ CUtensorMap tmW11,
+                  const __grid_constant__ CUtensorMap tmW21, const __grid_constant__ CUtensorMap tmY1,
+                  const __grid_constant__ FfnMulti P)
 {
     using Sh = FfnShape<D>;
     constexpr int KS = Sh::KS;
     constexpr uint32_t IDESC1 = make_idesc(FF_BM, FF_BH1, 1, 0, 0);
     constexpr uint32_t IDESC2 = make_idesc(FF_BM, D, 1, 0, 0);
-    const FfnArgs &a = P.a;
+    const FfnArgs &a = P.q[0].a; // launch-wide: F, eps, wait control
     const int NC = a.F / FF_BH; // hidden chunks per tile
+    const bool two = P.tiles > P.split;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -160,24 +184,31 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
         const bool w1_side = warp == 0;
         if (lane == 0) {
             if (w1_side) {
-                tma_prefetch(&tmH);
-                tma_prefetch(&tmY);
+                tma_prefetch(&tmH0);
+                tma_prefetch(&tmY0);
+                if (two) {
+                    tma_prefetch(&tmH1);
+                    tma_prefetch(&tmY1);
+                }
             }
-            tma_prefetch(w1_side ? &tmW1 : &tmW2);
+            tma_prefetch(w1_side ? &tmW10 : &tmW20);
+            if (two) tma_prefetch(w1_side ? &tmW11 : &tmW21);
             long long gc = 0; // global chunk counter
             int tl = 0, n_h = 0;
             bool ok = true;
             for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x, ++tl) {
-                const int g = static_cast<int>(tile / P.m_tiles);
-                const int m0 = static_cast<int>(tile % P.m_tiles) * FF_BM;
+                int g, m0;
+                const int pi = ffn_tile(P, tile, g, m0);
+                const CUtensorMap *tH = pi ? &tmH1 : &tmH0;
+                const CUtensorMap *tW1 = pi ? &tmW11 : &tmW10, *tW2 = pi ? &tmW21 : &tmW20;
                 if (w1_side) {
                     if (!mbar_wait(h_free, (tl & 1) ^ 1, a.wait, abort_flag)) break;
                     mbar_arrive_expect_tx(h_full, Sh::H_BYTES);
                     for (int k = 0; k < KS; ++k) {
-                        if (P.grouped)
-                            tma_load_3d(sH + k * FF_SLAB, &tmH, h_full, k * 64, g, m0);
+                        if (P.q[pi].grouped)
+                            tma_load_3d(sH + k * FF_SLAB, tH, h_full, k * 64, g, m0);
                         else
-                            tma_load_3d(sH + k * FF_SLAB, &tmH, h_full, k * 64, m0, 0);
+                            tma_load_3d(sH + k * FF_SLAB, tH, h_full, k * 64, m0, 0);
                     }
                     ++n_h;
                 } else if (tl > 0 && !mbar_wait(stg_free, (tl - 1) & 1, a.wait, abort_flag)) {
@@ -194,7 +225,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                         }
                         mbar_arrive_expect_tx(&w1_full[st], Sh::W1_BYTES);
                         for (int k = 0; k < KS / 2; ++k)
-                            tma_load_3d(sW1 + st * Sh::W1_BYTES + k * FF_SLAB, &tmW1, &w1_full[st],
+                            tma_load_3d(sW1 + st * Sh::W1_BYTES + k * FF_SLAB, tW1, &w1_full[st],
                                         (st * (KS / 2) + k) * 64, (c >> 1) * FF_BH1, g);
                     } else {
                         if (!mbar_wait(&w2_empty[st], ph ^ 1, a.wait, abort_flag)) {
@@ -202,7 +233,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                             break;
                         }
                         mbar_arrive_expect_tx(&w2_full[st], Sh::W2_BYTES);
-                        tma_load_3d(sW2 + st * Sh::W2_BYTES, &tmW2, &w2_full[st], c * FF_BH, 0, g);
+                        tma_load_3d(sW2 + st * Sh::W2_BYTES, tW2, &w2_full[st], c * FF_BH, 0, g);
                     }
                 }
             }
@@ -301,8 +332,8 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
         int tl = 0;
         bool ok = true;
         for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x, ++tl) {
-            const int g = static_cast<int>(tile / P.m_tiles);
-            const int m0 = static_cast<int>(tile % P.m_tiles) * FF_BM;
+            int g, m0;
+            const int pi = ffn_tile(P, tile, g, m0);
             if (!mbar_wait(h_full, tl & 1, a.wait, abort_flag)) break;
             // This warp's half of its rows of H (columns hf*HALF ..): the
             // RMSNorm partial sum of squares, and the values in fp32 into
@@ -415,11 +446,12 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             fence_proxy_async_smem();
             named_bar_sync(1, 32 * FF_EPI_WARPS);
             if (warp == FF_EPI0 && lane == 0) {
+                const CUtensorMap *tY = pi ? &tmY1 : &tmY0;
                 for (int k = 0; k < KS; ++k) {
-                    if (P.grouped)
-                        tma_store_3d(&tmY, stg + k * FF_SLAB, k * 64, g, m0);
+                    if (P.q[pi].grouped)
+                        tma_store_3d(tY, stg + k * FF_SLAB, k * 64, g, m0);
                     else
-                        tma_store_3d(&tmY, stg + k * FF_SLAB, k * 64, m0, 0);
+                        tma_store_3d(tY, stg + k * FF_SLAB, k * 64, m0, 0);
                 }
                 bulk_commit_group();
                 bulk_wait_group_read0();
@@ -437,12 +469,11 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
     }
 }
 
+// tile count and tensor maps of one problem
 template <int D>
-static cudaError_t launch_ffn_cfg(const FfnArgs &a, cudaStream_t s)
+static cudaError_t prepare_ffn(const FfnArgs &a, FfnParams &p, CUtensorMap *tmH, CUtensorMap *tmW1,
+                               CUtensorMap *tmW2, CUtensorMap *tmY)
 {
-    using Sh = FfnShape<D>;
-    alignas(64) CUtensorMap tmH, tmW1, tmW2, tmY;
-    FfnParams p;
     p.a = a;
     p.grouped = a.G > 1 && a.h_map.Gs != 0;
     p.m_tiles = (a.M + FF_BM - 1) / FF_BM;
@@ -452,13 +483,13 @@ static cudaError_t launch_ffn_cfg(const FfnArgs &a, cudaStream_t s)
         uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.G), static_cast<uint64_t>(a.M)};
         uint64_t str[2] = {static_cast<uint64_t>(a.h_map.Gs) * D * 2, static_cast<uint64_t>(a.h_map.A) * D * 2};
         uint32_t box[3] = {64, 1, FF_BM};
-        if (encode_tmap_3d(&tmH, 2, Hbase, dims, str, box)) return cudaErrorInvalidValue;
+        if (encode_tmap_3d(tmH, 2, Hbase, dims, str, box)) return cudaErrorInvalidValue;
     } else {
         uint64_t rs = static_cast<uint64_t>(a.h_map.A) * D * 2;
         uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.M), 1};
         uint64_t str[2] = {rs, rs * static_cast<uint64_t>(a.M)};
         uint32_t box[3] = {64, FF_BM, 1};
-        if (encode_tmap_3d(&tmH, 2, Hbase, dims, str, box)) return cudaErrorInvalidValue;
+        if (encode_tmap_3d(tmH, 2, Hbase, dims, str, box)) return cudaErrorInvalidValue;
     }
     // Y: same row structure as H (rows of a tile are H's rows of the same
     // tile under y_map)
@@ -468,25 +499,46 @@ static cudaError_t launch_ffn_cfg(const FfnArgs &a, cudaStream_t s)
         uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.G), static_cast<uint64_t>(a.M)};
         uint64_t str[2] = {static_cast<uint64_t>(a.y_map.Gs) * D * 2, static_cast<uint64_t>(a.y_map.A) * D * 2};
         uint32_t box[3] = {64, 1, FF_BM};
-        if (encode_tmap_3d(&tmY, 2, Ybase, dims, str, box)) return cudaErrorInvalidValue;
+        if (encode_tmap_3d(tmY, 2, Ybase, dims, str, box)) return cudaErrorInvalidValue;
     } else {
         uint64_t rs = static_cast<uint64_t>(a.y_map.A) * D * 2;
         uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.M), 1};
         uint64_t str[2] = {rs, rs * static_cast<uint64_t>(a.M)};
         uint32_t box[3] = {64, FF_BM, 1};
-        if (encode_tmap_3d(&tmY, 2, Ybase, dims, str, box)) return cudaErrorInvalidValue;
+        if (encode_tmap_3d(tmY, 2, Ybase, dims, str, box)) return cudaErrorInvalidValue;
     }
     {
         uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.F), static_cast<uint64_t>(a.G)};
         uint64_t str[2] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(a.w1_gstride) * 2};
         uint32_t box[3] = {64, FF_BH1, 1};
-        if (encode_tmap_3d(&tmW1, 2, a.W1, dims, str, box)) return cudaErrorInvalidValue;
+        if (encode_tmap_3d(tmW1, 2, a.W1, dims, str, box)) return cudaErrorInvalidValue;
     }
     {
         uint64_t dims[3] = {static_cast<uint64_t>(a.F), static_cast<uint64_t>(D), static_cast<uint64_t>(a.G)};
         uint64_t str[2] = {static_cast<uint64_t>(a.F) * 2, static_cast<uint64_t>(a.w2_gstride) * 2};
         uint32_t box[3] = {64, static_cast<uint32_t>(D), 1};
-        if (encode_tmap_3d(&tmW2, 2, a.W2, dims, str, box)) return cudaErrorInvalidValue;
+        if (encode_tmap_3d(tmW2, 2, a.W2, dims, str, box)) return cudaErrorInvalidValue;
+    }
+    return cudaSuccess;
+}
+
+template <int D>
+static cudaError_t launch_ffn_cfg(const FfnArgs &a, const FfnArgs *a1, cudaStream_t s)
+{
+    using Sh = FfnShape<D>;
+    alignas(64) CUtensorMap tm[2][4];
+    FfnMulti P;
+    memset(&P, 0, sizeof(P));
+    cudaError_t e = prepare_ffn<D>(a, P.q[0], &tm[0][0], &tm[0][1], &tm[0][2], &tm[0][3]);
+    if (e != cudaSuccess) return e;
+    P.split = P.q[0].tiles;
+    P.tiles = P.split;
+    if (a1) {
+        if ((e = prepare_ffn<D>(*a1, P.q[1], &tm[1][0], &tm[1][1], &tm[1][2], &tm[1][3])) != cudaSuccess)
+            return e;
+        P.tiles += P.q[1].tiles;
+    } else {
+        for (int k = 0; k < 4; ++k) tm[1][k] = tm[0][k];
     }
     static int num_sms = 0;
     if (num_sms == 0) {
@@ -497,22 +549,28 @@ static cudaError_t launch_ffn_cfg(const FfnArgs &a, cudaStream_t s)
             num_sms = 148;
     }
     auto kern = ffn_tc_kernel<D>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(Sh::SMEM));
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Sh::SMEM));
     if (e != cudaSuccess) return e;
-    const long long grid = p.tiles < num_sms ? p.tiles : num_sms;
-    return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(FF_THREADS), Sh::SMEM, s, tmH, tmW1,
-                      tmW2, tmY, p);
+    const long long grid = P.tiles < num_sms ? P.tiles : num_sms;
+    return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(FF_THREADS), Sh::SMEM, s, tm[0][0],
+                      tm[0][1], tm[0][2], tm[0][3], tm[1][0], tm[1][1], tm[1][2], tm[1][3], P);
 }
 
 bool ffn_tc_supported(int D, int F) { return (D == 128 || D == 256) && F % FF_BH1 == 0 && F >= FF_BH1; }
 
-cudaError_t launch_ffn_tc(const FfnArgs &a, cudaStream_t s)
+static bool ffn_ok(const FfnArgs &a)
 {
-    if (!ffn_tc_supported(a.D, a.F) || a.M < 1 || a.G < 1 || a.h_map.P != 1 || a.y_map.P != 1)
-        return cudaErrorInvalidValue;
-    if (a.D == 256) return launch_ffn_cfg<256>(a, s);
-    return launch_ffn_cfg<128>(a, s);
+    return ffn_tc_supported(a.D, a.F) && a.M >= 1 && a.G >= 1 && a.h_map.P == 1 && a.y_map.P == 1;
 }
+
+cudaError_t launch_ffn_tc_multi(const FfnArgs &a, const FfnArgs *a1, cudaStream_t s)
+{
+    if (!ffn_ok(a)) return cudaErrorInvalidValue;
+    if (a1 && (!ffn_ok(*a1) || a1->D != a.D || a1->F != a.F || a1->eps != a.eps)) return cudaErrorInvalidValue;
+    if (a.D == 256) return launch_ffn_cfg<256>(a, a1, s);
+    return launch_ffn_cfg<128>(a, a1, s);
+}
+
+cudaError_t launch_ffn_tc(const FfnArgs &a, cudaStream_t s) { return launch_ffn_tc_multi(a, nullptr, s); }
 
 } // namespace ot

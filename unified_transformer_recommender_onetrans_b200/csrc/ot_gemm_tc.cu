@@ -25,6 +25,8 @@
 // A stage returns to the producer when its MMAs completed (tcgen05.commit)
 // and, for norm GEMMs, the four norm warps read it (their generic-proxy reads
 // are ordered before the next TMA write by fence.proxy.async).
+#include <cstring>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -59,6 +61,30 @@ struct TcGemmParams {
     int m_tiles, n_tiles;
     long long tiles;
 };
+
+// One launch over one or two problems with the same K, tile shape and norm
+// (the S and NS projections of a layer): problem 0's tiles, then problem 1's,
+// so the second fills the first's last partial wave.
+struct TcGemmMulti {
+    TcGemmParams q[2];
+    long long split; // first tile of problem 1 (= q[0].tiles)
+    long long tiles; // all tiles
+};
+
+// the problem a tile of the launch belongs to, and its tile index within it
+// (ONE: a single-problem launch; every parameter read then has a constant
+// offset, which the epilogue's per-tile reads depend on for speed)
+template <bool ONE>
+__device__ __forceinline__ int tile_problem(const TcGemmMulti &P, long long tile, long long &local)
+{
+    if (ONE) {
+        local = tile;
+        return 0;
+    }
+    const int pi = tile >= P.split ? 1 : 0;
+    local = tile - (pi ? P.split : 0);
+    return pi;
+}
 
 // exact-erf GELU, z * Phi(z), with Phi(z) ~ 1/2 + 1/2 tanh(z (A + B z^2)):
 // fitted A, B (max |Phi error| 1.4e-4) and the hardware tanh, six instructions
@@ -102,10 +128,11 @@ __device__ __forceinline__ bool rowmap_keep_dev(const RowMap &m, int r)
     return static_cast<long long>(static_cast<unsigned>(r) % P) >= m.min_t;
 }
 
-template <int BN, bool FP8>
+template <int BN, bool FP8, bool MULTI>
 __global__ void __launch_bounds__(G_THREADS, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ TcGemmParams P)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                   const __grid_constant__ TcGemmMulti P)
 {
     using Sh = GemmShape<BN>;
     constexpr int G_STAGES = Sh::STAGES;
@@ -114,7 +141,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     constexpr uint32_t G_STAGING = Sh::STAGING;
     constexpr int ROWB = G_EPI_COLS * 2; // staging row bytes
     constexpr uint32_t IDESC = make_idesc(G_BM, G_BN, FP8 ? 0 : 1, 0, 0);
-    const GemmArgs &a = P.a;
+    const GemmArgs &a0 = P.q[0].a; // launch-wide: K, norm, wait control
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -134,8 +161,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_kb = a.K / (FP8 ? 128 : 64);
-    const bool norm = a.norm != 0 && !FP8;
+    const int num_kb = a0.K / (FP8 ? 128 : 64);
+    const bool norm = a0.norm != 0 && !FP8;
     pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
@@ -152,8 +179,12 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
-        tma_prefetch(&tmA);
-        tma_prefetch(&tmB);
+        tma_prefetch(&tmA0);
+        tma_prefetch(&tmB0);
+        if (P.tiles > P.split) {
+            tma_prefetch(&tmA1);
+            tma_prefetch(&tmB1);
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 2 * G_BN);
@@ -164,7 +195,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // waits at the end ignore the abort flag and never use a test-lowered limit
-    const WaitCtl final_wait{a.wait.err, a.wait.limit > (1LL << 24) ? a.wait.limit : (1LL << 24)};
+    const WaitCtl wctl = a0.wait;
+    const WaitCtl final_wait{wctl.err, wctl.limit > (1LL << 24) ? wctl.limit : (1LL << 24)};
     volatile int no_abort = 0;
     pdl_wait(); // prologue done; from here on the previous kernel's memory is read / written
 
@@ -174,19 +206,23 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             long long it = 0;
             bool ok = true;
             for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x) {
+                long long lt;
+                const int pi = tile_problem<!MULTI>(P, tile, lt);
+                const TcGemmParams &Q = P.q[pi];
+                const CUtensorMap *tA = pi ? &tmA1 : &tmA0, *tB = pi ? &tmB1 : &tmB0;
                 int g, m0, n0;
-                decode_tile(P, tile, G_BN, g, m0, n0);
+                decode_tile(Q, lt, G_BN, g, m0, n0);
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const int s = static_cast<int>(it % G_STAGES);
                     const uint32_t ph = static_cast<uint32_t>((it / G_STAGES) & 1);
-                    if (!mbar_wait(&empty[s], ph ^ 1, a.wait, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(&empty[s], ph ^ 1, wctl, abort_flag)) { ok = false; break; }
                     mbar_arrive_expect_tx(&full[s], Sh::A_BYTES + Sh::B_BYTES);
                     const int kx = kb * (FP8 ? 128 : 64);
-                    if (P.a_grouped)
-                        tma_load_3d(sA + s * Sh::A_BYTES, &tmA, &full[s], kx, g, m0);
+                    if (Q.a_grouped)
+                        tma_load_3d(sA + s * Sh::A_BYTES, tA, &full[s], kx, g, m0);
                     else
-                        tma_load_3d(sA + s * Sh::A_BYTES, &tmA, &full[s], kx, m0, 0);
-                    tma_load_3d(sB + s * Sh::B_BYTES, &tmB, &full[s], kx, n0, g);
+                        tma_load_3d(sA + s * Sh::A_BYTES, tA, &full[s], kx, m0, 0);
+                    tma_load_3d(sB + s * Sh::B_BYTES, tB, &full[s], kx, n0, g);
                 }
             }
             // never leave a load in flight
@@ -202,12 +238,12 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             bool ok = true;
             for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x, ++t) {
                 const int b = t & 1;
-                if (!mbar_wait(&tempty[b], ((t >> 1) & 1) ^ 1, a.wait, abort_flag)) break;
+                if (!mbar_wait(&tempty[b], ((t >> 1) & 1) ^ 1, wctl, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t acc = tmem + b * G_BN;
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const int s = static_cast<int>(it % G_STAGES);
-                    if (!mbar_wait(&full[s], static_cast<uint32_t>((it / G_STAGES) & 1), a.wait,
+                    if (!mbar_wait(&full[s], static_cast<uint32_t>((it / G_STAGES) & 1), wctl,
                                    abort_flag)) {
                         ok = false;
                         break;
@@ -238,11 +274,14 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         const int q = warp & 3;              // TMEM lane quarter = rows 32q .. 32q+31
         const int half = (warp - 2) >> 2;    // columns 64*half .. 64*half+63 of the tile
         uint8_t *stage = sOut + (warp - 2) * G_STAGING;
-        const __nv_bfloat16 *res = static_cast<const __nv_bfloat16 *>(a.res);
         int t = 0;
         for (long long tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++t) {
+            long long lt;
+            const TcGemmParams &Q = P.q[tile_problem<!MULTI>(P, tile, lt)];
+            const GemmArgs &a = Q.a;
+            const __nv_bfloat16 *res = static_cast<const __nv_bfloat16 *>(a.res);
             int g, m0, n0;
-            decode_tile(P, tile, G_BN, g, m0, n0);
+            decode_tile(Q, lt, G_BN, g, m0, n0);
             const int b = t & 1;
             const int c0 = n0 + half * G_EPI_COLS; // first output column of this warp
             const int r = m0 + 32 * q + lane;      // this lane's row
@@ -274,11 +313,11 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                 for (int i = 0; i < 32 / RPI; ++i)
                     *stage_chunk<ROWB>(stage, RPI * i + lane / LPR, lane % LPR) = rv[i];
             }
-            if (!mbar_wait(&tfull[b], (t >> 1) & 1, a.wait, abort_flag)) break;
+            if (!mbar_wait(&tfull[b], (t >> 1) & 1, wctl, abort_flag)) break;
             tc_fence_after();
             float rs = 1.f;
             if (norm) {
-                if (!mbar_wait(&nfull[b], (t >> 1) & 1, a.wait, abort_flag)) break;
+                if (!mbar_wait(&nfull[b], (t >> 1) & 1, wctl, abort_flag)) break;
                 rs = rsqrtf(ssbuf[b * G_BM + 32 * q + lane] / static_cast<float>(a.K) + a.eps);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&nempty[b]);
@@ -342,11 +381,11 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         bool ok = true;
         for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x, ++t) {
             const int b = t & 1;
-            if (!mbar_wait(&nempty[b], ((t >> 1) & 1) ^ 1, a.wait, abort_flag)) break;
+            if (!mbar_wait(&nempty[b], ((t >> 1) & 1) ^ 1, wctl, abort_flag)) break;
             float ss = 0.f;
             for (int kb = 0; kb < num_kb; ++kb, ++it) {
                 const int s = static_cast<int>(it % G_STAGES);
-                if (!mbar_wait(&full[s], static_cast<uint32_t>((it / G_STAGES) & 1), a.wait,
+                if (!mbar_wait(&full[s], static_cast<uint32_t>((it / G_STAGES) & 1), wctl,
                                abort_flag)) {
                     ok = false;
                     break;
@@ -388,15 +427,13 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 
 static int g_num_sms = 0;
 
+// tile counts and the operand tensor maps of one problem
 template <int BN, bool FP8>
-static cudaError_t launch_tc_cfg(const GemmArgs &a, cudaStream_t s)
+static cudaError_t prepare_problem(const GemmArgs &a, TcGemmParams &p, CUtensorMap *tmA, CUtensorMap *tmB)
 {
     constexpr int G_BN = BN;
-    using Sh = GemmShape<BN>;
     const int esz = FP8 ? 1 : 2;
     const int kbox = FP8 ? 128 : 64;
-    alignas(64) CUtensorMap tmA, tmB;
-    TcGemmParams p;
     p.a = a;
     p.a_grouped = a.G > 1 && a.a_map.Gs != 0;
     p.m_tiles = (a.M + G_BM - 1) / G_BM;
@@ -409,23 +446,42 @@ static cudaError_t launch_tc_cfg(const GemmArgs &a, cudaStream_t s)
         uint64_t str[2] = {static_cast<uint64_t>(a.a_map.Gs * a.lda * esz),
                            static_cast<uint64_t>(a.a_map.A * a.lda * esz)};
         uint32_t box[3] = {static_cast<uint32_t>(kbox), 1, G_BM};
-        if (encode_tmap_3d(&tmA, esz, Abase, dims, str, box)) return cudaErrorInvalidValue;
+        if (encode_tmap_3d(tmA, esz, Abase, dims, str, box)) return cudaErrorInvalidValue;
     } else {
         uint64_t dims[3] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M), 1};
         uint64_t rs = static_cast<uint64_t>(a.a_map.A * a.lda * esz);
         uint64_t str[2] = {rs, rs * static_cast<uint64_t>(a.M)};
         uint32_t box[3] = {static_cast<uint32_t>(kbox), G_BM, 1};
-        if (encode_tmap_3d(&tmA, esz, Abase, dims, str, box)) return cudaErrorInvalidValue;
+        if (encode_tmap_3d(tmA, esz, Abase, dims, str, box)) return cudaErrorInvalidValue;
     }
-    {
-        uint64_t dims[3] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.N),
-                            static_cast<uint64_t>(a.G)};
-        uint64_t str[2] = {static_cast<uint64_t>(a.K) * esz,
-                           static_cast<uint64_t>(a.b_gstride > 0 ? a.b_gstride
-                                                                 : static_cast<long long>(a.N) * a.K) *
-                               esz};
-        uint32_t box[3] = {static_cast<uint32_t>(kbox), G_BN, 1};
-        if (encode_tmap_3d(&tmB, esz, a.B, dims, str, box)) return cudaErrorInvalidValue;
+    uint64_t dims[3] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.N),
+                        static_cast<uint64_t>(a.G)};
+    uint64_t str[2] = {static_cast<uint64_t>(a.K) * esz,
+                       static_cast<uint64_t>(a.b_gstride > 0 ? a.b_gstride
+                                                             : static_cast<long long>(a.N) * a.K) *
+                           esz};
+    uint32_t box[3] = {static_cast<uint32_t>(kbox), G_BN, 1};
+    if (encode_tmap_3d(tmB, esz, a.B, dims, str, box)) return cudaErrorInvalidValue;
+    return cudaSuccess;
+}
+
+template <int BN, bool FP8, bool MULTI>
+static cudaError_t launch_tc_cfg(const GemmArgs &a, const GemmArgs *a1, cudaStream_t s)
+{
+    using Sh = GemmShape<BN>;
+    alignas(64) CUtensorMap tmA0, tmB0, tmA1, tmB1;
+    TcGemmMulti P;
+    memset(&P, 0, sizeof(P));
+    cudaError_t e = prepare_problem<BN, FP8>(a, P.q[0], &tmA0, &tmB0);
+    if (e != cudaSuccess) return e;
+    P.split = P.q[0].tiles;
+    P.tiles = P.split;
+    if (a1) {
+        if ((e = prepare_problem<BN, FP8>(*a1, P.q[1], &tmA1, &tmB1)) != cudaSuccess) return e;
+        P.tiles += P.q[1].tiles;
+    } else {
+        tmA1 = tmA0;
+        tmB1 = tmB0;
     }
     if (g_num_sms == 0) {
         int dev = 0;
@@ -434,28 +490,51 @@ static cudaError_t launch_tc_cfg(const GemmArgs &a, cudaStream_t s)
             g_num_sms < 1)
             g_num_sms = 148;
     }
-    auto kern = gemm_tc_kernel<BN, FP8>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(Sh::SMEM));
+    auto kern = gemm_tc_kernel<BN, FP8, MULTI>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Sh::SMEM));
     if (e != cudaSuccess) return e;
-    const long long grid = p.tiles < g_num_sms ? p.tiles : g_num_sms;
-    return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(G_THREADS), Sh::SMEM, s, tmA,
-                      tmB, p);
+    const long long grid = P.tiles < g_num_sms ? P.tiles : g_num_sms;
+    return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(G_THREADS), Sh::SMEM, s, tmA0,
+                      tmB0, tmA1, tmB1, P);
+}
+
+// shape checks of one problem; wide: 128 x 256 tiles fit its column segments
+static bool gemm_ok(const GemmArgs &a, bool &wide)
+{
+    const bool fp8 = a.in_dtype == OT_DTYPE_FP8;
+    if (a.store != OT_STORE_BF16) return false;
+    if (a.K % (fp8 ? 128 : 64) != 0 || a.a_map.P != 1 || a.N % 128 != 0 || a.M < 1 || a.G < 1)
+        return false;
+    wide = a.N % 256 == 0;
+    for (int i = 0; i < a.nseg; ++i) {
+        if (a.seg[i].c_lo % 128 || a.seg[i].c_hi % 128) return false;
+        if (a.seg[i].c_lo % 256 || a.seg[i].c_hi % 256) wide = false;
+    }
+    return true;
+}
+
+cudaError_t launch_gemm_tc_multi(const GemmArgs &a, const GemmArgs *a1, cudaStream_t s)
+{
+    bool wide = false, wide1 = true;
+    if (!gemm_ok(a, wide)) return cudaErrorInvalidValue;
+    const bool fp8 = a.in_dtype == OT_DTYPE_FP8;
+    if (a1) {
+        // one launch-wide K and norm, bf16 / fp32 operands
+        if (fp8 || !gemm_ok(*a1, wide1) || a1->K != a.K || a1->in_dtype == OT_DTYPE_FP8 ||
+            (a1->norm != 0) != (a.norm != 0))
+            return cudaErrorInvalidValue;
+    }
+    if (a1) {
+        if (wide && wide1) return launch_tc_cfg<256, false, true>(a, a1, s);
+        return launch_tc_cfg<128, false, true>(a, a1, s);
+    }
+    if (wide) return fp8 ? launch_tc_cfg<256, true, false>(a, a1, s) : launch_tc_cfg<256, false, false>(a, a1, s);
+    return fp8 ? launch_tc_cfg<128, true, false>(a, a1, s) : launch_tc_cfg<128, false, false>(a, a1, s);
 }
 
 cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s)
 {
-    const bool fp8 = a.in_dtype == OT_DTYPE_FP8;
-    if (a.store != OT_STORE_BF16) return cudaErrorInvalidValue;
-    if (a.K % (fp8 ? 128 : 64) != 0 || a.a_map.P != 1 || a.N % 128 != 0 || a.M < 1)
-        return cudaErrorInvalidValue;
-    bool wide = a.N % 256 == 0;
-    for (int i = 0; i < a.nseg; ++i) {
-        if (a.seg[i].c_lo % 128 || a.seg[i].c_hi % 128) return cudaErrorInvalidValue;
-        if (a.seg[i].c_lo % 256 || a.seg[i].c_hi % 256) wide = false;
-    }
-    if (wide) return fp8 ? launch_tc_cfg<256, true>(a, s) : launch_tc_cfg<256, false>(a, s);
-    return fp8 ? launch_tc_cfg<128, true>(a, s) : launch_tc_cfg<128, false>(a, s);
+    return launch_gemm_tc_multi(a, nullptr, s);
 }
 
 } // namespace ot

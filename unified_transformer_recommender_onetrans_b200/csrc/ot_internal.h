@@ -139,10 +139,14 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 // Launchers (return cudaGetLastError() after the launch).
 cudaError_t launch_gemm_simt(const GemmArgs &a, cudaStream_t s);
 cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s);
+// two problems with the same K, operand dtype and norm in one launch (a1 may be null)
+cudaError_t launch_gemm_tc_multi(const GemmArgs &a, const GemmArgs *a1, cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s);
 bool ffn_tc_supported(int D, int F);
 cudaError_t launch_ffn_tc(const FfnArgs &a, cudaStream_t s);
+// two problems with the same D, F and eps in one launch (a1 may be null)
+cudaError_t launch_ffn_tc_multi(const FfnArgs &a, const FfnArgs *a1, cudaStream_t s);
 cudaError_t launch_fold_gain(const void *W, const void *g, void *out, long long rows, int cols,
                              long long groups, long long g_gstride, int dtype, cudaStream_t s);
 cudaError_t launch_embed_gather(const void *table, long long rows, int d, const int64_t *ids,
