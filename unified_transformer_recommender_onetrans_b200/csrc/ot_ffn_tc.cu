@@ -177,7 +177,9 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
     const uint32_t t_acc2 = tmem, t_acc1 = tmem + D;
     const WaitCtl final_wait{a.wait.err, a.wait.limit > (1LL << 24) ? a.wait.limit : (1LL << 24)};
     volatile int no_abort = 0;
-    pdl_wait(); // prologue done; from here on the previous kernel's memory is read / written
+    // prologue done; from here on the previous kernel's memory is read / written
+    // (the producers wait after issuing the weight loads that do not depend on it)
+    if (warp != 0 && warp != 3) pdl_wait();
 
     if (warp == 0 || warp == 3) {
         // ------------------------------------------------ TMA producers
@@ -193,6 +195,28 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             }
             tma_prefetch(w1_side ? &tmW10 : &tmW20);
             if (two) tma_prefetch(w1_side ? &tmW11 : &tmW21);
+            // The weights are not written by any kernel in flight: the first
+            // tile's first two W1 / W2 stages load while the previous kernel
+            // finishes (fresh stages, no empty wait); H follows once its
+            // outputs are visible.
+            const int n_pre = static_cast<long long>(blockIdx.x) < P.tiles ? (NC < 2 ? NC : 2) : 0;
+            if (n_pre > 0) {
+                int g, m0;
+                const int pi = ffn_tile(P, blockIdx.x, g, m0);
+                const CUtensorMap *tW1 = pi ? &tmW11 : &tmW10, *tW2 = pi ? &tmW21 : &tmW20;
+                for (int c = 0; c < n_pre; ++c) {
+                    if (w1_side) {
+                        mbar_arrive_expect_tx(&w1_full[c], Sh::W1_BYTES);
+                        for (int k = 0; k < KS / 2; ++k)
+                            tma_load_3d(sW1 + c * Sh::W1_BYTES + k * FF_SLAB, tW1, &w1_full[c],
+                                        (c * (KS / 2) + k) * 64, (c >> 1) * FF_BH1, g);
+                    } else {
+                        mbar_arrive_expect_tx(&w2_full[c], Sh::W2_BYTES);
+                        tma_load_3d(sW2 + c * Sh::W2_BYTES, tW2, &w2_full[c], c * FF_BH, 0, g);
+                    }
+                }
+            }
+            pdl_wait();
             long long gc = 0; // global chunk counter
             int tl = 0, n_h = 0;
             bool ok = true;
@@ -217,6 +241,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                 for (int c = 0; c < NC; ++c, ++gc) {
                     const int st = static_cast<int>(gc & 1);
                     const uint32_t ph = static_cast<uint32_t>((gc >> 1) & 1);
+                    if (gc < n_pre) continue; // issued before the wait
                     if (w1_side) {
                         // FFN1 chunk gc / 2 (128 hidden rows of W1), its K-half gc % 2
                         if (!mbar_wait(&w1_empty[st], ph ^ 1, a.wait, abort_flag)) {

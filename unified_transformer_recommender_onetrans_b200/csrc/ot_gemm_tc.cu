@@ -198,11 +198,31 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const WaitCtl wctl = a0.wait;
     const WaitCtl final_wait{wctl.err, wctl.limit > (1LL << 24) ? wctl.limit : (1LL << 24)};
     volatile int no_abort = 0;
-    pdl_wait(); // prologue done; from here on the previous kernel's memory is read / written
+    // prologue done; from here on the previous kernel's memory is read / written
+    // (the producer waits after issuing the weight loads that do not depend on it)
+    if (warp != 0) pdl_wait();
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
+            // The weights are not written by any kernel in flight: the first
+            // tile's B tiles of the first stages load while the previous
+            // kernel finishes (the stages are fresh, so no empty wait); their
+            // A tiles follow once its outputs are visible.
+            int n_pre = 0;
+            if (static_cast<long long>(blockIdx.x) < P.tiles) {
+                long long lt;
+                const int pi = tile_problem<!MULTI>(P, blockIdx.x, lt);
+                const CUtensorMap *tB = pi ? &tmB1 : &tmB0;
+                int g, m0, n0;
+                decode_tile(P.q[pi], lt, G_BN, g, m0, n0);
+                n_pre = num_kb < G_STAGES ? num_kb : G_STAGES;
+                for (int kb = 0; kb < n_pre; ++kb) {
+                    mbar_arrive_expect_tx(&full[kb], Sh::A_BYTES + Sh::B_BYTES);
+                    tma_load_3d(sB + kb * Sh::B_BYTES, tB, &full[kb], kb * (FP8 ? 128 : 64), n0, g);
+                }
+            }
+            pdl_wait();
             long long it = 0;
             bool ok = true;
             for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x) {
@@ -215,14 +235,17 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const int s = static_cast<int>(it % G_STAGES);
                     const uint32_t ph = static_cast<uint32_t>((it / G_STAGES) & 1);
-                    if (!mbar_wait(&empty[s], ph ^ 1, wctl, abort_flag)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&full[s], Sh::A_BYTES + Sh::B_BYTES);
+                    const bool pre = it < n_pre; // B already issued, transaction bytes armed
+                    if (!pre) {
+                        if (!mbar_wait(&empty[s], ph ^ 1, wctl, abort_flag)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&full[s], Sh::A_BYTES + Sh::B_BYTES);
+                    }
                     const int kx = kb * (FP8 ? 128 : 64);
                     if (Q.a_grouped)
                         tma_load_3d(sA + s * Sh::A_BYTES, tA, &full[s], kx, g, m0);
                     else
                         tma_load_3d(sA + s * Sh::A_BYTES, tA, &full[s], kx, m0, 0);
-                    tma_load_3d(sB + s * Sh::B_BYTES, tB, &full[s], kx, n0, g);
+                    if (!pre) tma_load_3d(sB + s * Sh::B_BYTES, tB, &full[s], kx, n0, g);
                 }
             }
             // never leave a load in flight
