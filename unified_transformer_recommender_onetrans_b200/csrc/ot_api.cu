@@ -12,9 +12,9 @@
 // Per layer of the NS-side (score, U users x C candidates x N tokens):
 //   the same four steps with grouped GEMMs (group = NS position n, its own
 //   weights), and NS attention against layer l of the cache.
-// Full forward (both sides): steps 3 and 4 of the two sides share one launch
-// each (the NS tiles fill the S launch's last partial wave); the NS QKV and
-// attention run on a second stream beside the S attention.
+// Full forward (both sides): steps 1, 3 and 4 of the two sides share one
+// launch each (the NS tiles fill the S launch's last partial wave); the NS
+// attention runs on a second stream beside the S attention.
 #include <cudaTypedefs.h>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -188,7 +188,7 @@ size_t score_ws_bytes(const ot_config &c, int U, int C, int esz)
 enum { ROLE_S_QKV = 0, ROLE_S_ATTN, ROLE_S_O, ROLE_S_FFN1, ROLE_S_FFN2, ROLE_NS_QKV, ROLE_NS_ATTN,
        ROLE_NS_O, ROLE_NS_FFN1, ROLE_NS_FFN2, ROLE_AUTO_SPLIT, ROLE_OTHER, ROLE_S_FFN, ROLE_NS_FFN,
        // one launch for the S and NS sides of a layer (full forward)
-       ROLE_O, ROLE_FFN };
+       ROLE_O, ROLE_FFN, ROLE_QKV };
 
 cudaEvent_t pooled_event(ot_model *m)
 {
@@ -668,12 +668,12 @@ bool merged_supported(const ot_model *m)
     return use_fused_ffn(m) && m->cfg.d / m->cfg.heads == 64;
 }
 
-// Full forward with the S and NS sides sharing the O-projection and FFN
+// Full forward with the S and NS sides sharing the QKV, O-projection and FFN
 // launches of each layer: the NS work units come after the S ones and fill
 // the S launches' last partial waves (at small C a whole NS step costs
-// almost nothing there).  The NS QKV projection and attention of layer l run
-// on the side stream once layer l's S K/V are cached, beside the S attention;
-// the merged O launch waits for them.  Same arithmetic, buffers and workspace
+// almost nothing there).  The NS attention of layer l runs on the side
+// stream once the layer's QKV launch is done, beside the S attention; the
+// merged O launch waits for it.  Same arithmetic, buffers and workspace
 // layouts as run_encode + run_score.
 ot_status run_full_merged(ot_model *m, const void *X0, int U, const void *ns, int C, void *kv,
                           void *s_out, void *out, Ws ws_enc, Ws ws_sc, cudaStream_t st)
@@ -708,7 +708,7 @@ ot_status run_full_merged(ot_model *m, const void *X0, int U, const void *ns, in
         char *V = K + static_cast<long long>(L) * d * m->esz;
         const RowMap cache_map{L, ustride / d, 0, 0, 0};
         const long long lN = static_cast<long long>(l) * N;
-        // 1. S QKV: K / V into the cache, Q of the tail rows
+        // 1. QKV: S rows (K / V into the cache, Q of the tail rows) and NS rows
         GemmArgs gs = gemm_base(c, U * L, 3 * d, d, 1);
         if ((r = projection(m, gs, X, d, rowmap_identity(),
                             at(m->Wqkv_s, static_cast<long long>(l) * 3 * d * d, m->esz), 3LL * d * d, nullptr,
@@ -718,21 +718,20 @@ ot_status run_full_merged(ot_model *m, const void *X0, int U, const void *ns, in
         gs.seg[0] = seg_of(Qb, d, 0, d, RowMap{L, q, -(L - q), 0, L - q});
         gs.seg[1] = seg_of(K, d, d, 2 * d, cache_map);
         gs.seg[2] = seg_of(V, d, 2 * d, 3 * d, cache_map);
-        if ((r = gemm(m, gs, st, ROLE_S_QKV)) != OT_OK) return r;
-        // the NS side of this layer needs these K/V and the previous layer's NS output
-        if (two && (cudaEventRecord(m->kv_ready[l], st) != cudaSuccess ||
-                    cudaStreamWaitEvent(side, m->kv_ready[l], 0) != cudaSuccess))
-            return OT_ERR_CUDA;
-        // 2. NS QKV + NS attention (side stream)
+        // NS rows of the same layer, in the same launch
         GemmArgs gn = gemm_base(c, Mc, 3 * d, d, N);
         if ((r = projection(m, gn, Y, d, grp, at(m->Wqkv_ns, lN * 3 * d * d, m->esz), 3LL * d * d, nullptr,
-                            nullptr, d, true, no_f8, side)) != OT_OK)
+                            nullptr, d, true, no_f8, st)) != OT_OK)
             return r;
         gn.nseg = 3;
         gn.seg[0] = seg_of(Qn, d, 0, d, grp);
         gn.seg[1] = seg_of(Kn, d, d, 2 * d, grp);
         gn.seg[2] = seg_of(Vn, d, 2 * d, 3 * d, grp);
-        if ((r = gemm(m, gn, side, ROLE_NS_QKV)) != OT_OK) return r;
+        if ((r = gemm2(m, &gs, &gn, st, ROLE_QKV)) != OT_OK) return r;
+        // 2. NS attention (side stream) needs this layer's S K/V and NS Q/K/V
+        if (two && (cudaEventRecord(m->kv_ready[l], st) != cudaSuccess ||
+                    cudaStreamWaitEvent(side, m->kv_ready[l], 0) != cudaSuccess))
+            return OT_ERR_CUDA;
         AttnArgs as_, an_;
         memset(&as_, 0, sizeof(as_));
         as_.mode = 0;

@@ -128,6 +128,62 @@ __device__ __forceinline__ bool rowmap_keep_dev(const RowMap &m, int r)
     return static_cast<long long>(static_cast<unsigned>(r) % P) >= m.min_t;
 }
 
+// Everything the epilogue needs from a tile's problem, read at constant
+// offsets of the parameter block (called once per problem with P.q[0] /
+// P.q[1] and the results selected: runtime indexing into the parameters
+// turns every read into a dependent global load on the tile's critical path).
+struct EpiTile {
+    int g, m0, n0;
+    int M, gelu;
+    long long out_off;          // this lane's row in the output segment (-1: not stored)
+    long long res_off;          // this lane's row in the residual
+    const __nv_bfloat16 *res;   // null: no residual
+    __nv_bfloat16 *obase;       // output segment base
+    const float *row_scale;     // fp8: per-row scale (indexed through the A row map), or null
+    long long row_scale_idx;
+    float g_scale;              // fp8: per-matrix scale (1 otherwise)
+    float inv_k, eps;           // RMSNorm
+};
+
+// the tile's residual rows first: their loads are the epilogue's longest wait
+template <int BN>
+__device__ __forceinline__ void epi_res(const TcGemmParams &Q, long long lt, int q, int lane, int half, EpiTile &e)
+{
+    const GemmArgs &a = Q.a;
+    decode_tile(Q, lt, BN, e.g, e.m0, e.n0);
+    e.M = a.M;
+    const int r = e.m0 + 32 * q + lane;
+    e.res = static_cast<const __nv_bfloat16 *>(a.res);
+    e.res_off = 0;
+    if (r < a.M && e.res) e.res_off = rowmap_dev(a.res_map, r, e.g) * a.res_ld + e.n0 + half * (BN / 2);
+}
+
+template <int BN>
+__device__ __forceinline__ void epi_tile(const TcGemmParams &Q, int q, int lane, int half, EpiTile &e)
+{
+    const GemmArgs &a = Q.a;
+    e.gelu = a.gelu;
+    e.inv_k = 1.f / static_cast<float>(a.K);
+    e.eps = a.eps;
+    const int c0 = e.n0 + half * (BN / 2); // first output column of this warp
+    const int r = e.m0 + 32 * q + lane;    // this lane's row
+    const bool live = r < a.M;
+    // column segment of the tile (at most three): constant indices only
+    const EpiSeg &s0 = a.seg[0], &s1 = a.seg[1], &s2 = a.seg[2];
+    const int sidx = (a.nseg < 2 || (e.n0 >= s0.c_lo && e.n0 < s0.c_hi))   ? 0
+                     : (a.nseg < 3 || (e.n0 >= s1.c_lo && e.n0 < s1.c_hi)) ? 1
+                                                                            : 2;
+#define OT_SEGF(f) (sidx == 0 ? s0.f : sidx == 1 ? s1.f : s2.f)
+    const RowMap mp{OT_SEGF(map.P), OT_SEGF(map.A), OT_SEGF(map.B), OT_SEGF(map.Gs), OT_SEGF(map.min_t)};
+    e.obase = static_cast<__nv_bfloat16 *>(OT_SEGF(out));
+    e.out_off = -1;
+    if (live && rowmap_keep_dev(mp, r)) e.out_off = rowmap_dev(mp, r, e.g) * OT_SEGF(ld) + (c0 - OT_SEGF(c_lo));
+#undef OT_SEGF
+    e.row_scale = live ? a.row_scale : nullptr;
+    e.row_scale_idx = e.row_scale ? rowmap_dev(a.a_map, r, e.g) : 0;
+    e.g_scale = a.g_scale ? a.g_scale[e.g] : 1.f;
+}
+
 template <int BN, bool FP8, bool MULTI>
 __global__ void __launch_bounds__(G_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
@@ -228,10 +284,16 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x) {
                 long long lt;
                 const int pi = tile_problem<!MULTI>(P, tile, lt);
-                const TcGemmParams &Q = P.q[pi];
                 const CUtensorMap *tA = pi ? &tmA1 : &tmA0, *tB = pi ? &tmB1 : &tmB0;
                 int g, m0, n0;
-                decode_tile(Q, lt, G_BN, g, m0, n0);
+                int a_grouped;
+                if (MULTI && pi) {
+                    decode_tile(P.q[1], lt, G_BN, g, m0, n0);
+                    a_grouped = P.q[1].a_grouped;
+                } else {
+                    decode_tile(P.q[0], lt, G_BN, g, m0, n0);
+                    a_grouped = P.q[0].a_grouped;
+                }
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const int s = static_cast<int>(it % G_STAGES);
                     const uint32_t ph = static_cast<uint32_t>((it / G_STAGES) & 1);
@@ -241,7 +303,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                         mbar_arrive_expect_tx(&full[s], Sh::A_BYTES + Sh::B_BYTES);
                     }
                     const int kx = kb * (FP8 ? 128 : 64);
-                    if (Q.a_grouped)
+                    if (a_grouped)
                         tma_load_3d(sA + s * Sh::A_BYTES, tA, &full[s], kx, g, m0);
                     else
                         tma_load_3d(sA + s * Sh::A_BYTES, tA, &full[s], kx, m0, 0);
@@ -300,23 +362,17 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         int t = 0;
         for (long long tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++t) {
             long long lt;
-            const TcGemmParams &Q = P.q[tile_problem<!MULTI>(P, tile, lt)];
-            const GemmArgs &a = Q.a;
-            const __nv_bfloat16 *res = static_cast<const __nv_bfloat16 *>(a.res);
-            int g, m0, n0;
-            decode_tile(Q, lt, G_BN, g, m0, n0);
-            const int b = t & 1;
-            const int c0 = n0 + half * G_EPI_COLS; // first output column of this warp
-            const int r = m0 + 32 * q + lane;      // this lane's row
-            const bool live = r < a.M;
+            const int pi = tile_problem<!MULTI>(P, tile, lt);
             // per-row addresses, computed once by the lane that owns the row
-            int sidx = 0;
-            while (sidx + 1 < a.nseg && !(n0 >= a.seg[sidx].c_lo && n0 < a.seg[sidx].c_hi)) ++sidx;
-            const EpiSeg &sg = a.seg[sidx];
-            long long out_off = -1, res_off = 0;
-            if (live && rowmap_keep_dev(sg.map, r))
-                out_off = rowmap_dev(sg.map, r, g) * sg.ld + (c0 - sg.c_lo);
-            if (live && res) res_off = rowmap_dev(a.res_map, r, g) * a.res_ld + c0;
+            EpiTile et;
+            if (MULTI && pi)
+                epi_res<G_BN>(P.q[1], lt, q, lane, half, et);
+            else
+                epi_res<G_BN>(P.q[0], lt, q, lane, half, et);
+            const __nv_bfloat16 *res = et.res;
+            const int m0 = et.m0;
+            const int b = t & 1;
+            const long long res_off = et.res_off;
             constexpr int LPR = ROWB / 16;       // lanes per staged row
             constexpr int RPI = 32 / LPR;        // rows per warp instruction
             if (res) {
@@ -329,24 +385,29 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                     const int rl = RPI * i + lane / LPR, ch = lane % LPR;
                     const long long ro = __shfl_sync(0xffffffffu, res_off, rl);
                     rv[i] = make_uint4(0, 0, 0, 0);
-                    if (m0 + 32 * q + rl < a.M)
+                    if (m0 + 32 * q + rl < et.M)
                         rv[i] = __ldg(reinterpret_cast<const uint4 *>(res + ro + ch * 8));
                 }
 #pragma unroll
                 for (int i = 0; i < 32 / RPI; ++i)
                     *stage_chunk<ROWB>(stage, RPI * i + lane / LPR, lane % LPR) = rv[i];
             }
+            if (MULTI && pi)
+                epi_tile<G_BN>(P.q[1], q, lane, half, et);
+            else
+                epi_tile<G_BN>(P.q[0], q, lane, half, et);
+            const long long out_off = et.out_off;
             if (!mbar_wait(&tfull[b], (t >> 1) & 1, wctl, abort_flag)) break;
             tc_fence_after();
             float rs = 1.f;
             if (norm) {
                 if (!mbar_wait(&nfull[b], (t >> 1) & 1, wctl, abort_flag)) break;
-                rs = rsqrtf(ssbuf[b * G_BM + 32 * q + lane] / static_cast<float>(a.K) + a.eps);
+                rs = rsqrtf(ssbuf[b * G_BM + 32 * q + lane] * et.inv_k + et.eps);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&nempty[b]);
             }
-            if (live && a.row_scale) rs *= a.row_scale[rowmap_dev(a.a_map, r, g)];
-            if (a.g_scale) rs *= a.g_scale[g];
+            if (et.row_scale) rs *= et.row_scale[et.row_scale_idx];
+            rs *= et.g_scale;
             __syncwarp(); // residual staging complete before rows are read back
 #pragma unroll 1
             for (int c = 0; c < G_EPI_COLS / 32; ++c) {
@@ -363,7 +424,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         f[e] = __uint_as_float(v[8 * j + e]) * rs;
-                        if (a.gelu) f[e] = gelu_fast(f[e]);
+                        if (et.gelu) f[e] = gelu_fast(f[e]);
                     }
                     if (res) {
                         const uint4 x = *p;
@@ -386,7 +447,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[b]); // accumulator b may be overwritten
             // coalesced stores: LPR lanes per row, ROWB contiguous bytes
-            __nv_bfloat16 *obase = static_cast<__nv_bfloat16 *>(sg.out);
+            __nv_bfloat16 *obase = et.obase;
 #pragma unroll
             for (int i = 0; i < 32 / RPI; ++i) {
                 const int rl = RPI * i + lane / LPR, ch = lane % LPR;
