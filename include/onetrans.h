@@ -216,7 +216,8 @@ ot_status ot_set_kernel_path(ot_model *m, int path);
  * (negative on error).  Records beyond an internal 1 << 16 are dropped. */
 typedef enum {
     OT_KIND_GEMM_TC = 0, OT_KIND_GEMM_SIMT = 1, OT_KIND_ATTN_TC = 2, OT_KIND_ATTN_SIMT = 3,
-    OT_KIND_GATHER = 4, OT_KIND_QUANT = 5, OT_KIND_FFN_TC = 6 /* fused FFN1 + GELU + FFN2 */
+    OT_KIND_GATHER = 4, OT_KIND_QUANT = 5, OT_KIND_FFN_TC = 6 /* fused FFN1 + GELU + FFN2 */,
+    OT_KIND_ATTN_NS = 7 /* NS attention, <= 64 query rows per (user, head) */
 } ot_kernel_kind;
 
 typedef struct {

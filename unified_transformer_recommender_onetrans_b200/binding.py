@@ -45,7 +45,7 @@ class OtLaunchRecord(C.Structure):
 
 
 KINDS = {0: "gemm_tc", 1: "gemm_simt", 2: "attn_tc", 3: "attn_simt", 4: "gather", 5: "quant",
-         6: "ffn_tc"}
+         6: "ffn_tc", 7: "attn_ns"}
 ROLES = {0: "S_QKV", 1: "S_attn", 2: "S_O", 3: "S_FFN1", 4: "S_FFN2", 5: "NS_QKV", 6: "NS_attn",
          7: "NS_O", 8: "NS_FFN1", 9: "NS_FFN2", 10: "auto_split", 11: "other", 12: "S_FFN",
          13: "NS_FFN", 14: "O", 15: "FFN", 16: "QKV"}

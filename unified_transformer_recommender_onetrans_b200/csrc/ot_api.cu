@@ -284,9 +284,13 @@ ot_status attn(ot_model *m, AttnArgs &a, cudaStream_t s)
     const bool simt = m->cfg.dtype == OT_DTYPE_F32 || m->path == 1;
     double flops = 0, bytes = 0;
     if (m->profiling) attn_cost(m, a, flops, bytes);
-    return profiled(m, s, simt ? OT_KIND_ATTN_SIMT : OT_KIND_ATTN_TC,
+    // a few NS rows per (user, head): the decode-shaped kernel
+    const bool ns_small = !simt && attn_ns_small_supported(a);
+    return profiled(m, s, simt ? OT_KIND_ATTN_SIMT : ns_small ? OT_KIND_ATTN_NS : OT_KIND_ATTN_TC,
                     a.mode == 0 ? ROLE_S_ATTN : ROLE_NS_ATTN, flops, bytes, [&] {
-                        return simt ? launch_attn_simt(a, s) : launch_attn_tc(a, s);
+                        return simt ? launch_attn_simt(a, s)
+                               : ns_small ? launch_attn_ns_small(a, s)
+                                          : launch_attn_tc(a, s);
                     });
 }
 

@@ -143,6 +143,9 @@ cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s);
 cudaError_t launch_gemm_tc_multi(const GemmArgs &a, const GemmArgs *a1, cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s);
+// NS attention with all query rows of a (user, head) within 64 (decode-shaped)
+bool attn_ns_small_supported(const AttnArgs &a);
+cudaError_t launch_attn_ns_small(const AttnArgs &a, cudaStream_t s);
 bool ffn_tc_supported(int D, int F);
 cudaError_t launch_ffn_tc(const FfnArgs &a, cudaStream_t s);
 // two problems with the same D, F and eps in one launch (a1 may be null)
