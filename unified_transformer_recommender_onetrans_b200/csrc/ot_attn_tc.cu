@@ -99,12 +99,14 @@ __device__ __forceinline__ void softmax_unit(uint32_t tS_row, float c2, int klo,
 #pragma unroll
     for (int q = 0; q < 4; ++q) tmem_reg_fence(v[q]);
     released();
+    // four independent chains of three-input maxima: 64 instructions for 128 scores
     float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
     for (int q = 0; q < 4; ++q)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[q][e]));
-    const float mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c2;
+        for (int e = 0; e < 32; e += 2)
+            mx[(e >> 1) & 3] = fmax3(mx[(e >> 1) & 3], __uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1]));
+    const float mb = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * c2;
     alpha = 1.f;
     if (m == -INFINITY) {
         m = mb; // the row's first block: l is 0 and O holds nothing for it
@@ -112,23 +114,31 @@ __device__ __forceinline__ void softmax_unit(uint32_t tS_row, float c2, int klo,
         alpha = fast_exp2(m - mb);
         m = mb;
     }
-    const float mneg = -m;
-    float rs[4] = {0.f, 0.f, 0.f, 0.f};
+    // per pair of scores: one packed FMA for the exponents, two exponentials,
+    // one packed add into the row sum (two independent pair accumulators)
+    const uint64_t c2x2 = f32x2(c2, c2), mnx2 = f32x2(-m, -m);
+    uint64_t rs2[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
 #pragma unroll
     for (int q = 0; q < 4; ++q)
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-            float p2[2];
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const int k = 32 * q + 2 * j + t;
-                const float ex = fast_exp2(fmaf(__uint_as_float(v[q][2 * j + t]), c2, mneg));
-                p2[t] = (FULL || (k >= klo && k <= khi)) ? ex : 0.f;
-                rs[t + 2 * (j & 1)] += p2[t];
+            float x0, x1;
+            f32x2_split(fma_f32x2(f32x2(__uint_as_float(v[q][2 * j]), __uint_as_float(v[q][2 * j + 1])), c2x2,
+                                  mnx2),
+                        x0, x1);
+            float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            if (!FULL) {
+                const int k = 32 * q + 2 * j;
+                p0 = (k >= klo && k <= khi) ? p0 : 0.f;
+                p1 = (k + 1 >= klo && k + 1 <= khi) ? p1 : 0.f;
             }
-            pk[q][j] = pack_bf16x2(p2[0], p2[1]);
+            rs2[j & 1] = add_f32x2(rs2[j & 1], f32x2(p0, p1));
+            pk[q][j] = pack_bf16x2(p0, p1);
         }
-    rsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+    float a0, a1, b0, b1;
+    f32x2_split(rs2[0], a0, a1);
+    f32x2_split(rs2[1], b0, b1);
+    rsum = (a0 + b0) + (a1 + b1);
 }
 
 // One work item of the persistent kernel: a (user, head, query pair) and its
