@@ -521,35 +521,33 @@ def run_ours(args, wl):
     tokens_per_step = U * wl.L0 * world
     value = tokens_per_step / (ms_per_step / 1e3)
 
-    # ---- end to end through the public API: pinned host inputs -> device -> host outputs
+    # ---- end to end through the public API: pinned host inputs -> device -> host outputs.
+    # ot_full_forward_host copies each call's inputs on the model's copy stream into
+    # one of two staging slots, so back-to-back calls overlap the next input copy
+    # with this call's work, as a serving loop would; the number is the span of
+    # all K calls (L2 flushes between calls included) divided by K.
     S_h = S_cpu.pin_memory()
     x_h = x_cpu.pin_memory()
     s_tail_h = torch.empty(s_tail.shape, dtype=s_tail.dtype).pin_memory()
     out_ns_h = torch.empty(out_ns.shape, dtype=out_ns.dtype).pin_memory()
-    S_e2e = torch.empty_like(S)
-    x_e2e = torch.empty_like(x)
+    ws_host = torch.empty(m.host_workspace_bytes(U, C), dtype=torch.uint8, device=dev)
 
     def step_e2e():
-        S_e2e.copy_(S_h, non_blocking=True)
-        x_e2e.copy_(x_h, non_blocking=True)
-        m.auto_split(x_e2e, ns)
-        m.full_forward(S_e2e, ns, kv=kv, out_s_tail=s_tail, out_ns=out_ns, ws=ws)
-        s_tail_h.copy_(s_tail, non_blocking=True)
-        out_ns_h.copy_(out_ns, non_blocking=True)
+        m.full_forward_host(S_h, x_h, s_tail_h, out_ns_h, kv=kv, ws=ws_host)
 
-    for _ in range(2):
+    for _ in range(3):
         step_e2e()
-    barrier()
-    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for e0, e1 in ev2:
-        e0.record(stream)
-        step_e2e()
-        e1.record(stream)
         flush.zero_()
     barrier()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2) / args.steps, world, dist,
-                            dev)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(args.steps):
+        step_e2e()
+        flush.zero_()
+    e_end.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, world, dist, dev)
+    del ws_host
     h2d = S_h.numel() * S_h.element_size() + x_h.numel() * x_h.element_size()
     d2h = s_tail_h.numel() * s_tail_h.element_size() + out_ns_h.numel() * out_ns_h.element_size()
 

@@ -188,6 +188,22 @@ ot_status ot_full_forward(ot_model *m, const void *S, const void *ns, int B, int
                           void *out_s_tail, void *out_ns, void *kv_cache, void *ws,
                           size_t ws_bytes, void *stream);
 
+/* The same batch from pinned host memory: S_host [B][L0][d], x_host [B][C][F]
+ * (the Auto-Split input, F = cfg.F > 0) -> out_s_tail_host [B][q_last][d],
+ * out_ns_host [B][C][N][d], all in the storage dtype.  The inputs are copied
+ * on the model's own copy stream into one of two staging slots of the
+ * workspace (alternating per call; a slot is rewritten only after the
+ * forward that read it has run), then Auto-Split, the forward and the output
+ * copies run on `stream`.  Calls issued back to back on one stream with the
+ * same workspace therefore overlap the next call's input copy with this
+ * call's work.  ws >= ot_host_workspace_bytes(m, B, C) bytes, device; the
+ * host buffers must stay valid until the call's work on `stream` completes.
+ * Returns as ot_full_forward; OT_ERR_SHAPE if the model has no Auto-Split. */
+size_t ot_host_workspace_bytes(const ot_model *m, int users, int cands);
+ot_status ot_full_forward_host(ot_model *m, const void *S_host, const void *x_host, int B, int C,
+                               void *out_s_tail_host, void *out_ns_host, void *kv_cache,
+                               void *ws, size_t ws_bytes, void *stream);
+
 /* Synchronise `stream`, then read and clear the model's device error word.
  * Returns OT_OK, OT_ERR_DEVICE_TIMEOUT, OT_ERR_DEVICE_BOUNDS or OT_ERR_CUDA. */
 ot_status ot_poll_device_error(ot_model *m, void *stream);

@@ -79,6 +79,8 @@ def test_calls_reject_null_model(lib):
     assert lib.ot_encode_user(None, None, 1, None, None, None, 0, None) == 1
     assert lib.ot_score_candidates(None, None, 1, None, 1, None, None, 0, None) == 1
     assert lib.ot_full_forward(None, None, None, 1, 1, None, None, None, None, 0, None) == 1
+    assert lib.ot_full_forward_host(None, None, None, 1, 1, None, None, None, None, 0, None) == 1
+    assert lib.ot_host_workspace_bytes(None, 1, 1) == 0
     assert lib.ot_auto_split(None, None, 1, None, None) == 1
     assert lib.ot_embed_gather(None, 1, 8, None, 1, None, None, None) == 1
     assert lib.ot_embed_gather(16, 1, 12, 16, 1, 16, None, None) == 2

@@ -297,6 +297,38 @@ def test_bf16_many_items_per_cta():
         assert O.rel_l2(x.double().cpu().numpy(), y.double().cpu().numpy()) < 1e-2
 
 
+# ----------------------------------------------------------------- host-buffer entry point
+def test_full_forward_host_matches_device_path():
+    """ot_full_forward_host (pinned host in / out, inputs staged through two
+    alternating workspace slots on the model's copy stream) against Auto-Split
+    + ot_full_forward on device tensors, bit for bit, over three back-to-back
+    calls so both slots are used and one is reused."""
+    wl = WORKLOADS["onetrans_s_full"]
+    w = gen_weights(wl)
+    m = model_of(wl, w)
+    m.set_wait_limit(TEST_WAIT)
+    groups = ([0, 1, 2], [3, 4, 5], [6, 7, 8])
+    B, C = len(groups[0]), wl.cands
+    ws = torch.empty(m.host_workspace_bytes(B, C), dtype=torch.uint8, device="cuda")
+    host_runs, dev_runs = [], []
+    for users in groups:
+        S = gen_s_tokens(wl, users=users, weights=w)
+        x = gen_auto_split_features(wl, users=users)
+        S_h, x_h = S.pin_memory(), x.pin_memory()
+        tail_h = torch.empty(B, m.q[-1], wl.d, dtype=m.storage).pin_memory()
+        ns_h = torch.empty(B, C, wl.n_ns, wl.d, dtype=m.storage).pin_memory()
+        m.full_forward_host(S_h, x_h, tail_h, ns_h, ws=ws)
+        host_runs.append((S_h, x_h, tail_h, ns_h))
+    torch.cuda.synchronize()
+    m.poll()
+    for S_h, x_h, tail_h, ns_h in host_runs:
+        ns = m.auto_split(x_h.cuda())
+        tail_d, ns_d = m.full_forward(S_h.cuda(), ns)
+        m.poll()
+        assert torch.equal(tail_h, tail_d.cpu()) and torch.equal(ns_h, ns_d.cpu())
+    assert not torch.equal(host_runs[0][2], host_runs[1][2])
+
+
 # ----------------------------------------------------------------- split-key NS attention
 @pytest.mark.parametrize("shape", ["nq128_odd_even_blocks", "nq1_two_blocks"])
 def test_split_key_ns_attention(shape):

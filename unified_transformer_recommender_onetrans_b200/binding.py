@@ -60,6 +60,8 @@ SIGNATURES = {
     "ot_encode_user": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
     "ot_score_candidates": (_i, [_vp, _vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
     "ot_full_forward": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "ot_host_workspace_bytes": (_sz, [_vp, _i, _i]),
+    "ot_full_forward_host": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "ot_poll_device_error": (_i, [_vp, _vp]),
     "ot_set_wait_limit": (_i, [_vp, _ll]),
     "ot_set_kernel_path": (_i, [_vp, _i]),
@@ -119,6 +121,15 @@ def pyramid_schedule(L0: int, q_end: int | None, layers: int) -> list[int]:
 
 
 # ------------------------------------------------------------------ torch face
+def _host_ptr(t) -> int:
+    """Address of a pinned, contiguous host tensor (ot_full_forward_host)."""
+    if t.is_cuda or not t.is_pinned():
+        raise ValueError("host buffers passed to the library must be pinned CPU tensors")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return t.data_ptr()
+
+
 def _ptr(t) -> int:
     if t is None:
         return 0
@@ -292,6 +303,24 @@ class Model:
                                     ws.numel() * ws.element_size(), _stream(stream)),
               "ot_full_forward")
         return out_s_tail, out_ns
+
+    def host_workspace_bytes(self, users: int, cands: int) -> int:
+        return int(lib().ot_host_workspace_bytes(self.handle, users, cands))
+
+    def full_forward_host(self, S_host, x_host, out_s_tail_host, out_ns_host, kv=None, ws=None,
+                          stream=None):
+        """Auto-Split + full forward from pinned host tensors S_host [B, L0, d] and
+        x_host [B, C, F] into pinned host outputs [B, q_last, d] and [B, C, N, d]
+        (ot_full_forward_host).  Consecutive calls on one stream with the same
+        workspace overlap the next call's input copy with this call's work."""
+        B, Cn = x_host.shape[0], x_host.shape[1]
+        ws = self._ws(ws, self.host_workspace_bytes(B, Cn))
+        check(lib().ot_full_forward_host(self.handle, _host_ptr(S_host), _host_ptr(x_host), B, Cn,
+                                         _host_ptr(out_s_tail_host), _host_ptr(out_ns_host), _ptr(kv),
+                                         _ptr(ws), ws.numel() * ws.element_size(),
+                                         _stream(stream)),
+              "ot_full_forward_host")
+        return out_s_tail_host, out_ns_host
 
 
 def embed_gather(table, ids, out=None, err=None, stream=None):

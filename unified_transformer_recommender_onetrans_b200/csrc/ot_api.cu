@@ -58,7 +58,15 @@ struct ot_model {
     cudaEvent_t kv_ready[OT_MAX_LAYERS];
     cudaEvent_t ns_attn_done[OT_MAX_LAYERS]; // merged full forward: NS attention of layer l
     cudaEvent_t fork_ev = nullptr, join_ev = nullptr;
-    std::mutex enqueue_mu; // event re-recording must not interleave between calls
+    // ot_full_forward_host: inputs travel on their own stream into one of two
+    // staging slots; in_ready[s] = slot s holds its inputs, in_free[s] = the
+    // forward that read slot s is done with it
+    cudaStream_t copy_stream = nullptr;
+    cudaEvent_t in_ready[2] = {nullptr, nullptr}, in_free[2] = {nullptr, nullptr};
+    unsigned long long host_calls = 0;
+    // event re-recording must not interleave between calls (recursive: a host
+    // call holds it across the forward it enqueues)
+    std::recursive_mutex enqueue_mu;
 };
 
 namespace ot {
@@ -896,8 +904,13 @@ ot_status ot_model_create(const ot_config *cfg, const ot_weights *w, ot_model **
         m->allocs.push_back(m->err);
         if (cudaMemset(m->err, 0, sizeof(int)) != cudaSuccess) { r = OT_ERR_CUDA; break; }
         if (cudaStreamCreateWithFlags(&m->side, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&m->copy_stream, cudaStreamNonBlocking) != cudaSuccess ||
             cudaEventCreateWithFlags(&m->fork_ev, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&m->join_ev, cudaEventDisableTiming) != cudaSuccess) {
+            cudaEventCreateWithFlags(&m->join_ev, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&m->in_ready[0], cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&m->in_ready[1], cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&m->in_free[0], cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&m->in_free[1], cudaEventDisableTiming) != cudaSuccess) {
             r = OT_ERR_CUDA;
             break;
         }
@@ -966,6 +979,11 @@ void ot_model_destroy(ot_model *m)
     }
     if (m->fork_ev) cudaEventDestroy(m->fork_ev);
     if (m->join_ev) cudaEventDestroy(m->join_ev);
+    for (int i = 0; i < 2; ++i) {
+        if (m->in_ready[i]) cudaEventDestroy(m->in_ready[i]);
+        if (m->in_free[i]) cudaEventDestroy(m->in_free[i]);
+    }
+    if (m->copy_stream) cudaStreamDestroy(m->copy_stream);
     if (m->side) cudaStreamDestroy(m->side);
     delete m;
 }
@@ -1121,7 +1139,7 @@ ot_status ot_full_forward(ot_model *m, const void *S, const void *ns, int B, int
     }
     // Shared O / FFN launches for both sides where the kernels allow it
     if (merged_supported(m) && m->side && w.left >= enc + sc) {
-        std::lock_guard<std::mutex> lock(m->enqueue_mu);
+        std::lock_guard<std::recursive_mutex> lock(m->enqueue_mu);
         Ws w_enc = w;
         Ws w_sc{w.p + enc, w.left - enc, m->esz};
         return run_full_merged(m, S, B, ns, C, kv, out_s_tail, out_ns, w_enc, w_sc, st);
@@ -1135,7 +1153,7 @@ ot_status ot_full_forward(ot_model *m, const void *S, const void *ns, int B, int
         if (r != OT_OK) return r;
         return run_score(m, kv, B, ns, C, out_ns, w, st);
     }
-    std::lock_guard<std::mutex> lock(m->enqueue_mu);
+    std::lock_guard<std::recursive_mutex> lock(m->enqueue_mu);
     Ws w_enc = w;
     Ws w_sc{w.p + enc, w.left - enc, m->esz};
     if (cudaEventRecord(m->fork_ev, st) != cudaSuccess ||
@@ -1149,6 +1167,80 @@ ot_status ot_full_forward(ot_model *m, const void *S, const void *ns, int B, int
         cudaStreamWaitEvent(st, m->join_ev, 0) != cudaSuccess)
         return OT_ERR_CUDA;
     return r != OT_OK ? r : r2;
+}
+
+// Workspace of ot_full_forward_host: two staging slots (S and x), the NS
+// tokens, the device outputs, then the forward's own workspace; every region
+// starts on a 256-byte boundary.
+struct HostWs {
+    size_t s_bytes, x_bytes, ns_bytes, tail_bytes, slot, total_fixed;
+};
+
+static size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+static HostWs host_ws(const ot_model *m, int B, int C)
+{
+    const ot_config &c = m->cfg;
+    HostWs h;
+    h.s_bytes = align256(bytes_of(static_cast<long long>(B) * c.L0 * c.d, m->esz));
+    h.x_bytes = align256(bytes_of(static_cast<long long>(B) * C * c.F, m->esz));
+    h.ns_bytes = align256(bytes_of(static_cast<long long>(B) * C * c.n_ns * c.d, m->esz));
+    h.tail_bytes = align256(bytes_of(static_cast<long long>(B) * c.q[c.layers - 1] * c.d, m->esz));
+    h.slot = h.s_bytes + h.x_bytes;
+    h.total_fixed = 2 * h.slot + 2 * h.ns_bytes + h.tail_bytes; // ns in, ns out, S tail
+    return h;
+}
+
+size_t ot_host_workspace_bytes(const ot_model *m, int users, int cands)
+{
+    if (!m || users < 1 || cands < 1 || m->cfg.F <= 0) return 0;
+    return host_ws(m, users, cands).total_fixed + ot_workspace_bytes(m, users, cands);
+}
+
+ot_status ot_full_forward_host(ot_model *m, const void *S_host, const void *x_host, int B, int C,
+                               void *out_s_tail_host, void *out_ns_host, void *kv_cache, void *ws,
+                               size_t ws_bytes, void *stream)
+{
+    if (!m || !S_host || !x_host || !out_s_tail_host || !out_ns_host || !ws || B < 1 || C < 1)
+        return OT_ERR_ARG;
+    if (m->cfg.F <= 0) return OT_ERR_SHAPE;
+    if (!aligned16(ws) || (kv_cache && !aligned16(kv_cache))) return OT_ERR_ALIGN;
+    if (ws_bytes < ot_host_workspace_bytes(m, B, C)) return OT_ERR_WORKSPACE_TOO_SMALL;
+    if (!m->copy_stream) return OT_ERR_CUDA;
+    const HostWs h = host_ws(m, B, C);
+    char *base = static_cast<char *>(ws);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    std::lock_guard<std::recursive_mutex> lock(m->enqueue_mu);
+    const int slot = static_cast<int>(m->host_calls & 1);
+    char *S_dev = base + slot * h.slot, *x_dev = S_dev + h.s_bytes;
+    char *ns_dev = base + 2 * h.slot, *out_ns_dev = ns_dev + h.ns_bytes, *tail_dev = out_ns_dev + h.ns_bytes;
+    char *fw = base + h.total_fixed;
+    // inputs: once the forward two calls back has finished reading this slot
+    if (cudaStreamWaitEvent(m->copy_stream, m->in_free[slot], 0) != cudaSuccess ||
+        cudaMemcpyAsync(S_dev, S_host, bytes_of(static_cast<long long>(B) * m->cfg.L0 * m->cfg.d, m->esz),
+                        cudaMemcpyHostToDevice, m->copy_stream) != cudaSuccess ||
+        cudaMemcpyAsync(x_dev, x_host, bytes_of(static_cast<long long>(B) * C * m->cfg.F, m->esz),
+                        cudaMemcpyHostToDevice, m->copy_stream) != cudaSuccess ||
+        cudaEventRecord(m->in_ready[slot], m->copy_stream) != cudaSuccess ||
+        cudaStreamWaitEvent(st, m->in_ready[slot], 0) != cudaSuccess)
+        return OT_ERR_CUDA;
+    ++m->host_calls;
+    ot_status r = ot_auto_split(m, x_dev, static_cast<long>(B) * C, ns_dev, stream);
+    if (r == OT_OK)
+        r = ot_full_forward(m, S_dev, ns_dev, B, C, tail_dev, out_ns_dev, kv_cache, fw,
+                            ws_bytes - h.total_fixed, stream);
+    // the slot is free again once the forward has run (also after an error,
+    // so later calls do not wait on a stale record)
+    if (cudaEventRecord(m->in_free[slot], st) != cudaSuccess) return OT_ERR_CUDA;
+    if (r != OT_OK) return r;
+    const ot_config &c = m->cfg;
+    if (cudaMemcpyAsync(out_s_tail_host, tail_dev,
+                        bytes_of(static_cast<long long>(B) * c.q[c.layers - 1] * c.d, m->esz),
+                        cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemcpyAsync(out_ns_host, out_ns_dev, bytes_of(static_cast<long long>(B) * C * c.n_ns * c.d, m->esz),
+                        cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return OT_ERR_CUDA;
+    return OT_OK;
 }
 
 } // extern "C"
