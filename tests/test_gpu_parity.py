@@ -330,18 +330,20 @@ def test_full_forward_host_matches_device_path():
 
 
 # ----------------------------------------------------------------- split-key NS attention
-@pytest.mark.parametrize("shape", ["nq128_odd_even_blocks", "nq1_two_blocks"])
+@pytest.mark.parametrize("shape", ["nq128_odd_even_blocks", "nq1_two_blocks", "nq80_partial_tiles"])
 def test_split_key_ns_attention(shape):
-    """NS attention with every query row of a (user, head) in one tile: the
-    two tiles of a CTA take alternate key blocks and merge their softmax
-    states.  Layers with an even (4) and an odd (3) number of key blocks and
-    with exactly two (one S block, one NS block), a full tile of NS rows
-    (C N = 128) and a single NS row; every user against the oracle and the
-    CUDA-core path."""
+    """NS attention with at most 128 query rows per (user, head): 128 and 80
+    rows take the tensor-memory kernel's split-key mode (the two tiles of a
+    CTA take alternate key blocks and merge their softmax states; layers with
+    an even and an odd number of key blocks, a partly filled tile), a single
+    row the decode-shaped kernel (key splits over four warps, a layer with
+    two key blocks); every user against the oracle and the CUDA-core path."""
     if shape == "nq128_odd_even_blocks":
         layers, d, H, f, N, U, C, L0, q = 3, 128, 2, 256, 16, 4, 8, 260, [260, 200, 60]
-    else:
+    elif shape == "nq1_two_blocks":
         layers, d, H, f, N, U, C, L0, q = 3, 128, 2, 256, 1, 5, 1, 100, [100, 64, 1]
+    else:
+        layers, d, H, f, N, U, C, L0, q = 3, 128, 2, 256, 16, 3, 5, 200, [200, 150, 70]
     w = rand_weights(layers, d, f, N, seed=51, dtype=torch.bfloat16)
     S, ns = rand_inputs(U, C, L0, N, d, seed=52, dtype=torch.bfloat16)
     m = make_model(w, layers=layers, d=d, heads=H, ffn=f, n_ns=N, L0=L0, q=q)
