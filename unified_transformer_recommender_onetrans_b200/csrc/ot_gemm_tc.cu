@@ -608,6 +608,19 @@ cudaError_t launch_gemm_tc_multi(const GemmArgs &a, const GemmArgs *a1, cudaStre
             (a1->norm != 0) != (a.norm != 0))
             return cudaErrorInvalidValue;
     }
+    // a single problem whose 128 x 256 tiles would leave SMs idle (the grouped
+    // NS projections at small C) gets twice as many 128 x 128 tiles instead
+    if (!a1 && wide) {
+        if (g_num_sms == 0) {
+            int dev = 0;
+            cudaGetDevice(&dev);
+            if (cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+                g_num_sms < 1)
+                g_num_sms = 148;
+        }
+        const long long tiles256 = static_cast<long long>((a.M + G_BM - 1) / G_BM) * (a.N / 256) * a.G;
+        if (tiles256 < g_num_sms) wide = false;
+    }
     if (a1) {
         if (wide && wide1) return launch_tc_cfg<256, false, true>(a, a1, s);
         return launch_tc_cfg<128, false, true>(a, a1, s);
