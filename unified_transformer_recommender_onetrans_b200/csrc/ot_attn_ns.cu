@@ -1,5 +1,5 @@
-// NS attention when every NS query row of a user fits in 64 (C N <= 64, the
-// common case in serving and in the full forward): query i = NS token i % N
+// NS attention when every NS query row of a user fits in 64 (C N <= 64; the
+// dispatcher uses it up to 16, e.g. the full forward at C = 1): query i = NS token i % N
 // of candidate i / N sees all L cached S keys of the layer and the NS keys
 // m <= i % N of its own candidate (the OneTrans mask).  head_dim 64, bf16
 // operands, fp32 scores, softmax and accumulation.
@@ -35,7 +35,8 @@ constexpr int NA_KB = 32;                         // keys per block
 constexpr int NA_NT = NA_KB / 8;                  // 8-key column tiles of a block (S = Q K^T)
 constexpr int NA_KS = NA_KB / 16;                 // 16-key steps of a block (O += P V)
 constexpr int NA_HD = 64;
-constexpr int NA_MAXQ = 64;                       // query rows per (user, head)
+constexpr int NA_MAXQ = 64;                       // query rows per (user, head) the kernel handles
+constexpr int NA_MAXQ_FAST = 16;                  // ... and where it beats the tensor-memory kernel
 constexpr int NA_STAGES = 3;                      // K / V ring depth per warp
 constexpr uint32_t NA_TILE = NA_KB * 128;         // NA_KB rows x 128 bytes
 constexpr uint32_t NA_STAGE = 2 * NA_TILE;        // K and V
@@ -324,9 +325,13 @@ __global__ void __launch_bounds__(NA_WARPS * 32, 2)
 
 bool attn_ns_small_supported(const AttnArgs &a)
 {
-    // bf16 operands (the e4m3 models keep bf16 activations and caches)
+    // bf16 operands (the e4m3 models keep bf16 activations and caches).  Only
+    // up to 16 rows, where all four warps split the keys: with 2-4 query
+    // tiles each warp walks half or all of the keys alone and the tensor-memory
+    // kernel's split-key mode is faster (C sweep: 32 rows 0.368 ms, 64 rows
+    // 0.505 ms against 0.319 ms at 128 rows on tcgen05)
     return a.mode == 1 && a.hd == NA_HD && (a.dtype == OT_DTYPE_BF16 || a.dtype == OT_DTYPE_FP8) &&
-           a.nq >= 1 && a.nq <= NA_MAXQ &&
+           a.nq >= 1 && a.nq <= NA_MAXQ_FAST &&
            a.N >= 1 && a.L >= 0 && a.U >= 1 && a.H >= 1;
 }
 
