@@ -357,6 +357,31 @@ def test_split_key_ns_attention(shape):
         assert O.rel_l2(x.double().cpu().numpy(), y.double().cpu().numpy()) < 1e-2
 
 
+def test_ns_attention_two_row_tiles_ragged():
+    """NS attention with 190 query rows per (user, head): both row tiles of a
+    CTA live, the second partly past the last row (a warp with 30 live rows,
+    two warps with none); 10 NS tokens per candidate, so NS key blocks split
+    candidates and some warps see no key of a block.  Full forward (NS
+    attention on the side stream) against the oracle and the CUDA-core path;
+    cached scoring bit-identical to it."""
+    layers, d, H, f, N, U, C, L0, q = 3, 128, 2, 1024, 10, 2, 19, 850, [850, 200, 100]
+    w = rand_weights(layers, d, f, N, seed=61, dtype=torch.bfloat16)
+    S, ns = rand_inputs(U, C, L0, N, d, seed=62, dtype=torch.bfloat16)
+    m = make_model(w, layers=layers, d=d, heads=H, ffn=f, n_ns=N, L0=L0, q=q)
+    m.set_wait_limit(TEST_WAIT)
+    a = _run_full(m, S.cuda(), ns.cuda())
+    errs = _errors_vs_oracle(m, w, S, ns, *a, list(range(U)))
+    assert_within(errs, TOL["bf16"])
+    kv2, _ = m.encode_user(S.cuda(), want_s_tail=False)
+    sc = m.score_candidates(kv2, ns.cuda())
+    m.poll()
+    assert torch.equal(sc, a[1])
+    m.set_kernel_path(1)
+    b = _run_full(m, S.cuda(), ns.cuda())
+    for x, y in zip(a, b):
+        assert O.rel_l2(x.double().cpu().numpy(), y.double().cpu().numpy()) < 1e-2
+
+
 # ----------------------------------------------------------------- fused feed-forward
 @pytest.mark.parametrize("shape", ["small_d128", "onetrans_s_d256"])
 def test_fused_ffn_matches_two_gemm_path(shape):

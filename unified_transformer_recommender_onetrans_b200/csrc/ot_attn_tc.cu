@@ -1,8 +1,9 @@
 // tcgen05 attention for one layer of the block (head_dim 64, bf16 operands,
 // fp32 scores and softmax).  Persistent: one CTA per SM walks a list of work
 // items, each a (user, head) and two 128-query tiles (256 consecutive query
-// rows); the next item's Q and K/V loads and its first scores overlap the
-// current item's last blocks and output read-out.
+// rows), or, in NS mode's split-key form, one 128-query tile whose key blocks
+// the two tiles of the CTA share out; the next item's Q and K/V loads and its
+// first scores overlap the current item's last blocks and output read-out.
 //
 // Key blocks of 128 rows are visited in order: first the user's S keys (from
 // the KV cache), then, in NS mode, the NS keys of the candidates the item's
@@ -150,10 +151,15 @@ struct AtItem {
     int n_blocks;     // S blocks + NS blocks
 };
 
+// Query rows per item: two tiles of 128, or one in split-key mode, where
+// both tiles of the CTA work on the same rows.
+template <bool SPLIT> __host__ __device__ constexpr int at_item_rows() { return SPLIT ? AT_BM : AT_BM * AT_TILES; }
+
 // Item k.  S mode orders the pairs longest first (pairs later in the tail see
 // more keys), so the snake assignment below balances the CTAs; NS mode keeps
-// the pairs of one (user, head) together so they share K/V tiles in L2.
-template <bool NS>
+// the pairs (row tiles in split-key mode) of one (user, head) together so
+// they share K/V tiles in L2.
+template <bool NS, bool SPLIT>
 __device__ __forceinline__ AtItem at_item(const AttnArgs &a, int n_pairs, int k)
 {
     AtItem it;
@@ -168,8 +174,8 @@ __device__ __forceinline__ AtItem at_item(const AttnArgs &a, int n_pairs, int k)
     }
     it.u = uh / a.H;
     it.h = uh % a.H;
-    it.i0 = pair * (AT_BM * AT_TILES);
-    const int i_last = min(it.i0 + AT_BM * AT_TILES, a.nq) - 1;
+    it.i0 = pair * at_item_rows<SPLIT>();
+    const int i_last = min(it.i0 + at_item_rows<SPLIT>(), a.nq) - 1;
     it.k_begin = 0;
     if (!NS) {
         const int t_last = a.L - a.nq + i_last;
@@ -195,9 +201,9 @@ __device__ __forceinline__ int at_item_of(int r, int n_items)
 }
 
 // The key blocks tile w works on, in order, across this CTA's items.  Every
-// tile takes every block, except in split-key mode (SPLIT: NS mode with all
-// query rows in one tile), where tile w takes the blocks b = w (mod 2) of an
-// item and the two tiles' partial softmax states are merged at its end.
+// tile takes every block, except in split-key mode (SPLIT: NS mode with
+// items of one 128-row tile), where tile w takes the blocks b = w (mod 2) of
+// an item and the two tiles' partial softmax states are merged at its end.
 // gb counts all blocks of the CTA (the K/V ring position), lb this tile's.
 template <bool NS, bool SPLIT>
 struct BlockCursor {
@@ -214,7 +220,7 @@ struct BlockCursor {
         if (++b < it.n_blocks) return;
         b = 0;
         k = at_item_of(++r, n_items);
-        if (k >= 0) it = at_item<NS>(a, n_pairs, k);
+        if (k >= 0) it = at_item<NS, SPLIT>(a, n_pairs, k);
     }
     __device__ __forceinline__ void init(const AttnArgs &a, int n_pairs, int n_items, int tile)
     {
@@ -224,7 +230,7 @@ struct BlockCursor {
         gb = 0;
         lb = 0;
         k = at_item_of(0, n_items);
-        if (k >= 0) it = at_item<NS>(a, n_pairs, k);
+        if (k >= 0) it = at_item<NS, SPLIT>(a, n_pairs, k);
         while (valid() && !owned()) step(a, n_pairs, n_items);
     }
     __device__ __forceinline__ void next(const AttnArgs &a, int n_pairs, int n_items)
@@ -270,7 +276,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     float *xch = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + AT_BAR_BYTES); // [2][AT_BM]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_pairs = (a.nq + AT_BM * AT_TILES - 1) / (AT_BM * AT_TILES);
+    const int n_pairs = (a.nq + at_item_rows<SPLIT>() - 1) / at_item_rows<SPLIT>();
     const int n_items = n_pairs * a.U * a.H;
     pdl_launch_dependents();
 
@@ -333,7 +339,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             for (; ok; ++r) {
                 const int k = at_item_of(r, n_items);
                 if (k < 0) break;
-                const AtItem it = at_item<NS>(a, n_pairs, k);
+                const AtItem it = at_item<NS, SPLIT>(a, n_pairs, k);
                 const int qb = r & 1;
                 // the Q buffer of item r - 2 is free once all its S MMAs completed
                 if (!mbar_wait(&q_empty[qb], ((r >> 1) & 1) ^ 1, a.wait, abort_flag)) break;
@@ -477,7 +483,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         for (int r = 0; ok; ++r) {
             const int k = at_item_of(r, n_items);
             if (k < 0) break;
-            const AtItem it = at_item<NS>(a, n_pairs, k);
+            const AtItem it = at_item<NS, SPLIT>(a, n_pairs, k);
             const int i = it.i0 + (SPLIT ? 0 : w * AT_BM) + row; // query row within the user
             const bool warp_dead = __all_sync(0xffffffffu, i >= a.nq);
             const int t_self = a.L - a.nq + i;      // S mode
@@ -658,13 +664,32 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
             num_sms < 1)
             num_sms = 148;
     }
-    const long long items = static_cast<long long>((a.nq + AT_BM * AT_TILES - 1) / (AT_BM * AT_TILES)) *
-                            a.H * a.U;
+    // Split-key mode (NS mode with at least one S block, so every item has
+    // two or more key blocks and each tile gets one): items of one 128-row
+    // tile whose key blocks the CTA's two tiles take alternately, instead of
+    // items of two row tiles that both walk every block.  Always with at most
+    // 128 rows; above that where the estimated time is lower by a tenth, the
+    // estimate being waves of items x (key blocks a tile walks + one for the
+    // item's read-out), taken on the first item.  Split-key items read each
+    // K/V tile once per row tile rather than once per pair of them (the row
+    // tiles of a (user, head) run side by side, so mostly from L2).
+    auto key_blocks = [&](int rows) {
+        const int k_end = ((min(rows, a.nq) - 1) / a.N + 1) * a.N; // NS keys of the first item
+        return static_cast<long long>((a.L + AT_BK - 1) / AT_BK + (k_end + AT_BK - 1) / AT_BK);
+    };
+    bool split = false;
+    if (a.mode == 1 && a.L >= 1 && a.N >= 1) {
+        const long long uh = static_cast<long long>(a.U) * a.H;
+        const long long items2 = uh * ((a.nq + AT_BM * AT_TILES - 1) / (AT_BM * AT_TILES));
+        const long long items1 = uh * ((a.nq + AT_BM - 1) / AT_BM);
+        const long long t2 = (items2 + num_sms - 1) / num_sms * (key_blocks(AT_BM * AT_TILES) + 1);
+        const long long t1 = (items1 + num_sms - 1) / num_sms * ((key_blocks(AT_BM) + 1) / 2 + 1);
+        split = a.nq <= AT_BM || t1 * 10 < t2 * 9;
+    }
+    const int rows = split ? AT_BM : AT_BM * AT_TILES;
+    const long long items = static_cast<long long>((a.nq + rows - 1) / rows) * a.H * a.U;
     if (items < 1 || items > (1LL << 30)) return cudaErrorInvalidValue;
     dim3 grid(static_cast<unsigned>(items < num_sms ? items : num_sms));
-    // split-key mode: every query row in one tile and at least one S block,
-    // so each item has two or more key blocks and each tile gets one
-    const bool split = a.mode == 1 && a.nq <= AT_BM && a.L >= 1;
     auto run = [&](auto kernel) -> cudaError_t {
         // the setmaxnreg split must fit the registers the launch allocates,
         // or the softmax warpgroups' increase would wait forever
