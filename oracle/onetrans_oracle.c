@@ -328,6 +328,81 @@ int orc_encode_user(const orc_cfg *c, const orc_weights *w, const float *S, int 
 }
 
 /* ------------------------------------------------------------------------- */
+/* Appending S rows to encoded users (sequence KV caching across requests,     */
+/* summary page, KV-cache paragraph; the pages give no schedule for it).      */
+/* Reading: the pyramid windows stay anchored at their first row, so every    */
+/* layer's row set and query tail grow by the `delta` new rows: c is the grown */
+/* configuration (L0 and each q[l] include the new rows) and the previous      */
+/* encode used L0 - delta and q[l] - delta.  An old row then sees exactly the */
+/* keys it saw before at every layer (the mask is causal and no window loses  */
+/* a row), so its K/V and outputs are unchanged; only the new rows are run:   */
+/* per layer their K/V join the old ones, and new row t attends to keys 0..t. */
+/* kv_old is the previous cache, S_new [U][delta][d]; kv_new receives the      */
+/* cache in the grown layout, out_new [U][delta][d] the new rows' outputs of  */
+/* the last layer (the last delta rows of the grown S output).               */
+int orc_encode_append(const orc_cfg *c, const orc_weights *w, const double *kv_old,
+                      const float *S_new, int U, int delta, double *kv_new, double *out_new)
+{
+    if (check_cfg(c) || delta < 1) return 1;
+    orc_cfg old = *c;
+    old.L0 -= delta;
+    for (int l = 0; l < c->layers; ++l) old.q[l] -= delta;
+    if (check_cfg(&old)) return 1;
+    int d = c->d, H = c->heads, hd = d / H, f = c->ffn;
+    long kv_user = orc_kv_user_elems(c), kv_user_old = orc_kv_user_elems(&old);
+    for (int u = 0; u < U; ++u) {
+        double *X = (double *)malloc(sizeof(double) * (long)delta * d);
+        for (long i = 0; i < (long)delta * d; ++i) X[i] = S_new[(long)u * delta * d + i];
+        for (int l = 0; l < c->layers; ++l) {
+            int L = rows_at(c, l), Lo = L - delta;
+            pset_t p = s_params(c, w, l);
+            double *K = kv_new + (long)u * kv_user + orc_kv_layer_offset(c, l);
+            double *V = K + (long)L * d;
+            const double *Ko = kv_old + (long)u * kv_user_old + orc_kv_layer_offset(&old, l);
+            const double *Vo = Ko + (long)Lo * d;
+            memcpy(K, Ko, sizeof(double) * (long)Lo * d);
+            memcpy(V, Vo, sizeof(double) * (long)Lo * d);
+            double *Q = (double *)malloc(sizeof(double) * (long)delta * d);
+            double *Y = (double *)malloc(sizeof(double) * (long)delta * d);
+            double *xn = (double *)malloc(sizeof(double) * d);
+            double *qkv = (double *)malloc(sizeof(double) * 3 * d);
+            double *xq = (double *)malloc(sizeof(double) * (d > f ? d : f));
+            for (int i = 0; i < delta; ++i) {
+                int t = Lo + i;
+                rmsnorm(X + (long)i * d, p.g1, d, c->eps, xn);
+                project(&p.qkv, xn, 0, 3 * d, qkv, xq);
+                memcpy(Q + (long)i * d, qkv, sizeof(double) * d);
+                memcpy(K + (long)t * d, qkv + d, sizeof(double) * d);
+                memcpy(V + (long)t * d, qkv + 2 * d, sizeof(double) * d);
+            }
+            free(xn); free(qkv); free(xq);
+#pragma omp parallel
+            {
+                double *a = (double *)malloc(sizeof(double) * d);
+                double *sc = (double *)malloc(sizeof(double) * L);
+                double *scr = (double *)malloc(sizeof(double) * (3 * d + 2 * f + d));
+#pragma omp for schedule(dynamic, 4)
+                for (int i = 0; i < delta; ++i) {
+                    int t = Lo + i; /* the new row t sees keys 0..t: the old rows and new rows up to itself */
+                    for (int h = 0; h < H; ++h)
+                        attend(Q + (long)i * d + h * hd, hd, h * hd, d, K, V, t + 1, NULL, NULL, 0,
+                               a + h * hd, sc);
+                    block_tail(c, &p, X + (long)i * d, a, Y + (long)i * d, scr);
+                }
+                free(a); free(sc); free(scr);
+            }
+            pset_free(&p);
+            free(Q);
+            free(X);
+            X = Y;
+        }
+        memcpy(out_new + (long)u * delta * d, X, sizeof(double) * (long)delta * d);
+        free(X);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
 /* NS-side per candidate against the cached S K/V ("NS-side runs per          */
 /* candidate").  ns_in / ns_out are [U][C][N][d].                             */
 int orc_score_candidates(const orc_cfg *c, const orc_weights *w, const double *kv, int U,

@@ -47,6 +47,8 @@ def lib():
         L.orc_encode_user.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), fp, C.c_int, dp, dp]
         L.orc_score_candidates.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, C.c_int, dp,
                                            C.c_int, dp]
+        L.orc_encode_append.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, fp, C.c_int, C.c_int,
+                                        dp, dp]
         L.orc_full_forward_joint.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), fp, C.c_int, dp,
                                              C.c_int, dp, dp, dp]
         L.orc_auto_split.argtypes = [fp, C.c_long, C.c_int, fp, C.c_int, dp]
@@ -117,6 +119,13 @@ class Config:
         c.fp8 = int(bool(self.fp8))
         return c
 
+    def grown(self, delta: int) -> "Config":
+        """The configuration after appending `delta` S rows: L0 and every
+        query tail longer by delta (pyramid windows anchored at their first
+        row)."""
+        return Config(self.layers, self.d, self.heads, self.ffn, self.n_ns, self.L0 + delta,
+                      [v + delta for v in self.q], self.eps, self.fp8)
+
     def kv_user_elems(self) -> int:
         return int(lib().orc_kv_user_elems(C.byref(self._c())))
 
@@ -177,6 +186,26 @@ def encode_user(cfg: Config, w, S):
     if rc:
         raise ValueError("oracle rejected the configuration")
     return kv, s_out
+
+
+def encode_append(cfg: Config, w, kv_old, S_new):
+    """Append S_new [U, delta, d] to users encoded with the configuration
+    that `cfg` (the grown one) was grown from.  kv_old [U, old kv_user_elems]
+    -> (kv [U, kv_user_elems], out_new [U, delta, d]): the grown cache and
+    the new rows' outputs of the last layer."""
+    S_new, kv_old = _f32(S_new), _f64(kv_old)
+    U, delta = S_new.shape[0], S_new.shape[1]
+    assert S_new.shape == (U, delta, cfg.d), S_new.shape
+    old = cfg.grown(-delta)
+    assert kv_old.shape == (U, old.kv_user_elems()), kv_old.shape
+    W = _weights(w)
+    kv = np.zeros((U, cfg.kv_user_elems()))
+    out = np.zeros((U, delta, cfg.d))
+    rc = lib().orc_encode_append(C.byref(cfg._c()), C.byref(W.c), _dptr(kv_old), _fptr(S_new), U,
+                                 delta, _dptr(kv), _dptr(out))
+    if rc:
+        raise ValueError("oracle rejected the configuration")
+    return kv, out
 
 
 def score_candidates(cfg: Config, w, kv, ns):

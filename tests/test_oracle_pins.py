@@ -249,6 +249,64 @@ def test_invariant_kv_cache_equivalence_and_s_independence():
         np.testing.assert_allclose(jkv[:, c], kv, rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("fp8", [False, True], ids=["fp64", "e4m3"])
+def test_append_equals_encode_of_grown_sequence(fp8):
+    """Appending delta S rows (incremental: only the new rows run, against the
+    cached K/V) equals encoding the concatenated sequence with every pyramid
+    window grown by delta; the grown S output is the old output followed by
+    the new rows' outputs, and the old rows' K/V are unchanged.  Checked
+    against the brute-force token loop on the concatenated sequence too, and
+    twice in a row (append to an appended cache)."""
+    layers, d, H, f, N = 3, 16, 2, 24, 2
+    L0, q = 14, [14, 9, 4]
+    w = rand_weights(layers, d, f, N, seed=81)
+    S_all, _ = rand_inputs(2, 1, L0 + 5 + 3, N, d, seed=82)
+    cfg0 = cfg_of(layers, d, H, f, N, L0, q, fp8=fp8)
+    kv0, s0 = O.encode_user(cfg0, w, S_all[:, :L0])
+    cfg1 = cfg0.grown(5)
+    kv1, new1 = O.encode_append(cfg1, w, kv0, S_all[:, L0:L0 + 5])
+    kvf, sf = O.encode_user(cfg1, w, S_all[:, :L0 + 5])
+    np.testing.assert_allclose(kv1, kvf, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(new1, sf[:, -5:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(s0, sf[:, :-5], rtol=0, atol=1e-12)
+    for l in range(layers):  # the old rows' K/V moved unchanged into the grown layout
+        K0, V0 = O.kv_layer(cfg0, kv0[0], l)
+        K1, V1 = O.kv_layer(cfg1, kv1[0], l)
+        assert np.array_equal(K1[:K0.shape[0]], K0) and np.array_equal(V1[:V0.shape[0]], V0)
+    cfg2 = cfg1.grown(3)
+    kv2, new2 = O.encode_append(cfg2, w, kv1, S_all[:, L0 + 5:])
+    kvg, sg = O.encode_user(cfg2, w, S_all)
+    np.testing.assert_allclose(kv2, kvg, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(new2, sg[:, -3:], rtol=0, atol=1e-12)
+    if not fp8:
+        wl = to_lists(w)
+        bs, _, bkv = run_candidate(wl, S_all[1].double().tolist(), [[0.0] * d] * N, cfg2.q, H, 1e-6)
+        np.testing.assert_allclose(new2[1], np.array(bs)[-3:], rtol=0, atol=1e-12)
+        for l, (K, V) in enumerate(bkv):
+            Ko, Vo = O.kv_layer(cfg2, kv2[1], l)
+            np.testing.assert_allclose(Ko, np.array(K), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(Vo, np.array(V), rtol=0, atol=1e-12)
+
+
+def test_append_needs_anchored_windows():
+    """The reading the append rests on matters: re-deriving a shrinking
+    pyramid for the longer sequence (windows that slide) changes the old
+    rows' outputs, so the incremental result would not be a re-encode."""
+    layers, d, H, f, N = 2, 16, 2, 24, 1
+    w = rand_weights(layers, d, f, N, seed=83)
+    S_all, _ = rand_inputs(1, 1, 16, N, d, seed=84)
+    cfg0 = cfg_of(layers, d, H, f, N, 12, [12, 4])
+    kv0, _ = O.encode_user(cfg0, w, S_all[:, :12])
+    kv1, new1 = O.encode_append(cfg0.grown(4), w, kv0, S_all[:, 12:])
+    sliding = cfg_of(layers, d, H, f, N, 16, [12, 4])   # layer 1 keeps only the last 12 rows
+    _, ss = O.encode_user(sliding, w, S_all)
+    assert not np.allclose(new1[0], ss[0])
+    # the schedule the cache came from must be valid: every q[l] > delta
+    grown = cfg_of(layers, d, H, f, N, 12, [12, 4])
+    with pytest.raises(ValueError):
+        O.encode_append(grown, w, np.zeros((1, grown.grown(-4).kv_user_elems())), S_all[:, :4])
+
+
 def test_invariant_candidate_independence():
     layers, d, H, f, N, L0, q = _small()
     w = rand_weights(layers, d, f, N, seed=81)
