@@ -145,6 +145,36 @@ ot_status ot_embed_gather(const void *table, long rows, int d, const int64_t *id
 ot_status ot_encode_user(ot_model *m, const void *S, int U, void *kv_cache, void *out_s_tail,
                          void *ws, size_t ws_bytes, void *stream);
 
+/* Append `delta` new S tokens to each of U encoded users without encoding
+ * the old ones again (sequence KV caching across requests; summary page,
+ * KV-cache paragraph, which gives no schedule for it).  Reading: the pyramid
+ * windows stay anchored at their first row, so appending grows L0 and every
+ * query tail q[l] by delta; each old row then keeps exactly the keys it had at
+ * every layer (the mask is causal), so its K/V and outputs do not change and
+ * only the new rows are computed, against the cached K/V.
+ *   m        the model of the GROWN sequences: its L0 and q[l] include the
+ *            delta new rows (the old cache was written by a model with
+ *            L0 - delta and q[l] - delta and the same weights).
+ *   kv_old   device, the old cache (layout of that shorter configuration).
+ *   S_new    device [U][delta][d], the new rows in sequence order.
+ *   kv_new   device, ot_kv_cache_bytes(m, U) bytes: the grown cache, the old
+ *            rows' K/V copied into the grown layout and the new rows' K/V
+ *            after them in every layer; what ot_encode_user(m, old ++ new)
+ *            writes, up to rounding.
+ *   out_new  device [U][delta][d]: the new rows' outputs of the last layer,
+ *            i.e. the last delta rows of the grown S output (the rows before
+ *            them are the old call's output, unchanged).
+ * ws >= ot_append_workspace_bytes(m, U, delta).  kv_old and kv_new must not
+ * overlap.  Errors: OT_ERR_ARG (null pointer, delta < 1, overlapping
+ * caches), OT_ERR_SHAPE (q[last] <= delta, so the old schedule would be
+ * empty; d * sizeof(storage) not a multiple of 16; U > 65535),
+ * OT_ERR_ALIGN, OT_ERR_WORKSPACE_TOO_SMALL. */
+ot_status ot_encode_append(ot_model *m, const void *kv_old, int U, const void *S_new, int delta,
+                           void *kv_new, void *out_new, void *ws, size_t ws_bytes, void *stream);
+/* Workspace bytes of ot_encode_append for `users` users and `delta` new rows
+ * each: the encode buffers for users * delta rows. */
+size_t ot_append_workspace_bytes(const ot_model *m, int users, int delta);
+
 /* Score C candidates per user against the users' cached S K/V (NS-side):
  * ns device [U][C][N][d] -> out_ns device [U][C][N][d].  kv_cache as written
  * by ot_encode_user for the same U users.  ws >= ot_workspace_bytes(m, U, C).
@@ -233,7 +263,8 @@ ot_status ot_set_kernel_path(ot_model *m, int path);
 typedef enum {
     OT_KIND_GEMM_TC = 0, OT_KIND_GEMM_SIMT = 1, OT_KIND_ATTN_TC = 2, OT_KIND_ATTN_SIMT = 3,
     OT_KIND_GATHER = 4, OT_KIND_QUANT = 5, OT_KIND_FFN_TC = 6 /* fused FFN1 + GELU + FFN2 */,
-    OT_KIND_ATTN_NS = 7 /* NS attention, <= 64 query rows per (user, head) */
+    OT_KIND_ATTN_NS = 7 /* NS attention, <= 64 query rows per (user, head) */,
+    OT_KIND_KV_GROW = 8 /* old K/V rows into a grown cache (ot_encode_append) */
 } ot_kernel_kind;
 
 typedef struct {

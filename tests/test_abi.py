@@ -86,6 +86,8 @@ def test_calls_reject_null_model(lib):
     assert lib.ot_embed_gather(16, 1, 12, 16, 1, 16, None, None) == 2
     assert lib.ot_embed_gather(16, 1, 8, 16, 1, 24, None, None) == 4
     assert lib.ot_kv_cache_bytes(None, 1) == 0
+    assert lib.ot_encode_append(None, None, 1, None, 1, None, None, None, 0, None) == 1
+    assert lib.ot_append_workspace_bytes(None, 1, 1) == 0
     assert lib.ot_set_wait_limit(None, 5) == 1
     assert lib.ot_launch_count(None) == -1
 

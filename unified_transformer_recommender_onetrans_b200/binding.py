@@ -45,7 +45,7 @@ class OtLaunchRecord(C.Structure):
 
 
 KINDS = {0: "gemm_tc", 1: "gemm_simt", 2: "attn_tc", 3: "attn_simt", 4: "gather", 5: "quant",
-         6: "ffn_tc", 7: "attn_ns"}
+         6: "ffn_tc", 7: "attn_ns", 8: "kv_grow"}
 ROLES = {0: "S_QKV", 1: "S_attn", 2: "S_O", 3: "S_FFN1", 4: "S_FFN2", 5: "NS_QKV", 6: "NS_attn",
          7: "NS_O", 8: "NS_FFN1", 9: "NS_FFN2", 10: "auto_split", 11: "other", 12: "S_FFN",
          13: "NS_FFN", 14: "O", 15: "FFN", 16: "QKV"}
@@ -70,6 +70,8 @@ SIGNATURES = {
     "ot_profile_enable": (_i, [_vp, _i]),
     "ot_profile_read": (_i, [_vp, C.POINTER(OtLaunchRecord), _i]),
     "ot_score_candidates_noalloc": (_i, [_vp, _vp, _i, _vp, _i, _vp, _vp]),
+    "ot_encode_append": (_i, [_vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
+    "ot_append_workspace_bytes": (_sz, [_vp, _i, _i]),
 }
 
 _lib = None
@@ -266,6 +268,26 @@ class Model:
                                    ws.numel() * ws.element_size(), _stream(stream)),
               "ot_encode_user")
         return kv, out_s_tail
+
+    def append_workspace_bytes(self, users: int, delta: int) -> int:
+        return int(lib().ot_append_workspace_bytes(self.handle, users, delta))
+
+    def encode_append(self, kv_old, S_new, kv=None, out_new=None, ws=None, stream=None):
+        """Append S_new [U, delta, d] to users whose cache kv_old was written
+        by a model with L0 - delta and q[l] - delta (ot_encode_append); this
+        model is the grown one.  Returns (grown cache, the new rows' outputs
+        of the last layer [U, delta, d])."""
+        import torch
+        U, delta = S_new.shape[0], S_new.shape[1]
+        if kv is None:
+            kv = self.new_kv_cache(U)
+        if out_new is None:
+            out_new = torch.empty(U, delta, self.d, dtype=self.storage, device=S_new.device)
+        ws = self._ws(ws, self.append_workspace_bytes(U, delta))
+        check(lib().ot_encode_append(self.handle, _ptr(kv_old), U, _ptr(S_new), delta, _ptr(kv),
+                                     _ptr(out_new), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _stream(stream)), "ot_encode_append")
+        return kv, out_new
 
     def score_candidates(self, kv, ns, out=None, ws=None, stream=None):
         import torch

@@ -447,14 +447,19 @@ EpiSeg seg_of(void *out, long long ld, int lo, int hi, RowMap map)
 }
 
 // S-side of every layer for U users.  X0: [U][L0][d].  s_out may be null.
+// S-side of every layer for U users.  delta > 0 appends: X0 holds only the
+// delta new rows per user, and only they run through each layer (the last
+// delta of its L_l rows, all of them queries), attending to the cached K/V
+// of the old rows, which the caller has already placed in `kv`; their own
+// K/V go after the old rows.
 ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, Ws ws,
-                     cudaStream_t st, cudaEvent_t *kv_ready = nullptr)
+                     cudaStream_t st, cudaEvent_t *kv_ready = nullptr, int delta = 0)
 {
     const ot_config &c = m->cfg;
     const int d = c.d, f = c.ffn, esz = m->esz;
     const bool fp8 = c.dtype == OT_DTYPE_FP8;
     const int wesz = fp8 ? 1 : esz; // bytes per weight element as the GEMM reads it
-    const long long rows0 = static_cast<long long>(U) * c.L0;
+    const long long rows0 = static_cast<long long>(U) * (delta ? delta : c.L0);
     void *Xb[2] = {ws.take(rows0 * d), ws.take(rows0 * d)};
     void *Qb = ws.take(rows0 * d), *Ab = ws.take(rows0 * d), *Hb = ws.take(rows0 * d);
     void *hid = ws.take(rows0 * f);
@@ -471,16 +476,18 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
     const void *X = X0;
     ot_status r;
     for (int l = 0; l < c.layers; ++l) {
-        const int L = rows_at(c, l), q = c.q[l];
+        const int L = rows_at(c, l);
+        const int n = delta ? delta : L;        // rows run through this layer (the last n of L)
+        const int q = delta ? delta : c.q[l];   // their query tail
         const bool last = l == c.layers - 1;
         const bool kv_only = last && s_out == nullptr; // the S tail of the last layer is unused
         char *K = at(kv, kv_layer_off(c, l), esz);
         char *V = K + static_cast<long long>(L) * d * esz;
-        const RowMap cache_map{L, ustride / d, 0, 0, 0};
+        const RowMap cache_map{n, ustride / d, L - n, 0, 0};
         const void *g1 = fp8 ? at(m->g1_s, static_cast<long long>(l) * d, esz) : nullptr;
         const void *g2 = fp8 ? at(m->g2_s, static_cast<long long>(l) * d, esz) : nullptr;
         // 1. QKV (or KV only): RMSNorm1 + shared projection; K/V into the cache
-        GemmArgs g = gemm_base(c, U * L, kv_only ? 2 * d : 3 * d, d, 1);
+        GemmArgs g = gemm_base(c, U * n, kv_only ? 2 * d : 3 * d, d, 1);
         if ((r = projection(m, g, X, d, rowmap_identity(),
                             at(m->Wqkv_s, static_cast<long long>(l) * 3 * d * d + (kv_only ? d * d : 0), wesz),
                             3LL * d * d, fp8 ? m->sc_qkv_s + l : nullptr, g1, d, true, f8, st)) != OT_OK)
@@ -491,7 +498,7 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
             g.seg[1] = seg_of(V, d, d, 2 * d, cache_map);
         } else {
             g.nseg = 3;
-            g.seg[0] = seg_of(Qb, d, 0, d, RowMap{L, q, -(L - q), 0, L - q});
+            g.seg[0] = seg_of(Qb, d, 0, d, RowMap{n, q, -(n - q), 0, n - q});
             g.seg[1] = seg_of(K, d, d, 2 * d, cache_map);
             g.seg[2] = seg_of(V, d, 2 * d, 3 * d, cache_map);
         }
@@ -525,7 +532,7 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
             return r;
         g.res = X;
         g.res_ld = d;
-        g.res_map = RowMap{q, L, L - q, 0, 0};
+        g.res_map = RowMap{q, n, n - q, 0, 0};
         g.nseg = 1;
         g.seg[0] = seg_of(Hb, d, 0, d, rowmap_identity());
         if ((r = gemm(m, g, st, ROLE_S_O)) != OT_OK) return r;
@@ -1099,6 +1106,57 @@ ot_status ot_encode_user(ot_model *m, const void *S, int U, void *kv_cache, void
     if (ws_bytes < ot_workspace_bytes(m, U, 0)) return OT_ERR_WORKSPACE_TOO_SMALL;
     Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
     return run_encode(m, S, U, kv_cache, out_s_tail, w, static_cast<cudaStream_t>(stream));
+}
+
+size_t ot_append_workspace_bytes(const ot_model *m, int users, int delta)
+{
+    if (!m || users < 0 || delta < 0) return 0;
+    const long long rows = static_cast<long long>(users) * delta;
+    const ot_config &c = m->cfg;
+    return 5 * bytes_of(rows * c.d, m->esz) + bytes_of(rows * c.ffn, m->esz) + fp8_ws_bytes(c, rows);
+}
+
+ot_status ot_encode_append(ot_model *m, const void *kv_old, int U, const void *S_new, int delta,
+                           void *kv_new, void *out_new, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!m || !kv_old || !S_new || !kv_new || !out_new || !ws || U < 1 || delta < 1) return OT_ERR_ARG;
+    if (!aligned16(kv_old) || !aligned16(S_new) || !aligned16(kv_new) || !aligned16(out_new) ||
+        !aligned16(ws))
+        return OT_ERR_ALIGN;
+    const ot_config &c = m->cfg; // the grown sequences
+    // the configuration the old cache was written with: every window shorter by delta
+    ot_config o = c;
+    o.L0 -= delta;
+    for (int l = 0; l < c.layers; ++l) o.q[l] -= delta;
+    if (o.L0 < 1 || o.q[c.layers - 1] < 1) return OT_ERR_SHAPE;
+    if ((static_cast<long long>(c.d) * m->esz) % 16) return OT_ERR_SHAPE;
+    if (U > 65535 || static_cast<long long>(U) * c.L0 > (1LL << 31) - 1) return OT_ERR_SHAPE;
+    const long long bytes_old = static_cast<long long>(U) * kv_user_elems(o) * m->esz;
+    const long long bytes_new = static_cast<long long>(U) * kv_user_elems(c) * m->esz;
+    const char *po = static_cast<const char *>(kv_old), *pn = static_cast<const char *>(kv_new);
+    if (po < pn + bytes_new && pn < po + bytes_old) return OT_ERR_ARG; // the caches overlap
+    if (ws_bytes < ot_append_workspace_bytes(m, U, delta)) return OT_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // 1. the old rows' K/V into the grown layout (16-byte units)
+    KvGrowArgs g;
+    memset(&g, 0, sizeof(g));
+    const long long unit = 16 / m->esz; // elements per unit
+    g.src = static_cast<const uint4 *>(kv_old);
+    g.dst = static_cast<uint4 *>(kv_new);
+    g.ustride_src = kv_user_elems(o) / unit;
+    g.ustride_dst = kv_user_elems(c) / unit;
+    for (int l = 0; l < c.layers; ++l) {
+        g.off_src[l] = kv_layer_off(o, l) / unit;
+        g.off_dst[l] = kv_layer_off(c, l) / unit;
+        g.len_src[l] = static_cast<long long>(rows_at(o, l)) * c.d / unit;
+        g.len_dst[l] = static_cast<long long>(rows_at(c, l)) * c.d / unit;
+    }
+    ot_status r = profiled(m, st, OT_KIND_KV_GROW, ROLE_OTHER, 0.0,
+                           2.0 * static_cast<double>(bytes_old), [&] { return launch_kv_grow(g, U, c.layers, st); });
+    if (r != OT_OK) return r;
+    // 2. the new rows through every layer, against the grown cache
+    Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
+    return run_encode(m, S_new, U, kv_new, out_new, w, st, nullptr, delta);
 }
 
 ot_status ot_score_candidates(ot_model *m, const void *kv_cache, int U, const void *ns, int C,

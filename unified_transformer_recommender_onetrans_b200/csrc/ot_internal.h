@@ -152,6 +152,18 @@ cudaError_t launch_ffn_tc(const FfnArgs &a, cudaStream_t s);
 cudaError_t launch_ffn_tc_multi(const FfnArgs &a, const FfnArgs *a1, cudaStream_t s);
 cudaError_t launch_fold_gain(const void *W, const void *g, void *out, long long rows, int cols,
                              long long groups, long long g_gstride, int dtype, cudaStream_t s);
+// Copy of the old K/V rows of a cache into the layout of longer sequences
+// (appending S rows): per layer l, the len_src[l] units of K (then of V)
+// starting at off_src[l] of a user's cache go to off_dst[l] (V at
+// off_dst[l] + len_dst[l]) of the new one.  Units of 16 bytes.
+struct KvGrowArgs {
+    const uint4 *src;
+    uint4 *dst;
+    long long ustride_src, ustride_dst;
+    long long off_src[OT_MAX_LAYERS], off_dst[OT_MAX_LAYERS];
+    long long len_src[OT_MAX_LAYERS], len_dst[OT_MAX_LAYERS];
+};
+cudaError_t launch_kv_grow(const KvGrowArgs &a, int users, int layers, cudaStream_t s);
 cudaError_t launch_embed_gather(const void *table, long long rows, int d, const int64_t *ids,
                                 long long n, void *out, int *err, cudaStream_t s);
 cudaError_t launch_quant_rows(const void *X, long long lda, RowMap map, long long M, int G, int K,

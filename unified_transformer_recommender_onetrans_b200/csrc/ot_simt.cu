@@ -321,4 +321,34 @@ cudaError_t launch_embed_gather(const void *table, long long rows, int d, const 
     return cudaGetLastError();
 }
 
+// Old K/V rows of every (user, layer) into the layout of a longer sequence:
+// block (x, l * 2 + kv, u) copies a slice of user u's layer-l K (kv = 0) or
+// V (kv = 1) block, all offsets in 16-byte units.
+__global__ void kv_grow_kernel(const __grid_constant__ KvGrowArgs a)
+{
+    const int l = static_cast<int>(blockIdx.y) >> 1, kv = static_cast<int>(blockIdx.y) & 1;
+    const long long u = blockIdx.z;
+    const long long n = a.len_src[l];
+    const uint4 *src = a.src + u * a.ustride_src + a.off_src[l] + kv * n;
+    uint4 *dst = a.dst + u * a.ustride_dst + a.off_dst[l] + kv * a.len_dst[l];
+    const long long step = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n; i += step)
+        dst[i] = __ldg(src + i);
+}
+
+cudaError_t launch_kv_grow(const KvGrowArgs &a, int users, int layers, cudaStream_t s)
+{
+    if (users < 1 || users > 65535 || layers < 1 || layers > OT_MAX_LAYERS) return cudaErrorInvalidValue;
+    long long longest = 0;
+    for (int l = 0; l < layers; ++l) longest = a.len_src[l] > longest ? a.len_src[l] : longest;
+    // enough blocks per (user, layer, K|V) to cover its longest slice in a
+    // few strides, at least one
+    long long bx = (longest + 4 * 256 - 1) / (4 * 256);
+    if (bx < 1) bx = 1;
+    if (bx > 64) bx = 64;
+    kv_grow_kernel<<<dim3(static_cast<unsigned>(bx), static_cast<unsigned>(2 * layers), static_cast<unsigned>(users)),
+                     256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 } // namespace ot
