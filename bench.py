@@ -365,10 +365,50 @@ def measure_fp8_peak(dev, n=8192, seconds=2.0):
         return {"error": str(e).splitlines()[0][:200]}
 
 
-def run_serving(name, steps, flush, world, dist, dev, peaks, cands=None, sweep=None):
+def _append_point(m, wl, w, q, S, kv, delta, steps, flush, world, dist, dev):
+    """Append `delta` new S tokens per user to the encoded users
+    (ot_encode_append on the grown model: only the new rows run, against the
+    cached K/V) against encoding the grown sequences from scratch."""
+    import torch
+
+    import unified_transformer_recommender_onetrans_b200 as ot
+    from unified_transformer_recommender_onetrans_b200.binding import WEIGHT_NAMES
+
+    U = S.shape[0]
+    m2 = ot.Model(layers=wl.layers, d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns,
+                  L0=wl.L0 + delta, q=[v + delta for v in q], F=wl.F, eps=wl.eps, dtype=wl.dtype,
+                  weights={k: w[k].to(dev) for k in WEIGHT_NAMES})
+    g = torch.Generator().manual_seed(7)
+    S_new = torch.randn(U, delta, wl.d, generator=g).to(S.dtype).to(dev)
+    S_all = torch.cat([S, S_new], dim=1).contiguous()
+    kv2 = m2.new_kv_cache(U)
+    out_new = torch.empty(U, delta, wl.d, dtype=S.dtype, device=dev)
+    ws_a = torch.empty(m2.append_workspace_bytes(U, delta), dtype=torch.uint8, device=dev)
+    ws_e = torch.empty(m2.workspace_bytes(U, 0), dtype=torch.uint8, device=dev)
+
+    def append():
+        m2.encode_append(kv, S_new, kv=kv2, out_new=out_new, ws=ws_a)
+
+    def reencode():
+        m2.encode_user(S_all, kv=kv2, ws=ws_e, want_s_tail=False)
+
+    for _ in range(10):
+        append()
+        reencode()
+    m2.poll()
+    app_ms = _time_device(append, steps, flush, world, dist, dev)
+    enc_ms = _time_device(reencode, steps, flush, world, dist, dev)
+    m2.poll()
+    del m2, kv2, ws_a, ws_e
+    return {"delta": delta, "ms": app_ms, "new_s_tokens_per_s": world * U * delta / (app_ms / 1e3),
+            "reencode_ms": enc_ms, "speedup_vs_reencode": enc_ms / app_ms}
+
+
+def run_serving(name, steps, flush, world, dist, dev, peaks, cands=None, sweep=None, append_rows=0):
     """Encode once per user, then score every candidate against the cache
     (Auto-Split of the candidates' features included in scoring); with
-    `sweep`, score the same cache again at each candidate count in it."""
+    `sweep`, score the same cache again at each candidate count in it; with
+    `append_rows`, also time appending that many S tokens per user."""
     import torch
 
     import unified_transformer_recommender_onetrans_b200 as ot
@@ -418,6 +458,8 @@ def run_serving(name, steps, flush, world, dist, dev, peaks, cands=None, sweep=N
         "encode_ms": enc_ms,
         "encode_tflops": enc_flops / (enc_ms / 1e3) / 1e12,
     })
+    if append_rows and gather is None:
+        out["append"] = _append_point(m, wl, w, q, S, kv, append_rows, steps, flush, world, dist, dev)
     bf16_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     tensor_peak = {"gemm": bf16_peak, "attn": bf16_peak}
     peak_note = f"{peaks['_source']} bf16 dense sustained"
@@ -573,7 +615,8 @@ def run_ours(args, wl):
         for name, cands, sw in (("onetrans_s_serve", None, sweep), ("onetrans_l_full", 8, sweep),
                                 ("long_fp8", None, None)):
             # 10 warm-up calls, median of 50 per call
-            serving.append(run_serving(name, 50, flush, world, dist, dev, peaks, cands, sw))
+            serving.append(run_serving(name, 50, flush, world, dist, dev, peaks, cands, sw,
+                                       append_rows=64 if name == "onetrans_s_serve" else 0))
             torch.cuda.empty_cache()
 
     # ---- roofline of the dominant kernel (from the live per-launch events)
