@@ -338,12 +338,29 @@ void ffn_cost(const FfnArgs &a, double &flops, double &bytes)
     const double rows = static_cast<double>(a.M) * a.G, d = a.D, f = a.F;
     flops += 4.0 * rows * d * f;
     bytes += 2.0 * (2.0 * rows * d + 2.0 * a.G * d * f); // H in, Y out, W1 + W2 once
+    if (a.fuse_o) {
+        flops += 2.0 * rows * d * d;
+        bytes += 2.0 * (rows * d + a.G * d * d); // X in, Wo once (A in replaces H in)
+    }
 }
 
-ot_status ffn(ot_model *m, int M, int G, const void *H, RowMap h_map, const void *W1,
-              const void *W2, void *Y, RowMap y_map, cudaStream_t s, int role)
+// The FFN with the attention's output projection in front (FfnArgs::fuse_o):
+// H = X + A Wo^T, A read as the FFN's H otherwise is (rows under a_map), X
+// under x_map; then Y = H + GELU(n(H) W1^T) W2^T.
+FfnArgs ffn_o_args(const ot_model *m, int M, int G, const void *A, RowMap a_map, const void *Wo,
+                   const void *X, RowMap x_map, const void *W1, const void *W2, void *Y, RowMap y_map)
 {
-    FfnArgs a = ffn_args(m, M, G, H, h_map, W1, W2, Y, y_map);
+    FfnArgs a = ffn_args(m, M, G, A, a_map, W1, W2, Y, y_map);
+    a.fuse_o = 1;
+    a.Wo = Wo;
+    a.wo_gstride = static_cast<long long>(m->cfg.d) * m->cfg.d;
+    a.X = X;
+    a.x_map = x_map;
+    return a;
+}
+
+ot_status ffn_run(ot_model *m, const FfnArgs &a, cudaStream_t s, int role)
+{
     double flops = 0, bytes = 0;
     if (m->profiling) ffn_cost(a, flops, bytes);
     return profiled(m, s, OT_KIND_FFN_TC, role, flops, bytes, [&] { return launch_ffn_tc(a, s); });
@@ -523,6 +540,20 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
         at_.O = Ab;
         at_.scale = 1.0f / sqrtf(static_cast<float>(at_.hd));
         if ((r = attn(m, at_, st)) != OT_OK) return r;
+        void *Xn = (last && s_out) ? s_out : Xb[l & 1];
+        if (use_fused_ffn(m)) {
+            // 3 + 4 in one launch: O projection + residual from the tail rows
+            // of the layer input, RMSNorm2, W1, GELU, W2, residual
+            const FfnArgs fa = ffn_o_args(m, U * q, 1, Ab, rowmap_identity(),
+                                          at(m->Wo_s, static_cast<long long>(l) * d * d, esz), X,
+                                          RowMap{q, n, n - q, 0, 0},
+                                          at(m->W1_s, static_cast<long long>(l) * f * d, esz),
+                                          at(m->W2_s, static_cast<long long>(l) * d * f, esz), Xn,
+                                          rowmap_identity());
+            if ((r = ffn_run(m, fa, st, ROLE_S_FFN)) != OT_OK) return r;
+            X = Xn;
+            continue;
+        }
         // 3. O projection + residual from the tail rows of the layer input
         g = gemm_base(c, U * q, d, d, 1);
         if ((r = projection(m, g, Ab, d, rowmap_identity(),
@@ -537,15 +568,6 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
         g.seg[0] = seg_of(Hb, d, 0, d, rowmap_identity());
         if ((r = gemm(m, g, st, ROLE_S_O)) != OT_OK) return r;
         // 4. FFN: RMSNorm2 + W1 + GELU, then W2 + residual
-        void *Xn = (last && s_out) ? s_out : Xb[l & 1];
-        if (use_fused_ffn(m)) {
-            if ((r = ffn(m, U * q, 1, Hb, rowmap_identity(), at(m->W1_s, static_cast<long long>(l) * f * d, esz),
-                         at(m->W2_s, static_cast<long long>(l) * d * f, esz), Xn, rowmap_identity(), st,
-                         ROLE_S_FFN)) != OT_OK)
-                return r;
-            X = Xn;
-            continue;
-        }
         g = gemm_base(c, U * q, f, d, 1);
         if ((r = projection(m, g, Hb, d, rowmap_identity(),
                             at(m->W1_s, static_cast<long long>(l) * f * d, wesz),
@@ -636,6 +658,15 @@ ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, v
         at_.O = An;
         at_.scale = 1.0f / sqrtf(static_cast<float>(at_.hd));
         if ((r = attn(m, at_, st)) != OT_OK) return r;
+        void *Xn = last ? out : Xb[l & 1];
+        if (use_fused_ffn(m)) {
+            // O projection + residual and the FFN in one grouped launch
+            const FfnArgs fa = ffn_o_args(m, Mc, N, An, grp, at(m->Wo_ns, lN * d * d, esz), X, grp,
+                                          at(m->W1_ns, lN * f * d, esz), at(m->W2_ns, lN * d * f, esz), Xn, grp);
+            if ((r = ffn_run(m, fa, st, ROLE_NS_FFN)) != OT_OK) return r;
+            X = Xn;
+            continue;
+        }
         g = gemm_base(c, Mc, d, d, N);
         if ((r = projection(m, g, An, d, grp, at(m->Wo_ns, lN * d * d, wesz),
                             static_cast<long long>(d) * d, fp8 ? m->sc_o_ns + lN : nullptr, nullptr,
@@ -647,14 +678,6 @@ ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, v
         g.nseg = 1;
         g.seg[0] = seg_of(Hn, d, 0, d, grp);
         if ((r = gemm(m, g, st, ROLE_NS_O)) != OT_OK) return r;
-        void *Xn = last ? out : Xb[l & 1];
-        if (use_fused_ffn(m)) {
-            if ((r = ffn(m, Mc, N, Hn, grp, at(m->W1_ns, lN * f * d, esz), at(m->W2_ns, lN * d * f, esz), Xn,
-                         grp, st, ROLE_NS_FFN)) != OT_OK)
-                return r;
-            X = Xn;
-            continue;
-        }
         g = gemm_base(c, Mc, f, d, N);
         if ((r = projection(m, g, Hn, d, grp, at(m->W1_ns, lN * f * d, wesz),
                             static_cast<long long>(f) * d, fp8 ? m->sc_1_ns + lN : nullptr, g2, d,
@@ -779,33 +802,16 @@ ot_status run_full_merged(ot_model *m, const void *X0, int U, const void *ns, in
         // 3. S attention (main stream)
         if ((r = attn(m, as_, st)) != OT_OK) return r;
         if (two && cudaStreamWaitEvent(st, m->ns_attn_done[l], 0) != cudaSuccess) return OT_ERR_CUDA;
-        // 4. O projection + residual, both sides in one launch
-        GemmArgs os_ = gemm_base(c, U * q, d, d, 1);
-        if ((r = projection(m, os_, Ab, d, rowmap_identity(), at(m->Wo_s, static_cast<long long>(l) * d * d, m->esz),
-                            static_cast<long long>(d) * d, nullptr, nullptr, 0, false, no_f8, st)) != OT_OK)
-            return r;
-        os_.res = X;
-        os_.res_ld = d;
-        os_.res_map = RowMap{q, L, L - q, 0, 0};
-        os_.nseg = 1;
-        os_.seg[0] = seg_of(Hb, d, 0, d, rowmap_identity());
-        GemmArgs on_ = gemm_base(c, Mc, d, d, N);
-        if ((r = projection(m, on_, An, d, grp, at(m->Wo_ns, lN * d * d, m->esz), static_cast<long long>(d) * d,
-                            nullptr, nullptr, 0, false, no_f8, st)) != OT_OK)
-            return r;
-        on_.res = Y;
-        on_.res_ld = d;
-        on_.res_map = grp;
-        on_.nseg = 1;
-        on_.seg[0] = seg_of(Hn, d, 0, d, grp);
-        if ((r = gemm2(m, &os_, &on_, st, ROLE_O)) != OT_OK) return r;
-        // 5. FFN (RMSNorm, W1, GELU, W2, residual), both sides in one launch
+        // 4. O projection + residual, RMSNorm, W1, GELU, W2, residual: both
+        // sides in one launch
         void *Xn = (last && s_out) ? s_out : Xb[l & 1];
         void *Yn = last ? out : Yb[l & 1];
-        FfnArgs fs = ffn_args(m, U * q, 1, Hb, rowmap_identity(), at(m->W1_s, static_cast<long long>(l) * f * d, m->esz),
-                              at(m->W2_s, static_cast<long long>(l) * d * f, m->esz), Xn, rowmap_identity());
-        FfnArgs fn = ffn_args(m, Mc, N, Hn, grp, at(m->W1_ns, lN * f * d, m->esz), at(m->W2_ns, lN * d * f, m->esz),
-                              Yn, grp);
+        FfnArgs fs = ffn_o_args(m, U * q, 1, Ab, rowmap_identity(),
+                                at(m->Wo_s, static_cast<long long>(l) * d * d, m->esz), X, RowMap{q, L, L - q, 0, 0},
+                                at(m->W1_s, static_cast<long long>(l) * f * d, m->esz),
+                                at(m->W2_s, static_cast<long long>(l) * d * f, m->esz), Xn, rowmap_identity());
+        FfnArgs fn = ffn_o_args(m, Mc, N, An, grp, at(m->Wo_ns, lN * d * d, m->esz), Y, grp,
+                                at(m->W1_ns, lN * f * d, m->esz), at(m->W2_ns, lN * d * f, m->esz), Yn, grp);
         if ((r = ffn2(m, &fs, &fn, st)) != OT_OK) return r;
         X = Xn;
         Y = Yn;

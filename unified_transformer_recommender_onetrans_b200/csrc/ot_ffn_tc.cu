@@ -97,12 +97,19 @@ __device__ __forceinline__ float ffn_gelu(float z)
     return fmaf(hz, t, hz);
 }
 
-template <int D>
+// FO (fused output projection): the tile's TMA load brings the attention
+// output A instead of H; the epilogue first seeds acc2 with the block input
+// rows X, the FFN1 issuer accumulates A Wo^T onto them (Wo streamed through
+// the W1 stages ahead of the tile's W1 chunks), and the epilogue turns
+// acc2 = H into the bf16 H tile in shared memory (plus the norm's sums) that
+// FFN1 reads; FFN2 then accumulates onto H in fp32.
+template <int D, bool FO>
 __global__ void __launch_bounds__(FF_THREADS, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmH0, const __grid_constant__ CUtensorMap tmW10,
                   const __grid_constant__ CUtensorMap tmW20, const __grid_constant__ CUtensorMap tmY0,
                   const __grid_constant__ CUtensorMap tmH1, const __grid_constant__ CUtensorMap tmW11,
                   const __grid_constant__ CUtensorMap tmW21, const __grid_constant__ CUtensorMap tmY1,
+                  const __grid_constant__ CUtensorMap tmWo0, const __grid_constant__ CUtensorMap tmWo1,
                   const __grid_constant__ FfnMulti P)
 {
     using Sh = FfnShape<D>;
@@ -139,7 +146,9 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
     uint64_t *a2_init = a2_full + 1;   // acc2 holds the tile's H (the residual) in fp32
     uint64_t *stg_free = a2_init + 1;  // the W2 stages no longer hold the previous output
     uint64_t *mma_done = stg_free + 1; // [2] one per issuer
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 2);
+    uint64_t *o_done = mma_done + 2;   // FO: acc2 = X + A Wo^T complete
+    uint64_t *hb_full = o_done + 1;    // FO: the bf16 H tile is in sH
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(hb_full + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -163,6 +172,8 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
         mbar_init(a2_full, 1);
         mbar_init(a2_init, FF_EPI_WARPS);
         mbar_init(stg_free, 1);
+        mbar_init(o_done, 1);
+        mbar_init(hb_full, FF_EPI_WARPS);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -195,26 +206,42 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             }
             tma_prefetch(w1_side ? &tmW10 : &tmW20);
             if (two) tma_prefetch(w1_side ? &tmW11 : &tmW21);
+            if (FO && w1_side) {
+                tma_prefetch(&tmWo0);
+                if (two) tma_prefetch(&tmWo1);
+            }
+            // W1-side loads per tile: (FO) the KS chunks of Wo, then the NC
+            // half-chunks of W1; W2 side: the NC chunks of W2.  Load j of a
+            // side goes to stage j % 2 (KS and NC are even, so a W1 chunk's
+            // K-half h always lands in stage h)
+            constexpr int NWO = FO ? KS : 0;
+            const int n_side = (w1_side ? NWO : 0) + NC;
             // The weights are not written by any kernel in flight: the first
             // tile's first two W1 / W2 stages load while the previous kernel
             // finishes (fresh stages, no empty wait); H follows once its
             // outputs are visible.
-            const int n_pre = static_cast<long long>(blockIdx.x) < P.tiles ? (NC < 2 ? NC : 2) : 0;
+            const int n_pre = static_cast<long long>(blockIdx.x) < P.tiles ? (n_side < 2 ? n_side : 2) : 0;
+            // load j of this side for group g into stage st
+            auto load = [&](int pi, int g, int j, int st) {
+                if (w1_side) {
+                    mbar_arrive_expect_tx(&w1_full[st], Sh::W1_BYTES);
+                    if (j < NWO) { // Wo columns 64 j .. 64 j + 63, all D rows
+                        tma_load_3d(sW1 + st * Sh::W1_BYTES, pi ? &tmWo1 : &tmWo0, &w1_full[st], j * 64, 0, g);
+                        return;
+                    }
+                    const int c = j - NWO;
+                    for (int k = 0; k < KS / 2; ++k)
+                        tma_load_3d(sW1 + st * Sh::W1_BYTES + k * FF_SLAB, pi ? &tmW11 : &tmW10, &w1_full[st],
+                                    (st * (KS / 2) + k) * 64, (c >> 1) * FF_BH1, g);
+                } else {
+                    mbar_arrive_expect_tx(&w2_full[st], Sh::W2_BYTES);
+                    tma_load_3d(sW2 + st * Sh::W2_BYTES, pi ? &tmW21 : &tmW20, &w2_full[st], j * FF_BH, 0, g);
+                }
+            };
             if (n_pre > 0) {
                 int g, m0;
                 const int pi = ffn_tile(P, blockIdx.x, g, m0);
-                const CUtensorMap *tW1 = pi ? &tmW11 : &tmW10, *tW2 = pi ? &tmW21 : &tmW20;
-                for (int c = 0; c < n_pre; ++c) {
-                    if (w1_side) {
-                        mbar_arrive_expect_tx(&w1_full[c], Sh::W1_BYTES);
-                        for (int k = 0; k < KS / 2; ++k)
-                            tma_load_3d(sW1 + c * Sh::W1_BYTES + k * FF_SLAB, tW1, &w1_full[c],
-                                        (c * (KS / 2) + k) * 64, (c >> 1) * FF_BH1, g);
-                    } else {
-                        mbar_arrive_expect_tx(&w2_full[c], Sh::W2_BYTES);
-                        tma_load_3d(sW2 + c * Sh::W2_BYTES, tW2, &w2_full[c], c * FF_BH, 0, g);
-                    }
-                }
+                for (int j = 0; j < n_pre; ++j) load(pi, g, j, j);
             }
             pdl_wait();
             long long gc = 0; // global chunk counter
@@ -224,7 +251,6 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                 int g, m0;
                 const int pi = ffn_tile(P, tile, g, m0);
                 const CUtensorMap *tH = pi ? &tmH1 : &tmH0;
-                const CUtensorMap *tW1 = pi ? &tmW11 : &tmW10, *tW2 = pi ? &tmW21 : &tmW20;
                 if (w1_side) {
                     if (!mbar_wait(h_free, (tl & 1) ^ 1, a.wait, abort_flag)) break;
                     mbar_arrive_expect_tx(h_full, Sh::H_BYTES);
@@ -238,28 +264,15 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                 } else if (tl > 0 && !mbar_wait(stg_free, (tl - 1) & 1, a.wait, abort_flag)) {
                     break; // the W2 stages staged the previous tile's output
                 }
-                for (int c = 0; c < NC; ++c, ++gc) {
+                for (int j = 0; j < n_side; ++j, ++gc) {
                     const int st = static_cast<int>(gc & 1);
                     const uint32_t ph = static_cast<uint32_t>((gc >> 1) & 1);
                     if (gc < n_pre) continue; // issued before the wait
-                    if (w1_side) {
-                        // FFN1 chunk gc / 2 (128 hidden rows of W1), its K-half gc % 2
-                        if (!mbar_wait(&w1_empty[st], ph ^ 1, a.wait, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        mbar_arrive_expect_tx(&w1_full[st], Sh::W1_BYTES);
-                        for (int k = 0; k < KS / 2; ++k)
-                            tma_load_3d(sW1 + st * Sh::W1_BYTES + k * FF_SLAB, tW1, &w1_full[st],
-                                        (st * (KS / 2) + k) * 64, (c >> 1) * FF_BH1, g);
-                    } else {
-                        if (!mbar_wait(&w2_empty[st], ph ^ 1, a.wait, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        mbar_arrive_expect_tx(&w2_full[st], Sh::W2_BYTES);
-                        tma_load_3d(sW2 + st * Sh::W2_BYTES, tW2, &w2_full[st], c * FF_BH, 0, g);
+                    if (!mbar_wait(w1_side ? &w1_empty[st] : &w2_empty[st], ph ^ 1, a.wait, abort_flag)) {
+                        ok = false;
+                        break;
                     }
+                    load(pi, g, j, st);
                 }
             }
             // never leave a load in flight
@@ -272,21 +285,47 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
         // ------------------------------------------------ FFN1 issuer
         if (lane == 0) {
             long long gc1 = 0; // global FFN1 chunk counter (128 hidden each)
+            long long gw = 0;  // W1-stage loads consumed (stage gw % 2, use gw / 2 of it)
             int tl = 0;
             bool ok = true;
             for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x, ++tl) {
                 if (!mbar_wait(h_full, tl & 1, a.wait, abort_flag)) break;
+                if (FO) {
+                    // acc2 = X (seeded by the epilogue) + A Wo^T, A from the
+                    // H buffer, Wo chunk j (K = 64 j .. 64 j + 63) from the W1 stages
+                    if (!mbar_wait(a2_init, tl & 1, a.wait, abort_flag)) break;
+                    tc_fence_after();
+                    for (int j = 0; j < KS; ++j, ++gw) {
+                        const int st = static_cast<int>(gw & 1);
+                        if (!mbar_wait(&w1_full[st], static_cast<uint32_t>((gw >> 1) & 1), a.wait, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t a_addr = smem_u32(sH + j * FF_SLAB);
+                        const uint32_t w_addr = smem_u32(sW1 + st * Sh::W1_BYTES);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_f16(t_acc2, sw128_desc(a_addr + k * 32, 16), sw128_desc(w_addr + k * 32, 16),
+                                    IDESC2, 1);
+                        mma_commit(&w1_empty[st]);
+                    }
+                    if (!ok) break;
+                    mma_commit(o_done);
+                    // FFN1 reads the bf16 H the epilogue made of acc2
+                    if (!mbar_wait(hb_full, tl & 1, a.wait, abort_flag)) break;
+                }
                 tc_fence_after();
                 for (int c1 = 0; c1 < NC / 2 && ok; ++c1, ++gc1) {
                     const int b = static_cast<int>(gc1 & 1);
-                    const uint32_t ph = static_cast<uint32_t>(gc1 & 1);
                     if (!mbar_wait(&a1_free[b], static_cast<uint32_t>((gc1 >> 1) & 1) ^ 1, a.wait, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    for (int st = 0; st < 2; ++st) {
-                        if (!mbar_wait(&w1_full[st], ph, a.wait, abort_flag)) {
+                    for (int st = 0; st < 2; ++st, ++gw) {
+                        // K-half st of this chunk is W1-stage load gw, in stage st
+                        if (!mbar_wait(&w1_full[st], static_cast<uint32_t>((gw >> 1) & 1), a.wait, abort_flag)) {
                             ok = false;
                             break;
                         }
@@ -327,8 +366,9 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                         break;
                     }
                     // the tile's first chunk accumulates onto H, which the
-                    // epilogue has stored into acc2
-                    if (c == 0 && !mbar_wait(a2_init, tl & 1, a.wait, abort_flag)) {
+                    // epilogue has stored into acc2 (FO: which the output
+                    // projection left there and the epilogue has read)
+                    if (c == 0 && !mbar_wait(FO ? hb_full : a2_init, tl & 1, a.wait, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -359,43 +399,111 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
         for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x, ++tl) {
             int g, m0;
             const int pi = ffn_tile(P, tile, g, m0);
-            if (!mbar_wait(h_full, tl & 1, a.wait, abort_flag)) break;
-            // This warp's half of its rows of H (columns hf*HALF ..): the
-            // RMSNorm partial sum of squares, and the values in fp32 into
-            // acc2, onto which the second projection accumulates (so the
-            // residual needs no read at the end).  acc2 is free: the previous
-            // tile's output was read out of it by these warps.  Chunk j of a
-            // slab row sits at 16-byte position j ^ (r & 7).
             float ss = 0.f;
+            if (FO) {
+                // acc2 = X, the block input rows (the output projection's
+                // residual); acc2 is free: the previous tile's output was read
+                // out of it by these warps
+                const FfnArgs &pa = P.q[pi].a;
+                const long long gr = static_cast<long long>(m0) + r; // row of the problem in group g
+                const bool live = gr < pa.M;
+                const __nv_bfloat16 *xrow =
+                    static_cast<const __nv_bfloat16 *>(pa.X) + (live ? rowmap_apply(pa.x_map, gr, g) : 0) * D;
 #pragma unroll 1
-            for (int c32 = 0; c32 < HALF / 32; ++c32) {
-                const int col = hf * HALF + 32 * c32;
-                const uint8_t *row = sH + (col / 64) * FF_SLAB + r * 128;
-                uint32_t hv[32];
+                for (int c32 = 0; c32 < HALF / 32; ++c32) {
+                    const int col = hf * HALF + 32 * c32;
+                    uint32_t hv[32];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(row + ((((col % 64) / 8 + i) ^ (r & 7)) << 4));
-                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                    for (int i = 0; i < 4; ++i) {
+                        const uint4 v = live ? *reinterpret_cast<const uint4 *>(xrow + col + 8 * i) : make_uint4(0, 0, 0, 0);
+                        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float lo = __uint_as_float(w4[e] << 16);
-                        const float hi = __uint_as_float(w4[e] & 0xFFFF0000u);
-                        ss = fmaf(lo, lo, ss);
-                        ss = fmaf(hi, hi, ss);
-                        hv[8 * i + 2 * e] = __float_as_uint(lo);
-                        hv[8 * i + 2 * e + 1] = __float_as_uint(hi);
+                        for (int e = 0; e < 4; ++e) {
+                            hv[8 * i + 2 * e] = w4[e] << 16;
+                            hv[8 * i + 2 * e + 1] = w4[e] & 0xFFFF0000u;
+                        }
+                    }
+                    tmem_st32(t_acc2 + lane_off + col, hv);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(a2_init);
+                // acc2 = X + A Wo^T = H.  Its bf16 values become the H tile in
+                // shared memory (the first projection's operand, laid out as a
+                // 128-byte-swizzled TMA load would) and give the norm's sum of
+                // squares; acc2 keeps H in fp32 for the second projection
+                if (!mbar_wait(o_done, tl & 1, a.wait, abort_flag)) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int c32 = 0; c32 < HALF / 32; ++c32) {
+                    const int col = hf * HALF + 32 * c32;
+                    uint32_t v[32];
+                    tmem_ld32(t_acc2 + lane_off + col, v);
+                    tmem_ld_wait();
+                    tmem_reg_fence(v);
+                    uint8_t *row = sH + (col / 64) * FF_SLAB + r * 128;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint32_t ow[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            ow[e] = pack_bf16x2(__uint_as_float(v[8 * i + 2 * e]), __uint_as_float(v[8 * i + 2 * e + 1]));
+                            const float lo = __uint_as_float(ow[e] << 16);
+                            const float hi = __uint_as_float(ow[e] & 0xFFFF0000u);
+                            ss = fmaf(lo, lo, ss);
+                            ss = fmaf(hi, hi, ss);
+                        }
+                        *reinterpret_cast<uint4 *>(row + ((((col % 64) / 8 + i) ^ (r & 7)) << 4)) =
+                            make_uint4(ow[0], ow[1], ow[2], ow[3]);
                     }
                 }
-                tmem_st32(t_acc2 + lane_off + col, hv);
-            }
-            tmem_st_wait();
-            // H read (generic proxy) before its buffer is refilled by TMA
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(a2_init);
-                mbar_arrive(h_free);
+                // generic writes, read next by the tensor core (async proxy)
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(hb_full);
+                    mbar_arrive(h_free);
+                }
+            } else {
+                if (!mbar_wait(h_full, tl & 1, a.wait, abort_flag)) break;
+                // This warp's half of its rows of H (columns hf*HALF ..): the
+                // RMSNorm partial sum of squares, and the values in fp32 into
+                // acc2, onto which the second projection accumulates (so the
+                // residual needs no read at the end).  acc2 is free: the previous
+                // tile's output was read out of it by these warps.  Chunk j of a
+                // slab row sits at 16-byte position j ^ (r & 7).
+#pragma unroll 1
+                for (int c32 = 0; c32 < HALF / 32; ++c32) {
+                    const int col = hf * HALF + 32 * c32;
+                    const uint8_t *row = sH + (col / 64) * FF_SLAB + r * 128;
+                    uint32_t hv[32];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(row + ((((col % 64) / 8 + i) ^ (r & 7)) << 4));
+                        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float lo = __uint_as_float(w4[e] << 16);
+                            const float hi = __uint_as_float(w4[e] & 0xFFFF0000u);
+                            ss = fmaf(lo, lo, ss);
+                            ss = fmaf(hi, hi, ss);
+                            hv[8 * i + 2 * e] = __float_as_uint(lo);
+                            hv[8 * i + 2 * e + 1] = __float_as_uint(hi);
+                        }
+                    }
+                    tmem_st32(t_acc2 + lane_off + col, hv);
+                }
+                tmem_st_wait();
+                // H read (generic proxy) before its buffer is refilled by TMA
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(a2_init);
+                    mbar_arrive(h_free);
+                }
             }
             s_ss[hf * FF_BM + r] = ss;
             named_bar_sync(1, 32 * FF_EPI_WARPS);
@@ -497,7 +605,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
 // tile count and tensor maps of one problem
 template <int D>
 static cudaError_t prepare_ffn(const FfnArgs &a, FfnParams &p, CUtensorMap *tmH, CUtensorMap *tmW1,
-                               CUtensorMap *tmW2, CUtensorMap *tmY)
+                               CUtensorMap *tmW2, CUtensorMap *tmY, CUtensorMap *tmWo)
 {
     p.a = a;
     p.grouped = a.G > 1 && a.h_map.Gs != 0;
@@ -544,26 +652,36 @@ static cudaError_t prepare_ffn(const FfnArgs &a, FfnParams &p, CUtensorMap *tmH,
         uint32_t box[3] = {64, static_cast<uint32_t>(D), 1};
         if (encode_tmap_3d(tmW2, 2, a.W2, dims, str, box)) return cudaErrorInvalidValue;
     }
+    if (a.fuse_o) {
+        // Wo [G][D out][D in]: boxes of 64 input columns x all D output rows
+        uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(D), static_cast<uint64_t>(a.G)};
+        uint64_t str[2] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(a.wo_gstride) * 2};
+        uint32_t box[3] = {64, static_cast<uint32_t>(D), 1};
+        if (encode_tmap_3d(tmWo, 2, a.Wo, dims, str, box)) return cudaErrorInvalidValue;
+    } else {
+        *tmWo = *tmW2; // unused
+    }
     return cudaSuccess;
 }
 
-template <int D>
+template <int D, bool FO>
 static cudaError_t launch_ffn_cfg(const FfnArgs &a, const FfnArgs *a1, cudaStream_t s)
 {
     using Sh = FfnShape<D>;
-    alignas(64) CUtensorMap tm[2][4];
+    alignas(64) CUtensorMap tm[2][5];
     FfnMulti P;
     memset(&P, 0, sizeof(P));
-    cudaError_t e = prepare_ffn<D>(a, P.q[0], &tm[0][0], &tm[0][1], &tm[0][2], &tm[0][3]);
+    cudaError_t e = prepare_ffn<D>(a, P.q[0], &tm[0][0], &tm[0][1], &tm[0][2], &tm[0][3], &tm[0][4]);
     if (e != cudaSuccess) return e;
     P.split = P.q[0].tiles;
     P.tiles = P.split;
     if (a1) {
-        if ((e = prepare_ffn<D>(*a1, P.q[1], &tm[1][0], &tm[1][1], &tm[1][2], &tm[1][3])) != cudaSuccess)
+        if ((e = prepare_ffn<D>(*a1, P.q[1], &tm[1][0], &tm[1][1], &tm[1][2], &tm[1][3], &tm[1][4])) !=
+            cudaSuccess)
             return e;
         P.tiles += P.q[1].tiles;
     } else {
-        for (int k = 0; k < 4; ++k) tm[1][k] = tm[0][k];
+        for (int k = 0; k < 5; ++k) tm[1][k] = tm[0][k];
     }
     static int num_sms = 0;
     if (num_sms == 0) {
@@ -573,27 +691,30 @@ static cudaError_t launch_ffn_cfg(const FfnArgs &a, const FfnArgs *a1, cudaStrea
             num_sms < 1)
             num_sms = 148;
     }
-    auto kern = ffn_tc_kernel<D>;
+    auto kern = ffn_tc_kernel<D, FO>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Sh::SMEM));
     if (e != cudaSuccess) return e;
     const long long grid = P.tiles < num_sms ? P.tiles : num_sms;
     return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(FF_THREADS), Sh::SMEM, s, tm[0][0],
-                      tm[0][1], tm[0][2], tm[0][3], tm[1][0], tm[1][1], tm[1][2], tm[1][3], P);
+                      tm[0][1], tm[0][2], tm[0][3], tm[1][0], tm[1][1], tm[1][2], tm[1][3], tm[0][4], tm[1][4],
+                      P);
 }
 
 bool ffn_tc_supported(int D, int F) { return (D == 128 || D == 256) && F % FF_BH1 == 0 && F >= FF_BH1; }
 
 static bool ffn_ok(const FfnArgs &a)
 {
-    return ffn_tc_supported(a.D, a.F) && a.M >= 1 && a.G >= 1 && a.h_map.P == 1 && a.y_map.P == 1;
+    return ffn_tc_supported(a.D, a.F) && a.M >= 1 && a.G >= 1 && a.h_map.P == 1 && a.y_map.P == 1 &&
+           (!a.fuse_o || (a.Wo && a.X && a.x_map.P >= 1));
 }
 
 cudaError_t launch_ffn_tc_multi(const FfnArgs &a, const FfnArgs *a1, cudaStream_t s)
 {
     if (!ffn_ok(a)) return cudaErrorInvalidValue;
-    if (a1 && (!ffn_ok(*a1) || a1->D != a.D || a1->F != a.F || a1->eps != a.eps)) return cudaErrorInvalidValue;
-    if (a.D == 256) return launch_ffn_cfg<256>(a, a1, s);
-    return launch_ffn_cfg<128>(a, a1, s);
+    if (a1 && (!ffn_ok(*a1) || a1->D != a.D || a1->F != a.F || a1->eps != a.eps || a1->fuse_o != a.fuse_o))
+        return cudaErrorInvalidValue;
+    if (a.fuse_o) return a.D == 256 ? launch_ffn_cfg<256, true>(a, a1, s) : launch_ffn_cfg<128, true>(a, a1, s);
+    return a.D == 256 ? launch_ffn_cfg<256, false>(a, a1, s) : launch_ffn_cfg<128, false>(a, a1, s);
 }
 
 cudaError_t launch_ffn_tc(const FfnArgs &a, cudaStream_t s) { return launch_ffn_tc_multi(a, nullptr, s); }

@@ -102,6 +102,11 @@ struct AttnArgs {
 //   Y[row_y(r, g)] = H[row_h(r, g)] + GELU(n(H) W1[g]^T) W2[g]^T,
 // n(H) = H * rsqrt(mean(H^2) + eps) (the RMSNorm gain folded into W1).
 // H / Y rows are D wide; W1 is [G][F][D], W2 is [G][D][F] (bf16).
+//
+// fuse_o: the attention's output projection and residual come first, in the
+// same kernel: H = X + A Wo[g]^T, with A (the attention output) read where H
+// is otherwise read (`H`, h_map), X the block input rows under x_map, Wo
+// [G][D][D]; the residual of the FFN is then H in fp32.
 struct FfnArgs {
     int M, G, D, F;
     const void *H;
@@ -114,6 +119,11 @@ struct FfnArgs {
     RowMap y_map;
     float eps;
     WaitCtl wait;
+    int fuse_o;
+    const void *Wo;
+    long long wo_gstride;   // elements between groups of Wo
+    const void *X;
+    RowMap x_map;
 };
 
 // Launch with programmatic stream serialization: the kernel may start while
