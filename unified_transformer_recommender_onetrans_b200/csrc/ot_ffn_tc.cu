@@ -466,6 +466,19 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                     mbar_arrive(hb_full);
                     mbar_arrive(h_free);
                 }
+                // this thread's X half-row of its next tile toward L2: its seed
+                // pass then waits for L2, not DRAM
+                const long long nt = tile + gridDim.x;
+                if (nt < P.tiles) {
+                    int g2, m2;
+                    const FfnArgs &pb = P.q[ffn_tile(P, nt, g2, m2)].a;
+                    const long long r2 = static_cast<long long>(m2) + r;
+                    if (r2 < pb.M) {
+                        const char *xr = reinterpret_cast<const char *>(
+                            static_cast<const __nv_bfloat16 *>(pb.X) + rowmap_apply(pb.x_map, r2, g2) * D + hf * HALF);
+                        for (int o = 0; o < HALF * 2; o += 128) prefetch_l2(xr + o);
+                    }
+                }
             } else {
                 if (!mbar_wait(h_full, tl & 1, a.wait, abort_flag)) break;
                 // This warp's half of its rows of H (columns hf*HALF ..): the
