@@ -271,7 +271,11 @@ typedef struct {
     int kind;      /* ot_kernel_kind */
     int role;      /* 0 S-QKV, 1 S-attn, 2 S-O, 3 S-FFN1, 4 S-FFN2, 5..9 the NS ones, 10 Auto-Split,
                       11 other, 12 S-FFN (fused), 13 NS-FFN (fused); 14 O, 15 FFN, 16 QKV:
-                      one launch for both sides of a layer in ot_full_forward */
+                      one launch for both sides of a layer in ot_full_forward.
+                      Where the FFN kernel runs (bf16, d of 128 or 256) it also
+                      does the output projection, so the S-O / NS-O / O roles
+                      appear only on the other paths (FP8, d = 384, kernel
+                      path 2) */
     float ms;      /* device time between the two events */
     double flops;  /* algorithmic floating-point operations */
     double bytes;  /* algorithmic HBM bytes */
