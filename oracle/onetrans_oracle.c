@@ -30,11 +30,24 @@
  * Storage: every input is passed as float32, which holds the bf16 / fp32
  * values of the runs exactly; all arithmetic is fp64 (double).
  *
- * FP8 mode (cfg->fp8 = 1): every input row of a QKV/O/W1/W2 projection is
- * quantised to e4m3 with its own scale s = amax(row)/448 (RNE, saturating at
- * 448, s = 1 for an all-zero row); every weight matrix is quantised the same
- * way with one scale per matrix; the product is computed in fp64 on the
- * quantised values and multiplied by both scales.  Attention stays unquantised.
+ * FP8 modes (the V2 podcast page names "kernel fusion + FP8" and nothing
+ * more; the workload fixes e4m3 with per-tensor fp32 scales):
+ *   fp8 = 2 (per-tensor): every projection input tensor -- the input of the
+ *     QKV, O, W1 or W2 projection of one layer and one parameter set (S, or
+ *     NS position n) -- has one fixed fp32 scale s from cfg->act_scale; each
+ *     value is quantised as e4m3(x / s), round to nearest even, saturating
+ *     at +-448.  A calibrated scale does not depend on the batch, so a
+ *     candidate's result stays independent of the other candidates.
+ *   fp8 = 1 (per-row, the calibration pass): every input row gets its own
+ *     scale s = amax(row)/448 (s = 1 for an all-zero row).
+ *   In both modes every weight matrix is quantised with one scale
+ *   amax(W)/448, the product is computed in fp64 on the quantised values and
+ *   multiplied by both scales, and attention stays unquantised.
+ *   cfg->act_amax, if not NULL, receives max |x| over every row that entered
+ *   each projection input tensor (max-accumulated): the per-tensor amax a
+ *   calibration turns into scales amax/448.
+ *   Layout of act_scale / act_amax: [layer][set][4], set 0 = S, 1 + n = NS
+ *   position n; the 4 inputs in the order QKV, O, W1, W2.
  *
  * Layouts (row-major):
  *   Wqkv [3d][d] (rows Q | K | V), Wo [d][d], W1 [ffn][d], W2 [d][ffn],
@@ -56,8 +69,12 @@ typedef struct {
     int layers, d, heads, ffn, n_ns, L0;
     int q[ORC_MAX_LAYERS]; /* query tail per layer; L_{l+1} = q[l] */
     double eps;
-    int fp8;
+    int fp8;                  /* 0 off, 1 per-row scales, 2 per-tensor scales */
+    const double *act_scale;  /* fp8 == 2: [layers][1 + n_ns][4] */
+    double *act_amax;         /* optional, same layout: max |input| seen */
 } orc_cfg;
+
+enum { ORC_IN_QKV = 0, ORC_IN_O = 1, ORC_IN_W1 = 2, ORC_IN_W2 = 3 };
 
 typedef struct {
     const float *Wqkv_s, *Wo_s, *W1_s, *W2_s, *g1_s, *g2_s;
@@ -94,23 +111,28 @@ static double quantise_block(const double *x, long n, double *xq)
     return s;
 }
 
-/* A weight matrix as the projections read it: plain, or quantised + scale. */
+/* A weight matrix as the projections read it: plain, or quantised + scale,
+ * with the quantisation rule of its input tensor. */
 typedef struct {
     const float *w; /* [out][in] */
     double *wq;     /* quantised copy (fp8 mode) */
     double s;
     int out, in;
+    int fp8;        /* input rule: 0 none, 1 per-row scale, 2 per-tensor scale xs */
+    double xs;      /* per-tensor input scale (fp8 == 2) */
+    double *amax;   /* if not NULL: max |input| of this tensor, accumulated */
 } mat_t;
 
 static mat_t mat_plain(const float *w, int out, int in)
 {
-    mat_t m = {w, NULL, 1.0, out, in};
+    mat_t m = {w, NULL, 1.0, out, in, 0, 1.0, NULL};
     return m;
 }
 
 static mat_t mat_make(const float *w, int out, int in, int fp8)
 {
     mat_t m = mat_plain(w, out, in);
+    m.fp8 = fp8;
     if (fp8) {
         long n = (long)out * in;
         double *tmp = (double *)malloc(sizeof(double) * n);
@@ -124,12 +146,34 @@ static mat_t mat_make(const float *w, int out, int in, int fp8)
 
 static void mat_free(mat_t *m) { free(m->wq); m->wq = NULL; }
 
+/* Record max |x| of one input row into the tensor's amax slot. */
+static void record_amax(const mat_t *m, const double *x)
+{
+    if (!m->amax) return;
+    double a = 0.0;
+    for (int k = 0; k < m->in; ++k) if (fabs(x[k]) > a) a = fabs(x[k]);
+#pragma omp critical(orc_amax)
+    {
+        if (a > *m->amax) *m->amax = a;
+    }
+}
+
+/* Quantise one input row by the matrix's input rule; returns its scale. */
+static double quantise_input(const mat_t *m, const double *x, double *xq)
+{
+    if (m->fp8 == 1) return quantise_block(x, m->in, xq);
+    for (int k = 0; k < m->in; ++k) xq[k] = e4m3_round(x[k] / m->xs);
+    return m->xs;
+}
+
 /* y[o] = sum_k W[o][k] x[k] for o in [o0, o0+nout).  In fp8 mode the input
- * row x (the whole projection input, all `in` values) is quantised with its
- * own scale first.  xq is scratch of `in` doubles. */
+ * row x (the whole projection input, all `in` values) is quantised first,
+ * with its own scale (per-row) or the tensor's (per-tensor).  xq is scratch
+ * of `in` doubles. */
 static void project(const mat_t *m, const double *x, int o0, int nout, double *y, double *xq)
 {
     int in = m->in;
+    record_amax(m, x);
     if (!m->wq) {
         for (int o = 0; o < nout; ++o) {
             const float *row = m->w + (long)(o0 + o) * in;
@@ -139,7 +183,7 @@ static void project(const mat_t *m, const double *x, int o0, int nout, double *y
         }
         return;
     }
-    double sx = quantise_block(x, in, xq);
+    double sx = quantise_input(m, x, xq);
     for (int o = 0; o < nout; ++o) {
         const double *row = m->wq + (long)(o0 + o) * in;
         double acc = 0.0;
@@ -193,8 +237,17 @@ typedef struct {
     const float *g1, *g2;
 } pset_t;
 
-static pset_t pset_make(const orc_cfg *c, const float *Wqkv, const float *Wo, const float *W1,
-                        const float *W2, const float *g1, const float *g2)
+/* Attach the input rule of tensor (layer l, set, input t) to a matrix. */
+static void mat_input(const orc_cfg *c, mat_t *m, int l, int set, int t)
+{
+    long slot = ((long)l * (1 + c->n_ns) + set) * 4 + t;
+    if (c->fp8 == 2) m->xs = c->act_scale[slot];
+    if (c->act_amax) m->amax = c->act_amax + slot;
+}
+
+/* Parameter set `set` (0 = S, 1 + n = NS position n) of layer l. */
+static pset_t pset_make(const orc_cfg *c, int l, int set, const float *Wqkv, const float *Wo,
+                        const float *W1, const float *W2, const float *g1, const float *g2)
 {
     int d = c->d, f = c->ffn;
     pset_t p;
@@ -202,6 +255,10 @@ static pset_t pset_make(const orc_cfg *c, const float *Wqkv, const float *Wo, co
     p.o = mat_make(Wo, d, d, c->fp8);
     p.w1 = mat_make(W1, f, d, c->fp8);
     p.w2 = mat_make(W2, d, f, c->fp8);
+    mat_input(c, &p.qkv, l, set, ORC_IN_QKV);
+    mat_input(c, &p.o, l, set, ORC_IN_O);
+    mat_input(c, &p.w1, l, set, ORC_IN_W1);
+    mat_input(c, &p.w2, l, set, ORC_IN_W2);
     p.g1 = g1;
     p.g2 = g2;
     return p;
@@ -215,14 +272,14 @@ static void pset_free(pset_t *p)
 static pset_t s_params(const orc_cfg *c, const orc_weights *w, int l)
 {
     long d = c->d, f = c->ffn;
-    return pset_make(c, w->Wqkv_s + l * 3 * d * d, w->Wo_s + l * d * d, w->W1_s + l * f * d,
+    return pset_make(c, l, 0, w->Wqkv_s + l * 3 * d * d, w->Wo_s + l * d * d, w->W1_s + l * f * d,
                      w->W2_s + l * d * f, w->g1_s + l * d, w->g2_s + l * d);
 }
 
 static pset_t ns_params(const orc_cfg *c, const orc_weights *w, int l, int n)
 {
     long d = c->d, f = c->ffn, ln = (long)l * c->n_ns + n;
-    return pset_make(c, w->Wqkv_ns + ln * 3 * d * d, w->Wo_ns + ln * d * d, w->W1_ns + ln * f * d,
+    return pset_make(c, l, 1 + n, w->Wqkv_ns + ln * 3 * d * d, w->Wo_ns + ln * d * d, w->W1_ns + ln * f * d,
                      w->W2_ns + ln * d * f, w->g1_ns + ln * d, w->g2_ns + ln * d);
 }
 
@@ -255,8 +312,13 @@ long orc_kv_user_elems(const orc_cfg *c) { return orc_kv_layer_offset(c, c->laye
 static int check_cfg(const orc_cfg *c)
 {
     if (c->layers < 1 || c->layers > ORC_MAX_LAYERS || c->d < 1 || c->heads < 1 ||
-        c->d % c->heads || c->ffn < 1 || c->n_ns < 0 || c->L0 < 1)
+        c->d % c->heads || c->ffn < 1 || c->n_ns < 0 || c->L0 < 1 || c->fp8 < 0 || c->fp8 > 2)
         return 1;
+    if (c->fp8 == 2) {
+        if (!c->act_scale) return 1;
+        for (long i = 0; i < (long)c->layers * (1 + c->n_ns) * 4; ++i)
+            if (!(c->act_scale[i] > 0.0)) return 1;
+    }
     int L = c->L0;
     for (int l = 0; l < c->layers; ++l) {
         if (c->q[l] < 1 || c->q[l] > L) return 1;
@@ -550,6 +612,26 @@ int orc_full_forward_joint(const orc_cfg *c, const orc_weights *w, const float *
         memcpy(ns_out + uc * (long)N * d, X + (long)qlast * d, sizeof(double) * (long)N * d);
         free(X);
     }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* One projection of `rows` input rows under an FP8 rule, exactly as the      */
+/* block's projections run it (fp8 0 / 1 / 2 as in the config; xs is the     */
+/* per-tensor scale of rule 2; amax, if not NULL, accumulates max |x|).      */
+/* x [rows][in], W [out][in] -> y [rows][out].                                */
+int orc_project_rows(const double *x, long rows, int in, const float *W, int out, int fp8,
+                     double xs, double *amax, double *y)
+{
+    if (rows < 0 || in < 1 || out < 1 || fp8 < 0 || fp8 > 2 || (fp8 == 2 && !(xs > 0.0)))
+        return 1;
+    mat_t m = mat_make(W, out, in, fp8);
+    m.xs = xs;
+    m.amax = amax;
+    double *xq = (double *)malloc(sizeof(double) * in);
+    for (long r = 0; r < rows; ++r) project(&m, x + r * in, 0, out, y + r * out, xq);
+    free(xq);
+    mat_free(&m);
     return 0;
 }
 

@@ -25,7 +25,15 @@ MAX_LAYERS = 64
 class _Cfg(C.Structure):
     _fields_ = [("layers", C.c_int), ("d", C.c_int), ("heads", C.c_int), ("ffn", C.c_int),
                 ("n_ns", C.c_int), ("L0", C.c_int), ("q", C.c_int * MAX_LAYERS),
-                ("eps", C.c_double), ("fp8", C.c_int)]
+                ("eps", C.c_double), ("fp8", C.c_int), ("act_scale", C.POINTER(C.c_double)),
+                ("act_amax", C.POINTER(C.c_double))]
+
+
+# FP8 rules of the projection inputs (see onetrans_oracle.c): off, one scale
+# per input row (the calibration pass), one fixed scale per input tensor.
+FP8_OFF, FP8_ROW, FP8_TENSOR = 0, 1, 2
+# the four projection inputs of a parameter set, in the act_scale layout
+INPUTS = ("qkv", "o", "w1", "w2")
 
 
 _WNAMES = ("Wqkv_s", "Wo_s", "W1_s", "W2_s", "g1_s", "g2_s",
@@ -58,6 +66,8 @@ def lib():
         L.orc_kv_user_elems.restype = C.c_long
         L.orc_kv_layer_offset.argtypes = [C.POINTER(_Cfg), C.c_int]
         L.orc_kv_layer_offset.restype = C.c_long
+        L.orc_project_rows.argtypes = [dp, C.c_long, C.c_int, fp, C.c_int, C.c_int, C.c_double,
+                                       dp, dp]
         L.orc_e4m3_round.argtypes = [C.c_double]
         L.orc_e4m3_round.restype = C.c_double
         L.orc_set_threads.argtypes = [C.c_int]
@@ -90,6 +100,9 @@ def pyramid_schedule(L0: int, q_end: int | None, layers: int) -> list[int]:
 
 @dataclass
 class Config:
+    """Block-stack shape.  ``fp8``: FP8_OFF (also False), FP8_ROW (also True)
+    or FP8_TENSOR, which needs ``act_scale`` [layers][1 + n_ns][4] (set 0 =
+    S, 1 + n = NS position n; inputs of QKV, O, W1, W2)."""
     layers: int
     d: int
     heads: int
@@ -98,25 +111,44 @@ class Config:
     L0: int
     q: list = field(default_factory=list)
     eps: float = 1e-6
-    fp8: bool = False
+    fp8: int = FP8_OFF
+    act_scale: object = None
 
     @staticmethod
-    def of(wl, q=None, fp8=None) -> "Config":
+    def of(wl, q=None, fp8=None, act_scale=None) -> "Config":
         q = pyramid_schedule(wl.L0, wl.q_end, wl.layers) if q is None else list(q)
-        return Config(wl.layers, wl.d, wl.heads, wl.ffn, wl.n_ns, wl.L0, q, wl.eps,
-                      (wl.dtype == "fp8") if fp8 is None else fp8)
+        if fp8 is None:
+            fp8 = FP8_TENSOR if act_scale is not None else (
+                FP8_ROW if wl.dtype == "fp8" else FP8_OFF)
+        return Config(wl.layers, wl.d, wl.heads, wl.ffn, wl.n_ns, wl.L0, q, wl.eps, fp8,
+                      act_scale)
+
+    def scale_shape(self) -> tuple:
+        return (self.layers, 1 + self.n_ns, 4)
 
     def rows_at(self, l: int) -> int:
         return self.L0 if l == 0 else self.q[l - 1]
 
-    def _c(self) -> _Cfg:
+    def _c(self, amax=None) -> _Cfg:
+        """The C struct; ``amax`` (float64 [layers][1 + n_ns][4], C order) is
+        max-accumulated by the call it is passed to."""
         c = _Cfg()
         c.layers, c.d, c.heads, c.ffn, c.n_ns, c.L0 = (self.layers, self.d, self.heads, self.ffn,
                                                       self.n_ns, self.L0)
         for i, v in enumerate(self.q):
             c.q[i] = int(v)
         c.eps = float(self.eps)
-        c.fp8 = int(bool(self.fp8))
+        c.fp8 = int(self.fp8)
+        if self.fp8 == FP8_TENSOR:
+            if self.act_scale is None:
+                raise ValueError("per-tensor FP8 needs act_scale")
+            self._scale = np.ascontiguousarray(self.act_scale, dtype=np.float64)
+            assert self._scale.shape == self.scale_shape(), self._scale.shape
+            c.act_scale = _dptr(self._scale)
+        if amax is not None:
+            assert amax.shape == self.scale_shape() and amax.dtype == np.float64
+            assert amax.flags.c_contiguous
+            c.act_amax = _dptr(amax)
         return c
 
     def grown(self, delta: int) -> "Config":
@@ -124,7 +156,7 @@ class Config:
         query tail longer by delta (pyramid windows anchored at their first
         row)."""
         return Config(self.layers, self.d, self.heads, self.ffn, self.n_ns, self.L0 + delta,
-                      [v + delta for v in self.q], self.eps, self.fp8)
+                      [v + delta for v in self.q], self.eps, self.fp8, self.act_scale)
 
     def kv_user_elems(self) -> int:
         return int(lib().orc_kv_user_elems(C.byref(self._c())))
@@ -173,15 +205,17 @@ def kv_layer(cfg: Config, kv_user: np.ndarray, l: int):
     return K, V
 
 
-def encode_user(cfg: Config, w, S):
-    """S [U, L0, d] -> (kv [U, kv_user_elems], s_out [U, q_last, d])."""
+def encode_user(cfg: Config, w, S, amax=None):
+    """S [U, L0, d] -> (kv [U, kv_user_elems], s_out [U, q_last, d]).
+    ``amax``: optional float64 array of cfg.scale_shape(), max-accumulated
+    with every projection input's max |x| (calibration)."""
     S = _f32(S)
     U = S.shape[0]
     assert S.shape == (U, cfg.L0, cfg.d), S.shape
     W = _weights(w)
     kv = np.zeros((U, cfg.kv_user_elems()))
     s_out = np.zeros((U, cfg.q[-1], cfg.d))
-    rc = lib().orc_encode_user(C.byref(cfg._c()), C.byref(W.c), _fptr(S), U, _dptr(kv),
+    rc = lib().orc_encode_user(C.byref(cfg._c(amax)), C.byref(W.c), _fptr(S), U, _dptr(kv),
                                _dptr(s_out))
     if rc:
         raise ValueError("oracle rejected the configuration")
@@ -208,14 +242,15 @@ def encode_append(cfg: Config, w, kv_old, S_new):
     return kv, out
 
 
-def score_candidates(cfg: Config, w, kv, ns):
-    """kv [U, kv_user_elems], ns [U, C, N, d] -> ns_out [U, C, N, d]."""
+def score_candidates(cfg: Config, w, kv, ns, amax=None):
+    """kv [U, kv_user_elems], ns [U, C, N, d] -> ns_out [U, C, N, d].
+    ``amax`` as for encode_user."""
     kv, ns = _f64(kv), _f64(ns)
     U, Cn = ns.shape[0], ns.shape[1]
     assert ns.shape == (U, Cn, cfg.n_ns, cfg.d) and kv.shape == (U, cfg.kv_user_elems())
     W = _weights(w)
     out = np.zeros_like(ns)
-    rc = lib().orc_score_candidates(C.byref(cfg._c()), C.byref(W.c), _dptr(kv), U, _dptr(ns),
+    rc = lib().orc_score_candidates(C.byref(cfg._c(amax)), C.byref(W.c), _dptr(kv), U, _dptr(ns),
                                     Cn, _dptr(out))
     if rc:
         raise ValueError("oracle rejected the configuration")
@@ -263,6 +298,43 @@ def embed_gather(table, ids):
 
 def e4m3_round(v: float) -> float:
     return float(lib().orc_e4m3_round(float(v)))
+
+
+def project_rows(x, W, fp8=FP8_OFF, xs=1.0, amax=None):
+    """One projection y = x W^T of rows x [R, in] by W [out, in] under an FP8
+    rule, through the same code the block's projections use (weights
+    quantised with one scale amax(W)/448; inputs per row or with the
+    per-tensor scale xs).  ``amax``: optional float64 [1] accumulator."""
+    x = _f64(np.atleast_2d(_f64(x)))
+    Wf = _f32(W)
+    R, k = x.shape
+    assert Wf.shape[1] == k
+    y = np.zeros((R, Wf.shape[0]))
+    am = None
+    if amax is not None:
+        assert amax.dtype == np.float64 and amax.size == 1
+        am = _dptr(amax)
+    rc = lib().orc_project_rows(_dptr(x), R, k, _fptr(Wf), Wf.shape[0], int(fp8), float(xs), am,
+                                _dptr(y))
+    if rc:
+        raise ValueError("oracle rejected the projection")
+    return y
+
+
+def calibrate(cfg: Config, w, S, ns):
+    """Per-tensor FP8 scales from a calibration sample: the encode of users S
+    and the scoring of their candidates ns with per-row FP8 scales, recording
+    each projection input's max |x|; scale = amax / 448 (1 where amax is 0).
+    Returns (scales, amax), each [layers][1 + n_ns][4]."""
+    c1 = Config(cfg.layers, cfg.d, cfg.heads, cfg.ffn, cfg.n_ns, cfg.L0, list(cfg.q), cfg.eps,
+                FP8_ROW)
+    amax = np.zeros(c1.scale_shape())
+    W = _weights(w)
+    kv, _ = encode_user(c1, W, S, amax=amax)
+    score_candidates(c1, W, kv, ns, amax=amax)
+    # the scales as the GPU holds them (fp32), so both sides quantise alike
+    scales = np.where(amax > 0, amax / 448.0, 1.0).astype(np.float32).astype(np.float64)
+    return scales, amax
 
 
 def full_forward(cfg: Config, w, S, ns):

@@ -10,7 +10,10 @@
 * the invariants the pages' design rests on: causality, pyramid
   consistency, KV-cache equivalence, candidate independence, S-side
   independence from NS input;
-* e4m3 rounding against torch's float8_e4m3fn cast;
+* e4m3 rounding against torch's float8_e4m3fn cast; both FP8 rules (per-row
+  and per-tensor scales) against the brute force, exact results on
+  representable operands, a hand-worked row, the scale granularity and the
+  calibration amax;
 * Auto-Split and embedding gather against numpy.
 """
 
@@ -31,8 +34,8 @@ from oracle import oracle as O
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
-def cfg_of(layers, d, heads, ffn, N, L0, q, eps=1e-6, fp8=False):
-    return O.Config(layers, d, heads, ffn, N, L0, list(q), eps, fp8)
+def cfg_of(layers, d, heads, ffn, N, L0, q, eps=1e-6, fp8=O.FP8_OFF, act_scale=None):
+    return O.Config(layers, d, heads, ffn, N, L0, list(q), eps, fp8, act_scale)
 
 
 TINY_CASES = [
@@ -363,21 +366,167 @@ def test_e4m3_round_matches_torch_cast():
 
 
 def test_fp8_mode_quantises_and_stays_close():
-    """FP8 mode really quantises (results move) and stays inside the format's
-    bound: e4m3 keeps 3 mantissa bits, so each operand carries at most 2^-4
-    relative rounding error and a product of two at most about 2 * 2^-4."""
+    """Both FP8 rules really quantise (results move) and stay inside the
+    format's bound: e4m3 keeps 3 mantissa bits, so each operand carries at
+    most 2^-4 relative rounding error and a product of two at most about
+    2 * 2^-4."""
     layers, d, H, f, N, L0, q = _small()
     w = rand_weights(layers, d, f, N, seed=95)
     S, ns = rand_inputs(1, 2, L0, N, d, seed=96)
     c64 = cfg_of(layers, d, H, f, N, L0, q)
-    c8 = cfg_of(layers, d, H, f, N, L0, q, fp8=True)
     kv, s = O.encode_user(c64, w, S)
-    kv8, s8 = O.encode_user(c8, w, S)
     n64 = O.score_candidates(c64, w, kv, ns)
-    n8 = O.score_candidates(c8, w, kv8, ns)
-    for a, b in ((s8, s), (kv8, kv), (n8, n64)):
-        err = O.rel_l2(a, b)
-        assert 1e-4 < err < 2 * 2.0 ** -4, err
+    scales, _ = O.calibrate(c64, w, S, ns)
+    for c8 in (cfg_of(layers, d, H, f, N, L0, q, fp8=O.FP8_ROW),
+               cfg_of(layers, d, H, f, N, L0, q, fp8=O.FP8_TENSOR, act_scale=scales)):
+        kv8, s8 = O.encode_user(c8, w, S)
+        n8 = O.score_candidates(c8, w, kv8, ns)
+        for a, b in ((s8, s), (kv8, kv), (n8, n64)):
+            err = O.rel_l2(a, b)
+            assert 1e-4 < err < 2 * 2.0 ** -4, err
+
+
+def _fp8_scales(cfg, seed, lo=0.002, hi=0.01):
+    """Seeded per-tensor scales small enough that the larger inputs saturate."""
+    g = torch.Generator().manual_seed(seed)
+    return (lo + (hi - lo) * torch.rand(cfg.scale_shape(), generator=g)).double().numpy()
+
+
+@pytest.mark.parametrize("case", TINY_CASES[1:4])
+@pytest.mark.parametrize("rule", [O.FP8_ROW, O.FP8_TENSOR], ids=["per_row", "per_tensor"])
+def test_brute_force_matches_oracle_fp8(case, rule):
+    """Both FP8 rules against the brute-force token loop, whose e4m3 rounding
+    is torch's float8_e4m3fn cast: outputs, every layer's K / V, and the
+    calibration amax of every projection input tensor."""
+    from brute_force import Fp8
+    layers, d, H, f, N, L0, q, U, Cn = case
+    w = rand_weights(layers, d, f, N, seed=L0 + d + 1)
+    S, ns = rand_inputs(U, Cn, L0, N, d, seed=7 * L0 + N + 1)
+    cfg = cfg_of(layers, d, H, f, N, L0, q, fp8=rule)
+    if rule == O.FP8_TENSOR:
+        cfg.act_scale = _fp8_scales(cfg, seed=L0)
+    amax = np.zeros(cfg.scale_shape())
+    kv, s_out = O.encode_user(cfg, w, S, amax=amax)
+    ns_out = O.score_candidates(cfg, w, kv, ns, amax=amax)
+    wl = to_lists(w)
+    bam = np.zeros(cfg.scale_shape()).tolist()
+    st = Fp8(rule, None if cfg.act_scale is None else cfg.act_scale.tolist(), bam)
+    for u in range(U):
+        for c in range(Cn):
+            bs, bns, bkv = run_candidate(wl, S[u].double().tolist(), ns[u, c].double().tolist(),
+                                         q, H, 1e-6, fp8=st)
+            np.testing.assert_allclose(s_out[u], np.array(bs), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(ns_out[u, c], np.array(bns), rtol=0, atol=1e-12)
+            for l, (K, V) in enumerate(bkv):
+                Ko, Vo = O.kv_layer(cfg, kv[u], l)
+                np.testing.assert_allclose(Ko, np.array(K), rtol=0, atol=1e-12)
+                np.testing.assert_allclose(Vo, np.array(V), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(amax, np.array(bam), rtol=0, atol=1e-12)
+    assert np.all(amax > 0)
+
+
+def _e4m3_grid(g, shape, exp2):
+    """Random e4m3 values times 2^exp2, each row holding one +-448 entry."""
+    codes = torch.randint(0, 256, shape, generator=g, dtype=torch.uint8).view(torch.float8_e4m3fn)
+    v = codes.double()
+    v[~torch.isfinite(v)] = 0.0
+    v[:, 0] = 448.0 * torch.where(torch.rand(shape[0], generator=g) < 0.5, 1.0, -1.0).double()
+    return (v * 2.0 ** exp2).numpy()
+
+
+def test_fp8_exact_when_operands_are_representable():
+    """Inputs that are e4m3 values times the scale, weights likewise: both
+    rules must then reproduce the fp64 product bit for bit (every operand is
+    exact in e4m3 and every sum is exact in fp64)."""
+    g = torch.Generator().manual_seed(11)
+    x = _e4m3_grid(g, (9, 32), -3)       # per-row amax 448 * 2^-3: scale 2^-3
+    W = _e4m3_grid(g, (24, 32), -5)      # amax 448 * 2^-5: scale 2^-5
+    exact = x @ W.T
+    for rule in (O.FP8_ROW, O.FP8_TENSOR):
+        y = O.project_rows(x, W, fp8=rule, xs=2.0 ** -3)
+        assert np.array_equal(y, exact), rule
+    assert np.array_equal(O.project_rows(x, W), exact)
+
+
+def test_fp8_scale_constant_hand_worked():
+    """One row through an identity weight (exact in e4m3 after its scale
+    1/448): per row, y = e4m3(x / (amax/448)) * amax/448 with torch's cast;
+    per tensor with scale 0.01, the values above 4.48 saturate at 4.48."""
+    x = np.array([[0.3, -1.7, 2.9, 0.01, 5.5, -5.25, 1e-3, 0.0]])
+    W = np.eye(8)
+    s = 5.5 / 448.0
+    want = (torch.tensor(x / s).float().to(torch.float8_e4m3fn).double() * s).numpy()
+    # (the scale products are rounded in another order: equal to the last bits)
+    np.testing.assert_allclose(O.project_rows(x, W, fp8=O.FP8_ROW), want, rtol=1e-15, atol=0)
+    assert not np.allclose(want, x, rtol=1e-3)   # it did quantise
+    xs = 0.01
+    q = torch.tensor(x / xs).clamp(-448, 448).float().to(torch.float8_e4m3fn).double()
+    want2 = (q * xs).numpy()
+    np.testing.assert_allclose(O.project_rows(x, W, fp8=O.FP8_TENSOR, xs=xs), want2, rtol=1e-15,
+                               atol=0)
+    assert want2[0, 4] == pytest.approx(4.48) and want2[0, 5] == pytest.approx(-4.48)
+
+
+def test_fp8_scale_granularity():
+    """Per row: scaling one row by 2 scales exactly its own output by 2 and
+    leaves the other rows alone.  Per tensor: the other rows are unchanged
+    too, but the scaled row is quantised on the tensor's fixed grid, so its
+    output is not three times the old one when the row is scaled by 3."""
+    g = torch.Generator().manual_seed(12)
+    x = torch.randn(6, 40, generator=g).double().numpy()
+    W = (torch.randn(16, 40, generator=g) / 6).numpy()
+    y = O.project_rows(x, W, fp8=O.FP8_ROW)
+    x2 = x.copy()
+    x2[3] *= 2.0
+    y2 = O.project_rows(x2, W, fp8=O.FP8_ROW)
+    assert np.array_equal(np.delete(y2, 3, 0), np.delete(y, 3, 0))
+    assert np.array_equal(y2[3], 2.0 * y[3])
+    xs = 0.02
+    t = O.project_rows(x, W, fp8=O.FP8_TENSOR, xs=xs)
+    x3 = x.copy()
+    x3[3] *= 3.0
+    t3 = O.project_rows(x3, W, fp8=O.FP8_TENSOR, xs=xs)
+    assert np.array_equal(np.delete(t3, 3, 0), np.delete(t, 3, 0))
+    assert not np.allclose(t3[3], 3.0 * t[3], rtol=1e-4, atol=0)
+    # the same projection with per-row scales gives 3x exactly up to fp64 rounding
+    r3 = O.project_rows(x3, W, fp8=O.FP8_ROW)
+    np.testing.assert_allclose(r3[3], 3.0 * y[3], rtol=1e-14, atol=1e-14)
+    # amax accumulates max |x| over all rows of the tensor
+    am = np.zeros(1)
+    O.project_rows(x3, W, fp8=O.FP8_TENSOR, xs=xs, amax=am)
+    assert am[0] == np.abs(x3).max()
+
+
+def test_fp8_calibration_amax_of_first_projection():
+    """The calibration's amax slot of layer 0's QKV input is max |RMSNorm(x)
+    * g| over the rows that entered it: torch's rms_norm over the S rows (S
+    set) and over each NS position's rows of every candidate (NS sets)."""
+    layers, d, H, f, N, L0, q = _small()
+    w = rand_weights(layers, d, f, N, seed=97)
+    S, ns = rand_inputs(2, 3, L0, N, d, seed=98)
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    scales, amax = O.calibrate(cfg, w, S, ns)
+    want_s = Fnn.rms_norm(S.double(), (d,), weight=w["g1_s"][0].double(), eps=1e-6).abs().max()
+    assert amax[0, 0, 0] == pytest.approx(float(want_s), rel=1e-12)
+    for n in range(N):
+        xn = Fnn.rms_norm(ns[:, :, n].double(), (d,), weight=w["g1_ns"][0, n].double(), eps=1e-6)
+        assert amax[0, 1 + n, 0] == pytest.approx(float(xn.abs().max()), rel=1e-12)
+    np.testing.assert_allclose(scales, np.float32(amax / 448.0), rtol=0, atol=0)
+
+
+def test_fp8_per_tensor_candidate_independence():
+    """Fixed per-tensor scales keep a candidate's result independent of the
+    other candidates in the call."""
+    layers, d, H, f, N, L0, q = _small()
+    w = rand_weights(layers, d, f, N, seed=99)
+    S, ns = rand_inputs(1, 4, L0, N, d, seed=100)
+    cfg = cfg_of(layers, d, H, f, N, L0, q, fp8=O.FP8_TENSOR)
+    cfg.act_scale = _fp8_scales(cfg, seed=3)
+    kv, _ = O.encode_user(cfg, w, S)
+    batch = O.score_candidates(cfg, w, kv, ns)
+    for c in range(4):
+        alone = O.score_candidates(cfg, w, kv, ns[:, c:c + 1])
+        assert np.array_equal(alone[:, 0], batch[:, c])
 
 
 def test_auto_split_matches_numpy():
