@@ -25,14 +25,16 @@
  *     during the call.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls are asynchronous on it; nothing synchronises except
- *     ot_model_create, ot_model_destroy and ot_poll_device_error.
+ *     ot_model_create, ot_model_destroy, ot_set_act_scales and
+ *     ot_poll_device_error.
  *   - Arguments are checked on the host before anything is launched; a
  *     failed check returns its status and launches nothing.
  *   - Device-side failures (a bounded wait that expired, a failed index
  *     check) set the model's device error word instead of trapping; read it
  *     with ot_poll_device_error.
  *   - No C++ exception crosses this ABI.  The only allocations are made by
- *     ot_model_create (weights and the error word); hot calls never allocate.
+ *     ot_model_create (weights and the error word) and the first
+ *     ot_set_act_scales (the scale array); hot calls never allocate.
  *   - A model may be used from several streams at once if every concurrent
  *     call has its own workspace and output buffers.
  *
@@ -41,12 +43,19 @@
  * accumulation on tcgen05 tensor cores); OT_DTYPE_FP8 = bfloat16 storage with
  * every QKV / O / FFN projection run on e4m3 operands, attention and cache in
  * bf16.  FP8 rule (the V2 podcast page names "kernel fusion + FP8" without a
- * recipe; this is the library's reading): each projection input row, after
- * its RMSNorm and gain where the block has one, is quantised with its own
- * scale s = amax(row) / 448 (s = 1 for an all-zero row), round to nearest
- * even, saturating; each weight matrix (one layer's Wqkv, Wo, W1 or W2, per
- * NS position for the private sets) has one scale; the fp32 product is
- * multiplied by both scales.  Auto-Split stays bf16.
+ * recipe; e4m3 with per-tensor fp32 scales is the library's reading): every
+ * projection input tensor -- the input of one layer's QKV, O, W1 or W2
+ * projection for one parameter set (S, or NS position n), after its RMSNorm
+ * and gain where the block has one -- has one fixed fp32 scale s, set with
+ * ot_set_act_scales from a calibration (ot_fp8_calibrate); each value is
+ * quantised to e4m3(x / s), round to nearest even, saturating at +-448.
+ * Each weight matrix (one layer's Wqkv, Wo, W1 or W2, per NS position for
+ * the private sets) has one scale amax(W) / 448; the fp32 product is
+ * multiplied by both scales.  Until scales are set, and during calibration,
+ * each input row is quantised with its own scale amax(row) / 448 (s = 1 for
+ * an all-zero row).  Fixed scales do not depend on the batch, so a
+ * candidate's result never depends on the other candidates.  Auto-Split
+ * stays bf16.
  */
 #ifndef ONETRANS_H
 #define ONETRANS_H
@@ -138,7 +147,12 @@ ot_status ot_auto_split(ot_model *m, const void *x, long M, void *ns, void *stre
 ot_status ot_embed_gather(const void *table, long rows, int d, const int64_t *ids, long n,
                           void *out, int32_t *err_word, void *stream);
 
-/* Encode U users (S-side, once per user): S device [U][L0][d] ->
+/* Encode U users (S-side, once per user; summary page, pyramid / KV-cache
+ * paragraph: candidates of one request share the user sequence, so the
+ * S-side runs once; blog page, "Cross-Request KV Caching").  Every layer l:
+ * RMSNorm + shared QKV over its L_l S rows, K / V stored in the cache, causal
+ * attention of the q_l tail rows, O, FFN (summary page, block paragraph).
+ * S device [U][L0][d] ->
  * kv_cache device (ot_kv_cache_bytes(m, U) bytes) and, if out_s_tail is not
  * NULL, the last layer's S rows device [U][q_last][d].
  * ws: device workspace of ws_bytes >= ot_workspace_bytes(m, U, 0). */
@@ -175,7 +189,10 @@ ot_status ot_encode_append(ot_model *m, const void *kv_old, int U, const void *S
  * each: the encode buffers for users * delta rows. */
 size_t ot_append_workspace_bytes(const ot_model *m, int users, int delta);
 
-/* Score C candidates per user against the users' cached S K/V (NS-side):
+/* Score C candidates per user against the users' cached S K/V (NS-side;
+ * summary page, pyramid / KV-cache paragraph: the NS-side runs per
+ * candidate; block paragraph: NS token n has private weights and sees every
+ * S token of the layer and NS tokens 0..n of its own candidate):
  * ns device [U][C][N][d] -> out_ns device [U][C][N][d].  kv_cache as written
  * by ot_encode_user for the same U users.  ws >= ot_workspace_bytes(m, U, C).
  * A candidate's result does not depend on the other candidates in the call. */
@@ -186,31 +203,39 @@ ot_status ot_score_candidates(ot_model *m, const void *kv_cache, int U, const vo
 #define OT_NOALLOC_SCRATCH_BYTES (16u << 20)
 
 /* ot_score_candidates for callers that cannot allocate device memory (a
- * serving runtime that forbids allocation on its request path, a caller in
- * the middle of stream capture, a host that owns all GPU memory through its
- * own pool).  The pages have no counterpart: this is a deployment variant of
- * the NS-side call, computing exactly what ot_score_candidates computes.
+ * serving runtime that forbids allocation on its request path, or a host
+ * that owns all GPU memory through its own pool and lends none to
+ * libraries).  The pages have no counterpart: this is a deployment variant
+ * of the NS-side call, computing exactly what ot_score_candidates computes.
  * Same arguments minus the workspace: the scratch is a fixed device array of
  * OT_NOALLOC_SCRATCH_BYTES inside the library's device image, present on
  * every GPU that loads the library until the process exits.  The call makes
  * no cudaMalloc / cudaFree or other allocating call.
  *   - The model's device must be current.  The first call on a device looks
- *     up the array's address there (cudaGetSymbolAddress); make that first
- *     call before any stream capture.
+ *     up the array's address there (cudaGetSymbolAddress) and keeps it for
+ *     that device's current context; a call in a new context (after a
+ *     cudaDeviceReset, say) looks it up again.  Make the first call on a
+ *     device before any stream capture.
  *   - All calls on a device share the array; concurrent calls (other
  *     streams or threads) race on it and must be serialised by the caller.
  *     Contents persist between calls; the path never reads scratch it has
  *     not written in the same call.
- * Errors: OT_ERR_WORKSPACE_TOO_SMALL when U * C * N rows need more scratch
- * than OT_NOALLOC_SCRATCH_BYTES (the bytes ot_score_candidates would need
- * are 7 * rows * d + rows * ffn storage elements, fp8 adds rows * max(d, ffn)
- * + 4 * rows); OT_ERR_UNSUPPORTED while per-launch profiling is enabled;
- * OT_ERR_ARG if another device is current; otherwise as ot_score_candidates. */
+ * Errors, in this order: OT_ERR_ARG (null pointer, U or C < 1),
+ * OT_ERR_ALIGN, OT_ERR_SHAPE (U * C * N >= 2^31 or C * N > 2^30),
+ * OT_ERR_UNSUPPORTED while per-launch profiling is enabled,
+ * OT_ERR_WORKSPACE_TOO_SMALL when the rows need more scratch than
+ * OT_NOALLOC_SCRATCH_BYTES (the bytes ot_score_candidates would need: 7 *
+ * rows * d + rows * ffn storage elements, fp8 adds rows * max(d, ffn) + 4 *
+ * rows, rows = U * C * N), OT_ERR_ARG if another device is current; then as
+ * ot_score_candidates. */
 ot_status ot_score_candidates_noalloc(ot_model *m, const void *kv_cache, int U, const void *ns,
                                       int C, void *out_ns, void *stream);
 
-/* Training-style batch: B users with C candidates each, S and NS in one
- * call.  S device [B][L0][d], ns device [B][C][N][d] -> out_s_tail device
+/* Training-style batch (summary page, block and pyramid paragraphs: the
+ * whole token sequence of a candidate through the stack): B users with C
+ * candidates each, S and NS in one call.  Because S tokens never see NS
+ * tokens, this computes what ot_encode_user followed by ot_score_candidates
+ * computes.  S device [B][L0][d], ns device [B][C][N][d] -> out_s_tail device
  * [B][q_last][d], out_ns device [B][C][N][d]; the S K/V go to kv_cache if
  * not NULL (ot_kv_cache_bytes(m, B) bytes), else to the workspace.
  * ws >= ot_workspace_bytes(m, B, C). */
@@ -233,6 +258,29 @@ size_t ot_host_workspace_bytes(const ot_model *m, int users, int cands);
 ot_status ot_full_forward_host(ot_model *m, const void *S_host, const void *x_host, int B, int C,
                                void *out_s_tail_host, void *out_ns_host, void *kv_cache,
                                void *ws, size_t ws_bytes, void *stream);
+
+/* Per-tensor FP8 activation scales (OT_DTYPE_FP8 models only; see the FP8
+ * rule above).  scales: host float [layers][1 + n_ns][4] -- parameter set 0
+ * is the S side, set 1 + n NS position n; the four inputs of a set in the
+ * order QKV, O (attention output), W1, W2 -- each finite and > 0; copied
+ * into library-owned device memory (allocated on the first call; the call
+ * synchronises the device first, so calls enqueued earlier finish with the
+ * scales they were enqueued with).  scales = NULL returns the model to
+ * per-row scales.  Errors: OT_ERR_ARG (null model, a scale <= 0 or not
+ * finite), OT_ERR_DTYPE (not an FP8 model), OT_ERR_CUDA. */
+ot_status ot_set_act_scales(ot_model *m, const float *scales);
+
+/* Calibration for the per-tensor FP8 scales: encode U users S device
+ * [U][L0][d] and score their C candidates ns device [U][C][N][d] through
+ * every layer with per-row scales (whatever ot_set_act_scales set), and
+ * max-accumulate into amax (device float [layers][1 + n_ns][4], the layout
+ * of ot_set_act_scales; zero it before the first batch) the largest |x| of
+ * every projection input tensor.  Scales amax / 448 then quantise that
+ * sample's largest inputs to +-448 exactly.  The outputs are discarded.
+ * ws >= ot_workspace_bytes(m, U, C).  Errors: OT_ERR_ARG, OT_ERR_DTYPE (not
+ * an FP8 model), OT_ERR_ALIGN, OT_ERR_SHAPE, OT_ERR_WORKSPACE_TOO_SMALL. */
+ot_status ot_fp8_calibrate(ot_model *m, const void *S, const void *ns, int U, int C, float *amax,
+                           void *ws, size_t ws_bytes, void *stream);
 
 /* Synchronise `stream`, then read and clear the model's device error word.
  * Returns OT_OK, OT_ERR_DEVICE_TIMEOUT, OT_ERR_DEVICE_BOUNDS or OT_ERR_CUDA. */

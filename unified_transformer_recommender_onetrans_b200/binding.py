@@ -72,6 +72,8 @@ SIGNATURES = {
     "ot_score_candidates_noalloc": (_i, [_vp, _vp, _i, _vp, _i, _vp, _vp]),
     "ot_encode_append": (_i, [_vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
     "ot_append_workspace_bytes": (_sz, [_vp, _i, _i]),
+    "ot_set_act_scales": (_i, [_vp, _vp]),
+    "ot_fp8_calibrate": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp, _sz, _vp]),
 }
 
 _lib = None
@@ -325,6 +327,37 @@ class Model:
                                     ws.numel() * ws.element_size(), _stream(stream)),
               "ot_full_forward")
         return out_s_tail, out_ns
+
+    # fp8 per-tensor scales
+    def act_scale_shape(self) -> tuple:
+        return (self.layers, 1 + self.n_ns, 4)
+
+    def set_act_scales(self, scales):
+        """Per-tensor FP8 activation scales [layers, 1 + n_ns, 4] (a CPU tensor
+        or array; None: back to per-row scales)."""
+        import numpy as np
+        if scales is None:
+            check(lib().ot_set_act_scales(self.handle, None), "ot_set_act_scales")
+            return
+        a = np.ascontiguousarray(np.asarray(scales, dtype=np.float32))
+        if a.shape != self.act_scale_shape():
+            raise ValueError(f"scales must have shape {self.act_scale_shape()}")
+        check(lib().ot_set_act_scales(self.handle, a.ctypes.data_as(C.c_void_p)),
+              "ot_set_act_scales")
+
+    def fp8_calibrate(self, S, ns, amax=None, ws=None, stream=None):
+        """Max-accumulate every projection input's max |x| over users S [U, L0,
+        d] and candidates ns [U, C, N, d] into amax (a CUDA float32 tensor of
+        act_scale_shape(), zeros if None) and return it."""
+        import torch
+        U, Cn = ns.shape[0], ns.shape[1]
+        if amax is None:
+            amax = torch.zeros(self.act_scale_shape(), dtype=torch.float32, device=S.device)
+        ws = self._ws(ws, self.workspace_bytes(U, Cn))
+        check(lib().ot_fp8_calibrate(self.handle, _ptr(S), _ptr(ns), U, Cn, _ptr(amax), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)),
+              "ot_fp8_calibrate")
+        return amax
 
     def host_workspace_bytes(self, users: int, cands: int) -> int:
         return int(lib().ot_host_workspace_bytes(self.handle, users, cands))

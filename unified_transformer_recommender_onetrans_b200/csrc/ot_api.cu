@@ -38,6 +38,12 @@ struct ot_model {
     void *Wqkv_ns, *Wo_ns, *W1_ns, *W2_ns;
     void *W_split;
     float *sc_qkv_s, *sc_o_s, *sc_1_s, *sc_2_s, *sc_qkv_ns, *sc_o_ns, *sc_1_ns, *sc_2_ns;
+    // fp8: per-tensor activation scales [layers][1 + n_ns][4] (device; null =
+    // per-row scales), and while ot_fp8_calibrate enqueues, the caller's amax
+    // array (same layout) with per-row scales forced
+    float *act_scale = nullptr;
+    float *act_scale_mem = nullptr;
+    float *calib_amax = nullptr;
     void *g1_s, *g2_s, *g1_ns, *g2_ns;
     int *err;
     long long wait_limit;
@@ -105,6 +111,8 @@ int encode_tmap_3d(void *map, int esz, const void *base, const uint64_t dims[3],
 int internal_profiling(const ot_model *m) { return m->profiling; }
 
 int internal_device(const ot_model *m) { return m->device; }
+
+int internal_n_ns(const ot_model *m) { return m->cfg.n_ns; }
 
 } // namespace ot
 
@@ -415,16 +423,22 @@ struct Fp8Scratch {
     float *s;
 };
 
+// Projection inputs in the per-tensor scale layout [layer][set][4].
+enum { IN_QKV = 0, IN_O = 1, IN_W1 = 2, IN_W2 = 3 };
+
 // Attach the A operand and weights of a projection GEMM.  src: activation
 // rows (lda elements apart, through amap); W: weights of group 0 of this
 // layer (gstride elements between groups); norm: the projection follows an
 // RMSNorm with gain `gain` (gain_gstride elements between groups).
 // bf16 / fp32: the norm runs inside the GEMM and the gain is already folded
-// into W.  fp8: one pass quantises every (normalised) row to e4m3 with its own
-// scale and the GEMM reads the quantised weights and both scales.
+// into W.  fp8: one pass quantises every (normalised) row to e4m3 -- with the
+// input tensor's per-tensor scale (layer l, parameter set set0 + group, input
+// `in`) when the model has them, else with the row's own scale -- and the
+// GEMM reads the quantised weights and both scales.
 ot_status projection(ot_model *m, GemmArgs &g, const void *src, long long lda, RowMap amap,
                      const void *W, long long w_gstride, const float *wscale, const void *gain,
-                     long long gain_gstride, bool norm, const Fp8Scratch &f8, cudaStream_t st)
+                     long long gain_gstride, bool norm, const Fp8Scratch &f8, cudaStream_t st,
+                     int l = 0, int set0 = 0, int in = 0)
 {
     g.a_map = amap;
     g.b_gstride = w_gstride;
@@ -438,9 +452,13 @@ ot_status projection(ot_model *m, GemmArgs &g, const void *src, long long lda, R
     double bytes = 0;
     if (m->profiling)
         bytes = static_cast<double>(g.M) * g.G * g.K * (2 + 1) + static_cast<double>(g.M) * g.G * 4;
+    const long long slot = (static_cast<long long>(l) * (1 + m->cfg.n_ns) + set0) * 4 + in;
+    QuantRule rule{nullptr, nullptr, 4};
+    if (m->calib_amax) rule.amax = m->calib_amax + slot; // calibration: per-row scales
+    else if (m->act_scale) rule.xscale = m->act_scale + slot;
     ot_status r = profiled(m, st, OT_KIND_QUANT, ROLE_OTHER, 0.0, bytes, [&] {
         return launch_quant_rows(src, lda, amap, g.M, g.G, g.K, gain, gain_gstride, norm ? 1 : 0,
-                                 m->cfg.eps, f8.q, f8.s, st);
+                                 m->cfg.eps, rule, f8.q, f8.s, st);
     });
     if (r != OT_OK) return r;
     g.A = f8.q;
@@ -469,8 +487,11 @@ EpiSeg seg_of(void *out, long long ld, int lo, int hi, RowMap map)
 // delta of its L_l rows, all of them queries), attending to the cached K/V
 // of the old rows, which the caller has already placed in `kv`; their own
 // K/V go after the old rows.
+// full_last: run the whole last layer even when s_out is null (its output
+// goes to a workspace buffer; calibration needs its projections).
 ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, Ws ws,
-                     cudaStream_t st, cudaEvent_t *kv_ready = nullptr, int delta = 0)
+                     cudaStream_t st, cudaEvent_t *kv_ready = nullptr, int delta = 0,
+                     bool full_last = false)
 {
     const ot_config &c = m->cfg;
     const int d = c.d, f = c.ffn, esz = m->esz;
@@ -497,7 +518,8 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
         const int n = delta ? delta : L;        // rows run through this layer (the last n of L)
         const int q = delta ? delta : c.q[l];   // their query tail
         const bool last = l == c.layers - 1;
-        const bool kv_only = last && s_out == nullptr; // the S tail of the last layer is unused
+        // the S tail of the last layer is unused
+        const bool kv_only = last && s_out == nullptr && !full_last;
         char *K = at(kv, kv_layer_off(c, l), esz);
         char *V = K + static_cast<long long>(L) * d * esz;
         const RowMap cache_map{n, ustride / d, L - n, 0, 0};
@@ -507,7 +529,8 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
         GemmArgs g = gemm_base(c, U * n, kv_only ? 2 * d : 3 * d, d, 1);
         if ((r = projection(m, g, X, d, rowmap_identity(),
                             at(m->Wqkv_s, static_cast<long long>(l) * 3 * d * d + (kv_only ? d * d : 0), wesz),
-                            3LL * d * d, fp8 ? m->sc_qkv_s + l : nullptr, g1, d, true, f8, st)) != OT_OK)
+                            3LL * d * d, fp8 ? m->sc_qkv_s + l : nullptr, g1, d, true, f8, st, l, 0,
+                            IN_QKV)) != OT_OK)
             return r;
         if (kv_only) {
             g.nseg = 2;
@@ -559,7 +582,7 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
         if ((r = projection(m, g, Ab, d, rowmap_identity(),
                             at(m->Wo_s, static_cast<long long>(l) * d * d, wesz),
                             static_cast<long long>(d) * d, fp8 ? m->sc_o_s + l : nullptr, nullptr, 0,
-                            false, f8, st)) != OT_OK)
+                            false, f8, st, l, 0, IN_O)) != OT_OK)
             return r;
         g.res = X;
         g.res_ld = d;
@@ -572,7 +595,7 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
         if ((r = projection(m, g, Hb, d, rowmap_identity(),
                             at(m->W1_s, static_cast<long long>(l) * f * d, wesz),
                             static_cast<long long>(f) * d, fp8 ? m->sc_1_s + l : nullptr, g2, d, true,
-                            f8, st)) != OT_OK)
+                            f8, st, l, 0, IN_W1)) != OT_OK)
             return r;
         g.gelu = 1;
         g.nseg = 1;
@@ -582,7 +605,7 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
         if ((r = projection(m, g, hid, f, rowmap_identity(),
                             at(m->W2_s, static_cast<long long>(l) * d * f, wesz),
                             static_cast<long long>(d) * f, fp8 ? m->sc_2_s + l : nullptr, nullptr, 0,
-                            false, f8, st)) != OT_OK)
+                            false, f8, st, l, 0, IN_W2)) != OT_OK)
             return r;
         g.res = Hb;
         g.res_ld = d;
@@ -595,6 +618,7 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
 }
 
 // NS-side of every layer: U users x C candidates, N tokens each, against kv.
+// out may be null (calibration): the last layer then writes a workspace buffer.
 ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, void *out, Ws ws,
                     cudaStream_t st, cudaEvent_t *kv_ready = nullptr)
 {
@@ -632,7 +656,7 @@ ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, v
         const void *g2 = fp8 ? at(m->g2_ns, lN * d, esz) : nullptr;
         GemmArgs g = gemm_base(c, Mc, 3 * d, d, N);
         if ((r = projection(m, g, X, d, grp, at(m->Wqkv_ns, lN * 3 * d * d, wesz), 3LL * d * d,
-                            fp8 ? m->sc_qkv_ns + lN : nullptr, g1, d, true, f8, st)) != OT_OK)
+                            fp8 ? m->sc_qkv_ns + lN : nullptr, g1, d, true, f8, st, l, 1, IN_QKV)) != OT_OK)
             return r;
         g.nseg = 3;
         g.seg[0] = seg_of(Qn, d, 0, d, grp);
@@ -658,7 +682,7 @@ ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, v
         at_.O = An;
         at_.scale = 1.0f / sqrtf(static_cast<float>(at_.hd));
         if ((r = attn(m, at_, st)) != OT_OK) return r;
-        void *Xn = last ? out : Xb[l & 1];
+        void *Xn = last && out ? out : Xb[l & 1];
         if (use_fused_ffn(m)) {
             // O projection + residual and the FFN in one grouped launch
             const FfnArgs fa = ffn_o_args(m, Mc, N, An, grp, at(m->Wo_ns, lN * d * d, esz), X, grp,
@@ -670,7 +694,7 @@ ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, v
         g = gemm_base(c, Mc, d, d, N);
         if ((r = projection(m, g, An, d, grp, at(m->Wo_ns, lN * d * d, wesz),
                             static_cast<long long>(d) * d, fp8 ? m->sc_o_ns + lN : nullptr, nullptr,
-                            0, false, f8, st)) != OT_OK)
+                            0, false, f8, st, l, 1, IN_O)) != OT_OK)
             return r;
         g.res = X;
         g.res_ld = d;
@@ -681,7 +705,7 @@ ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, v
         g = gemm_base(c, Mc, f, d, N);
         if ((r = projection(m, g, Hn, d, grp, at(m->W1_ns, lN * f * d, wesz),
                             static_cast<long long>(f) * d, fp8 ? m->sc_1_ns + lN : nullptr, g2, d,
-                            true, f8, st)) != OT_OK)
+                            true, f8, st, l, 1, IN_W1)) != OT_OK)
             return r;
         g.gelu = 1;
         g.nseg = 1;
@@ -690,7 +714,7 @@ ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, v
         g = gemm_base(c, Mc, d, f, N);
         if ((r = projection(m, g, hid, f, grp, at(m->W2_ns, lN * d * f, wesz),
                             static_cast<long long>(d) * f, fp8 ? m->sc_2_ns + lN : nullptr, nullptr,
-                            0, false, f8, st)) != OT_OK)
+                            0, false, f8, st, l, 1, IN_W2)) != OT_OK)
             return r;
         g.res = Hn;
         g.res_ld = d;
@@ -1059,6 +1083,56 @@ ot_status ot_set_kernel_path(ot_model *m, int path)
 }
 
 long long ot_launch_count(const ot_model *m) { return m ? m->launches : -1; }
+
+ot_status ot_set_act_scales(ot_model *m, const float *scales)
+{
+    if (!m) return OT_ERR_ARG;
+    if (m->cfg.dtype != OT_DTYPE_FP8) return OT_ERR_DTYPE;
+    const long long n = static_cast<long long>(m->cfg.layers) * (1 + m->cfg.n_ns) * 4;
+    if (!scales) {
+        m->act_scale = nullptr; // back to per-row scales (the array stays allocated)
+        return OT_OK;
+    }
+    for (long long i = 0; i < n; ++i)
+        if (!(scales[i] > 0.f) || !(scales[i] < 3.0e38f)) return OT_ERR_ARG;
+    std::lock_guard<std::recursive_mutex> lock(m->enqueue_mu);
+    if (!m->act_scale_mem) {
+        if (cudaMalloc(reinterpret_cast<void **>(&m->act_scale_mem), sizeof(float) * n) != cudaSuccess)
+            return OT_ERR_CUDA;
+        m->allocs.push_back(m->act_scale_mem);
+    }
+    // synchronous: no call enqueued before this one still reads the old scales
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpy(m->act_scale_mem, scales, sizeof(float) * n, cudaMemcpyHostToDevice) != cudaSuccess)
+        return OT_ERR_CUDA;
+    m->act_scale = m->act_scale_mem;
+    return OT_OK;
+}
+
+ot_status ot_fp8_calibrate(ot_model *m, const void *S, const void *ns, int U, int C, float *amax,
+                           void *ws, size_t ws_bytes, void *stream)
+{
+    if (!m || !S || !ns || !amax || !ws || U < 1 || C < 1) return OT_ERR_ARG;
+    if (m->cfg.dtype != OT_DTYPE_FP8) return OT_ERR_DTYPE;
+    if (!aligned16(S) || !aligned16(ns) || !aligned16(ws) || (reinterpret_cast<uintptr_t>(amax) & 3))
+        return OT_ERR_ALIGN;
+    if (static_cast<long long>(U) * m->cfg.L0 > (1LL << 31) - 1 ||
+        static_cast<long long>(U) * C * m->cfg.n_ns > (1LL << 31) - 1)
+        return OT_ERR_SHAPE;
+    if (ws_bytes < ot_workspace_bytes(m, U, C)) return OT_ERR_WORKSPACE_TOO_SMALL;
+    const ot_config &c = m->cfg;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
+    void *kv = w.take(static_cast<long long>(U) * kv_user_elems(c));
+    if (!kv) return OT_ERR_WORKSPACE_TOO_SMALL;
+    std::lock_guard<std::recursive_mutex> lock(m->enqueue_mu);
+    m->calib_amax = amax;
+    // every layer in full, S side then NS side against the cache just written
+    ot_status r = run_encode(m, S, U, kv, nullptr, w, st, nullptr, 0, true);
+    if (r == OT_OK) r = run_score(m, kv, U, ns, C, nullptr, w, st);
+    m->calib_amax = nullptr;
+    return r;
+}
 
 ot_status ot_poll_device_error(ot_model *m, void *stream)
 {

@@ -2,12 +2,16 @@
 //
 // Activations: one warp per projection input row.  The row is read once
 // (bf16), optionally RMSNorm-ed with its gain (y = x * rsqrt(mean(x^2) + eps)
-// * gain), its amax taken, scale s = amax / 448 (1 for an all-zero row), and
-// y / s converted to e4m3 with round-to-nearest-even and saturation.  The
-// GEMM epilogue multiplies the fp32 accumulator by s (per row) and by the
-// weight matrix's own scale.  Per-row scales keep each token's projection
-// independent of every other row in the call, so a candidate's result does
-// not depend on which other candidates share the batch.
+// * gain) and converted to e4m3(y / s), round to nearest even, saturating.
+// The scale s is the input tensor's fixed per-tensor scale when one is given
+// (one fp32 value per projection input of a layer and parameter set, found
+// by calibration), else the row's own amax / 448 (1 for an all-zero row):
+// the calibration pass.  Either way s does not depend on the other rows of
+// the call, so a candidate's result does not depend on which other
+// candidates share the batch.  The row's scale is written beside it and the
+// GEMM epilogue multiplies the fp32 accumulator by it and by the weight
+// matrix's own scale.  Optionally the row's amax is max-accumulated into its
+// tensor's slot (calibration).
 //
 // Weights: one CTA per matrix computes its amax, then writes e4m3(w / s_w).
 #include <cuda_bf16.h>
@@ -38,7 +42,8 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16 *X,
                                                          RowMap map, long long M, int G, int K,
                                                          const __nv_bfloat16 *gain,
                                                          long long gain_gstride, int norm,
-                                                         float eps, uint8_t *q, float *scale)
+                                                         float eps, QuantRule rule, uint8_t *q,
+                                                         float *scale)
 {
     const int lane = threadIdx.x & 31;
     const long long warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
@@ -87,7 +92,12 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16 *X,
 #pragma unroll
             for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
         amax = warp_max(amax);
-        const float s = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        // non-negative floats order like their bit patterns as signed ints
+        if (rule.amax && lane == 0)
+            atomicMax(reinterpret_cast<int *>(rule.amax + g * rule.gstride), __float_as_int(amax));
+        const float s = rule.xscale ? rule.xscale[g * rule.gstride]
+                        : amax > 0.f ? __fdiv_rn(amax, 448.0f)
+                                     : 1.0f;
         uint2 *dst = reinterpret_cast<uint2 *>(q + arow * K);
 #pragma unroll
         for (int i = 0; i < QR_MAX_CHUNKS; ++i) {
@@ -112,7 +122,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16 *X,
 
 cudaError_t launch_quant_rows(const void *X, long long lda, RowMap map, long long M, int G, int K,
                               const void *gain, long long gain_gstride, int norm, float eps,
-                              uint8_t *q_out, float *scale_out, cudaStream_t s)
+                              QuantRule rule, uint8_t *q_out, float *scale_out, cudaStream_t s)
 {
     if (K % 8 || K > QR_MAX_CHUNKS * 8 * 32) return cudaErrorInvalidValue;
     const long long rows = M * G;
@@ -121,7 +131,7 @@ cudaError_t launch_quant_rows(const void *X, long long lda, RowMap map, long lon
     if (blocks < 1) blocks = 1;
     quant_rows_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
         static_cast<const __nv_bfloat16 *>(X), lda, map, M, G, K,
-        static_cast<const __nv_bfloat16 *>(gain), gain_gstride, norm, eps, q_out, scale_out);
+        static_cast<const __nv_bfloat16 *>(gain), gain_gstride, norm, eps, rule, q_out, scale_out);
     return cudaGetLastError();
 }
 

@@ -176,15 +176,24 @@ struct KvGrowArgs {
 cudaError_t launch_kv_grow(const KvGrowArgs &a, int users, int layers, cudaStream_t s);
 cudaError_t launch_embed_gather(const void *table, long long rows, int d, const int64_t *ids,
                                 long long n, void *out, int *err, cudaStream_t s);
+// Scale rule of an FP8 projection input (group g reads slot g * gstride):
+// xscale = the input tensor's fixed scale (NULL: each row's amax / 448);
+// amax = where each row's max |x| is max-accumulated (NULL: not recorded).
+struct QuantRule {
+    const float *xscale;
+    float *amax;
+    long long gstride;
+};
 cudaError_t launch_quant_rows(const void *X, long long lda, RowMap map, long long M, int G, int K,
                               const void *gain, long long gain_gstride, int norm, float eps,
-                              uint8_t *q_out, float *scale_out, cudaStream_t s);
+                              QuantRule rule, uint8_t *q_out, float *scale_out, cudaStream_t s);
 cudaError_t launch_quant_weights(const void *W, long long per_mat, long long mats, uint8_t *q_out,
                                  float *scale_out, float *amax_scratch, cudaStream_t s);
 
 // Read-only model queries for entry points defined outside ot_api.cu.
 int internal_profiling(const ot_model *m);
 int internal_device(const ot_model *m);
+int internal_n_ns(const ot_model *m);
 size_t internal_score_ws_bytes(const ot_model *m, int users, int cands);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point.
