@@ -34,6 +34,33 @@ sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM traffic of the dominant kernel (dram__bytes_read.sum + dram__bytes_write.sum),
+# summed over the launches of one step, from one ncu capture of the default
+# workload (the capture is summarised in profiles/, with its command).  It is
+# reported only while the kernel's source is the one that was captured.
+CAPTURED_TRAFFIC = {
+    # kernel kind -> (source file, its sha256 at capture time, bytes per step, launches per step)
+}
+
+
+def metric_name(wl) -> str:
+    """The headline metric's name: the same string in both arms."""
+    return f"S-tokens/s ({wl.name} full forward)"
+
+
+def captured_traffic(kind: str):
+    """(bytes per step, note) of the last ncu capture of `kind`, or (None, why)."""
+    import hashlib
+    ent = CAPTURED_TRAFFIC.get(kind)
+    if ent is None:
+        return None, "no ncu capture recorded for this kernel"
+    src, sha, nbytes, launches = ent
+    path = os.path.join(ROOT, "unified_transformer_recommender_onetrans_b200", "csrc", src)
+    with open(path, "rb") as fh:
+        if hashlib.sha256(fh.read()).hexdigest() != sha:
+            return None, f"{src} changed since the ncu capture"
+    return nbytes, f"ncu dram__bytes_read.sum + dram__bytes_write.sum over {launches} launches"
+
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -244,7 +271,7 @@ def run_reference(args, wl):
     sec_per_tok = sum(per) / len(per)
     value = 1.0 / sec_per_tok
     line = {
-        "impl": "reference", "metric": "S-tokens/s (full forward)", "value": value,
+        "impl": "reference", "metric": metric_name(wl), "value": value,
         "unit": "S-tokens/s", "n_gpus": ws, "steps": len(per), "warmup": args.warmup_ref,
         "ms_per_step": 1e3 * sec_per_tok * wl.L0, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -437,6 +464,18 @@ def run_serving(name, steps, flush, world, dist, dev, peaks, cands=None, sweep=N
         gather = None
     x = gen_auto_split_features(wl).to(dev)
     kv = m.new_kv_cache(U)
+    if wl.dtype == "fp8":
+        # per-tensor activation scales from a calibration sample (user 0 and
+        # 8 of its candidates): amax of every projection input / 448
+        if gather:
+            gather()
+        ns_cal = m.auto_split(x[:1, :8].contiguous())
+        amax = m.fp8_calibrate(S[:1].contiguous(), ns_cal)
+        m.poll()
+        scales = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax)).cpu()
+        m.set_act_scales(scales)
+        out["fp8_scales"] = "per-tensor, calibrated on user 0 x 8 candidates (ot_fp8_calibrate)"
+        del ns_cal
     ws = torch.empty(m.workspace_bytes(U, 0), dtype=torch.uint8, device=dev)
 
     def encode():
@@ -485,6 +524,53 @@ def run_serving(name, steps, flush, world, dist, dev, peaks, cands=None, sweep=N
             torch.cuda.empty_cache()
     m.close()
     return out
+
+
+def run_full_point(name, steps, flush, world, dist, dev, peaks):
+    """Auto-Split + full forward of a whole workload batch (C candidates per
+    user, S and NS sides in one call), 10 warm-ups + median of `steps` calls."""
+    import torch
+
+    import unified_transformer_recommender_onetrans_b200 as ot
+    from synth import WORKLOADS, gen_auto_split_features, gen_s_tokens, gen_weights
+    from unified_transformer_recommender_onetrans_b200.binding import WEIGHT_NAMES
+
+    wl = WORKLOADS[name]
+    w = gen_weights(wl)
+    q = ot.pyramid_schedule(wl.L0, wl.q_end, wl.layers)
+    m = ot.Model(layers=wl.layers, d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns, L0=wl.L0,
+                 q=q, F=wl.F, eps=wl.eps, dtype=wl.dtype,
+                 weights={k: w[k].to(dev) for k in WEIGHT_NAMES})
+    U, C = wl.users, wl.cands
+    S = gen_s_tokens(wl, weights=w).to(dev)
+    x = gen_auto_split_features(wl).to(dev)
+    del w
+    ns = torch.empty(U, C, wl.n_ns, wl.d, dtype=m.storage, device=dev)
+    out_ns = torch.empty_like(ns)
+    s_tail = torch.empty(U, q[-1], wl.d, dtype=m.storage, device=dev)
+    kv = m.new_kv_cache(U)
+    ws = torch.empty(m.workspace_bytes(U, C), dtype=torch.uint8, device=dev)
+
+    def step():
+        m.auto_split(x, ns)
+        m.full_forward(S, ns, kv=kv, out_s_tail=s_tail, out_ns=out_ns, ws=ws)
+
+    for _ in range(10):
+        step()
+    m.poll()
+    ms = _time_device(step, steps, flush, world, dist, dev)
+    m.poll()
+    m.profile(True)
+    step()
+    flops = sum(r["flops"] for r in m.profile_read())
+    m.profile(False)
+    m.close()
+    tf = flops / (ms / 1e3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    return {"workload": name, "users": U, "cands": C, "dtype": wl.dtype, "full_forward_ms": ms,
+            "full_forward_s_tokens_per_s": world * U * wl.L0 / (ms / 1e3),
+            "full_forward_tflops": tf, "full_forward_tensor_frac": tf / peak,
+            "peak_source": f"{peaks['_source']} bf16 dense sustained (whole calls back to back)"}
 
 
 # ---------------------------------------------------------------- our arm
@@ -618,6 +704,8 @@ def run_ours(args, wl):
             serving.append(run_serving(name, 50, flush, world, dist, dev, peaks, cands, sw,
                                        append_rows=64 if name == "onetrans_s_serve" else 0))
             torch.cuda.empty_cache()
+        serving.append(run_full_point("onetrans_l_full", 50, flush, world, dist, dev, peaks))
+        torch.cuda.empty_cache()
 
     # ---- roofline of the dominant kernel (from the live per-launch events)
     by_kind, by_role = {}, {}
@@ -631,10 +719,16 @@ def run_ours(args, wl):
     dom = max(by_kind, key=lambda k: by_kind[k]["ms"])
     dk = by_kind[dom]
     tf = dk["flops"] / (dk["ms"] / 1e3) / 1e12
-    peak_tf = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    # each launch is timed alone by its own event pair: the burst peak applies
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    traffic, traffic_note = captured_traffic(dom)
     roofline = {"kernel": dom, "bound": "tensor", "achieved": tf, "peak": peak_tf,
-                "unit": "TFLOP/s", "frac": tf / peak_tf, "traffic": None,
-                "peak_source": f"{peaks['_source']} bf16 dense sustained",
+                "unit": "TFLOP/s", "frac": tf / peak_tf,
+                "traffic": None if traffic is None else traffic * prof_steps / dk["launches"],
+                "traffic_unit": "bytes per launch (mean over the step's launches)",
+                "traffic_source": traffic_note,
+                "algorithmic_bytes_per_launch": dk["bytes"] / dk["launches"],
+                "peak_source": f"{peaks['_source']} bf16 dense burst",
                 "launches_per_step": dk["launches"] / prof_steps,
                 "algorithmic_tflop_per_step": dk["flops"] / prof_steps / 1e12}
     step_flops = sum(v["flops"] for v in by_kind.values()) / prof_steps
@@ -656,7 +750,7 @@ def run_ours(args, wl):
                              f"candidate each), "
                              f"Auto-Split + encode + score, C fp64 oracle, OpenMP"}
         line = {
-            "metric": "S-tokens/s (OneTransS full forward)", "value": value, "unit": "S-tokens/s",
+            "metric": metric_name(wl), "value": value, "unit": "S-tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
@@ -695,7 +789,7 @@ def main():
                     help="also score the serving caches at C = 1, 2, 4, 8, 16, 64, 512")
     args = ap.parse_args()
     args.steps_ref = max(1, args.steps)
-    args.warmup_ref = min(args.warmup, 3)
+    args.warmup_ref = args.warmup
     from synth import WORKLOADS
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":

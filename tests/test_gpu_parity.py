@@ -254,6 +254,37 @@ def test_onetrans_l_full_forward_sampled_users():
     assert_within(_full_size("onetrans_l_full", [5]), TOL["bf16"])
 
 
+def test_onetrans_l_cached_scoring_sampled():
+    """OneTransL serving with the cross-request cache at the cached-candidate
+    shape: all 32 users (1500 S tokens, d = 384) encoded once, 8 candidates
+    per user scored against the cache (24 NS tokens each: 192 NS rows per
+    user and head, the split-key NS attention; the two-GEMM d = 384 FFN).
+    Sampled users and candidates against the oracle: NS outputs and every
+    layer's K / V."""
+    wl = WORKLOADS["onetrans_l_full"].with_(cands=8)
+    w = gen_weights(wl)
+    S = gen_s_tokens(wl, weights=w)
+    x = gen_auto_split_features(wl)                    # [32, 8, 1024]
+    m = model_of(wl, w)
+    m.set_wait_limit(TEST_WAIT)
+    kv, _ = m.encode_user(S.cuda(), want_s_tail=False)
+    ns = m.auto_split(x.cuda())
+    out = m.score_candidates(kv, ns)
+    m.poll()
+    users, cands = [2, 31], [0, 3, 7]
+    cfg = oracle_cfg(m)
+    kv_o, _ = O.encode_user(cfg, w, S[users])
+    ns_o = O.auto_split(x[users][:, cands], w["W_split"], wl.n_ns, wl.d)
+    out_o = O.score_candidates(cfg, w, kv_o, ns_o)
+    errs = {"ns_out": O.rel_l2(out[users][:, cands].double().cpu().numpy(), out_o)}
+    errs.update(kv_errors(m, kv[users], kv_o, cfg))
+    assert_within(errs, TOL["bf16"])
+    # the full forward of the same batch gives the same NS outputs
+    s_tail, ns_full, kv2 = _run_full(m, S.cuda(), ns)
+    assert torch.equal(kv2, kv)
+    assert O.rel_l2(ns_full.double().cpu().numpy(), out.double().cpu().numpy()) < 2 * 2.0 ** -8
+
+
 def test_onetrans_s_serving_sampled():
     wl = WORKLOADS["onetrans_s_serve"]
     w = gen_weights(wl)
