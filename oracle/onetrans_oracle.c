@@ -21,6 +21,11 @@
  *              that tail (L_{l+1} = q_l), in order.
  *   KV cache : S never attends to NS, so the S-side K/V of every layer are a
  *              per-user quantity; candidates are scored against them.
+ *   full attention (cfg->full_attn = 1; summary page, limitations paragraph:
+ *              full attention matches causal attention offline, causal wins
+ *              only through the KV cache): every token sees every token of
+ *              its own candidate's sequence, S and NS alike.  S then depends
+ *              on the candidate, so only the joint formulation runs it.
  *
  * Readings where the pages are silent (each listed in the design notes):
  *   RMSNorm n(x; g) = x * (mean(x^2) + eps)^(-1/2) * g, eps from the config;
@@ -72,6 +77,7 @@ typedef struct {
     int fp8;                  /* 0 off, 1 per-row scales, 2 per-tensor scales */
     const double *act_scale;  /* fp8 == 2: [layers][1 + n_ns][4] */
     double *act_amax;         /* optional, same layout: max |input| seen */
+    int full_attn;            /* 1: full (non-causal) attention, joint form only */
 } orc_cfg;
 
 enum { ORC_IN_QKV = 0, ORC_IN_O = 1, ORC_IN_W1 = 2, ORC_IN_W2 = 3 };
@@ -333,7 +339,7 @@ static int check_cfg(const orc_cfg *c)
 int orc_encode_user(const orc_cfg *c, const orc_weights *w, const float *S, int U,
                     double *kv, double *s_out)
 {
-    if (check_cfg(c)) return 1;
+    if (check_cfg(c) || c->full_attn) return 1; /* S would depend on the candidate */
     int d = c->d, H = c->heads, hd = d / H, f = c->ffn;
     long kv_user = orc_kv_user_elems(c);
     for (int u = 0; u < U; ++u) {
@@ -405,7 +411,7 @@ int orc_encode_user(const orc_cfg *c, const orc_weights *w, const float *S, int 
 int orc_encode_append(const orc_cfg *c, const orc_weights *w, const double *kv_old,
                       const float *S_new, int U, int delta, double *kv_new, double *out_new)
 {
-    if (check_cfg(c) || delta < 1) return 1;
+    if (check_cfg(c) || c->full_attn || delta < 1) return 1;
     orc_cfg old = *c;
     old.L0 -= delta;
     for (int l = 0; l < c->layers; ++l) old.q[l] -= delta;
@@ -470,7 +476,7 @@ int orc_encode_append(const orc_cfg *c, const orc_weights *w, const double *kv_o
 int orc_score_candidates(const orc_cfg *c, const orc_weights *w, const double *kv, int U,
                          const double *ns_in, int C, double *ns_out)
 {
-    if (check_cfg(c)) return 1;
+    if (check_cfg(c) || c->full_attn) return 1;
     int d = c->d, H = c->heads, hd = d / H, f = c->ffn, N = c->n_ns;
     long kv_user = orc_kv_user_elems(c);
     pset_t *P = (pset_t *)malloc(sizeof(pset_t) * (long)c->layers * (N > 0 ? N : 1));
@@ -527,7 +533,8 @@ int orc_score_candidates(const orc_cfg *c, const orc_weights *w, const double *k
 /* ------------------------------------------------------------------------- */
 /* Joint formulation: every candidate's own token sequence [S rows; NS rows]  */
 /* run through the stack with no cache, each token picking its parameter set  */
-/* by type and position and its visible keys by the S/NS mask rule.           */
+/* by type and position and its visible keys by the S/NS mask rule (or, with  */
+/* full attention, every key of the sequence).                                */
 /* s_out [U][C][q_last][d]; kv [U][C][cache]; ns_out [U][C][N][d].            */
 int orc_full_forward_joint(const orc_cfg *c, const orc_weights *w, const float *S, int U,
                            const double *ns_in, int C, double *s_out, double *kv, double *ns_out)
@@ -588,7 +595,7 @@ int orc_full_forward_joint(const orc_cfg *c, const orc_weights *w, const float *
                     int nv = 0;
                     for (long j = 0; j < T; ++j) {
                         int j_ns = j >= L;
-                        int ok = is_ns ? (!j_ns || j <= i) : (!j_ns && j <= i);
+                        int ok = c->full_attn ? 1 : is_ns ? (!j_ns || j <= i) : (!j_ns && j <= i);
                         if (ok) {
                             memcpy(Kv + (long)nv * d, Ka + j * d, sizeof(double) * d);
                             memcpy(Vv + (long)nv * d, Va + j * d, sizeof(double) * d);

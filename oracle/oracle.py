@@ -26,7 +26,7 @@ class _Cfg(C.Structure):
     _fields_ = [("layers", C.c_int), ("d", C.c_int), ("heads", C.c_int), ("ffn", C.c_int),
                 ("n_ns", C.c_int), ("L0", C.c_int), ("q", C.c_int * MAX_LAYERS),
                 ("eps", C.c_double), ("fp8", C.c_int), ("act_scale", C.POINTER(C.c_double)),
-                ("act_amax", C.POINTER(C.c_double))]
+                ("act_amax", C.POINTER(C.c_double)), ("full_attn", C.c_int)]
 
 
 # FP8 rules of the projection inputs (see onetrans_oracle.c): off, one scale
@@ -113,6 +113,7 @@ class Config:
     eps: float = 1e-6
     fp8: int = FP8_OFF
     act_scale: object = None
+    full_attn: bool = False     # full (non-causal) attention: joint form only
 
     @staticmethod
     def of(wl, q=None, fp8=None, act_scale=None) -> "Config":
@@ -139,6 +140,7 @@ class Config:
             c.q[i] = int(v)
         c.eps = float(self.eps)
         c.fp8 = int(self.fp8)
+        c.full_attn = int(bool(self.full_attn))
         if self.fp8 == FP8_TENSOR:
             if self.act_scale is None:
                 raise ValueError("per-tensor FP8 needs act_scale")
@@ -156,7 +158,8 @@ class Config:
         query tail longer by delta (pyramid windows anchored at their first
         row)."""
         return Config(self.layers, self.d, self.heads, self.ffn, self.n_ns, self.L0 + delta,
-                      [v + delta for v in self.q], self.eps, self.fp8, self.act_scale)
+                      [v + delta for v in self.q], self.eps, self.fp8, self.act_scale,
+                      self.full_attn)
 
     def kv_user_elems(self) -> int:
         return int(lib().orc_kv_user_elems(C.byref(self._c())))

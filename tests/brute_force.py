@@ -91,7 +91,9 @@ def _gelu(z):
     return 0.5 * z * (1.0 + math.erf(z / math.sqrt(2.0)))
 
 
-def _visible(qt: Token, kt: Token) -> bool:
+def _visible(qt: Token, kt: Token, full: bool = False) -> bool:
+    if full:            # full attention: every token of the sequence
+        return True
     if qt.kind == "S":
         return kt.kind == "S" and kt.index <= qt.index
     return kt.kind == "S" or kt.index <= qt.index
@@ -112,12 +114,12 @@ def _params(w, l, tok: Token):
             w["g1_ns"][l][n], w["g2_ns"][l][n])
 
 
-def run_candidate(w, S_rows, ns_rows, q_sched, heads, eps, fp8=None):
+def run_candidate(w, S_rows, ns_rows, q_sched, heads, eps, fp8=None, full=False):
     """One candidate: S_rows [L0][d], ns_rows [N][d] (lists).
 
     Returns (S tail rows after the last layer, NS rows, per-layer (K, V) of
     the S tokens).  ``w`` holds nested Python lists; ``fp8`` an Fp8 state or
-    None.
+    None; ``full``: full (non-causal) attention over the candidate's sequence.
     """
     d = len(S_rows[0])
     hd = d // heads
@@ -142,7 +144,7 @@ def run_candidate(w, S_rows, ns_rows, q_sched, heads, eps, fp8=None):
                 qv = proj[i][0][h * hd:(h + 1) * hd]
                 scores, vals = [], []
                 for j, kt in enumerate(seq):
-                    if not _visible(t, kt):
+                    if not _visible(t, kt, full):
                         continue
                     kvec = proj[j][1][h * hd:(h + 1) * hd]
                     scores.append(sum(a_ * b_ for a_, b_ in zip(qv, kvec)) / math.sqrt(hd))

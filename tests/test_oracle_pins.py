@@ -72,15 +72,16 @@ def test_brute_force_matches_oracle(case):
                 np.testing.assert_allclose(Vo, np.array(V), rtol=0, atol=1e-12)
 
 
-def _torch_causal_layer(x, Wqkv, Wo, W1, W2, g1, g2, H, eps):
-    """Pre-norm causal Transformer layer from torch library routines (fp64)."""
+def _torch_causal_layer(x, Wqkv, Wo, W1, W2, g1, g2, H, eps, causal=True):
+    """Pre-norm causal (or, causal=False, bidirectional) Transformer layer from
+    torch library routines (fp64)."""
     T, d = x.shape
     hd = d // H
     xn = Fnn.rms_norm(x, (d,), weight=g1, eps=eps)
     qkv = xn @ Wqkv.T
     q, k, v = qkv.split(d, dim=-1)
     heads = lambda t: t.view(T, H, hd).transpose(0, 1)  # noqa: E731
-    a = Fnn.scaled_dot_product_attention(heads(q), heads(k), heads(v), is_causal=True)
+    a = Fnn.scaled_dot_product_attention(heads(q), heads(k), heads(v), is_causal=causal)
     h = x + a.transpose(0, 1).reshape(T, d) @ Wo.T
     return h + Fnn.gelu(Fnn.rms_norm(h, (d,), weight=g2, eps=eps) @ W1.T) @ W2.T
 
@@ -110,6 +111,87 @@ def test_textbook_reduction_causal_transformer(pyramid):
             L = q[l]
         np.testing.assert_allclose(s_out[0], x[:L].numpy(), rtol=0, atol=1e-11)
         np.testing.assert_allclose(ns_out[0, c], x[L:].numpy(), rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("pyramid", [False, True])
+def test_textbook_reduction_full_attention(pyramid):
+    """Full attention with every NS parameter set equal to the S set: each
+    block is a plain bidirectional pre-norm Transformer layer over [S; NS]
+    (scaled_dot_product_attention with is_causal=False), and with a pyramid
+    the kept rows are the tail S rows and the NS rows of that layer."""
+    layers, d, H, f, N, L0 = 2, 16, 2, 32, 3, 11
+    q = [7, 3] if pyramid else [L0, L0]
+    w = rand_weights(layers, d, f, N, seed=4, dtype=torch.float64)
+    for name in ("Wqkv", "Wo", "W1", "W2", "g1", "g2"):
+        w[name + "_ns"] = w[name + "_s"][:, None].expand(-1, N, *w[name + "_s"].shape[1:]).clone()
+    S, ns = rand_inputs(1, 2, L0, N, d, seed=6, dtype=torch.float64)
+    w = {k: v.float().double() for k, v in w.items()}
+    S, ns = S.float().double(), ns.float().double()
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    cfg.full_attn = True
+    js, jkv, jns = O.full_forward_joint(cfg, w, S, ns)
+    for c in range(2):
+        x = torch.cat([S[0], ns[0, c]])
+        L = L0
+        for l in range(layers):
+            y = _torch_causal_layer(x, w["Wqkv_s"][l], w["Wo_s"][l], w["W1_s"][l], w["W2_s"][l],
+                                    w["g1_s"][l], w["g2_s"][l], H, 1e-6, causal=False)
+            x = torch.cat([y[L - q[l]:L], y[L:]])
+            L = q[l]
+        np.testing.assert_allclose(js[0, c], x[:L].numpy(), rtol=0, atol=1e-11)
+        np.testing.assert_allclose(jns[0, c], x[L:].numpy(), rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("case", TINY_CASES[1:4])
+def test_brute_force_matches_oracle_full_attention(case):
+    """Full attention: the joint oracle against the brute-force token loop
+    with its every-key visibility; the split (cached) form refuses it."""
+    layers, d, H, f, N, L0, q, U, Cn = case
+    w = rand_weights(layers, d, f, N, seed=L0 + d + 2)
+    S, ns = rand_inputs(U, Cn, L0, N, d, seed=7 * L0 + N + 2)
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    cfg.full_attn = True
+    js, jkv, jns = O.full_forward_joint(cfg, w, S, ns)
+    wl = to_lists(w)
+    for u in range(U):
+        for c in range(Cn):
+            bs, bns, bkv = run_candidate(wl, S[u].double().tolist(), ns[u, c].double().tolist(),
+                                         q, H, 1e-6, full=True)
+            np.testing.assert_allclose(js[u, c], np.array(bs), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(jns[u, c], np.array(bns), rtol=0, atol=1e-12)
+            for l, (K, V) in enumerate(bkv):
+                Ko, Vo = O.kv_layer(cfg, jkv[u, c], l)
+                np.testing.assert_allclose(Ko, np.array(K), rtol=0, atol=1e-12)
+                np.testing.assert_allclose(Vo, np.array(V), rtol=0, atol=1e-12)
+    with pytest.raises(ValueError):
+        O.encode_user(cfg, w, S)
+
+
+def test_full_attention_breaks_the_cache_invariants():
+    """What makes full attention uncacheable: S outputs change with the
+    candidate's NS input and with later S rows (both are fixed under the
+    causal mask); with a single layer and no pyramid the layer-0 K / V still
+    do not (they come before any attention)."""
+    layers, d, H, f, N, L0, q = _small()
+    w = rand_weights(layers, d, f, N, seed=93)
+    S, ns = rand_inputs(1, 1, L0, N, d, seed=94)
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    cfg.full_attn = True
+    s1, kv1, n1 = O.full_forward_joint(cfg, w, S, ns)
+    ns2 = ns.clone()
+    ns2[0, 0, N - 1] += 1.0
+    s2, kv2, n2 = O.full_forward_joint(cfg, w, S, ns2)
+    assert not np.allclose(s1, s2)
+    K1, _ = O.kv_layer(cfg, kv1[0, 0], 0)
+    K2, _ = O.kv_layer(cfg, kv2[0, 0], 0)
+    assert np.array_equal(K1, K2)
+    K1b, _ = O.kv_layer(cfg, kv1[0, 0], 1)
+    K2b, _ = O.kv_layer(cfg, kv2[0, 0], 1)
+    assert not np.allclose(K1b, K2b)
+    S3 = S.clone()
+    S3[0, L0 - 1] += 1.0
+    s3, _, _ = O.full_forward_joint(cfg, w, S3, ns)
+    assert not np.allclose(s1[0, 0, 0], s3[0, 0, 0])
 
 
 def _zero_rows(w, key, rows):
