@@ -21,6 +21,14 @@
  *              that tail (L_{l+1} = q_l), in order.
  *   KV cache : S never attends to NS, so the S-side K/V of every layer are a
  *              per-user quantity; candidates are scored against them.
+ *   sparse MoE (cfg->moe_experts = E > 0; the OneTrans-V2 summary page names
+ *              a sparse mixture of experts for capacity, without a recipe):
+ *              the shared S-side FFN of every block becomes E expert FFNs of
+ *              the same shape.  With z = n(h; g2) the FFN's normalised input,
+ *              a linear router gives logits W_r z; the top-k logits (ties to
+ *              the lower expert index) are softmax-ed into gates g_j, and
+ *              y = h + sum_j g_j W2_e(j) GELU(W1_e(j) z).  NS tokens keep
+ *              their private dense FFNs.
  *   full attention (cfg->full_attn = 1; summary page, limitations paragraph:
  *              full attention matches causal attention offline, causal wins
  *              only through the KV cache): every token sees every token of
@@ -78,6 +86,8 @@ typedef struct {
     const double *act_scale;  /* fp8 == 2: [layers][1 + n_ns][4] */
     double *act_amax;         /* optional, same layout: max |input| seen */
     int full_attn;            /* 1: full (non-causal) attention, joint form only */
+    int moe_experts;          /* E > 0: the S-side FFN is a sparse mixture of E experts */
+    int moe_topk;             /* experts per S row (1 or 2) */
 } orc_cfg;
 
 enum { ORC_IN_QKV = 0, ORC_IN_O = 1, ORC_IN_W1 = 2, ORC_IN_W2 = 3 };
@@ -85,6 +95,9 @@ enum { ORC_IN_QKV = 0, ORC_IN_O = 1, ORC_IN_W1 = 2, ORC_IN_W2 = 3 };
 typedef struct {
     const float *Wqkv_s, *Wo_s, *W1_s, *W2_s, *g1_s, *g2_s;
     const float *Wqkv_ns, *Wo_ns, *W1_ns, *W2_ns, *g1_ns, *g2_ns;
+    const float *W_router; /* [layers][E][d] (moe_experts > 0) */
+    const float *W1_moe;   /* [layers][E][ffn][d] */
+    const float *W2_moe;   /* [layers][E][d][ffn] */
 } orc_weights;
 
 /* ------------------------------------------------------------------------- */
@@ -241,6 +254,9 @@ static void attend(const double *q, int hd, int coff, int d,
 typedef struct {
     mat_t qkv, o, w1, w2;
     const float *g1, *g2;
+    int moe_E, moe_k;        /* S set with a mixture of experts: E, top-k */
+    const float *router;     /* [E][d] */
+    mat_t *ew1, *ew2;        /* [E] expert W1 [ffn][d], W2 [d][ffn] */
 } pset_t;
 
 /* Attach the input rule of tensor (layer l, set, input t) to a matrix. */
@@ -267,19 +283,67 @@ static pset_t pset_make(const orc_cfg *c, int l, int set, const float *Wqkv, con
     mat_input(c, &p.w2, l, set, ORC_IN_W2);
     p.g1 = g1;
     p.g2 = g2;
+    p.moe_E = 0;
+    p.moe_k = 0;
+    p.router = NULL;
+    p.ew1 = p.ew2 = NULL;
     return p;
 }
 
 static void pset_free(pset_t *p)
 {
     mat_free(&p->qkv); mat_free(&p->o); mat_free(&p->w1); mat_free(&p->w2);
+    free(p->ew1);
+    free(p->ew2);
 }
 
 static pset_t s_params(const orc_cfg *c, const orc_weights *w, int l)
 {
     long d = c->d, f = c->ffn;
+    if (c->moe_experts > 0) {
+        /* the dense S FFN weights are not used: point them at expert 0 */
+        long E = c->moe_experts;
+        pset_t p = pset_make(c, l, 0, w->Wqkv_s + l * 3 * d * d, w->Wo_s + l * d * d,
+                             w->W1_moe + l * E * f * d, w->W2_moe + l * E * d * f, w->g1_s + l * d,
+                             w->g2_s + l * d);
+        p.moe_E = (int)E;
+        p.moe_k = c->moe_topk;
+        p.router = w->W_router + l * E * d;
+        p.ew1 = (mat_t *)malloc(sizeof(mat_t) * E);
+        p.ew2 = (mat_t *)malloc(sizeof(mat_t) * E);
+        for (long e = 0; e < E; ++e) {
+            p.ew1[e] = mat_plain(w->W1_moe + (l * E + e) * f * d, (int)f, (int)d);
+            p.ew2[e] = mat_plain(w->W2_moe + (l * E + e) * d * f, (int)d, (int)f);
+        }
+        return p;
+    }
     return pset_make(c, l, 0, w->Wqkv_s + l * 3 * d * d, w->Wo_s + l * d * d, w->W1_s + l * f * d,
                      w->W2_s + l * d * f, w->g1_s + l * d, w->g2_s + l * d);
+}
+
+/* Router of a mixture of experts: the top-k of the logits W_r z (ties to
+ * the lower expert index) and their softmax gates. */
+static void moe_route(const pset_t *p, const double *z, int d, int *sel, double *gate)
+{
+    double logit[64];
+    for (int e = 0; e < p->moe_E; ++e) {
+        const float *r = p->router + (long)e * d;
+        double acc = 0.0;
+        for (int k = 0; k < d; ++k) acc += (double)r[k] * z[k];
+        logit[e] = acc;
+    }
+    for (int j = 0; j < p->moe_k; ++j) {
+        int best = -1;
+        for (int e = 0; e < p->moe_E; ++e) {
+            int taken = 0;
+            for (int i = 0; i < j; ++i) taken |= sel[i] == e;
+            if (!taken && (best < 0 || logit[e] > logit[best])) best = e;
+        }
+        sel[j] = best;
+    }
+    double mx = logit[sel[0]], sum = 0.0;
+    for (int j = 0; j < p->moe_k; ++j) { gate[j] = exp(logit[sel[j]] - mx); sum += gate[j]; }
+    for (int j = 0; j < p->moe_k; ++j) gate[j] /= sum;
 }
 
 static pset_t ns_params(const orc_cfg *c, const orc_weights *w, int l, int n)
@@ -289,7 +353,8 @@ static pset_t ns_params(const orc_cfg *c, const orc_weights *w, int l, int n)
                      w->W2_ns + ln * d * f, w->g1_ns + ln * d, w->g2_ns + ln * d);
 }
 
-/* Second half of the block for one row: h = x + a.Wo^T; y = h + W2 GELU(W1 n(h)). */
+/* Second half of the block for one row: h = x + a.Wo^T; y = h + W2 GELU(W1 n(h)),
+ * or with a mixture of experts y = h + sum_j g_j W2_e(j) GELU(W1_e(j) n(h)). */
 static void block_tail(const orc_cfg *c, const pset_t *p, const double *x, const double *a, double *y,
                        double *scr /* >= 3d + 2 ffn */)
 {
@@ -298,6 +363,19 @@ static void block_tail(const orc_cfg *c, const pset_t *p, const double *x, const
     project(&p->o, a, 0, d, t, xq);
     for (int k = 0; k < d; ++k) h[k] = x[k] + t[k];
     rmsnorm(h, p->g2, d, c->eps, z);
+    if (p->moe_E > 0) {
+        int sel[2];
+        double gate[2];
+        moe_route(p, z, d, sel, gate);
+        for (int k = 0; k < d; ++k) y[k] = h[k];
+        for (int j = 0; j < p->moe_k; ++j) {
+            project(&p->ew1[sel[j]], z, 0, f, hid, xq);
+            for (int k = 0; k < f; ++k) hid[k] = gelu(hid[k]);
+            project(&p->ew2[sel[j]], hid, 0, d, t, xq);
+            for (int k = 0; k < d; ++k) y[k] += gate[j] * t[k];
+        }
+        return;
+    }
     project(&p->w1, z, 0, f, hid, xq);
     for (int k = 0; k < f; ++k) hid[k] = gelu(hid[k]);
     project(&p->w2, hid, 0, d, t, xq);
@@ -319,6 +397,10 @@ static int check_cfg(const orc_cfg *c)
 {
     if (c->layers < 1 || c->layers > ORC_MAX_LAYERS || c->d < 1 || c->heads < 1 ||
         c->d % c->heads || c->ffn < 1 || c->n_ns < 0 || c->L0 < 1 || c->fp8 < 0 || c->fp8 > 2)
+        return 1;
+    if (c->moe_experts < 0 || c->moe_experts > 64 ||
+        (c->moe_experts > 0 && (c->moe_topk < 1 || c->moe_topk > 2 || c->moe_topk > c->moe_experts ||
+                                c->fp8)))
         return 1;
     if (c->fp8 == 2) {
         if (!c->act_scale) return 1;

@@ -26,7 +26,8 @@ class _Cfg(C.Structure):
     _fields_ = [("layers", C.c_int), ("d", C.c_int), ("heads", C.c_int), ("ffn", C.c_int),
                 ("n_ns", C.c_int), ("L0", C.c_int), ("q", C.c_int * MAX_LAYERS),
                 ("eps", C.c_double), ("fp8", C.c_int), ("act_scale", C.POINTER(C.c_double)),
-                ("act_amax", C.POINTER(C.c_double)), ("full_attn", C.c_int)]
+                ("act_amax", C.POINTER(C.c_double)), ("full_attn", C.c_int),
+                ("moe_experts", C.c_int), ("moe_topk", C.c_int)]
 
 
 # FP8 rules of the projection inputs (see onetrans_oracle.c): off, one scale
@@ -38,10 +39,13 @@ INPUTS = ("qkv", "o", "w1", "w2")
 
 _WNAMES = ("Wqkv_s", "Wo_s", "W1_s", "W2_s", "g1_s", "g2_s",
            "Wqkv_ns", "Wo_ns", "W1_ns", "W2_ns", "g1_ns", "g2_ns")
+# sparse-MoE S-side FFN (optional): router [layers][E][d], experts
+# W1 [layers][E][ffn][d], W2 [layers][E][d][ffn]
+_MOE_NAMES = ("W_router", "W1_moe", "W2_moe")
 
 
 class _W(C.Structure):
-    _fields_ = [(n, C.POINTER(C.c_float)) for n in _WNAMES]
+    _fields_ = [(n, C.POINTER(C.c_float)) for n in _WNAMES + _MOE_NAMES]
 
 
 _lib = None
@@ -114,6 +118,8 @@ class Config:
     fp8: int = FP8_OFF
     act_scale: object = None
     full_attn: bool = False     # full (non-causal) attention: joint form only
+    moe_experts: int = 0        # E > 0: sparse mixture of E experts as the S-side FFN
+    moe_topk: int = 1           # experts per S row (1 or 2)
 
     @staticmethod
     def of(wl, q=None, fp8=None, act_scale=None) -> "Config":
@@ -141,6 +147,8 @@ class Config:
         c.eps = float(self.eps)
         c.fp8 = int(self.fp8)
         c.full_attn = int(bool(self.full_attn))
+        c.moe_experts = int(self.moe_experts)
+        c.moe_topk = int(self.moe_topk)
         if self.fp8 == FP8_TENSOR:
             if self.act_scale is None:
                 raise ValueError("per-tensor FP8 needs act_scale")
@@ -159,7 +167,7 @@ class Config:
         row)."""
         return Config(self.layers, self.d, self.heads, self.ffn, self.n_ns, self.L0 + delta,
                       [v + delta for v in self.q], self.eps, self.fp8, self.act_scale,
-                      self.full_attn)
+                      self.full_attn, self.moe_experts, self.moe_topk)
 
     def kv_user_elems(self) -> int:
         return int(lib().orc_kv_user_elems(C.byref(self._c())))
@@ -193,6 +201,7 @@ class Weights:
 
     def __init__(self, w: dict):
         self.arrays = {n: _f32(w[n]) for n in _WNAMES}
+        self.arrays.update({n: _f32(w[n]) for n in _MOE_NAMES if w.get(n) is not None})
         self.c = _W(**{n: _fptr(a) for n, a in self.arrays.items()})
 
 

@@ -114,12 +114,27 @@ def _params(w, l, tok: Token):
             w["g1_ns"][l][n], w["g2_ns"][l][n])
 
 
-def run_candidate(w, S_rows, ns_rows, q_sched, heads, eps, fp8=None, full=False):
+def _moe_ffn(w, l, z, topk):
+    """Sparse mixture of experts on the S side: top-k router logits (ties to
+    the lower index), softmax over them, gated sum of the experts' FFNs."""
+    logits = _mv(w["W_router"][l], z)
+    order = sorted(range(len(logits)), key=lambda e: (-logits[e], e))[:topk]
+    mx = logits[order[0]]
+    ex = [math.exp(logits[e] - mx) for e in order]
+    out = [0.0] * len(z)
+    for e, x in zip(order, ex):
+        f = [_gelu(v) for v in _mv(w["W1_moe"][l][e], z)]
+        out = [o + x / sum(ex) * v for o, v in zip(out, _mv(w["W2_moe"][l][e], f))]
+    return out
+
+
+def run_candidate(w, S_rows, ns_rows, q_sched, heads, eps, fp8=None, full=False, moe_topk=0):
     """One candidate: S_rows [L0][d], ns_rows [N][d] (lists).
 
     Returns (S tail rows after the last layer, NS rows, per-layer (K, V) of
     the S tokens).  ``w`` holds nested Python lists; ``fp8`` an Fp8 state or
-    None; ``full``: full (non-causal) attention over the candidate's sequence.
+    None; ``full``: full (non-causal) attention over the candidate's sequence;
+    ``moe_topk`` > 0: the S tokens' FFN is the mixture of experts in ``w``.
     """
     d = len(S_rows[0])
     hd = d // heads
@@ -156,8 +171,11 @@ def run_candidate(w, S_rows, ns_rows, q_sched, heads, eps, fp8=None, full=False)
             _, Wo, W1, W2, _, g2 = _params(w, l, t)
             st = _set(t)
             hrow = [xv + ov for xv, ov in zip(t.x, _proj(Wo, a, fp8, (l, st, 1)))]
-            f = [_gelu(v) for v in _proj(W1, _rms(hrow, g2, eps), fp8, (l, st, 2))]
-            y = [hv + fv for hv, fv in zip(hrow, _proj(W2, f, fp8, (l, st, 3)))]
+            if moe_topk and t.kind == "S":
+                y = [hv + fv for hv, fv in zip(hrow, _moe_ffn(w, l, _rms(hrow, g2, eps), moe_topk))]
+            else:
+                f = [_gelu(v) for v in _proj(W1, _rms(hrow, g2, eps), fp8, (l, st, 2))]
+                y = [hv + fv for hv, fv in zip(hrow, _proj(W2, f, fp8, (l, st, 3)))]
             new_seq.append(Token(t.kind, t.index, y))
         # re-index the S tail 0..q-1 so the next layer's S stream starts at 0
         s_tail = [t for t in new_seq if t.kind == "S"]

@@ -194,6 +194,73 @@ def test_full_attention_breaks_the_cache_invariants():
     assert not np.allclose(s1[0, 0, 0], s3[0, 0, 0])
 
 
+# ----------------------------------------------------------------- sparse MoE
+@pytest.mark.parametrize("topk", [1, 2])
+@pytest.mark.parametrize("case", TINY_CASES[2:5])
+def test_brute_force_matches_oracle_moe(case, topk):
+    """The sparse-MoE S-side FFN (router top-k, softmax gates, gated expert
+    sum) against the brute-force token loop: split and joint forms."""
+    layers, d, H, f, N, L0, q, U, Cn = case
+    w = rand_weights(layers, d, f, N, seed=L0 + d + 3, experts=4)
+    S, ns = rand_inputs(U, Cn, L0, N, d, seed=7 * L0 + N + 3)
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    cfg.moe_experts, cfg.moe_topk = 4, topk
+    kv, s_out = O.encode_user(cfg, w, S)
+    ns_out = O.score_candidates(cfg, w, kv, ns)
+    js, jkv, jns = O.full_forward_joint(cfg, w, S, ns)
+    wl = to_lists(w)
+    for u in range(U):
+        for c in range(Cn):
+            bs, bns, bkv = run_candidate(wl, S[u].double().tolist(), ns[u, c].double().tolist(),
+                                         q, H, 1e-6, moe_topk=topk)
+            np.testing.assert_allclose(s_out[u], np.array(bs), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(js[u, c], np.array(bs), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(ns_out[u, c], np.array(bns), rtol=0, atol=1e-12)
+            for l, (K, V) in enumerate(bkv):
+                Ko, Vo = O.kv_layer(cfg, kv[u], l)
+                np.testing.assert_allclose(Ko, np.array(K), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("topk", [1, 2])
+def test_moe_identical_experts_equal_the_dense_ffn(topk):
+    """Closed form: with every expert equal to the dense FFN the gates sum to
+    one, so the mixture is the dense block whatever the router says."""
+    layers, d, H, f, N, L0, q = _small()
+    w = rand_weights(layers, d, f, N, seed=101, experts=3)
+    w["W1_moe"] = w["W1_s"][:, None].expand(-1, 3, -1, -1).clone()
+    w["W2_moe"] = w["W2_s"][:, None].expand(-1, 3, -1, -1).clone()
+    S, ns = rand_inputs(1, 2, L0, N, d, seed=102)
+    dense = cfg_of(layers, d, H, f, N, L0, q)
+    moe = cfg_of(layers, d, H, f, N, L0, q)
+    moe.moe_experts, moe.moe_topk = 3, topk
+    kv_d, s_d = O.encode_user(dense, w, S)
+    kv_m, s_m = O.encode_user(moe, w, S)
+    np.testing.assert_allclose(s_m, s_d, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(kv_m, kv_d, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(O.score_candidates(moe, w, kv_m, ns),
+                               O.score_candidates(dense, w, kv_d, ns), rtol=0, atol=1e-12)
+
+
+def test_moe_zero_router_picks_the_lowest_experts():
+    """Closed form: a zero router ties every logit, so the top-1 expert is
+    expert 0 (gate 1) and the top-2 are experts 0 and 1 (gates 1/2 each)."""
+    layers, d, H, f, N, L0 = 1, 16, 2, 32, 2, 9
+    w = rand_weights(layers, d, f, N, seed=103, experts=4)
+    w["W_router"] = torch.zeros_like(w["W_router"])
+    S, _ = rand_inputs(1, 1, L0, N, d, seed=104)
+    moe1 = cfg_of(layers, d, H, f, N, L0, [L0])
+    moe1.moe_experts, moe1.moe_topk = 4, 1
+    dense = cfg_of(layers, d, H, f, N, L0, [L0])
+    w0 = dict(w, W1_s=w["W1_moe"][:, 0].clone(), W2_s=w["W2_moe"][:, 0].clone())
+    np.testing.assert_array_equal(O.encode_user(moe1, w, S)[1], O.encode_user(dense, w0, S)[1])
+    moe2 = cfg_of(layers, d, H, f, N, L0, [L0])
+    moe2.moe_experts, moe2.moe_topk = 4, 2
+    w1 = dict(w, W1_s=w["W1_moe"][:, 1].clone(), W2_s=w["W2_moe"][:, 1].clone())
+    y0, y1, y2 = (O.encode_user(c, ww, S)[1] for c, ww in ((dense, w0), (dense, w1), (moe2, w)))
+    # y = h + (f0 + f1) / 2 = (y0 + y1) / 2 (both share h)
+    np.testing.assert_allclose(y2, (y0 + y1) / 2, rtol=0, atol=1e-12)
+
+
 def _zero_rows(w, key, rows):
     w[key] = w[key].clone()
     w[key][..., rows, :] = 0
