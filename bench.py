@@ -526,6 +526,62 @@ def run_serving(name, steps, flush, world, dist, dev, peaks, cands=None, sweep=N
     return out
 
 
+def run_moe_point(name, experts, topk, steps, flush, world, dist, dev, peaks):
+    """The workload's full forward with a sparse mixture of `experts` experts
+    (top-`topk`) as the S-side FFN: router, experts and combine timed with
+    the rest of the step; seeded random router and experts of the dense FFN's
+    shape."""
+    import torch
+
+    import unified_transformer_recommender_onetrans_b200 as ot
+    from synth import WORKLOADS, gen_auto_split_features, gen_s_tokens, gen_weights
+    from unified_transformer_recommender_onetrans_b200.binding import MOE_WEIGHT_NAMES, WEIGHT_NAMES
+
+    wl = WORKLOADS[name]
+    w = gen_weights(wl)
+    g = torch.Generator().manual_seed(11)
+    L, d, f, E = wl.layers, wl.d, wl.ffn, experts
+    w["W_router"] = (torch.randn(L, E, d, generator=g) * d ** -0.5).to(torch.bfloat16)
+    w["W1_moe"] = (torch.randn(L, E, f, d, generator=g) * d ** -0.5).to(torch.bfloat16)
+    w["W2_moe"] = (torch.randn(L, E, d, f, generator=g) * f ** -0.5).to(torch.bfloat16)
+    q = ot.pyramid_schedule(wl.L0, wl.q_end, wl.layers)
+    m = ot.Model(layers=wl.layers, d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns, L0=wl.L0,
+                 q=q, F=wl.F, eps=wl.eps, dtype=wl.dtype, moe_experts=E, moe_topk=topk,
+                 weights={k: w[k].to(dev) for k in WEIGHT_NAMES + MOE_WEIGHT_NAMES})
+    U, C = wl.users, wl.cands
+    S = gen_s_tokens(wl, weights=w).to(dev)
+    x = gen_auto_split_features(wl).to(dev)
+    del w
+    ns = torch.empty(U, C, wl.n_ns, wl.d, dtype=m.storage, device=dev)
+    out_ns = torch.empty_like(ns)
+    s_tail = torch.empty(U, q[-1], wl.d, dtype=m.storage, device=dev)
+    kv = m.new_kv_cache(U)
+    ws = torch.empty(m.workspace_bytes(U, C), dtype=torch.uint8, device=dev)
+
+    def step():
+        m.auto_split(x, ns)
+        m.full_forward(S, ns, kv=kv, out_s_tail=s_tail, out_ns=out_ns, ws=ws)
+
+    for _ in range(5):
+        step()
+    m.poll()
+    ms = _time_device(step, steps, flush, world, dist, dev)
+    m.poll()
+    m.profile(True)
+    step()
+    recs = m.profile_read()
+    m.profile(False)
+    m.close()
+    by_role = {}
+    for r in recs:
+        by_role[r["role"]] = by_role.get(r["role"], 0.0) + r["ms"]
+    flops = sum(r["flops"] for r in recs)
+    return {"workload": name, "moe_experts": E, "moe_topk": topk, "users": U, "cands": C,
+            "full_forward_ms": ms, "full_forward_s_tokens_per_s": world * U * wl.L0 / (ms / 1e3),
+            "algorithmic_tflops": flops / (ms / 1e3) / 1e12,
+            "ms_by_role_serialised": by_role}
+
+
 def run_full_point(name, steps, flush, world, dist, dev, peaks):
     """Auto-Split + full forward of a whole workload batch (C candidates per
     user, S and NS sides in one call), 10 warm-ups + median of `steps` calls."""
@@ -706,6 +762,8 @@ def run_ours(args, wl):
             torch.cuda.empty_cache()
         serving.append(run_full_point("onetrans_l_full", 50, flush, world, dist, dev, peaks))
         torch.cuda.empty_cache()
+        serving.append(run_moe_point("onetrans_s_full", 8, 2, 20, flush, world, dist, dev, peaks))
+        torch.cuda.empty_cache()
 
     # ---- roofline of the dominant kernel (from the live per-launch events)
     by_kind, by_role = {}, {}
@@ -785,6 +843,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-users", type=int, default=8)
     ap.add_argument("--no-serving", action="store_true")
+    ap.add_argument("--users", type=int, default=0,
+                    help="users per GPU instead of the workload's (a small case for profiling)")
     ap.add_argument("--c-sweep", action="store_true",
                     help="also score the serving caches at C = 1, 2, 4, 8, 16, 64, 512")
     args = ap.parse_args()
@@ -792,6 +852,8 @@ def main():
     args.warmup_ref = args.warmup
     from synth import WORKLOADS
     wl = WORKLOADS[args.workload]
+    if args.users > 0:
+        wl = wl.with_(users=args.users)
     if args.impl == "reference":
         run_reference(args, wl)
     else:

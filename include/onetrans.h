@@ -89,13 +89,30 @@ typedef enum { OT_DTYPE_F32 = 0, OT_DTYPE_BF16 = 1, OT_DTYPE_FP8 = 2 } ot_dtype;
  * L_0 = L0, L_{l+1} = q[l]).  F is the Auto-Split input width (0: no
  * Auto-Split weights).  heads must divide d; d / heads must be 64 for the
  * bf16 / fp8 kernels (16, 32 or 64 for fp32); bf16 / fp8: d and ffn
- * multiples of 128 and F a multiple of 64; fp8: d, ffn <= 1536. */
+ * multiples of 128 and F a multiple of 64; fp8: d, ffn <= 1536.
+ * full_attn = 1 selects full (non-causal) attention (summary page,
+ * limitations paragraph: full attention matches causal attention offline;
+ * causal wins only through the KV cache): every token sees every token of
+ * its own candidate's sequence, S and NS alike.  S rows then depend on the
+ * candidate, so such a model runs only ot_full_forward with one candidate
+ * per user (C = 1; give a user with several candidates one row of the batch
+ * per candidate); the cached calls return OT_ERR_UNSUPPORTED.
+ * moe_experts = E > 0 makes the shared S-side FFN of every block a sparse
+ * mixture of E experts (the OneTrans-V2 summary page names a sparse MoE for
+ * capacity without a recipe; this is the library's reading): with z the
+ * FFN's normalised input n(h; g2), a linear router gives E logits
+ * W_router z; the moe_topk (1 or 2) largest, ties to the lower expert index,
+ * are softmax-ed into gates g_j, and y = h + sum_j g_j W2_e GELU(W1_e z),
+ * each expert of the dense FFN's shape.  NS tokens keep their private dense
+ * FFNs.  E <= 64, d <= 256; bf16 or fp32 (not fp8). */
 typedef struct {
     int layers, d, heads, ffn, n_ns, L0;
     int q[OT_MAX_LAYERS];
     int F;
     float eps;
     int dtype; /* ot_dtype */
+    int full_attn; /* 0 = the OneTrans causal mask, 1 = full attention */
+    int moe_experts, moe_topk; /* 0 = dense S-side FFN */
 } ot_config;
 
 /* Weights, device pointers in the storage dtype (float32 for OT_DTYPE_F32,
@@ -105,11 +122,15 @@ typedef struct {
  *   Wqkv_ns [layers][N][3d][d], Wo_ns [layers][N][d][d],
  *   W1_ns [layers][N][ffn][d], W2_ns [layers][N][d][ffn],
  *   g1_ns, g2_ns [layers][N][d];  W_split [N*d][F] (may be NULL if F == 0).
- * g1 / g2 are the RMSNorm gains before attention and before the FFN. */
+ * g1 / g2 are the RMSNorm gains before attention and before the FFN.
+ * Mixture of experts (moe_experts = E > 0; W1_s / W2_s are then unused and
+ * may be NULL): W_router [layers][E][d], W1_moe [layers][E][ffn][d],
+ * W2_moe [layers][E][d][ffn]; NULL for a dense model. */
 typedef struct {
     const void *Wqkv_s, *Wo_s, *W1_s, *W2_s, *g1_s, *g2_s;
     const void *Wqkv_ns, *Wo_ns, *W1_ns, *W2_ns, *g1_ns, *g2_ns;
     const void *W_split;
+    const void *W_router, *W1_moe, *W2_moe;
 } ot_weights;
 
 typedef struct ot_model ot_model;
@@ -312,7 +333,8 @@ typedef enum {
     OT_KIND_GEMM_TC = 0, OT_KIND_GEMM_SIMT = 1, OT_KIND_ATTN_TC = 2, OT_KIND_ATTN_SIMT = 3,
     OT_KIND_GATHER = 4, OT_KIND_QUANT = 5, OT_KIND_FFN_TC = 6 /* fused FFN1 + GELU + FFN2 */,
     OT_KIND_ATTN_NS = 7 /* NS attention, <= 64 query rows per (user, head) */,
-    OT_KIND_KV_GROW = 8 /* old K/V rows into a grown cache (ot_encode_append) */
+    OT_KIND_KV_GROW = 8 /* old K/V rows into a grown cache (ot_encode_append) */,
+    OT_KIND_MOE = 9 /* mixture of experts: routing or combining the rows */
 } ot_kernel_kind;
 
 typedef struct {
@@ -323,7 +345,8 @@ typedef struct {
                       Where the FFN kernel runs (bf16, d of 128 or 256) it also
                       does the output projection, so the S-O / NS-O / O roles
                       appear only on the other paths (FP8, d = 384, kernel
-                      path 2) */
+                      path 2, mixture of experts); 17 S-MoE: the experts'
+                      routing and combining */
     float ms;      /* device time between the two events */
     double flops;  /* algorithmic floating-point operations */
     double bytes;  /* algorithmic HBM bytes */

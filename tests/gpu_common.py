@@ -8,16 +8,18 @@ import torch
 
 import unified_transformer_recommender_onetrans_b200 as ot
 from oracle import oracle as O
-from unified_transformer_recommender_onetrans_b200.binding import WEIGHT_NAMES
+from unified_transformer_recommender_onetrans_b200.binding import MOE_WEIGHT_NAMES, WEIGHT_NAMES
 
 # Max relative L2 error per output tensor (stated workload tolerances).
 TOL = {"f32": 1e-5, "bf16": 2e-2, "fp8": 6e-2}
 
 
-def make_model(w, *, layers, d, heads, ffn, n_ns, L0, q, F=0, dtype="bf16", eps=1e-6):
-    dev = {k: w[k].cuda() for k in WEIGHT_NAMES if k in w and w[k] is not None}
+def make_model(w, *, layers, d, heads, ffn, n_ns, L0, q, F=0, dtype="bf16", eps=1e-6,
+               full_attn=False, moe_experts=0, moe_topk=1):
+    dev = {k: w[k].cuda() for k in WEIGHT_NAMES + MOE_WEIGHT_NAMES if k in w and w[k] is not None}
     return ot.Model(layers=layers, d=d, heads=heads, ffn=ffn, n_ns=n_ns, L0=L0, q=q, F=F,
-                    eps=eps, dtype=dtype, weights=dev)
+                    eps=eps, dtype=dtype, weights=dev, full_attn=full_attn,
+                    moe_experts=moe_experts, moe_topk=moe_topk)
 
 
 def model_of(wl, w, q=None):
@@ -27,7 +29,10 @@ def model_of(wl, w, q=None):
 
 
 def oracle_cfg(m: ot.Model, fp8=False):
-    return O.Config(m.layers, m.d, m.heads, m.ffn, m.n_ns, m.L0, list(m.q), m.eps, fp8)
+    c = O.Config(m.layers, m.d, m.heads, m.ffn, m.n_ns, m.L0, list(m.q), m.eps, fp8)
+    c.full_attn = m.full_attn
+    c.moe_experts, c.moe_topk = m.moe_experts, m.moe_topk
+    return c
 
 
 def kv_errors(m, kv_gpu_users, kv_oracle_users, cfg):

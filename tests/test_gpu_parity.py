@@ -450,3 +450,172 @@ def test_fused_ffn_matches_two_gemm_path(shape):
         assert_within(errs, TOL["bf16"])
         for x, y in zip(a, b):
             assert O.rel_l2(x.double().cpu().numpy(), y.double().cpu().numpy()) < tol
+
+
+# ----------------------------------------------------------------- full (non-causal) attention
+def _full_model(w, path=0, **shapes):
+    m = make_model(w, full_attn=True, **shapes)
+    m.set_wait_limit(TEST_WAIT)
+    m.set_kernel_path(path)
+    return m
+
+
+def _full_errors(m, w, S, ns, s_tail, ns_out, kv, users):
+    cfg = oracle_cfg(m)
+    cfg.full_attn = True
+    js, jkv, jns = O.full_forward_joint(cfg, w, S[users], ns[users])
+    errs = {"s_tail": O.rel_l2(s_tail[users].double().cpu().numpy(), js[:, 0]),
+            "ns_out": O.rel_l2(ns_out[users].double().cpu().numpy(), jns)}
+    errs.update(kv_errors(m, kv[users], jkv[:, 0], cfg))
+    return errs
+
+
+@pytest.mark.parametrize("path", [0, 1, 2], ids=["tcgen05_fused", "cuda_core", "tcgen05_two_gemm"])
+def test_full_attention_parity(path):
+    """Full attention (every token sees its whole sequence, one candidate per
+    user) against the oracle's joint form: the tensor-core path with the S and
+    NS sides in shared launches, the CUDA-core path and the two-GEMM FFN path
+    (layer by layer: both sides' projections, then both attentions)."""
+    shapes = dict(layers=3, d=128, heads=2, ffn=256, n_ns=5, L0=300, q=[300, 170, 37])
+    w = rand_weights(3, 128, 256, 5, seed=111, dtype=torch.bfloat16)
+    S, ns = rand_inputs(4, 1, 300, 5, 128, seed=112, dtype=torch.bfloat16)
+    m = _full_model(w, path, **shapes)
+    s_tail, ns_out, kv = _run_full(m, S.cuda(), ns.cuda())
+    assert_within(_full_errors(m, w, S, ns, s_tail, ns_out, kv, [0, 3]), TOL["bf16"])
+    # the cached calls refuse a full-attention model; several candidates per user too
+    with pytest.raises(ot.OtError) as e:
+        m.encode_user(S.cuda())
+    assert e.value.code == 10
+    with pytest.raises(ot.OtError) as e:
+        m.full_forward(S.cuda(), torch.cat([ns, ns], dim=1).cuda())
+    assert e.value.code == 2
+
+
+def test_full_attention_onetrans_s_shapes():
+    """Full attention at the OneTransS widths (d = 256, 4 heads, 16 NS tokens,
+    a 600 -> 300 pyramid) on sampled users against the oracle."""
+    wl = WORKLOADS["onetrans_s_full"]
+    shapes = dict(layers=2, d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns, L0=600, q=[600, 300])
+    w = rand_weights(2, wl.d, wl.ffn, wl.n_ns, seed=113, dtype=torch.bfloat16)
+    S, ns = rand_inputs(6, 1, 600, wl.n_ns, wl.d, seed=114, dtype=torch.bfloat16)
+    m = _full_model(w, 0, **shapes)
+    s_tail, ns_out, kv = _run_full(m, S.cuda(), ns.cuda())
+    assert_within(_full_errors(m, w, S, ns, s_tail, ns_out, kv, [0, 5]), TOL["bf16"])
+
+
+def test_full_attention_tiny_fp32():
+    """The tiny fp32 block with full attention (CUDA-core kernels) at 1e-5."""
+    wl = WORKLOADS["tiny_fp32"]
+    w = gen_weights(wl)
+    S = gen_s_tokens(wl, weights=w)
+    x = gen_auto_split_features(wl)[:, :1]                 # one candidate
+    q = ot.pyramid_schedule(wl.L0, wl.q_end, wl.layers)
+    m = make_model(w, layers=wl.layers, d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns,
+                   L0=wl.L0, q=q, F=wl.F, eps=wl.eps, dtype="f32", full_attn=True)
+    ns = m.auto_split(x.cuda())
+    s_tail, ns_out, kv = _run_full(m, S.cuda(), ns)
+    cfg = oracle_cfg(m)
+    cfg.full_attn = True
+    ns_o = O.auto_split(x, w["W_split"], wl.n_ns, wl.d)
+    js, jkv, jns = O.full_forward_joint(cfg, w, S, ns_o)
+    errs = {"s_tail": O.rel_l2(s_tail.double().cpu().numpy(), js[:, 0]),
+            "ns_out": O.rel_l2(ns_out.double().cpu().numpy(), jns)}
+    errs.update(kv_errors(m, kv, jkv[:, 0], cfg))
+    assert_within(errs, TOL["f32"])
+
+
+def test_full_attention_mask_probe_bitexact():
+    """The mask probe of the causal test with full attention: every output
+    row has a non-zero in every S column and every NS column of its user."""
+    L0, N, d, q = 100, 8, 128, 60
+    w = rand_weights(1, d, 256, N, seed=5, dtype=torch.bfloat16)
+    eye = torch.eye(d, dtype=torch.bfloat16)
+    for k, shape in (("Wqkv_s", (1, 3 * d, d)), ("Wqkv_ns", (1, N, 3 * d, d))):
+        t = torch.zeros(shape, dtype=torch.bfloat16)
+        t[..., 2 * d:, :] = eye
+        w[k] = t
+    w["g1_s"] = torch.ones_like(w["g1_s"])
+    w["g1_ns"] = torch.ones_like(w["g1_ns"])
+    w["Wo_s"] = eye.expand(1, d, d).clone()
+    w["Wo_ns"] = eye.expand(1, N, d, d).clone()
+    w["W2_s"] = torch.zeros_like(w["W2_s"])
+    w["W2_ns"] = torch.zeros_like(w["W2_ns"])
+    S = torch.zeros(2, L0, d, dtype=torch.bfloat16)
+    S[:, torch.arange(L0), torch.arange(L0)] = 1
+    ns = torch.zeros(2, 1, N, d, dtype=torch.bfloat16)
+    ns[:, 0, torch.arange(N), L0 + torch.arange(N)] = 1
+    want = torch.zeros(d, dtype=torch.bool)
+    want[:L0 + N] = True
+    for path in (0, 1):
+        m = _full_model(w, path, layers=1, d=d, heads=2, ffn=256, n_ns=N, L0=L0, q=[q])
+        s_tail, ns_out, _ = _run_full(m, S.cuda(), ns.cuda())
+        assert torch.equal(s_tail.float().cpu() != 0, want.expand(2, q, d)), path
+        assert torch.equal(ns_out.float().cpu() != 0, want.expand(2, 1, N, d)), path
+
+
+# ----------------------------------------------------------------- sparse mixture of experts
+def _moe_inputs(U, C, L0, N, d, E, seed):
+    """S rows whose router logits are decisive: row t carries a large
+    component on coordinate t % E (its first expert) and a smaller one on a
+    second coordinate (its second expert), and the router reads those
+    coordinates, so no rounding difference between the GPU and the oracle
+    can swap the chosen experts (both sides decide in their own precision)."""
+    S, ns = rand_inputs(U, C, L0, N, d, seed=seed, dtype=torch.float32)
+    t = torch.arange(L0)
+    e1 = t % E
+    e2 = (t + 1 + t // E) % E
+    e2 = torch.where(e2 == e1, (e1 + 1) % E, e2)
+    S[:, t, e1] += 45.0
+    S[:, t, e2] += 22.0
+    return S.to(torch.bfloat16), ns.to(torch.bfloat16)
+
+
+def _moe_weights(layers, d, f, N, E, seed):
+    w = rand_weights(layers, d, f, N, seed=seed, dtype=torch.bfloat16, experts=E)
+    r = torch.zeros(layers, E, d)
+    r[:, torch.arange(E), torch.arange(E)] = 0.3
+    w["W_router"] = r.to(torch.bfloat16)
+    return w
+
+
+@pytest.mark.parametrize("topk", [1, 2])
+@pytest.mark.parametrize("path", [0, 1, 2], ids=["tcgen05_fused", "cuda_core", "tcgen05_two_gemm"])
+def test_moe_parity(path, topk):
+    """The sparse-MoE S-side FFN (router, expert-major rows, the experts' FFN,
+    combine) against the oracle: the fused-FFN path computing only each
+    expert's filled rows, the CUDA-core path and the two-GEMM path; the NS
+    side keeps its dense private FFNs; cached scoring matches the full
+    forward, and a second run is bit-identical (the slots an expert's rows
+    take depend on atomic order, the results must not)."""
+    E = 4
+    shapes = dict(layers=3, d=128, heads=2, ffn=256, n_ns=5, L0=300, q=[300, 170, 37])
+    w = _moe_weights(3, 128, 256, 5, E, seed=121)
+    S, ns = _moe_inputs(3, 4, 300, 5, 128, E, seed=122)
+    m = make_model(w, moe_experts=E, moe_topk=topk, **shapes)
+    m.set_wait_limit(TEST_WAIT)
+    m.set_kernel_path(path)
+    a = _run_full(m, S.cuda(), ns.cuda())
+    errs = _errors_vs_oracle(m, w, S, ns, *a, [0, 2])
+    assert_within(errs, TOL["bf16"])
+    b = _run_full(m, S.cuda(), ns.cuda())
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    kv2, s2 = m.encode_user(S.cuda())
+    sc = m.score_candidates(kv2, ns.cuda())
+    m.poll()
+    assert torch.equal(kv2, a[2]) and torch.equal(s2, a[0]) and torch.equal(sc, a[1])
+
+
+def test_moe_onetrans_s_shapes():
+    """Eight experts, top-2, at the OneTransS widths (d = 256, 4 heads, FFN
+    1024, 16 NS tokens, 600 -> 300 pyramid): sampled users against the
+    oracle."""
+    E = 8
+    wl = WORKLOADS["onetrans_s_full"]
+    shapes = dict(layers=2, d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns, L0=600, q=[600, 300])
+    w = _moe_weights(2, wl.d, wl.ffn, wl.n_ns, E, seed=123)
+    S, ns = _moe_inputs(6, 2, 600, wl.n_ns, wl.d, E, seed=124)
+    m = make_model(w, moe_experts=E, moe_topk=2, **shapes)
+    m.set_wait_limit(TEST_WAIT)
+    a = _run_full(m, S.cuda(), ns.cuda())
+    assert_within(_errors_vs_oracle(m, w, S, ns, *a, [1, 4]), TOL["bf16"])

@@ -28,15 +28,18 @@ _vp, _i, _l, _ll, _sz = C.c_void_p, C.c_int, C.c_long, C.c_longlong, C.c_size_t
 class OtConfig(C.Structure):
     _fields_ = [("layers", C.c_int), ("d", C.c_int), ("heads", C.c_int), ("ffn", C.c_int),
                 ("n_ns", C.c_int), ("L0", C.c_int), ("q", C.c_int * MAX_LAYERS), ("F", C.c_int),
-                ("eps", C.c_float), ("dtype", C.c_int)]
+                ("eps", C.c_float), ("dtype", C.c_int), ("full_attn", C.c_int),
+                ("moe_experts", C.c_int), ("moe_topk", C.c_int)]
 
 
 WEIGHT_NAMES = ("Wqkv_s", "Wo_s", "W1_s", "W2_s", "g1_s", "g2_s", "Wqkv_ns", "Wo_ns", "W1_ns",
                 "W2_ns", "g1_ns", "g2_ns", "W_split")
+# a mixture of experts as the S-side FFN (ot_config.moe_experts > 0)
+MOE_WEIGHT_NAMES = ("W_router", "W1_moe", "W2_moe")
 
 
 class OtWeights(C.Structure):
-    _fields_ = [(n, C.c_void_p) for n in WEIGHT_NAMES]
+    _fields_ = [(n, C.c_void_p) for n in WEIGHT_NAMES + MOE_WEIGHT_NAMES]
 
 
 class OtLaunchRecord(C.Structure):
@@ -45,10 +48,10 @@ class OtLaunchRecord(C.Structure):
 
 
 KINDS = {0: "gemm_tc", 1: "gemm_simt", 2: "attn_tc", 3: "attn_simt", 4: "gather", 5: "quant",
-         6: "ffn_tc", 7: "attn_ns", 8: "kv_grow"}
+         6: "ffn_tc", 7: "attn_ns", 8: "kv_grow", 9: "moe"}
 ROLES = {0: "S_QKV", 1: "S_attn", 2: "S_O", 3: "S_FFN1", 4: "S_FFN2", 5: "NS_QKV", 6: "NS_attn",
          7: "NS_O", 8: "NS_FFN1", 9: "NS_FFN2", 10: "auto_split", 11: "other", 12: "S_FFN",
-         13: "NS_FFN", 14: "O", 15: "FFN", 16: "QKV"}
+         13: "NS_FFN", 14: "O", 15: "FFN", 16: "QKV", 17: "S_MoE"}
 
 SIGNATURES = {
     "ot_model_create": (_i, [C.POINTER(OtConfig), C.POINTER(OtWeights), C.POINTER(_vp)]),
@@ -158,7 +161,7 @@ class Model:
     """
 
     def __init__(self, *, layers, d, heads, ffn, n_ns, L0, q, F=0, eps=1e-6, dtype="bf16",
-                 weights: dict):
+                 weights: dict, full_attn: bool = False, moe_experts: int = 0, moe_topk: int = 1):
         import torch
         if not torch.cuda.is_available():
             raise RuntimeError("the OneTrans library needs a CUDA GPU")
@@ -171,12 +174,17 @@ class Model:
         for i, v in enumerate(self.q):
             cfg.q[i] = int(v)
         cfg.F, cfg.eps, cfg.dtype = F, eps, DTYPES[dtype]
+        cfg.full_attn = int(bool(full_attn))
+        self.full_attn = bool(full_attn)
+        cfg.moe_experts, cfg.moe_topk = int(moe_experts), int(moe_topk)
+        self.moe_experts, self.moe_topk = int(moe_experts), int(moe_topk)
         self._cfg = cfg
-        self._w = {k: weights[k].contiguous() for k in WEIGHT_NAMES if weights.get(k) is not None}
+        self._w = {k: weights[k].contiguous() for k in WEIGHT_NAMES + MOE_WEIGHT_NAMES
+                   if weights.get(k) is not None}
         for k, t in self._w.items():
             if t.dtype != self.storage:
                 raise ValueError(f"weight {k} must be {self.storage}")
-        w = OtWeights(**{k: _ptr(self._w.get(k)) for k in WEIGHT_NAMES})
+        w = OtWeights(**{k: _ptr(self._w.get(k)) for k in WEIGHT_NAMES + MOE_WEIGHT_NAMES})
         h = C.c_void_p()
         check(lib().ot_model_create(C.byref(cfg), C.byref(w), C.byref(h)), "ot_model_create")
         self.handle = h

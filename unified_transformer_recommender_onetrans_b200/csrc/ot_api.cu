@@ -25,6 +25,8 @@
 #include <new>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "ot_internal.h"
 
 struct ot_model {
@@ -37,6 +39,8 @@ struct ot_model {
     void *Wqkv_s, *Wo_s, *W1_s, *W2_s;
     void *Wqkv_ns, *Wo_ns, *W1_ns, *W2_ns;
     void *W_split;
+    // mixture of experts: router, experts' W1 (gain g2 folded), W2
+    void *W_router = nullptr, *W1_moe = nullptr, *W2_moe = nullptr;
     float *sc_qkv_s, *sc_o_s, *sc_1_s, *sc_2_s, *sc_qkv_ns, *sc_o_ns, *sc_1_ns, *sc_2_ns;
     // fp8: per-tensor activation scales [layers][1 + n_ns][4] (device; null =
     // per-row scales), and while ot_fp8_calibrate enqueues, the caller's amax
@@ -145,6 +149,13 @@ ot_status check_config(const ot_config &c)
         return OT_ERR_ARG;
     if (c.dtype != OT_DTYPE_F32 && c.dtype != OT_DTYPE_BF16 && c.dtype != OT_DTYPE_FP8)
         return OT_ERR_DTYPE;
+    if (c.full_attn != 0 && c.full_attn != 1) return OT_ERR_ARG;
+    if (c.moe_experts < 0 || c.moe_experts > 64) return OT_ERR_SHAPE;
+    if (c.moe_experts > 0) {
+        if (c.moe_topk < 1 || c.moe_topk > 2 || c.moe_topk > c.moe_experts) return OT_ERR_ARG;
+        if (c.dtype == OT_DTYPE_FP8) return OT_ERR_DTYPE;
+        if (c.d % 32 || c.d > 256) return OT_ERR_SHAPE;
+    }
     if (c.d % c.heads) return OT_ERR_SHAPE;
     int L = c.L0;
     for (int l = 0; l < c.layers; ++l) {
@@ -189,10 +200,22 @@ size_t fp8_ws_bytes(const ot_config &c, long long rows)
     return bytes_of(rows * (c.d > c.ffn ? c.d : c.ffn), 1) + bytes_of(rows, 4);
 }
 
+// mixture of experts: expert-major rows in (Hp) and out (Yp), the experts'
+// hidden (two-GEMM paths), routes (int64) and gates of 2 choices per row,
+// the experts' row counts
+size_t moe_ws_bytes(const ot_config &c, long long rows, int esz)
+{
+    if (c.moe_experts <= 0) return 0;
+    const long long er = rows * c.moe_experts;
+    return 2 * bytes_of(er * c.d, esz) + bytes_of(er * c.ffn, esz) + bytes_of(rows * 2, 8) +
+           bytes_of(rows * 2, 4) + bytes_of(c.moe_experts, 4);
+}
+
 size_t encode_ws_bytes(const ot_config &c, int U, int esz)
 {
     long long rows = static_cast<long long>(U) * c.L0;
-    return 5 * bytes_of(rows * c.d, esz) + bytes_of(rows * c.ffn, esz) + fp8_ws_bytes(c, rows);
+    return 5 * bytes_of(rows * c.d, esz) + bytes_of(rows * c.ffn, esz) + fp8_ws_bytes(c, rows) +
+           moe_ws_bytes(c, rows, esz);
 }
 
 size_t score_ws_bytes(const ot_config &c, int U, int C, int esz)
@@ -204,7 +227,8 @@ size_t score_ws_bytes(const ot_config &c, int U, int C, int esz)
 enum { ROLE_S_QKV = 0, ROLE_S_ATTN, ROLE_S_O, ROLE_S_FFN1, ROLE_S_FFN2, ROLE_NS_QKV, ROLE_NS_ATTN,
        ROLE_NS_O, ROLE_NS_FFN1, ROLE_NS_FFN2, ROLE_AUTO_SPLIT, ROLE_OTHER, ROLE_S_FFN, ROLE_NS_FFN,
        // one launch for the S and NS sides of a layer (full forward)
-       ROLE_O, ROLE_FFN, ROLE_QKV };
+       ROLE_O, ROLE_FFN, ROLE_QKV,
+       ROLE_S_MOE }; // routing / combining the rows of a mixture of experts
 
 cudaEvent_t pooled_event(ot_model *m)
 {
@@ -218,11 +242,23 @@ cudaEvent_t pooled_event(ot_model *m)
     return e;
 }
 
-// Launch `fn` bracketed by profiling events when profiling is on.
+// Name of a launch role for NVTX ranges (the same order as ot_launch_record::role).
+const char *role_name(int role)
+{
+    static const char *names[] = {"S-QKV", "S-attn", "S-O", "S-FFN1", "S-FFN2", "NS-QKV", "NS-attn",
+                                  "NS-O", "NS-FFN1", "NS-FFN2", "Auto-Split", "other", "S-FFN",
+                                  "NS-FFN", "O", "FFN", "QKV", "S-MoE"};
+    return role >= 0 && role <= ROLE_S_MOE ? names[role] : "launch";
+}
+
+// Launch `fn` bracketed by profiling events when profiling is on, inside an
+// NVTX range named for its role (free when no tool is attached; a profiler
+// timeline then shows which step of the block each kernel is).
 template <typename F>
 ot_status profiled(ot_model *m, cudaStream_t s, int kind, int role, double flops, double bytes,
                    F fn)
 {
+    nvtxRangePushA(role_name(role));
     cudaEvent_t e0 = nullptr, e1 = nullptr;
     const bool prof = m->profiling && m->recs.size() < (1u << 16);
     if (prof) {
@@ -236,6 +272,7 @@ ot_status profiled(ot_model *m, cudaStream_t s, int kind, int role, double flops
         cudaEventRecord(e1, s);
         m->recs.push_back(ot_model::Rec{kind, role, flops, bytes, e0, e1});
     }
+    nvtxRangePop();
     return e == cudaSuccess ? OT_OK : OT_ERR_CUDA;
 }
 
@@ -285,17 +322,21 @@ void attn_cost(const ot_model *m, const AttnArgs &a, double &flops, double &byte
 {
     const double L = a.L, nq = a.nq, N = a.N, U = a.U, esz = m->esz;
     double pairs; // visible (query, key) pairs per user and head
-    if (a.mode == 0)
+    if (a.full)
+        pairs = a.mode == 0 ? nq * (L + a.nkn) : nq * (L + N);
+    else if (a.mode == 0)
         pairs = nq * (L - nq) + nq * (nq + 1) / 2;
     else
         pairs = (nq / N) * (N * L + N * (N + 1) / 2);
     flops += 4.0 * a.hd * pairs * a.H * U;
-    bytes += esz * U * a.d * (2 * nq + 2 * L + (a.mode == 1 ? 2 * nq : 0));
+    bytes += esz * U * a.d * (2 * nq + 2 * L + ((a.mode == 1 || a.full) ? 2.0 * a.nkn : 0.0));
 }
 
 ot_status attn(ot_model *m, AttnArgs &a, cudaStream_t s)
 {
     a.wait = WaitCtl{m->err, m->wait_limit};
+    if (a.mode == 1) a.nkn = a.nq;
+    if (a.mode == 0 && a.full && (!a.KN || !a.VN || a.nkn < 1)) return OT_ERR_ARG;
     a.dtype = m->cfg.dtype;
     const bool simt = m->cfg.dtype == OT_DTYPE_F32 || m->path == 1;
     double flops = 0, bytes = 0;
@@ -341,9 +382,12 @@ FfnArgs ffn_args(const ot_model *m, int M, int G, const void *H, RowMap h_map, c
     return a;
 }
 
-void ffn_cost(const FfnArgs &a, double &flops, double &bytes)
+// rows_override > 0: the rows actually computed (a mixture's routed rows,
+// not every slot of every expert)
+void ffn_cost(const FfnArgs &a, double &flops, double &bytes, double rows_override = 0)
 {
-    const double rows = static_cast<double>(a.M) * a.G, d = a.D, f = a.F;
+    const double rows = rows_override > 0 ? rows_override : static_cast<double>(a.M) * a.G,
+                 d = a.D, f = a.F;
     flops += 4.0 * rows * d * f;
     bytes += 2.0 * (2.0 * rows * d + 2.0 * a.G * d * f); // H in, Y out, W1 + W2 once
     if (a.fuse_o) {
@@ -367,10 +411,10 @@ FfnArgs ffn_o_args(const ot_model *m, int M, int G, const void *A, RowMap a_map,
     return a;
 }
 
-ot_status ffn_run(ot_model *m, const FfnArgs &a, cudaStream_t s, int role)
+ot_status ffn_run(ot_model *m, const FfnArgs &a, cudaStream_t s, int role, double routed_rows = 0)
 {
     double flops = 0, bytes = 0;
-    if (m->profiling) ffn_cost(a, flops, bytes);
+    if (m->profiling) ffn_cost(a, flops, bytes, routed_rows);
     return profiled(m, s, OT_KIND_FFN_TC, role, flops, bytes, [&] { return launch_ffn_tc(a, s); });
 }
 
@@ -481,52 +525,112 @@ EpiSeg seg_of(void *out, long long ld, int lo, int hi, RowMap map)
     return s;
 }
 
-// S-side of every layer for U users.  X0: [U][L0][d].  s_out may be null.
-// S-side of every layer for U users.  delta > 0 appends: X0 holds only the
-// delta new rows per user, and only they run through each layer (the last
-// delta of its L_l rows, all of them queries), attending to the cached K/V
-// of the old rows, which the caller has already placed in `kv`; their own
-// K/V go after the old rows.
+// Attention arguments shared by both sides of a layer.
+AttnArgs attn_base(const ot_config &c, int mode, int U, int L, int nq, const void *Q,
+                   const void *K, const void *V, void *O)
+{
+    AttnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.mode = mode;
+    a.U = U;
+    a.H = c.heads;
+    a.hd = c.d / c.heads;
+    a.d = c.d;
+    a.L = L;
+    a.nq = nq;
+    a.N = c.n_ns;
+    a.Q = Q;
+    a.KS = K;
+    a.VS = V;
+    a.s_ustride = kv_user_elems(c);
+    a.O = O;
+    a.scale = 1.0f / sqrtf(static_cast<float>(a.hd));
+    a.full = c.full_attn;
+    return a;
+}
+
+// S-side of every layer for U users, one layer at a time: qkv(l), then
+// rest(l) (attention, output projection, FFN).  X0: [U][L0][d]; s_out may
+// be null.  delta > 0 appends: X0 holds only the delta new rows per user,
+// and only they run through each layer (the last delta of its L_l rows, all
+// of them queries), attending to the cached K/V of the old rows, which the
+// caller has already placed in `kv`; their own K/V go after the old rows.
 // full_last: run the whole last layer even when s_out is null (its output
 // goes to a workspace buffer; calibration needs its projections).
-ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, Ws ws,
-                     cudaStream_t st, cudaEvent_t *kv_ready = nullptr, int delta = 0,
-                     bool full_last = false)
-{
-    const ot_config &c = m->cfg;
-    const int d = c.d, f = c.ffn, esz = m->esz;
-    const bool fp8 = c.dtype == OT_DTYPE_FP8;
-    const int wesz = fp8 ? 1 : esz; // bytes per weight element as the GEMM reads it
-    const long long rows0 = static_cast<long long>(U) * (delta ? delta : c.L0);
-    void *Xb[2] = {ws.take(rows0 * d), ws.take(rows0 * d)};
-    void *Qb = ws.take(rows0 * d), *Ab = ws.take(rows0 * d), *Hb = ws.take(rows0 * d);
-    void *hid = ws.take(rows0 * f);
-    if (!Xb[0] || !Xb[1] || !Qb || !Ab || !Hb || !hid) return OT_ERR_WORKSPACE_TOO_SMALL;
+// Full attention: ns_K / ns_V / ns_rows name the NS keys and values of the
+// layer (one candidate per user) that the S rows also see.
+struct EncodeRun {
+    ot_model *m;
+    int U;
+    void *kv, *s_out;
+    cudaStream_t st;
+    cudaEvent_t *kv_ready;
+    int delta;
+    bool full_last;
+    void *Xb[2], *Qb, *Ab, *Hb, *hid;
     Fp8Scratch f8{nullptr, nullptr};
-    if (fp8) {
-        Ws w1{ws.p, ws.left, 1};
-        f8.q = static_cast<uint8_t *>(w1.take(rows0 * (d > f ? d : f)));
-        Ws w4{w1.p, w1.left, 4};
-        f8.s = static_cast<float *>(w4.take(rows0));
-        if (!f8.q || !f8.s) return OT_ERR_WORKSPACE_TOO_SMALL;
+    // mixture of experts: expert-major rows, hidden, routes, gates, counts
+    void *Hp = nullptr, *Yp = nullptr, *ehid = nullptr;
+    long long *route = nullptr;
+    float *gate = nullptr;
+    int *counts = nullptr;
+    const void *X;
+    bool done = false; // the last layer ran its K/V projection only
+    const void *ns_K = nullptr, *ns_V = nullptr;
+    int ns_rows = 0;
+
+    ot_status init(const void *X0, Ws ws)
+    {
+        const ot_config &c = m->cfg;
+        const long long rows0 = static_cast<long long>(U) * (delta ? delta : c.L0);
+        Xb[0] = ws.take(rows0 * c.d);
+        Xb[1] = ws.take(rows0 * c.d);
+        Qb = ws.take(rows0 * c.d);
+        Ab = ws.take(rows0 * c.d);
+        Hb = ws.take(rows0 * c.d);
+        hid = ws.take(rows0 * c.ffn);
+        if (!Xb[0] || !Xb[1] || !Qb || !Ab || !Hb || !hid) return OT_ERR_WORKSPACE_TOO_SMALL;
+        if (c.dtype == OT_DTYPE_FP8) {
+            Ws w1{ws.p, ws.left, 1};
+            f8.q = static_cast<uint8_t *>(w1.take(rows0 * (c.d > c.ffn ? c.d : c.ffn)));
+            Ws w4{w1.p, w1.left, 4};
+            f8.s = static_cast<float *>(w4.take(rows0));
+            if (!f8.q || !f8.s) return OT_ERR_WORKSPACE_TOO_SMALL;
+        }
+        if (c.moe_experts > 0) {
+            const long long er = rows0 * c.moe_experts;
+            Hp = ws.take(er * c.d);
+            Yp = ws.take(er * c.d);
+            ehid = ws.take(er * c.ffn);
+            Ws w8{ws.p, ws.left, 8};
+            route = static_cast<long long *>(w8.take(rows0 * 2));
+            Ws w4{w8.p, w8.left, 4};
+            gate = static_cast<float *>(w4.take(rows0 * 2));
+            counts = static_cast<int *>(w4.take(c.moe_experts));
+            if (!Hp || !Yp || !ehid || !route || !gate || !counts) return OT_ERR_WORKSPACE_TOO_SMALL;
+        }
+        X = X0;
+        return OT_OK;
     }
-    const long long ustride = kv_user_elems(c);
-    const void *X = X0;
-    ot_status r;
-    for (int l = 0; l < c.layers; ++l) {
-        const int L = rows_at(c, l);
-        const int n = delta ? delta : L;        // rows run through this layer (the last n of L)
-        const int q = delta ? delta : c.q[l];   // their query tail
+    int rows(int l) const { return delta ? delta : rows_at(m->cfg, l); }   // rows run through layer l
+    int tail(int l) const { return delta ? delta : m->cfg.q[l]; }          // their query tail
+    char *K(int l) const { return at(kv, kv_layer_off(m->cfg, l), m->esz); }
+    char *V(int l) const { return K(l) + static_cast<long long>(rows_at(m->cfg, l)) * m->cfg.d * m->esz; }
+
+    // 1. QKV (or KV only): RMSNorm1 + shared projection; K/V into the cache
+    ot_status qkv(int l)
+    {
+        const ot_config &c = m->cfg;
+        const int d = c.d, esz = m->esz, L = rows_at(c, l), n = rows(l), q = tail(l);
+        const bool fp8 = c.dtype == OT_DTYPE_FP8;
+        const int wesz = fp8 ? 1 : esz; // bytes per weight element as the GEMM reads it
         const bool last = l == c.layers - 1;
         // the S tail of the last layer is unused
         const bool kv_only = last && s_out == nullptr && !full_last;
-        char *K = at(kv, kv_layer_off(c, l), esz);
-        char *V = K + static_cast<long long>(L) * d * esz;
-        const RowMap cache_map{n, ustride / d, L - n, 0, 0};
+        const RowMap cache_map{n, kv_user_elems(c) / d, L - n, 0, 0};
         const void *g1 = fp8 ? at(m->g1_s, static_cast<long long>(l) * d, esz) : nullptr;
-        const void *g2 = fp8 ? at(m->g2_s, static_cast<long long>(l) * d, esz) : nullptr;
-        // 1. QKV (or KV only): RMSNorm1 + shared projection; K/V into the cache
         GemmArgs g = gemm_base(c, U * n, kv_only ? 2 * d : 3 * d, d, 1);
+        ot_status r;
         if ((r = projection(m, g, X, d, rowmap_identity(),
                             at(m->Wqkv_s, static_cast<long long>(l) * 3 * d * d + (kv_only ? d * d : 0), wesz),
                             3LL * d * d, fp8 ? m->sc_qkv_s + l : nullptr, g1, d, true, f8, st, l, 0,
@@ -534,36 +638,42 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
             return r;
         if (kv_only) {
             g.nseg = 2;
-            g.seg[0] = seg_of(K, d, 0, d, cache_map);
-            g.seg[1] = seg_of(V, d, d, 2 * d, cache_map);
+            g.seg[0] = seg_of(K(l), d, 0, d, cache_map);
+            g.seg[1] = seg_of(V(l), d, d, 2 * d, cache_map);
         } else {
             g.nseg = 3;
             g.seg[0] = seg_of(Qb, d, 0, d, RowMap{n, q, -(n - q), 0, n - q});
-            g.seg[1] = seg_of(K, d, d, 2 * d, cache_map);
-            g.seg[2] = seg_of(V, d, 2 * d, 3 * d, cache_map);
+            g.seg[1] = seg_of(K(l), d, d, 2 * d, cache_map);
+            g.seg[2] = seg_of(V(l), d, 2 * d, 3 * d, cache_map);
         }
         if ((r = gemm(m, g, st, ROLE_S_QKV)) != OT_OK) return r;
         if (kv_ready && cudaEventRecord(kv_ready[l], st) != cudaSuccess) return OT_ERR_CUDA;
-        if (kv_only) break;
-        // 2. attention over the tail
-        AttnArgs at_;
-        memset(&at_, 0, sizeof(at_));
-        at_.mode = 0;
-        at_.U = U;
-        at_.H = c.heads;
-        at_.hd = d / c.heads;
-        at_.d = d;
-        at_.L = L;
-        at_.nq = q;
-        at_.N = c.n_ns;
-        at_.Q = Qb;
-        at_.KS = K;
-        at_.VS = V;
-        at_.s_ustride = ustride;
-        at_.O = Ab;
-        at_.scale = 1.0f / sqrtf(static_cast<float>(at_.hd));
+        done = kv_only;
+        return OT_OK;
+    }
+
+    // 2. attention over the tail, 3. O projection + residual, 4. FFN
+    ot_status rest(int l)
+    {
+        if (done) return OT_OK;
+        const ot_config &c = m->cfg;
+        const int d = c.d, f = c.ffn, esz = m->esz, n = rows(l), q = tail(l);
+        const bool fp8 = c.dtype == OT_DTYPE_FP8;
+        const int wesz = fp8 ? 1 : esz;
+        const bool last = l == c.layers - 1;
+        const void *g2 = fp8 ? at(m->g2_s, static_cast<long long>(l) * d, esz) : nullptr;
+        AttnArgs at_ = attn_base(c, 0, U, rows_at(c, l), q, Qb, K(l), V(l), Ab);
+        at_.KN = ns_K;
+        at_.VN = ns_V;
+        at_.nkn = ns_rows;
+        ot_status r;
         if ((r = attn(m, at_, st)) != OT_OK) return r;
         void *Xn = (last && s_out) ? s_out : Xb[l & 1];
+        if (c.moe_experts > 0) {
+            if ((r = moe_ffn(l, Xn)) != OT_OK) return r;
+            X = Xn;
+            return OT_OK;
+        }
         if (use_fused_ffn(m)) {
             // 3 + 4 in one launch: O projection + residual from the tail rows
             // of the layer input, RMSNorm2, W1, GELU, W2, residual
@@ -575,10 +685,10 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
                                           rowmap_identity());
             if ((r = ffn_run(m, fa, st, ROLE_S_FFN)) != OT_OK) return r;
             X = Xn;
-            continue;
+            return OT_OK;
         }
         // 3. O projection + residual from the tail rows of the layer input
-        g = gemm_base(c, U * q, d, d, 1);
+        GemmArgs g = gemm_base(c, U * q, d, d, 1);
         if ((r = projection(m, g, Ab, d, rowmap_identity(),
                             at(m->Wo_s, static_cast<long long>(l) * d * d, wesz),
                             static_cast<long long>(d) * d, fp8 ? m->sc_o_s + l : nullptr, nullptr, 0,
@@ -613,125 +723,266 @@ ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, 
         g.seg[0] = seg_of(Xn, d, 0, d, rowmap_identity());
         if ((r = gemm(m, g, st, ROLE_S_FFN2)) != OT_OK) return r;
         X = Xn;
+        return OT_OK;
     }
-    return OT_OK;
+
+    // 3. O projection + residual into H, then the mixture of experts: route
+    // every row to its top-k experts (rows copied expert-major), the experts'
+    // FFN (Yp = h + FFN_e(n(h)) per slot), combine into Xn
+    ot_status moe_ffn(int l, void *Xn)
+    {
+        const ot_config &c = m->cfg;
+        const int d = c.d, f = c.ffn, esz = m->esz, n = rows(l), q = tail(l), E = c.moe_experts;
+        const long long cap = static_cast<long long>(U) * q; // an expert takes at most every row
+        GemmArgs g = gemm_base(c, U * q, d, d, 1);
+        ot_status r;
+        if ((r = projection(m, g, Ab, d, rowmap_identity(), at(m->Wo_s, static_cast<long long>(l) * d * d, esz),
+                            static_cast<long long>(d) * d, nullptr, nullptr, 0, false, f8, st, l, 0, IN_O)) !=
+            OT_OK)
+            return r;
+        g.res = X;
+        g.res_ld = d;
+        g.res_map = RowMap{q, n, n - q, 0, 0};
+        g.nseg = 1;
+        g.seg[0] = seg_of(Hb, d, 0, d, rowmap_identity());
+        if ((r = gemm(m, g, st, ROLE_S_O)) != OT_OK) return r;
+        if (cudaMemsetAsync(counts, 0, sizeof(int) * E, st) != cudaSuccess) return OT_ERR_CUDA;
+        MoeRouteArgs ra;
+        memset(&ra, 0, sizeof(ra));
+        ra.rows = cap;
+        ra.d = d;
+        ra.E = E;
+        ra.topk = c.moe_topk;
+        ra.dtype = c.dtype;
+        ra.eps = c.eps;
+        ra.H = Hb;
+        ra.gain = at(m->g2_s, static_cast<long long>(l) * d, esz);
+        ra.Wr = at(m->W_router, static_cast<long long>(l) * E * d, esz);
+        ra.Hp = Hp;
+        ra.cap = cap;
+        ra.counts = counts;
+        ra.route = route;
+        ra.gate = gate;
+        const double rbytes = static_cast<double>(cap) * d * esz * (1 + c.moe_topk) +
+                              static_cast<double>(E) * d * esz;
+        if ((r = profiled(m, st, OT_KIND_MOE, ROLE_S_MOE, 2.0 * cap * d * E, rbytes,
+                          [&] { return launch_moe_route(ra, st); })) != OT_OK)
+            return r;
+        const RowMap seg_rows{1, 1, 0, cap, 0}; // expert e, slot s -> row e * cap + s
+        const char *W1e = at(m->W1_moe, static_cast<long long>(l) * E * f * d, esz);
+        const char *W2e = at(m->W2_moe, static_cast<long long>(l) * E * d * f, esz);
+        if (use_fused_ffn(m)) {
+            // the experts' FFN in one launch: group = expert, only its filled rows
+            FfnArgs fa = ffn_args(m, static_cast<int>(cap), E, Hp, seg_rows, W1e, W2e, Yp, seg_rows);
+            fa.group_rows = counts;
+            if ((r = ffn_run(m, fa, st, ROLE_S_FFN, static_cast<double>(cap) * c.moe_topk)) != OT_OK) return r;
+        } else {
+            // two grouped GEMMs over every slot of every expert
+            g = gemm_base(c, static_cast<int>(cap), f, d, E);
+            if ((r = projection(m, g, Hp, d, seg_rows, W1e, static_cast<long long>(f) * d, nullptr, nullptr, 0,
+                                true, f8, st)) != OT_OK)
+                return r;
+            g.gelu = 1;
+            g.nseg = 1;
+            g.seg[0] = seg_of(ehid, f, 0, f, seg_rows);
+            if ((r = gemm(m, g, st, ROLE_S_FFN1)) != OT_OK) return r;
+            g = gemm_base(c, static_cast<int>(cap), d, f, E);
+            if ((r = projection(m, g, ehid, f, seg_rows, W2e, static_cast<long long>(d) * f, nullptr, nullptr, 0,
+                                false, f8, st)) != OT_OK)
+                return r;
+            g.res = Hp;
+            g.res_ld = d;
+            g.res_map = seg_rows;
+            g.nseg = 1;
+            g.seg[0] = seg_of(Yp, d, 0, d, seg_rows);
+            if ((r = gemm(m, g, st, ROLE_S_FFN2)) != OT_OK) return r;
+        }
+        MoeCombineArgs ca;
+        memset(&ca, 0, sizeof(ca));
+        ca.rows = cap;
+        ca.d = d;
+        ca.topk = c.moe_topk;
+        ca.dtype = c.dtype;
+        ca.H = Hb;
+        ca.Yp = Yp;
+        ca.Y = Xn;
+        ca.route = route;
+        ca.gate = gate;
+        const double cbytes = static_cast<double>(cap) * d * esz * (2 + c.moe_topk);
+        return profiled(m, st, OT_KIND_MOE, ROLE_S_MOE, 0.0, cbytes, [&] { return launch_moe_combine(ca, st); });
+    }
+};
+
+ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, Ws ws,
+                     cudaStream_t st, cudaEvent_t *kv_ready = nullptr, int delta = 0,
+                     bool full_last = false)
+{
+    EncodeRun e{m, U, kv, s_out, st, kv_ready, delta, full_last};
+    ot_status r = e.init(X0, ws);
+    for (int l = 0; r == OT_OK && l < m->cfg.layers && !e.done; ++l)
+        if ((r = e.qkv(l)) == OT_OK) r = e.rest(l);
+    return r;
 }
 
-// NS-side of every layer: U users x C candidates, N tokens each, against kv.
-// out may be null (calibration): the last layer then writes a workspace buffer.
-ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, void *out, Ws ws,
-                    cudaStream_t st, cudaEvent_t *kv_ready = nullptr)
-{
-    const ot_config &c = m->cfg;
-    const int d = c.d, f = c.ffn, N = c.n_ns, esz = m->esz;
-    const bool fp8 = c.dtype == OT_DTYPE_FP8;
-    const int wesz = fp8 ? 1 : esz;
-    const int Mc = U * C;
-    const long long R = static_cast<long long>(Mc) * N;
-    void *Xb[2] = {ws.take(R * d), ws.take(R * d)};
-    void *Qn = ws.take(R * d), *Kn = ws.take(R * d), *Vn = ws.take(R * d);
-    void *An = ws.take(R * d), *Hn = ws.take(R * d), *hid = ws.take(R * f);
-    if (!Xb[0] || !Xb[1] || !Qn || !Kn || !Vn || !An || !Hn || !hid)
-        return OT_ERR_WORKSPACE_TOO_SMALL;
+// NS-side of every layer, one layer at a time (qkv(l), then rest(l)): U
+// users x C candidates, N tokens each, against the S K/V in kv.  out may be
+// null (calibration): the last layer then writes a workspace buffer.
+struct ScoreRun {
+    ot_model *m;
+    const void *kv;
+    int U, C;
+    void *out;
+    cudaStream_t st;
+    cudaEvent_t *kv_ready;
+    void *Xb[2], *Qn, *Kn, *Vn, *An, *Hn, *hid;
     Fp8Scratch f8{nullptr, nullptr};
-    if (fp8) {
-        Ws w1{ws.p, ws.left, 1};
-        f8.q = static_cast<uint8_t *>(w1.take(R * (d > f ? d : f)));
-        Ws w4{w1.p, w1.left, 4};
-        f8.s = static_cast<float *>(w4.take(R));
-        if (!f8.q || !f8.s) return OT_ERR_WORKSPACE_TOO_SMALL;
+    const void *X;
+
+    ot_status init(const void *ns, Ws ws)
+    {
+        const ot_config &c = m->cfg;
+        const long long R = static_cast<long long>(U) * C * c.n_ns;
+        Xb[0] = ws.take(R * c.d);
+        Xb[1] = ws.take(R * c.d);
+        Qn = ws.take(R * c.d);
+        Kn = ws.take(R * c.d);
+        Vn = ws.take(R * c.d);
+        An = ws.take(R * c.d);
+        Hn = ws.take(R * c.d);
+        hid = ws.take(R * c.ffn);
+        if (!Xb[0] || !Xb[1] || !Qn || !Kn || !Vn || !An || !Hn || !hid)
+            return OT_ERR_WORKSPACE_TOO_SMALL;
+        if (c.dtype == OT_DTYPE_FP8) {
+            Ws w1{ws.p, ws.left, 1};
+            f8.q = static_cast<uint8_t *>(w1.take(R * (c.d > c.ffn ? c.d : c.ffn)));
+            Ws w4{w1.p, w1.left, 4};
+            f8.s = static_cast<float *>(w4.take(R));
+            if (!f8.q || !f8.s) return OT_ERR_WORKSPACE_TOO_SMALL;
+        }
+        X = ns;
+        return OT_OK;
     }
-    const long long ustride = kv_user_elems(c);
-    const RowMap grp{1, N, 0, 1, 0}; // candidate m, position g -> row m*N + g
-    const void *X = ns;
-    ot_status r;
-    for (int l = 0; l < c.layers; ++l) {
-        const int L = rows_at(c, l);
-        const bool last = l == c.layers - 1;
-        const char *K = at(kv, kv_layer_off(c, l), esz);
-        const char *V = K + static_cast<long long>(L) * d * esz;
+    RowMap grp() const { return RowMap{1, m->cfg.n_ns, 0, 1, 0}; } // candidate m, position g -> row m*N + g
+
+    ot_status qkv(int l)
+    {
+        const ot_config &c = m->cfg;
+        const int d = c.d, N = c.n_ns, esz = m->esz;
+        const bool fp8 = c.dtype == OT_DTYPE_FP8;
+        const int wesz = fp8 ? 1 : esz;
         const long long lN = static_cast<long long>(l) * N;
         if (kv_ready && cudaStreamWaitEvent(st, kv_ready[l], 0) != cudaSuccess) return OT_ERR_CUDA;
         const void *g1 = fp8 ? at(m->g1_ns, lN * d, esz) : nullptr;
-        const void *g2 = fp8 ? at(m->g2_ns, lN * d, esz) : nullptr;
-        GemmArgs g = gemm_base(c, Mc, 3 * d, d, N);
-        if ((r = projection(m, g, X, d, grp, at(m->Wqkv_ns, lN * 3 * d * d, wesz), 3LL * d * d,
+        GemmArgs g = gemm_base(c, U * C, 3 * d, d, N);
+        ot_status r;
+        if ((r = projection(m, g, X, d, grp(), at(m->Wqkv_ns, lN * 3 * d * d, wesz), 3LL * d * d,
                             fp8 ? m->sc_qkv_ns + lN : nullptr, g1, d, true, f8, st, l, 1, IN_QKV)) != OT_OK)
             return r;
         g.nseg = 3;
-        g.seg[0] = seg_of(Qn, d, 0, d, grp);
-        g.seg[1] = seg_of(Kn, d, d, 2 * d, grp);
-        g.seg[2] = seg_of(Vn, d, 2 * d, 3 * d, grp);
-        if ((r = gemm(m, g, st, ROLE_NS_QKV)) != OT_OK) return r;
-        AttnArgs at_;
-        memset(&at_, 0, sizeof(at_));
-        at_.mode = 1;
-        at_.U = U;
-        at_.H = c.heads;
-        at_.hd = d / c.heads;
-        at_.d = d;
-        at_.L = L;
-        at_.nq = C * N;
-        at_.N = N;
-        at_.Q = Qn;
-        at_.KS = K;
-        at_.VS = V;
-        at_.s_ustride = ustride;
+        g.seg[0] = seg_of(Qn, d, 0, d, grp());
+        g.seg[1] = seg_of(Kn, d, d, 2 * d, grp());
+        g.seg[2] = seg_of(Vn, d, 2 * d, 3 * d, grp());
+        return gemm(m, g, st, ROLE_NS_QKV);
+    }
+
+    ot_status rest(int l)
+    {
+        const ot_config &c = m->cfg;
+        const int d = c.d, f = c.ffn, N = c.n_ns, esz = m->esz, Mc = U * C, L = rows_at(c, l);
+        const bool fp8 = c.dtype == OT_DTYPE_FP8;
+        const int wesz = fp8 ? 1 : esz;
+        const bool last = l == c.layers - 1;
+        const long long lN = static_cast<long long>(l) * N;
+        const void *g2 = fp8 ? at(m->g2_ns, lN * d, esz) : nullptr;
+        const char *K = at(kv, kv_layer_off(c, l), esz);
+        const char *V = K + static_cast<long long>(L) * d * esz;
+        AttnArgs at_ = attn_base(c, 1, U, L, C * N, Qn, K, V, An);
         at_.KN = Kn;
         at_.VN = Vn;
-        at_.O = An;
-        at_.scale = 1.0f / sqrtf(static_cast<float>(at_.hd));
+        at_.nkn = C * N;
+        ot_status r;
         if ((r = attn(m, at_, st)) != OT_OK) return r;
         void *Xn = last && out ? out : Xb[l & 1];
+        const RowMap gm = grp();
         if (use_fused_ffn(m)) {
             // O projection + residual and the FFN in one grouped launch
-            const FfnArgs fa = ffn_o_args(m, Mc, N, An, grp, at(m->Wo_ns, lN * d * d, esz), X, grp,
-                                          at(m->W1_ns, lN * f * d, esz), at(m->W2_ns, lN * d * f, esz), Xn, grp);
+            const FfnArgs fa = ffn_o_args(m, Mc, N, An, gm, at(m->Wo_ns, lN * d * d, esz), X, gm,
+                                          at(m->W1_ns, lN * f * d, esz), at(m->W2_ns, lN * d * f, esz), Xn, gm);
             if ((r = ffn_run(m, fa, st, ROLE_NS_FFN)) != OT_OK) return r;
             X = Xn;
-            continue;
+            return OT_OK;
         }
-        g = gemm_base(c, Mc, d, d, N);
-        if ((r = projection(m, g, An, d, grp, at(m->Wo_ns, lN * d * d, wesz),
+        GemmArgs g = gemm_base(c, Mc, d, d, N);
+        if ((r = projection(m, g, An, d, gm, at(m->Wo_ns, lN * d * d, wesz),
                             static_cast<long long>(d) * d, fp8 ? m->sc_o_ns + lN : nullptr, nullptr,
                             0, false, f8, st, l, 1, IN_O)) != OT_OK)
             return r;
         g.res = X;
         g.res_ld = d;
-        g.res_map = grp;
+        g.res_map = gm;
         g.nseg = 1;
-        g.seg[0] = seg_of(Hn, d, 0, d, grp);
+        g.seg[0] = seg_of(Hn, d, 0, d, gm);
         if ((r = gemm(m, g, st, ROLE_NS_O)) != OT_OK) return r;
         g = gemm_base(c, Mc, f, d, N);
-        if ((r = projection(m, g, Hn, d, grp, at(m->W1_ns, lN * f * d, wesz),
+        if ((r = projection(m, g, Hn, d, gm, at(m->W1_ns, lN * f * d, wesz),
                             static_cast<long long>(f) * d, fp8 ? m->sc_1_ns + lN : nullptr, g2, d,
                             true, f8, st, l, 1, IN_W1)) != OT_OK)
             return r;
         g.gelu = 1;
         g.nseg = 1;
-        g.seg[0] = seg_of(hid, f, 0, f, grp);
+        g.seg[0] = seg_of(hid, f, 0, f, gm);
         if ((r = gemm(m, g, st, ROLE_NS_FFN1)) != OT_OK) return r;
         g = gemm_base(c, Mc, d, f, N);
-        if ((r = projection(m, g, hid, f, grp, at(m->W2_ns, lN * d * f, wesz),
+        if ((r = projection(m, g, hid, f, gm, at(m->W2_ns, lN * d * f, wesz),
                             static_cast<long long>(d) * f, fp8 ? m->sc_2_ns + lN : nullptr, nullptr,
                             0, false, f8, st, l, 1, IN_W2)) != OT_OK)
             return r;
         g.res = Hn;
         g.res_ld = d;
-        g.res_map = grp;
+        g.res_map = gm;
         g.nseg = 1;
-        g.seg[0] = seg_of(Xn, d, 0, d, grp);
+        g.seg[0] = seg_of(Xn, d, 0, d, gm);
         if ((r = gemm(m, g, st, ROLE_NS_FFN2)) != OT_OK) return r;
         X = Xn;
+        return OT_OK;
     }
-    return OT_OK;
+};
+
+ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, void *out, Ws ws,
+                    cudaStream_t st, cudaEvent_t *kv_ready = nullptr)
+{
+    ScoreRun sc{m, kv, U, C, out, st, kv_ready};
+    ot_status r = sc.init(ns, ws);
+    for (int l = 0; r == OT_OK && l < m->cfg.layers; ++l)
+        if ((r = sc.qkv(l)) == OT_OK) r = sc.rest(l);
+    return r;
+}
+
+// Full attention (one candidate per user): the S rows of layer l also see
+// the layer's NS keys, so both sides' projections run before either side's
+// attention, layer by layer, on one stream.
+ot_status run_full_joint(ot_model *m, const void *X0, int U, const void *ns, void *kv, void *s_out,
+                         void *out, Ws ws_enc, Ws ws_sc, cudaStream_t st)
+{
+    EncodeRun e{m, U, kv, s_out, st, nullptr, 0, true};
+    ScoreRun sc{m, kv, U, 1, out, st, nullptr};
+    ot_status r = e.init(X0, ws_enc);
+    if (r == OT_OK) r = sc.init(ns, ws_sc);
+    e.ns_K = sc.Kn;
+    e.ns_V = sc.Vn;
+    e.ns_rows = m->cfg.n_ns;
+    for (int l = 0; r == OT_OK && l < m->cfg.layers; ++l) {
+        if ((r = e.qkv(l)) != OT_OK || (r = sc.qkv(l)) != OT_OK || (r = e.rest(l)) != OT_OK) break;
+        r = sc.rest(l);
+    }
+    return r;
 }
 
 // The S and NS sides can share launches: bf16 tensor-core path with the
 // fused FFN and head_dim 64 attention.
 bool merged_supported(const ot_model *m)
 {
-    return use_fused_ffn(m) && m->cfg.d / m->cfg.heads == 64;
+    return use_fused_ffn(m) && m->cfg.d / m->cfg.heads == 64 && m->cfg.moe_experts == 0;
 }
 
 // Full forward with the S and NS sides sharing the QKV, O-projection and FFN
@@ -761,7 +1012,6 @@ ot_status run_full_merged(ot_model *m, const void *X0, int U, const void *ns, in
     const long long ustride = kv_user_elems(c);
     const RowMap grp{1, N, 0, 1, 0}; // candidate m, position g -> row m*N + g
     const Fp8Scratch no_f8{nullptr, nullptr};
-    const float scale = 1.0f / sqrtf(static_cast<float>(d / c.heads));
     // per-launch profiling times each kernel alone: everything on one stream
     cudaStream_t side = m->profiling ? st : m->side;
     const bool two = side != st;
@@ -798,29 +1048,15 @@ ot_status run_full_merged(ot_model *m, const void *X0, int U, const void *ns, in
         if (two && (cudaEventRecord(m->kv_ready[l], st) != cudaSuccess ||
                     cudaStreamWaitEvent(side, m->kv_ready[l], 0) != cudaSuccess))
             return OT_ERR_CUDA;
-        AttnArgs as_, an_;
-        memset(&as_, 0, sizeof(as_));
-        as_.mode = 0;
-        as_.U = U;
-        as_.H = c.heads;
-        as_.hd = d / c.heads;
-        as_.d = d;
-        as_.L = L;
-        as_.nq = q;
-        as_.N = N;
-        as_.Q = Qb;
-        as_.KS = K;
-        as_.VS = V;
-        as_.s_ustride = ustride;
-        as_.O = Ab;
-        as_.scale = scale;
-        an_ = as_;
-        an_.mode = 1;
-        an_.nq = C * N;
-        an_.Q = Qn;
+        AttnArgs as_ = attn_base(c, 0, U, L, q, Qb, K, V, Ab);
+        if (c.full_attn) { // the S rows also see the layer's NS keys (one candidate per user)
+            as_.KN = Kn;
+            as_.VN = Vn;
+            as_.nkn = C * N;
+        }
+        AttnArgs an_ = attn_base(c, 1, U, L, C * N, Qn, K, V, An);
         an_.KN = Kn;
         an_.VN = Vn;
-        an_.O = An;
         if ((r = attn(m, an_, side)) != OT_OK) return r;
         if (two && cudaEventRecord(m->ns_attn_done[l], side) != cudaSuccess) return OT_ERR_CUDA;
         // 3. S attention (main stream)
@@ -915,8 +1151,11 @@ ot_status ot_model_create(const ot_config *cfg, const ot_weights *w, ot_model **
     *out = nullptr;
     ot_status r = check_config(*cfg);
     if (r != OT_OK) return r;
-    const void *need[] = {w->Wqkv_s, w->Wo_s, w->W1_s, w->W2_s, w->g1_s, w->g2_s,
-                          w->Wqkv_ns, w->Wo_ns, w->W1_ns, w->W2_ns, w->g1_ns, w->g2_ns};
+    const bool moe = cfg->moe_experts > 0;
+    // a mixture of experts replaces the dense S-side FFN weights
+    const void *need[] = {w->Wqkv_s, w->Wo_s, moe ? w->W_router : w->W1_s, moe ? w->W1_moe : w->W2_s,
+                          w->g1_s, w->g2_s, w->Wqkv_ns, w->Wo_ns, w->W1_ns, w->W2_ns, w->g1_ns, w->g2_ns,
+                          moe ? w->W2_moe : w->Wqkv_s};
     for (const void *p : need) {
         if (!p) return OT_ERR_ARG;
         if (!aligned16(p)) return OT_ERR_ALIGN;
@@ -979,12 +1218,31 @@ ot_status ot_model_create(const ot_config *cfg, const ot_weights *w, ot_model **
         }
         // gains folded into the projection that follows each norm
         if ((r = device_fold(m, &m->Wqkv_s, w->Wqkv_s, w->g1_s, 3 * d, d, L)) != OT_OK) break;
-        if ((r = device_fold(m, &m->W1_s, w->W1_s, w->g2_s, f, d, L)) != OT_OK) break;
+        if (moe) {
+            // experts: g2 folded into every expert's W1 (one gain per layer);
+            // the router reads the gain itself, so g2 is kept as well
+            const long long E = cfg->moe_experts;
+            const size_t w1b = static_cast<size_t>(L * E * f * d) * esz;
+            if (cudaMalloc(&m->W1_moe, w1b) != cudaSuccess) { r = OT_ERR_CUDA; break; }
+            m->allocs.push_back(m->W1_moe);
+            for (long long l = 0; l < L && r == OT_OK; ++l)
+                if (launch_fold_gain(at(w->W1_moe, l * E * f * d, esz), at(w->g2_s, l * d, esz),
+                                     at(m->W1_moe, l * E * f * d, esz), f, static_cast<int>(d), E, 0,
+                                     cfg->dtype == OT_DTYPE_F32 ? OT_DTYPE_F32 : OT_DTYPE_BF16,
+                                     0) != cudaSuccess)
+                    r = OT_ERR_CUDA;
+            if (r != OT_OK) break;
+            if ((r = device_copy(m, &m->W2_moe, w->W2_moe, L * E * d * f * esz)) != OT_OK) break;
+            if ((r = device_copy(m, &m->W_router, w->W_router, L * E * d * esz)) != OT_OK) break;
+            if ((r = device_copy(m, &m->g2_s, w->g2_s, L * d * esz)) != OT_OK) break;
+        } else if ((r = device_fold(m, &m->W1_s, w->W1_s, w->g2_s, f, d, L)) != OT_OK) {
+            break;
+        }
         if ((r = device_fold(m, &m->Wqkv_ns, w->Wqkv_ns, w->g1_ns, 3 * d, d, L * N)) != OT_OK)
             break;
         if ((r = device_fold(m, &m->W1_ns, w->W1_ns, w->g2_ns, f, d, L * N)) != OT_OK) break;
         if ((r = device_copy(m, &m->Wo_s, w->Wo_s, L * d * d * esz)) != OT_OK) break;
-        if ((r = device_copy(m, &m->W2_s, w->W2_s, L * d * f * esz)) != OT_OK) break;
+        if (!moe && (r = device_copy(m, &m->W2_s, w->W2_s, L * d * f * esz)) != OT_OK) break;
         if ((r = device_copy(m, &m->Wo_ns, w->Wo_ns, L * N * d * d * esz)) != OT_OK) break;
         if ((r = device_copy(m, &m->W2_ns, w->W2_ns, L * N * d * f * esz)) != OT_OK) break;
         if (cfg->F > 0 &&
@@ -1114,6 +1372,7 @@ ot_status ot_fp8_calibrate(ot_model *m, const void *S, const void *ns, int U, in
 {
     if (!m || !S || !ns || !amax || !ws || U < 1 || C < 1) return OT_ERR_ARG;
     if (m->cfg.dtype != OT_DTYPE_FP8) return OT_ERR_DTYPE;
+    if (m->cfg.full_attn) return OT_ERR_UNSUPPORTED;
     if (!aligned16(S) || !aligned16(ns) || !aligned16(ws) || (reinterpret_cast<uintptr_t>(amax) & 3))
         return OT_ERR_ALIGN;
     if (static_cast<long long>(U) * m->cfg.L0 > (1LL << 31) - 1 ||
@@ -1179,6 +1438,7 @@ ot_status ot_encode_user(ot_model *m, const void *S, int U, void *kv_cache, void
                          void *ws, size_t ws_bytes, void *stream)
 {
     if (!m || !S || !kv_cache || !ws || U < 1) return OT_ERR_ARG;
+    if (m->cfg.full_attn) return OT_ERR_UNSUPPORTED; // S rows depend on the candidate
     if (!aligned16(S) || !aligned16(kv_cache) || !aligned16(ws) ||
         (out_s_tail && !aligned16(out_s_tail)))
         return OT_ERR_ALIGN;
@@ -1193,13 +1453,15 @@ size_t ot_append_workspace_bytes(const ot_model *m, int users, int delta)
     if (!m || users < 0 || delta < 0) return 0;
     const long long rows = static_cast<long long>(users) * delta;
     const ot_config &c = m->cfg;
-    return 5 * bytes_of(rows * c.d, m->esz) + bytes_of(rows * c.ffn, m->esz) + fp8_ws_bytes(c, rows);
+    return 5 * bytes_of(rows * c.d, m->esz) + bytes_of(rows * c.ffn, m->esz) + fp8_ws_bytes(c, rows) +
+           moe_ws_bytes(c, rows, m->esz);
 }
 
 ot_status ot_encode_append(ot_model *m, const void *kv_old, int U, const void *S_new, int delta,
                            void *kv_new, void *out_new, void *ws, size_t ws_bytes, void *stream)
 {
     if (!m || !kv_old || !S_new || !kv_new || !out_new || !ws || U < 1 || delta < 1) return OT_ERR_ARG;
+    if (m->cfg.full_attn) return OT_ERR_UNSUPPORTED;
     if (!aligned16(kv_old) || !aligned16(S_new) || !aligned16(kv_new) || !aligned16(out_new) ||
         !aligned16(ws))
         return OT_ERR_ALIGN;
@@ -1243,6 +1505,7 @@ ot_status ot_score_candidates(ot_model *m, const void *kv_cache, int U, const vo
                               void *out_ns, void *ws, size_t ws_bytes, void *stream)
 {
     if (!m || !kv_cache || !ns || !out_ns || !ws || U < 1 || C < 1) return OT_ERR_ARG;
+    if (m->cfg.full_attn) return OT_ERR_UNSUPPORTED;
     if (!aligned16(kv_cache) || !aligned16(ns) || !aligned16(out_ns) || !aligned16(ws))
         return OT_ERR_ALIGN;
     if (static_cast<long long>(U) * C * m->cfg.n_ns > (1LL << 31) - 1) return OT_ERR_SHAPE;
@@ -1274,6 +1537,17 @@ ot_status ot_full_forward(ot_model *m, const void *S, const void *ns, int B, int
     if (!kv) {
         kv = w.take(static_cast<long long>(B) * kv_user_elems(c));
         if (!kv) return OT_ERR_WORKSPACE_TOO_SMALL;
+    }
+    if (c.full_attn) {
+        // full attention: the S rows see their candidate's NS keys, one candidate per user
+        if (C != 1) return OT_ERR_SHAPE;
+        if (w.left < enc + sc) return OT_ERR_WORKSPACE_TOO_SMALL;
+        std::lock_guard<std::recursive_mutex> lock(m->enqueue_mu);
+        Ws w_enc = w;
+        Ws w_sc{w.p + enc, w.left - enc, m->esz};
+        if (merged_supported(m) && m->side)
+            return run_full_merged(m, S, B, ns, C, kv, out_s_tail, out_ns, w_enc, w_sc, st);
+        return run_full_joint(m, S, B, ns, kv, out_s_tail, out_ns, w_enc, w_sc, st);
     }
     // Shared O / FFN launches for both sides where the kernels allow it
     if (merged_supported(m) && m->side && w.left >= enc + sc) {

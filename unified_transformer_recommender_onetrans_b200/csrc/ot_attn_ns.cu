@@ -1,7 +1,8 @@
 // NS attention when every NS query row of a user fits in 64 (C N <= 64; the
 // dispatcher uses it up to 16, e.g. the full forward at C = 1): query i = NS token i % N
 // of candidate i / N sees all L cached S keys of the layer and the NS keys
-// m <= i % N of its own candidate (the OneTrans mask).  head_dim 64, bf16
+// m <= i % N of its own candidate (the OneTrans mask; with full attention
+// every NS key of its candidate).  head_dim 64, bf16
 // operands, fp32 scores, softmax and accumulation.
 //
 // With a handful of query rows a 128-row tensor-memory tile would hold mostly
@@ -202,7 +203,8 @@ __global__ void __launch_bounds__(NA_WARPS * 32, 2)
             for (int e = 0; e < 4; ++e) {
                 const int hi = e >> 1, key = j0 + n * 8 + 2 * t + (e & 1);
                 const bool vis = s_block ? key < a.L
-                                         : (key < a.nq && key / a.N == cand[hi] && key % a.N <= tok[hi]);
+                                         : (key < a.nq && key / a.N == cand[hi] &&
+                                            (a.full || key % a.N <= tok[hi]));
                 sc[n][e] = vis ? sc[n][e] * c2 : -INFINITY;
                 bm[hi] = fmaxf(bm[hi], sc[n][e]);
             }

@@ -15,6 +15,9 @@
 //             every S key 0..L-1 and NS keys m <= n of candidate c.  Each
 //             cached S K/V tile is read once per item and shared by all the
 //             item's candidates (256 / N of them).
+//   full attention (AttnArgs::full, one candidate per user): an S row sees
+//             every S key and then the user's nkn NS keys, which follow the S
+//             blocks in its item; an NS row every NS key of its candidate.
 //
 // A tcgen05.mma issued from one thread takes about 100-130 cycles whatever
 // its N up to 128, so at head_dim 64 (12 MMAs per tile and key block) the
@@ -142,7 +145,7 @@ __device__ __forceinline__ void softmax_unit(uint32_t tS_row, float c2, int klo,
     rsum = (a0 + b0) + (a1 + b1);
 }
 
-// One work item of the persistent kernel: a (user, head, query pair) and its
+// One work item of the persistent kernel (FA: full attention, AttnArgs::full): a (user, head, query pair) and its
 // key-block schedule, shared by every role of the CTA.
 struct AtItem {
     int u, h, i0;     // user, head, first query row of the pair
@@ -159,7 +162,7 @@ template <bool SPLIT> __host__ __device__ constexpr int at_item_rows() { return 
 // more keys), so the snake assignment below balances the CTAs; NS mode keeps
 // the pairs (row tiles in split-key mode) of one (user, head) together so
 // they share K/V tiles in L2.
-template <bool NS, bool SPLIT>
+template <bool NS, bool SPLIT, bool FA>
 __device__ __forceinline__ AtItem at_item(const AttnArgs &a, int n_pairs, int k)
 {
     AtItem it;
@@ -178,9 +181,11 @@ __device__ __forceinline__ AtItem at_item(const AttnArgs &a, int n_pairs, int k)
     const int i_last = min(it.i0 + at_item_rows<SPLIT>(), a.nq) - 1;
     it.k_begin = 0;
     if (!NS) {
+        // causal: the keys up to the item's last row; full attention: every
+        // S key, then the user's NS keys
         const int t_last = a.L - a.nq + i_last;
-        it.n_s_blocks = (t_last + AT_BK) / AT_BK;
-        it.n_blocks = it.n_s_blocks;
+        it.n_s_blocks = FA ? (a.L + AT_BK - 1) / AT_BK : (t_last + AT_BK) / AT_BK;
+        it.n_blocks = it.n_s_blocks + (FA ? (a.nkn + AT_BK - 1) / AT_BK : 0);
     } else {
         it.n_s_blocks = (a.L + AT_BK - 1) / AT_BK;
         it.k_begin = (it.i0 / a.N) * a.N;
@@ -205,7 +210,7 @@ __device__ __forceinline__ int at_item_of(int r, int n_items)
 // items of one 128-row tile), where tile w takes the blocks b = w (mod 2) of
 // an item and the two tiles' partial softmax states are merged at its end.
 // gb counts all blocks of the CTA (the K/V ring position), lb this tile's.
-template <bool NS, bool SPLIT>
+template <bool NS, bool SPLIT, bool FA>
 struct BlockCursor {
     int r, k;      // item ordinal within the CTA, item index (k < 0: past the end)
     AtItem it;
@@ -220,7 +225,7 @@ struct BlockCursor {
         if (++b < it.n_blocks) return;
         b = 0;
         k = at_item_of(++r, n_items);
-        if (k >= 0) it = at_item<NS, SPLIT>(a, n_pairs, k);
+        if (k >= 0) it = at_item<NS, SPLIT, FA>(a, n_pairs, k);
     }
     __device__ __forceinline__ void init(const AttnArgs &a, int n_pairs, int n_items, int tile)
     {
@@ -230,7 +235,7 @@ struct BlockCursor {
         gb = 0;
         lb = 0;
         k = at_item_of(0, n_items);
-        if (k >= 0) it = at_item<NS, SPLIT>(a, n_pairs, k);
+        if (k >= 0) it = at_item<NS, SPLIT, FA>(a, n_pairs, k);
         while (valid() && !owned()) step(a, n_pairs, n_items);
     }
     __device__ __forceinline__ void next(const AttnArgs &a, int n_pairs, int n_items)
@@ -247,7 +252,7 @@ struct BlockCursor {
     }
 };
 
-template <bool NS, bool SPLIT>
+template <bool NS, bool SPLIT, bool FA>
 __global__ void __launch_bounds__(AT_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKS,
                    const __grid_constant__ CUtensorMap tmVS, const __grid_constant__ CUtensorMap tmKN,
@@ -339,7 +344,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             for (; ok; ++r) {
                 const int k = at_item_of(r, n_items);
                 if (k < 0) break;
-                const AtItem it = at_item<NS, SPLIT>(a, n_pairs, k);
+                const AtItem it = at_item<NS, SPLIT, FA>(a, n_pairs, k);
                 const int qb = r & 1;
                 // the Q buffer of item r - 2 is free once all its S MMAs completed
                 if (!mbar_wait(&q_empty[qb], ((r >> 1) & 1) ^ 1, a.wait, abort_flag)) break;
@@ -390,7 +395,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         if (lane == 0 && !aborted_at_start) {
             const uint32_t tS = tmem + w * 256, tP = tS + 128, tO = tS + 192;
             auto live = [&](const AtItem &it) { return SPLIT || it.i0 + w * AT_BM < a.nq; };
-            auto issue_s = [&](const BlockCursor<NS, SPLIT> &c) {
+            auto issue_s = [&](const BlockCursor<NS, SPLIT, FA> &c) {
                 if (live(c.it)) {
                     const uint32_t q_addr = smem_u32(sQ + ((c.r & 1) * AT_TILES + (SPLIT ? 0 : w)) * AT_TILE);
                     const uint32_t k_addr = smem_u32(sKV + 2 * (c.gb % AT_STAGES) * AT_TILE);
@@ -403,12 +408,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 // the item's last S of this tile: its Q buffer is free once they completed
                 if (c.last_in_item()) mma_commit(&q_empty[c.r & 1]);
             };
-            auto ready_s = [&](const BlockCursor<NS, SPLIT> &c) {
+            auto ready_s = [&](const BlockCursor<NS, SPLIT, FA> &c) {
                 return mbar_wait(&kv_full[c.gb % AT_STAGES], static_cast<uint32_t>((c.gb / AT_STAGES) & 1),
                                  a.wait, abort_flag) &&
                        mbar_wait(&q_full[c.r & 1], (c.r >> 1) & 1, a.wait, abort_flag);
             };
-            BlockCursor<NS, SPLIT> cur;
+            BlockCursor<NS, SPLIT, FA> cur;
             cur.init(a, n_pairs, n_items, w);
             bool run = cur.valid() && ready_s(cur);
             if (run) {
@@ -416,7 +421,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 issue_s(cur);
             }
             while (run) {
-                BlockCursor<NS, SPLIT> nxt = cur;
+                BlockCursor<NS, SPLIT, FA> nxt = cur;
                 nxt.next(a, n_pairs, n_items);
                 if (nxt.valid()) {
                     if (!mbar_wait(&s_free[w], static_cast<uint32_t>(cur.lb & 1), a.wait, abort_flag) ||
@@ -483,11 +488,14 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         for (int r = 0; ok; ++r) {
             const int k = at_item_of(r, n_items);
             if (k < 0) break;
-            const AtItem it = at_item<NS, SPLIT>(a, n_pairs, k);
+            const AtItem it = at_item<NS, SPLIT, FA>(a, n_pairs, k);
             const int i = it.i0 + (SPLIT ? 0 : w * AT_BM) + row; // query row within the user
             const bool warp_dead = __all_sync(0xffffffffu, i >= a.nq);
             const int t_self = a.L - a.nq + i;      // S mode
-            const int my_c = NS ? i / a.N : 0, my_n = NS ? i % a.N : 0;
+            // the row's candidate and the last NS key of it the row sees (S
+            // rows meet NS keys only with full attention: all nkn of the user)
+            const int my_c = NS ? i / a.N : 0;
+            const int my_n = !NS ? (FA ? a.nkn - 1 : 0) : FA ? a.N - 1 : i % a.N;
             float m = -INFINITY, l = 0.f;
             const int b0 = SPLIT ? w : 0; // this tile's first block of the item
             for (int b = b0; ok && b < it.n_blocks; b += SPLIT ? 2 : 1, ++lb) {
@@ -496,7 +504,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 // visible key range [klo, khi] of this row inside the block
                 int klo = 0, khi;
                 if (s_block) {
-                    khi = NS ? min(a.L - 1 - j0, AT_BK - 1) : min(t_self - j0, AT_BK - 1);
+                    khi = (NS || FA) ? min(a.L - 1 - j0, AT_BK - 1) : min(t_self - j0, AT_BK - 1);
                 } else {
                     const int first = my_c * a.N - j0; // key index of (my_c, 0)
                     klo = max(first, 0);
@@ -648,9 +656,11 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
         tmap_rows(&tks, a.KS, a.d, a.L, a.U, a.s_ustride) ||
         tmap_rows(&tvs, a.VS, a.d, a.L, a.U, a.s_ustride))
         return cudaErrorInvalidValue;
-    if (a.mode == 1) {
-        if (tmap_rows(&tkn, a.KN, a.d, a.nq, a.U, static_cast<long long>(a.nq) * a.d) ||
-            tmap_rows(&tvn, a.VN, a.d, a.nq, a.U, static_cast<long long>(a.nq) * a.d))
+    if (a.mode == 1 || a.full) {
+        // NS keys / values: nkn rows per user (NS mode: the query rows themselves)
+        const int nk = a.mode == 1 ? a.nq : a.nkn;
+        if (nk < 1 || tmap_rows(&tkn, a.KN, a.d, nk, a.U, static_cast<long long>(nk) * a.d) ||
+            tmap_rows(&tvn, a.VN, a.d, nk, a.U, static_cast<long long>(nk) * a.d))
             return cudaErrorInvalidValue;
     } else {
         tkn = tks;
@@ -703,8 +713,12 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
         if (err != cudaSuccess) return err;
         return launch_pdl(kernel, grid, dim3(AT_THREADS), AT_SMEM, s, tq, tks, tvs, tkn, tvn, a);
     };
-    if (a.mode != 1) return run(attn_tc_kernel<false, false>);
-    return split ? run(attn_tc_kernel<true, true>) : run(attn_tc_kernel<true, false>);
+    if (a.full) {
+        if (a.mode != 1) return run(attn_tc_kernel<false, false, true>);
+        return split ? run(attn_tc_kernel<true, true, true>) : run(attn_tc_kernel<true, false, true>);
+    }
+    if (a.mode != 1) return run(attn_tc_kernel<false, false, false>);
+    return split ? run(attn_tc_kernel<true, true, false>) : run(attn_tc_kernel<true, false, false>);
 }
 
 } // namespace ot

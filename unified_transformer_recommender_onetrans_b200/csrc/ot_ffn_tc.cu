@@ -88,6 +88,17 @@ __device__ __forceinline__ int ffn_tile(const FfnMulti &P, long long tile, int &
     return pi;
 }
 
+// Whether tile `tile` holds a filled row: a group with group_rows set (the
+// experts of a mixture) has only its first group_rows[g] rows filled, and
+// every role skips the tiles past them alike.
+__device__ __forceinline__ bool ffn_tile_live(const FfnMulti &P, long long tile)
+{
+    int g, m0;
+    const int pi = ffn_tile(P, tile, g, m0);
+    const int *gr = P.q[pi].a.group_rows;
+    return !gr || m0 < gr[g];
+}
+
 // exact-erf GELU, z * Phi(z), with Phi(z) ~ 1/2 + 1/2 tanh(z (A + B z^2)):
 // the same fitted form as the GEMM epilogue
 __device__ __forceinline__ float ffn_gelu(float z)
@@ -220,7 +231,10 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             // tile's first two W1 / W2 stages load while the previous kernel
             // finishes (fresh stages, no empty wait); H follows once its
             // outputs are visible.
-            const int n_pre = static_cast<long long>(blockIdx.x) < P.tiles ? (n_side < 2 ? n_side : 2) : 0;
+            // (not with filled-row counts: which tile comes first is known
+            // only once the previous kernel's counts are visible)
+            const bool counted = P.q[0].a.group_rows || (two && P.q[1].a.group_rows);
+            const int n_pre = !counted && static_cast<long long>(blockIdx.x) < P.tiles ? (n_side < 2 ? n_side : 2) : 0;
             // load j of this side for group g into stage st
             auto load = [&](int pi, int g, int j, int st) {
                 if (w1_side) {
@@ -248,6 +262,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             int tl = 0, n_h = 0;
             bool ok = true;
             for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x, ++tl) {
+                if (!ffn_tile_live(P, tile)) { --tl; continue; } // past its group's filled rows
                 int g, m0;
                 const int pi = ffn_tile(P, tile, g, m0);
                 const CUtensorMap *tH = pi ? &tmH1 : &tmH0;
@@ -289,6 +304,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             int tl = 0;
             bool ok = true;
             for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x, ++tl) {
+                if (!ffn_tile_live(P, tile)) { --tl; continue; } // past its group's filled rows
                 if (!mbar_wait(h_full, tl & 1, a.wait, abort_flag)) break;
                 if (FO) {
                     // acc2 = X (seeded by the epilogue) + A Wo^T, A from the
@@ -357,6 +373,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             int tl = 0;
             bool ok = true;
             for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x, ++tl) {
+                if (!ffn_tile_live(P, tile)) { --tl; continue; } // past its group's filled rows
                 for (int c = 0; c < NC; ++c, ++gc) {
                     const int st = static_cast<int>(gc & 1);
                     const uint32_t ph = static_cast<uint32_t>((gc >> 1) & 1);
@@ -397,6 +414,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
         int tl = 0;
         bool ok = true;
         for (long long tile = blockIdx.x; ok && tile < P.tiles; tile += gridDim.x, ++tl) {
+            if (!ffn_tile_live(P, tile)) { --tl; continue; } // past its group's filled rows
             int g, m0;
             const int pi = ffn_tile(P, tile, g, m0);
             float ss = 0.f;

@@ -77,17 +77,22 @@ struct GemmArgs {
 
 // Attention over one layer.  Query rows come from Q [U][nq][d] (head h at
 // columns h*hd); S keys / values from the per-user cache rows
-// [U][L][d] (user stride s_ustride elements); NS keys / values (NS mode)
-// from KN / VN [U][nq][d].
+// [U][L][d] (user stride s_ustride elements); NS keys / values from KN / VN
+// [U][nkn][d] (NS mode, and S mode with full attention).
 //   S mode  : query i is S row t = L - nq + i; it sees S keys 0..t.
 //   NS mode : query i is NS token n = i % N of candidate c = i / N; it sees
 //             all L S keys and NS keys m <= n of candidate c.
+//   full    : full (non-causal) attention, one candidate per user in S mode:
+//             an S row sees all L S keys and all nkn NS keys of its user; an
+//             NS row all L S keys and all N NS keys of its candidate.
 struct AttnArgs {
     int mode;           // 0 = S, 1 = NS
     int U, H, hd, d;
     int L;              // S keys
     int nq;             // query rows per user
-    int N;              // NS tokens per candidate (NS mode)
+    int N;              // NS tokens per candidate
+    int full;           // 1: full attention
+    int nkn;            // NS key rows per user in KN / VN (NS mode: nq)
     const void *Q;
     const void *KS, *VS;
     long long s_ustride; // elements between users in KS / VS
@@ -124,6 +129,9 @@ struct FfnArgs {
     long long wo_gstride;   // elements between groups of Wo
     const void *X;
     RowMap x_map;
+    // rows of each group actually filled (device, [G]; null: M each): tiles
+    // past a group's count are skipped (the experts of a mixture)
+    const int *group_rows;
 };
 
 // Launch with programmatic stream serialization: the kernel may start while
@@ -189,6 +197,33 @@ cudaError_t launch_quant_rows(const void *X, long long lda, RowMap map, long lon
                               QuantRule rule, uint8_t *q_out, float *scale_out, cudaStream_t s);
 cudaError_t launch_quant_weights(const void *W, long long per_mat, long long mats, uint8_t *q_out,
                                  float *scale_out, float *amax_scratch, cudaStream_t s);
+
+// Sparse mixture of experts (S-side FFN).  Router: rows of H [rows][d] ->
+// for each row its top-k experts; choice j of row r takes slot counts[e]++
+// of expert e, its row is copied to Hp[e * cap + slot] and route[2 r + j] =
+// e * cap + slot, gate[2 r + j] = its gate.  counts must start at zero.
+struct MoeRouteArgs {
+    long long rows;
+    int d, E, topk, dtype;
+    float eps;
+    const void *H, *gain, *Wr;   // gain [d] (RMSNorm before the FFN), Wr [E][d]
+    void *Hp;                    // [E][cap][d]
+    long long cap;
+    int *counts;                 // [E]
+    long long *route;            // [rows][2]
+    float *gate;                 // [rows][2]
+};
+// Combine: Y[r] = H[r] + sum_j gate[2 r + j] (Yp[route[2 r + j]] - H[r]).
+struct MoeCombineArgs {
+    long long rows;
+    int d, topk, dtype;
+    const void *H, *Yp;
+    void *Y;
+    const long long *route;
+    const float *gate;
+};
+cudaError_t launch_moe_route(const MoeRouteArgs &a, cudaStream_t s);
+cudaError_t launch_moe_combine(const MoeCombineArgs &a, cudaStream_t s);
 
 // Read-only model queries for entry points defined outside ot_api.cu.
 int internal_profiling(const ot_model *m);

@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(SA_ROWS) attn_simt_kernel(AttnArgs a)
     const int i_last = min(i0 + SA_ROWS, a.nq) - 1;
     // ---- S keys
     int s_keys;
-    if (a.mode == 0)
+    if (a.mode == 0 && !a.full)
         s_keys = a.L - a.nq + i_last + 1; // the last query row's S row + 1
     else
         s_keys = a.L;
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(SA_ROWS) attn_simt_kernel(AttnArgs a)
         __syncthreads();
         if (!valid) continue;
         int jend = min(SA_KT, s_keys - j0);
-        if (a.mode == 0) jend = min(jend, t_self - j0 + 1);
+        if (a.mode == 0 && !a.full) jend = min(jend, t_self - j0 + 1);
         for (int j = 0; j < jend; ++j) {
             float sc = 0.f;
 #pragma unroll
@@ -183,13 +183,16 @@ __global__ void __launch_bounds__(SA_ROWS) attn_simt_kernel(AttnArgs a)
             for (int e = 0; e < HD; ++e) o[e] = fmaf(p, Vs[j][e], o[e]);
         }
     }
-    // ---- NS keys of the candidates this CTA's rows belong to
-    if (a.mode == 1) {
-        const int c_first = i0 / a.N, c_last = i_last / a.N;
-        const int k_begin = c_first * a.N, k_end = (c_last + 1) * a.N;
-        const T *KN = static_cast<const T *>(a.KN) + static_cast<long long>(u) * a.nq * a.d + h * HD;
-        const T *VN = static_cast<const T *>(a.VN) + static_cast<long long>(u) * a.nq * a.d + h * HD;
-        const int my_c = i / a.N, my_n = i % a.N;
+    // ---- NS keys of the candidates this CTA's rows belong to (NS mode), or
+    // with full attention in S mode all nkn NS keys of the user
+    if (a.mode == 1 || a.full) {
+        const int c_first = a.mode == 1 ? i0 / a.N : 0, c_last = a.mode == 1 ? i_last / a.N : 0;
+        const int k_begin = c_first * a.N, k_end = a.mode == 1 ? (c_last + 1) * a.N : a.nkn;
+        const T *KN = static_cast<const T *>(a.KN) + static_cast<long long>(u) * a.nkn * a.d + h * HD;
+        const T *VN = static_cast<const T *>(a.VN) + static_cast<long long>(u) * a.nkn * a.d + h * HD;
+        // the row's candidate and position; in full attention every NS key of
+        // the candidate is visible (S mode: the user's only candidate)
+        const int my_c = a.mode == 1 ? i / a.N : 0, my_n = a.full ? a.N - 1 : i % a.N;
         for (int j0 = k_begin; j0 < k_end; j0 += SA_KT) {
             __syncthreads();
             for (int e = threadIdx.x; e < SA_KT * HD; e += SA_ROWS) {
