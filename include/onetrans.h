@@ -68,6 +68,8 @@ extern "C" {
 #endif
 
 #define OT_MAX_LAYERS 32
+/* Rows of K (and of V) in one page of a paged KV cache. */
+#define OT_PAGE_ROWS 128
 
 typedef enum {
     OT_OK = 0,
@@ -219,6 +221,34 @@ size_t ot_append_workspace_bytes(const ot_model *m, int users, int delta);
  * A candidate's result does not depend on the other candidates in the call. */
 ot_status ot_score_candidates(ot_model *m, const void *kv_cache, int U, const void *ns, int C,
                               void *out_ns, void *ws, size_t ws_bytes, void *stream);
+
+/* Paged KV cache (the blog page's engineering reading list points at
+ * PagedAttention and prefix caching for the cross-request KV cache; the
+ * layout here is the library's).  Instead of one dense block per user the
+ * cache is a caller-owned pool of pages, each OT_PAGE_ROWS rows of K [128][d]
+ * followed by the same rows of V, and a page table, device int32
+ * [U][ot_kv_pages_per_user(m)]: entry off(l) + b of user u names the page
+ * holding rows 128 b .. 128 b + 127 of layer l (off(l) = sum over j < l of
+ * ceil(L_j / 128); the last page of a layer may be partly used).  Pages may
+ * be listed by several users when their K/V rows are identical: users with
+ * the same schedule and the same S rows up to the page's last row (a shared
+ * prefix) -- every user's encode writes the page, with identical values.
+ * A page id outside [0, n_pages) is never dereferenced: the store is
+ * skipped, reads use page 0, and OT_ERR_DEVICE_BOUNDS is raised. */
+int ot_kv_pages_per_user(const ot_model *m);
+/* Bytes of one page: 2 * OT_PAGE_ROWS * d * sizeof(storage). */
+size_t ot_kv_page_bytes(const ot_model *m);
+/* ot_encode_user into a paged cache: pool device (n_pages pages), pages
+ * device int32 [U][ot_kv_pages_per_user(m)]; otherwise as ot_encode_user
+ * (same workspace).  Errors as ot_encode_user, plus OT_ERR_ARG for a null
+ * pool or table or n_pages < 1. */
+ot_status ot_encode_user_paged(ot_model *m, const void *S, int U, void *pool, long long n_pages,
+                               const int32_t *pages, void *out_s_tail, void *ws, size_t ws_bytes,
+                               void *stream);
+/* ot_score_candidates against a paged cache written by ot_encode_user_paged. */
+ot_status ot_score_candidates_paged(ot_model *m, const void *pool, long long n_pages,
+                                    const int32_t *pages, int U, const void *ns, int C,
+                                    void *out_ns, void *ws, size_t ws_bytes, void *stream);
 
 /* Capacity of the scratch array used by ot_score_candidates_noalloc (bytes). */
 #define OT_NOALLOC_SCRATCH_BYTES (16u << 20)

@@ -619,3 +619,123 @@ def test_moe_onetrans_s_shapes():
     m.set_wait_limit(TEST_WAIT)
     a = _run_full(m, S.cuda(), ns.cuda())
     assert_within(_errors_vs_oracle(m, w, S, ns, *a, [1, 4]), TOL["bf16"])
+
+
+# ----------------------------------------------------------------- paged KV cache
+def _page_table(m, U, n_pages, seed, share=None):
+    """A random assignment of distinct pages to every (user, layer block);
+    share = (a, b): user b lists user a's pages (their rows are identical)."""
+    ppu = m.kv_pages_per_user()
+    g = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(n_pages, generator=g)[: U * ppu].view(U, ppu)
+    if share:
+        perm[share[1]] = perm[share[0]]
+    return perm.to(torch.int32).cuda()
+
+
+@pytest.mark.parametrize("shape", ["small", "onetrans_s_c1", "onetrans_s_c8"])
+def test_paged_cache_matches_dense_cache(shape):
+    """ot_encode_user_paged / ot_score_candidates_paged against the dense
+    cache, bit for bit: the S tails, the NS outputs and every layer's K / V
+    gathered from the pages (shuffled page ids in a pool with spare pages;
+    layers whose last page is partly used); small-NS, split-key and
+    two-tile NS attention read the pages."""
+    if shape == "small":
+        shapes = dict(layers=3, d=128, heads=2, ffn=256, n_ns=5, L0=300, q=[300, 170, 37])
+        U, C = 3, 7
+    else:
+        wl = WORKLOADS["onetrans_s_full"]
+        shapes = dict(layers=3, d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns, L0=700,
+                      q=[700, 333, 60])
+        U, C = 4, (1 if shape == "onetrans_s_c1" else 8)
+    w = rand_weights(shapes["layers"], shapes["d"], shapes["ffn"], shapes["n_ns"], seed=131,
+                     dtype=torch.bfloat16)
+    S, ns = rand_inputs(U, C, shapes["L0"], shapes["n_ns"], shapes["d"], seed=132, dtype=torch.bfloat16)
+    m = make_model(w, **shapes)
+    m.set_wait_limit(TEST_WAIT)
+    Sd, nsd = S.cuda(), ns.cuda()
+    kv, s_dense = m.encode_user(Sd)
+    out_dense = m.score_candidates(kv, nsd)
+    n_pages = U * m.kv_pages_per_user() + 9
+    pool = m.new_page_pool(n_pages)
+    pool.fill_(float("nan"))  # stale pages: nothing unwritten may leak into the results
+    pages = _page_table(m, U, n_pages, seed=133)
+    s_paged = m.encode_user_paged(Sd, pool, pages)
+    out_paged = m.score_candidates_paged(pool, pages, nsd)
+    m.poll()
+    assert torch.equal(s_paged, s_dense)
+    assert torch.equal(out_paged, out_dense)
+    for u in range(U):
+        for l in range(m.layers):
+            K, V = m.kv_from_pages(pool, pages[u].cpu(), l)
+            Kd, Vd = m.kv_layer(kv[u], l)
+            assert torch.equal(K, Kd) and torch.equal(V, Vd), (u, l)
+
+
+def test_paged_cache_shared_prefix_pages():
+    """Users with identical S rows list the same pages (a shared prefix
+    covering the whole sequence): their results equal each other and the
+    dense cache's, and a third user with its own pages is unaffected."""
+    shapes = dict(layers=3, d=128, heads=2, ffn=256, n_ns=5, L0=300, q=[300, 170, 37])
+    w = rand_weights(3, 128, 256, 5, seed=134, dtype=torch.bfloat16)
+    S, ns = rand_inputs(3, 4, 300, 5, 128, seed=135, dtype=torch.bfloat16)
+    S[1] = S[0]
+    m = make_model(w, **shapes)
+    m.set_wait_limit(TEST_WAIT)
+    n_pages = 3 * m.kv_pages_per_user()
+    pool = m.new_page_pool(n_pages)
+    pages = _page_table(m, 3, n_pages, seed=136, share=(0, 1))
+    s_paged = m.encode_user_paged(S.cuda(), pool, pages)
+    out_paged = m.score_candidates_paged(pool, pages, ns.cuda())
+    kv, s_dense = m.encode_user(S.cuda())
+    out_dense = m.score_candidates(kv, ns.cuda())
+    m.poll()
+    assert torch.equal(s_paged, s_dense) and torch.equal(out_paged, out_dense)
+    assert torch.equal(s_paged[0], s_paged[1])
+
+
+def test_paged_cache_fp32_cuda_core_and_oracle():
+    """The tiny fp32 block on the CUDA-core kernels with a paged cache,
+    against the oracle at 1e-5."""
+    wl = WORKLOADS["tiny_fp32"]
+    w = gen_weights(wl)
+    S = gen_s_tokens(wl, weights=w)
+    x = gen_auto_split_features(wl)
+    m = model_of(wl, w)
+    ns = m.auto_split(x.cuda())
+    pool = m.new_page_pool(m.kv_pages_per_user() + 2)
+    pages = _page_table(m, 1, pool.shape[0], seed=137)
+    s_tail = m.encode_user_paged(S.cuda(), pool, pages)
+    out = m.score_candidates_paged(pool, pages, ns)
+    m.poll()
+    cfg = oracle_cfg(m)
+    kv_o, s_o = O.encode_user(cfg, w, S)
+    out_o = O.score_candidates(cfg, w, kv_o, O.auto_split(x, w["W_split"], wl.n_ns, wl.d))
+    errs = {"s_tail": O.rel_l2(s_tail.double().cpu().numpy(), s_o),
+            "ns_out": O.rel_l2(out.double().cpu().numpy(), out_o)}
+    assert_within(errs, TOL["f32"])
+
+
+def test_paged_cache_bad_page_id_is_reported():
+    """A page id outside the pool is never dereferenced: the call completes,
+    the device error word reports OT_ERR_DEVICE_BOUNDS, and the context is
+    fine for the next call."""
+    shapes = dict(layers=2, d=128, heads=2, ffn=256, n_ns=3, L0=200, q=[200, 90])
+    w = rand_weights(2, 128, 256, 3, seed=138, dtype=torch.bfloat16)
+    S, ns = rand_inputs(2, 2, 200, 3, 128, seed=139, dtype=torch.bfloat16)
+    m = make_model(w, **shapes)
+    m.set_wait_limit(TEST_WAIT)
+    n_pages = 2 * m.kv_pages_per_user()
+    pool = m.new_page_pool(n_pages)
+    pages = _page_table(m, 2, n_pages, seed=140)
+    bad = pages.clone()
+    bad[1, 1] = n_pages + 5
+    m.encode_user_paged(S.cuda(), pool, bad)
+    with pytest.raises(ot.OtError) as e:
+        m.poll()
+    assert e.value.code == 9
+    s_tail = m.encode_user_paged(S.cuda(), pool, pages)
+    m.poll()
+    kv, s_dense = m.encode_user(S.cuda())
+    m.poll()
+    assert torch.equal(s_tail, s_dense)

@@ -76,6 +76,10 @@ SIGNATURES = {
     "ot_encode_append": (_i, [_vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
     "ot_append_workspace_bytes": (_sz, [_vp, _i, _i]),
     "ot_set_act_scales": (_i, [_vp, _vp]),
+    "ot_kv_pages_per_user": (_i, [_vp]),
+    "ot_kv_page_bytes": (_sz, [_vp]),
+    "ot_encode_user_paged": (_i, [_vp, _vp, _i, _vp, _ll, _vp, _vp, _vp, _sz, _vp]),
+    "ot_score_candidates_paged": (_i, [_vp, _vp, _ll, _vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
     "ot_fp8_calibrate": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp, _sz, _vp]),
 }
 
@@ -335,6 +339,58 @@ class Model:
                                     ws.numel() * ws.element_size(), _stream(stream)),
               "ot_full_forward")
         return out_s_tail, out_ns
+
+    # paged KV cache
+    PAGE_ROWS = 128
+
+    def kv_pages_per_user(self) -> int:
+        return int(lib().ot_kv_pages_per_user(self.handle))
+
+    def kv_page_bytes(self) -> int:
+        return int(lib().ot_kv_page_bytes(self.handle))
+
+    def new_page_pool(self, n_pages: int):
+        """A pool of n_pages pages ([n_pages, 2, 128, d]: K rows, then V rows)."""
+        import torch
+        return torch.empty((n_pages, 2, self.PAGE_ROWS, self.d), dtype=self.storage, device="cuda")
+
+    def encode_user_paged(self, S, pool, pages, out_s_tail=None, ws=None, want_s_tail=True,
+                          stream=None):
+        """ot_encode_user into a paged cache: pool from new_page_pool, pages an
+        int32 CUDA tensor [U, kv_pages_per_user()] of page ids."""
+        import torch
+        U = S.shape[0]
+        if out_s_tail is None and want_s_tail:
+            out_s_tail = torch.empty(U, self.q[-1], self.d, dtype=self.storage, device=S.device)
+        ws = self._ws(ws, self.workspace_bytes(U, 0))
+        check(lib().ot_encode_user_paged(self.handle, _ptr(S), U, _ptr(pool), pool.shape[0],
+                                         _ptr(pages), _ptr(out_s_tail), _ptr(ws),
+                                         ws.numel() * ws.element_size(), _stream(stream)),
+              "ot_encode_user_paged")
+        return out_s_tail
+
+    def score_candidates_paged(self, pool, pages, ns, out=None, ws=None, stream=None):
+        import torch
+        U, Cn = ns.shape[0], ns.shape[1]
+        if out is None:
+            out = torch.empty_like(ns)
+        ws = self._ws(ws, self.workspace_bytes(U, Cn))
+        check(lib().ot_score_candidates_paged(self.handle, _ptr(pool), pool.shape[0], _ptr(pages), U,
+                                              _ptr(ns), Cn, _ptr(out), _ptr(ws),
+                                              ws.numel() * ws.element_size(), _stream(stream)),
+              "ot_score_candidates_paged")
+        return out
+
+    def kv_from_pages(self, pool, pages_u, l: int):
+        """(K, V) [L_l, d] of layer l of one user, gathered from its pages."""
+        import torch
+        L = self.rows_at(l)
+        off = sum((self.rows_at(j) + self.PAGE_ROWS - 1) // self.PAGE_ROWS for j in range(l))
+        nb = (L + self.PAGE_ROWS - 1) // self.PAGE_ROWS
+        pg = pages_u[off: off + nb].long()
+        K = pool[pg, 0].reshape(-1, self.d)[:L]
+        V = pool[pg, 1].reshape(-1, self.d)[:L]
+        return K, V
 
     # fp8 per-tensor scales
     def act_scale_shape(self) -> tuple:

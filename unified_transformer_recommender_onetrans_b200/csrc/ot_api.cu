@@ -135,6 +135,23 @@ inline long long kv_layer_off(const ot_config &c, int l)
 
 inline long long kv_user_elems(const ot_config &c) { return kv_layer_off(c, c.layers); }
 
+// Paged KV cache: first page-table entry of layer l (one entry per
+// OT_PAGE_ROWS rows of each layer) and the entries of one user.
+inline int page_off(const ot_config &c, int l)
+{
+    int off = 0;
+    for (int j = 0; j < l; ++j) off += (rows_at(c, j) + OT_PAGE_ROWS - 1) / OT_PAGE_ROWS;
+    return off;
+}
+
+// A paged cache as the runs address it.
+struct PagedKv {
+    void *pool;
+    const int *pages;
+    long long n_pages;
+    long long ustride; // page-table entries per user
+};
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 inline char *at(const void *base, long long elems, int esz)
@@ -549,6 +566,28 @@ AttnArgs attn_base(const ot_config &c, int mode, int U, int L, int nq, const voi
     return a;
 }
 
+// Read the S keys / values of layer l from a paged cache.
+void attn_paged(AttnArgs &a, const ot_config &c, const PagedKv *pg, int l)
+{
+    if (!pg) return;
+    a.KS = a.VS = pg->pool;
+    a.pages = pg->pages;
+    a.pg_ustride = pg->ustride;
+    a.n_pages = pg->n_pages;
+    a.pg_off = page_off(c, l);
+}
+
+// Write the K (kv = 0) or V (kv = 1) segment of layer l into a paged cache.
+void seg_paged(EpiSeg &s, const ot_config &c, const PagedKv *pg, int l, int kv)
+{
+    s.out = pg->pool;
+    s.pages = pg->pages;
+    s.pg_ustride = pg->ustride;
+    s.n_pages = pg->n_pages;
+    s.pg_off = page_off(c, l);
+    s.pg_kv = kv;
+}
+
 // S-side of every layer for U users, one layer at a time: qkv(l), then
 // rest(l) (attention, output projection, FFN).  X0: [U][L0][d]; s_out may
 // be null.  delta > 0 appends: X0 holds only the delta new rows per user,
@@ -578,6 +617,7 @@ struct EncodeRun {
     bool done = false; // the last layer ran its K/V projection only
     const void *ns_K = nullptr, *ns_V = nullptr;
     int ns_rows = 0;
+    const PagedKv *pg = nullptr; // the cache is paged (kv unused)
 
     ot_status init(const void *X0, Ws ws)
     {
@@ -638,13 +678,17 @@ struct EncodeRun {
             return r;
         if (kv_only) {
             g.nseg = 2;
-            g.seg[0] = seg_of(K(l), d, 0, d, cache_map);
-            g.seg[1] = seg_of(V(l), d, d, 2 * d, cache_map);
+            g.seg[0] = seg_of(pg ? nullptr : K(l), d, 0, d, cache_map);
+            g.seg[1] = seg_of(pg ? nullptr : V(l), d, d, 2 * d, cache_map);
         } else {
             g.nseg = 3;
             g.seg[0] = seg_of(Qb, d, 0, d, RowMap{n, q, -(n - q), 0, n - q});
-            g.seg[1] = seg_of(K(l), d, d, 2 * d, cache_map);
-            g.seg[2] = seg_of(V(l), d, 2 * d, 3 * d, cache_map);
+            g.seg[1] = seg_of(pg ? nullptr : K(l), d, d, 2 * d, cache_map);
+            g.seg[2] = seg_of(pg ? nullptr : V(l), d, 2 * d, 3 * d, cache_map);
+        }
+        if (pg) {
+            seg_paged(g.seg[kv_only ? 0 : 1], c, pg, l, 0);
+            seg_paged(g.seg[kv_only ? 1 : 2], c, pg, l, 1);
         }
         if ((r = gemm(m, g, st, ROLE_S_QKV)) != OT_OK) return r;
         if (kv_ready && cudaEventRecord(kv_ready[l], st) != cudaSuccess) return OT_ERR_CUDA;
@@ -662,7 +706,8 @@ struct EncodeRun {
         const int wesz = fp8 ? 1 : esz;
         const bool last = l == c.layers - 1;
         const void *g2 = fp8 ? at(m->g2_s, static_cast<long long>(l) * d, esz) : nullptr;
-        AttnArgs at_ = attn_base(c, 0, U, rows_at(c, l), q, Qb, K(l), V(l), Ab);
+        AttnArgs at_ = attn_base(c, 0, U, rows_at(c, l), q, Qb, pg ? nullptr : K(l), pg ? nullptr : V(l), Ab);
+        attn_paged(at_, c, pg, l);
         at_.KN = ns_K;
         at_.VN = ns_V;
         at_.nkn = ns_rows;
@@ -815,9 +860,10 @@ struct EncodeRun {
 
 ot_status run_encode(ot_model *m, const void *X0, int U, void *kv, void *s_out, Ws ws,
                      cudaStream_t st, cudaEvent_t *kv_ready = nullptr, int delta = 0,
-                     bool full_last = false)
+                     bool full_last = false, const PagedKv *pg = nullptr)
 {
     EncodeRun e{m, U, kv, s_out, st, kv_ready, delta, full_last};
+    e.pg = pg;
     ot_status r = e.init(X0, ws);
     for (int l = 0; r == OT_OK && l < m->cfg.layers && !e.done; ++l)
         if ((r = e.qkv(l)) == OT_OK) r = e.rest(l);
@@ -834,6 +880,7 @@ struct ScoreRun {
     void *out;
     cudaStream_t st;
     cudaEvent_t *kv_ready;
+    const PagedKv *pg = nullptr; // the cache is paged (kv unused)
     void *Xb[2], *Qn, *Kn, *Vn, *An, *Hn, *hid;
     Fp8Scratch f8{nullptr, nullptr};
     const void *X;
@@ -894,9 +941,10 @@ struct ScoreRun {
         const bool last = l == c.layers - 1;
         const long long lN = static_cast<long long>(l) * N;
         const void *g2 = fp8 ? at(m->g2_ns, lN * d, esz) : nullptr;
-        const char *K = at(kv, kv_layer_off(c, l), esz);
-        const char *V = K + static_cast<long long>(L) * d * esz;
+        const char *K = pg ? nullptr : at(kv, kv_layer_off(c, l), esz);
+        const char *V = pg ? nullptr : K + static_cast<long long>(L) * d * esz;
         AttnArgs at_ = attn_base(c, 1, U, L, C * N, Qn, K, V, An);
+        attn_paged(at_, c, pg, l);
         at_.KN = Kn;
         at_.VN = Vn;
         at_.nkn = C * N;
@@ -949,9 +997,10 @@ struct ScoreRun {
 };
 
 ot_status run_score(ot_model *m, const void *kv, int U, const void *ns, int C, void *out, Ws ws,
-                    cudaStream_t st, cudaEvent_t *kv_ready = nullptr)
+                    cudaStream_t st, cudaEvent_t *kv_ready = nullptr, const PagedKv *pg = nullptr)
 {
     ScoreRun sc{m, kv, U, C, out, st, kv_ready};
+    sc.pg = pg;
     ot_status r = sc.init(ns, ws);
     for (int l = 0; r == OT_OK && l < m->cfg.layers; ++l)
         if ((r = sc.qkv(l)) == OT_OK) r = sc.rest(l);
@@ -1513,6 +1562,70 @@ ot_status ot_score_candidates(ot_model *m, const void *kv_cache, int U, const vo
     if (ws_bytes < score_ws_bytes(m->cfg, U, C, m->esz)) return OT_ERR_WORKSPACE_TOO_SMALL;
     Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
     return run_score(m, kv_cache, U, ns, C, out_ns, w, static_cast<cudaStream_t>(stream));
+}
+
+int ot_kv_pages_per_user(const ot_model *m) { return m ? page_off(m->cfg, m->cfg.layers) : 0; }
+
+size_t ot_kv_page_bytes(const ot_model *m)
+{
+    return m ? 2 * static_cast<size_t>(OT_PAGE_ROWS) * m->cfg.d * m->esz : 0;
+}
+
+ot_status ot_encode_user_paged(ot_model *m, const void *S, int U, void *pool, long long n_pages,
+                               const int32_t *pages, void *out_s_tail, void *ws, size_t ws_bytes,
+                               void *stream)
+{
+    if (!m || !S || !pool || !pages || !ws || U < 1 || n_pages < 1) return OT_ERR_ARG;
+    if (m->cfg.full_attn) return OT_ERR_UNSUPPORTED;
+    if (!aligned16(S) || !aligned16(pool) || !aligned16(ws) || (reinterpret_cast<uintptr_t>(pages) & 3) ||
+        (out_s_tail && !aligned16(out_s_tail)))
+        return OT_ERR_ALIGN;
+    const ot_config &c = m->cfg;
+    if (static_cast<long long>(U) * c.L0 > (1LL << 31) - 1 || 2 * n_pages > (1LL << 31) - 1 ||
+        (static_cast<long long>(c.d) * m->esz) % 16)
+        return OT_ERR_SHAPE;
+    if (ws_bytes < ot_workspace_bytes(m, U, 0)) return OT_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const PagedKv pg{pool, pages, n_pages, page_off(c, c.layers)};
+    // the unused rows of every layer's last page hold zeros before any layer
+    // reads its keys (the kernels read whole key blocks)
+    PageTailArgs pt;
+    memset(&pt, 0, sizeof(pt));
+    pt.pool = pool;
+    pt.pages = pages;
+    pt.pg_ustride = pg.ustride;
+    pt.n_pages = n_pages;
+    pt.layers = c.layers;
+    pt.d = c.d;
+    pt.esz = m->esz;
+    pt.err = m->err;
+    for (int l = 0; l < c.layers; ++l) {
+        pt.L[l] = rows_at(c, l);
+        pt.off[l] = page_off(c, l);
+    }
+    ot_status r = profiled(m, st, OT_KIND_KV_GROW, ROLE_OTHER, 0.0, 0.0,
+                           [&] { return launch_page_tail_clear(pt, U, st); });
+    if (r != OT_OK) return r;
+    Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
+    return run_encode(m, S, U, nullptr, out_s_tail, w, st, nullptr, 0, false, &pg);
+}
+
+ot_status ot_score_candidates_paged(ot_model *m, const void *pool, long long n_pages,
+                                    const int32_t *pages, int U, const void *ns, int C,
+                                    void *out_ns, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!m || !pool || !pages || !ns || !out_ns || !ws || U < 1 || C < 1 || n_pages < 1) return OT_ERR_ARG;
+    if (m->cfg.full_attn) return OT_ERR_UNSUPPORTED;
+    if (!aligned16(pool) || !aligned16(ns) || !aligned16(out_ns) || !aligned16(ws) ||
+        (reinterpret_cast<uintptr_t>(pages) & 3))
+        return OT_ERR_ALIGN;
+    if (static_cast<long long>(U) * C * m->cfg.n_ns > (1LL << 31) - 1 ||
+        static_cast<long long>(C) * m->cfg.n_ns > (1LL << 30) || 2 * n_pages > (1LL << 31) - 1)
+        return OT_ERR_SHAPE;
+    if (ws_bytes < score_ws_bytes(m->cfg, U, C, m->esz)) return OT_ERR_WORKSPACE_TOO_SMALL;
+    const PagedKv pg{const_cast<void *>(pool), pages, n_pages, page_off(m->cfg, m->cfg.layers)};
+    Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
+    return run_score(m, nullptr, U, ns, C, out_ns, w, static_cast<cudaStream_t>(stream), nullptr, &pg);
 }
 
 ot_status ot_full_forward(ot_model *m, const void *S, const void *ns, int B, int C,

@@ -132,7 +132,13 @@ __global__ void __launch_bounds__(NA_WARPS * 32, 2)
         uint64_t *bar = &kv_full[warp * NA_STAGES + s];
         ++issued;
         mbar_arrive_expect_tx(bar, NA_STAGE);
-        if (b < P.nb_s) {
+        if (b < P.nb_s && a.pages) {
+            // paged cache: block b lies in page b / (OT_PAGE_ROWS / NA_KB)
+            constexpr int per = OT_PAGE_ROWS / NA_KB;
+            const int pg = static_cast<int>(attn_page(a, u, b / per));
+            tma_load_3d(k_dst, &tmKS, bar, h * NA_HD, (b % per) * NA_KB, 2 * pg);
+            tma_load_3d(v_dst, &tmVS, bar, h * NA_HD, (b % per) * NA_KB, 2 * pg + 1);
+        } else if (b < P.nb_s) {
             tma_load_3d(k_dst, &tmKS, bar, h * NA_HD, b * NA_KB, u);
             tma_load_3d(v_dst, &tmVS, bar, h * NA_HD, b * NA_KB, u);
         } else {
@@ -363,7 +369,14 @@ cudaError_t launch_attn_ns_small(const AttnArgs &a, cudaStream_t s)
     if (tmap_ns(&tq, a.Q, a.d, a.nq, a.U, nqd, NA_MAXQ) || tmap_ns(&tkn, a.KN, a.d, a.nq, a.U, nqd, NA_KB) ||
         tmap_ns(&tvn, a.VN, a.d, a.nq, a.U, nqd, NA_KB))
         return cudaErrorInvalidValue;
-    if (a.L > 0) {
+    if (a.L > 0 && a.pages) {
+        // paged cache: (d, OT_PAGE_ROWS rows, 2 n_pages), K / V of page p at 2 p / 2 p + 1
+        if (a.n_pages < 1 || 2 * a.n_pages > (1LL << 31) - 1 ||
+            tmap_ns(&tks, a.KS, a.d, OT_PAGE_ROWS, 2 * a.n_pages, static_cast<long long>(OT_PAGE_ROWS) * a.d,
+                    NA_KB))
+            return cudaErrorInvalidValue;
+        tvs = tks;
+    } else if (a.L > 0) {
         if (tmap_ns(&tks, a.KS, a.d, a.L, a.U, a.s_ustride, NA_KB) ||
             tmap_ns(&tvs, a.VS, a.d, a.L, a.U, a.s_ustride, NA_KB))
             return cudaErrorInvalidValue;

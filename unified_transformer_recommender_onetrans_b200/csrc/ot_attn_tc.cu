@@ -363,7 +363,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                     }
                     mbar_arrive_expect_tx(&kv_full[st], 2 * AT_TILE);
                     uint8_t *k_dst = sKV + 2 * st * AT_TILE, *v_dst = k_dst + AT_TILE;
-                    if (b < it.n_s_blocks) {
+                    if (b < it.n_s_blocks && a.pages) {
+                        // paged cache: one page per key block (K rows, then V rows)
+                        const int pg = static_cast<int>(attn_page(a, it.u, b));
+                        tma_load_3d(k_dst, &tmKS, &kv_full[st], it.h * AT_HD, 0, 2 * pg);
+                        tma_load_3d(v_dst, &tmVS, &kv_full[st], it.h * AT_HD, 0, 2 * pg + 1);
+                    } else if (b < it.n_s_blocks) {
                         tma_load_3d(k_dst, &tmKS, &kv_full[st], it.h * AT_HD, b * AT_BK, it.u);
                         tma_load_3d(v_dst, &tmVS, &kv_full[st], it.h * AT_HD, b * AT_BK, it.u);
                     } else {
@@ -652,10 +657,20 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
 {
     if (a.hd != AT_HD || a.dtype == OT_DTYPE_F32) return cudaErrorInvalidValue;
     alignas(64) CUtensorMap tq, tks, tvs, tkn, tvn;
-    if (tmap_rows(&tq, a.Q, a.d, a.nq, a.U, static_cast<long long>(a.nq) * a.d) ||
-        tmap_rows(&tks, a.KS, a.d, a.L, a.U, a.s_ustride) ||
-        tmap_rows(&tvs, a.VS, a.d, a.L, a.U, a.s_ustride))
+    if (tmap_rows(&tq, a.Q, a.d, a.nq, a.U, static_cast<long long>(a.nq) * a.d))
         return cudaErrorInvalidValue;
+    if (a.pages) {
+        // paged cache: the pool as (d, OT_PAGE_ROWS rows, 2 n_pages) -- K and V
+        // of page p are slices 2 p and 2 p + 1
+        static_assert(OT_PAGE_ROWS == AT_BK, "one page per key block");
+        if (a.n_pages < 1 || 2 * a.n_pages > (1LL << 31) - 1 ||
+            tmap_rows(&tks, a.KS, a.d, OT_PAGE_ROWS, 2 * a.n_pages, static_cast<long long>(OT_PAGE_ROWS) * a.d))
+            return cudaErrorInvalidValue;
+        tvs = tks;
+    } else if (tmap_rows(&tks, a.KS, a.d, a.L, a.U, a.s_ustride) ||
+               tmap_rows(&tvs, a.VS, a.d, a.L, a.U, a.s_ustride)) {
+        return cudaErrorInvalidValue;
+    }
     if (a.mode == 1 || a.full) {
         // NS keys / values: nkn rows per user (NS mode: the query rows themselves)
         const int nk = a.mode == 1 ? a.nq : a.nkn;

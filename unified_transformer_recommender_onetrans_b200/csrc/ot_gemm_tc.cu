@@ -177,7 +177,26 @@ __device__ __forceinline__ void epi_tile(const TcGemmParams &Q, int q, int lane,
     const RowMap mp{OT_SEGF(map.P), OT_SEGF(map.A), OT_SEGF(map.B), OT_SEGF(map.Gs), OT_SEGF(map.min_t)};
     e.obase = static_cast<__nv_bfloat16 *>(OT_SEGF(out));
     e.out_off = -1;
-    if (live && rowmap_keep_dev(mp, r)) e.out_off = rowmap_dev(mp, r, e.g) * OT_SEGF(ld) + (c0 - OT_SEGF(c_lo));
+    const int *pages = OT_SEGF(pages);
+    if (live && rowmap_keep_dev(mp, r)) {
+        if (pages) {
+            // paged KV cache: the row's page from the table (a bad id: no store)
+            EpiSeg sg;
+            sg.map = mp;
+            sg.pages = pages;
+            sg.pg_ustride = OT_SEGF(pg_ustride);
+            sg.n_pages = OT_SEGF(n_pages);
+            sg.pg_off = OT_SEGF(pg_off);
+            sg.pg_kv = OT_SEGF(pg_kv);
+            const long long pr = paged_row(sg, r);
+            if (pr >= 0)
+                e.out_off = pr * OT_SEGF(ld) + (c0 - OT_SEGF(c_lo));
+            else if (a.wait.err)
+                atomicCAS(a.wait.err, 0, OT_ERR_DEVICE_BOUNDS);
+        } else {
+            e.out_off = rowmap_dev(mp, r, e.g) * OT_SEGF(ld) + (c0 - OT_SEGF(c_lo));
+        }
+    }
 #undef OT_SEGF
     e.row_scale = live ? a.row_scale : nullptr;
     e.row_scale_idx = e.row_scale ? rowmap_dev(a.a_map, r, e.g) : 0;

@@ -41,12 +41,30 @@ __host__ __device__ inline bool rowmap_keep(const RowMap &m, long long r)
 
 // One output column segment [c_lo, c_hi) of a GEMM: written to
 // out + row(r, g) * ld + (c - c_lo).
+// Paged KV cache (pages != null): out is the page pool, each page K rows
+// [OT_PAGE_ROWS][d] then V rows; the GEMM row r is user u = r / map.P,
+// position t = r % map.P + map.B, and goes to row
+//   (page * 2 + pg_kv) * OT_PAGE_ROWS + t % OT_PAGE_ROWS,
+//   page = pages[u * pg_ustride + pg_off + t / OT_PAGE_ROWS].
 struct EpiSeg {
     void *out;
     long long ld;
     int c_lo, c_hi;
     RowMap map;
+    const int *pages;
+    long long pg_ustride, n_pages;
+    int pg_off, pg_kv;
 };
+
+// Row of the page pool for GEMM row r of a paged segment; -1 when the page
+// id is outside [0, n_pages) (the caller skips the store and reports it).
+__host__ __device__ inline long long paged_row(const EpiSeg &s, long long r)
+{
+    const long long u = r / s.map.P, t = r % s.map.P + s.map.B;
+    const long long page = s.pages[u * s.pg_ustride + s.pg_off + t / OT_PAGE_ROWS];
+    if (page < 0 || page >= s.n_pages) return -1;
+    return (page * 2 + s.pg_kv) * OT_PAGE_ROWS + t % OT_PAGE_ROWS;
+}
 
 enum { OT_STORE_F32 = 0, OT_STORE_BF16 = 1 };
 
@@ -93,6 +111,11 @@ struct AttnArgs {
     int N;              // NS tokens per candidate
     int full;           // 1: full attention
     int nkn;            // NS key rows per user in KN / VN (NS mode: nq)
+    // paged S keys / values (pages != null): KS = VS = the page pool, key
+    // block j / OT_PAGE_ROWS of user u in page pages[u * pg_ustride + pg_off + ...]
+    const int *pages;
+    long long pg_ustride, n_pages;
+    int pg_off;
     const void *Q;
     const void *KS, *VS;
     long long s_ustride; // elements between users in KS / VS
@@ -133,6 +156,19 @@ struct FfnArgs {
     // past a group's count are skipped (the experts of a mixture)
     const int *group_rows;
 };
+
+// Page of key block b (OT_PAGE_ROWS keys) of user u in a paged cache;
+// an id outside [0, n_pages) gives page 0 and sets the device error word,
+// so no access ever leaves the pool.
+__device__ inline long long attn_page(const AttnArgs &a, long long u, long long b)
+{
+    long long page = a.pages[u * a.pg_ustride + a.pg_off + b];
+    if (page < 0 || page >= a.n_pages) {
+        if (a.wait.err) atomicCAS(a.wait.err, 0, OT_ERR_DEVICE_BOUNDS);
+        page = 0;
+    }
+    return page;
+}
 
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel in the stream finishes; it must call pdl_wait() before
@@ -182,6 +218,16 @@ struct KvGrowArgs {
     long long len_src[OT_MAX_LAYERS], len_dst[OT_MAX_LAYERS];
 };
 cudaError_t launch_kv_grow(const KvGrowArgs &a, int users, int layers, cudaStream_t s);
+// Zero the unused rows of every layer's last page of a paged cache.
+struct PageTailArgs {
+    void *pool;
+    const int *pages;
+    long long pg_ustride, n_pages;
+    int layers, d, esz;
+    int L[OT_MAX_LAYERS], off[OT_MAX_LAYERS]; // rows and first page-table entry of each layer
+    int *err;
+};
+cudaError_t launch_page_tail_clear(const PageTailArgs &a, int users, cudaStream_t s);
 cudaError_t launch_embed_gather(const void *table, long long rows, int d, const int64_t *ids,
                                 long long n, void *out, int *err, cudaStream_t s);
 // Scale rule of an FP8 projection input (group g reads slot g * gstride):

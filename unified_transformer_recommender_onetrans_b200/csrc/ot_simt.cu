@@ -106,7 +106,17 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a)
             for (int s = 0; s < a.nseg; ++s) {
                 const EpiSeg &sg = a.seg[s];
                 if (c < sg.c_lo || c >= sg.c_hi || !rowmap_keep(sg.map, r)) continue;
-                st_out(sg.out, rowmap_apply(sg.map, r, g) * sg.ld + (c - sg.c_lo), a.store, v);
+                long long orow;
+                if (sg.pages) { // paged KV cache: a bad page id is reported, not written
+                    orow = paged_row(sg, r);
+                    if (orow < 0) {
+                        if (a.wait.err) atomicCAS(a.wait.err, 0, OT_ERR_DEVICE_BOUNDS);
+                        continue;
+                    }
+                } else {
+                    orow = rowmap_apply(sg.map, r, g);
+                }
+                st_out(sg.out, orow * sg.ld + (c - sg.c_lo), a.store, v);
             }
         }
     }
@@ -154,13 +164,21 @@ __global__ void __launch_bounds__(SA_ROWS) attn_simt_kernel(AttnArgs a)
     const int t_self = a.L - a.nq + i; // S mode: this row's S position
     const T *KS = static_cast<const T *>(a.KS) + static_cast<long long>(u) * a.s_ustride + h * HD;
     const T *VS = static_cast<const T *>(a.VS) + static_cast<long long>(u) * a.s_ustride + h * HD;
+    // key row j of this user: dense rows, or its page of a paged cache
+    auto key_off = [&](int j, int kv) -> long long {
+        if (!a.pages) return static_cast<long long>(j) * a.d;
+        const long long pg = attn_page(a, u, j / OT_PAGE_ROWS);
+        return ((pg * 2 + kv) * OT_PAGE_ROWS + j % OT_PAGE_ROWS) * a.d;
+    };
+    const T *KB = a.pages ? static_cast<const T *>(a.KS) + h * HD : KS;
+    const T *VB = a.pages ? static_cast<const T *>(a.KS) + h * HD : VS;
     for (int j0 = 0; j0 < s_keys; j0 += SA_KT) {
         __syncthreads();
         for (int e = threadIdx.x; e < SA_KT * HD; e += SA_ROWS) {
             int j = e / HD, c = e % HD;
             bool in = j0 + j < s_keys;
-            Ks[j][c] = in ? ld_f(KS + static_cast<long long>(j0 + j) * a.d + c) : 0.f;
-            Vs[j][c] = in ? ld_f(VS + static_cast<long long>(j0 + j) * a.d + c) : 0.f;
+            Ks[j][c] = in ? ld_f(KB + key_off(j0 + j, 0) + c) : 0.f;
+            Vs[j][c] = in ? ld_f(VB + key_off(j0 + j, 1) + c) : 0.f;
         }
         __syncthreads();
         if (!valid) continue;
@@ -289,6 +307,37 @@ cudaError_t launch_fold_gain(const void *W, const void *g, void *out, long long 
         fold_gain_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
             static_cast<const __nv_bfloat16 *>(W), static_cast<const __nv_bfloat16 *>(g),
             static_cast<__nv_bfloat16 *>(out), rows, cols, groups, g_gstride);
+    return cudaGetLastError();
+}
+
+// --------------------------------------------------------------------------
+// Paged KV cache: zero the unused rows of every layer's last page (rows
+// L_l % OT_PAGE_ROWS .. OT_PAGE_ROWS - 1, K and V), so the attention kernels,
+// which read whole key blocks, never multiply a masked probability by stale
+// values.  One CTA per (user, layer).
+__global__ void page_tail_clear_kernel(PageTailArgs a)
+{
+    const int u = blockIdx.x / a.layers, l = blockIdx.x % a.layers;
+    const int used = a.L[l] % OT_PAGE_ROWS;
+    if (used == 0) return;
+    long long pg = a.pages[static_cast<long long>(u) * a.pg_ustride + a.off[l] + a.L[l] / OT_PAGE_ROWS];
+    if (pg < 0 || pg >= a.n_pages) {
+        if (threadIdx.x == 0 && a.err) atomicCAS(a.err, 0, OT_ERR_DEVICE_BOUNDS);
+        return;
+    }
+    const long long row16 = static_cast<long long>(a.d) * a.esz / 16; // 16-byte units per row
+    uint4 *base = static_cast<uint4 *>(a.pool);
+    for (int kv = 0; kv < 2; ++kv) {
+        uint4 *p = base + ((pg * 2 + kv) * OT_PAGE_ROWS + used) * row16;
+        const long long n = (OT_PAGE_ROWS - used) * row16;
+        for (long long i = threadIdx.x; i < n; i += blockDim.x) p[i] = make_uint4(0, 0, 0, 0);
+    }
+}
+
+cudaError_t launch_page_tail_clear(const PageTailArgs &a, int users, cudaStream_t s)
+{
+    if ((static_cast<long long>(a.d) * a.esz) % 16) return cudaErrorInvalidValue;
+    page_tail_clear_kernel<<<users * a.layers, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 
