@@ -1,0 +1,108 @@
+"""Gradients of the OneTrans block stack: the oracle of the backward pass
+(TEST INFRASTRUCTURE ONLY; only tests/ and bench.py's CPU legs may use it).
+
+The forward is restated here in plain fp64 PyTorch ops, step by step as in
+onetrans_oracle.c (summary page, block / pyramid / KV-cache paragraphs):
+per user the S side layer by layer (RMSNorm, shared QKV, causal attention of
+the query tail over the layer's S keys, output projection, RMSNorm, GELU
+FFN, residuals; the next layer's S rows are the tail), and per candidate the
+NS side (private weights per NS position, attention over every S key of the
+layer and the candidate's NS keys m <= n).  The gradients are torch
+autograd's of the scalar loss
+    sum(s_out * G_s) + sum(ns_out * G_ns)
+for given upstream gradients G_s [U, q_last, d] and G_ns [U, C, N, d]:
+autograd is the library step; the restated forward is pinned to the C
+oracle and the gradients to central finite differences of the C oracle.
+
+Dense FFN and the causal mask only.
+"""
+
+from __future__ import annotations
+
+import math
+
+import torch
+
+W_NAMES = ("Wqkv_s", "Wo_s", "W1_s", "W2_s", "g1_s", "g2_s",
+           "Wqkv_ns", "Wo_ns", "W1_ns", "W2_ns", "g1_ns", "g2_ns")
+
+
+def _rms(x, g, eps):
+    return x * torch.rsqrt((x * x).mean(-1, keepdim=True) + eps) * g
+
+
+def _gelu(z):
+    return 0.5 * z * (1.0 + torch.erf(z / math.sqrt(2.0)))
+
+
+def _attend(q, k, v, mask, heads):
+    """q [Tq, d], k / v [Tk, d], mask [Tq, Tk] (True = visible) -> [Tq, d]."""
+    Tq, d = q.shape
+    hd = d // heads
+    qh = q.view(Tq, heads, hd).transpose(0, 1)
+    kh = k.view(-1, heads, hd).transpose(0, 1)
+    vh = v.view(-1, heads, hd).transpose(0, 1)
+    s = qh @ kh.transpose(1, 2) / math.sqrt(hd)
+    s = s.masked_fill(~mask, float("-inf"))
+    p = torch.softmax(s, dim=-1)
+    return (p @ vh).transpose(0, 1).reshape(Tq, d)
+
+
+def forward(cfg, w, S, ns):
+    """S [U, L0, d], ns [U, C, N, d] (fp64 tensors) -> (s_out [U, q_last, d],
+    ns_out [U, C, N, d]) with the weights of dict w (fp64 tensors)."""
+    d, H, N, eps = cfg.d, cfg.heads, cfg.n_ns, cfg.eps
+    s_outs, ns_outs = [], []
+    for u in range(S.shape[0]):
+        x = S[u]
+        kvs = []
+        for l in range(cfg.layers):
+            L, q = x.shape[0], cfg.q[l]
+            z = _rms(x, w["g1_s"][l], eps)
+            qkv = z @ w["Wqkv_s"][l].T
+            Q, K, V = qkv[L - q:, :d], qkv[:, d:2 * d], qkv[:, 2 * d:]
+            kvs.append((K, V))
+            t = torch.arange(L - q, L).unsqueeze(1)
+            mask = torch.arange(L).unsqueeze(0) <= t            # S row t sees S keys 0..t
+            a = _attend(Q, K, V, mask, H)
+            h = x[L - q:] + a @ w["Wo_s"][l].T
+            f = _gelu(_rms(h, w["g2_s"][l], eps) @ w["W1_s"][l].T) @ w["W2_s"][l].T
+            x = h + f
+        s_outs.append(x)
+        cand = []
+        for c in range(ns.shape[1]):
+            y = ns[u, c]
+            for l in range(cfg.layers):
+                K_s, V_s = kvs[l]
+                L = K_s.shape[0]
+                rows = []
+                qkv = torch.stack([_rms(y[n], w["g1_ns"][l, n], eps) @ w["Wqkv_ns"][l, n].T
+                                   for n in range(N)])
+                Qn, Kn, Vn = qkv[:, :d], qkv[:, d:2 * d], qkv[:, 2 * d:]
+                K = torch.cat([K_s, Kn])
+                V = torch.cat([V_s, Vn])
+                mask = torch.cat([torch.ones(N, L, dtype=torch.bool),
+                                  torch.arange(N).unsqueeze(0) <= torch.arange(N).unsqueeze(1)], dim=1)
+                a = _attend(Qn, K, V, mask, H)
+                for n in range(N):
+                    h = y[n] + a[n] @ w["Wo_ns"][l, n].T
+                    f = _gelu(_rms(h, w["g2_ns"][l, n], eps) @ w["W1_ns"][l, n].T) @ w["W2_ns"][l, n].T
+                    rows.append(h + f)
+                y = torch.stack(rows)
+            cand.append(y)
+        ns_outs.append(torch.stack(cand))
+    return torch.stack(s_outs), torch.stack(ns_outs)
+
+
+def gradients(cfg, w, S, ns, G_s, G_ns):
+    """(loss, grads): grads maps "S", "ns" and every weight name to the
+    gradient of sum(s_out * G_s) + sum(ns_out * G_ns), fp64 CPU tensors."""
+    wt = {k: torch.as_tensor(w[k]).detach().double().clone().requires_grad_(True) for k in W_NAMES}
+    St = torch.as_tensor(S).detach().double().clone().requires_grad_(True)
+    nst = torch.as_tensor(ns).detach().double().clone().requires_grad_(True)
+    s_out, ns_out = forward(cfg, wt, St, nst)
+    loss = (s_out * torch.as_tensor(G_s).double()).sum() + (ns_out * torch.as_tensor(G_ns).double()).sum()
+    loss.backward()
+    grads = {"S": St.grad, "ns": nst.grad}
+    grads.update({k: wt[k].grad for k in W_NAMES})
+    return float(loss.detach()), grads

@@ -695,3 +695,60 @@ def test_embed_gather_matches_numpy():
     assert np.array_equal(out, table.double().numpy()[ids.numpy()])
     with pytest.raises(IndexError):
         O.embed_gather(table, np.array([50]))
+
+
+# ----------------------------------------------------------------- backward
+def _bw_case(seed=150):
+    layers, d, H, f, N, L0, q = 2, 8, 2, 12, 2, 7, [5, 3]
+    w = rand_weights(layers, d, f, N, seed=seed, dtype=torch.float64)
+    w = {k: v.float().double() for k, v in w.items()}
+    S, ns = rand_inputs(2, 2, L0, N, d, seed=seed + 1, dtype=torch.float64)
+    S, ns = S.float().double(), ns.float().double()
+    g = torch.Generator().manual_seed(seed + 2)
+    G_s = torch.randn(2, q[-1], d, generator=g, dtype=torch.float64)
+    G_ns = torch.randn(2, 2, N, d, generator=g, dtype=torch.float64)
+    return cfg_of(layers, d, H, f, N, L0, q), w, S, ns, G_s, G_ns
+
+
+def test_backward_oracle_forward_matches_c_oracle():
+    """The PyTorch restatement the gradients come from computes what the
+    pinned C oracle computes (the S tails and the NS outputs)."""
+    from oracle import backward as OB
+    cfg, w, S, ns, _, _ = _bw_case()
+    s_t, ns_t = OB.forward(cfg, w, S, ns)
+    kv, s_c = O.encode_user(cfg, w, S)
+    ns_c = O.score_candidates(cfg, w, kv, ns)
+    np.testing.assert_allclose(s_t.detach().numpy(), s_c, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(ns_t.detach().numpy(), ns_c, rtol=0, atol=1e-12)
+
+
+def test_backward_oracle_matches_finite_differences():
+    """Every gradient along random directions against central differences of
+    the C oracle's loss: (L(p + e v) - L(p - e v)) / 2e = grad . v."""
+    from oracle import backward as OB
+    cfg, w, S, ns, G_s, G_ns = _bw_case()
+    _, grads = OB.gradients(cfg, w, S, ns, G_s, G_ns)
+
+    def loss(w_, S_, ns_):
+        kv, s_c = O.encode_user(cfg, w_, S_.float())
+        return float((s_c * G_s.numpy()).sum() +
+                     (O.score_candidates(cfg, w_, kv, ns_) * G_ns.numpy()).sum())
+
+    g = torch.Generator().manual_seed(7)
+    eps = 1e-3
+    for name in ["S", "ns"] + list(OB.W_NAMES):
+        base = {"S": S, "ns": ns}.get(name, w.get(name))
+        v = torch.randn(base.shape, generator=g, dtype=torch.float64)
+        # float32-representable probes (the C oracle reads its inputs as float32)
+        p_plus, p_minus = (base + eps * v).float().double(), (base - eps * v).float().double()
+        step = (p_plus - p_minus).double() / 2
+
+        def with_(p):
+            if name == "S":
+                return w, p, ns
+            if name == "ns":
+                return w, S, p
+            return dict(w, **{name: p}), S, ns
+        fd = (loss(*with_(p_plus)) - loss(*with_(p_minus)))
+        an = 2.0 * float((grads[name] * step).sum())
+        assert abs(fd - an) <= 2e-5 * max(1.0, abs(an)), (name, fd, an)
