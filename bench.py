@@ -582,6 +582,74 @@ def run_moe_point(name, experts, topk, steps, flush, world, dist, dev, peaks):
             "ms_by_role_serialised": by_role}
 
 
+def forward_flops(wl, q, U, C) -> float:
+    """Algorithmic FLOPs of one forward of U users x C candidates: the
+    projections and FFNs of both sides, and 4 d FLOPs per attended
+    (query, key) pair (Q K^T and P V)."""
+    d, f, N = wl.d, wl.ffn, wl.n_ns
+    L, total = wl.L0, 0.0
+    RN = U * C * N
+    for ql in q:
+        pairs_s = ql * (L - ql) + ql * (ql + 1) // 2
+        pairs_ns = N * L + N * (N + 1) // 2
+        total += 2.0 * U * L * 3 * d * d + 4.0 * d * U * pairs_s
+        total += 2.0 * U * ql * d * d + 4.0 * U * ql * d * f
+        total += 2.0 * RN * 3 * d * d + 4.0 * d * U * C * pairs_ns + 2.0 * RN * d * d + 4.0 * RN * d * f
+        L = ql
+    return total
+
+
+def run_backward_point(name, users, steps, flush, world, dist, dev, peaks):
+    """One training step of the workload's shapes in fp32 through
+    ot_full_backward: checkpointing forward, then per layer (top first) the
+    recomputed forward and the gradients of every weight, gain and input.
+    Synthetic S rows of the workload, seeded NS rows and upstream gradients."""
+    import torch
+
+    import unified_transformer_recommender_onetrans_b200 as ot
+    from synth import WORKLOADS, gen_s_tokens, gen_weights
+
+    wl = WORKLOADS[name].with_(dtype="f32", users=users, cands=1)
+    w = gen_weights(wl)
+    q = ot.pyramid_schedule(wl.L0, wl.q_end, wl.layers)
+    cfg = ot.make_config(layers=wl.layers, d=wl.d, heads=wl.heads, ffn=wl.ffn, n_ns=wl.n_ns,
+                         L0=wl.L0, q=q, eps=wl.eps)
+    U, C = wl.users, wl.cands
+    g = torch.Generator().manual_seed(21)
+    S = gen_s_tokens(wl, weights=w).to(dev)
+    ns = torch.randn(U, C, wl.n_ns, wl.d, generator=g).to(dev)
+    G_s = torch.randn(U, q[-1], wl.d, generator=g).to(dev)
+    G_ns = torch.randn(U, C, wl.n_ns, wl.d, generator=g).to(dev)
+    wd = {k: w[k].to(dev) for k in ot.GRAD_NAMES}
+    del w
+    grads = {k: torch.empty_like(wd[k]) for k in ot.GRAD_NAMES}
+    dS, dns = torch.empty_like(S), torch.empty_like(ns)
+    s_tail = torch.empty(U, q[-1], wl.d, device=dev)
+    out_ns = torch.empty_like(ns)
+    ws = torch.empty(ot.backward_workspace_bytes(cfg, U, C), dtype=torch.uint8, device=dev)
+
+    def step():
+        ot.full_backward(cfg, wd, S, ns, G_s, G_ns, grads=grads, dS=dS, dns=dns,
+                         out_s_tail=s_tail, out_ns=out_ns, ws=ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    ms = _time_device(step, steps, flush, world, dist, dev)
+    F = forward_flops(wl, q, U, C)
+    # fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 FLOPs x max SM clock
+    fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    model = 3 * F / (ms / 1e3) / 1e12
+    executed = 4 * F / (ms / 1e3) / 1e12
+    return {"workload": name, "dtype": "f32", "training_step": "ot_full_backward (checkpointed)",
+            "users": U, "cands": C, "ms": ms, "s_tokens_per_s": world * U * wl.L0 / (ms / 1e3),
+            "launches": ot.backward_launches(cfg, U, C),
+            "model_tflops": model, "executed_tflops": executed,
+            "fp32_peak_tflops": fp32_peak, "executed_frac_fp32_peak": executed / fp32_peak,
+            "flops_rule": "model = 3 x forward FLOPs (forward + backward); executed adds the "
+                          "recomputed forward (4 x)"}
+
+
 def run_full_point(name, steps, flush, world, dist, dev, peaks):
     """Auto-Split + full forward of a whole workload batch (C candidates per
     user, S and NS sides in one call), 10 warm-ups + median of `steps` calls."""
@@ -763,6 +831,7 @@ def run_ours(args, wl):
         serving.append(run_full_point("onetrans_l_full", 50, flush, world, dist, dev, peaks))
         torch.cuda.empty_cache()
         serving.append(run_moe_point("onetrans_s_full", 8, 2, 20, flush, world, dist, dev, peaks))
+        serving.append(run_backward_point("onetrans_s_full", 16, 5, flush, world, dist, dev, peaks))
         torch.cuda.empty_cache()
 
     # ---- roofline of the dominant kernel (from the live per-launch events)

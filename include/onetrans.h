@@ -106,7 +106,7 @@ typedef enum { OT_DTYPE_F32 = 0, OT_DTYPE_BF16 = 1, OT_DTYPE_FP8 = 2 } ot_dtype;
  * W_router z; the moe_topk (1 or 2) largest, ties to the lower expert index,
  * are softmax-ed into gates g_j, and y = h + sum_j g_j W2_e GELU(W1_e z),
  * each expert of the dense FFN's shape.  NS tokens keep their private dense
- * FFNs.  E <= 64, d <= 256; bf16 or fp32 (not fp8). */
+ * FFNs.  E <= 64, d of 64, 128 or 256; bf16 or fp32 (not fp8). */
 typedef struct {
     int layers, d, heads, ffn, n_ns, L0;
     int q[OT_MAX_LAYERS];
@@ -384,6 +384,48 @@ typedef struct {
 
 ot_status ot_profile_enable(ot_model *m, int enable);
 int ot_profile_read(ot_model *m, ot_launch_record *out, int max);
+
+/* ---- Backward pass (training) ----
+ * The summary page lists activation checkpointing among the training
+ * optimisations on top of the stack (systems paragraph).  ot_full_backward
+ * computes, for an fp32 config with the causal mask and dense FFNs, the
+ * gradients of
+ *     loss = sum(s_tail * G_s) + sum(ns_out * G_ns)
+ * (s_tail, ns_out: the outputs of ot_full_forward; G_s, G_ns: the upstream
+ * gradients) with respect to every weight and gain and to S and ns.
+ * Activation checkpointing: a forward pass keeps only each layer's input
+ * rows; the backward then recomputes one layer at a time from them, top
+ * layer first, and takes its gradients.  CUDA-core fp32 kernels.
+ * All pointers are device pointers to fp32, 16-byte aligned:
+ *   w      the twelve dense tensors of ot_weights (Wqkv_s .. g2_ns), fp32,
+ *          gains NOT folded (W_split and the MoE fields are not read);
+ *   S [U][L0][d], ns [U][C][N][d], G_s [U][q_last][d], G_ns [U][C][N][d];
+ *   out_s_tail [U][q_last][d], out_ns [U][C][N][d]: the forward's outputs
+ *          (NULL: not written);
+ *   g      gradients in the weights' shapes, all twelve non-NULL,
+ *          overwritten (not accumulated);
+ *   dS [U][L0][d], dns [U][C][N][d] (NULL: not written).
+ * C = 0 runs the S side alone (ns, G_ns, out_ns and dns are not read or
+ * written; the NS gradients are set to zero).  No atomics: the same inputs
+ * give the same bits.  Nothing is allocated; ws >=
+ * ot_backward_workspace_bytes(cfg, U, C).  Errors, in this order:
+ * OT_ERR_ARG (null pointer, U < 1, C < 0, a bad config field),
+ * OT_ERR_DTYPE (not OT_DTYPE_F32), OT_ERR_UNSUPPORTED (full_attn or
+ * moe_experts), OT_ERR_SHAPE (the config rules; rows beyond the kernels'
+ * 32-bit row counts), OT_ERR_ALIGN, OT_ERR_WORKSPACE_TOO_SMALL,
+ * OT_ERR_CUDA. */
+typedef struct {
+    float *Wqkv_s, *Wo_s, *W1_s, *W2_s, *g1_s, *g2_s;
+    float *Wqkv_ns, *Wo_ns, *W1_ns, *W2_ns, *g1_ns, *g2_ns;
+} ot_grads;
+
+size_t ot_backward_workspace_bytes(const ot_config *cfg, int U, int C);
+/* Kernel launches one ot_full_backward call issues (0 for a rejected shape). */
+long long ot_backward_launches(const ot_config *cfg, int U, int C);
+ot_status ot_full_backward(const ot_config *cfg, const ot_weights *w, const float *S, const float *ns,
+                           int U, int C, const float *G_s, const float *G_ns, float *out_s_tail,
+                           float *out_ns, const ot_grads *g, float *dS, float *dns, void *ws,
+                           size_t ws_bytes, void *stream);
 
 /* Static string for a status code. */
 const char *ot_status_str(ot_status s);

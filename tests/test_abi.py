@@ -111,3 +111,55 @@ def test_product_path_does_not_import_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in src.replace("oracle-free", ""), f
+
+
+def _bw_args(cfg, U=2, Cn=3, misalign=None, ws_bytes=None):
+    """ot_full_backward arguments with placeholder (never dereferenced)
+    device addresses: the host checks return before any device work."""
+    names = list(B.GRAD_NAMES)
+    w = B.OtWeights(**{n: 4096 * (i + 1) for i, n in enumerate(names)})
+    g = B.OtGrads(**{n: 4096 * (i + 101) for i, n in enumerate(names)})
+    if misalign:
+        setattr(g, misalign, getattr(g, misalign) + 4)
+    nbytes = lib_bw_bytes(cfg, U, Cn) if ws_bytes is None else ws_bytes
+    return (C.byref(cfg), C.byref(w), 1 << 20, 2 << 20, U, Cn, 3 << 20, 4 << 20, 0, 0, C.byref(g),
+            0, 0, 5 << 20, nbytes, None)
+
+
+def lib_bw_bytes(cfg, U, Cn):
+    return B.lib().ot_backward_workspace_bytes(C.byref(cfg), U, Cn)
+
+
+def test_backward_host_checks(lib):
+    f32 = dict(dtype=0, d=64, heads=2, ffn=96, n_ns=3, L0=40, q=[40, 10])
+    cfg = _cfg(**f32)
+    ws = lib_bw_bytes(cfg, 2, 3)
+    assert ws > 0 and ws % 256 == 0
+    # the workspace grows with the batch; C = 0 needs no NS buffers
+    assert lib_bw_bytes(cfg, 4, 3) > ws > lib_bw_bytes(cfg, 2, 0) > 0
+    assert lib.ot_full_backward(None, None, None, None, 1, 1, None, None, None, None, None, None,
+                                None, None, 0, None) == 1
+    assert lib.ot_full_backward(*_bw_args(_cfg(**dict(f32, dtype=1)))) == 3          # bf16
+    assert lib.ot_full_backward(*_bw_args(_cfg(**dict(f32, full_attn=1)))) == 10
+    assert lib.ot_full_backward(*_bw_args(_cfg(**dict(f32, moe_experts=4, moe_topk=1)))) == 10
+    assert lib.ot_full_backward(*_bw_args(_cfg(**dict(f32, q=[41, 10])))) == 2
+    assert lib.ot_full_backward(*_bw_args(cfg, misalign="W1_ns")) == 4
+    assert lib.ot_full_backward(*_bw_args(cfg, ws_bytes=ws - 1)) == 6
+    args = list(_bw_args(cfg))
+    args[4] = 0                                                                      # U = 0
+    assert lib.ot_full_backward(*args) == 1
+    assert lib_bw_bytes(_cfg(**dict(f32, dtype=1)), 2, 3) == 0
+
+
+def test_backward_launch_count(lib):
+    """Kernel launches per call.  Per layer, with candidates: the forward is
+    8 launches per side (norm, QKV, attention, O, norm, FFN1, GELU, FFN2),
+    7 when only recomputed (no output GEMM); the backward 10 per side for the
+    FFN and O projection, 4 attention kernels, 5 per side for QKV and the
+    first norm, 1 residual add.  The top layer is not recomputed."""
+    f32 = dict(dtype=0, d=64, heads=2, ffn=96, n_ns=3, L0=40)
+    for layers, q in ((1, [40]), (2, [40, 10]), (3, [40, 20, 5])):
+        c = _cfg(**dict(f32, layers=layers, q=q))
+        assert lib.ot_backward_launches(C.byref(c), 2, 3) == 16 * layers + 14 * (layers - 1) + 35 * layers
+        assert lib.ot_backward_launches(C.byref(c), 2, 0) == 8 * layers + 7 * (layers - 1) + 18 * layers
+    assert lib.ot_backward_launches(C.byref(_cfg(**dict(f32, dtype=1, layers=1, q=[40]))), 2, 3) == 0

@@ -6,11 +6,16 @@ Build it with ``python -m unified_transformer_recommender_onetrans_b200.build``.
 """
 
 from .binding import (  # noqa: F401
+    GRAD_NAMES,
     LIB_PATH,
     SIGNATURES,
     Model,
     OtError,
+    backward_launches,
+    backward_workspace_bytes,
     embed_gather,
+    full_backward,
     lib,
+    make_config,
     pyramid_schedule,
 )

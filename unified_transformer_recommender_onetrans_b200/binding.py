@@ -42,6 +42,14 @@ class OtWeights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in WEIGHT_NAMES + MOE_WEIGHT_NAMES]
 
 
+# the tensors ot_full_backward differentiates (fp32, gains not folded)
+GRAD_NAMES = WEIGHT_NAMES[:12]
+
+
+class OtGrads(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in GRAD_NAMES]
+
+
 class OtLaunchRecord(C.Structure):
     _fields_ = [("kind", C.c_int), ("role", C.c_int), ("ms", C.c_float), ("flops", C.c_double),
                 ("bytes", C.c_double)]
@@ -81,6 +89,10 @@ SIGNATURES = {
     "ot_encode_user_paged": (_i, [_vp, _vp, _i, _vp, _ll, _vp, _vp, _vp, _sz, _vp]),
     "ot_score_candidates_paged": (_i, [_vp, _vp, _ll, _vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
     "ot_fp8_calibrate": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp, _sz, _vp]),
+    "ot_backward_workspace_bytes": (_sz, [C.POINTER(OtConfig), _i, _i]),
+    "ot_backward_launches": (_ll, [C.POINTER(OtConfig), _i, _i]),
+    "ot_full_backward": (_i, [C.POINTER(OtConfig), C.POINTER(OtWeights), _vp, _vp, _i, _i, _vp,
+                              _vp, _vp, _vp, C.POINTER(OtGrads), _vp, _vp, _vp, _sz, _vp]),
 }
 
 _lib = None
@@ -451,3 +463,59 @@ def embed_gather(table, ids, out=None, err=None, stream=None):
     check(lib().ot_embed_gather(_ptr(table), table.shape[0], d, _ptr(ids), n, _ptr(out),
                                 _ptr(err), _stream(stream)), "ot_embed_gather")
     return out
+
+
+# ------------------------------------------------------------------ training
+def make_config(*, layers, d, heads, ffn, n_ns, L0, q, F=0, eps=1e-6, dtype="f32",
+                full_attn=False, moe_experts=0, moe_topk=1) -> OtConfig:
+    cfg = OtConfig()
+    cfg.layers, cfg.d, cfg.heads, cfg.ffn, cfg.n_ns, cfg.L0 = layers, d, heads, ffn, n_ns, L0
+    for i, v in enumerate(q):
+        cfg.q[i] = int(v)
+    cfg.F, cfg.eps, cfg.dtype = F, eps, DTYPES[dtype]
+    cfg.full_attn, cfg.moe_experts, cfg.moe_topk = int(bool(full_attn)), moe_experts, moe_topk
+    return cfg
+
+
+def backward_workspace_bytes(cfg: OtConfig, users: int, cands: int) -> int:
+    return lib().ot_backward_workspace_bytes(C.byref(cfg), users, cands)
+
+
+def backward_launches(cfg: OtConfig, users: int, cands: int) -> int:
+    return lib().ot_backward_launches(C.byref(cfg), users, cands)
+
+
+def full_backward(cfg: OtConfig, weights: dict, S, ns, G_s, G_ns, *, grads=None, dS=None,
+                  dns=None, out_s_tail=None, out_ns=None, ws=None, want_outputs=True,
+                  want_input_grads=True, stream=None):
+    """ot_full_backward on fp32 CUDA tensors.  ``weights``: the twelve dense
+    tensors of GRAD_NAMES (gains not folded).  Returns (s_tail, ns_out,
+    grads, dS, dns); the gradients are those of sum(s_tail * G_s) +
+    sum(ns_out * G_ns)."""
+    import torch
+    U, Cn = S.shape[0], (ns.shape[1] if ns is not None else 0)
+    dev = S.device
+    if grads is None:
+        grads = {k: torch.empty_like(weights[k]) for k in GRAD_NAMES}
+    if want_outputs:
+        if out_s_tail is None:
+            out_s_tail = torch.empty(U, cfg.q[cfg.layers - 1], cfg.d, dtype=torch.float32, device=dev)
+        if out_ns is None and Cn:
+            out_ns = torch.empty_like(ns)
+    if want_input_grads:
+        if dS is None:
+            dS = torch.empty_like(S)
+        if dns is None and Cn:
+            dns = torch.empty_like(ns)
+    nbytes = backward_workspace_bytes(cfg, U, Cn)
+    if ws is None:
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    w = OtWeights(**{k: _ptr(weights[k]) for k in GRAD_NAMES})
+    g = OtGrads(**{k: _ptr(grads[k]) for k in GRAD_NAMES})
+    check(lib().ot_full_backward(C.byref(cfg), C.byref(w), _ptr(S), _ptr(ns) if Cn else 0, U, Cn,
+                                 _ptr(G_s), _ptr(G_ns) if Cn else 0, _ptr(out_s_tail),
+                                 _ptr(out_ns) if Cn else 0, C.byref(g), _ptr(dS),
+                                 _ptr(dns) if Cn else 0, _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)),
+          "ot_full_backward")
+    return out_s_tail, out_ns, grads, dS, dns

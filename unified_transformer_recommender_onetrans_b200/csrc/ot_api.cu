@@ -171,7 +171,7 @@ ot_status check_config(const ot_config &c)
     if (c.moe_experts > 0) {
         if (c.moe_topk < 1 || c.moe_topk > 2 || c.moe_topk > c.moe_experts) return OT_ERR_ARG;
         if (c.dtype == OT_DTYPE_FP8) return OT_ERR_DTYPE;
-        if (c.d % 32 || c.d > 256) return OT_ERR_SHAPE;
+        if (c.d != 64 && c.d != 128 && c.d != 256) return OT_ERR_SHAPE; // the router's row widths
     }
     if (c.d % c.heads) return OT_ERR_SHAPE;
     int L = c.L0;
@@ -1167,6 +1167,8 @@ ot_status device_quant(ot_model *m, void **dst, float **scales, const void *W, l
 } // namespace
 
 namespace ot {
+ot_status internal_check_config(const ot_config &c) { return check_config(c); }
+
 size_t internal_score_ws_bytes(const ot_model *m, int users, int cands)
 {
     if (!m || users < 1 || cands < 1) return 0;

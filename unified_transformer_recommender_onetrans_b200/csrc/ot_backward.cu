@@ -1,0 +1,952 @@
+// Backward pass of the block stack: ot_full_backward (fp32 models, the
+// OneTrans causal mask, dense FFNs).  The summary page puts activation
+// checkpointing on top of the stack for training (systems paragraph): a
+// forward pass keeps every layer's input rows only, and the backward
+// recomputes one layer at a time from them, top layer first, before taking
+// its gradients.  CUDA-core fp32 kernels, deterministic (no atomics).
+//
+// Per layer l (S rows X [U][L][d], query tail q; NS rows Y [U][C][N][d]):
+//   recompute  Z1 = n(X; g1), QKV = Z1 Wqkv^T, A = attn(QKV), H = X_tail +
+//              A Wo^T, Z2 = n(H; g2), U1 = Z2 W1^T, Act = GELU(U1); the NS
+//              side the same with its private weights per position n
+//              (grouped GEMMs, group = n) and attention over the layer's S
+//              keys and the candidate's NS keys m <= n;
+//   gradients  dH = dOut + n'(dOut W2 * GELU'(U1) W1), dW2 = dOut^T Act,
+//              dW1 = dU1^T Z2, dA = dH Wo, dWo = dH^T A; attention: dQ per
+//              query row, dK / dV per key row (S keys collect the S tail
+//              rows at or after them and every NS row of the user);
+//              dWqkv = dQKV^T Z1, dX = n'(dQKV Wqkv) + dH on the tail rows.
+// n'(.) is the RMSNorm backward: with r = (mean(x^2) + eps)^(-1/2),
+//   dx = r g dz - x r^3 mean(x g dz),  dg = sum over rows of dz x r.
+#include <math.h>
+#include <stdint.h>
+
+#include "ot_internal.h"
+
+namespace ot {
+
+__device__ __forceinline__ float bw_warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ long long bw_warp_id()
+{
+    return (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
+}
+
+__device__ __forceinline__ long long bw_warp_count()
+{
+    return (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+}
+
+// ---------------------------------------------------------------- RMSNorm
+// One warp per row; rows are taken group-major (row r of group g is warp
+// item g * rows + r).
+__global__ void rms_fwd_kernel(BwRows a, const float *g, long long g_gstride, float eps, float *z,
+                               float *r_out)
+{
+    const int lane = threadIdx.x & 31;
+    for (long long w = bw_warp_id(); w < a.rows * a.G; w += bw_warp_count()) {
+        const long long grp = w / a.rows, R = rowmap_apply(a.map, w % a.rows, grp);
+        const float *x = a.X + R * a.d;
+        const float *gg = g + grp * g_gstride;
+        float ss = 0.f;
+        for (int k = lane; k < a.d; k += 32) ss = fmaf(x[k], x[k], ss);
+        const float rs = 1.0f / sqrtf(bw_warp_sum(ss) / static_cast<float>(a.d) + eps);
+        for (int k = lane; k < a.d; k += 32) z[R * a.d + k] = x[k] * rs * gg[k];
+        if (lane == 0) r_out[R] = rs;
+    }
+}
+
+__global__ void rms_bwd_kernel(BwRows a, const float *g, long long g_gstride, const float *r_in,
+                               const float *dz, float *dx, int accumulate)
+{
+    const int lane = threadIdx.x & 31;
+    for (long long w = bw_warp_id(); w < a.rows * a.G; w += bw_warp_count()) {
+        const long long grp = w / a.rows, R = rowmap_apply(a.map, w % a.rows, grp);
+        const float *x = a.X + R * a.d;
+        const float *dzr = dz + R * a.d;
+        const float *gg = g + grp * g_gstride;
+        const float rs = r_in[R];
+        float s = 0.f;
+        for (int k = lane; k < a.d; k += 32) s = fmaf(x[k] * gg[k], dzr[k], s);
+        const float c = bw_warp_sum(s) * rs * rs * rs / static_cast<float>(a.d);
+        float *dxr = dx + R * a.d;
+        for (int k = lane; k < a.d; k += 32) {
+            const float v = rs * gg[k] * dzr[k] - x[k] * c;
+            dxr[k] = accumulate ? dxr[k] + v : v;
+        }
+    }
+}
+
+// Gain gradient in two deterministic steps: partial column sums over row
+// chunks ([splits][G][d]), then their sum in chunk order.
+__global__ void gain_partial_kernel(BwRows a, const float *r_in, const float *dz, float *partial, int splits)
+{
+    __shared__ float red[8][33];
+    const int k = blockIdx.x * 32 + threadIdx.x, grp = blockIdx.y, zc = blockIdx.z;
+    const long long chunk = (a.rows + splits - 1) / splits;
+    const long long r0 = zc * chunk, r1 = min(a.rows, r0 + chunk);
+    float acc = 0.f;
+    if (k < a.d)
+        for (long long r = r0 + threadIdx.y; r < r1; r += 8) {
+            const long long R = rowmap_apply(a.map, r, grp);
+            acc = fmaf(dz[R * a.d + k] * a.X[R * a.d + k], r_in[R], acc);
+        }
+    red[threadIdx.y][threadIdx.x] = acc;
+    __syncthreads();
+    if (threadIdx.y == 0 && k < a.d) {
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s += red[i][threadIdx.x];
+        partial[(static_cast<long long>(zc) * a.G + grp) * a.d + k] = s;
+    }
+}
+
+__global__ void gain_reduce_kernel(const float *partial, int splits, int G, int d, float *dg, long long g_gstride)
+{
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < static_cast<long long>(G) * d;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long grp = i / d, k = i % d;
+        float s = 0.f;
+        for (int zc = 0; zc < splits; ++zc) s += partial[(static_cast<long long>(zc) * G + grp) * d + k];
+        dg[grp * g_gstride + k] = s;
+    }
+}
+
+// ---------------------------------------------------------------- elementwise
+__global__ void gelu_fwd_kernel(const float *u, float *a, long long n)
+{
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x)
+        a[i] = 0.5f * u[i] * (1.0f + erff(u[i] * 0.70710678118654752f));
+}
+
+// d GELU(u) / du = Phi(u) + u phi(u) (exact-erf GELU); du may alias da.
+__global__ void gelu_bwd_kernel(const float *u, const float *da, float *du, long long n)
+{
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const float x = u[i];
+        const float cdf = 0.5f * (1.0f + erff(x * 0.70710678118654752f));
+        const float pdf = 0.39894228040143268f * expf(-0.5f * x * x);
+        du[i] = da[i] * (cdf + x * pdf);
+    }
+}
+
+// dst[map(r)] += src[r] over rows of d floats
+__global__ void rows_add_kernel(float *dst, RowMap map, const float *src, long long rows, int d)
+{
+    const long long n = rows * d;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long r = i / d, k = i % d;
+        dst[rowmap_apply(map, r, 0) * d + k] += src[i];
+    }
+}
+
+// ---------------------------------------------------------------- GEMM
+// 64 x 64 output tile per CTA, 16-deep k steps staged in shared memory,
+// 4 x 4 outputs per thread.
+constexpr int GB_M = 64, GB_N = 64, GB_K = 16, GB_T = 256;
+
+template <int FORM>
+__global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
+{
+    __shared__ __align__(16) float As[GB_K][GB_M + 4];
+    __shared__ __align__(16) float Bs[GB_K][GB_N + 4];
+    const int tid = threadIdx.x, g = blockIdx.z;
+    const int m0 = blockIdx.y * GB_M, n0 = blockIdx.x * GB_N;
+    const int tm = (tid >> 4) * 4, tn = (tid & 15) * 4;
+    // rows of A (NT, NN) and of B (NT) this thread stages: fixed for the kernel
+    const float *arow[4] = {nullptr, nullptr, nullptr, nullptr};
+    const float *brow[4] = {nullptr, nullptr, nullptr, nullptr};
+    if (FORM != BW_TN) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int m = m0 + (tid >> 4) + 16 * j;
+            if (m < p.M) arow[j] = p.A + rowmap_apply(p.a_map, m, g) * p.lda;
+        }
+    }
+    if (FORM == BW_NT) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = n0 + (tid >> 4) + 16 * j;
+            if (n < p.N) brow[j] = p.B + g * p.b_gstride + static_cast<long long>(n) * p.ldb;
+        }
+    }
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+    for (int k0 = 0; k0 < p.K; k0 += GB_K) {
+        if (FORM != BW_TN) {
+            const int kk = tid & 15, k = k0 + kk;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) As[kk][(tid >> 4) + 16 * j] = (arow[j] && k < p.K) ? arow[j][k] : 0.f;
+        } else {
+            const int mm = tid & 63, m = m0 + mm;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int kk = (tid >> 6) + 4 * j, k = k0 + kk;
+                As[kk][mm] = (k < p.K && m < p.M) ? p.A[rowmap_apply(p.a_map, k, g) * p.lda + m] : 0.f;
+            }
+        }
+        if (FORM == BW_NT) {
+            const int kk = tid & 15, k = k0 + kk;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) Bs[kk][(tid >> 4) + 16 * j] = (brow[j] && k < p.K) ? brow[j][k] : 0.f;
+        } else {
+            const int nn = tid & 63, n = n0 + nn;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int kk = (tid >> 6) + 4 * j, k = k0 + kk;
+                float v = 0.f;
+                if (k < p.K && n < p.N) {
+                    const long long row = FORM == BW_NN ? static_cast<long long>(k) : rowmap_apply(p.b_map, k, g);
+                    v = p.B[(FORM == BW_NN ? g * p.b_gstride : 0) + row * p.ldb + n];
+                }
+                Bs[kk][nn] = v;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < GB_K; ++k) {
+            const float4 a = *reinterpret_cast<const float4 *>(&As[k][tm]);
+            const float4 b = *reinterpret_cast<const float4 *>(&Bs[k][tn]);
+            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int m = m0 + tm + i;
+        if (m >= p.M) continue;
+        float *crow = FORM == BW_TN ? p.C + g * p.c_gstride + static_cast<long long>(m) * p.ldc
+                                    : p.C + rowmap_apply(p.c_map, m, g) * p.ldc;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = n0 + tn + j;
+            if (n < p.N) crow[n] = p.accumulate ? crow[n] + acc[i][j] : acc[i][j];
+        }
+    }
+}
+
+// ---------------------------------------------------------------- attention
+// Lane's two dims (lane, lane + 32) of head h of a row; hd <= 64.
+__device__ __forceinline__ float2 bw_ld2(const float *row, int h, int hd, int lane)
+{
+    const float *p = row + h * hd;
+    return make_float2(lane < hd ? p[lane] : 0.f, lane + 32 < hd ? p[lane + 32] : 0.f);
+}
+
+__device__ __forceinline__ void bw_st2(float *row, int h, int hd, int lane, float2 v)
+{
+    float *p = row + h * hd;
+    if (lane < hd) p[lane] = v.x;
+    if (lane + 32 < hd) p[lane + 32] = v.y;
+}
+
+__device__ __forceinline__ float bw_dot(float2 a, float2 b) { return bw_warp_sum(a.x * b.x + a.y * b.y); }
+
+// The keys of query i of user u, in order: S keys 0 .. s_end - 1 (rows
+// u * L + j of skv), then n_cnt NS keys (rows n_row0 + m of qkv).
+struct BwKeys {
+    int s_end, n_cnt;
+    long long n_row0;
+};
+
+__device__ __forceinline__ BwKeys bw_keys(const BwAttn &a, int u, int i)
+{
+    BwKeys k;
+    if (a.mode == 0) {
+        k.s_end = a.L - a.nq + i + 1;
+        k.n_cnt = 0;
+        k.n_row0 = 0;
+    } else {
+        k.s_end = a.L;
+        k.n_cnt = i % a.N + 1;
+        k.n_row0 = static_cast<long long>(u) * a.q_ustride + (i / a.N) * a.N;
+    }
+    return k;
+}
+
+__device__ __forceinline__ const float *bw_key_row(const BwAttn &a, const BwKeys &ks, int u, int j)
+{
+    return j < ks.s_end ? a.skv + (static_cast<long long>(u) * a.L + j) * a.ld
+                        : a.qkv + (ks.n_row0 + (j - ks.s_end)) * a.ld;
+}
+
+// One warp per (query row, head): online softmax; O and the row's softmax
+// statistics (running max m, sum l, base e).
+__global__ void attn_fwd_kernel(BwAttn a)
+{
+    const int lane = threadIdx.x & 31;
+    const long long total = static_cast<long long>(a.U) * a.nq * a.H;
+    for (long long w = bw_warp_id(); w < total; w += bw_warp_count()) {
+        const int h = static_cast<int>(w % a.H);
+        const long long orow = w / a.H;
+        const int u = static_cast<int>(orow / a.nq), i = static_cast<int>(orow % a.nq);
+        const float2 q = bw_ld2(a.qkv + (static_cast<long long>(u) * a.q_ustride + a.q_off + i) * a.ld, h, a.hd, lane);
+        const BwKeys ks = bw_keys(a, u, i);
+        float m = -INFINITY, l = 0.f;
+        float2 o = make_float2(0.f, 0.f);
+        for (int j = 0; j < ks.s_end + ks.n_cnt; ++j) {
+            const float *kr = bw_key_row(a, ks, u, j);
+            const float s = bw_dot(q, bw_ld2(kr + a.d, h, a.hd, lane)) * a.scale;
+            if (s > m) {
+                const float corr = expf(m - s);
+                l *= corr;
+                o.x *= corr;
+                o.y *= corr;
+                m = s;
+            }
+            const float pj = expf(s - m);
+            const float2 v = bw_ld2(kr + 2 * a.d, h, a.hd, lane);
+            l += pj;
+            o.x = fmaf(pj, v.x, o.x);
+            o.y = fmaf(pj, v.y, o.y);
+        }
+        bw_st2(a.O + orow * a.d, h, a.hd, lane, make_float2(o.x / l, o.y / l));
+        if (lane == 0) {
+            a.stat_m[orow * a.H + h] = m;
+            a.stat_l[orow * a.H + h] = l;
+        }
+    }
+}
+
+// One warp per (query row, head): D = dO . O and
+// dQ = scale sum_j p_j (dO . v_j - D) k_j.
+__global__ void attn_bwd_q_kernel(BwAttn a)
+{
+    const int lane = threadIdx.x & 31;
+    const long long total = static_cast<long long>(a.U) * a.nq * a.H;
+    for (long long w = bw_warp_id(); w < total; w += bw_warp_count()) {
+        const int h = static_cast<int>(w % a.H);
+        const long long orow = w / a.H;
+        const int u = static_cast<int>(orow / a.nq), i = static_cast<int>(orow % a.nq);
+        const long long qrow = static_cast<long long>(u) * a.q_ustride + a.q_off + i;
+        const float2 q = bw_ld2(a.qkv + qrow * a.ld, h, a.hd, lane);
+        const float2 dO = bw_ld2(a.dO + orow * a.d, h, a.hd, lane);
+        const float D = bw_dot(dO, bw_ld2(a.O + orow * a.d, h, a.hd, lane));
+        const float m = a.stat_m[orow * a.H + h], inv_l = 1.0f / a.stat_l[orow * a.H + h];
+        const BwKeys ks = bw_keys(a, u, i);
+        float2 dq = make_float2(0.f, 0.f);
+        for (int j = 0; j < ks.s_end + ks.n_cnt; ++j) {
+            const float *kr = bw_key_row(a, ks, u, j);
+            const float2 k = bw_ld2(kr + a.d, h, a.hd, lane);
+            const float p = expf(bw_dot(q, k) * a.scale - m) * inv_l;
+            const float ds = p * (bw_dot(dO, bw_ld2(kr + 2 * a.d, h, a.hd, lane)) - D) * a.scale;
+            dq.x = fmaf(ds, k.x, dq.x);
+            dq.y = fmaf(ds, k.y, dq.y);
+        }
+        bw_st2(a.dqkv + qrow * a.ld, h, a.hd, lane, dq);
+        if (lane == 0) a.stat_D[orow * a.H + h] = D;
+    }
+}
+
+// Contribution of query (qrow, orow) of problem a to the key (k, v):
+// dK += ds q, dV += p dO.
+__device__ __forceinline__ void bw_kv_add(const BwAttn &a, long long qrow, long long orow, int h, int lane, float2 k,
+                                          float2 v, float2 &dk, float2 &dv)
+{
+    const float2 q = bw_ld2(a.qkv + qrow * a.ld, h, a.hd, lane);
+    const float2 dO = bw_ld2(a.dO + orow * a.d, h, a.hd, lane);
+    const long long st = orow * a.H + h;
+    const float p = expf(bw_dot(q, k) * a.scale - a.stat_m[st]) / a.stat_l[st];
+    const float ds = p * (bw_dot(dO, v) - a.stat_D[st]) * a.scale;
+    dk.x = fmaf(ds, q.x, dk.x);
+    dk.y = fmaf(ds, q.y, dk.y);
+    dv.x = fmaf(p, dO.x, dv.x);
+    dv.y = fmaf(p, dO.y, dv.y);
+}
+
+// S keys of the layer: the S tail queries (problem sq) at or after the key
+// and, if has_ns, every NS query of the user (problem nsq).
+__global__ void attn_bwd_kv_s_kernel(BwAttn sq, BwAttn nsq, int has_ns)
+{
+    const int lane = threadIdx.x & 31;
+    const long long total = static_cast<long long>(sq.U) * sq.L * sq.H;
+    for (long long w = bw_warp_id(); w < total; w += bw_warp_count()) {
+        const int h = static_cast<int>(w % sq.H);
+        const long long krow = w / sq.H; // = u * L + j
+        const int u = static_cast<int>(krow / sq.L), j = static_cast<int>(krow % sq.L);
+        const float *kr = sq.skv + krow * sq.ld;
+        const float2 k = bw_ld2(kr + sq.d, h, sq.hd, lane), v = bw_ld2(kr + 2 * sq.d, h, sq.hd, lane);
+        float2 dk = make_float2(0.f, 0.f), dv = make_float2(0.f, 0.f);
+        // tail query i is S row L - nq + i; it sees key j when that row is >= j
+        for (int i = max(0, j - (sq.L - sq.nq)); i < sq.nq; ++i)
+            bw_kv_add(sq, static_cast<long long>(u) * sq.q_ustride + sq.q_off + i,
+                      static_cast<long long>(u) * sq.nq + i, h, lane, k, v, dk, dv);
+        if (has_ns)
+            for (int i = 0; i < nsq.nq; ++i)
+                bw_kv_add(nsq, static_cast<long long>(u) * nsq.q_ustride + i, static_cast<long long>(u) * nsq.nq + i,
+                          h, lane, k, v, dk, dv);
+        float *dr = sq.dskv + krow * sq.ld;
+        bw_st2(dr + sq.d, h, sq.hd, lane, dk);
+        bw_st2(dr + 2 * sq.d, h, sq.hd, lane, dv);
+    }
+}
+
+// NS keys: key m of candidate c is seen by the candidate's NS rows n >= m.
+__global__ void attn_bwd_kv_ns_kernel(BwAttn a)
+{
+    const int lane = threadIdx.x & 31;
+    const long long total = static_cast<long long>(a.U) * a.nq * a.H;
+    for (long long w = bw_warp_id(); w < total; w += bw_warp_count()) {
+        const int h = static_cast<int>(w % a.H);
+        const long long orow = w / a.H;
+        const int u = static_cast<int>(orow / a.nq), j = static_cast<int>(orow % a.nq);
+        const long long ubase = static_cast<long long>(u) * a.q_ustride;
+        const float *kr = a.qkv + (ubase + j) * a.ld;
+        const float2 k = bw_ld2(kr + a.d, h, a.hd, lane), v = bw_ld2(kr + 2 * a.d, h, a.hd, lane);
+        float2 dk = make_float2(0.f, 0.f), dv = make_float2(0.f, 0.f);
+        const int c_end = (j / a.N + 1) * a.N;
+        for (int i = j; i < c_end; ++i)
+            bw_kv_add(a, ubase + i, static_cast<long long>(u) * a.nq + i, h, lane, k, v, dk, dv);
+        float *dr = a.dqkv + (ubase + j) * a.ld;
+        bw_st2(dr + a.d, h, a.hd, lane, dk);
+        bw_st2(dr + 2 * a.d, h, a.hd, lane, dv);
+    }
+}
+
+// ---------------------------------------------------------------- launchers
+static int bw_blocks(long long threads)
+{
+    long long b = (threads + 255) / 256;
+    if (b > 148 * 16) b = 148 * 16;
+    return b < 1 ? 1 : static_cast<int>(b);
+}
+
+cudaError_t bw_rms_fwd(const BwRows &a, const float *g, long long g_gstride, float eps, float *z, float *r,
+                       cudaStream_t s)
+{
+    rms_fwd_kernel<<<bw_blocks(a.rows * a.G * 32), 256, 0, s>>>(a, g, g_gstride, eps, z, r);
+    return cudaGetLastError();
+}
+
+cudaError_t bw_rms_bwd(const BwRows &a, const float *g, long long g_gstride, const float *r, const float *dz,
+                       float *dx, int accumulate, cudaStream_t s)
+{
+    rms_bwd_kernel<<<bw_blocks(a.rows * a.G * 32), 256, 0, s>>>(a, g, g_gstride, r, dz, dx, accumulate);
+    return cudaGetLastError();
+}
+
+int bw_gain_splits(const BwRows &a)
+{
+    const long long col_blocks = static_cast<long long>((a.d + 31) / 32) * a.G;
+    long long sp = (2 * 148 + col_blocks - 1) / col_blocks;
+    const long long by_rows = (a.rows + 63) / 64;
+    if (sp > by_rows) sp = by_rows;
+    if (sp > 64) sp = 64;
+    return sp < 1 ? 1 : static_cast<int>(sp);
+}
+
+cudaError_t bw_gain_grad(const BwRows &a, const float *r, const float *dz, float *partial, int splits, float *dg,
+                         long long g_gstride, cudaStream_t s)
+{
+    if (a.G > 65535 || splits > 64) return cudaErrorInvalidValue;
+    gain_partial_kernel<<<dim3((a.d + 31) / 32, a.G, splits), dim3(32, 8), 0, s>>>(a, r, dz, partial, splits);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    gain_reduce_kernel<<<bw_blocks(static_cast<long long>(a.G) * a.d), 256, 0, s>>>(partial, splits, a.G, a.d, dg,
+                                                                                    g_gstride);
+    return cudaGetLastError();
+}
+
+cudaError_t bw_gelu_fwd(const float *u, float *a, long long n, cudaStream_t s)
+{
+    gelu_fwd_kernel<<<bw_blocks(n), 256, 0, s>>>(u, a, n);
+    return cudaGetLastError();
+}
+
+cudaError_t bw_gelu_bwd(const float *u, const float *da, float *du, long long n, cudaStream_t s)
+{
+    gelu_bwd_kernel<<<bw_blocks(n), 256, 0, s>>>(u, da, du, n);
+    return cudaGetLastError();
+}
+
+cudaError_t bw_rows_add(float *dst, RowMap dst_map, const float *src, long long rows, int d, cudaStream_t s)
+{
+    rows_add_kernel<<<bw_blocks(rows * d), 256, 0, s>>>(dst, dst_map, src, rows, d);
+    return cudaGetLastError();
+}
+
+cudaError_t bw_gemm(const BwGemm &p, cudaStream_t s)
+{
+    const dim3 grid((p.N + GB_N - 1) / GB_N, (p.M + GB_M - 1) / GB_M, p.G);
+    if (p.M < 1 || p.N < 1 || p.K < 1 || p.G < 1 || grid.y > 65535 || grid.z > 65535) return cudaErrorInvalidValue;
+    switch (p.form) {
+    case BW_NT: bw_gemm_kernel<BW_NT><<<grid, GB_T, 0, s>>>(p); break;
+    case BW_NN: bw_gemm_kernel<BW_NN><<<grid, GB_T, 0, s>>>(p); break;
+    case BW_TN: bw_gemm_kernel<BW_TN><<<grid, GB_T, 0, s>>>(p); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+static long long attn_threads(const BwAttn &a) { return static_cast<long long>(a.U) * a.nq * a.H * 32; }
+
+cudaError_t bw_attn_fwd(const BwAttn &a, cudaStream_t s)
+{
+    if (a.hd > 64) return cudaErrorInvalidValue;
+    attn_fwd_kernel<<<bw_blocks(attn_threads(a)), 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t bw_attn_bwd_q(const BwAttn &a, cudaStream_t s)
+{
+    if (a.hd > 64) return cudaErrorInvalidValue;
+    attn_bwd_q_kernel<<<bw_blocks(attn_threads(a)), 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t bw_attn_bwd_kv_s(const BwAttn &sq, const BwAttn *nsq, cudaStream_t s)
+{
+    if (sq.hd > 64) return cudaErrorInvalidValue;
+    attn_bwd_kv_s_kernel<<<bw_blocks(static_cast<long long>(sq.U) * sq.L * sq.H * 32), 256, 0, s>>>(
+        sq, nsq ? *nsq : sq, nsq ? 1 : 0);
+    return cudaGetLastError();
+}
+
+cudaError_t bw_attn_bwd_kv_ns(const BwAttn &a, cudaStream_t s)
+{
+    if (a.hd > 64) return cudaErrorInvalidValue;
+    attn_bwd_kv_ns_kernel<<<bw_blocks(attn_threads(a)), 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+} // namespace ot
+
+// ==================================================================== host
+namespace {
+
+using namespace ot;
+
+constexpr RowMap kIdentity{1, 1, 0, 0, 0};
+
+// Workspace carving.  With a null base it only sums the sizes and hands out
+// non-null placeholder addresses (a dry run never dereferences them, but
+// takes the same branches as a real one).
+struct Carve {
+    char *base;
+    size_t off;
+    float *take(long long n)
+    {
+        float *p = base ? reinterpret_cast<float *>(base + off)
+                        : reinterpret_cast<float *>(static_cast<uintptr_t>(off) + 256);
+        off += (static_cast<size_t>(n) * sizeof(float) + 255) & ~static_cast<size_t>(255);
+        return p;
+    }
+};
+
+// Intermediates of one side (S or NS) of one layer.
+struct Side {
+    float *r1, *Z1, *QKV, *A, *H, *r2, *Z2, *U1, *Act; // recomputed forward
+    float *dH, *dAct, *dZ2, *dA, *dQKV, *dZ1;           // gradients
+    float *sm, *sl, *sD;                                // softmax statistics
+};
+
+struct Backward {
+    ot_config c;
+    int U, C, N, d, f, H, hd, Lyr;
+    int Ls[OT_MAX_LAYERS + 1]; // S rows per user entering layer l
+    bool dry;
+    cudaStream_t st;
+    long long launches;
+    cudaError_t err;
+    const ot_weights *w;
+    const ot_grads *g;
+    const float *X[OT_MAX_LAYERS + 1], *Y[OT_MAX_LAYERS + 1];
+    float *Xout_last, *Yout_last;
+    Side s, n;
+    float *partial;
+    float *dXbuf[2], *dYbuf[2];
+    const float *G_s, *G_ns;
+    float *dS, *dns;
+    size_t bytes;
+
+    const float *wt(const void *p, long long off) const { return static_cast<const float *>(p) + off; }
+    long long T(int l) const { return static_cast<long long>(U) * c.q[l]; }
+    long long RS(int l) const { return static_cast<long long>(U) * Ls[l]; }
+    long long RN() const { return static_cast<long long>(U) * C * N; }
+    RowMap nmap() const { return RowMap{1, N, 0, 1, 0}; }
+
+    // a kernel launch (counted; skipped in a dry run or after an error)
+    template <typename F> void k(F &&fn)
+    {
+        ++launches;
+        if (!dry && err == cudaSuccess) err = fn();
+    }
+    void copy(void *dst, const void *src, size_t nbytes)
+    {
+        if (!dry && err == cudaSuccess) err = cudaMemcpyAsync(dst, src, nbytes, cudaMemcpyDeviceToDevice, st);
+    }
+    void zero(void *dst, size_t nbytes)
+    {
+        if (!dry && err == cudaSuccess) err = cudaMemsetAsync(dst, 0, nbytes, st);
+    }
+
+    void plan(char *base, const float *S, const float *ns, float *out_s, float *out_ns)
+    {
+        Carve cv{base, 0};
+        X[0] = S;
+        Y[0] = ns;
+        for (int l = 1; l < Lyr; ++l) {
+            X[l] = cv.take(RS(l) * d);
+            Y[l] = C ? cv.take(RN() * d) : nullptr;
+        }
+        Xout_last = out_s;
+        Yout_last = out_ns;
+        const long long R = RS(0), Tq = T(0), RN_ = RN();
+        auto side = [&](Side &x, long long rows, long long tail) {
+            x.r1 = cv.take(rows);
+            x.Z1 = cv.take(rows * d);
+            x.QKV = cv.take(rows * 3 * d);
+            x.A = cv.take(tail * d);
+            x.H = cv.take(tail * d);
+            x.r2 = cv.take(tail);
+            x.Z2 = cv.take(tail * d);
+            x.U1 = cv.take(tail * f);
+            x.Act = cv.take(tail * f);
+            x.dH = cv.take(tail * d);
+            x.dAct = cv.take(tail * f);
+            x.dZ2 = cv.take(tail * d);
+            x.dA = cv.take(tail * d);
+            x.dQKV = cv.take(rows * 3 * d);
+            x.dZ1 = cv.take(rows * d);
+            x.sm = cv.take(tail * H);
+            x.sl = cv.take(tail * H);
+            x.sD = cv.take(tail * H);
+        };
+        side(s, R, Tq);
+        if (C) side(n, RN_, RN_);
+        partial = cv.take(64LL * d * (C ? N : 1)); // gain partials: <= 64 chunks, 1 or N groups
+        dXbuf[0] = cv.take(R * d);
+        dXbuf[1] = cv.take(R * d);
+        if (C) {
+            dYbuf[0] = cv.take(RN_ * d);
+            dYbuf[1] = cv.take(RN_ * d);
+        }
+        bytes = cv.off;
+    }
+
+    BwAttn attn_s(int l) const
+    {
+        BwAttn a{};
+        a.mode = 0;
+        a.U = U, a.H = H, a.hd = hd, a.d = d, a.L = Ls[l], a.nq = c.q[l], a.N = N;
+        a.ld = 3LL * d, a.q_ustride = Ls[l], a.q_off = Ls[l] - c.q[l];
+        a.qkv = a.skv = s.QKV;
+        a.dqkv = a.dskv = s.dQKV;
+        a.O = s.A, a.dO = s.dA;
+        a.stat_m = s.sm, a.stat_l = s.sl, a.stat_D = s.sD;
+        a.scale = 1.0f / sqrtf(static_cast<float>(hd));
+        return a;
+    }
+    BwAttn attn_ns(int l) const
+    {
+        BwAttn a{};
+        a.mode = 1;
+        a.U = U, a.H = H, a.hd = hd, a.d = d, a.L = Ls[l], a.nq = C * N, a.N = N;
+        a.ld = 3LL * d, a.q_ustride = static_cast<long long>(C) * N, a.q_off = 0;
+        a.qkv = n.QKV, a.skv = s.QKV;
+        a.dqkv = n.dQKV, a.dskv = s.dQKV;
+        a.O = n.A, a.dO = n.dA;
+        a.stat_m = n.sm, a.stat_l = n.sl, a.stat_D = n.sD;
+        a.scale = 1.0f / sqrtf(static_cast<float>(hd));
+        return a;
+    }
+
+    // C = A B^T with B a weight [G][Nn][K]
+    void nt(const float *A, long long lda, RowMap am, const float *B, long long bgs, float *Cp, long long ldc,
+            RowMap cm, int M, int Nn, int K, int G, int acc)
+    {
+        BwGemm p{};
+        p.form = BW_NT, p.M = M, p.N = Nn, p.K = K, p.G = G;
+        p.A = A, p.lda = lda, p.a_map = am;
+        p.B = B, p.ldb = K, p.b_gstride = bgs;
+        p.C = Cp, p.ldc = ldc, p.c_map = cm, p.accumulate = acc;
+        k([&] { return bw_gemm(p, st); });
+    }
+    // C = A B with B a weight [G][K][Nn]
+    void nn(const float *A, long long lda, RowMap am, const float *B, long long bgs, float *Cp, long long ldc,
+            RowMap cm, int M, int Nn, int K, int G)
+    {
+        BwGemm p{};
+        p.form = BW_NN, p.M = M, p.N = Nn, p.K = K, p.G = G;
+        p.A = A, p.lda = lda, p.a_map = am;
+        p.B = B, p.ldb = Nn, p.b_gstride = bgs;
+        p.C = Cp, p.ldc = ldc, p.c_map = cm;
+        k([&] { return bw_gemm(p, st); });
+    }
+    // weight gradient: C[g] [M][Nn] = sum over the group's K rows of A[row][m] B[row][n]
+    void tn(const float *A, long long lda, RowMap am, const float *B, long long ldb, RowMap bm, float *Cp,
+            long long cgs, int M, int Nn, int K, int G)
+    {
+        BwGemm p{};
+        p.form = BW_TN, p.M = M, p.N = Nn, p.K = K, p.G = G;
+        p.A = A, p.lda = lda, p.a_map = am;
+        p.B = B, p.ldb = ldb, p.b_map = bm;
+        p.C = Cp, p.ldc = Nn, p.c_gstride = cgs;
+        k([&] { return bw_gemm(p, st); });
+    }
+
+    // Recompute layer l (both sides); with s_out / n_out also its output rows.
+    void forward(int l, float *s_out, float *n_out)
+    {
+        const int L = Ls[l], q = c.q[l];
+        const long long R = RS(l), Tq = T(l);
+        const long long d3 = 3LL * d, fd = static_cast<long long>(f) * d, dd = static_cast<long long>(d) * d;
+        // ---- S side
+        const BwRows x1{X[l], kIdentity, R, 1, d};
+        k([&] { return bw_rms_fwd(x1, wt(w->g1_s, static_cast<long long>(l) * d), 0, c.eps, s.Z1, s.r1, st); });
+        nt(s.Z1, d, kIdentity, wt(w->Wqkv_s, l * d3 * d), 0, s.QKV, d3, kIdentity, static_cast<int>(R), 3 * d, d, 1, 0);
+        const BwAttn sa = attn_s(l);
+        k([&] { return bw_attn_fwd(sa, st); });
+        if (!dry && err == cudaSuccess)
+            err = cudaMemcpy2DAsync(s.H, static_cast<size_t>(q) * d * 4, X[l] + static_cast<long long>(L - q) * d,
+                                    static_cast<size_t>(L) * d * 4, static_cast<size_t>(q) * d * 4, U,
+                                    cudaMemcpyDeviceToDevice, st);
+        nt(s.A, d, kIdentity, wt(w->Wo_s, l * dd), 0, s.H, d, kIdentity, static_cast<int>(Tq), d, d, 1, 1);
+        const BwRows h2{s.H, kIdentity, Tq, 1, d};
+        k([&] { return bw_rms_fwd(h2, wt(w->g2_s, static_cast<long long>(l) * d), 0, c.eps, s.Z2, s.r2, st); });
+        nt(s.Z2, d, kIdentity, wt(w->W1_s, l * fd), 0, s.U1, f, kIdentity, static_cast<int>(Tq), f, d, 1, 0);
+        k([&] { return bw_gelu_fwd(s.U1, s.Act, Tq * f, st); });
+        if (s_out) {
+            copy(s_out, s.H, static_cast<size_t>(Tq) * d * 4);
+            nt(s.Act, f, kIdentity, wt(w->W2_s, l * fd), 0, s_out, d, kIdentity, static_cast<int>(Tq), d, f, 1, 1);
+        }
+        if (!C) return;
+        // ---- NS side: group = NS position, rows of a group = the U * C candidates
+        const RowMap nm = nmap();
+        const long long RN_ = RN();
+        const int M = U * C;
+        const long long ln = static_cast<long long>(l) * N;
+        const BwRows y1{Y[l], nm, M, N, d};
+        k([&] { return bw_rms_fwd(y1, wt(w->g1_ns, ln * d), d, c.eps, n.Z1, n.r1, st); });
+        nt(n.Z1, d, nm, wt(w->Wqkv_ns, ln * d3 * d), d3 * d, n.QKV, d3, nm, M, 3 * d, d, N, 0);
+        const BwAttn na = attn_ns(l);
+        k([&] { return bw_attn_fwd(na, st); });
+        copy(n.H, Y[l], static_cast<size_t>(RN_) * d * 4);
+        nt(n.A, d, nm, wt(w->Wo_ns, ln * dd), dd, n.H, d, nm, M, d, d, N, 1);
+        const BwRows h2n{n.H, nm, M, N, d};
+        k([&] { return bw_rms_fwd(h2n, wt(w->g2_ns, ln * d), d, c.eps, n.Z2, n.r2, st); });
+        nt(n.Z2, d, nm, wt(w->W1_ns, ln * fd), fd, n.U1, f, nm, M, f, d, N, 0);
+        k([&] { return bw_gelu_fwd(n.U1, n.Act, RN_ * f, st); });
+        if (n_out) {
+            copy(n_out, n.H, static_cast<size_t>(RN_) * d * 4);
+            nt(n.Act, f, nm, wt(w->W2_ns, ln * fd), fd, n_out, d, nm, M, d, f, N, 1);
+        }
+    }
+
+    // FFN and output-projection backward of one side: dOut -> x.dH, x.dA and
+    // the gradients of W1, W2, Wo and g2.  M rows in each of G groups under map.
+    void ffn_back(Side &x, const float *dOut, RowMap map, int M, int G, const float *W1, const float *W2,
+                  const float *Wo, const float *g2, long long ggs, float *dW1, float *dW2, float *dWo, float *dg2)
+    {
+        const long long rows = static_cast<long long>(M) * G;
+        const long long fd = static_cast<long long>(f) * d, dd = static_cast<long long>(d) * d;
+        copy(x.dH, dOut, static_cast<size_t>(rows) * d * 4);
+        nn(dOut, d, map, W2, fd, x.dAct, f, map, M, f, d, G); // dAct = dOut W2
+        tn(dOut, d, map, x.Act, f, map, dW2, fd, d, f, M, G);  // dW2 = dOut^T Act
+        k([&] { return bw_gelu_bwd(x.U1, x.dAct, x.dAct, rows * f, st); });
+        tn(x.dAct, f, map, x.Z2, d, map, dW1, fd, f, d, M, G); // dW1 = dU1^T Z2
+        nn(x.dAct, f, map, W1, fd, x.dZ2, d, map, M, d, f, G); // dZ2 = dU1 W1
+        const BwRows hr{x.H, map, M, G, d};
+        k([&] { return bw_rms_bwd(hr, g2, ggs, x.r2, x.dZ2, x.dH, 1, st); });
+        const int sp = bw_gain_splits(hr);
+        k([&] { return bw_gain_grad(hr, x.r2, x.dZ2, partial, sp, dg2, ggs, st); });
+        ++launches; // bw_gain_grad issues two kernels
+        nn(x.dH, d, map, Wo, dd, x.dA, d, map, M, d, d, G); // dA = dH Wo
+        tn(x.dH, d, map, x.A, d, map, dWo, dd, d, d, M, G);  // dWo = dH^T A
+    }
+
+    // QKV projection and first-norm backward of one side: x.dQKV -> dX
+    // (written, or added when accumulate), gradients of Wqkv and g1.
+    void qkv_back(Side &x, const float *Xin, RowMap map, int M, int G, const float *Wqkv, const float *g1,
+                  long long ggs, float *dWqkv, float *dg1, float *dX, int accumulate)
+    {
+        const long long d3 = 3LL * d;
+        tn(x.dQKV, d3, map, x.Z1, d, map, dWqkv, d3 * d, 3 * d, d, M, G); // dWqkv = dQKV^T Z1
+        nn(x.dQKV, d3, map, Wqkv, d3 * d, x.dZ1, d, map, M, d, 3 * d, G); // dZ1 = dQKV Wqkv
+        const BwRows xr{Xin, map, M, G, d};
+        k([&] { return bw_rms_bwd(xr, g1, ggs, x.r1, x.dZ1, dX, accumulate, st); });
+        const int sp = bw_gain_splits(xr);
+        k([&] { return bw_gain_grad(xr, x.r1, x.dZ1, partial, sp, dg1, ggs, st); });
+        ++launches;
+    }
+
+    void backward(int l, const float *dXin, float *dXout, const float *dYin, float *dYout)
+    {
+        const int L = Ls[l], q = c.q[l];
+        const long long R = RS(l), Tq = T(l);
+        const long long d3 = 3LL * d, fd = static_cast<long long>(f) * d, dd = static_cast<long long>(d) * d;
+        const long long ln = static_cast<long long>(l) * N;
+        const RowMap nm = nmap();
+        const int M = U * C;
+        // FFN + output projection, both sides
+        ffn_back(s, dXin, kIdentity, static_cast<int>(Tq), 1, wt(w->W1_s, l * fd), wt(w->W2_s, l * fd),
+                 wt(w->Wo_s, l * dd), wt(w->g2_s, static_cast<long long>(l) * d), 0, g->W1_s + l * fd,
+                 g->W2_s + l * fd, g->Wo_s + l * dd, g->g2_s + static_cast<long long>(l) * d);
+        if (C)
+            ffn_back(n, dYin, nm, M, N, wt(w->W1_ns, ln * fd), wt(w->W2_ns, ln * fd), wt(w->Wo_ns, ln * dd),
+                     wt(w->g2_ns, ln * d), d, g->W1_ns + ln * fd, g->W2_ns + ln * fd, g->Wo_ns + ln * dd,
+                     g->g2_ns + ln * d);
+        // attention
+        zero(s.dQKV, static_cast<size_t>(R) * d3 * 4); // Q columns of the rows above the tail stay 0
+        const BwAttn sa = attn_s(l);
+        k([&] { return bw_attn_bwd_q(sa, st); });
+        BwAttn na{};
+        if (C) {
+            na = attn_ns(l);
+            k([&] { return bw_attn_bwd_q(na, st); });
+        }
+        k([&] { return bw_attn_bwd_kv_s(sa, C ? &na : nullptr, st); });
+        if (C) k([&] { return bw_attn_bwd_kv_ns(na, st); });
+        // QKV + first norm; the residual adds dH to the tail rows
+        qkv_back(s, X[l], kIdentity, static_cast<int>(R), 1, wt(w->Wqkv_s, l * d3 * d),
+                 wt(w->g1_s, static_cast<long long>(l) * d), 0, g->Wqkv_s + l * d3 * d,
+                 g->g1_s + static_cast<long long>(l) * d, dXout, 0);
+        const RowMap tail{q, L, L - q, 0, 0};
+        k([&] { return bw_rows_add(dXout, tail, s.dH, Tq, d, st); });
+        if (C) {
+            copy(dYout, n.dH, static_cast<size_t>(RN()) * d * 4);
+            qkv_back(n, Y[l], nm, M, N, wt(w->Wqkv_ns, ln * d3 * d), wt(w->g1_ns, ln * d), d,
+                     g->Wqkv_ns + ln * d3 * d, g->g1_ns + ln * d, dYout, 1);
+        }
+    }
+
+    void run()
+    {
+        if (!C) {
+            const long long fd = static_cast<long long>(f) * d, dd = static_cast<long long>(d) * d;
+            const long long LN = static_cast<long long>(Lyr) * N;
+            zero(g->Wqkv_ns, LN * 3 * dd * 4);
+            zero(g->Wo_ns, LN * dd * 4);
+            zero(g->W1_ns, LN * fd * 4);
+            zero(g->W2_ns, LN * fd * 4);
+            zero(g->g1_ns, LN * d * 4);
+            zero(g->g2_ns, LN * d * 4);
+        }
+        // checkpointing forward: keep every layer's input rows
+        for (int l = 0; l < Lyr; ++l) {
+            const bool last = l == Lyr - 1;
+            forward(l, last ? Xout_last : const_cast<float *>(X[l + 1]),
+                    last ? Yout_last : const_cast<float *>(Y[l + 1]));
+        }
+        // backward, top layer first (its intermediates are still in place)
+        for (int l = Lyr - 1; l >= 0; --l) {
+            if (l != Lyr - 1) forward(l, nullptr, nullptr);
+            const float *dXin = l == Lyr - 1 ? G_s : dXbuf[(l + 1) & 1];
+            float *dXout = (l == 0 && dS) ? dS : dXbuf[l & 1];
+            const float *dYin = !C ? nullptr : (l == Lyr - 1 ? G_ns : dYbuf[(l + 1) & 1]);
+            float *dYout = !C ? nullptr : ((l == 0 && dns) ? dns : dYbuf[l & 1]);
+            backward(l, dXin, dXout, dYin, dYout);
+        }
+    }
+};
+
+ot_status bw_validate(const ot_config *cfg, int U, int C)
+{
+    if (!cfg || U < 1 || C < 0) return OT_ERR_ARG;
+    if (cfg->dtype != OT_DTYPE_F32) return OT_ERR_DTYPE;
+    if (cfg->full_attn || cfg->moe_experts) return OT_ERR_UNSUPPORTED;
+    const ot_status r = internal_check_config(*cfg);
+    if (r != OT_OK) return r;
+    if (cfg->d / cfg->heads > 64) return OT_ERR_SHAPE;
+    // GEMM rows stay below 2^31 / 64 (the grid's 65535 row tiles) and U * C fits an int
+    const long long rs = static_cast<long long>(U) * cfg->L0, rn = static_cast<long long>(U) * C;
+    if (rs > 65535LL * 64 || rn > 65535LL * 64) return OT_ERR_SHAPE;
+    return OT_OK;
+}
+
+void bw_init(Backward &b, const ot_config *cfg, int U, int C)
+{
+    b.c = *cfg;
+    b.U = U, b.C = C, b.N = cfg->n_ns, b.d = cfg->d, b.f = cfg->ffn, b.H = cfg->heads;
+    b.hd = cfg->d / cfg->heads, b.Lyr = cfg->layers;
+    b.Ls[0] = cfg->L0;
+    for (int l = 0; l < cfg->layers; ++l) b.Ls[l + 1] = cfg->q[l];
+    b.launches = 0;
+    b.err = cudaSuccess;
+    b.bytes = 0;
+}
+
+} // namespace
+
+extern "C" {
+
+size_t ot_backward_workspace_bytes(const ot_config *cfg, int U, int C)
+{
+    if (bw_validate(cfg, U, C) != OT_OK) return 0;
+    Backward b{};
+    bw_init(b, cfg, U, C);
+    b.dry = true;
+    b.plan(nullptr, nullptr, nullptr, nullptr, nullptr);
+    return b.bytes;
+}
+
+long long ot_backward_launches(const ot_config *cfg, int U, int C)
+{
+    if (bw_validate(cfg, U, C) != OT_OK) return 0;
+    Backward b{};
+    bw_init(b, cfg, U, C);
+    b.dry = true;
+    // the output pointers only decide whether the last layer's output GEMMs run
+    static float dummy;
+    b.plan(nullptr, nullptr, nullptr, &dummy, C ? &dummy : nullptr);
+    const ot_weights w0{};
+    const ot_grads g0{};
+    b.w = &w0;
+    b.g = &g0;
+    b.run();
+    return b.launches;
+}
+
+ot_status ot_full_backward(const ot_config *cfg, const ot_weights *w, const float *S, const float *ns, int U, int C,
+                           const float *G_s, const float *G_ns, float *out_s_tail, float *out_ns, const ot_grads *g,
+                           float *dS, float *dns, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!cfg || !w || !g || !S || !G_s || !ws || U < 1 || C < 0) return OT_ERR_ARG;
+    if (C && (!ns || !G_ns)) return OT_ERR_ARG;
+    const void *wp[] = {w->Wqkv_s,  w->Wo_s,  w->W1_s,  w->W2_s,  w->g1_s,  w->g2_s,
+                        w->Wqkv_ns, w->Wo_ns, w->W1_ns, w->W2_ns, w->g1_ns, w->g2_ns};
+    const void *gp[] = {g->Wqkv_s,  g->Wo_s,  g->W1_s,  g->W2_s,  g->g1_s,  g->g2_s,
+                        g->Wqkv_ns, g->Wo_ns, g->W1_ns, g->W2_ns, g->g1_ns, g->g2_ns};
+    for (int i = 0; i < 12; ++i)
+        if (!wp[i] || !gp[i]) return OT_ERR_ARG;
+    const ot_status v = bw_validate(cfg, U, C);
+    if (v != OT_OK) return v;
+    auto al = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+    for (int i = 0; i < 12; ++i)
+        if (!al(wp[i]) || !al(gp[i])) return OT_ERR_ALIGN;
+    if (!al(S) || !al(G_s) || !al(ws) || (C && (!al(ns) || !al(G_ns))) || (out_s_tail && !al(out_s_tail)) ||
+        (C && out_ns && !al(out_ns)) || (dS && !al(dS)) || (C && dns && !al(dns)))
+        return OT_ERR_ALIGN;
+    Backward b{};
+    bw_init(b, cfg, U, C);
+    b.dry = false;
+    b.plan(static_cast<char *>(ws), S, C ? ns : nullptr, out_s_tail, C ? out_ns : nullptr);
+    if (b.bytes > ws_bytes) return OT_ERR_WORKSPACE_TOO_SMALL;
+    b.st = static_cast<cudaStream_t>(stream);
+    b.w = w;
+    b.g = g;
+    b.G_s = G_s;
+    b.G_ns = C ? G_ns : nullptr;
+    b.dS = dS;
+    b.dns = C ? dns : nullptr;
+    b.run();
+    return b.err == cudaSuccess ? OT_OK : OT_ERR_CUDA;
+}
+
+} // extern "C"

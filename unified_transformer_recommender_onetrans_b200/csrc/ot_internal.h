@@ -271,6 +271,72 @@ struct MoeCombineArgs {
 cudaError_t launch_moe_route(const MoeRouteArgs &a, cudaStream_t s);
 cudaError_t launch_moe_combine(const MoeCombineArgs &a, cudaStream_t s);
 
+// Backward pass (fp32, CUDA cores).  Row sets of the backward kernels: row
+// r of group g is buffer row map(r, g), rows of d floats.
+struct BwRows {
+    const float *X; // input rows
+    RowMap map;
+    long long rows;
+    int G, d;
+};
+// C = A B^T (NT), A B (NN) or A^T B (TN), C an M x N block, reduction K:
+//   NT: C[cmap(m, g)][n] (+)= sum_k A[amap(m, g)][k] B[g][n][k]
+//   NN: C[cmap(m, g)][n] (+)= sum_k A[amap(m, g)][k] B[g][k][n]
+//   TN: C[g][m][n]       (+)= sum_k A[amap(k, g)][m] B[bmap(k, g)][n]
+// B[g] starts at B + g * b_gstride (NT / NN) with row stride ldb; C[g] of
+// TN at C + g * c_gstride.
+enum { BW_NT = 0, BW_NN = 1, BW_TN = 2 };
+struct BwGemm {
+    int form, M, N, K, G;
+    const float *A;
+    long long lda;
+    RowMap a_map;
+    const float *B;
+    long long ldb, b_gstride;
+    RowMap b_map;
+    float *C;
+    long long ldc, c_gstride;
+    RowMap c_map;
+    int accumulate;
+};
+// One attention problem of a layer over QKV rows [.][3d] (Q | K | V):
+//   mode 0 (S queries): query i of user u is S row t = L - nq + i of the
+//     layer, buffer row u * q_ustride + q_off + i of qkv (= skv); it sees S
+//     keys 0..t.
+//   mode 1 (NS queries): query i = c * N + n of user u is row
+//     u * q_ustride + i of qkv; it sees the user's L S keys (rows u * L + j
+//     of skv) and NS keys c * N + m, m <= n (rows of qkv).
+// O / dO are [U * nq][d]; stat_* [U * nq][H]; dqkv / dskv take dQ and dK, dV
+// in the layout of qkv / skv.
+struct BwAttn {
+    int mode, U, H, hd, d, L, nq, N;
+    long long ld, q_ustride, q_off;
+    const float *qkv, *skv;
+    float *dqkv, *dskv;
+    float *O;
+    const float *dO;
+    float *stat_m, *stat_l, *stat_D;
+    float scale;
+};
+cudaError_t bw_rms_fwd(const BwRows &a, const float *g, long long g_gstride, float eps, float *z, float *r,
+                       cudaStream_t s);
+cudaError_t bw_rms_bwd(const BwRows &a, const float *g, long long g_gstride, const float *r,
+                       const float *dz, float *dx, int accumulate, cudaStream_t s);
+cudaError_t bw_gain_grad(const BwRows &a, const float *r, const float *dz, float *partial, int splits,
+                         float *dg, long long g_gstride, cudaStream_t s);
+int bw_gain_splits(const BwRows &a);
+cudaError_t bw_gelu_fwd(const float *u, float *a, long long n, cudaStream_t s);
+cudaError_t bw_gelu_bwd(const float *u, const float *da, float *du, long long n, cudaStream_t s);
+cudaError_t bw_rows_add(float *dst, RowMap dst_map, const float *src, long long rows, int d, cudaStream_t s);
+cudaError_t bw_gemm(const BwGemm &p, cudaStream_t s);
+cudaError_t bw_attn_fwd(const BwAttn &a, cudaStream_t s);
+cudaError_t bw_attn_bwd_q(const BwAttn &a, cudaStream_t s);
+cudaError_t bw_attn_bwd_kv_s(const BwAttn &sq, const BwAttn *nsq, cudaStream_t s);
+cudaError_t bw_attn_bwd_kv_ns(const BwAttn &a, cudaStream_t s);
+
+// Shape / dtype check of a config (the rules of ot_model_create).
+ot_status internal_check_config(const ot_config &c);
+
 // Read-only model queries for entry points defined outside ot_api.cu.
 int internal_profiling(const ot_model *m);
 int internal_device(const ot_model *m);
