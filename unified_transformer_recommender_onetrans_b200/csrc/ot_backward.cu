@@ -32,6 +32,13 @@ __device__ __forceinline__ float bw_warp_sum(float v)
     return v;
 }
 
+// rowmap_apply with the common P == 1 case (flat and NS-group maps) taken
+// without a division
+__device__ __forceinline__ long long bw_row(const RowMap &m, long long r, long long g)
+{
+    return m.P == 1 ? r * m.A + m.B + g * m.Gs : rowmap_apply(m, r, g);
+}
+
 __device__ __forceinline__ long long bw_warp_id()
 {
     return (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
@@ -50,7 +57,7 @@ __global__ void rms_fwd_kernel(BwRows a, const float *g, long long g_gstride, fl
 {
     const int lane = threadIdx.x & 31;
     for (long long w = bw_warp_id(); w < a.rows * a.G; w += bw_warp_count()) {
-        const long long grp = w / a.rows, R = rowmap_apply(a.map, w % a.rows, grp);
+        const long long grp = w / a.rows, R = bw_row(a.map, w % a.rows, grp);
         const float *x = a.X + R * a.d;
         const float *gg = g + grp * g_gstride;
         float ss = 0.f;
@@ -66,7 +73,7 @@ __global__ void rms_bwd_kernel(BwRows a, const float *g, long long g_gstride, co
 {
     const int lane = threadIdx.x & 31;
     for (long long w = bw_warp_id(); w < a.rows * a.G; w += bw_warp_count()) {
-        const long long grp = w / a.rows, R = rowmap_apply(a.map, w % a.rows, grp);
+        const long long grp = w / a.rows, R = bw_row(a.map, w % a.rows, grp);
         const float *x = a.X + R * a.d;
         const float *dzr = dz + R * a.d;
         const float *gg = g + grp * g_gstride;
@@ -93,7 +100,7 @@ __global__ void gain_partial_kernel(BwRows a, const float *r_in, const float *dz
     float acc = 0.f;
     if (k < a.d)
         for (long long r = r0 + threadIdx.y; r < r1; r += 8) {
-            const long long R = rowmap_apply(a.map, r, grp);
+            const long long R = bw_row(a.map, r, grp);
             acc = fmaf(dz[R * a.d + k] * a.X[R * a.d + k], r_in[R], acc);
         }
     red[threadIdx.y][threadIdx.x] = acc;
@@ -158,8 +165,17 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
 {
     __shared__ __align__(16) float As[GB_K][GB_M + 4];
     __shared__ __align__(16) float Bs[GB_K][GB_N + 4];
-    const int tid = threadIdx.x, g = blockIdx.z;
+    const int tid = threadIdx.x;
+    const int g = FORM == BW_TN ? static_cast<int>(blockIdx.z) / p.splits : static_cast<int>(blockIdx.z);
+    const int split = FORM == BW_TN ? static_cast<int>(blockIdx.z) % p.splits : 0;
     const int m0 = blockIdx.y * GB_M, n0 = blockIdx.x * GB_N;
+    // reduction range of this CTA (TN: one of `splits` chunks, GB_K aligned)
+    int k_lo = 0, k_hi = p.K;
+    if (FORM == BW_TN && p.splits > 1) {
+        const int chunk = ((p.K + p.splits - 1) / p.splits + GB_K - 1) / GB_K * GB_K;
+        k_lo = min(p.K, split * chunk);
+        k_hi = min(p.K, k_lo + chunk);
+    }
     const int tm = (tid >> 4) * 4, tn = (tid & 15) * 4;
     // rows of A (NT, NN) and of B (NT) this thread stages: fixed for the kernel
     const float *arow[4] = {nullptr, nullptr, nullptr, nullptr};
@@ -168,7 +184,7 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int m = m0 + (tid >> 4) + 16 * j;
-            if (m < p.M) arow[j] = p.A + rowmap_apply(p.a_map, m, g) * p.lda;
+            if (m < p.M) arow[j] = p.A + bw_row(p.a_map, m, g) * p.lda;
         }
     }
     if (FORM == BW_NT) {
@@ -184,7 +200,7 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 
-    for (int k0 = 0; k0 < p.K; k0 += GB_K) {
+    for (int k0 = k_lo; k0 < k_hi; k0 += GB_K) {
         if (FORM != BW_TN) {
             const int kk = tid & 15, k = k0 + kk;
 #pragma unroll
@@ -194,7 +210,7 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int kk = (tid >> 6) + 4 * j, k = k0 + kk;
-                As[kk][mm] = (k < p.K && m < p.M) ? p.A[rowmap_apply(p.a_map, k, g) * p.lda + m] : 0.f;
+                As[kk][mm] = (k < k_hi && m < p.M) ? p.A[bw_row(p.a_map, k, g) * p.lda + m] : 0.f;
             }
         }
         if (FORM == BW_NT) {
@@ -207,8 +223,8 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
             for (int j = 0; j < 4; ++j) {
                 const int kk = (tid >> 6) + 4 * j, k = k0 + kk;
                 float v = 0.f;
-                if (k < p.K && n < p.N) {
-                    const long long row = FORM == BW_NN ? static_cast<long long>(k) : rowmap_apply(p.b_map, k, g);
+                if (k < k_hi && n < p.N) {
+                    const long long row = FORM == BW_NN ? static_cast<long long>(k) : bw_row(p.b_map, k, g);
                     v = p.B[(FORM == BW_NN ? g * p.b_gstride : 0) + row * p.ldb + n];
                 }
                 Bs[kk][nn] = v;
@@ -231,13 +247,32 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
     for (int i = 0; i < 4; ++i) {
         const int m = m0 + tm + i;
         if (m >= p.M) continue;
-        float *crow = FORM == BW_TN ? p.C + g * p.c_gstride + static_cast<long long>(m) * p.ldc
-                                    : p.C + rowmap_apply(p.c_map, m, g) * p.ldc;
+        float *crow;
+        if (FORM == BW_TN && p.splits > 1)
+            crow = p.partial + ((static_cast<long long>(split) * p.G + g) * p.M + m) * p.N;
+        else if (FORM == BW_TN)
+            crow = p.C + g * p.c_gstride + static_cast<long long>(m) * p.ldc;
+        else
+            crow = p.C + bw_row(p.c_map, m, g) * p.ldc;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int n = n0 + tn + j;
-            if (n < p.N) crow[n] = p.accumulate ? crow[n] + acc[i][j] : acc[i][j];
+            if (n < p.N) crow[n] = p.accumulate && !(FORM == BW_TN && p.splits > 1) ? crow[n] + acc[i][j] : acc[i][j];
         }
+    }
+}
+
+// C[g][m][n] (+)= sum over splits, in split order, of partial[s][g][m][n]
+__global__ void tn_reduce_kernel(BwGemm p)
+{
+    const long long per = static_cast<long long>(p.M) * p.N, n_all = per * p.G;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n_all;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long g = i / per, mn = i % per, m = mn / p.N, n = mn % p.N;
+        float v = 0.f;
+        for (int sp = 0; sp < p.splits; ++sp) v += p.partial[sp * n_all + i];
+        float *c = p.C + g * p.c_gstride + m * p.ldc + n;
+        *c = p.accumulate ? *c + v : v;
     }
 }
 
@@ -481,16 +516,38 @@ cudaError_t bw_rows_add(float *dst, RowMap dst_map, const float *src, long long 
     return cudaGetLastError();
 }
 
+int bw_tn_splits(int M, int N, int K, int G)
+{
+    const long long tiles = static_cast<long long>((M + GB_M - 1) / GB_M) * ((N + GB_N - 1) / GB_N) * G;
+    long long sp = (2 * 148 + tiles - 1) / tiles;
+    const long long by_k = (K + 255) / 256; // at least 256 reduction rows per split
+    if (sp > by_k) sp = by_k;
+    if (sp > 64) sp = 64;
+    return sp < 1 ? 1 : static_cast<int>(sp);
+}
+
+long long bw_tn_partial_floats(int M, int N, int K, int G)
+{
+    const int sp = bw_tn_splits(M, N, K, G);
+    return sp > 1 ? static_cast<long long>(sp) * G * M * N : 0;
+}
+
 cudaError_t bw_gemm(const BwGemm &p, cudaStream_t s)
 {
-    const dim3 grid((p.N + GB_N - 1) / GB_N, (p.M + GB_M - 1) / GB_M, p.G);
-    if (p.M < 1 || p.N < 1 || p.K < 1 || p.G < 1 || grid.y > 65535 || grid.z > 65535) return cudaErrorInvalidValue;
+    const int splits = p.form == BW_TN ? p.splits : 1;
+    const dim3 grid((p.N + GB_N - 1) / GB_N, (p.M + GB_M - 1) / GB_M, p.G * splits);
+    if (p.M < 1 || p.N < 1 || p.K < 1 || p.G < 1 || splits < 1 || grid.y > 65535 || grid.z > 65535 ||
+        (splits > 1 && !p.partial))
+        return cudaErrorInvalidValue;
     switch (p.form) {
     case BW_NT: bw_gemm_kernel<BW_NT><<<grid, GB_T, 0, s>>>(p); break;
     case BW_NN: bw_gemm_kernel<BW_NN><<<grid, GB_T, 0, s>>>(p); break;
     case BW_TN: bw_gemm_kernel<BW_TN><<<grid, GB_T, 0, s>>>(p); break;
     default: return cudaErrorInvalidValue;
     }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || splits == 1) return e;
+    tn_reduce_kernel<<<bw_blocks(static_cast<long long>(p.M) * p.N * p.G), 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -570,6 +627,8 @@ struct Backward {
     float *Xout_last, *Yout_last;
     Side s, n;
     float *partial;
+    float *tn_partial; // split TN GEMMs: < 2 * 296 tiles of 64 x 64 floats
+    static constexpr long long kTnPartialFloats = 2LL * 296 * 64 * 64;
     float *dXbuf[2], *dYbuf[2];
     const float *G_s, *G_ns;
     float *dS, *dns;
@@ -631,6 +690,7 @@ struct Backward {
         side(s, R, Tq);
         if (C) side(n, RN_, RN_);
         partial = cv.take(64LL * d * (C ? N : 1)); // gain partials: <= 64 chunks, 1 or N groups
+        tn_partial = cv.take(kTnPartialFloats);
         dXbuf[0] = cv.take(R * d);
         dXbuf[1] = cv.take(R * d);
         if (C) {
@@ -698,7 +758,11 @@ struct Backward {
         p.A = A, p.lda = lda, p.a_map = am;
         p.B = B, p.ldb = ldb, p.b_map = bm;
         p.C = Cp, p.ldc = Nn, p.c_gstride = cgs;
+        p.splits = bw_tn_splits(M, Nn, K, G);
+        p.partial = tn_partial;
+        if (bw_tn_partial_floats(M, Nn, K, G) > kTnPartialFloats && err == cudaSuccess) err = cudaErrorInvalidValue;
         k([&] { return bw_gemm(p, st); });
+        if (p.splits > 1) ++launches; // the split-order reduction
     }
 
     // Recompute layer l (both sides); with s_out / n_out also its output rows.

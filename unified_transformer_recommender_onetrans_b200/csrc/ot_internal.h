@@ -298,6 +298,11 @@ struct BwGemm {
     long long ldc, c_gstride;
     RowMap c_map;
     int accumulate;
+    // TN only: the reduction split over `splits` CTAs, each writing its
+    // partial block to partial[split][G][M][N]; a second kernel sums them in
+    // split order into C (splits == 1: straight into C)
+    int splits;
+    float *partial;
 };
 // One attention problem of a layer over QKV rows [.][3d] (Q | K | V):
 //   mode 0 (S queries): query i of user u is S row t = L - nq + i of the
@@ -329,6 +334,10 @@ cudaError_t bw_gelu_fwd(const float *u, float *a, long long n, cudaStream_t s);
 cudaError_t bw_gelu_bwd(const float *u, const float *da, float *du, long long n, cudaStream_t s);
 cudaError_t bw_rows_add(float *dst, RowMap dst_map, const float *src, long long rows, int d, cudaStream_t s);
 cudaError_t bw_gemm(const BwGemm &p, cudaStream_t s);
+// reduction split of a TN GEMM (2 * 148 CTAs as the target) and the partial
+// buffer floats it needs (0 when not split)
+int bw_tn_splits(int M, int N, int K, int G);
+long long bw_tn_partial_floats(int M, int N, int K, int G);
 cudaError_t bw_attn_fwd(const BwAttn &a, cudaStream_t s);
 cudaError_t bw_attn_bwd_q(const BwAttn &a, cudaStream_t s);
 cudaError_t bw_attn_bwd_kv_s(const BwAttn &sq, const BwAttn *nsq, cudaStream_t s);
