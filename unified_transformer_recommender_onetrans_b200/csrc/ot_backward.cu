@@ -12,9 +12,10 @@
 //              (grouped GEMMs, group = n) and attention over the layer's S
 //              keys and the candidate's NS keys m <= n;
 //   gradients  dH = dOut + n'(dOut W2 * GELU'(U1) W1), dW2 = dOut^T Act,
-//              dW1 = dU1^T Z2, dA = dH Wo, dWo = dH^T A; attention: dQ per
-//              query row, dK / dV per key row (S keys collect the S tail
-//              rows at or after them and every NS row of the user);
+//              dW1 = dU1^T Z2, dA = dH Wo, dWo = dH^T A; attention
+//              (ot_backward_attn.cu): dQ per query block, dK / dV per key
+//              block (S keys collect the S tail rows at or after them and
+//              every NS row of the user);
 //              dWqkv = dQKV^T Z1, dX = n'(dQKV Wqkv) + dH on the tail rows.
 // n'(.) is the RMSNorm backward: with r = (mean(x^2) + eps)^(-1/2),
 //   dx = r g dz - x r^3 mean(x g dz),  dg = sum over rows of dz x r.
@@ -276,184 +277,6 @@ __global__ void tn_reduce_kernel(BwGemm p)
     }
 }
 
-// ---------------------------------------------------------------- attention
-// Lane's two dims (lane, lane + 32) of head h of a row; hd <= 64.
-__device__ __forceinline__ float2 bw_ld2(const float *row, int h, int hd, int lane)
-{
-    const float *p = row + h * hd;
-    return make_float2(lane < hd ? p[lane] : 0.f, lane + 32 < hd ? p[lane + 32] : 0.f);
-}
-
-__device__ __forceinline__ void bw_st2(float *row, int h, int hd, int lane, float2 v)
-{
-    float *p = row + h * hd;
-    if (lane < hd) p[lane] = v.x;
-    if (lane + 32 < hd) p[lane + 32] = v.y;
-}
-
-__device__ __forceinline__ float bw_dot(float2 a, float2 b) { return bw_warp_sum(a.x * b.x + a.y * b.y); }
-
-// The keys of query i of user u, in order: S keys 0 .. s_end - 1 (rows
-// u * L + j of skv), then n_cnt NS keys (rows n_row0 + m of qkv).
-struct BwKeys {
-    int s_end, n_cnt;
-    long long n_row0;
-};
-
-__device__ __forceinline__ BwKeys bw_keys(const BwAttn &a, int u, int i)
-{
-    BwKeys k;
-    if (a.mode == 0) {
-        k.s_end = a.L - a.nq + i + 1;
-        k.n_cnt = 0;
-        k.n_row0 = 0;
-    } else {
-        k.s_end = a.L;
-        k.n_cnt = i % a.N + 1;
-        k.n_row0 = static_cast<long long>(u) * a.q_ustride + (i / a.N) * a.N;
-    }
-    return k;
-}
-
-__device__ __forceinline__ const float *bw_key_row(const BwAttn &a, const BwKeys &ks, int u, int j)
-{
-    return j < ks.s_end ? a.skv + (static_cast<long long>(u) * a.L + j) * a.ld
-                        : a.qkv + (ks.n_row0 + (j - ks.s_end)) * a.ld;
-}
-
-// One warp per (query row, head): online softmax; O and the row's softmax
-// statistics (running max m, sum l, base e).
-__global__ void attn_fwd_kernel(BwAttn a)
-{
-    const int lane = threadIdx.x & 31;
-    const long long total = static_cast<long long>(a.U) * a.nq * a.H;
-    for (long long w = bw_warp_id(); w < total; w += bw_warp_count()) {
-        const int h = static_cast<int>(w % a.H);
-        const long long orow = w / a.H;
-        const int u = static_cast<int>(orow / a.nq), i = static_cast<int>(orow % a.nq);
-        const float2 q = bw_ld2(a.qkv + (static_cast<long long>(u) * a.q_ustride + a.q_off + i) * a.ld, h, a.hd, lane);
-        const BwKeys ks = bw_keys(a, u, i);
-        float m = -INFINITY, l = 0.f;
-        float2 o = make_float2(0.f, 0.f);
-        for (int j = 0; j < ks.s_end + ks.n_cnt; ++j) {
-            const float *kr = bw_key_row(a, ks, u, j);
-            const float s = bw_dot(q, bw_ld2(kr + a.d, h, a.hd, lane)) * a.scale;
-            if (s > m) {
-                const float corr = expf(m - s);
-                l *= corr;
-                o.x *= corr;
-                o.y *= corr;
-                m = s;
-            }
-            const float pj = expf(s - m);
-            const float2 v = bw_ld2(kr + 2 * a.d, h, a.hd, lane);
-            l += pj;
-            o.x = fmaf(pj, v.x, o.x);
-            o.y = fmaf(pj, v.y, o.y);
-        }
-        bw_st2(a.O + orow * a.d, h, a.hd, lane, make_float2(o.x / l, o.y / l));
-        if (lane == 0) {
-            a.stat_m[orow * a.H + h] = m;
-            a.stat_l[orow * a.H + h] = l;
-        }
-    }
-}
-
-// One warp per (query row, head): D = dO . O and
-// dQ = scale sum_j p_j (dO . v_j - D) k_j.
-__global__ void attn_bwd_q_kernel(BwAttn a)
-{
-    const int lane = threadIdx.x & 31;
-    const long long total = static_cast<long long>(a.U) * a.nq * a.H;
-    for (long long w = bw_warp_id(); w < total; w += bw_warp_count()) {
-        const int h = static_cast<int>(w % a.H);
-        const long long orow = w / a.H;
-        const int u = static_cast<int>(orow / a.nq), i = static_cast<int>(orow % a.nq);
-        const long long qrow = static_cast<long long>(u) * a.q_ustride + a.q_off + i;
-        const float2 q = bw_ld2(a.qkv + qrow * a.ld, h, a.hd, lane);
-        const float2 dO = bw_ld2(a.dO + orow * a.d, h, a.hd, lane);
-        const float D = bw_dot(dO, bw_ld2(a.O + orow * a.d, h, a.hd, lane));
-        const float m = a.stat_m[orow * a.H + h], inv_l = 1.0f / a.stat_l[orow * a.H + h];
-        const BwKeys ks = bw_keys(a, u, i);
-        float2 dq = make_float2(0.f, 0.f);
-        for (int j = 0; j < ks.s_end + ks.n_cnt; ++j) {
-            const float *kr = bw_key_row(a, ks, u, j);
-            const float2 k = bw_ld2(kr + a.d, h, a.hd, lane);
-            const float p = expf(bw_dot(q, k) * a.scale - m) * inv_l;
-            const float ds = p * (bw_dot(dO, bw_ld2(kr + 2 * a.d, h, a.hd, lane)) - D) * a.scale;
-            dq.x = fmaf(ds, k.x, dq.x);
-            dq.y = fmaf(ds, k.y, dq.y);
-        }
-        bw_st2(a.dqkv + qrow * a.ld, h, a.hd, lane, dq);
-        if (lane == 0) a.stat_D[orow * a.H + h] = D;
-    }
-}
-
-// Contribution of query (qrow, orow) of problem a to the key (k, v):
-// dK += ds q, dV += p dO.
-__device__ __forceinline__ void bw_kv_add(const BwAttn &a, long long qrow, long long orow, int h, int lane, float2 k,
-                                          float2 v, float2 &dk, float2 &dv)
-{
-    const float2 q = bw_ld2(a.qkv + qrow * a.ld, h, a.hd, lane);
-    const float2 dO = bw_ld2(a.dO + orow * a.d, h, a.hd, lane);
-    const long long st = orow * a.H + h;
-    const float p = expf(bw_dot(q, k) * a.scale - a.stat_m[st]) / a.stat_l[st];
-    const float ds = p * (bw_dot(dO, v) - a.stat_D[st]) * a.scale;
-    dk.x = fmaf(ds, q.x, dk.x);
-    dk.y = fmaf(ds, q.y, dk.y);
-    dv.x = fmaf(p, dO.x, dv.x);
-    dv.y = fmaf(p, dO.y, dv.y);
-}
-
-// S keys of the layer: the S tail queries (problem sq) at or after the key
-// and, if has_ns, every NS query of the user (problem nsq).
-__global__ void attn_bwd_kv_s_kernel(BwAttn sq, BwAttn nsq, int has_ns)
-{
-    const int lane = threadIdx.x & 31;
-    const long long total = static_cast<long long>(sq.U) * sq.L * sq.H;
-    for (long long w = bw_warp_id(); w < total; w += bw_warp_count()) {
-        const int h = static_cast<int>(w % sq.H);
-        const long long krow = w / sq.H; // = u * L + j
-        const int u = static_cast<int>(krow / sq.L), j = static_cast<int>(krow % sq.L);
-        const float *kr = sq.skv + krow * sq.ld;
-        const float2 k = bw_ld2(kr + sq.d, h, sq.hd, lane), v = bw_ld2(kr + 2 * sq.d, h, sq.hd, lane);
-        float2 dk = make_float2(0.f, 0.f), dv = make_float2(0.f, 0.f);
-        // tail query i is S row L - nq + i; it sees key j when that row is >= j
-        for (int i = max(0, j - (sq.L - sq.nq)); i < sq.nq; ++i)
-            bw_kv_add(sq, static_cast<long long>(u) * sq.q_ustride + sq.q_off + i,
-                      static_cast<long long>(u) * sq.nq + i, h, lane, k, v, dk, dv);
-        if (has_ns)
-            for (int i = 0; i < nsq.nq; ++i)
-                bw_kv_add(nsq, static_cast<long long>(u) * nsq.q_ustride + i, static_cast<long long>(u) * nsq.nq + i,
-                          h, lane, k, v, dk, dv);
-        float *dr = sq.dskv + krow * sq.ld;
-        bw_st2(dr + sq.d, h, sq.hd, lane, dk);
-        bw_st2(dr + 2 * sq.d, h, sq.hd, lane, dv);
-    }
-}
-
-// NS keys: key m of candidate c is seen by the candidate's NS rows n >= m.
-__global__ void attn_bwd_kv_ns_kernel(BwAttn a)
-{
-    const int lane = threadIdx.x & 31;
-    const long long total = static_cast<long long>(a.U) * a.nq * a.H;
-    for (long long w = bw_warp_id(); w < total; w += bw_warp_count()) {
-        const int h = static_cast<int>(w % a.H);
-        const long long orow = w / a.H;
-        const int u = static_cast<int>(orow / a.nq), j = static_cast<int>(orow % a.nq);
-        const long long ubase = static_cast<long long>(u) * a.q_ustride;
-        const float *kr = a.qkv + (ubase + j) * a.ld;
-        const float2 k = bw_ld2(kr + a.d, h, a.hd, lane), v = bw_ld2(kr + 2 * a.d, h, a.hd, lane);
-        float2 dk = make_float2(0.f, 0.f), dv = make_float2(0.f, 0.f);
-        const int c_end = (j / a.N + 1) * a.N;
-        for (int i = j; i < c_end; ++i)
-            bw_kv_add(a, ubase + i, static_cast<long long>(u) * a.nq + i, h, lane, k, v, dk, dv);
-        float *dr = a.dqkv + (ubase + j) * a.ld;
-        bw_st2(dr + a.d, h, a.hd, lane, dk);
-        bw_st2(dr + 2 * a.d, h, a.hd, lane, dv);
-    }
-}
-
 // ---------------------------------------------------------------- launchers
 static int bw_blocks(long long threads)
 {
@@ -548,37 +371,6 @@ cudaError_t bw_gemm(const BwGemm &p, cudaStream_t s)
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || splits == 1) return e;
     tn_reduce_kernel<<<bw_blocks(static_cast<long long>(p.M) * p.N * p.G), 256, 0, s>>>(p);
-    return cudaGetLastError();
-}
-
-static long long attn_threads(const BwAttn &a) { return static_cast<long long>(a.U) * a.nq * a.H * 32; }
-
-cudaError_t bw_attn_fwd(const BwAttn &a, cudaStream_t s)
-{
-    if (a.hd > 64) return cudaErrorInvalidValue;
-    attn_fwd_kernel<<<bw_blocks(attn_threads(a)), 256, 0, s>>>(a);
-    return cudaGetLastError();
-}
-
-cudaError_t bw_attn_bwd_q(const BwAttn &a, cudaStream_t s)
-{
-    if (a.hd > 64) return cudaErrorInvalidValue;
-    attn_bwd_q_kernel<<<bw_blocks(attn_threads(a)), 256, 0, s>>>(a);
-    return cudaGetLastError();
-}
-
-cudaError_t bw_attn_bwd_kv_s(const BwAttn &sq, const BwAttn *nsq, cudaStream_t s)
-{
-    if (sq.hd > 64) return cudaErrorInvalidValue;
-    attn_bwd_kv_s_kernel<<<bw_blocks(static_cast<long long>(sq.U) * sq.L * sq.H * 32), 256, 0, s>>>(
-        sq, nsq ? *nsq : sq, nsq ? 1 : 0);
-    return cudaGetLastError();
-}
-
-cudaError_t bw_attn_bwd_kv_ns(const BwAttn &a, cudaStream_t s)
-{
-    if (a.hd > 64) return cudaErrorInvalidValue;
-    attn_bwd_kv_ns_kernel<<<bw_blocks(attn_threads(a)), 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 
