@@ -263,6 +263,123 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
     }
 }
 
+// The same three forms on 128 x 128 tiles, 8-deep k steps, 8 x 8 outputs
+// per thread (rows ty*4 + i and 64 + ty*4 + i, columns likewise), the next
+// k step's operands fetched into registers while the current one computes.
+constexpr int GL_M = 128, GL_N = 128, GL_K = 8;
+
+template <int FORM>
+__global__ void __launch_bounds__(GB_T) bw_gemm_big_kernel(BwGemm p)
+{
+    __shared__ __align__(16) float As[GL_K][GL_M + 4];
+    __shared__ __align__(16) float Bs[GL_K][GL_N + 4];
+    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+    const int g = FORM == BW_TN ? static_cast<int>(blockIdx.z) / p.splits : static_cast<int>(blockIdx.z);
+    const int split = FORM == BW_TN ? static_cast<int>(blockIdx.z) % p.splits : 0;
+    const int m0 = blockIdx.y * GL_M, n0 = blockIdx.x * GL_N;
+    int k_lo = 0, k_hi = p.K;
+    if (FORM == BW_TN && p.splits > 1) {
+        const int chunk = ((p.K + p.splits - 1) / p.splits + GL_K - 1) / GL_K * GL_K;
+        k_lo = min(p.K, split * chunk);
+        k_hi = min(p.K, k_lo + chunk);
+    }
+    // staging: NT / NN A and NT B are row-major in k (thread: row t / 2,
+    // k quad (t % 2) * 4); TN A and NN / TN B are row-major in m / n
+    // (thread: k row t / 32, 4 columns (t % 32) * 4)
+    const int rq = tid >> 1, kq = (tid & 1) * 4, kr = tid >> 5, cq = (tid & 31) * 4;
+    const float *arow = nullptr, *brow = nullptr;
+    if (FORM != BW_TN && m0 + rq < p.M) arow = p.A + bw_row(p.a_map, m0 + rq, g) * p.lda;
+    if (FORM == BW_NT && n0 + rq < p.N) brow = p.B + g * p.b_gstride + static_cast<long long>(n0 + rq) * p.ldb;
+    float ra[4], rb[4];
+    auto fetch = [&](int k0) {
+        if (FORM != BW_TN) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) ra[q] = (arow && k0 + kq + q < k_hi) ? arow[k0 + kq + q] : 0.f;
+        } else {
+            const int k = k0 + kr;
+            const float *src = k < k_hi ? p.A + bw_row(p.a_map, k, g) * p.lda : nullptr;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) ra[q] = (src && m0 + cq + q < p.M) ? src[m0 + cq + q] : 0.f;
+        }
+        if (FORM == BW_NT) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) rb[q] = (brow && k0 + kq + q < k_hi) ? brow[k0 + kq + q] : 0.f;
+        } else {
+            const int k = k0 + kr;
+            const float *src = nullptr;
+            if (k < k_hi)
+                src = FORM == BW_NN ? p.B + g * p.b_gstride + static_cast<long long>(k) * p.ldb
+                                    : p.B + bw_row(p.b_map, k, g) * p.ldb;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) rb[q] = (src && n0 + cq + q < p.N) ? src[n0 + cq + q] : 0.f;
+        }
+    };
+    auto stage = [&]() {
+        if (FORM != BW_TN) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) As[kq + q][rq] = ra[q];
+        } else {
+            *reinterpret_cast<float4 *>(&As[kr][cq]) = make_float4(ra[0], ra[1], ra[2], ra[3]);
+        }
+        if (FORM == BW_NT) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) Bs[kq + q][rq] = rb[q];
+        } else {
+            *reinterpret_cast<float4 *>(&Bs[kr][cq]) = make_float4(rb[0], rb[1], rb[2], rb[3]);
+        }
+    };
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    if (k_lo < k_hi) {
+        fetch(k_lo);
+        stage();
+    }
+    __syncthreads();
+    for (int k0 = k_lo; k0 < k_hi; k0 += GL_K) {
+        const bool more = k0 + GL_K < k_hi;
+        if (more) fetch(k0 + GL_K);
+#pragma unroll
+        for (int k = 0; k < GL_K; ++k) {
+            const float4 a0 = *reinterpret_cast<const float4 *>(&As[k][ty * 4]);
+            const float4 a1 = *reinterpret_cast<const float4 *>(&As[k][64 + ty * 4]);
+            const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[k][tx * 4]);
+            const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[k][64 + tx * 4]);
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+        __syncthreads();
+        if (more) {
+            stage();
+            __syncthreads();
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
+        if (m >= p.M) continue;
+        float *crow;
+        if (FORM == BW_TN && p.splits > 1)
+            crow = p.partial + ((static_cast<long long>(split) * p.G + g) * p.M + m) * p.N;
+        else if (FORM == BW_TN)
+            crow = p.C + g * p.c_gstride + static_cast<long long>(m) * p.ldc;
+        else
+            crow = p.C + bw_row(p.c_map, m, g) * p.ldc;
+        const bool add = p.accumulate && !(FORM == BW_TN && p.splits > 1);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int n = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
+            if (n < p.N) crow[n] = add ? crow[n] + acc[i][j] : acc[i][j];
+        }
+    }
+}
+
 // C[g][m][n] (+)= sum over splits, in split order, of partial[s][g][m][n]
 __global__ void tn_reduce_kernel(BwGemm p)
 {
@@ -339,9 +456,13 @@ cudaError_t bw_rows_add(float *dst, RowMap dst_map, const float *src, long long 
     return cudaGetLastError();
 }
 
+// 128 x 128 tiles where both output dimensions fill them
+static bool bw_big(int M, int N) { return M >= GL_M && N >= GL_N; }
+
 int bw_tn_splits(int M, int N, int K, int G)
 {
-    const long long tiles = static_cast<long long>((M + GB_M - 1) / GB_M) * ((N + GB_N - 1) / GB_N) * G;
+    const int tm = bw_big(M, N) ? GL_M : GB_M, tn = bw_big(M, N) ? GL_N : GB_N;
+    const long long tiles = static_cast<long long>((M + tm - 1) / tm) * ((N + tn - 1) / tn) * G;
     long long sp = (2 * 148 + tiles - 1) / tiles;
     const long long by_k = (K + 255) / 256; // at least 256 reduction rows per split
     if (sp > by_k) sp = by_k;
@@ -358,14 +479,19 @@ long long bw_tn_partial_floats(int M, int N, int K, int G)
 cudaError_t bw_gemm(const BwGemm &p, cudaStream_t s)
 {
     const int splits = p.form == BW_TN ? p.splits : 1;
-    const dim3 grid((p.N + GB_N - 1) / GB_N, (p.M + GB_M - 1) / GB_M, p.G * splits);
+    const bool big = bw_big(p.M, p.N);
+    const int tm = big ? GL_M : GB_M, tn = big ? GL_N : GB_N;
+    const dim3 grid((p.N + tn - 1) / tn, (p.M + tm - 1) / tm, p.G * splits);
     if (p.M < 1 || p.N < 1 || p.K < 1 || p.G < 1 || splits < 1 || grid.y > 65535 || grid.z > 65535 ||
         (splits > 1 && !p.partial))
         return cudaErrorInvalidValue;
-    switch (p.form) {
-    case BW_NT: bw_gemm_kernel<BW_NT><<<grid, GB_T, 0, s>>>(p); break;
-    case BW_NN: bw_gemm_kernel<BW_NN><<<grid, GB_T, 0, s>>>(p); break;
-    case BW_TN: bw_gemm_kernel<BW_TN><<<grid, GB_T, 0, s>>>(p); break;
+    switch (p.form * 2 + (big ? 1 : 0)) {
+    case BW_NT * 2: bw_gemm_kernel<BW_NT><<<grid, GB_T, 0, s>>>(p); break;
+    case BW_NN * 2: bw_gemm_kernel<BW_NN><<<grid, GB_T, 0, s>>>(p); break;
+    case BW_TN * 2: bw_gemm_kernel<BW_TN><<<grid, GB_T, 0, s>>>(p); break;
+    case BW_NT * 2 + 1: bw_gemm_big_kernel<BW_NT><<<grid, GB_T, 0, s>>>(p); break;
+    case BW_NN * 2 + 1: bw_gemm_big_kernel<BW_NN><<<grid, GB_T, 0, s>>>(p); break;
+    case BW_TN * 2 + 1: bw_gemm_big_kernel<BW_TN><<<grid, GB_T, 0, s>>>(p); break;
     default: return cudaErrorInvalidValue;
     }
     cudaError_t e = cudaGetLastError();
@@ -419,8 +545,8 @@ struct Backward {
     float *Xout_last, *Yout_last;
     Side s, n;
     float *partial;
-    float *tn_partial; // split TN GEMMs: < 2 * 296 tiles of 64 x 64 floats
-    static constexpr long long kTnPartialFloats = 2LL * 296 * 64 * 64;
+    float *tn_partial; // split TN GEMMs: < 2 * 296 tiles of at most 128 x 128 floats
+    static constexpr long long kTnPartialFloats = 2LL * 296 * 128 * 128;
     float *dXbuf[2], *dYbuf[2];
     const float *G_s, *G_ns;
     float *dS, *dns;
