@@ -920,6 +920,9 @@ def main():
                     help="users per GPU instead of the workload's (a small case for profiling)")
     ap.add_argument("--c-sweep", action="store_true",
                     help="also score the serving caches at C = 1, 2, 4, 8, 16, 64, 512")
+    ap.add_argument("--training", action="store_true",
+                    help="time only the fp32 training step (ot_full_backward) at the workload's "
+                         "shapes, --users users (default 16), and print its JSON object")
     args = ap.parse_args()
     args.steps_ref = max(1, args.steps)
     args.warmup_ref = args.warmup
@@ -927,7 +930,15 @@ def main():
     wl = WORKLOADS[args.workload]
     if args.users > 0:
         wl = wl.with_(users=args.users)
-    if args.impl == "reference":
+    if args.training:
+        import torch
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        res = run_backward_point(args.workload, args.users or 16, args.steps, flush, 1, None, dev,
+                                 load_peaks())
+        print(json.dumps(res))
+    elif args.impl == "reference":
         run_reference(args, wl)
     else:
         run_ours(args, wl)

@@ -265,14 +265,16 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
 
 // The same three forms on 128 x 128 tiles, 8-deep k steps, 8 x 8 outputs
 // per thread (rows ty*4 + i and 64 + ty*4 + i, columns likewise), the next
-// k step's operands fetched into registers while the current one computes.
+// k step's operands fetched into registers while the current one computes
+// and staged into the other of two shared-memory buffers (one barrier per
+// k step).
 constexpr int GL_M = 128, GL_N = 128, GL_K = 8;
 
 template <int FORM>
-__global__ void __launch_bounds__(GB_T) bw_gemm_big_kernel(BwGemm p)
+__global__ void __launch_bounds__(GB_T, 2) bw_gemm_big_kernel(BwGemm p)
 {
-    __shared__ __align__(16) float As[GL_K][GL_M + 4];
-    __shared__ __align__(16) float Bs[GL_K][GL_N + 4];
+    __shared__ __align__(16) float As[2][GL_K][GL_M + 4];
+    __shared__ __align__(16) float Bs[2][GL_K][GL_N + 4];
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
     const int g = FORM == BW_TN ? static_cast<int>(blockIdx.z) / p.splits : static_cast<int>(blockIdx.z);
     const int split = FORM == BW_TN ? static_cast<int>(blockIdx.z) % p.splits : 0;
@@ -314,18 +316,18 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_big_kernel(BwGemm p)
             for (int q = 0; q < 4; ++q) rb[q] = (src && n0 + cq + q < p.N) ? src[n0 + cq + q] : 0.f;
         }
     };
-    auto stage = [&]() {
+    auto stage = [&](int bf) {
         if (FORM != BW_TN) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) As[kq + q][rq] = ra[q];
+            for (int q = 0; q < 4; ++q) As[bf][kq + q][rq] = ra[q];
         } else {
-            *reinterpret_cast<float4 *>(&As[kr][cq]) = make_float4(ra[0], ra[1], ra[2], ra[3]);
+            *reinterpret_cast<float4 *>(&As[bf][kr][cq]) = make_float4(ra[0], ra[1], ra[2], ra[3]);
         }
         if (FORM == BW_NT) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) Bs[kq + q][rq] = rb[q];
+            for (int q = 0; q < 4; ++q) Bs[bf][kq + q][rq] = rb[q];
         } else {
-            *reinterpret_cast<float4 *>(&Bs[kr][cq]) = make_float4(rb[0], rb[1], rb[2], rb[3]);
+            *reinterpret_cast<float4 *>(&Bs[bf][kr][cq]) = make_float4(rb[0], rb[1], rb[2], rb[3]);
         }
     };
     float acc[8][8];
@@ -335,18 +337,19 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_big_kernel(BwGemm p)
         for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
     if (k_lo < k_hi) {
         fetch(k_lo);
-        stage();
+        stage(0);
     }
     __syncthreads();
+    int bf = 0;
     for (int k0 = k_lo; k0 < k_hi; k0 += GL_K) {
         const bool more = k0 + GL_K < k_hi;
         if (more) fetch(k0 + GL_K);
 #pragma unroll
         for (int k = 0; k < GL_K; ++k) {
-            const float4 a0 = *reinterpret_cast<const float4 *>(&As[k][ty * 4]);
-            const float4 a1 = *reinterpret_cast<const float4 *>(&As[k][64 + ty * 4]);
-            const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[k][tx * 4]);
-            const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[k][64 + tx * 4]);
+            const float4 a0 = *reinterpret_cast<const float4 *>(&As[bf][k][ty * 4]);
+            const float4 a1 = *reinterpret_cast<const float4 *>(&As[bf][k][64 + ty * 4]);
+            const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[bf][k][tx * 4]);
+            const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[bf][k][64 + tx * 4]);
             const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -354,11 +357,11 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_big_kernel(BwGemm p)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
+        // the other buffer was last read in the previous step, before the
+        // barrier that ended it
+        if (more) stage(bf ^ 1);
         __syncthreads();
-        if (more) {
-            stage();
-            __syncthreads();
-        }
+        bf ^= 1;
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -849,6 +852,7 @@ ot_status bw_validate(const ot_config *cfg, int U, int C)
     // GEMM rows stay below 2^31 / 64 (the grid's 65535 row tiles) and U * C fits an int
     const long long rs = static_cast<long long>(U) * cfg->L0, rn = static_cast<long long>(U) * C;
     if (rs > 65535LL * 64 || rn > 65535LL * 64) return OT_ERR_SHAPE;
+    if (static_cast<long long>(C) * cfg->n_ns >= (1LL << 30)) return OT_ERR_SHAPE; // NS rows of a user: int
     return OT_OK;
 }
 

@@ -1,6 +1,7 @@
 // Attention of the backward pass (fp32, CUDA cores), tiled in the order of
 // the FlashAttention-2 backward: a forward per 64-row query block that keeps
-// each row's softmax statistics (max m, sum l), dQ per 64-row query block,
+// each row's softmax statistics (max m of the scores in base-2 units, sum l
+// of 2^(s log2(e) - m); exponentials by ex2.approx), dQ per 64-row query block,
 // and dK / dV per 64-key block, each CTA summing over the query blocks that
 // see its keys — every output is written by exactly one CTA, so there are no
 // atomics and the result is the same bit for bit run to run.
@@ -19,6 +20,7 @@
 #include <stdint.h>
 
 #include "ot_internal.h"
+#include "ot_ptx.cuh"
 
 namespace ot {
 
@@ -27,12 +29,22 @@ namespace {
 constexpr int TB = 64;      // query rows / keys per tile
 constexpr int TP = TB + 4;  // pitch of transposed tiles (16-byte rows)
 constexpr int NT = 256;     // threads
+constexpr float LOG2E = 1.4426950408889634f;
 
 struct KeySpace {
-    int nks;            // S keys
-    int nkn;            // NS keys
-    long long k_begin;  // first NS key row (within the user's NS rows)
+    int nks;      // S keys
+    int nkn;      // NS keys
+    int k_begin;  // first NS key row (within the user's NS rows, < 2^30)
 };
+
+// [64][64] tiles of P / dS, written as 4 x 4 blocks by the 16 x 16 threads
+// and read as float4 rows: 16-byte chunk c of row r sits at chunk
+// c ^ ((r / 4) % 8), so the 16 threads writing rows 4 tx + j of one column
+// hit 8 different chunks (2-way instead of 8-way bank conflicts).
+__device__ __forceinline__ int sw(int r, int k)
+{
+    return r * TB + ((((k >> 2) ^ ((r >> 2) & 7)) << 2) | (k & 3));
+}
 
 __device__ __forceinline__ long long q_row(const BwAttn &a, int u, int i)
 {
@@ -51,7 +63,7 @@ __device__ __forceinline__ KeySpace key_space(const BwAttn &a, int i0, int i1)
         const int c0 = i0 / a.N, c1 = (i1 - 1) / a.N + 1;
         ks.nks = a.L;
         ks.nkn = (c1 - c0) * a.N;
-        ks.k_begin = static_cast<long long>(c0) * a.N;
+        ks.k_begin = c0 * a.N;
     }
     return ks;
 }
@@ -65,8 +77,17 @@ __device__ __forceinline__ const float *key_row(const BwAttn &a, const KeySpace 
 __device__ __forceinline__ bool visible(const BwAttn &a, const KeySpace &ks, int i, int j)
 {
     if (j < ks.nks) return a.mode == 1 || j <= a.L - a.nq + i;
-    const long long r = ks.k_begin + (j - ks.nks);
-    return r / a.N == i / a.N && r % a.N <= i % a.N;
+    const int r = ks.k_begin + (j - ks.nks);
+    const int ci = i / a.N;
+    return r >= ci * a.N && r <= i; // same candidate, position m <= n
+}
+
+// every (row, key) of rows [i0, i0 + 64) x keys [j0, j0 + 64) visible and
+// every key valid (rows past the problem do not matter to the caller)
+__device__ __forceinline__ bool block_full(const BwAttn &a, const KeySpace &ks, int i0, int j0)
+{
+    if (j0 + TB > ks.nks) return false; // reaches NS keys or past the S keys
+    return a.mode == 1 || j0 + TB - 1 <= a.L - a.nq + i0;
 }
 
 __device__ __forceinline__ float half_warp_max(float v)
@@ -120,9 +141,9 @@ __device__ __forceinline__ void tile_dot(const float *A, int a0, const float *B,
     }
 }
 
-template <int HD> constexpr int fwd_smem_floats() { return 2 * HD * TP + TB * (HD + 4) + TB * TP; }
-template <int HD> constexpr int dq_smem_floats() { return 4 * HD * TP + TB * (HD + 4) + TB * TP + 3 * TB; }
-template <int HD> constexpr int dkv_smem_floats() { return 4 * HD * TP + 2 * TB * (HD + 4) + 2 * TB * TP + 3 * TB; }
+template <int HD> constexpr int fwd_smem_floats() { return 2 * HD * TP + TB * (HD + 4) + TB * TB; }
+template <int HD> constexpr int dq_smem_floats() { return 4 * HD * TP + TB * (HD + 4) + TB * TB + 3 * TB; }
+template <int HD> constexpr int dkv_smem_floats() { return 4 * HD * TP + 2 * TB * (HD + 4) + 2 * TB * TB + 3 * TB; }
 
 // ------------------------------------------------------------ forward
 template <int HD>
@@ -130,7 +151,7 @@ __global__ void __launch_bounds__(NT) attn_fwd_tiled(BwAttn a, int n_qb)
 {
     constexpr int CPT = HD / 16, VP = HD + 4;
     extern __shared__ __align__(16) float sm[];
-    float *QT = sm, *KT = QT + HD * TP, *Vs = KT + HD * TP, *PT = Vs + TB * VP;
+    float *QT = sm, *KT = QT + HD * TP, *Vs = KT + HD * TP, *PT = Vs + TB * VP; // PT: [key][row], sw()
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
     const long long items = static_cast<long long>(a.U) * a.H * n_qb;
     for (long long item = blockIdx.x; item < items; item += gridDim.x) {
@@ -149,6 +170,7 @@ __global__ void __launch_bounds__(NT) attn_fwd_tiled(BwAttn a, int n_qb)
 #pragma unroll
             for (int c = 0; c < CPT; ++c) o[i][c] = 0.f;
         }
+        const float c2 = a.scale * LOG2E; // scores in base-2 units
         for (int j0 = 0; j0 < nk; j0 += TB) {
             __syncthreads();
             for (int e = tid; e < TB * HD; e += NT) {
@@ -165,6 +187,7 @@ __global__ void __launch_bounds__(NT) attn_fwd_tiled(BwAttn a, int n_qb)
             __syncthreads();
             float s[4][4] = {};
             tile_dot<HD>(QT, ty * 4, KT, tx * 4, s);
+            const bool full = block_full(a, ks, i0, j0);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int qi = i0 + ty * 4 + i;
@@ -172,18 +195,18 @@ __global__ void __launch_bounds__(NT) attn_fwd_tiled(BwAttn a, int n_qb)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int kj = j0 + tx * 4 + j;
-                    const bool vis = qi < i1 && kj < nk && visible(a, ks, qi, kj);
-                    s[i][j] = vis ? s[i][j] * a.scale : -INFINITY;
+                    const bool vis = full || (qi < i1 && kj < nk && visible(a, ks, qi, kj));
+                    s[i][j] = vis ? s[i][j] * c2 : -INFINITY;
                     bmax = fmaxf(bmax, s[i][j]);
                 }
                 bmax = half_warp_max(bmax);
-                const float mn = fmaxf(m[i], bmax), corr = expf(m[i] - mn);
+                const float mn = fmaxf(m[i], bmax), corr = fast_exp2(m[i] - mn);
                 m[i] = mn;
                 float ps = 0.f;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const float p = expf(s[i][j] - mn);
-                    PT[(tx * 4 + j) * TP + ty * 4 + i] = p;
+                    const float p = fast_exp2(s[i][j] - mn);
+                    PT[sw(tx * 4 + j, ty * 4 + i)] = p;
                     ps += p;
                 }
                 l[i] = l[i] * corr + half_warp_sum(ps);
@@ -193,7 +216,7 @@ __global__ void __launch_bounds__(NT) attn_fwd_tiled(BwAttn a, int n_qb)
             __syncthreads();
 #pragma unroll 4
             for (int kk = 0; kk < TB; ++kk) {
-                const float4 p4 = ld4(PT + kk * TP + ty * 4);
+                const float4 p4 = ld4(PT + sw(kk, ty * 4));
                 const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
                 float v[CPT];
 #pragma unroll
@@ -228,7 +251,7 @@ __global__ void __launch_bounds__(NT) attn_dq_tiled(BwAttn a, int n_qb)
     constexpr int CPT = HD / 16, VP = HD + 4;
     extern __shared__ __align__(16) float sm[];
     float *QT = sm, *dOT = QT + HD * TP, *KT = dOT + HD * TP, *VT = KT + HD * TP;
-    float *Ks = VT + HD * TP, *dST = Ks + TB * VP, *sM = dST + TB * TP, *sL = sM + TB, *sD = sL + TB;
+    float *Ks = VT + HD * TP, *dST = Ks + TB * VP, *sM = dST + TB * TB, *sL = sM + TB, *sD = sL + TB;
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15, lane = tid & 31, warp = tid >> 5;
     const long long items = static_cast<long long>(a.U) * a.H * n_qb;
     for (long long item = blockIdx.x; item < items; item += gridDim.x) {
@@ -252,7 +275,7 @@ __global__ void __launch_bounds__(NT) attn_dq_tiled(BwAttn a, int n_qb)
                 const long long st = (orow0 + r) * a.H + h;
                 sD[r] = dsum;
                 sM[r] = r < n ? a.stat_m[st] : 0.f;
-                sL[r] = r < n ? a.stat_l[st] : 1.f;
+                sL[r] = r < n ? 1.0f / a.stat_l[st] : 1.f; // 1 / l
                 if (r < n) a.stat_D[st] = dsum;
             }
         }
@@ -279,24 +302,27 @@ __global__ void __launch_bounds__(NT) attn_dq_tiled(BwAttn a, int n_qb)
             float s[4][4] = {}, dp[4][4] = {};
             tile_dot<HD>(QT, ty * 4, KT, tx * 4, s);
             tile_dot<HD>(dOT, ty * 4, VT, tx * 4, dp);
+            const bool full = block_full(a, ks, i0, j0);
+            const float c2 = a.scale * LOG2E;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int r = ty * 4 + i, qi = i0 + r;
+                const float mr = sM[r], il = sL[r], dr = sD[r];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int kj = j0 + tx * 4 + j;
                     float ds = 0.f;
-                    if (qi < i1 && kj < nk && visible(a, ks, qi, kj)) {
-                        const float p = expf(s[i][j] * a.scale - sM[r]) / sL[r];
-                        ds = p * (dp[i][j] - sD[r]) * a.scale;
+                    if (full || (qi < i1 && kj < nk && visible(a, ks, qi, kj))) {
+                        const float p = fast_exp2(s[i][j] * c2 - mr) * il;
+                        ds = p * (dp[i][j] - dr) * a.scale;
                     }
-                    dST[(tx * 4 + j) * TP + r] = ds;
+                    dST[sw(tx * 4 + j, r)] = ds;
                 }
             }
             __syncthreads();
 #pragma unroll 4
             for (int kk = 0; kk < TB; ++kk) {
-                const float4 d4 = ld4(dST + kk * TP + ty * 4);
+                const float4 d4 = ld4(dST + sw(kk, ty * 4));
                 const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
                 float kv[CPT];
 #pragma unroll
@@ -329,8 +355,8 @@ __global__ void __launch_bounds__(NT) attn_dkv_tiled(BwAttn p0, BwAttn p1, int n
     constexpr int CPT = HD / 16, VP = HD + 4;
     extern __shared__ __align__(16) float sm[];
     float *KT = sm, *VT = KT + HD * TP, *QT = VT + HD * TP, *dOT = QT + HD * TP;
-    float *Qs = dOT + HD * TP, *dOs = Qs + TB * VP, *PS = dOs + TB * VP, *dSs = PS + TB * TP;
-    float *sM = dSs + TB * TP, *sL = sM + TB, *sD = sL + TB;
+    float *Qs = dOT + HD * TP, *dOs = Qs + TB * VP, *PS = dOs + TB * VP, *dSs = PS + TB * TB;
+    float *sM = dSs + TB * TB, *sL = sM + TB, *sD = sL + TB;
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
     const int nkeys = kind == 0 ? p0.L : p0.nq;
     const KeySpace ks{kind == 0 ? p0.L : 0, kind == 0 ? 0 : p0.nq, 0};
@@ -381,33 +407,38 @@ __global__ void __launch_bounds__(NT) attn_dkv_tiled(BwAttn p0, BwAttn p1, int n
                 for (int r = tid; r < TB; r += NT) {
                     const long long st = (orow0 + r) * P.H + h;
                     sM[r] = r < n ? P.stat_m[st] : 0.f;
-                    sL[r] = r < n ? P.stat_l[st] : 1.f;
+                    sL[r] = r < n ? 1.0f / P.stat_l[st] : 1.f; // 1 / l
                     sD[r] = r < n ? P.stat_D[st] : 0.f;
                 }
                 __syncthreads();
-                // thread: keys ty*4 + i, query rows tx*4 + j
+                // thread: keys ty*4 + i, query rows tx*4 + j.  Rows past n
+                // hold Q = dO = 0 and D = 0: their p multiplies dO = 0 and
+                // their dS is 0, so only the mask needs them
                 float s[4][4] = {}, dp[4][4] = {};
                 tile_dot<HD>(KT, ty * 4, QT, tx * 4, s);
                 tile_dot<HD>(VT, ty * 4, dOT, tx * 4, dp);
+                const bool full = kind == 0 && n == TB && (P.mode == 1 || j0 + TB - 1 <= P.L - P.nq + i0);
+                const float c2 = P.scale * LOG2E;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int r = tx * 4 + j, qi = i0 + r;
+                    const float mr = sM[r], il = sL[r], dr = sD[r];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int kj = j0 + ty * 4 + i;
                         float p = 0.f, ds = 0.f;
-                        if (r < n && kj < j1 && visible(P, ks, qi, kj)) {
-                            p = expf(s[i][j] * P.scale - sM[r]) / sL[r];
-                            ds = p * (dp[i][j] - sD[r]) * P.scale;
+                        if (full || (r < n && kj < j1 && visible(P, ks, qi, kj))) {
+                            p = fast_exp2(s[i][j] * c2 - mr) * il;
+                            ds = p * (dp[i][j] - dr) * P.scale;
                         }
-                        PS[r * TP + ty * 4 + i] = p;
-                        dSs[r * TP + ty * 4 + i] = ds;
+                        PS[sw(r, ty * 4 + i)] = p;
+                        dSs[sw(r, ty * 4 + i)] = ds;
                     }
                 }
                 __syncthreads();
 #pragma unroll 4
                 for (int r = 0; r < TB; ++r) {
-                    const float4 p4 = ld4(PS + r * TP + ty * 4), d4 = ld4(dSs + r * TP + ty * 4);
+                    const float4 p4 = ld4(PS + sw(r, ty * 4)), d4 = ld4(dSs + sw(r, ty * 4));
                     const float pv[4] = {p4.x, p4.y, p4.z, p4.w}, dsv[4] = {d4.x, d4.y, d4.z, d4.w};
                     float qv[CPT], ov[CPT];
 #pragma unroll

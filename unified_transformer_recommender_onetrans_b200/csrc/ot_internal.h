@@ -311,8 +311,9 @@ struct BwGemm {
 //   mode 1 (NS queries): query i = c * N + n of user u is row
 //     u * q_ustride + i of qkv; it sees the user's L S keys (rows u * L + j
 //     of skv) and NS keys c * N + m, m <= n (rows of qkv).
-// O / dO are [U * nq][d]; stat_* [U * nq][H]; dqkv / dskv take dQ and dK, dV
-// in the layout of qkv / skv.
+// O / dO are [U * nq][d]; stat_* [U * nq][H] (m: the row's max score in
+// base-2 units, s * scale * log2(e); l: the sum of 2^(s' - m); D: dO . O);
+// dqkv / dskv take dQ and dK, dV in the layout of qkv / skv.
 struct BwAttn {
     int mode, U, H, hd, d, L, nq, N;
     long long ld, q_ustride, q_off;
