@@ -319,7 +319,7 @@ void gemm_prepare(const ot_model *m, GemmArgs &a)
     a.in_dtype = m->cfg.dtype == OT_DTYPE_F32 ? OT_DTYPE_F32
                  : a.in_dtype == OT_DTYPE_FP8 ? OT_DTYPE_FP8
                                               : OT_DTYPE_BF16;
-    a.store = m->cfg.dtype == OT_DTYPE_F32 ? OT_STORE_F32 : OT_STORE_BF16;
+    a.store = m->cfg.dtype == OT_DTYPE_F32 ? OT_STORE_F32 : a.qscale ? OT_STORE_E4M3 : OT_STORE_BF16;
 }
 
 ot_status gemm(ot_model *m, GemmArgs &a, cudaStream_t s, int role)
@@ -529,6 +529,39 @@ ot_status projection(ot_model *m, GemmArgs &g, const void *src, long long lda, R
     g.g_scale = wscale;
     g.in_dtype = OT_DTYPE_FP8;
     return OT_OK;
+}
+
+// FP8 with per-tensor activation scales (and not calibrating): the first
+// FFN projection's epilogue writes the hidden as e4m3 with the second
+// projection's input scale, and the second projection reads it as is — no
+// quantisation pass over the 4d-wide hidden.
+bool fp8_fused_hidden(const ot_model *m)
+{
+    return m->cfg.dtype == OT_DTYPE_FP8 && m->act_scale && !m->calib_amax;
+}
+
+// per-tensor scale of input `in` of layer l, parameter set `set` (sets of
+// consecutive groups are 4 slots apart)
+const float *act_slot(const ot_model *m, int l, int set, int in)
+{
+    return m->act_scale + (static_cast<long long>(l) * (1 + m->cfg.n_ns) + set) * 4 + in;
+}
+
+// The second FFN projection on the e4m3 hidden the first one wrote.
+void fp8_hidden_operand(GemmArgs &g, const void *hid, long long lda, RowMap amap, const void *W, long long w_gstride,
+                        const float *wscale, const float *xscale)
+{
+    g.A = hid;
+    g.lda = lda;
+    g.a_map = amap;
+    g.B = W;
+    g.b_gstride = w_gstride;
+    g.norm = 0;
+    g.row_scale = nullptr;
+    g.g_scale = wscale;
+    g.xg_scale = xscale;
+    g.xg_gstride = 4;
+    g.in_dtype = OT_DTYPE_FP8;
 }
 
 EpiSeg seg_of(void *out, long long ld, int lo, int hi, RowMap map)
@@ -755,12 +788,20 @@ struct EncodeRun {
         g.gelu = 1;
         g.nseg = 1;
         g.seg[0] = seg_of(hid, f, 0, f, rowmap_identity());
+        const bool fh = fp8_fused_hidden(m);
+        if (fh) {
+            g.qscale = act_slot(m, l, 0, IN_W2);
+            g.qscale_gstride = 4;
+        }
         if ((r = gemm(m, g, st, ROLE_S_FFN1)) != OT_OK) return r;
         g = gemm_base(c, U * q, d, f, 1);
-        if ((r = projection(m, g, hid, f, rowmap_identity(),
-                            at(m->W2_s, static_cast<long long>(l) * d * f, wesz),
-                            static_cast<long long>(d) * f, fp8 ? m->sc_2_s + l : nullptr, nullptr, 0,
-                            false, f8, st, l, 0, IN_W2)) != OT_OK)
+        if (fh)
+            fp8_hidden_operand(g, hid, f, rowmap_identity(), at(m->W2_s, static_cast<long long>(l) * d * f, wesz),
+                               static_cast<long long>(d) * f, m->sc_2_s + l, act_slot(m, l, 0, IN_W2));
+        else if ((r = projection(m, g, hid, f, rowmap_identity(),
+                                 at(m->W2_s, static_cast<long long>(l) * d * f, wesz),
+                                 static_cast<long long>(d) * f, fp8 ? m->sc_2_s + l : nullptr, nullptr, 0,
+                                 false, f8, st, l, 0, IN_W2)) != OT_OK)
             return r;
         g.res = Hb;
         g.res_ld = d;
@@ -979,11 +1020,19 @@ struct ScoreRun {
         g.gelu = 1;
         g.nseg = 1;
         g.seg[0] = seg_of(hid, f, 0, f, gm);
+        const bool fh = fp8_fused_hidden(m);
+        if (fh) {
+            g.qscale = act_slot(m, l, 1, IN_W2); // group g: parameter set 1 + g
+            g.qscale_gstride = 4;
+        }
         if ((r = gemm(m, g, st, ROLE_NS_FFN1)) != OT_OK) return r;
         g = gemm_base(c, Mc, d, f, N);
-        if ((r = projection(m, g, hid, f, gm, at(m->W2_ns, lN * d * f, wesz),
-                            static_cast<long long>(d) * f, fp8 ? m->sc_2_ns + lN : nullptr, nullptr,
-                            0, false, f8, st, l, 1, IN_W2)) != OT_OK)
+        if (fh)
+            fp8_hidden_operand(g, hid, f, gm, at(m->W2_ns, lN * d * f, wesz), static_cast<long long>(d) * f,
+                               m->sc_2_ns + lN, act_slot(m, l, 1, IN_W2));
+        else if ((r = projection(m, g, hid, f, gm, at(m->W2_ns, lN * d * f, wesz),
+                                 static_cast<long long>(d) * f, fp8 ? m->sc_2_ns + lN : nullptr, nullptr,
+                                 0, false, f8, st, l, 1, IN_W2)) != OT_OK)
             return r;
         g.res = Hn;
         g.res_ld = d;

@@ -29,6 +29,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <math.h>
 
 #include "ot_gelu_fit.h"
@@ -105,6 +106,15 @@ __device__ __forceinline__ void decode_tile(const TcGemmParams &P, long long til
     n0 = nt * bn;
 }
 
+// four values -> e4m3 bytes (first value in the lowest byte), round to
+// nearest even, saturating
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d)
+{
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+    return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
 // staging layout: row r (0..31) is ROWB bytes, 16-byte chunk c stored at
 // (c & ~7) | ((c ^ r) & 7), so 8 consecutive rows hit 8 different bank groups
 template <int ROWB>
@@ -141,7 +151,8 @@ struct EpiTile {
     __nv_bfloat16 *obase;       // output segment base
     const float *row_scale;     // fp8: per-row scale (indexed through the A row map), or null
     long long row_scale_idx;
-    float g_scale;              // fp8: per-matrix scale (1 otherwise)
+    float g_scale;              // fp8: per-matrix scale (1 otherwise), times the A operand's per-group scale
+    float q_inv;                // e4m3 output: 1 / its scale
     float inv_k, eps;           // RMSNorm
 };
 
@@ -201,6 +212,8 @@ __device__ __forceinline__ void epi_tile(const TcGemmParams &Q, int q, int lane,
     e.row_scale = live ? a.row_scale : nullptr;
     e.row_scale_idx = e.row_scale ? rowmap_dev(a.a_map, r, e.g) : 0;
     e.g_scale = a.g_scale ? a.g_scale[e.g] : 1.f;
+    if (a.xg_scale) e.g_scale *= a.xg_scale[e.g * a.xg_gstride];
+    e.q_inv = a.qscale ? __frcp_rn(a.qscale[e.g * a.qscale_gstride]) : 1.f;
 }
 
 template <int BN, bool FP8, bool MULTI>
@@ -238,6 +251,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_kb = a0.K / (FP8 ? 128 : 64);
     const bool norm = a0.norm != 0 && !FP8;
+    const bool q8 = a0.store == OT_STORE_E4M3; // launch-wide (both problems agree)
     pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
@@ -428,6 +442,48 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             if (et.row_scale) rs *= et.row_scale[et.row_scale_idx];
             rs *= et.g_scale;
             __syncwarp(); // residual staging complete before rows are read back
+            if (q8) {
+                // e4m3 output (no residual): 32 columns -> two 16-byte chunks
+                // of the staging row (its first ROWB / 2 bytes), then
+                // coalesced stores
+#pragma unroll 1
+                for (int c = 0; c < G_EPI_COLS / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + b * G_BN + (static_cast<uint32_t>(q * 32) << 16) +
+                                  half * G_EPI_COLS + c * 32,
+                              v);
+                    tmem_ld_wait();
+                    tmem_reg_fence(v);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            f[e] = __uint_as_float(v[8 * j + e]) * rs;
+                            if (et.gelu) f[e] = gelu_fast(f[e]);
+                            f[e] *= et.q_inv;
+                        }
+                        uint2 o;
+                        o.x = pack_e4m3x4(f[0], f[1], f[2], f[3]);
+                        o.y = pack_e4m3x4(f[4], f[5], f[6], f[7]);
+                        reinterpret_cast<uint2 *>(stage_chunk<ROWB>(stage, lane, 2 * c + (j >> 1)))[j & 1] = o;
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[b]); // accumulator b may be overwritten
+                constexpr int LPR8 = ROWB / 32, RPI8 = 32 / LPR8; // e4m3 row: ROWB / 2 bytes
+                uint8_t *ob8 = reinterpret_cast<uint8_t *>(et.obase);
+#pragma unroll
+                for (int i = 0; i < 32 / RPI8; ++i) {
+                    const int rl = RPI8 * i + lane / LPR8, ch = lane % LPR8;
+                    const long long oo = __shfl_sync(0xffffffffu, out_off, rl);
+                    if (oo < 0) continue;
+                    *reinterpret_cast<uint4 *>(ob8 + oo + ch * 16) = *stage_chunk<ROWB>(stage, rl, ch);
+                }
+                __syncwarp(); // staging free for the next tile
+                continue;
+            }
 #pragma unroll 1
             for (int c = 0; c < G_EPI_COLS / 32; ++c) {
                 uint32_t v[32];
@@ -605,7 +661,8 @@ static cudaError_t launch_tc_cfg(const GemmArgs &a, const GemmArgs *a1, cudaStre
 static bool gemm_ok(const GemmArgs &a, bool &wide)
 {
     const bool fp8 = a.in_dtype == OT_DTYPE_FP8;
-    if (a.store != OT_STORE_BF16) return false;
+    if (a.store != OT_STORE_BF16 && a.store != OT_STORE_E4M3) return false;
+    if (a.store == OT_STORE_E4M3 && (a.res || !a.qscale)) return false;
     if (a.K % (fp8 ? 128 : 64) != 0 || a.a_map.P != 1 || a.N % 128 != 0 || a.M < 1 || a.G < 1)
         return false;
     wide = a.N % 256 == 0;
@@ -624,7 +681,7 @@ cudaError_t launch_gemm_tc_multi(const GemmArgs &a, const GemmArgs *a1, cudaStre
     if (a1) {
         // one launch-wide K and norm, bf16 / fp32 operands
         if (fp8 || !gemm_ok(*a1, wide1) || a1->K != a.K || a1->in_dtype == OT_DTYPE_FP8 ||
-            (a1->norm != 0) != (a.norm != 0))
+            (a1->norm != 0) != (a.norm != 0) || a1->store != a.store)
             return cudaErrorInvalidValue;
     }
     // a single problem whose 128 x 256 tiles would leave SMs idle (the grouped

@@ -66,7 +66,10 @@ __host__ __device__ inline long long paged_row(const EpiSeg &s, long long r)
     return (page * 2 + s.pg_kv) * OT_PAGE_ROWS + t % OT_PAGE_ROWS;
 }
 
-enum { OT_STORE_F32 = 0, OT_STORE_BF16 = 1 };
+// OT_STORE_E4M3: e4m3 of (value / qscale[g * qscale_gstride]), rounded to
+// nearest even and saturating (the per-tensor FP8 scale of the tensor the
+// output feeds, so the next projection reads it without a quantisation pass)
+enum { OT_STORE_F32 = 0, OT_STORE_BF16 = 1, OT_STORE_E4M3 = 2 };
 
 // C[r, c] (group g) = epilogue( sum_k A[row_a(r,g), k] * B[g][c][k] ).
 // Epilogue, in order: * rsqrt(mean_k A^2 + eps) if norm; * row_scale[row_a]
@@ -86,6 +89,10 @@ struct GemmArgs {
     float eps;
     const float *row_scale; // indexed by row_a(r, g)
     const float *g_scale;   // indexed by g
+    const float *xg_scale;  // fp8 A operand with a per-group scale: xg_scale[g * xg_gstride]
+    long long xg_gstride;
+    const float *qscale;    // e4m3 output (OT_STORE_E4M3): its scale per group
+    long long qscale_gstride;
     int gelu;
     const void *res;
     long long res_ld;
