@@ -14,7 +14,10 @@ for given upstream gradients G_s [U, q_last, d] and G_ns [U, C, N, d]:
 autograd is the library step; the restated forward is pinned to the C
 oracle and the gradients to central finite differences of the C oracle.
 
-Dense FFN and the causal mask only.
+Dense FFN; the OneTrans causal mask, or full (non-causal) attention
+(cfg.full_attn, one candidate per user: summary page, limitations paragraph
+— every token of a candidate's sequence sees every other, so the S rows
+depend on the candidate and the two sides run jointly per layer).
 """
 
 from __future__ import annotations
@@ -48,9 +51,40 @@ def _attend(q, k, v, mask, heads):
     return (p @ vh).transpose(0, 1).reshape(Tq, d)
 
 
+def _forward_full(cfg, w, S, ns):
+    """Full attention, one candidate per user: per layer the joint sequence
+    [S rows; NS rows], queries = the S tail and every NS row, keys = every
+    row, all visible."""
+    d, H, N, eps = cfg.d, cfg.heads, cfg.n_ns, cfg.eps
+    assert ns.shape[1] == 1, "full attention runs one candidate per user"
+    s_outs, ns_outs = [], []
+    for u in range(S.shape[0]):
+        x, y = S[u], ns[u, 0]
+        for l in range(cfg.layers):
+            L, q = x.shape[0], cfg.q[l]
+            qkv_s = _rms(x, w["g1_s"][l], eps) @ w["Wqkv_s"][l].T
+            qkv_n = torch.stack([_rms(y[n], w["g1_ns"][l, n], eps) @ w["Wqkv_ns"][l, n].T for n in range(N)])
+            Q = torch.cat([qkv_s[L - q:, :d], qkv_n[:, :d]])
+            K = torch.cat([qkv_s[:, d:2 * d], qkv_n[:, d:2 * d]])
+            V = torch.cat([qkv_s[:, 2 * d:], qkv_n[:, 2 * d:]])
+            a = _attend(Q, K, V, torch.ones(q + N, L + N, dtype=torch.bool), H)
+            h = x[L - q:] + a[:q] @ w["Wo_s"][l].T
+            x = h + _gelu(_rms(h, w["g2_s"][l], eps) @ w["W1_s"][l].T) @ w["W2_s"][l].T
+            rows = []
+            for n in range(N):
+                hn = y[n] + a[q + n] @ w["Wo_ns"][l, n].T
+                rows.append(hn + _gelu(_rms(hn, w["g2_ns"][l, n], eps) @ w["W1_ns"][l, n].T) @ w["W2_ns"][l, n].T)
+            y = torch.stack(rows)
+        s_outs.append(x)
+        ns_outs.append(y[None])
+    return torch.stack(s_outs), torch.stack(ns_outs)
+
+
 def forward(cfg, w, S, ns):
     """S [U, L0, d], ns [U, C, N, d] (fp64 tensors) -> (s_out [U, q_last, d],
     ns_out [U, C, N, d]) with the weights of dict w (fp64 tensors)."""
+    if getattr(cfg, "full_attn", False):
+        return _forward_full(cfg, w, S, ns)
     d, H, N, eps = cfg.d, cfg.heads, cfg.n_ns, cfg.eps
     s_outs, ns_outs = [], []
     for u in range(S.shape[0]):

@@ -752,3 +752,70 @@ def test_backward_oracle_matches_finite_differences():
         fd = (loss(*with_(p_plus)) - loss(*with_(p_minus)))
         an = 2.0 * float((grads[name] * step).sum())
         assert abs(fd - an) <= 2e-5 * max(1.0, abs(an)), (name, fd, an)
+
+
+def _bw_full_case(seed=160):
+    layers, d, H, f, N, L0, q = 2, 8, 2, 12, 3, 7, [5, 3]
+    w = rand_weights(layers, d, f, N, seed=seed, dtype=torch.float64)
+    w = {k: v.float().double() for k, v in w.items()}
+    S, ns = rand_inputs(2, 1, L0, N, d, seed=seed + 1, dtype=torch.float64)
+    S, ns = S.float().double(), ns.float().double()
+    g = torch.Generator().manual_seed(seed + 2)
+    G_s = torch.randn(2, q[-1], d, generator=g, dtype=torch.float64)
+    G_ns = torch.randn(2, 1, N, d, generator=g, dtype=torch.float64)
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    cfg.full_attn = True
+    return cfg, w, S, ns, G_s, G_ns
+
+
+def test_backward_oracle_full_attention_forward_matches_c_oracle():
+    """Full attention: the restated forward equals the C oracle's joint form
+    (its every-key visibility pinned by the brute force) to 1e-12."""
+    from oracle import backward as OB
+    cfg, w, S, ns, _, _ = _bw_full_case()
+    s_t, ns_t = OB.forward(cfg, w, S, ns)
+    s_c, _, ns_c = O.full_forward_joint(cfg, w, S, ns)
+    np.testing.assert_allclose(s_t.detach().numpy(), s_c[:, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(ns_t.detach().numpy(), ns_c, rtol=0, atol=1e-12)
+
+
+def test_backward_oracle_full_attention_matches_finite_differences():
+    """Full attention: every gradient along a random direction against the
+    central difference of the C oracle's joint-form loss."""
+    from oracle import backward as OB
+    cfg, w, S, ns, G_s, G_ns = _bw_full_case()
+    _, grads = OB.gradients(cfg, w, S, ns, G_s, G_ns)
+
+    def loss(w_, S_, ns_):
+        s_c, _, ns_c = O.full_forward_joint(cfg, w_, S_.float(), ns_)
+        return float((s_c[:, 0] * G_s.numpy()).sum() + (ns_c * G_ns.numpy()).sum())
+
+    g = torch.Generator().manual_seed(9)
+    eps = 1e-3
+    for name in ["S", "ns"] + list(OB.W_NAMES):
+        base = {"S": S, "ns": ns}.get(name, w.get(name))
+        v = torch.randn(base.shape, generator=g, dtype=torch.float64)
+        p_plus, p_minus = (base + eps * v).float().double(), (base - eps * v).float().double()
+        step = (p_plus - p_minus).double() / 2
+
+        def with_(p):
+            if name == "S":
+                return w, p, ns
+            if name == "ns":
+                return w, S, p
+            return dict(w, **{name: p}), S, ns
+        fd = loss(*with_(p_plus)) - loss(*with_(p_minus))
+        an = 2.0 * float((grads[name] * step).sum())
+        assert abs(fd - an) <= 2e-5 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_backward_oracle_full_attention_differs_from_causal():
+    """The switch is live: the same inputs give other gradients under the
+    causal mask (S rows then see neither later S rows nor NS rows)."""
+    from oracle import backward as OB
+    cfg, w, S, ns, G_s, G_ns = _bw_full_case()
+    _, g_full = OB.gradients(cfg, w, S, ns, G_s, G_ns)
+    cfg.full_attn = False
+    _, g_causal = OB.gradients(cfg, w, S, ns, G_s, G_ns)
+    assert float((g_full["Wqkv_s"] - g_causal["Wqkv_s"]).abs().max()) > 1e-6
+    assert float((g_full["S"] - g_causal["S"]).abs().max()) > 1e-6
