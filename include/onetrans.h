@@ -388,8 +388,9 @@ int ot_profile_read(ot_model *m, ot_launch_record *out, int max);
 /* ---- Backward pass (training) ----
  * The summary page lists activation checkpointing among the training
  * optimisations on top of the stack (systems paragraph).  ot_full_backward
- * computes, for an fp32 config with the causal mask and dense FFNs, the
- * gradients of
+ * computes, for an fp32 config with dense FFNs and the causal mask or full
+ * attention (full_attn = 1: one candidate per user, C = 1, as the forward),
+ * the gradients of
  *     loss = sum(s_tail * G_s) + sum(ns_out * G_ns)
  * (s_tail, ns_out: the outputs of ot_full_forward; G_s, G_ns: the upstream
  * gradients) with respect to every weight and gain and to S and ns.
@@ -410,9 +411,9 @@ int ot_profile_read(ot_model *m, ot_launch_record *out, int max);
  * give the same bits.  Nothing is allocated; ws >=
  * ot_backward_workspace_bytes(cfg, U, C).  Errors, in this order:
  * OT_ERR_ARG (null pointer, U < 1, C < 0, a bad config field),
- * OT_ERR_DTYPE (not OT_DTYPE_F32), OT_ERR_UNSUPPORTED (full_attn or
- * moe_experts), OT_ERR_SHAPE (the config rules; rows beyond the kernels'
- * 32-bit row counts), OT_ERR_ALIGN, OT_ERR_WORKSPACE_TOO_SMALL,
+ * OT_ERR_DTYPE (not OT_DTYPE_F32), OT_ERR_UNSUPPORTED (moe_experts),
+ * OT_ERR_SHAPE (the config rules; full_attn with C != 1; rows beyond the
+ * kernels' 32-bit row counts), OT_ERR_ALIGN, OT_ERR_WORKSPACE_TOO_SMALL,
  * OT_ERR_CUDA. */
 typedef struct {
     float *Wqkv_s, *Wo_s, *W1_s, *W2_s, *g1_s, *g2_s;

@@ -32,15 +32,16 @@ def _build():
     build()
 
 
-def _case(layers, d, heads, ffn, N, L0, q, U, C, seed):
+def _case(layers, d, heads, ffn, N, L0, q, U, C, seed, full=False):
     w = rand_weights(layers, d, ffn, N, seed=seed)
     S, ns = rand_inputs(U, max(C, 1), L0, N, d, seed=seed + 1)
     ns = ns[:, :C].contiguous()
     g = torch.Generator().manual_seed(seed + 2)
     G_s = torch.randn(U, q[-1], d, generator=g)
     G_ns = torch.randn(U, C, N, d, generator=g)
-    cfg = ot.make_config(layers=layers, d=d, heads=heads, ffn=ffn, n_ns=N, L0=L0, q=q)
+    cfg = ot.make_config(layers=layers, d=d, heads=heads, ffn=ffn, n_ns=N, L0=L0, q=q, full_attn=full)
     ocfg = O.Config(layers, d, heads, ffn, N, L0, list(q), 1e-6)
+    ocfg.full_attn = full
     return cfg, ocfg, w, S, ns, G_s, G_ns
 
 
@@ -100,6 +101,37 @@ def test_backward_parity(name):
     assert max(errs.values()) <= TOL_GRAD, {k: f"{v:.2e}" for k, v in errs.items()}
 
 
+FULL_CASES = {
+    # full attention, one candidate per user: S rows also see the NS keys
+    "hd64_ragged": dict(layers=2, d=128, heads=2, ffn=192, N=4, L0=150, q=[150, 61], U=2, C=1),
+    "hd16_3layers": dict(layers=3, d=64, heads=4, ffn=96, N=3, L0=70, q=[70, 33, 1], U=3, C=1),
+}
+
+
+@pytest.mark.parametrize("name", list(FULL_CASES))
+def test_backward_full_attention_parity(name):
+    cfg, ocfg, w, S, ns, G_s, G_ns = _case(**FULL_CASES[name], seed=800 + len(name), full=True)
+    errs, fwd = _errors(ocfg, w, S, ns, G_s, G_ns, _run(cfg, w, S, ns, G_s, G_ns))
+    assert max(fwd.values()) <= TOL_FWD, fwd
+    assert max(errs.values()) <= TOL_GRAD, {k: f"{v:.2e}" for k, v in errs.items()}
+
+
+def test_backward_full_attention_matches_full_forward():
+    """The backward's recomputed outputs equal what the library's own full
+    forward (ot_full_forward, fp32, full attention) computes, to fp32
+    rounding."""
+    spec = dict(FULL_CASES["hd64_ragged"])
+    cfg, ocfg, w, S, ns, G_s, G_ns = _case(**spec, seed=901, full=True)
+    s_tail, ns_out, _, _, _ = _run(cfg, w, S, ns, G_s, G_ns)
+    from gpu_common import make_model
+    m = make_model(w, layers=spec["layers"], d=spec["d"], heads=spec["heads"], ffn=spec["ffn"],
+                   n_ns=spec["N"], L0=spec["L0"], q=spec["q"], dtype="f32", full_attn=True)
+    s_f, ns_f = m.full_forward(S.cuda(), ns.cuda())
+    m.poll()
+    assert O.rel_l2(s_tail.double().cpu().numpy(), s_f.double().cpu().numpy()) < 1e-5
+    assert O.rel_l2(ns_out.double().cpu().numpy(), ns_f.double().cpu().numpy()) < 1e-5
+
+
 def test_backward_s_only():
     """C = 0: the S side alone; the NS gradients are zero."""
     cfg, ocfg, w, S, ns, G_s, G_ns = _case(layers=2, d=64, heads=2, ffn=128, N=2, L0=90, q=[50, 20],
@@ -134,7 +166,7 @@ def test_backward_rejects():
     bad = ot.make_config(layers=1, d=64, heads=4, ffn=64, n_ns=1, L0=70, q=[70], dtype="bf16")
     with pytest.raises(ot.OtError, match="DTYPE"):
         ot.full_backward(bad, *args)
-    bad = ot.make_config(layers=1, d=64, heads=4, ffn=64, n_ns=1, L0=70, q=[70], full_attn=True)
+    bad = ot.make_config(layers=1, d=64, heads=4, ffn=64, n_ns=1, L0=70, q=[70], moe_experts=2)
     with pytest.raises(ot.OtError, match="UNSUPPORTED"):
         ot.full_backward(bad, *args)
     bad = ot.make_config(layers=1, d=64, heads=4, ffn=64, n_ns=1, L0=70, q=[71])

@@ -1,5 +1,5 @@
 // Backward pass of the block stack: ot_full_backward (fp32 models, the
-// OneTrans causal mask, dense FFNs).  The summary page puts activation
+// OneTrans causal mask or full attention, dense FFNs).  The summary page puts activation
 // checkpointing on top of the stack for training (systems paragraph): a
 // forward pass keeps every layer's input rows only, and the backward
 // recomputes one layer at a time from them, top layer first, before taking
@@ -629,6 +629,8 @@ struct Backward {
         a.ld = 3LL * d, a.q_ustride = Ls[l], a.q_off = Ls[l] - c.q[l];
         a.qkv = a.skv = s.QKV;
         a.dqkv = a.dskv = s.dQKV;
+        a.full = c.full_attn;
+        a.nkv = C ? n.QKV : nullptr, a.n_ustride = static_cast<long long>(C) * N, a.nkn = C * N;
         a.O = s.A, a.dO = s.dA;
         a.stat_m = s.sm, a.stat_l = s.sl, a.stat_D = s.sD;
         a.scale = 1.0f / sqrtf(static_cast<float>(hd));
@@ -642,6 +644,8 @@ struct Backward {
         a.ld = 3LL * d, a.q_ustride = static_cast<long long>(C) * N, a.q_off = 0;
         a.qkv = n.QKV, a.skv = s.QKV;
         a.dqkv = n.dQKV, a.dskv = s.dQKV;
+        a.full = c.full_attn;
+        a.nkv = n.QKV, a.n_ustride = static_cast<long long>(C) * N, a.nkn = C * N;
         a.O = n.A, a.dO = n.dA;
         a.stat_m = n.sm, a.stat_l = n.sl, a.stat_D = n.sD;
         a.scale = 1.0f / sqrtf(static_cast<float>(hd));
@@ -692,10 +696,21 @@ struct Backward {
         const int L = Ls[l], q = c.q[l];
         const long long R = RS(l), Tq = T(l);
         const long long d3 = 3LL * d, fd = static_cast<long long>(f) * d, dd = static_cast<long long>(d) * d;
-        // ---- S side
+        const RowMap nm = nmap();
+        const long long RN_ = RN();
+        const int M = U * C;
+        const long long ln = static_cast<long long>(l) * N;
+        // ---- both sides' QKV first (under full attention the S rows read NS keys)
         const BwRows x1{X[l], kIdentity, R, 1, d};
         k([&] { return bw_rms_fwd(x1, wt(w->g1_s, static_cast<long long>(l) * d), 0, c.eps, s.Z1, s.r1, st); });
         nt(s.Z1, d, kIdentity, wt(w->Wqkv_s, l * d3 * d), 0, s.QKV, d3, kIdentity, static_cast<int>(R), 3 * d, d, 1, 0);
+        if (C) {
+            // NS side: group = NS position, rows of a group = the U * C candidates
+            const BwRows y1{Y[l], nm, M, N, d};
+            k([&] { return bw_rms_fwd(y1, wt(w->g1_ns, ln * d), d, c.eps, n.Z1, n.r1, st); });
+            nt(n.Z1, d, nm, wt(w->Wqkv_ns, ln * d3 * d), d3 * d, n.QKV, d3, nm, M, 3 * d, d, N, 0);
+        }
+        // ---- S side
         const BwAttn sa = attn_s(l);
         k([&] { return bw_attn_fwd(sa, st); });
         if (!dry && err == cudaSuccess)
@@ -712,14 +727,7 @@ struct Backward {
             nt(s.Act, f, kIdentity, wt(w->W2_s, l * fd), 0, s_out, d, kIdentity, static_cast<int>(Tq), d, f, 1, 1);
         }
         if (!C) return;
-        // ---- NS side: group = NS position, rows of a group = the U * C candidates
-        const RowMap nm = nmap();
-        const long long RN_ = RN();
-        const int M = U * C;
-        const long long ln = static_cast<long long>(l) * N;
-        const BwRows y1{Y[l], nm, M, N, d};
-        k([&] { return bw_rms_fwd(y1, wt(w->g1_ns, ln * d), d, c.eps, n.Z1, n.r1, st); });
-        nt(n.Z1, d, nm, wt(w->Wqkv_ns, ln * d3 * d), d3 * d, n.QKV, d3, nm, M, 3 * d, d, N, 0);
+        // ---- NS side
         const BwAttn na = attn_ns(l);
         k([&] { return bw_attn_fwd(na, st); });
         copy(n.H, Y[l], static_cast<size_t>(RN_) * d * 4);
@@ -797,7 +805,7 @@ struct Backward {
             k([&] { return bw_attn_bwd_q(na, st); });
         }
         k([&] { return bw_attn_bwd_kv_s(sa, C ? &na : nullptr, st); });
-        if (C) k([&] { return bw_attn_bwd_kv_ns(na, st); });
+        if (C) k([&] { return bw_attn_bwd_kv_ns(na, c.full_attn ? &sa : nullptr, st); });
         // QKV + first norm; the residual adds dH to the tail rows
         qkv_back(s, X[l], kIdentity, static_cast<int>(R), 1, wt(w->Wqkv_s, l * d3 * d),
                  wt(w->g1_s, static_cast<long long>(l) * d), 0, g->Wqkv_s + l * d3 * d,
@@ -845,7 +853,8 @@ ot_status bw_validate(const ot_config *cfg, int U, int C)
 {
     if (!cfg || U < 1 || C < 0) return OT_ERR_ARG;
     if (cfg->dtype != OT_DTYPE_F32) return OT_ERR_DTYPE;
-    if (cfg->full_attn || cfg->moe_experts) return OT_ERR_UNSUPPORTED;
+    if (cfg->moe_experts) return OT_ERR_UNSUPPORTED;
+    if (cfg->full_attn && C != 1) return OT_ERR_SHAPE; // one candidate per user, as the forward
     const ot_status r = internal_check_config(*cfg);
     if (r != OT_OK) return r;
     if (cfg->d / cfg->heads > 64) return OT_ERR_SHAPE;

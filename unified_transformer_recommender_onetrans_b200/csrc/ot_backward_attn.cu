@@ -15,7 +15,9 @@
 // the layer's S QKV buffer), then, for NS queries, the NS keys of the
 // candidates the block spans (rows of the NS QKV buffer).  Visibility: an S
 // tail row t = L - nq + i sees S keys j <= t; an NS row sees every S key and
-// the NS keys m <= n of its own candidate.
+// the NS keys m <= n of its own candidate.  Full attention (one candidate
+// per user): an S row sees every S key and every NS key of the user, an NS
+// row every NS key of its candidate.
 #include <math.h>
 #include <stdint.h>
 
@@ -55,7 +57,11 @@ __device__ __forceinline__ long long q_row(const BwAttn &a, int u, int i)
 __device__ __forceinline__ KeySpace key_space(const BwAttn &a, int i0, int i1)
 {
     KeySpace ks;
-    if (a.mode == 0) {
+    if (a.mode == 0 && a.full) {
+        ks.nks = a.L;
+        ks.nkn = a.nkn; // every NS key of the user (its one candidate)
+        ks.k_begin = 0;
+    } else if (a.mode == 0) {
         ks.nks = min(a.L, a.L - a.nq + i1); // the last row sees keys 0 .. L - nq + i1 - 1
         ks.nkn = 0;
         ks.k_begin = 0;
@@ -71,23 +77,25 @@ __device__ __forceinline__ KeySpace key_space(const BwAttn &a, int i0, int i1)
 __device__ __forceinline__ const float *key_row(const BwAttn &a, const KeySpace &ks, int u, int j)
 {
     return j < ks.nks ? a.skv + (static_cast<long long>(u) * a.L + j) * a.ld
-                      : a.qkv + (static_cast<long long>(u) * a.q_ustride + ks.k_begin + (j - ks.nks)) * a.ld;
+                      : a.nkv + (static_cast<long long>(u) * a.n_ustride + ks.k_begin + (j - ks.nks)) * a.ld;
 }
 
 __device__ __forceinline__ bool visible(const BwAttn &a, const KeySpace &ks, int i, int j)
 {
-    if (j < ks.nks) return a.mode == 1 || j <= a.L - a.nq + i;
+    if (j < ks.nks) return a.full || a.mode == 1 || j <= a.L - a.nq + i;
+    if (a.mode == 0) return true; // S rows meet NS keys only under full attention
     const int r = ks.k_begin + (j - ks.nks);
-    const int ci = i / a.N;
-    return r >= ci * a.N && r <= i; // same candidate, position m <= n
+    const int c0 = (i / a.N) * a.N;
+    return r >= c0 && (a.full ? r < c0 + a.N : r <= i); // same candidate (and m <= n)
 }
 
 // every (row, key) of rows [i0, i0 + 64) x keys [j0, j0 + 64) visible and
 // every key valid (rows past the problem do not matter to the caller)
 __device__ __forceinline__ bool block_full(const BwAttn &a, const KeySpace &ks, int i0, int j0)
 {
+    if (a.full && a.mode == 0) return j0 + TB <= ks.nks + ks.nkn;
     if (j0 + TB > ks.nks) return false; // reaches NS keys or past the S keys
-    return a.mode == 1 || j0 + TB - 1 <= a.L - a.nq + i0;
+    return a.full || a.mode == 1 || j0 + TB - 1 <= a.L - a.nq + i0;
 }
 
 __device__ __forceinline__ float half_warp_max(float v)
@@ -386,11 +394,11 @@ __global__ void __launch_bounds__(NT) attn_dkv_tiled(BwAttn p0, BwAttn p1, int n
             const BwAttn &P = pi == 0 ? p0 : p1;
             // the query rows that can see a key of [j0, j1)
             int qa, qe;
-            if (kind == 1) {
-                qa = (j0 / P.N) * P.N;
+            if (kind == 1 && P.mode == 1) {
+                qa = (j0 / P.N) * P.N; // the candidates of the keys
                 qe = min(P.nq, ((j1 - 1) / P.N + 1) * P.N);
-            } else if (P.mode == 0) {
-                qa = max(0, j0 - (P.L - P.nq));
+            } else if (kind == 0 && P.mode == 0 && !P.full) {
+                qa = max(0, j0 - (P.L - P.nq)); // tail rows at or after the keys
                 qe = P.nq;
             } else {
                 qa = 0;
@@ -417,7 +425,9 @@ __global__ void __launch_bounds__(NT) attn_dkv_tiled(BwAttn p0, BwAttn p1, int n
                 float s[4][4] = {}, dp[4][4] = {};
                 tile_dot<HD>(KT, ty * 4, QT, tx * 4, s);
                 tile_dot<HD>(VT, ty * 4, dOT, tx * 4, dp);
-                const bool full = kind == 0 && n == TB && (P.mode == 1 || j0 + TB - 1 <= P.L - P.nq + i0);
+                const bool full =
+                    n == TB && (kind == 0 ? (P.mode == 1 || P.full || j0 + TB - 1 <= P.L - P.nq + i0)
+                                          : P.mode == 0); // NS keys of S rows: full attention only
                 const float c2 = P.scale * LOG2E;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -548,12 +558,14 @@ cudaError_t bw_attn_bwd_kv_s(const BwAttn &sq, const BwAttn *nsq, cudaStream_t s
     return cudaErrorInvalidValue;
 }
 
-cudaError_t bw_attn_bwd_kv_ns(const BwAttn &a, cudaStream_t s)
+cudaError_t bw_attn_bwd_kv_ns(const BwAttn &a, const BwAttn *sq, cudaStream_t s)
 {
+    const BwAttn &p1 = sq ? *sq : a;
+    const int n_prob = sq ? 2 : 1;
     switch (a.hd) {
-    case 16: return dkv_launch<16>(a, a, 1, 1, s);
-    case 32: return dkv_launch<32>(a, a, 1, 1, s);
-    case 64: return dkv_launch<64>(a, a, 1, 1, s);
+    case 16: return dkv_launch<16>(a, p1, n_prob, 1, s);
+    case 32: return dkv_launch<32>(a, p1, n_prob, 1, s);
+    case 64: return dkv_launch<64>(a, p1, n_prob, 1, s);
     }
     return cudaErrorInvalidValue;
 }

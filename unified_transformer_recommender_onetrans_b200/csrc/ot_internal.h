@@ -314,17 +314,19 @@ struct BwGemm {
 // One attention problem of a layer over QKV rows [.][3d] (Q | K | V):
 //   mode 0 (S queries): query i of user u is S row t = L - nq + i of the
 //     layer, buffer row u * q_ustride + q_off + i of qkv (= skv); it sees S
-//     keys 0..t.
+//     keys 0..t (full: all L S keys and the user's nkn NS keys).
 //   mode 1 (NS queries): query i = c * N + n of user u is row
 //     u * q_ustride + i of qkv; it sees the user's L S keys (rows u * L + j
-//     of skv) and NS keys c * N + m, m <= n (rows of qkv).
+//     of skv) and NS keys c * N + m, m <= n (full: every m of candidate c).
+// NS keys of user u are rows u * n_ustride + r of nkv (mode 1: nkv = qkv).
 // O / dO are [U * nq][d]; stat_* [U * nq][H] (m: the row's max score in
 // base-2 units, s * scale * log2(e); l: the sum of 2^(s' - m); D: dO . O);
 // dqkv / dskv take dQ and dK, dV in the layout of qkv / skv.
 struct BwAttn {
     int mode, U, H, hd, d, L, nq, N;
-    long long ld, q_ustride, q_off;
-    const float *qkv, *skv;
+    int full, nkn;      // full attention; NS key rows per user
+    long long ld, q_ustride, q_off, n_ustride;
+    const float *qkv, *skv, *nkv;
     float *dqkv, *dskv;
     float *O;
     const float *dO;
@@ -349,7 +351,9 @@ long long bw_tn_partial_floats(int M, int N, int K, int G);
 cudaError_t bw_attn_fwd(const BwAttn &a, cudaStream_t s);
 cudaError_t bw_attn_bwd_q(const BwAttn &a, cudaStream_t s);
 cudaError_t bw_attn_bwd_kv_s(const BwAttn &sq, const BwAttn *nsq, cudaStream_t s);
-cudaError_t bw_attn_bwd_kv_ns(const BwAttn &a, cudaStream_t s);
+// NS keys: the NS queries of problem a and, if sq (full attention), the S
+// queries of sq
+cudaError_t bw_attn_bwd_kv_ns(const BwAttn &a, const BwAttn *sq, cudaStream_t s);
 
 // Shape / dtype check of a config (the rules of ot_model_create).
 ot_status internal_check_config(const ot_config &c);
