@@ -14,7 +14,11 @@ for given upstream gradients G_s [U, q_last, d] and G_ns [U, C, N, d]:
 autograd is the library step; the restated forward is pinned to the C
 oracle and the gradients to central finite differences of the C oracle.
 
-Dense FFN; the OneTrans causal mask, or full (non-causal) attention
+The S-side FFN dense or a sparse mixture of experts (cfg.moe_experts = E,
+top cfg.moe_topk: the router reads the FFN's normalised input, the k largest
+logits (ties to the lower expert index) are softmax-ed into gates, y = h +
+sum_j g_j FFN_e(j)(z); the selection itself carries no gradient); the
+OneTrans causal mask, or full (non-causal) attention
 (cfg.full_attn, one candidate per user: summary page, limitations paragraph
 — every token of a candidate's sequence sees every other, so the S rows
 depend on the candidate and the two sides run jointly per layer).
@@ -28,6 +32,13 @@ import torch
 
 W_NAMES = ("Wqkv_s", "Wo_s", "W1_s", "W2_s", "g1_s", "g2_s",
            "Wqkv_ns", "Wo_ns", "W1_ns", "W2_ns", "g1_ns", "g2_ns")
+MOE_NAMES = ("W_router", "W1_moe", "W2_moe")
+
+
+def names(cfg):
+    """The tensors a config differentiates (a mixture adds its router and
+    experts; the dense S-side W1_s / W2_s then get zero gradients)."""
+    return W_NAMES + (MOE_NAMES if getattr(cfg, "moe_experts", 0) else ())
 
 
 def _rms(x, g, eps):
@@ -51,6 +62,26 @@ def _attend(q, k, v, mask, heads):
     return (p @ vh).transpose(0, 1).reshape(Tq, d)
 
 
+def _s_ffn(cfg, w, l, h):
+    """The S-side FFN of layer l on rows h [q, d], residual included."""
+    z = _rms(h, w["g2_s"][l], cfg.eps)
+    E = getattr(cfg, "moe_experts", 0)
+    if not E:
+        return h + _gelu(z @ w["W1_s"][l].T) @ w["W2_s"][l].T
+    k = cfg.moe_topk
+    logits = z @ w["W_router"][l].T                                   # [q, E]
+    # top-k by a stable sort of the negated logits: equal logits keep the
+    # lower expert index first
+    sel = torch.sort(-logits.detach(), dim=-1, stable=True).indices[:, :k]
+    gates = torch.softmax(torch.gather(logits, 1, sel), dim=-1)       # [q, k]
+    ys = torch.stack([_gelu(z @ w["W1_moe"][l, e].T) @ w["W2_moe"][l, e].T for e in range(E)])  # [E, q, d]
+    rows = torch.arange(h.shape[0])
+    out = h
+    for j in range(k):
+        out = out + gates[:, j:j + 1] * ys[sel[:, j], rows]
+    return out
+
+
 def _forward_full(cfg, w, S, ns):
     """Full attention, one candidate per user: per layer the joint sequence
     [S rows; NS rows], queries = the S tail and every NS row, keys = every
@@ -69,7 +100,7 @@ def _forward_full(cfg, w, S, ns):
             V = torch.cat([qkv_s[:, 2 * d:], qkv_n[:, 2 * d:]])
             a = _attend(Q, K, V, torch.ones(q + N, L + N, dtype=torch.bool), H)
             h = x[L - q:] + a[:q] @ w["Wo_s"][l].T
-            x = h + _gelu(_rms(h, w["g2_s"][l], eps) @ w["W1_s"][l].T) @ w["W2_s"][l].T
+            x = _s_ffn(cfg, w, l, h)
             rows = []
             for n in range(N):
                 hn = y[n] + a[q + n] @ w["Wo_ns"][l, n].T
@@ -100,8 +131,7 @@ def forward(cfg, w, S, ns):
             mask = torch.arange(L).unsqueeze(0) <= t            # S row t sees S keys 0..t
             a = _attend(Q, K, V, mask, H)
             h = x[L - q:] + a @ w["Wo_s"][l].T
-            f = _gelu(_rms(h, w["g2_s"][l], eps) @ w["W1_s"][l].T) @ w["W2_s"][l].T
-            x = h + f
+            x = _s_ffn(cfg, w, l, h)
         s_outs.append(x)
         cand = []
         for c in range(ns.shape[1]):
@@ -131,12 +161,12 @@ def forward(cfg, w, S, ns):
 def gradients(cfg, w, S, ns, G_s, G_ns):
     """(loss, grads): grads maps "S", "ns" and every weight name to the
     gradient of sum(s_out * G_s) + sum(ns_out * G_ns), fp64 CPU tensors."""
-    wt = {k: torch.as_tensor(w[k]).detach().double().clone().requires_grad_(True) for k in W_NAMES}
+    wt = {k: torch.as_tensor(w[k]).detach().double().clone().requires_grad_(True) for k in names(cfg)}
     St = torch.as_tensor(S).detach().double().clone().requires_grad_(True)
     nst = torch.as_tensor(ns).detach().double().clone().requires_grad_(True)
     s_out, ns_out = forward(cfg, wt, St, nst)
     loss = (s_out * torch.as_tensor(G_s).double()).sum() + (ns_out * torch.as_tensor(G_ns).double()).sum()
     loss.backward()
     grads = {"S": St.grad, "ns": nst.grad}
-    grads.update({k: wt[k].grad for k in W_NAMES})
+    grads.update({k: wt[k].grad if wt[k].grad is not None else torch.zeros_like(wt[k]) for k in names(cfg)})
     return float(loss.detach()), grads

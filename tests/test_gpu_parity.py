@@ -672,6 +672,35 @@ def test_paged_cache_matches_dense_cache(shape):
             assert torch.equal(K, Kd) and torch.equal(V, Vd), (u, l)
 
 
+def test_paged_cache_fp8_per_tensor_matches_dense_cache():
+    """FP8 with per-tensor activation scales (the e4m3 hidden written by the
+    first FFN projection) through the paged calls: bit for bit the dense
+    cache's S tails, NS outputs and K / V."""
+    shapes = dict(layers=3, d=128, heads=2, ffn=256, n_ns=5, L0=300, q=[300, 170, 37])
+    w = rand_weights(3, 128, 256, 5, seed=137, dtype=torch.bfloat16)
+    S, ns = rand_inputs(3, 6, 300, 5, 128, seed=138, dtype=torch.bfloat16)
+    m = make_model(w, dtype="fp8", **shapes)
+    m.set_wait_limit(TEST_WAIT)
+    scales, _ = O.calibrate(oracle_cfg(m), w, S[:1], ns[:1])
+    m.set_act_scales(scales)
+    Sd, nsd = S.cuda(), ns.cuda()
+    kv, s_dense = m.encode_user(Sd)
+    out_dense = m.score_candidates(kv, nsd)
+    n_pages = 3 * m.kv_pages_per_user() + 5
+    pool = m.new_page_pool(n_pages)
+    pool.fill_(float("nan"))
+    pages = _page_table(m, 3, n_pages, seed=139)
+    s_paged = m.encode_user_paged(Sd, pool, pages)
+    out_paged = m.score_candidates_paged(pool, pages, nsd)
+    m.poll()
+    assert torch.equal(s_paged, s_dense) and torch.equal(out_paged, out_dense)
+    for u in range(3):
+        for l in range(m.layers):
+            K, V = m.kv_from_pages(pool, pages[u].cpu(), l)
+            Kd, Vd = m.kv_layer(kv[u], l)
+            assert torch.equal(K, Kd) and torch.equal(V, Vd), (u, l)
+
+
 def test_paged_cache_shared_prefix_pages():
     """Users with identical S rows list the same pages (a shared prefix
     covering the whole sequence): their results equal each other and the

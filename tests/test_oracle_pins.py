@@ -819,3 +819,87 @@ def test_backward_oracle_full_attention_differs_from_causal():
     _, g_causal = OB.gradients(cfg, w, S, ns, G_s, G_ns)
     assert float((g_full["Wqkv_s"] - g_causal["Wqkv_s"]).abs().max()) > 1e-6
     assert float((g_full["S"] - g_causal["S"]).abs().max()) > 1e-6
+
+
+def _bw_moe_case(topk, seed=170):
+    layers, d, H, f, N, L0, q = 2, 8, 2, 12, 2, 9, [6, 3]
+    w = rand_weights(layers, d, f, N, seed=seed, dtype=torch.float64, experts=3)
+    w = {k: v.float().double() for k, v in w.items()}
+    S, ns = rand_inputs(2, 2, L0, N, d, seed=seed + 1, dtype=torch.float64)
+    S, ns = S.float().double(), ns.float().double()
+    g = torch.Generator().manual_seed(seed + 2)
+    G_s = torch.randn(2, q[-1], d, generator=g, dtype=torch.float64)
+    G_ns = torch.randn(2, 2, N, d, generator=g, dtype=torch.float64)
+    cfg = cfg_of(layers, d, H, f, N, L0, q)
+    cfg.moe_experts, cfg.moe_topk = 3, topk
+    return cfg, w, S, ns, G_s, G_ns
+
+
+def _moe_margins(cfg, w, S, ns, monkeypatch):
+    """Smallest gap, over every S row of every layer, between the k-th and
+    the (k+1)-th router logit: the room a perturbation has before the
+    selection changes."""
+    from oracle import backward as OB
+    seen = []
+    orig = OB._s_ffn
+
+    def spy(cfg_, w_, l, h):
+        seen.append((l, h.detach()))
+        return orig(cfg_, w_, l, h)
+    monkeypatch.setattr(OB, "_s_ffn", spy)
+    OB.forward(cfg, {k: torch.as_tensor(v) for k, v in w.items()}, S, ns)
+    gaps = []
+    for l, h in seen:
+        z = OB._rms(h, w["g2_s"][l], cfg.eps)
+        lg = torch.sort(z @ w["W_router"][l].T, dim=-1, descending=True).values
+        gaps.append(float((lg[:, cfg.moe_topk - 1] - lg[:, cfg.moe_topk]).min()))
+    return min(gaps)
+
+
+@pytest.mark.parametrize("topk", [1, 2])
+def test_backward_oracle_moe_forward_matches_c_oracle(topk):
+    """The restated mixture (stable-sort top-k, softmax gates over the chosen
+    logits) equals the C oracle's (pinned by the brute force) to 1e-12."""
+    from oracle import backward as OB
+    cfg, w, S, ns, _, _ = _bw_moe_case(topk)
+    s_t, ns_t = OB.forward(cfg, w, S, ns)
+    kv, s_c = O.encode_user(cfg, w, S)
+    ns_c = O.score_candidates(cfg, w, kv, ns)
+    np.testing.assert_allclose(s_t.detach().numpy(), s_c, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(ns_t.detach().numpy(), ns_c, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("topk", [1, 2])
+def test_backward_oracle_moe_matches_finite_differences(topk, monkeypatch):
+    """Gradients of a mixture (router, experts, every other tensor) against
+    central differences of the C oracle's loss; the routing margins are
+    checked to be far above what the perturbations can move a logit by, so
+    no selection changes between the two evaluations."""
+    from oracle import backward as OB
+    cfg, w, S, ns, G_s, G_ns = _bw_moe_case(topk)
+    assert _moe_margins(cfg, w, S, ns, monkeypatch) > 2e-2
+    _, grads = OB.gradients(cfg, w, S, ns, G_s, G_ns)
+    assert float(grads["W1_s"].abs().max()) == 0.0  # the dense S FFN is unused
+
+    def loss(w_, S_, ns_):
+        kv, s_c = O.encode_user(cfg, w_, S_.float())
+        return float((s_c * G_s.numpy()).sum() +
+                     (O.score_candidates(cfg, w_, kv, ns_) * G_ns.numpy()).sum())
+
+    g = torch.Generator().manual_seed(11)
+    eps = 1e-4
+    for name in ["S", "ns"] + list(OB.names(cfg)):
+        base = {"S": S, "ns": ns}.get(name, w.get(name))
+        v = torch.randn(base.shape, generator=g, dtype=torch.float64)
+        p_plus, p_minus = (base + eps * v).float().double(), (base - eps * v).float().double()
+        step = (p_plus - p_minus).double() / 2
+
+        def with_(p):
+            if name == "S":
+                return w, p, ns
+            if name == "ns":
+                return w, S, p
+            return dict(w, **{name: p}), S, ns
+        fd = loss(*with_(p_plus)) - loss(*with_(p_minus))
+        an = 2.0 * float((grads[name] * step).sum())
+        assert abs(fd - an) <= 2e-5 * max(1.0, abs(an)) + 1e-9, (name, fd, an)
