@@ -388,9 +388,10 @@ int ot_profile_read(ot_model *m, ot_launch_record *out, int max);
 /* ---- Backward pass (training) ----
  * The summary page lists activation checkpointing among the training
  * optimisations on top of the stack (systems paragraph).  ot_full_backward
- * computes, for an fp32 config with dense FFNs and the causal mask or full
- * attention (full_attn = 1: one candidate per user, C = 1, as the forward),
- * the gradients of
+ * computes, for an fp32 config with the causal mask or full attention
+ * (full_attn = 1: one candidate per user, C = 1, as the forward) and a dense
+ * or mixture-of-experts S-side FFN (moe_experts = E: gradients of the router
+ * and the experts; the selection carries none), the gradients of
  *     loss = sum(s_tail * G_s) + sum(ns_out * G_ns)
  * (s_tail, ns_out: the outputs of ot_full_forward; G_s, G_ns: the upstream
  * gradients) with respect to every weight and gain and to S and ns.
@@ -398,26 +399,29 @@ int ot_profile_read(ot_model *m, ot_launch_record *out, int max);
  * rows; the backward then recomputes one layer at a time from them, top
  * layer first, and takes its gradients.  CUDA-core fp32 kernels.
  * All pointers are device pointers to fp32, 16-byte aligned:
- *   w      the twelve dense tensors of ot_weights (Wqkv_s .. g2_ns), fp32,
- *          gains NOT folded (W_split and the MoE fields are not read);
+ *   w      the tensors of ot_weights, fp32, gains NOT folded: Wqkv_s ..
+ *          g2_ns, and with E > 0 W_router, W1_moe, W2_moe (then W1_s / W2_s
+ *          are not read and may be NULL); W_split is not read;
  *   S [U][L0][d], ns [U][C][N][d], G_s [U][q_last][d], G_ns [U][C][N][d];
  *   out_s_tail [U][q_last][d], out_ns [U][C][N][d]: the forward's outputs
  *          (NULL: not written);
- *   g      gradients in the weights' shapes, all twelve non-NULL,
- *          overwritten (not accumulated);
+ *   g      gradients in the weights' shapes, overwritten (not
+ *          accumulated): the twelve dense ones non-NULL (W1_s / W2_s may be
+ *          NULL with E > 0, else they are zeroed), the three MoE ones
+ *          non-NULL with E > 0 (not read otherwise);
  *   dS [U][L0][d], dns [U][C][N][d] (NULL: not written).
  * C = 0 runs the S side alone (ns, G_ns, out_ns and dns are not read or
  * written; the NS gradients are set to zero).  No atomics: the same inputs
  * give the same bits.  Nothing is allocated; ws >=
  * ot_backward_workspace_bytes(cfg, U, C).  Errors, in this order:
  * OT_ERR_ARG (null pointer, U < 1, C < 0, a bad config field),
- * OT_ERR_DTYPE (not OT_DTYPE_F32), OT_ERR_UNSUPPORTED (moe_experts),
- * OT_ERR_SHAPE (the config rules; full_attn with C != 1; rows beyond the
- * kernels' 32-bit row counts), OT_ERR_ALIGN, OT_ERR_WORKSPACE_TOO_SMALL,
- * OT_ERR_CUDA. */
+ * OT_ERR_DTYPE (not OT_DTYPE_F32), OT_ERR_SHAPE (the config rules;
+ * full_attn with C != 1; rows beyond the kernels' 32-bit row counts),
+ * OT_ERR_ALIGN, OT_ERR_WORKSPACE_TOO_SMALL, OT_ERR_CUDA. */
 typedef struct {
     float *Wqkv_s, *Wo_s, *W1_s, *W2_s, *g1_s, *g2_s;
     float *Wqkv_ns, *Wo_ns, *W1_ns, *W2_ns, *g1_ns, *g2_ns;
+    float *W_router, *W1_moe, *W2_moe; /* mixture of experts only */
 } ot_grads;
 
 size_t ot_backward_workspace_bytes(const ot_config *cfg, int U, int C);

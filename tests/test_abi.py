@@ -142,7 +142,7 @@ def test_backward_host_checks(lib):
     assert lib.ot_full_backward(*_bw_args(_cfg(**dict(f32, dtype=1)))) == 3          # bf16
     assert lib.ot_full_backward(*_bw_args(_cfg(**dict(f32, full_attn=1)))) == 2     # full: C must be 1
     assert lib_bw_bytes(_cfg(**dict(f32, full_attn=1)), 2, 1) > 0
-    assert lib.ot_full_backward(*_bw_args(_cfg(**dict(f32, moe_experts=4, moe_topk=1)))) == 10
+    assert lib.ot_full_backward(*_bw_args(_cfg(**dict(f32, moe_experts=4, moe_topk=1)))) == 1   # no MoE tensors
     assert lib.ot_full_backward(*_bw_args(_cfg(**dict(f32, q=[41, 10])))) == 2
     assert lib.ot_full_backward(*_bw_args(cfg, misalign="W1_ns")) == 4
     assert lib.ot_full_backward(*_bw_args(cfg, ws_bytes=ws - 1)) == 6

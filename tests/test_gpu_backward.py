@@ -32,21 +32,23 @@ def _build():
     build()
 
 
-def _case(layers, d, heads, ffn, N, L0, q, U, C, seed, full=False):
-    w = rand_weights(layers, d, ffn, N, seed=seed)
+def _case(layers, d, heads, ffn, N, L0, q, U, C, seed, full=False, experts=0, topk=1):
+    w = rand_weights(layers, d, ffn, N, seed=seed, experts=experts)
     S, ns = rand_inputs(U, max(C, 1), L0, N, d, seed=seed + 1)
     ns = ns[:, :C].contiguous()
     g = torch.Generator().manual_seed(seed + 2)
     G_s = torch.randn(U, q[-1], d, generator=g)
     G_ns = torch.randn(U, C, N, d, generator=g)
-    cfg = ot.make_config(layers=layers, d=d, heads=heads, ffn=ffn, n_ns=N, L0=L0, q=q, full_attn=full)
+    cfg = ot.make_config(layers=layers, d=d, heads=heads, ffn=ffn, n_ns=N, L0=L0, q=q, full_attn=full,
+                         moe_experts=experts, moe_topk=topk)
     ocfg = O.Config(layers, d, heads, ffn, N, L0, list(q), 1e-6)
     ocfg.full_attn = full
+    ocfg.moe_experts, ocfg.moe_topk = experts, topk
     return cfg, ocfg, w, S, ns, G_s, G_ns
 
 
 def _run(cfg, w, S, ns, G_s, G_ns):
-    dw = {k: w[k].cuda() for k in ot.GRAD_NAMES}
+    dw = {k: v.cuda() for k, v in w.items()}
     C = ns.shape[1]
     out = ot.full_backward(cfg, dw, S.cuda(), ns.cuda() if C else None, G_s.cuda(),
                            G_ns.cuda() if C else None)
@@ -57,7 +59,7 @@ def _run(cfg, w, S, ns, G_s, G_ns):
 def _errors(ocfg, w, S, ns, G_s, G_ns, out):
     s_tail, ns_out, grads, dS, dns = out
     C = ns.shape[1]
-    w64 = {k: w[k].double() for k in OB.W_NAMES}
+    w64 = {k: w[k].double() for k in OB.names(ocfg)}
     if C:
         ns_o_in, G_ns_o = ns.double(), G_ns.double()
     else:
@@ -66,8 +68,12 @@ def _errors(ocfg, w, S, ns, G_s, G_ns, out):
         ns_o_in = torch.randn(S.shape[0], 1, ocfg.n_ns, ocfg.d, dtype=torch.float64)
         G_ns_o = torch.zeros_like(ns_o_in)
     _, want = OB.gradients(ocfg, w64, S.double(), ns_o_in, G_s.double(), G_ns_o)
+    moe = getattr(ocfg, "moe_experts", 0)
     errs = {k: O.rel_l2(grads[k].double().cpu().numpy(), want[k].numpy())
-            for k in OB.W_NAMES if C or not k.endswith("_ns")}
+            for k in OB.names(ocfg) if (C or not k.endswith("_ns")) and not (moe and k in ("W1_s", "W2_s"))}
+    if moe:
+        for k in ("W1_s", "W2_s"):
+            assert torch.count_nonzero(grads[k]) == 0, k
     errs["S"] = O.rel_l2(dS.double().cpu().numpy(), want["S"].numpy())
     fwd = {}
     s_o, ns_o = OB.forward(ocfg, w64, S.double(), ns_o_in)
@@ -132,6 +138,52 @@ def test_backward_full_attention_matches_full_forward():
     assert O.rel_l2(ns_out.double().cpu().numpy(), ns_f.double().cpu().numpy()) < 1e-5
 
 
+def _moe_decisive(w, experts, layers, d, scale=4.0):
+    """Router weights that read a few coordinates strongly, so the logit gaps
+    between experts are far above fp32 rounding (the GPU routes in fp32, the
+    oracle in fp64: the same choices need clear margins)."""
+    g = torch.Generator().manual_seed(1234)
+    wr = torch.zeros(layers, experts, d)
+    for l in range(layers):
+        for e in range(experts):
+            wr[l, e, (7 * e + l) % d] = scale * (1.0 + 0.37 * e)
+            wr[l, e] += 0.05 * torch.randn(d, generator=g)
+    w["W_router"] = wr
+    return w
+
+
+MOE_CASES = {
+    "top1_e3": dict(layers=2, d=64, heads=2, ffn=96, N=3, L0=90, q=[90, 41], U=2, C=2, experts=3, topk=1),
+    "top2_e4": dict(layers=2, d=128, heads=2, ffn=192, N=2, L0=150, q=[150, 61], U=2, C=2, experts=4, topk=2),
+}
+
+
+@pytest.mark.parametrize("name", list(MOE_CASES))
+def test_backward_moe_parity(name, monkeypatch):
+    """A mixture-of-experts S-side FFN: gradients of the router, the
+    experts and every other tensor against the oracle (the routing margins
+    are checked to be clear of fp32 rounding first)."""
+    spec = MOE_CASES[name]
+    cfg, ocfg, w, S, ns, G_s, G_ns = _case(**spec, seed=950 + len(name))
+    w = _moe_decisive(w, spec["experts"], spec["layers"], spec["d"])
+    seen = []
+    orig = OB._s_ffn
+
+    def spy(c_, w_, l, h):
+        seen.append((l, h.detach()))
+        return orig(c_, w_, l, h)
+    monkeypatch.setattr(OB, "_s_ffn", spy)
+    OB.forward(ocfg, {k: v.double() for k, v in w.items()}, S.double(), ns.double())
+    monkeypatch.setattr(OB, "_s_ffn", orig)
+    for l, h in seen:
+        z = OB._rms(h, w["g2_s"][l].double(), 1e-6)
+        lg = torch.sort(z @ w["W_router"][l].double().T, dim=-1, descending=True).values
+        assert float((lg[:, spec["topk"] - 1] - lg[:, spec["topk"]]).min()) > 1e-3
+    errs, fwd = _errors(ocfg, w, S, ns, G_s, G_ns, _run(cfg, w, S, ns, G_s, G_ns))
+    assert max(fwd.values()) <= TOL_FWD, fwd
+    assert max(errs.values()) <= TOL_GRAD, {k: f"{v:.2e}" for k, v in errs.items()}
+
+
 def test_backward_s_only():
     """C = 0: the S side alone; the NS gradients are zero."""
     cfg, ocfg, w, S, ns, G_s, G_ns = _case(layers=2, d=64, heads=2, ffn=128, N=2, L0=90, q=[50, 20],
@@ -167,7 +219,7 @@ def test_backward_rejects():
     with pytest.raises(ot.OtError, match="DTYPE"):
         ot.full_backward(bad, *args)
     bad = ot.make_config(layers=1, d=64, heads=4, ffn=64, n_ns=1, L0=70, q=[70], moe_experts=2)
-    with pytest.raises(ot.OtError, match="UNSUPPORTED"):
+    with pytest.raises(ot.OtError, match="ARG"):  # a mixture without its router and experts
         ot.full_backward(bad, *args)
     bad = ot.make_config(layers=1, d=64, heads=4, ffn=64, n_ns=1, L0=70, q=[71])
     with pytest.raises(ot.OtError, match="SHAPE"):

@@ -47,7 +47,7 @@ GRAD_NAMES = WEIGHT_NAMES[:12]
 
 
 class OtGrads(C.Structure):
-    _fields_ = [(n, C.c_void_p) for n in GRAD_NAMES]
+    _fields_ = [(n, C.c_void_p) for n in GRAD_NAMES + MOE_WEIGHT_NAMES]
 
 
 class OtLaunchRecord(C.Structure):
@@ -489,14 +489,16 @@ def full_backward(cfg: OtConfig, weights: dict, S, ns, G_s, G_ns, *, grads=None,
                   dns=None, out_s_tail=None, out_ns=None, ws=None, want_outputs=True,
                   want_input_grads=True, stream=None):
     """ot_full_backward on fp32 CUDA tensors.  ``weights``: the twelve dense
-    tensors of GRAD_NAMES (gains not folded).  Returns (s_tail, ns_out,
-    grads, dS, dns); the gradients are those of sum(s_tail * G_s) +
-    sum(ns_out * G_ns)."""
+    tensors of GRAD_NAMES (gains not folded) and, for a mixture of experts,
+    those of MOE_WEIGHT_NAMES (W1_s / W2_s may then be absent).  Returns
+    (s_tail, ns_out, grads, dS, dns); the gradients are those of
+    sum(s_tail * G_s) + sum(ns_out * G_ns)."""
     import torch
     U, Cn = S.shape[0], (ns.shape[1] if ns is not None else 0)
     dev = S.device
+    present = [k for k in GRAD_NAMES + MOE_WEIGHT_NAMES if weights.get(k) is not None]
     if grads is None:
-        grads = {k: torch.empty_like(weights[k]) for k in GRAD_NAMES}
+        grads = {k: torch.empty_like(weights[k]) for k in present}
     if want_outputs:
         if out_s_tail is None:
             out_s_tail = torch.empty(U, cfg.q[cfg.layers - 1], cfg.d, dtype=torch.float32, device=dev)
@@ -510,8 +512,8 @@ def full_backward(cfg: OtConfig, weights: dict, S, ns, G_s, G_ns, *, grads=None,
     nbytes = backward_workspace_bytes(cfg, U, Cn)
     if ws is None:
         ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
-    w = OtWeights(**{k: _ptr(weights[k]) for k in GRAD_NAMES})
-    g = OtGrads(**{k: _ptr(grads[k]) for k in GRAD_NAMES})
+    w = OtWeights(**{k: _ptr(weights.get(k)) for k in GRAD_NAMES + MOE_WEIGHT_NAMES})
+    g = OtGrads(**{k: _ptr(grads.get(k)) for k in GRAD_NAMES + MOE_WEIGHT_NAMES})
     check(lib().ot_full_backward(C.byref(cfg), C.byref(w), _ptr(S), _ptr(ns) if Cn else 0, U, Cn,
                                  _ptr(G_s), _ptr(G_ns) if Cn else 0, _ptr(out_s_tail),
                                  _ptr(out_ns) if Cn else 0, C.byref(g), _ptr(dS),

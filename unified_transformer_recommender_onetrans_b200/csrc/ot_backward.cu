@@ -40,6 +40,19 @@ __device__ __forceinline__ long long bw_row(const RowMap &m, long long r, long l
     return m.P == 1 ? r * m.A + m.B + g * m.Gs : rowmap_apply(m, r, g);
 }
 
+// row r of group g of a GEMM operand: its segment when the GEMM has
+// segments, else the row map
+__device__ __forceinline__ long long bw_grow(const BwGemm &p, const RowMap &m, long long r, int g)
+{
+    return p.g_off ? static_cast<long long>(p.g_off[g]) + r : bw_row(m, r, g);
+}
+
+// rows of group g (M for NT / NN, K for TN)
+__device__ __forceinline__ int bw_grows(const BwGemm &p, int g, int all)
+{
+    return p.g_cnt ? min(all, p.g_cnt[g]) : all;
+}
+
 __device__ __forceinline__ long long bw_warp_id()
 {
     return (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
@@ -170,12 +183,13 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
     const int g = FORM == BW_TN ? static_cast<int>(blockIdx.z) / p.splits : static_cast<int>(blockIdx.z);
     const int split = FORM == BW_TN ? static_cast<int>(blockIdx.z) % p.splits : 0;
     const int m0 = blockIdx.y * GB_M, n0 = blockIdx.x * GB_N;
+    const int Mg = FORM == BW_TN ? p.M : bw_grows(p, g, p.M); // output rows of this group
     // reduction range of this CTA (TN: one of `splits` chunks, GB_K aligned)
-    int k_lo = 0, k_hi = p.K;
+    int k_lo = 0, k_hi = FORM == BW_TN ? bw_grows(p, g, p.K) : p.K;
     if (FORM == BW_TN && p.splits > 1) {
         const int chunk = ((p.K + p.splits - 1) / p.splits + GB_K - 1) / GB_K * GB_K;
-        k_lo = min(p.K, split * chunk);
-        k_hi = min(p.K, k_lo + chunk);
+        k_lo = min(k_hi, split * chunk);
+        k_hi = min(k_hi, k_lo + chunk);
     }
     const int tm = (tid >> 4) * 4, tn = (tid & 15) * 4;
     // rows of A (NT, NN) and of B (NT) this thread stages: fixed for the kernel
@@ -185,7 +199,7 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int m = m0 + (tid >> 4) + 16 * j;
-            if (m < p.M) arow[j] = p.A + bw_row(p.a_map, m, g) * p.lda;
+            if (m < Mg) arow[j] = p.A + bw_grow(p, p.a_map, m, g) * p.lda;
         }
     }
     if (FORM == BW_NT) {
@@ -211,7 +225,7 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int kk = (tid >> 6) + 4 * j, k = k0 + kk;
-                As[kk][mm] = (k < k_hi && m < p.M) ? p.A[bw_row(p.a_map, k, g) * p.lda + m] : 0.f;
+                As[kk][mm] = (k < k_hi && m < p.M) ? p.A[bw_grow(p, p.a_map, k, g) * p.lda + m] : 0.f;
             }
         }
         if (FORM == BW_NT) {
@@ -225,7 +239,7 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
                 const int kk = (tid >> 6) + 4 * j, k = k0 + kk;
                 float v = 0.f;
                 if (k < k_hi && n < p.N) {
-                    const long long row = FORM == BW_NN ? static_cast<long long>(k) : bw_row(p.b_map, k, g);
+                    const long long row = FORM == BW_NN ? static_cast<long long>(k) : bw_grow(p, p.b_map, k, g);
                     v = p.B[(FORM == BW_NN ? g * p.b_gstride : 0) + row * p.ldb + n];
                 }
                 Bs[kk][nn] = v;
@@ -247,14 +261,14 @@ __global__ void __launch_bounds__(GB_T) bw_gemm_kernel(BwGemm p)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int m = m0 + tm + i;
-        if (m >= p.M) continue;
+        if (m >= Mg) continue;
         float *crow;
         if (FORM == BW_TN && p.splits > 1)
             crow = p.partial + ((static_cast<long long>(split) * p.G + g) * p.M + m) * p.N;
         else if (FORM == BW_TN)
             crow = p.C + g * p.c_gstride + static_cast<long long>(m) * p.ldc;
         else
-            crow = p.C + bw_row(p.c_map, m, g) * p.ldc;
+            crow = p.C + bw_grow(p, p.c_map, m, g) * p.ldc;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int n = n0 + tn + j;
@@ -279,18 +293,19 @@ __global__ void __launch_bounds__(GB_T, 2) bw_gemm_big_kernel(BwGemm p)
     const int g = FORM == BW_TN ? static_cast<int>(blockIdx.z) / p.splits : static_cast<int>(blockIdx.z);
     const int split = FORM == BW_TN ? static_cast<int>(blockIdx.z) % p.splits : 0;
     const int m0 = blockIdx.y * GL_M, n0 = blockIdx.x * GL_N;
-    int k_lo = 0, k_hi = p.K;
+    const int Mg = FORM == BW_TN ? p.M : bw_grows(p, g, p.M);
+    int k_lo = 0, k_hi = FORM == BW_TN ? bw_grows(p, g, p.K) : p.K;
     if (FORM == BW_TN && p.splits > 1) {
         const int chunk = ((p.K + p.splits - 1) / p.splits + GL_K - 1) / GL_K * GL_K;
-        k_lo = min(p.K, split * chunk);
-        k_hi = min(p.K, k_lo + chunk);
+        k_lo = min(k_hi, split * chunk);
+        k_hi = min(k_hi, k_lo + chunk);
     }
     // staging: NT / NN A and NT B are row-major in k (thread: row t / 2,
     // k quad (t % 2) * 4); TN A and NN / TN B are row-major in m / n
     // (thread: k row t / 32, 4 columns (t % 32) * 4)
     const int rq = tid >> 1, kq = (tid & 1) * 4, kr = tid >> 5, cq = (tid & 31) * 4;
     const float *arow = nullptr, *brow = nullptr;
-    if (FORM != BW_TN && m0 + rq < p.M) arow = p.A + bw_row(p.a_map, m0 + rq, g) * p.lda;
+    if (FORM != BW_TN && m0 + rq < Mg) arow = p.A + bw_grow(p, p.a_map, m0 + rq, g) * p.lda;
     if (FORM == BW_NT && n0 + rq < p.N) brow = p.B + g * p.b_gstride + static_cast<long long>(n0 + rq) * p.ldb;
     float ra[4], rb[4];
     auto fetch = [&](int k0) {
@@ -299,7 +314,7 @@ __global__ void __launch_bounds__(GB_T, 2) bw_gemm_big_kernel(BwGemm p)
             for (int q = 0; q < 4; ++q) ra[q] = (arow && k0 + kq + q < k_hi) ? arow[k0 + kq + q] : 0.f;
         } else {
             const int k = k0 + kr;
-            const float *src = k < k_hi ? p.A + bw_row(p.a_map, k, g) * p.lda : nullptr;
+            const float *src = k < k_hi ? p.A + bw_grow(p, p.a_map, k, g) * p.lda : nullptr;
 #pragma unroll
             for (int q = 0; q < 4; ++q) ra[q] = (src && m0 + cq + q < p.M) ? src[m0 + cq + q] : 0.f;
         }
@@ -311,7 +326,7 @@ __global__ void __launch_bounds__(GB_T, 2) bw_gemm_big_kernel(BwGemm p)
             const float *src = nullptr;
             if (k < k_hi)
                 src = FORM == BW_NN ? p.B + g * p.b_gstride + static_cast<long long>(k) * p.ldb
-                                    : p.B + bw_row(p.b_map, k, g) * p.ldb;
+                                    : p.B + bw_grow(p, p.b_map, k, g) * p.ldb;
 #pragma unroll
             for (int q = 0; q < 4; ++q) rb[q] = (src && n0 + cq + q < p.N) ? src[n0 + cq + q] : 0.f;
         }
@@ -366,14 +381,14 @@ __global__ void __launch_bounds__(GB_T, 2) bw_gemm_big_kernel(BwGemm p)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
-        if (m >= p.M) continue;
+        if (m >= Mg) continue;
         float *crow;
         if (FORM == BW_TN && p.splits > 1)
             crow = p.partial + ((static_cast<long long>(split) * p.G + g) * p.M + m) * p.N;
         else if (FORM == BW_TN)
             crow = p.C + g * p.c_gstride + static_cast<long long>(m) * p.ldc;
         else
-            crow = p.C + bw_row(p.c_map, m, g) * p.ldc;
+            crow = p.C + bw_grow(p, p.c_map, m, g) * p.ldc;
         const bool add = p.accumulate && !(FORM == BW_TN && p.splits > 1);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -549,6 +564,10 @@ struct Backward {
     Side s, n;
     float *partial;
     float *tn_partial; // split TN GEMMs: < 2 * 296 tiles of at most 128 x 128 floats
+    // mixture of experts (E > 0): routing and the experts' rows, P = T k slots
+    int E, K;
+    BwMoe moe;
+    float *Zp, *U1e, *Acte, *Ye, *dYe, *dActe, *dZp, *logits, *dlogits;
     static constexpr long long kTnPartialFloats = 2LL * 296 * 128 * 128;
     float *dXbuf[2], *dYbuf[2];
     const float *G_s, *G_ns;
@@ -610,6 +629,26 @@ struct Backward {
         };
         side(s, R, Tq);
         if (C) side(n, RN_, RN_);
+        if (E) {
+            const long long P = Tq * K;
+            auto ints = [&](long long cnt) { return reinterpret_cast<int *>(cv.take(cnt)); };
+            logits = cv.take(Tq * E);
+            dlogits = cv.take(Tq * E);
+            moe.sel = ints(Tq * 2);
+            moe.gate = cv.take(Tq * 2);
+            moe.lrank = ints(Tq * 2);
+            moe.slot = ints(Tq * 2);
+            moe.hist = ints(static_cast<long long>(bw_moe_chunks(static_cast<int>(Tq))) * E);
+            moe.seg_off = ints(E);
+            moe.seg_cnt = ints(E);
+            Zp = cv.take(P * d);
+            U1e = cv.take(P * f);
+            Acte = cv.take(P * f);
+            Ye = cv.take(P * d);
+            dYe = cv.take(P * d);
+            dActe = cv.take(P * f);
+            dZp = cv.take(P * d);
+        }
         partial = cv.take(64LL * d * (C ? N : 1)); // gain partials: <= 64 chunks, 1 or N groups
         tn_partial = cv.take(kTnPartialFloats);
         dXbuf[0] = cv.take(R * d);
@@ -652,11 +691,25 @@ struct Backward {
         return a;
     }
 
+    // segments of the experts (group = expert) for the next GEMM
+    const int *seg_off_ = nullptr, *seg_cnt_ = nullptr;
+    void segs(bool on)
+    {
+        seg_off_ = on ? moe.seg_off : nullptr;
+        seg_cnt_ = on ? moe.seg_cnt : nullptr;
+    }
+    void seg_fill(BwGemm &p) const
+    {
+        p.g_off = seg_off_;
+        p.g_cnt = seg_cnt_;
+    }
+
     // C = A B^T with B a weight [G][Nn][K]
     void nt(const float *A, long long lda, RowMap am, const float *B, long long bgs, float *Cp, long long ldc,
             RowMap cm, int M, int Nn, int K, int G, int acc)
     {
         BwGemm p{};
+        seg_fill(p);
         p.form = BW_NT, p.M = M, p.N = Nn, p.K = K, p.G = G;
         p.A = A, p.lda = lda, p.a_map = am;
         p.B = B, p.ldb = K, p.b_gstride = bgs;
@@ -668,6 +721,7 @@ struct Backward {
             RowMap cm, int M, int Nn, int K, int G)
     {
         BwGemm p{};
+        seg_fill(p);
         p.form = BW_NN, p.M = M, p.N = Nn, p.K = K, p.G = G;
         p.A = A, p.lda = lda, p.a_map = am;
         p.B = B, p.ldb = Nn, p.b_gstride = bgs;
@@ -679,6 +733,7 @@ struct Backward {
             long long cgs, int M, int Nn, int K, int G)
     {
         BwGemm p{};
+        seg_fill(p);
         p.form = BW_TN, p.M = M, p.N = Nn, p.K = K, p.G = G;
         p.A = A, p.lda = lda, p.a_map = am;
         p.B = B, p.ldb = ldb, p.b_map = bm;
@@ -720,11 +775,16 @@ struct Backward {
         nt(s.A, d, kIdentity, wt(w->Wo_s, l * dd), 0, s.H, d, kIdentity, static_cast<int>(Tq), d, d, 1, 1);
         const BwRows h2{s.H, kIdentity, Tq, 1, d};
         k([&] { return bw_rms_fwd(h2, wt(w->g2_s, static_cast<long long>(l) * d), 0, c.eps, s.Z2, s.r2, st); });
-        nt(s.Z2, d, kIdentity, wt(w->W1_s, l * fd), 0, s.U1, f, kIdentity, static_cast<int>(Tq), f, d, 1, 0);
-        k([&] { return bw_gelu_fwd(s.U1, s.Act, Tq * f, st); });
-        if (s_out) {
-            copy(s_out, s.H, static_cast<size_t>(Tq) * d * 4);
-            nt(s.Act, f, kIdentity, wt(w->W2_s, l * fd), 0, s_out, d, kIdentity, static_cast<int>(Tq), d, f, 1, 1);
+        if (E) {
+            moe_forward(l, s_out);
+        } else {
+            nt(s.Z2, d, kIdentity, wt(w->W1_s, l * fd), 0, s.U1, f, kIdentity, static_cast<int>(Tq), f, d, 1, 0);
+            k([&] { return bw_gelu_fwd(s.U1, s.Act, Tq * f, st); });
+            if (s_out) {
+                copy(s_out, s.H, static_cast<size_t>(Tq) * d * 4);
+                nt(s.Act, f, kIdentity, wt(w->W2_s, l * fd), 0, s_out, d, kIdentity, static_cast<int>(Tq), d, f, 1,
+                   1);
+            }
         }
         if (!C) return;
         // ---- NS side
@@ -742,19 +802,61 @@ struct Backward {
         }
     }
 
+    // The S-side mixture of layer l on Z2 = n(H; g2): router logits, routing,
+    // the experts' FFNs over their segments; with s_out also y = H + sum g Y.
+    void moe_forward(int l, float *s_out)
+    {
+        const int Tq = static_cast<int>(T(l));
+        const long long fd = static_cast<long long>(f) * d, Eed = static_cast<long long>(E) * d;
+        moe.T = Tq, moe.d = d, moe.E = E, moe.k = K, moe.logits = logits;
+        nt(s.Z2, d, kIdentity, wt(w->W_router, l * Eed), 0, logits, E, kIdentity, Tq, E, d, 1, 0);
+        k([&] { return bw_moe_route(moe, s.Z2, Zp, st); });
+        launches += 3; // top-k, rank, offsets and dispatch
+        segs(true);
+        nt(Zp, d, kIdentity, wt(w->W1_moe, l * E * fd), fd, U1e, f, kIdentity, Tq, f, d, E, 0);
+        k([&] { return bw_gelu_fwd(U1e, Acte, static_cast<long long>(Tq) * K * f, st); });
+        nt(Acte, f, kIdentity, wt(w->W2_moe, l * E * fd), fd, Ye, d, kIdentity, Tq, d, f, E, 0);
+        segs(false);
+        if (s_out) k([&] { return bw_moe_combine(moe, s.H, Ye, s_out, st); });
+    }
+
+    // The S-side mixture's backward: dOut -> x.dZ2 (router and experts) and
+    // the gradients of the router and the experts of layer l.
+    void moe_back(int l, const float *dOut)
+    {
+        const int Tq = static_cast<int>(T(l));
+        const long long fd = static_cast<long long>(f) * d, Eed = static_cast<long long>(E) * d;
+        k([&] { return bw_moe_combine_bwd(moe, dOut, Ye, dYe, dlogits, st); });
+        tn(dlogits, E, kIdentity, s.Z2, d, kIdentity, g->W_router + l * Eed, 0, E, d, Tq, 1); // dW_r
+        nn(dlogits, E, kIdentity, wt(w->W_router, l * Eed), 0, s.dZ2, d, kIdentity, Tq, d, E, 1); // dZ2 = dlogits W_r
+        segs(true);
+        nn(dYe, d, kIdentity, wt(w->W2_moe, l * E * fd), fd, dActe, f, kIdentity, Tq, f, d, E);      // dAct = dY W2
+        tn(dYe, d, kIdentity, Acte, f, kIdentity, g->W2_moe + l * E * fd, fd, d, f, Tq, E);          // dW2
+        k([&] { return bw_gelu_bwd(U1e, dActe, dActe, static_cast<long long>(Tq) * K * f, st); });
+        tn(dActe, f, kIdentity, Zp, d, kIdentity, g->W1_moe + l * E * fd, fd, f, d, Tq, E);          // dW1
+        nn(dActe, f, kIdentity, wt(w->W1_moe, l * E * fd), fd, dZp, d, kIdentity, Tq, d, f, E);      // dZp = dU1 W1
+        segs(false);
+        k([&] { return bw_moe_gather(moe, dZp, s.dZ2, st); });
+    }
+
     // FFN and output-projection backward of one side: dOut -> x.dH, x.dA and
     // the gradients of W1, W2, Wo and g2.  M rows in each of G groups under map.
     void ffn_back(Side &x, const float *dOut, RowMap map, int M, int G, const float *W1, const float *W2,
-                  const float *Wo, const float *g2, long long ggs, float *dW1, float *dW2, float *dWo, float *dg2)
+                  const float *Wo, const float *g2, long long ggs, float *dW1, float *dW2, float *dWo, float *dg2,
+                  int moe_layer = -1)
     {
         const long long rows = static_cast<long long>(M) * G;
         const long long fd = static_cast<long long>(f) * d, dd = static_cast<long long>(d) * d;
         copy(x.dH, dOut, static_cast<size_t>(rows) * d * 4);
-        nn(dOut, d, map, W2, fd, x.dAct, f, map, M, f, d, G); // dAct = dOut W2
-        tn(dOut, d, map, x.Act, f, map, dW2, fd, d, f, M, G);  // dW2 = dOut^T Act
-        k([&] { return bw_gelu_bwd(x.U1, x.dAct, x.dAct, rows * f, st); });
-        tn(x.dAct, f, map, x.Z2, d, map, dW1, fd, f, d, M, G); // dW1 = dU1^T Z2
-        nn(x.dAct, f, map, W1, fd, x.dZ2, d, map, M, d, f, G); // dZ2 = dU1 W1
+        if (moe_layer >= 0) {
+            moe_back(moe_layer, dOut);
+        } else {
+            nn(dOut, d, map, W2, fd, x.dAct, f, map, M, f, d, G); // dAct = dOut W2
+            tn(dOut, d, map, x.Act, f, map, dW2, fd, d, f, M, G);  // dW2 = dOut^T Act
+            k([&] { return bw_gelu_bwd(x.U1, x.dAct, x.dAct, rows * f, st); });
+            tn(x.dAct, f, map, x.Z2, d, map, dW1, fd, f, d, M, G); // dW1 = dU1^T Z2
+            nn(x.dAct, f, map, W1, fd, x.dZ2, d, map, M, d, f, G); // dZ2 = dU1 W1
+        }
         const BwRows hr{x.H, map, M, G, d};
         k([&] { return bw_rms_bwd(hr, g2, ggs, x.r2, x.dZ2, x.dH, 1, st); });
         const int sp = bw_gain_splits(hr);
@@ -789,8 +891,9 @@ struct Backward {
         const int M = U * C;
         // FFN + output projection, both sides
         ffn_back(s, dXin, kIdentity, static_cast<int>(Tq), 1, wt(w->W1_s, l * fd), wt(w->W2_s, l * fd),
-                 wt(w->Wo_s, l * dd), wt(w->g2_s, static_cast<long long>(l) * d), 0, g->W1_s + l * fd,
-                 g->W2_s + l * fd, g->Wo_s + l * dd, g->g2_s + static_cast<long long>(l) * d);
+                 wt(w->Wo_s, l * dd), wt(w->g2_s, static_cast<long long>(l) * d), 0,
+                 E ? nullptr : g->W1_s + l * fd, E ? nullptr : g->W2_s + l * fd, g->Wo_s + l * dd,
+                 g->g2_s + static_cast<long long>(l) * d, E ? l : -1);
         if (C)
             ffn_back(n, dYin, nm, M, N, wt(w->W1_ns, ln * fd), wt(w->W2_ns, ln * fd), wt(w->Wo_ns, ln * dd),
                      wt(w->g2_ns, ln * d), d, g->W1_ns + ln * fd, g->W2_ns + ln * fd, g->Wo_ns + ln * dd,
@@ -821,6 +924,12 @@ struct Backward {
 
     void run()
     {
+        if (E) {
+            // the dense S-side FFN is unused: its gradients are zero
+            const long long fdL = static_cast<long long>(Lyr) * f * d * 4;
+            if (g->W1_s) zero(g->W1_s, fdL);
+            if (g->W2_s) zero(g->W2_s, fdL);
+        }
         if (!C) {
             const long long fd = static_cast<long long>(f) * d, dd = static_cast<long long>(d) * d;
             const long long LN = static_cast<long long>(Lyr) * N;
@@ -853,7 +962,6 @@ ot_status bw_validate(const ot_config *cfg, int U, int C)
 {
     if (!cfg || U < 1 || C < 0) return OT_ERR_ARG;
     if (cfg->dtype != OT_DTYPE_F32) return OT_ERR_DTYPE;
-    if (cfg->moe_experts) return OT_ERR_UNSUPPORTED;
     if (cfg->full_attn && C != 1) return OT_ERR_SHAPE; // one candidate per user, as the forward
     const ot_status r = internal_check_config(*cfg);
     if (r != OT_OK) return r;
@@ -872,6 +980,8 @@ void bw_init(Backward &b, const ot_config *cfg, int U, int C)
     b.hd = cfg->d / cfg->heads, b.Lyr = cfg->layers;
     b.Ls[0] = cfg->L0;
     for (int l = 0; l < cfg->layers; ++l) b.Ls[l + 1] = cfg->q[l];
+    b.E = cfg->moe_experts;
+    b.K = cfg->moe_experts ? cfg->moe_topk : 0;
     b.launches = 0;
     b.err = cudaSuccess;
     b.bytes = 0;
@@ -914,17 +1024,22 @@ ot_status ot_full_backward(const ot_config *cfg, const ot_weights *w, const floa
 {
     if (!cfg || !w || !g || !S || !G_s || !ws || U < 1 || C < 0) return OT_ERR_ARG;
     if (C && (!ns || !G_ns)) return OT_ERR_ARG;
-    const void *wp[] = {w->Wqkv_s,  w->Wo_s,  w->W1_s,  w->W2_s,  w->g1_s,  w->g2_s,
-                        w->Wqkv_ns, w->Wo_ns, w->W1_ns, w->W2_ns, w->g1_ns, w->g2_ns};
-    const void *gp[] = {g->Wqkv_s,  g->Wo_s,  g->W1_s,  g->W2_s,  g->g1_s,  g->g2_s,
-                        g->Wqkv_ns, g->Wo_ns, g->W1_ns, g->W2_ns, g->g1_ns, g->g2_ns};
-    for (int i = 0; i < 12; ++i)
-        if (!wp[i] || !gp[i]) return OT_ERR_ARG;
+    const bool moe = cfg->moe_experts > 0;
+    const void *wp[] = {w->Wqkv_s,  w->Wo_s,   w->W1_s,  w->W2_s,  w->g1_s,   w->g2_s,
+                        w->Wqkv_ns, w->Wo_ns,  w->W1_ns, w->W2_ns, w->g1_ns,  w->g2_ns,
+                        w->W_router, w->W1_moe, w->W2_moe};
+    const void *gp[] = {g->Wqkv_s,  g->Wo_s,   g->W1_s,  g->W2_s,  g->g1_s,   g->g2_s,
+                        g->Wqkv_ns, g->Wo_ns,  g->W1_ns, g->W2_ns, g->g1_ns,  g->g2_ns,
+                        g->W_router, g->W1_moe, g->W2_moe};
+    // required: the dense twelve (W1_s / W2_s not with a mixture), the MoE three with one
+    auto needed = [&](int i) { return i < 12 ? !(moe && (i == 2 || i == 3)) : moe; };
+    for (int i = 0; i < 15; ++i)
+        if (needed(i) && (!wp[i] || !gp[i])) return OT_ERR_ARG;
     const ot_status v = bw_validate(cfg, U, C);
     if (v != OT_OK) return v;
     auto al = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
-    for (int i = 0; i < 12; ++i)
-        if (!al(wp[i]) || !al(gp[i])) return OT_ERR_ALIGN;
+    for (int i = 0; i < 15; ++i)
+        if ((needed(i) || (i < 12 && gp[i])) && (!al(wp[i]) || !al(gp[i]))) return OT_ERR_ALIGN;
     if (!al(S) || !al(G_s) || !al(ws) || (C && (!al(ns) || !al(G_ns))) || (out_s_tail && !al(out_s_tail)) ||
         (C && out_ns && !al(out_ns)) || (dS && !al(dS)) || (C && dns && !al(dns)))
         return OT_ERR_ALIGN;

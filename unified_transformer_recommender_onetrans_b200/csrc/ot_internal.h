@@ -310,6 +310,11 @@ struct BwGemm {
     // split order into C (splits == 1: straight into C)
     int splits;
     float *partial;
+    // segments (the experts of a mixture): group g owns buffer rows
+    // g_off[g] .. g_off[g] + g_cnt[g] - 1, in place of the row maps of the
+    // M rows (NT / NN: A and C) or of the K rows (TN: A and B); rows past
+    // g_cnt[g] are not read or written.  Null: the row maps.
+    const int *g_off, *g_cnt;
 };
 // One attention problem of a layer over QKV rows [.][3d] (Q | K | V):
 //   mode 0 (S queries): query i of user u is S row t = L - nq + i of the
@@ -354,6 +359,31 @@ cudaError_t bw_attn_bwd_kv_s(const BwAttn &sq, const BwAttn *nsq, cudaStream_t s
 // NS keys: the NS queries of problem a and, if sq (full attention), the S
 // queries of sq
 cudaError_t bw_attn_bwd_kv_ns(const BwAttn &a, const BwAttn *sq, cudaStream_t s);
+
+// Mixture-of-experts routing of T rows in the backward pass: top-k of the
+// E logits per row (ties to the lower index) and softmax gates; a fixed,
+// expert-major slot per choice (experts in order, rows in order within an
+// expert, no atomics): segment e = slots seg_off[e] .. + seg_cnt[e].
+struct BwMoe {
+    int T, d, E, k;
+    const float *logits; // [T][E]
+    int *sel;            // [T][2] chosen experts
+    float *gate;         // [T][2]
+    int *lrank;          // [T][2] rank within the choice's 128-row chunk
+    int *hist;           // [chunks][E]
+    int *seg_off, *seg_cnt; // [E]
+    int *slot;           // [T][2]
+};
+int bw_moe_chunks(int T);
+// route + copy z rows to their slots (Zp [T k][d]); 4 launches
+cudaError_t bw_moe_route(const BwMoe &m, const float *z, float *Zp, cudaStream_t s);
+// y = h + sum_j gate_j Y[slot_j]
+cudaError_t bw_moe_combine(const BwMoe &m, const float *h, const float *Y, float *y, cudaStream_t s);
+// dY[slot_j] = gate_j dy; dlogits [T][E] from the gates' softmax
+cudaError_t bw_moe_combine_bwd(const BwMoe &m, const float *dy, const float *Y, float *dY, float *dlogits,
+                               cudaStream_t s);
+// dz[r] += sum_j dZp[slot_j]
+cudaError_t bw_moe_gather(const BwMoe &m, const float *dZp, float *dz, cudaStream_t s);
 
 // Shape / dtype check of a config (the rules of ot_model_create).
 ot_status internal_check_config(const ot_config &c);
