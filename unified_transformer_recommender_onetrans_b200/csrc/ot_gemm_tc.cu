@@ -169,7 +169,7 @@ __device__ __forceinline__ void epi_res(const TcGemmParams &Q, long long lt, int
     if (r < a.M && e.res) e.res_off = rowmap_dev(a.res_map, r, e.g) * a.res_ld + e.n0 + half * (BN / 2);
 }
 
-template <int BN>
+template <int BN, bool FP8>
 __device__ __forceinline__ void epi_tile(const TcGemmParams &Q, int q, int lane, int half, EpiTile &e)
 {
     const GemmArgs &a = Q.a;
@@ -212,8 +212,11 @@ __device__ __forceinline__ void epi_tile(const TcGemmParams &Q, int q, int lane,
     e.row_scale = live ? a.row_scale : nullptr;
     e.row_scale_idx = e.row_scale ? rowmap_dev(a.a_map, r, e.g) : 0;
     e.g_scale = a.g_scale ? a.g_scale[e.g] : 1.f;
-    if (a.xg_scale) e.g_scale *= a.xg_scale[e.g * a.xg_gstride];
-    e.q_inv = a.qscale ? __frcp_rn(a.qscale[e.g * a.qscale_gstride]) : 1.f;
+    e.q_inv = 1.f;
+    if (FP8) { // per-group activation scale of the A operand; e4m3 output scale
+        if (a.xg_scale) e.g_scale *= a.xg_scale[e.g * a.xg_gstride];
+        if (a.qscale) e.q_inv = __frcp_rn(a.qscale[e.g * a.qscale_gstride]);
+    }
 }
 
 template <int BN, bool FP8, bool MULTI>
@@ -251,7 +254,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_kb = a0.K / (FP8 ? 128 : 64);
     const bool norm = a0.norm != 0 && !FP8;
-    const bool q8 = a0.store == OT_STORE_E4M3; // launch-wide (both problems agree)
+    // e4m3 output: launch-wide, and only with e4m3 operands (the bf16
+    // instantiations compile without the branch)
+    const bool q8 = FP8 && a0.store == OT_STORE_E4M3;
     pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
@@ -426,9 +431,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                     *stage_chunk<ROWB>(stage, RPI * i + lane / LPR, lane % LPR) = rv[i];
             }
             if (MULTI && pi)
-                epi_tile<G_BN>(P.q[1], q, lane, half, et);
+                epi_tile<G_BN, FP8>(P.q[1], q, lane, half, et);
             else
-                epi_tile<G_BN>(P.q[0], q, lane, half, et);
+                epi_tile<G_BN, FP8>(P.q[0], q, lane, half, et);
             const long long out_off = et.out_off;
             if (!mbar_wait(&tfull[b], (t >> 1) & 1, wctl, abort_flag)) break;
             tc_fence_after();
@@ -662,7 +667,7 @@ static bool gemm_ok(const GemmArgs &a, bool &wide)
 {
     const bool fp8 = a.in_dtype == OT_DTYPE_FP8;
     if (a.store != OT_STORE_BF16 && a.store != OT_STORE_E4M3) return false;
-    if (a.store == OT_STORE_E4M3 && (a.res || !a.qscale)) return false;
+    if (a.store == OT_STORE_E4M3 && (a.res || !a.qscale || !fp8)) return false;
     if (a.K % (fp8 ? 128 : 64) != 0 || a.a_map.P != 1 || a.N % 128 != 0 || a.M < 1 || a.G < 1)
         return false;
     wide = a.N % 256 == 0;
