@@ -12,7 +12,9 @@ import ctypes as C
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "_lib", "libonetrans.so")
+# OT_CHECKED=1: the debug build with device bounds checks (build --checked)
+LIB_PATH = os.path.join(HERE, "_lib", "libonetrans_checked.so" if os.environ.get("OT_CHECKED") == "1"
+                        else "libonetrans.so")
 MAX_LAYERS = 32
 
 OT_OK = 0

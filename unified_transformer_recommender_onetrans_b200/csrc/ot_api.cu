@@ -21,7 +21,10 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <cstdlib>
+#include <initializer_list>
 #include <mutex>
+#include <utility>
 #include <new>
 #include <vector>
 
@@ -312,6 +315,8 @@ void gemm_cost(const ot_model *m, const GemmArgs &a, double &flops, double &byte
                         (a.res ? static_cast<double>(a.M) * a.N : 0.0));
 }
 
+long long cap_of(const void *p); // extent of a caller buffer (checked build)
+
 void gemm_prepare(const ot_model *m, GemmArgs &a)
 {
     a.wait = WaitCtl{m->err, m->wait_limit};
@@ -320,6 +325,7 @@ void gemm_prepare(const ot_model *m, GemmArgs &a)
                  : a.in_dtype == OT_DTYPE_FP8 ? OT_DTYPE_FP8
                                               : OT_DTYPE_BF16;
     a.store = m->cfg.dtype == OT_DTYPE_F32 ? OT_STORE_F32 : a.qscale ? OT_STORE_E4M3 : OT_STORE_BF16;
+    a.res_cap = cap_of(a.res);
 }
 
 ot_status gemm(ot_model *m, GemmArgs &a, cudaStream_t s, int role)
@@ -352,6 +358,7 @@ void attn_cost(const ot_model *m, const AttnArgs &a, double &flops, double &byte
 ot_status attn(ot_model *m, AttnArgs &a, cudaStream_t s)
 {
     a.wait = WaitCtl{m->err, m->wait_limit};
+    a.o_cap = cap_of(a.O);
     if (a.mode == 1) a.nkn = a.nq;
     if (a.mode == 0 && a.full && (!a.KN || !a.VN || a.nkn < 1)) return OT_ERR_ARG;
     a.dtype = m->cfg.dtype;
@@ -564,10 +571,60 @@ void fp8_hidden_operand(GemmArgs &g, const void *hid, long long lda, RowMap amap
     g.in_dtype = OT_DTYPE_FP8;
 }
 
+// Extents of the caller's buffers during one call (used by the checked
+// build): a pointer inside one of them gets the bytes to its end as the
+// bound of the kernels' plain accesses through it.  Thread-local, set by
+// each entry point for the length of the call.
+struct Region {
+    const char *b, *e;
+};
+thread_local Region t_regions[8];
+thread_local int t_nregions = 0;
+
+struct RegionScope {
+    RegionScope(std::initializer_list<std::pair<const void *, size_t>> rs)
+    {
+        t_nregions = 0;
+        for (const auto &r : rs)
+            if (r.first && r.second && t_nregions < 8)
+                t_regions[t_nregions++] = Region{static_cast<const char *>(r.first),
+                                                 static_cast<const char *>(r.first) + r.second};
+    }
+    ~RegionScope() { t_nregions = 0; }
+};
+
+// Checked build test hook: OT_CHECK_SHRINK=1 halves every extent, so that
+// the kernels' checks fire (and skip the accesses) on a correct call.
+bool check_shrink()
+{
+    static const bool on = kDeviceChecks && getenv("OT_CHECK_SHRINK") && atoi(getenv("OT_CHECK_SHRINK")) == 1;
+    return on;
+}
+
+long long cap_of(const void *p)
+{
+    if (!kDeviceChecks || !p) return 0;
+    const char *c = static_cast<const char *>(p);
+    for (int i = 0; i < t_nregions; ++i)
+        if (c >= t_regions[i].b && c < t_regions[i].e) {
+            const long long cap = t_regions[i].e - c;
+            return check_shrink() ? (cap + 1) / 2 : cap;
+        }
+    return 0;
+}
+
+size_t kv_bytes(const ot_model *m, int U) { return static_cast<size_t>(U) * kv_user_elems(m->cfg) * m->esz; }
+size_t tail_bytes(const ot_model *m, int U)
+{
+    return static_cast<size_t>(U) * m->cfg.q[m->cfg.layers - 1] * m->cfg.d * m->esz;
+}
+size_t ns_bytes(const ot_model *m, long long rows) { return static_cast<size_t>(rows) * m->cfg.n_ns * m->cfg.d * m->esz; }
+
 EpiSeg seg_of(void *out, long long ld, int lo, int hi, RowMap map)
 {
-    EpiSeg s;
+    EpiSeg s{};
     s.out = out;
+    s.cap = cap_of(out);
     s.ld = ld;
     s.c_lo = lo;
     s.c_hi = hi;
@@ -1518,6 +1575,7 @@ ot_status ot_auto_split(ot_model *m, const void *x, long M, void *ns, void *stre
     g.B = m->W_split;
     g.b_gstride = static_cast<long long>(Nd) * c.F;
     g.nseg = 1;
+    RegionScope rs{{ns, ns_bytes(m, M)}};
     g.seg[0] = seg_of(ns, Nd, 0, Nd, rowmap_identity());
     return gemm(m, g, static_cast<cudaStream_t>(stream), ROLE_AUTO_SPLIT);
 }
@@ -1545,6 +1603,7 @@ ot_status ot_encode_user(ot_model *m, const void *S, int U, void *kv_cache, void
     if (static_cast<long long>(U) * m->cfg.L0 > (1LL << 31) - 1) return OT_ERR_SHAPE;
     if (ws_bytes < ot_workspace_bytes(m, U, 0)) return OT_ERR_WORKSPACE_TOO_SMALL;
     Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
+    RegionScope rs{{ws, ws_bytes}, {kv_cache, kv_bytes(m, U)}, {out_s_tail, tail_bytes(m, U)}};
     return run_encode(m, S, U, kv_cache, out_s_tail, w, static_cast<cudaStream_t>(stream));
 }
 
@@ -1598,6 +1657,8 @@ ot_status ot_encode_append(ot_model *m, const void *kv_old, int U, const void *S
     if (r != OT_OK) return r;
     // 2. the new rows through every layer, against the grown cache
     Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
+    RegionScope rs{{ws, ws_bytes}, {kv_new, static_cast<size_t>(bytes_new)},
+                   {out_new, static_cast<size_t>(U) * c.q[c.layers - 1] * c.d * m->esz}};
     return run_encode(m, S_new, U, kv_new, out_new, w, st, nullptr, delta);
 }
 
@@ -1612,6 +1673,7 @@ ot_status ot_score_candidates(ot_model *m, const void *kv_cache, int U, const vo
     if (static_cast<long long>(C) * m->cfg.n_ns > (1LL << 30)) return OT_ERR_SHAPE;
     if (ws_bytes < score_ws_bytes(m->cfg, U, C, m->esz)) return OT_ERR_WORKSPACE_TOO_SMALL;
     Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
+    RegionScope rs{{ws, ws_bytes}, {out_ns, ns_bytes(m, static_cast<long long>(U) * C)}};
     return run_score(m, kv_cache, U, ns, C, out_ns, w, static_cast<cudaStream_t>(stream));
 }
 
@@ -1658,6 +1720,8 @@ ot_status ot_encode_user_paged(ot_model *m, const void *S, int U, void *pool, lo
                            [&] { return launch_page_tail_clear(pt, U, st); });
     if (r != OT_OK) return r;
     Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
+    RegionScope rs{{ws, ws_bytes}, {pool, static_cast<size_t>(n_pages) * ot_kv_page_bytes(m)},
+                   {out_s_tail, tail_bytes(m, U)}};
     return run_encode(m, S, U, nullptr, out_s_tail, w, st, nullptr, 0, false, &pg);
 }
 
@@ -1676,6 +1740,7 @@ ot_status ot_score_candidates_paged(ot_model *m, const void *pool, long long n_p
     if (ws_bytes < score_ws_bytes(m->cfg, U, C, m->esz)) return OT_ERR_WORKSPACE_TOO_SMALL;
     const PagedKv pg{const_cast<void *>(pool), pages, n_pages, page_off(m->cfg, m->cfg.layers)};
     Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
+    RegionScope rs{{ws, ws_bytes}, {out_ns, ns_bytes(m, static_cast<long long>(U) * C)}};
     return run_score(m, nullptr, U, ns, C, out_ns, w, static_cast<cudaStream_t>(stream), nullptr, &pg);
 }
 
@@ -1696,6 +1761,8 @@ ot_status ot_full_forward(ot_model *m, const void *S, const void *ns, int B, int
     const size_t serial_need = (enc > sc ? enc : sc) + kvb;
     if (ws_bytes < serial_need) return OT_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    RegionScope rs{{ws, ws_bytes}, {kv_cache, kv_bytes(m, B)}, {out_s_tail, tail_bytes(m, B)},
+                   {out_ns, ns_bytes(m, static_cast<long long>(B) * C)}};
     Ws w{static_cast<char *>(ws), ws_bytes, m->esz};
     void *kv = kv_cache;
     if (!kv) {

@@ -326,8 +326,9 @@ __global__ void __launch_bounds__(NA_WARPS * 32, 2)
         out.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
         out.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
         out.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-        *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.O) +
-                                   (static_cast<long long>(u) * a.nq + row) * a.d + h * NA_HD + c8 * 8) = out;
+        const long long o_off = (static_cast<long long>(u) * a.nq + row) * a.d + h * NA_HD + c8 * 8;
+        if (ot_dev_ok(o_off * 2, 16, a.o_cap, a.wait.err))
+            *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.O) + o_off) = out;
     }
 }
 

@@ -625,10 +625,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             // O may now be overwritten by the next item's first PV
             release(&o_free[w]);
             if (SPLIT) release(&o_free[1]);
-            if (i < a.nq) {
-                uint4 *dp = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.O) +
-                                                      (static_cast<long long>(it.u) * a.nq + i) * a.d +
-                                                      it.h * AT_HD);
+            const long long o_off = (static_cast<long long>(it.u) * a.nq + i) * a.d + it.h * AT_HD;
+            if (i < a.nq && ot_dev_ok(o_off * 2, AT_HD * 2, a.o_cap, a.wait.err)) {
+                uint4 *dp = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.O) + o_off);
 #pragma unroll
                 for (int qd = 0; qd < 8; ++qd)
                     dp[qd] = make_uint4(ob[4 * qd], ob[4 * qd + 1], ob[4 * qd + 2], ob[4 * qd + 3]);

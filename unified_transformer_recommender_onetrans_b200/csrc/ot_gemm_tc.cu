@@ -148,7 +148,9 @@ struct EpiTile {
     long long out_off;          // this lane's row in the output segment (-1: not stored)
     long long res_off;          // this lane's row in the residual
     const __nv_bfloat16 *res;   // null: no residual
+    long long res_cap;          // checked build: bytes of the residual buffer from res
     __nv_bfloat16 *obase;       // output segment base
+    long long cap;              // checked build: bytes of the output buffer from obase
     const float *row_scale;     // fp8: per-row scale (indexed through the A row map), or null
     long long row_scale_idx;
     float g_scale;              // fp8: per-matrix scale (1 otherwise), times the A operand's per-group scale
@@ -165,6 +167,7 @@ __device__ __forceinline__ void epi_res(const TcGemmParams &Q, long long lt, int
     e.M = a.M;
     const int r = e.m0 + 32 * q + lane;
     e.res = static_cast<const __nv_bfloat16 *>(a.res);
+    e.res_cap = a.res_cap;
     e.res_off = 0;
     if (r < a.M && e.res) e.res_off = rowmap_dev(a.res_map, r, e.g) * a.res_ld + e.n0 + half * (BN / 2);
 }
@@ -187,6 +190,7 @@ __device__ __forceinline__ void epi_tile(const TcGemmParams &Q, int q, int lane,
 #define OT_SEGF(f) (sidx == 0 ? s0.f : sidx == 1 ? s1.f : s2.f)
     const RowMap mp{OT_SEGF(map.P), OT_SEGF(map.A), OT_SEGF(map.B), OT_SEGF(map.Gs), OT_SEGF(map.min_t)};
     e.obase = static_cast<__nv_bfloat16 *>(OT_SEGF(out));
+    e.cap = OT_SEGF(cap);
     e.out_off = -1;
     const int *pages = OT_SEGF(pages);
     if (live && rowmap_keep_dev(mp, r)) {
@@ -423,7 +427,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                     const int rl = RPI * i + lane / LPR, ch = lane % LPR;
                     const long long ro = __shfl_sync(0xffffffffu, res_off, rl);
                     rv[i] = make_uint4(0, 0, 0, 0);
-                    if (m0 + 32 * q + rl < et.M)
+                    if (m0 + 32 * q + rl < et.M && ot_dev_ok((ro + ch * 8) * 2, 16, et.res_cap, wctl.err))
                         rv[i] = __ldg(reinterpret_cast<const uint4 *>(res + ro + ch * 8));
                 }
 #pragma unroll
@@ -483,7 +487,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                 for (int i = 0; i < 32 / RPI8; ++i) {
                     const int rl = RPI8 * i + lane / LPR8, ch = lane % LPR8;
                     const long long oo = __shfl_sync(0xffffffffu, out_off, rl);
-                    if (oo < 0) continue;
+                    if (oo < 0 || !ot_dev_ok(oo + ch * 16, 16, et.cap, wctl.err)) continue;
                     *reinterpret_cast<uint4 *>(ob8 + oo + ch * 16) = *stage_chunk<ROWB>(stage, rl, ch);
                 }
                 __syncwarp(); // staging free for the next tile
@@ -532,7 +536,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             for (int i = 0; i < 32 / RPI; ++i) {
                 const int rl = RPI * i + lane / LPR, ch = lane % LPR;
                 const long long oo = __shfl_sync(0xffffffffu, out_off, rl);
-                if (oo < 0) continue;
+                if (oo < 0 || !ot_dev_ok((oo + ch * 8) * 2, 16, et.cap, wctl.err)) continue;
                 *reinterpret_cast<uint4 *>(obase + oo + ch * 8) = *stage_chunk<ROWB>(stage, rl, ch);
             }
             __syncwarp(); // staging free for the next tile

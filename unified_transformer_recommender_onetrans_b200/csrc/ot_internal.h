@@ -8,6 +8,26 @@
 
 namespace ot {
 
+// Device bounds checks of the checked build (compiled with OT_DEVICE_CHECKS):
+// a plain global access of n bytes at byte offset off from a buffer whose
+// extent from that base is cap bytes (0: not known, not checked) is made
+// only inside the extent; otherwise the model's error word gets
+// OT_ERR_DEVICE_BOUNDS and the access is skipped.  The release build
+// compiles every check away.
+#ifdef OT_DEVICE_CHECKS
+constexpr bool kDeviceChecks = true;
+#else
+constexpr bool kDeviceChecks = false;
+#endif
+
+__device__ __forceinline__ bool ot_dev_ok(long long off, long long n, long long cap, int *err)
+{
+    if (!kDeviceChecks || cap <= 0) return true;
+    if (off >= 0 && off + n <= cap) return true;
+    if (err) atomicCAS(err, 0, OT_ERR_DEVICE_BOUNDS);
+    return false;
+}
+
 // Bounded-wait control passed to every kernel that waits on device state.
 struct WaitCtl {
     int *err;         // model error word (device)
@@ -54,6 +74,7 @@ struct EpiSeg {
     const int *pages;
     long long pg_ustride, n_pages;
     int pg_off, pg_kv;
+    long long cap; // bytes from out to the end of its buffer (checked build; 0: unknown)
 };
 
 // Row of the page pool for GEMM row r of a paged segment; -1 when the page
@@ -97,6 +118,7 @@ struct GemmArgs {
     const void *res;
     long long res_ld;
     RowMap res_map;
+    long long res_cap;  // bytes from res to the end of its buffer (checked build; 0: unknown)
     WaitCtl wait;
 };
 
@@ -128,6 +150,7 @@ struct AttnArgs {
     long long s_ustride; // elements between users in KS / VS
     const void *KN, *VN;
     void *O;            // [U][nq][d]
+    long long o_cap;    // bytes from O to the end of its buffer (checked build; 0: unknown)
     float scale;        // 1/sqrt(hd)
     int dtype;
     WaitCtl wait;

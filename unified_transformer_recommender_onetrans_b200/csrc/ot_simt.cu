@@ -102,7 +102,11 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a)
             if (c >= a.N) continue;
             float v = acc[i][j] * rs;
             if (a.gelu) v = gelu_erf(v);
-            if (a.res) v += ld_res(a.res, rowmap_apply(a.res_map, r, g) * a.res_ld + c, a.store);
+            if (a.res) {
+                const long long ri = rowmap_apply(a.res_map, r, g) * a.res_ld + c;
+                const long long esz = a.store == OT_STORE_F32 ? 4 : 2;
+                if (ot_dev_ok(ri * esz, esz, a.res_cap, a.wait.err)) v += ld_res(a.res, ri, a.store);
+            }
             for (int s = 0; s < a.nseg; ++s) {
                 const EpiSeg &sg = a.seg[s];
                 if (c < sg.c_lo || c >= sg.c_hi || !rowmap_keep(sg.map, r)) continue;
@@ -116,7 +120,8 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a)
                 } else {
                     orow = rowmap_apply(sg.map, r, g);
                 }
-                st_out(sg.out, orow * sg.ld + (c - sg.c_lo), a.store, v);
+                const long long oi = orow * sg.ld + (c - sg.c_lo), esz = a.store == OT_STORE_F32 ? 4 : 2;
+                if (ot_dev_ok(oi * esz, esz, sg.cap, a.wait.err)) st_out(sg.out, oi, a.store, v);
             }
         }
     }
@@ -245,6 +250,9 @@ __global__ void __launch_bounds__(SA_ROWS) attn_simt_kernel(AttnArgs a)
     if (!valid) return;
     float inv = 1.0f / l;
     long long orow = (static_cast<long long>(u) * a.nq + i) * a.d + h * HD;
+    if (!ot_dev_ok(orow * (a.dtype == OT_DTYPE_F32 ? 4 : 2), HD * (a.dtype == OT_DTYPE_F32 ? 4 : 2), a.o_cap,
+                   a.wait.err))
+        return;
 #pragma unroll
     for (int e = 0; e < HD; ++e) {
         if (a.dtype == OT_DTYPE_F32)
