@@ -801,6 +801,13 @@ struct EncodeRun {
         at_.KN = ns_K;
         at_.VN = ns_V;
         at_.nkn = ns_rows;
+        // FP8 with per-tensor scales: the attention writes e4m3 for the O
+        // projection (not for the fused-FFN or mixture paths, bf16 only)
+        const bool oq = fp8_fused_hidden(m) && !use_fused_ffn(m) && c.moe_experts == 0;
+        if (oq) {
+            at_.o_qscale = act_slot(m, l, 0, IN_O);
+            at_.o_qstride = 4;
+        }
         ot_status r;
         if ((r = attn(m, at_, st)) != OT_OK) return r;
         void *Xn = (last && s_out) ? s_out : Xb[l & 1];
@@ -824,10 +831,13 @@ struct EncodeRun {
         }
         // 3. O projection + residual from the tail rows of the layer input
         GemmArgs g = gemm_base(c, U * q, d, d, 1);
-        if ((r = projection(m, g, Ab, d, rowmap_identity(),
-                            at(m->Wo_s, static_cast<long long>(l) * d * d, wesz),
-                            static_cast<long long>(d) * d, fp8 ? m->sc_o_s + l : nullptr, nullptr, 0,
-                            false, f8, st, l, 0, IN_O)) != OT_OK)
+        if (oq)
+            fp8_hidden_operand(g, Ab, d, rowmap_identity(), at(m->Wo_s, static_cast<long long>(l) * d * d, wesz),
+                               static_cast<long long>(d) * d, m->sc_o_s + l, act_slot(m, l, 0, IN_O));
+        else if ((r = projection(m, g, Ab, d, rowmap_identity(),
+                                 at(m->Wo_s, static_cast<long long>(l) * d * d, wesz),
+                                 static_cast<long long>(d) * d, fp8 ? m->sc_o_s + l : nullptr, nullptr, 0,
+                                 false, f8, st, l, 0, IN_O)) != OT_OK)
             return r;
         g.res = X;
         g.res_ld = d;
@@ -1046,6 +1056,11 @@ struct ScoreRun {
         at_.KN = Kn;
         at_.VN = Vn;
         at_.nkn = C * N;
+        const bool oq = fp8_fused_hidden(m) && !use_fused_ffn(m); // e4m3 attention output for the O projection
+        if (oq) {
+            at_.o_qscale = act_slot(m, l, 1, IN_O); // NS position n: parameter set 1 + n
+            at_.o_qstride = 4;
+        }
         ot_status r;
         if ((r = attn(m, at_, st)) != OT_OK) return r;
         void *Xn = last && out ? out : Xb[l & 1];
@@ -1059,9 +1074,12 @@ struct ScoreRun {
             return OT_OK;
         }
         GemmArgs g = gemm_base(c, Mc, d, d, N);
-        if ((r = projection(m, g, An, d, gm, at(m->Wo_ns, lN * d * d, wesz),
-                            static_cast<long long>(d) * d, fp8 ? m->sc_o_ns + lN : nullptr, nullptr,
-                            0, false, f8, st, l, 1, IN_O)) != OT_OK)
+        if (oq)
+            fp8_hidden_operand(g, An, d, gm, at(m->Wo_ns, lN * d * d, wesz), static_cast<long long>(d) * d,
+                               m->sc_o_ns + lN, act_slot(m, l, 1, IN_O));
+        else if ((r = projection(m, g, An, d, gm, at(m->Wo_ns, lN * d * d, wesz),
+                                 static_cast<long long>(d) * d, fp8 ? m->sc_o_ns + lN : nullptr, nullptr,
+                                 0, false, f8, st, l, 1, IN_O)) != OT_OK)
             return r;
         g.res = X;
         g.res_ld = d;

@@ -327,8 +327,18 @@ __global__ void __launch_bounds__(NA_WARPS * 32, 2)
         out.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
         out.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
         const long long o_off = (static_cast<long long>(u) * a.nq + row) * a.d + h * NA_HD + c8 * 8;
-        if (ot_dev_ok(o_off * 2, 16, a.o_cap, a.wait.err))
+        if (a.o_qscale) {
+            // e4m3 output: the bf16 values quantised with the O projection's input scale
+            const float qi = __frcp_rn(a.o_qscale[static_cast<long long>(row % a.N) * a.o_qstride]);
+            const uint2 q8 = make_uint2(static_cast<uint32_t>(bf16x2_to_e4m3x2(out.x, qi)) |
+                                            (static_cast<uint32_t>(bf16x2_to_e4m3x2(out.y, qi)) << 16),
+                                        static_cast<uint32_t>(bf16x2_to_e4m3x2(out.z, qi)) |
+                                            (static_cast<uint32_t>(bf16x2_to_e4m3x2(out.w, qi)) << 16));
+            if (ot_dev_ok(o_off, 8, a.o_cap, a.wait.err))
+                *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(a.O) + o_off) = q8;
+        } else if (ot_dev_ok(o_off * 2, 16, a.o_cap, a.wait.err)) {
             *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.O) + o_off) = out;
+        }
     }
 }
 

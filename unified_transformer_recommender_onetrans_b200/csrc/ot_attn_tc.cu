@@ -626,7 +626,19 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             release(&o_free[w]);
             if (SPLIT) release(&o_free[1]);
             const long long o_off = (static_cast<long long>(it.u) * a.nq + i) * a.d + it.h * AT_HD;
-            if (i < a.nq && ot_dev_ok(o_off * 2, AT_HD * 2, a.o_cap, a.wait.err)) {
+            if (a.o_qscale && i < a.nq && ot_dev_ok(o_off, AT_HD, a.o_cap, a.wait.err)) {
+                // e4m3 output: the bf16 row quantised with the O projection's input scale
+                const float qi = __frcp_rn(a.o_qscale[NS ? static_cast<long long>(i % a.N) * a.o_qstride : 0]);
+                uint32_t q8[AT_HD / 4];
+#pragma unroll
+                for (int e = 0; e < AT_HD / 4; ++e)
+                    q8[e] = static_cast<uint32_t>(bf16x2_to_e4m3x2(ob[2 * e], qi)) |
+                            (static_cast<uint32_t>(bf16x2_to_e4m3x2(ob[2 * e + 1], qi)) << 16);
+                uint4 *dp = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.O) + o_off);
+#pragma unroll
+                for (int qd = 0; qd < AT_HD / 16; ++qd)
+                    dp[qd] = make_uint4(q8[4 * qd], q8[4 * qd + 1], q8[4 * qd + 2], q8[4 * qd + 3]);
+            } else if (!a.o_qscale && i < a.nq && ot_dev_ok(o_off * 2, AT_HD * 2, a.o_cap, a.wait.err)) {
                 uint4 *dp = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.O) + o_off);
 #pragma unroll
                 for (int qd = 0; qd < 8; ++qd)

@@ -1,6 +1,7 @@
 // Internal types shared by the host entry points and the kernels.
 #pragma once
 
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -77,6 +78,14 @@ struct EpiSeg {
     long long cap; // bytes from out to the end of its buffer (checked build; 0: unknown)
 };
 
+// bf16 pair (lo, hi halves of w) -> two e4m3 bytes of x / s (x * inv),
+// round to nearest even, saturating; first value in the low byte
+__device__ __forceinline__ uint16_t bf16x2_to_e4m3x2(uint32_t w, float inv)
+{
+    const float2 f = make_float2(__uint_as_float(w << 16) * inv, __uint_as_float(w & 0xFFFF0000u) * inv);
+    return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3));
+}
+
 // Row of the page pool for GEMM row r of a paged segment; -1 when the page
 // id is outside [0, n_pages) (the caller skips the store and reports it).
 __host__ __device__ inline long long paged_row(const EpiSeg &s, long long r)
@@ -151,6 +160,10 @@ struct AttnArgs {
     const void *KN, *VN;
     void *O;            // [U][nq][d]
     long long o_cap;    // bytes from O to the end of its buffer (checked build; 0: unknown)
+    // e4m3 output (FP8 models with per-tensor scales): O holds e4m3(o / s),
+    // s = o_qscale[0] for S rows, o_qscale[(i % N) * o_qstride] for NS row i
+    const float *o_qscale;
+    long long o_qstride;
     float scale;        // 1/sqrt(hd)
     int dtype;
     WaitCtl wait;
