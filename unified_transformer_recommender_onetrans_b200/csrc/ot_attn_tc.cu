@@ -54,27 +54,41 @@
 namespace ot {
 
 constexpr int AT_BM = 128;  // query rows per tile
-constexpr int AT_TILES = 2; // tiles per CTA
 constexpr int AT_BK = 128;  // keys per block
 constexpr int AT_HD = 64;
 constexpr uint32_t AT_TILE = AT_BM * 128; // 16 KB: 128 rows x 128 bytes
-constexpr int AT_STAGES = 5;              // K/V ring depth
 constexpr int AT_QBUF = 2;                // Q buffers (items in flight)
-// Q[AT_QBUF][AT_TILES], then per stage K and V, then barriers, then the
+// Q[AT_QBUF][TILES], then per stage K and V, then barriers, then the
 // split-key exchange (tile 1's running max and sum per row)
 constexpr size_t AT_BAR_BYTES = 256;
 constexpr size_t AT_XCH_BYTES = AT_BM * 2 * sizeof(float);
-constexpr size_t AT_SMEM = (AT_QBUF * AT_TILES + 2 * AT_STAGES) * AT_TILE + AT_BAR_BYTES + AT_XCH_BYTES;
-static_assert((2 * AT_QBUF + 2 * AT_STAGES + 6 * AT_TILES + 1) * 8 + 8 <= AT_BAR_BYTES, "barrier area");
-static_assert(AT_SMEM <= 227 * 1024, "shared memory per CTA");
-constexpr int AT_THREADS = 128 * (1 + AT_TILES); // producer warpgroup + one softmax warpgroup per tile
-// Register split (setmaxnreg): the producer warpgroup (TMA warp, MMA warp, two
-// idle warps) drops to AT_REG_PRODUCER per thread and the softmax warpgroups
-// rise to AT_REG_SOFTMAX, which holds a row's 128 scores at once.  The sum
-// must stay within what the launch allocated (registers per thread x
-// AT_THREADS); the launcher checks it against the compiled kernel.
-constexpr int AT_REG_PRODUCER = 64;
-constexpr int AT_REG_SOFTMAX = 216;
+
+// Two shapes of the persistent kernel:
+//   TILES = 2  one CTA per SM with two 128-row query tiles (all 512 TMEM
+//              columns), a 5-deep K/V ring shared by both tiles; the NS
+//              modes (split-key items need both tiles on the same rows);
+//   TILES = 1  two CTAs per SM, one tile each (256 TMEM columns, a 2-deep
+//              ring per CTA): the two tiles of an SM run independent
+//              pipelines and drift out of step, so one softmax warpgroup's
+//              exponentials overlap the other's waits (S attention of the
+//              OneTransS layer 0: 0.140 -> 0.133 ms against TILES = 2).
+// Register split (setmaxnreg): the producer warpgroup (TMA warp, MMA warps,
+// idle warps) drops to REG_PRODUCER per thread and the softmax warpgroups
+// rise to REG_SOFTMAX, which holds a row's 128 scores at once.  The sum must
+// stay within what the launch allocated (registers per thread x THREADS);
+// the launcher checks it against the compiled kernel.
+template <int TILES> struct AtCfg {
+    static_assert(TILES == 1 || TILES == 2, "one or two tiles per CTA");
+    static constexpr int STAGES = TILES == 1 ? 2 : 5;       // K/V ring depth
+    static constexpr int CTAS = TILES == 1 ? 2 : 1;         // CTAs per SM
+    static constexpr int THREADS = 128 * (1 + TILES);       // producer warpgroup + a softmax warpgroup per tile
+    static constexpr int REG_PRODUCER = TILES == 1 ? 40 : 64;
+    static constexpr int REG_SOFTMAX = 216;
+    static constexpr size_t SMEM = (AT_QBUF * TILES + 2 * STAGES) * AT_TILE + AT_BAR_BYTES + AT_XCH_BYTES;
+    static_assert((2 * AT_QBUF + 2 * STAGES + 6 * TILES + 1) * 8 + 8 <= AT_BAR_BYTES, "barrier area");
+    static_assert(CTAS * (SMEM + 1024) <= 228 * 1024, "shared memory per SM");
+    static_assert(128 * REG_PRODUCER + 128 * TILES * REG_SOFTMAX <= 65536 / CTAS, "register split");
+};
 
 // Lazy rescale threshold (base-2): the running max moves only when it would
 // grow by more than 2^8; until then p <= 2^8, well inside fp32 / bf16 range.
@@ -156,13 +170,16 @@ struct AtItem {
 
 // Query rows per item: two tiles of 128, or one in split-key mode, where
 // both tiles of the CTA work on the same rows.
-template <bool SPLIT> __host__ __device__ constexpr int at_item_rows() { return SPLIT ? AT_BM : AT_BM * AT_TILES; }
+template <bool SPLIT, int TILES> __host__ __device__ constexpr int at_item_rows()
+{
+    return SPLIT ? AT_BM : AT_BM * TILES;
+}
 
 // Item k.  S mode orders the pairs longest first (pairs later in the tail see
 // more keys), so the snake assignment below balances the CTAs; NS mode keeps
 // the pairs (row tiles in split-key mode) of one (user, head) together so
 // they share K/V tiles in L2.
-template <bool NS, bool SPLIT, bool FA>
+template <bool NS, bool SPLIT, bool FA, int TILES>
 __device__ __forceinline__ AtItem at_item(const AttnArgs &a, int n_pairs, int k)
 {
     AtItem it;
@@ -177,8 +194,8 @@ __device__ __forceinline__ AtItem at_item(const AttnArgs &a, int n_pairs, int k)
     }
     it.u = uh / a.H;
     it.h = uh % a.H;
-    it.i0 = pair * at_item_rows<SPLIT>();
-    const int i_last = min(it.i0 + at_item_rows<SPLIT>(), a.nq) - 1;
+    it.i0 = pair * at_item_rows<SPLIT, TILES>();
+    const int i_last = min(it.i0 + at_item_rows<SPLIT, TILES>(), a.nq) - 1;
     it.k_begin = 0;
     if (!NS) {
         // causal: the keys up to the item's last row; full attention: every
@@ -210,7 +227,7 @@ __device__ __forceinline__ int at_item_of(int r, int n_items)
 // items of one 128-row tile), where tile w takes the blocks b = w (mod 2) of
 // an item and the two tiles' partial softmax states are merged at its end.
 // gb counts all blocks of the CTA (the K/V ring position), lb this tile's.
-template <bool NS, bool SPLIT, bool FA>
+template <bool NS, bool SPLIT, bool FA, int TILES>
 struct BlockCursor {
     int r, k;      // item ordinal within the CTA, item index (k < 0: past the end)
     AtItem it;
@@ -225,7 +242,7 @@ struct BlockCursor {
         if (++b < it.n_blocks) return;
         b = 0;
         k = at_item_of(++r, n_items);
-        if (k >= 0) it = at_item<NS, SPLIT, FA>(a, n_pairs, k);
+        if (k >= 0) it = at_item<NS, SPLIT, FA, TILES>(a, n_pairs, k);
     }
     __device__ __forceinline__ void init(const AttnArgs &a, int n_pairs, int n_items, int tile)
     {
@@ -235,7 +252,7 @@ struct BlockCursor {
         gb = 0;
         lb = 0;
         k = at_item_of(0, n_items);
-        if (k >= 0) it = at_item<NS, SPLIT, FA>(a, n_pairs, k);
+        if (k >= 0) it = at_item<NS, SPLIT, FA, TILES>(a, n_pairs, k);
         while (valid() && !owned()) step(a, n_pairs, n_items);
     }
     __device__ __forceinline__ void next(const AttnArgs &a, int n_pairs, int n_items)
@@ -252,8 +269,8 @@ struct BlockCursor {
     }
 };
 
-template <bool NS, bool SPLIT, bool FA>
-__global__ void __launch_bounds__(AT_THREADS, 1)
+template <bool NS, bool SPLIT, bool FA, int TILES>
+__global__ void __launch_bounds__(AtCfg<TILES>::THREADS, AtCfg<TILES>::CTAS)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKS,
                    const __grid_constant__ CUtensorMap tmVS, const __grid_constant__ CUtensorMap tmKN,
                    const __grid_constant__ CUtensorMap tmVN, const __grid_constant__ AttnArgs a)
@@ -262,6 +279,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     constexpr uint32_t IDESC_O = make_idesc(128, 64, 1, 0, 1);
 
     extern __shared__ __align__(1024) uint8_t smem[];
+    constexpr int AT_TILES = TILES, AT_STAGES = AtCfg<TILES>::STAGES;
     uint8_t *sQ = smem;                                  // [AT_QBUF][AT_TILES]
     uint8_t *sKV = smem + AT_QBUF * AT_TILES * AT_TILE;  // [stage][K | V]
     uint64_t *bars = reinterpret_cast<uint64_t *>(sKV + 2 * AT_STAGES * AT_TILE);
@@ -281,7 +299,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     float *xch = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + AT_BAR_BYTES); // [2][AT_BM]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_pairs = (a.nq + at_item_rows<SPLIT>() - 1) / at_item_rows<SPLIT>();
+    const int n_pairs = (a.nq + at_item_rows<SPLIT, TILES>() - 1) / at_item_rows<SPLIT, TILES>();
     const int n_items = n_pairs * a.U * a.H;
     pdl_launch_dependents();
 
@@ -311,7 +329,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 512);
+        tmem_alloc(tmem_slot, 256 * AT_TILES);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -326,7 +344,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 
     if (warp < 4) {
         // producer warpgroup: hand registers to the softmax warpgroups
-        setmaxnreg_dec<AT_REG_PRODUCER>();
+        setmaxnreg_dec<AtCfg<TILES>::REG_PRODUCER>();
     }
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -344,7 +362,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             for (; ok; ++r) {
                 const int k = at_item_of(r, n_items);
                 if (k < 0) break;
-                const AtItem it = at_item<NS, SPLIT, FA>(a, n_pairs, k);
+                const AtItem it = at_item<NS, SPLIT, FA, TILES>(a, n_pairs, k);
                 const int qb = r & 1;
                 // the Q buffer of item r - 2 is free once all its S MMAs completed
                 if (!mbar_wait(&q_empty[qb], ((r >> 1) & 1) ^ 1, a.wait, abort_flag)) break;
@@ -389,7 +407,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 mbar_wait(&kv_full[j % AT_STAGES], static_cast<uint32_t>((j / AT_STAGES) & 1),
                           final_wait, &no_abort);
         }
-    } else if (warp == 1 || warp == 2) {
+    } else if (warp >= 1 && warp <= AT_TILES) {
         // ------------------------------------------------ MMA issuer of tile w
         // Issued from one thread, a short tcgen05.mma takes about 100 cycles:
         // one issuer per tile keeps both tiles' MMAs flowing.  Per key block:
@@ -400,7 +418,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         if (lane == 0 && !aborted_at_start) {
             const uint32_t tS = tmem + w * 256, tP = tS + 128, tO = tS + 192;
             auto live = [&](const AtItem &it) { return SPLIT || it.i0 + w * AT_BM < a.nq; };
-            auto issue_s = [&](const BlockCursor<NS, SPLIT, FA> &c) {
+            auto issue_s = [&](const BlockCursor<NS, SPLIT, FA, TILES> &c) {
                 if (live(c.it)) {
                     const uint32_t q_addr = smem_u32(sQ + ((c.r & 1) * AT_TILES + (SPLIT ? 0 : w)) * AT_TILE);
                     const uint32_t k_addr = smem_u32(sKV + 2 * (c.gb % AT_STAGES) * AT_TILE);
@@ -413,12 +431,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 // the item's last S of this tile: its Q buffer is free once they completed
                 if (c.last_in_item()) mma_commit(&q_empty[c.r & 1]);
             };
-            auto ready_s = [&](const BlockCursor<NS, SPLIT, FA> &c) {
+            auto ready_s = [&](const BlockCursor<NS, SPLIT, FA, TILES> &c) {
                 return mbar_wait(&kv_full[c.gb % AT_STAGES], static_cast<uint32_t>((c.gb / AT_STAGES) & 1),
                                  a.wait, abort_flag) &&
                        mbar_wait(&q_full[c.r & 1], (c.r >> 1) & 1, a.wait, abort_flag);
             };
-            BlockCursor<NS, SPLIT, FA> cur;
+            BlockCursor<NS, SPLIT, FA, TILES> cur;
             cur.init(a, n_pairs, n_items, w);
             bool run = cur.valid() && ready_s(cur);
             if (run) {
@@ -426,7 +444,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 issue_s(cur);
             }
             while (run) {
-                BlockCursor<NS, SPLIT, FA> nxt = cur;
+                BlockCursor<NS, SPLIT, FA, TILES> nxt = cur;
                 nxt.next(a, n_pairs, n_items);
                 if (nxt.valid()) {
                     if (!mbar_wait(&s_free[w], static_cast<uint32_t>(cur.lb & 1), a.wait, abort_flag) ||
@@ -466,7 +484,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         }
     } else if (warp >= 4) {
         // ------------------------------------------------ softmax warpgroups
-        setmaxnreg_inc<AT_REG_SOFTMAX>();
+        setmaxnreg_inc<AtCfg<TILES>::REG_SOFTMAX>();
         const int w = (warp - 4) >> 2;         // tile of this warpgroup
         const int quarter = warp & 3;          // TMEM lane quarter
         const int row = quarter * 32 + lane;   // row within the tile
@@ -493,7 +511,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         for (int r = 0; ok; ++r) {
             const int k = at_item_of(r, n_items);
             if (k < 0) break;
-            const AtItem it = at_item<NS, SPLIT, FA>(a, n_pairs, k);
+            const AtItem it = at_item<NS, SPLIT, FA, TILES>(a, n_pairs, k);
             const int i = it.i0 + (SPLIT ? 0 : w * AT_BM) + row; // query row within the user
             const bool warp_dead = __all_sync(0xffffffffu, i >= a.nq);
             const int t_self = a.L - a.nq + i;      // S mode
@@ -650,7 +668,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, 256 * AT_TILES);
     }
 }
 
@@ -716,35 +734,40 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
     bool split = false;
     if (a.mode == 1 && a.L >= 1 && a.N >= 1) {
         const long long uh = static_cast<long long>(a.U) * a.H;
-        const long long items2 = uh * ((a.nq + AT_BM * AT_TILES - 1) / (AT_BM * AT_TILES));
+        const long long items2 = uh * ((a.nq + AT_BM * 2 - 1) / (AT_BM * 2));
         const long long items1 = uh * ((a.nq + AT_BM - 1) / AT_BM);
-        const long long t2 = (items2 + num_sms - 1) / num_sms * (key_blocks(AT_BM * AT_TILES) + 1);
+        const long long t2 = (items2 + num_sms - 1) / num_sms * (key_blocks(AT_BM * 2) + 1);
         const long long t1 = (items1 + num_sms - 1) / num_sms * ((key_blocks(AT_BM) + 1) / 2 + 1);
         split = a.nq <= AT_BM || t1 * 10 < t2 * 9;
     }
-    const int rows = split ? AT_BM : AT_BM * AT_TILES;
+    // S mode: one tile per CTA, two CTAs per SM; NS modes: two tiles per CTA
+    const int tiles = a.mode == 1 ? 2 : 1;
+    const int rows = split ? AT_BM : AT_BM * tiles;
     const long long items = static_cast<long long>((a.nq + rows - 1) / rows) * a.H * a.U;
     if (items < 1 || items > (1LL << 30)) return cudaErrorInvalidValue;
-    dim3 grid(static_cast<unsigned>(items < num_sms ? items : num_sms));
-    auto run = [&](auto kernel) -> cudaError_t {
+    auto run = [&](auto kernel, auto cfg) -> cudaError_t {
+        using Cfg = decltype(cfg);
+        const long long slots = static_cast<long long>(num_sms) * Cfg::CTAS;
+        const dim3 grid(static_cast<unsigned>(items < slots ? items : slots));
         // the setmaxnreg split must fit the registers the launch allocates,
         // or the softmax warpgroups' increase would wait forever
         cudaFuncAttributes fa;
         cudaError_t err = cudaFuncGetAttributes(&fa, kernel);
         if (err != cudaSuccess) return err;
-        if (128 * AT_REG_PRODUCER + 128 * AT_TILES * AT_REG_SOFTMAX > fa.numRegs * AT_THREADS)
+        if (128 * Cfg::REG_PRODUCER + 128 * (Cfg::THREADS / 128 - 1) * Cfg::REG_SOFTMAX > fa.numRegs * Cfg::THREADS)
             return cudaErrorInvalidConfiguration;
-        err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(AT_SMEM));
+        err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cfg::SMEM));
         if (err != cudaSuccess) return err;
-        return launch_pdl(kernel, grid, dim3(AT_THREADS), AT_SMEM, s, tq, tks, tvs, tkn, tvn, a);
+        return launch_pdl(kernel, grid, dim3(Cfg::THREADS), Cfg::SMEM, s, tq, tks, tvs, tkn, tvn, a);
     };
     if (a.full) {
-        if (a.mode != 1) return run(attn_tc_kernel<false, false, true>);
-        return split ? run(attn_tc_kernel<true, true, true>) : run(attn_tc_kernel<true, false, true>);
+        if (a.mode != 1) return run(attn_tc_kernel<false, false, true, 1>, AtCfg<1>{});
+        return split ? run(attn_tc_kernel<true, true, true, 2>, AtCfg<2>{})
+                     : run(attn_tc_kernel<true, false, true, 2>, AtCfg<2>{});
     }
-    if (a.mode != 1) return run(attn_tc_kernel<false, false, false>);
-    return split ? run(attn_tc_kernel<true, true, false>) : run(attn_tc_kernel<true, false, false>);
+    if (a.mode != 1) return run(attn_tc_kernel<false, false, false, 1>, AtCfg<1>{});
+    return split ? run(attn_tc_kernel<true, true, false, 2>, AtCfg<2>{})
+                 : run(attn_tc_kernel<true, false, false, 2>, AtCfg<2>{});
 }
 
 } // namespace ot
