@@ -41,9 +41,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 CAPTURED_TRAFFIC = {
     # kernel kind -> (source file, its sha256 at capture time, bytes per step, launches per step)
     # attn_tc: ncu dram__bytes_read.sum + dram__bytes_write.sum of the six S-attention launches
-    # of one onetrans_s_full step (536.4 MB read + 28.1 MB written)
-    "attn_tc": ("ot_attn_tc.cu", "461593d2e34f6b400d16785f42674a5f36e7215f3f5a4d8c54b23e6b7a6be733",
-                564471552, 6),
+    # of one onetrans_s_full step (655.0 MB read + 35.6 MB written)
+    "attn_tc": ("ot_attn_tc.cu", "55e776cf0e51e48953ffd861f5977b32d7ae13627f8173719350a5a906ff1cfc",
+                690605312, 6),
 }
 
 
