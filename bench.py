@@ -41,9 +41,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 CAPTURED_TRAFFIC = {
     # kernel kind -> (source file, its sha256 at capture time, bytes per step, launches per step)
     # attn_tc: ncu dram__bytes_read.sum + dram__bytes_write.sum of the six S-attention launches
-    # of one onetrans_s_full step (655.0 MB read + 35.6 MB written)
-    "attn_tc": ("ot_attn_tc.cu", "55e776cf0e51e48953ffd861f5977b32d7ae13627f8173719350a5a906ff1cfc",
-                690605312, 6),
+    # of one onetrans_s_full step (653.5 MB read + 35.3 MB written)
+    "attn_tc": ("ot_attn_tc.cu", "f7f088a65ddb4a12fb1aa96b20d829ba13650d3158db9ec3244588d6f2002d6d",
+                688931328, 6),
 }
 
 

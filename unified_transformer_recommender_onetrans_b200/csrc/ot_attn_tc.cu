@@ -65,13 +65,16 @@ constexpr size_t AT_XCH_BYTES = AT_BM * 2 * sizeof(float);
 
 // Two shapes of the persistent kernel:
 //   TILES = 2  one CTA per SM with two 128-row query tiles (all 512 TMEM
-//              columns), a 5-deep K/V ring shared by both tiles; the NS
-//              modes (split-key items need both tiles on the same rows);
+//              columns), a 5-deep K/V ring shared by both tiles; split-key
+//              NS items (their two tiles share the key blocks of one row
+//              tile);
 //   TILES = 1  two CTAs per SM, one tile each (256 TMEM columns, a 2-deep
-//              ring per CTA): the two tiles of an SM run independent
-//              pipelines and drift out of step, so one softmax warpgroup's
-//              exponentials overlap the other's waits (S attention of the
-//              OneTransS layer 0: 0.140 -> 0.133 ms against TILES = 2).
+//              ring per CTA): S items and the other NS items.  The two
+//              tiles of an SM run independent pipelines and drift out of
+//              step, so one softmax warpgroup's exponentials overlap the
+//              other's waits (OneTransS layer-0 S attention 0.140 -> 0.132
+//              ms, NS attention of 16 x 512 candidates 1.755 -> 1.714 ms
+//              against TILES = 2).
 // Register split (setmaxnreg): the producer warpgroup (TMA warp, MMA warps,
 // idle warps) drops to REG_PRODUCER per thread and the softmax warpgroups
 // rise to REG_SOFTMAX, which holds a row's 128 scores at once.  The sum must
@@ -740,8 +743,9 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
         const long long t1 = (items1 + num_sms - 1) / num_sms * ((key_blocks(AT_BM) + 1) / 2 + 1);
         split = a.nq <= AT_BM || t1 * 10 < t2 * 9;
     }
-    // S mode: one tile per CTA, two CTAs per SM; NS modes: two tiles per CTA
-    const int tiles = a.mode == 1 ? 2 : 1;
+    // split-key NS items: two tiles per CTA; everything else one tile per
+    // CTA, two CTAs per SM
+    const int tiles = (a.mode == 1 && split) ? 2 : 1;
     const int rows = split ? AT_BM : AT_BM * tiles;
     const long long items = static_cast<long long>((a.nq + rows - 1) / rows) * a.H * a.U;
     if (items < 1 || items > (1LL << 30)) return cudaErrorInvalidValue;
@@ -763,11 +767,11 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
     if (a.full) {
         if (a.mode != 1) return run(attn_tc_kernel<false, false, true, 1>, AtCfg<1>{});
         return split ? run(attn_tc_kernel<true, true, true, 2>, AtCfg<2>{})
-                     : run(attn_tc_kernel<true, false, true, 2>, AtCfg<2>{});
+                     : run(attn_tc_kernel<true, false, true, 1>, AtCfg<1>{});
     }
     if (a.mode != 1) return run(attn_tc_kernel<false, false, false, 1>, AtCfg<1>{});
     return split ? run(attn_tc_kernel<true, true, false, 2>, AtCfg<2>{})
-                 : run(attn_tc_kernel<true, false, false, 2>, AtCfg<2>{});
+                 : run(attn_tc_kernel<true, false, false, 1>, AtCfg<1>{});
 }
 
 } // namespace ot
