@@ -570,6 +570,10 @@ struct Backward {
     float *Zp, *U1e, *Acte, *Ye, *dYe, *dActe, *dZp, *logits, *dlogits;
     static constexpr long long kTnPartialFloats = 2LL * 296 * 128 * 128;
     float *dXbuf[2], *dYbuf[2];
+    // attention outputs and softmax statistics of every layer, kept from the
+    // checkpointing forward: the per-layer recompute skips the attention
+    float *sA[OT_MAX_LAYERS], *sM[OT_MAX_LAYERS], *sL[OT_MAX_LAYERS];
+    float *nA[OT_MAX_LAYERS], *nM[OT_MAX_LAYERS], *nL[OT_MAX_LAYERS];
     const float *G_s, *G_ns;
     float *dS, *dns;
     size_t bytes;
@@ -611,7 +615,6 @@ struct Backward {
             x.r1 = cv.take(rows);
             x.Z1 = cv.take(rows * d);
             x.QKV = cv.take(rows * 3 * d);
-            x.A = cv.take(tail * d);
             x.H = cv.take(tail * d);
             x.r2 = cv.take(tail);
             x.Z2 = cv.take(tail * d);
@@ -623,12 +626,20 @@ struct Backward {
             x.dA = cv.take(tail * d);
             x.dQKV = cv.take(rows * 3 * d);
             x.dZ1 = cv.take(rows * d);
-            x.sm = cv.take(tail * H);
-            x.sl = cv.take(tail * H);
             x.sD = cv.take(tail * H);
         };
         side(s, R, Tq);
         if (C) side(n, RN_, RN_);
+        for (int l = 0; l < Lyr; ++l) {
+            sA[l] = cv.take(T(l) * d);
+            sM[l] = cv.take(T(l) * H);
+            sL[l] = cv.take(T(l) * H);
+            if (C) {
+                nA[l] = cv.take(RN_ * d);
+                nM[l] = cv.take(RN_ * H);
+                nL[l] = cv.take(RN_ * H);
+            }
+        }
         if (E) {
             const long long P = Tq * K;
             auto ints = [&](long long cnt) { return reinterpret_cast<int *>(cv.take(cnt)); };
@@ -745,9 +756,13 @@ struct Backward {
         if (p.splits > 1) ++launches; // the split-order reduction
     }
 
-    // Recompute layer l (both sides); with s_out / n_out also its output rows.
-    void forward(int l, float *s_out, float *n_out)
+    // Layer l forward (both sides); with s_out / n_out also its output rows.
+    // The checkpointing pass runs the attention and keeps its outputs and
+    // statistics; the recompute (recompute = true) reuses them.
+    void forward(int l, float *s_out, float *n_out, bool recompute = false)
     {
+        s.A = sA[l], s.sm = sM[l], s.sl = sL[l];
+        if (C) n.A = nA[l], n.sm = nM[l], n.sl = nL[l];
         const int L = Ls[l], q = c.q[l];
         const long long R = RS(l), Tq = T(l);
         const long long d3 = 3LL * d, fd = static_cast<long long>(f) * d, dd = static_cast<long long>(d) * d;
@@ -767,7 +782,7 @@ struct Backward {
         }
         // ---- S side
         const BwAttn sa = attn_s(l);
-        k([&] { return bw_attn_fwd(sa, st); });
+        if (!recompute) k([&] { return bw_attn_fwd(sa, st); });
         if (!dry && err == cudaSuccess)
             err = cudaMemcpy2DAsync(s.H, static_cast<size_t>(q) * d * 4, X[l] + static_cast<long long>(L - q) * d,
                                     static_cast<size_t>(L) * d * 4, static_cast<size_t>(q) * d * 4, U,
@@ -789,7 +804,7 @@ struct Backward {
         if (!C) return;
         // ---- NS side
         const BwAttn na = attn_ns(l);
-        k([&] { return bw_attn_fwd(na, st); });
+        if (!recompute) k([&] { return bw_attn_fwd(na, st); });
         copy(n.H, Y[l], static_cast<size_t>(RN_) * d * 4);
         nt(n.A, d, nm, wt(w->Wo_ns, ln * dd), dd, n.H, d, nm, M, d, d, N, 1);
         const BwRows h2n{n.H, nm, M, N, d};
@@ -948,7 +963,7 @@ struct Backward {
         }
         // backward, top layer first (its intermediates are still in place)
         for (int l = Lyr - 1; l >= 0; --l) {
-            if (l != Lyr - 1) forward(l, nullptr, nullptr);
+            if (l != Lyr - 1) forward(l, nullptr, nullptr, true);
             const float *dXin = l == Lyr - 1 ? G_s : dXbuf[(l + 1) & 1];
             float *dXout = (l == 0 && dS) ? dS : dXbuf[l & 1];
             const float *dYin = !C ? nullptr : (l == Lyr - 1 ? G_ns : dYbuf[(l + 1) & 1]);
