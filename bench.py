@@ -44,6 +44,10 @@ CAPTURED_TRAFFIC = {
     # of one onetrans_s_full step (653.5 MB read + 35.3 MB written)
     "attn_tc": ("ot_attn_tc.cu", "f7f088a65ddb4a12fb1aa96b20d829ba13650d3158db9ec3244588d6f2002d6d",
                 688931328, 6),
+    # ffn_tc: the six fused O-projection + FFN launches of one onetrans_s_full step
+    # (363.4 MB read + 20.6 MB written)
+    "ffn_tc": ("ot_ffn_tc.cu", "675fae658dab54517d2954da43f31073cedb641fd3c4be7f406e1fea356bc07d",
+               383966464, 6),
 }
 
 
@@ -864,6 +868,23 @@ def run_ours(args, wl):
                 "peak_source": f"{peaks['_source']} bf16 dense burst",
                 "launches_per_step": dk["launches"] / prof_steps,
                 "algorithmic_tflop_per_step": dk["flops"] / prof_steps / 1e12}
+    # The S attention at head_dim 64 needs one exponential per visible (query,
+    # key) pair against 4 * 64 FLOPs: on B200 the special-function unit (16
+    # exp2 per clock per SM) is slower than the tensor core at that ratio, so
+    # its exponential rate is the kernel's binding roofline.
+    sa = by_role.get("S_attn")
+    if sa and sa["ms"] > 0:
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        mhz = clk.get("sm_max_mhz") or 1965.0
+        exp_peak = 16 * sms * mhz * 1e6
+        exps = sa["flops"] / (4 * 64)
+        roofline["s_attention_exp"] = {
+            "bound": "sfu", "achieved": exps / (sa["ms"] / 1e3), "peak": exp_peak, "unit": "exp2/s",
+            "frac": exps / (sa["ms"] / 1e3) / exp_peak,
+            "peak_source": f"16 exp2 per clock per SM x {sms} SMs x {mhz:.0f} MHz",
+            "exps_per_step": exps / prof_steps,
+            "tensor_floor_ms": sa["flops"] / prof_steps / (peak_tf * 1e12) * 1e3,
+            "exp_floor_ms": exps / prof_steps / exp_peak * 1e3}
     step_flops = sum(v["flops"] for v in by_kind.values()) / prof_steps
     kernels = {k: {"ms_per_step": v["ms"] / prof_steps,
                    "share": v["ms"] / max(sum(x["ms"] for x in by_kind.values()), 1e-9),
