@@ -348,8 +348,12 @@ def _score_point(m, wl, U, C, x, kv, steps, flush, world, dist, dev, peaks, tens
     # GEMMs at the GEMM dtype's peak, attention (always bf16) at the bf16 peak
     t_tc = gemm_flops / (tensor_peak["gemm"] * 1e12) + \
         (flops - gemm_flops) / (tensor_peak["attn"] * 1e12)
+    roles = {}
+    for r in recs:
+        roles[r["role"]] = roles.get(r["role"], 0.0) + r["ms"]
     return {
         "cands": C,
+        "roles_ms_profiled": roles,
         "candidates_per_s": world * U * C / (ms / 1e3),
         "ms": ms,
         "tflops": flops / (ms / 1e3) / 1e12,

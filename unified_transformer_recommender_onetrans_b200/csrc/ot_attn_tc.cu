@@ -31,7 +31,9 @@
 //               goes into the S columns, overlapping the exponentials; once
 //               P(b) is stored, O += P(b) V (8 MMAs, P from TMEM, V MN-major
 //               from its row-major tile).  A tile with no live query row gets
-//               no MMAs, only the signals.
+//               no MMAs, only the signals.  With one tile per CTA (two
+//               CTAs per SM, see AtCfg) warp 1 issues the S MMAs and warp 2
+//               the PV MMAs.
 //   warp 3      idle (it completes the producer warpgroup, whose registers
 //               go to the softmax warpgroups through setmaxnreg).
 //   warps 4-7   softmax warpgroup of tile 0, warps 8-11 of tile 1: one query
@@ -88,7 +90,7 @@ template <int TILES> struct AtCfg {
     static constexpr int REG_PRODUCER = TILES == 1 ? 40 : 64;
     static constexpr int REG_SOFTMAX = 216;
     static constexpr size_t SMEM = (AT_QBUF * TILES + 2 * STAGES) * AT_TILE + AT_BAR_BYTES + AT_XCH_BYTES;
-    static_assert((2 * AT_QBUF + 2 * STAGES + 6 * TILES + 1) * 8 + 8 <= AT_BAR_BYTES, "barrier area");
+    static_assert((2 * AT_QBUF + 2 * STAGES + 6 * TILES + 2) * 8 + 8 <= AT_BAR_BYTES, "barrier area");
     static_assert(CTAS * (SMEM + 1024) <= 228 * 1024, "shared memory per SM");
     static_assert(128 * REG_PRODUCER + 128 * TILES * REG_SOFTMAX <= 65536 / CTAS, "register split");
 };
@@ -295,8 +297,8 @@ __global__ void __launch_bounds__(AtCfg<TILES>::THREADS, AtCfg<TILES>::CTAS)
     uint64_t *p_full = s_free + AT_TILES;          // [tile] P stored
     uint64_t *o_full = p_full + AT_TILES;          // [tile] PV completed
     uint64_t *o_free = o_full + AT_TILES;          // [tile] O read out (end of an item)
-    uint64_t *mma_done = o_free + AT_TILES;        // [tile]
-    uint64_t *x_full = mma_done + AT_TILES;        // split-key: tile 1's state is in xch
+    uint64_t *mma_done = o_free + AT_TILES;        // [tile + 1] per issuing thread
+    uint64_t *x_full = mma_done + AT_TILES + 1;    // split-key: tile 1's state is in xch
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(x_full + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     float *xch = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + AT_BAR_BYTES); // [2][AT_BM]
@@ -323,6 +325,7 @@ __global__ void __launch_bounds__(AtCfg<TILES>::THREADS, AtCfg<TILES>::CTAS)
             mbar_init(&o_free[i], 4);
             mbar_init(&mma_done[i], 1);
         }
+        mbar_init(&mma_done[AT_TILES], 1);
         mbar_init(x_full, AT_BM);
         *abort_flag = 0;
         if (smem_u32(smem) & 1023) { // swizzle atoms need a 1024-byte aligned base
@@ -410,14 +413,21 @@ __global__ void __launch_bounds__(AtCfg<TILES>::THREADS, AtCfg<TILES>::CTAS)
                 mbar_wait(&kv_full[j % AT_STAGES], static_cast<uint32_t>((j / AT_STAGES) & 1),
                           final_wait, &no_abort);
         }
-    } else if (warp >= 1 && warp <= AT_TILES) {
-        // ------------------------------------------------ MMA issuer of tile w
-        // Issued from one thread, a short tcgen05.mma takes about 100 cycles:
-        // one issuer per tile keeps both tiles' MMAs flowing.  Per key block:
-        // once the softmax has S(b) in registers (s_free), S(b+1) = Q K^T goes
-        // into the S columns, so it runs while P(b) is being computed; then,
-        // once P(b) is stored (p_full), O += P(b) V.
-        const int w = warp - 1;
+    } else if (warp >= 1 && warp <= (TILES == 1 ? 2 : AT_TILES)) {
+        // ------------------------------------------------ MMA issuers
+        // Issued from one thread, a short tcgen05.mma takes about 100 cycles.
+        // Per key block: once the softmax has S(b) in registers (s_free),
+        // S(b+1) = Q K^T goes into the S columns, so it runs while P(b) is
+        // being computed; once P(b) is stored (p_full), O += P(b) V.
+        //   TILES = 2: warp 1 + w issues both for tile w (one issuer per tile
+        //              keeps both tiles' MMAs flowing);
+        //   TILES = 1: warp 1 issues the S MMAs, warp 2 the PV MMAs, so PV(b)
+        //              goes out as soon as P(b) is stored instead of queueing
+        //              behind S(b+1), which waits for its K/V tile (whose load
+        //              in turn waits for PV(b-1) to free the stage).
+        const int w = TILES == 1 ? 0 : warp - 1;
+        const bool issue_s_side = TILES == 2 || warp == 1;
+        const bool issue_pv_side = TILES == 2 || warp == 2;
         if (lane == 0 && !aborted_at_start) {
             const uint32_t tS = tmem + w * 256, tP = tS + 128, tO = tS + 192;
             auto live = [&](const AtItem &it) { return SPLIT || it.i0 + w * AT_BM < a.nq; };
@@ -439,51 +449,63 @@ __global__ void __launch_bounds__(AtCfg<TILES>::THREADS, AtCfg<TILES>::CTAS)
                                  a.wait, abort_flag) &&
                        mbar_wait(&q_full[c.r & 1], (c.r >> 1) & 1, a.wait, abort_flag);
             };
-            BlockCursor<NS, SPLIT, FA, TILES> cur;
-            cur.init(a, n_pairs, n_items, w);
-            bool run = cur.valid() && ready_s(cur);
-            if (run) {
-                tc_fence_after();
-                issue_s(cur);
-            }
-            while (run) {
-                BlockCursor<NS, SPLIT, FA, TILES> nxt = cur;
-                nxt.next(a, n_pairs, n_items);
-                if (nxt.valid()) {
-                    if (!mbar_wait(&s_free[w], static_cast<uint32_t>(cur.lb & 1), a.wait, abort_flag) ||
-                        !ready_s(nxt))
-                        break;
-                    tc_fence_after();
-                    issue_s(nxt);
-                }
-                if (!mbar_wait(&p_full[w], static_cast<uint32_t>(cur.lb & 1), a.wait, abort_flag)) break;
+            // O += P(b) V once P(b) is stored; false if a wait gave up
+            auto issue_pv = [&](const BlockCursor<NS, SPLIT, FA, TILES> &c) {
+                if (!mbar_wait(&p_full[w], static_cast<uint32_t>(c.lb & 1), a.wait, abort_flag)) return false;
                 tc_fence_after();
                 // the first PV of an item overwrites O: the previous item's
                 // output has been read out by then (the warpgroup did that
                 // before computing P of this block; in split-key mode tile 0
                 // reads both tiles' O)
-                const bool first = cur.first_in_item();
-                if (first && cur.r > 0) {
-                    if (!mbar_wait(&o_free[w], (cur.r - 1) & 1, a.wait, abort_flag)) break;
+                const bool first = c.first_in_item();
+                if (first && c.r > 0) {
+                    if (!mbar_wait(&o_free[w], (c.r - 1) & 1, a.wait, abort_flag)) return false;
                     tc_fence_after();
                 }
-                if (live(cur.it)) {
-                    const uint32_t v_addr = smem_u32(sKV + (2 * (cur.gb % AT_STAGES) + 1) * AT_TILE);
+                if (live(c.it)) {
+                    const uint32_t v_addr = smem_u32(sKV + (2 * (c.gb % AT_STAGES) + 1) * AT_TILE);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) // P from TMEM: 8 columns per 16 keys
                         mma_f16_ts(tO, tP + kk * 8, sw128_desc(v_addr + kk * 2048, AT_TILE), IDESC_O,
                                    !first || kk != 0);
                 }
                 mma_commit(&o_full[w]);
-                // both arrivals the stage waits for: split-key stages have one reader
-                mma_commit(&kv_empty[cur.gb % AT_STAGES]);
-                if (SPLIT) mma_commit(&kv_empty[cur.gb % AT_STAGES]);
-                if (!nxt.valid()) break;
-                cur = nxt;
+                // the arrivals the stage waits for (its S MMAs completed before
+                // P(b) existed): split-key stages have one reader
+                mma_commit(&kv_empty[c.gb % AT_STAGES]);
+                if (SPLIT) mma_commit(&kv_empty[c.gb % AT_STAGES]);
+                return true;
+            };
+            BlockCursor<NS, SPLIT, FA, TILES> cur;
+            cur.init(a, n_pairs, n_items, w);
+            if (issue_s_side) {
+                bool run = cur.valid() && ready_s(cur);
+                if (run) {
+                    tc_fence_after();
+                    issue_s(cur);
+                }
+                while (run) {
+                    BlockCursor<NS, SPLIT, FA, TILES> nxt = cur;
+                    nxt.next(a, n_pairs, n_items);
+                    if (nxt.valid()) {
+                        if (!mbar_wait(&s_free[w], static_cast<uint32_t>(cur.lb & 1), a.wait, abort_flag) ||
+                            !ready_s(nxt))
+                            break;
+                        tc_fence_after();
+                        issue_s(nxt);
+                    }
+                    if (issue_pv_side && !issue_pv(cur)) break;
+                    if (!nxt.valid()) break;
+                    cur = nxt;
+                }
+            } else {
+                for (; cur.valid(); cur.next(a, n_pairs, n_items))
+                    if (!issue_pv(cur)) break;
             }
             // every issued MMA must be complete before TMEM is released
-            mma_commit(&mma_done[w]);
-            mbar_wait(&mma_done[w], 0, final_wait, &no_abort);
+            uint64_t *done = &mma_done[TILES == 1 ? warp - 1 : w];
+            mma_commit(done);
+            mbar_wait(done, 0, final_wait, &no_abort);
         }
     } else if (warp >= 4) {
         // ------------------------------------------------ softmax warpgroups
