@@ -41,9 +41,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 CAPTURED_TRAFFIC = {
     # kernel kind -> (source file, its sha256 at capture time, bytes per step, launches per step)
     # attn_tc: ncu dram__bytes_read.sum + dram__bytes_write.sum of the six S-attention launches
-    # of one onetrans_s_full step (653.5 MB read + 35.3 MB written)
-    "attn_tc": ("ot_attn_tc.cu", "f7f088a65ddb4a12fb1aa96b20d829ba13650d3158db9ec3244588d6f2002d6d",
-                688931328, 6),
+    # of one onetrans_s_full step (651.1 MB read + 34.4 MB written)
+    "attn_tc": ("ot_attn_tc.cu", "4e9ab25b647c2a37ce94733adfd370f3024a6f8845cc1d9215fbd9a7504b1ec8",
+                685544192, 6),
     # ffn_tc: the six fused O-projection + FFN launches of one onetrans_s_full step
     # (363.4 MB read + 20.6 MB written)
     "ffn_tc": ("ot_ffn_tc.cu", "675fae658dab54517d2954da43f31073cedb641fd3c4be7f406e1fea356bc07d",

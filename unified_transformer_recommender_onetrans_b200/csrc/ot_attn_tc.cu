@@ -31,9 +31,9 @@
 //               goes into the S columns, overlapping the exponentials; once
 //               P(b) is stored, O += P(b) V (8 MMAs, P from TMEM, V MN-major
 //               from its row-major tile).  A tile with no live query row gets
-//               no MMAs, only the signals.  With one tile per CTA (two
-//               CTAs per SM, see AtCfg) warp 1 issues the S MMAs and warp 2
-//               the PV MMAs.
+//               no MMAs, only the signals.  In S mode (one tile per CTA,
+//               two CTAs per SM, see AtCfg) warp 1 issues the S MMAs and
+//               warp 2 the PV MMAs.
 //   warp 3      idle (it completes the producer warpgroup, whose registers
 //               go to the softmax warpgroups through setmaxnreg).
 //   warps 4-7   softmax warpgroup of tile 0, warps 8-11 of tile 1: one query
@@ -285,6 +285,8 @@ __global__ void __launch_bounds__(AtCfg<TILES>::THREADS, AtCfg<TILES>::CTAS)
 
     extern __shared__ __align__(1024) uint8_t smem[];
     constexpr int AT_TILES = TILES, AT_STAGES = AtCfg<TILES>::STAGES;
+    // S mode: separate S and PV issuing warps (see the MMA issuers below)
+    constexpr bool TWO_ISSUERS = TILES == 1 && !NS;
     uint8_t *sQ = smem;                                  // [AT_QBUF][AT_TILES]
     uint8_t *sKV = smem + AT_QBUF * AT_TILES * AT_TILE;  // [stage][K | V]
     uint64_t *bars = reinterpret_cast<uint64_t *>(sKV + 2 * AT_STAGES * AT_TILE);
@@ -413,21 +415,23 @@ __global__ void __launch_bounds__(AtCfg<TILES>::THREADS, AtCfg<TILES>::CTAS)
                 mbar_wait(&kv_full[j % AT_STAGES], static_cast<uint32_t>((j / AT_STAGES) & 1),
                           final_wait, &no_abort);
         }
-    } else if (warp >= 1 && warp <= (TILES == 1 ? 2 : AT_TILES)) {
+    } else if (warp >= 1 && warp <= (TWO_ISSUERS ? 2 : AT_TILES)) {
         // ------------------------------------------------ MMA issuers
         // Issued from one thread, a short tcgen05.mma takes about 100 cycles.
         // Per key block: once the softmax has S(b) in registers (s_free),
         // S(b+1) = Q K^T goes into the S columns, so it runs while P(b) is
         // being computed; once P(b) is stored (p_full), O += P(b) V.
-        //   TILES = 2: warp 1 + w issues both for tile w (one issuer per tile
+        //   in general warp 1 + w issues both for tile w (one issuer per tile
         //              keeps both tiles' MMAs flowing);
-        //   TILES = 1: warp 1 issues the S MMAs, warp 2 the PV MMAs, so PV(b)
-        //              goes out as soon as P(b) is stored instead of queueing
-        //              behind S(b+1), which waits for its K/V tile (whose load
-        //              in turn waits for PV(b-1) to free the stage).
-        const int w = TILES == 1 ? 0 : warp - 1;
-        const bool issue_s_side = TILES == 2 || warp == 1;
-        const bool issue_pv_side = TILES == 2 || warp == 2;
+        //   S mode (one tile per CTA): warp 1 issues the S MMAs, warp 2 the PV
+        //              MMAs, so PV(b) goes out as soon as P(b) is stored
+        //              instead of queueing behind S(b+1), which waits for its
+        //              K/V tile (whose load in turn waits for PV(b-1) to free
+        //              the stage).  NS items measured slower that way (their
+        //              K/V tiles mostly come from L2), so they keep one issuer.
+        const int w = TWO_ISSUERS ? 0 : warp - 1;
+        const bool issue_s_side = !TWO_ISSUERS || warp == 1;
+        const bool issue_pv_side = !TWO_ISSUERS || warp == 2;
         if (lane == 0 && !aborted_at_start) {
             const uint32_t tS = tmem + w * 256, tP = tS + 128, tO = tS + 192;
             auto live = [&](const AtItem &it) { return SPLIT || it.i0 + w * AT_BM < a.nq; };
@@ -503,7 +507,7 @@ __global__ void __launch_bounds__(AtCfg<TILES>::THREADS, AtCfg<TILES>::CTAS)
                     if (!issue_pv(cur)) break;
             }
             // every issued MMA must be complete before TMEM is released
-            uint64_t *done = &mma_done[TILES == 1 ? warp - 1 : w];
+            uint64_t *done = &mma_done[TWO_ISSUERS ? warp - 1 : w];
             mma_commit(done);
             mbar_wait(done, 0, final_wait, &no_abort);
         }
