@@ -606,7 +606,8 @@ def forward_flops(wl, q, U, C):
         pairs_ns = N * L + N * (N + 1) // 2
         a = 4.0 * d * U * pairs_s + 4.0 * d * U * C * pairs_ns
         attn += a
-        total += a + 2.0 * U * L * 3 * d * d + 2.0 * U * ql * d * d + 4.0 * U * ql * d * f
+        # S side: K and V of all L rows, Q, O and the FFN of the ql tail rows
+        total += a + 2.0 * U * (2 * L + ql) * d * d + 2.0 * U * ql * d * d + 4.0 * U * ql * d * f
         total += 2.0 * RN * 3 * d * d + 2.0 * RN * d * d + 4.0 * RN * d * f
         L = ql
     return total, attn
