@@ -69,8 +69,12 @@ __global__ void moe_topk_kernel(const float *logits, int T, int E, int k, int *s
     const int lane = threadIdx.x & 31;
     for (long long r = mb_warp_id(); r < T; r += mb_warps()) {
         const float *lg = logits + r * E;
-        // lane holds experts lane and lane + 32
+        // lane holds experts lane and lane + 32; a NaN logit counts as -inf,
+        // so every comparison below is ordered and the chosen indices stay
+        // below E (an unordered one could leave the out-of-range marker)
         float v0 = lane < E ? lg[lane] : -INFINITY, v1 = lane + 32 < E ? lg[lane + 32] : -INFINITY;
+        if (v0 != v0) v0 = -INFINITY;
+        if (v1 != v1) v1 = -INFINITY;
         float bv = v0;
         int be = lane < E ? lane : 1 << 20;
         mb_better(bv, be, v1, lane + 32 < E ? lane + 32 : 1 << 20);
