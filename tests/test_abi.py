@@ -165,3 +165,35 @@ def test_backward_launch_count(lib):
         assert lib.ot_backward_launches(C.byref(c), 2, 3) == 16 * layers + 12 * (layers - 1) + 35 * layers
         assert lib.ot_backward_launches(C.byref(c), 2, 0) == 8 * layers + 6 * (layers - 1) + 18 * layers
     assert lib.ot_backward_launches(C.byref(_cfg(**dict(f32, dtype=1, layers=1, q=[40]))), 2, 3) == 0
+
+
+def test_backward_binding_checks_tensor_shapes_on_host():
+    """full_backward refuses tensors that do not match an accepted
+    configuration before anything reaches the device (CPU tensors here: the
+    shape check comes first; a matching set then fails only on the device
+    check).  An invalid configuration is left to the library's status."""
+    import torch
+    import unified_transformer_recommender_onetrans_b200 as ot
+
+    L, d, H, f, N, L0, U, C = 1, 64, 2, 96, 3, 40, 2, 2
+    q = [9]
+    cfg = ot.make_config(layers=L, d=d, heads=H, ffn=f, n_ns=N, L0=L0, q=q)
+    shapes = {"Wqkv_s": (L, 3 * d, d), "Wo_s": (L, d, d), "W1_s": (L, f, d), "W2_s": (L, d, f),
+              "g1_s": (L, d), "g2_s": (L, d), "Wqkv_ns": (L, N, 3 * d, d), "Wo_ns": (L, N, d, d),
+              "W1_ns": (L, N, f, d), "W2_ns": (L, N, d, f), "g1_ns": (L, N, d), "g2_ns": (L, N, d)}
+    w = {k: torch.zeros(s) for k, s in shapes.items()}
+    S, ns = torch.zeros(U, L0, d), torch.zeros(U, C, N, d)
+    G_s, G_ns = torch.zeros(U, q[-1], d), torch.zeros(U, C, N, d)
+    with pytest.raises(ValueError, match="CUDA"):  # every shape right: the device check
+        ot.full_backward(cfg, w, S, ns, G_s, G_ns)
+    with pytest.raises(ValueError, match="shape"):
+        ot.full_backward(cfg, w, torch.zeros(U, L0 + 1, d), ns, G_s, G_ns)
+    with pytest.raises(ValueError, match="G_s must have shape"):
+        ot.full_backward(cfg, w, S, ns, torch.zeros(U, L0, d), G_ns)
+    bad_w = dict(w, W1_ns=torch.zeros(L, N, d, f))  # transposed
+    with pytest.raises(ValueError, match="W1_ns"):
+        ot.full_backward(cfg, bad_w, S, ns, G_s, G_ns)
+    with pytest.raises(ValueError, match="float32"):
+        ot.full_backward(cfg, w, S.double(), ns, G_s, G_ns)
+    with pytest.raises(ValueError, match="grads"):
+        ot.full_backward(cfg, w, S, ns, G_s, G_ns, grads={"Wo_s": torch.zeros(L, d, d + 1)})

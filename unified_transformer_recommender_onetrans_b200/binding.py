@@ -487,6 +487,32 @@ def backward_launches(cfg: OtConfig, users: int, cands: int) -> int:
     return lib().ot_backward_launches(C.byref(cfg), users, cands)
 
 
+def _expect(t, shape, name):
+    """A tensor handed to ot_full_backward: None, or fp32 of exactly this shape."""
+    import torch
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    if t.dtype != torch.float32:
+        raise ValueError(f"{name} must be float32, not {t.dtype}")
+
+
+def _backward_shapes(cfg: OtConfig, U: int, Cn: int) -> dict:
+    """Shapes of every tensor of ot_full_backward (include/onetrans.h layouts)."""
+    L, d, f, N, E = cfg.layers, cfg.d, cfg.ffn, cfg.n_ns, cfg.moe_experts
+    q_last = cfg.q[L - 1]
+    return {
+        "Wqkv_s": (L, 3 * d, d), "Wo_s": (L, d, d), "W1_s": (L, f, d), "W2_s": (L, d, f),
+        "g1_s": (L, d), "g2_s": (L, d),
+        "Wqkv_ns": (L, N, 3 * d, d), "Wo_ns": (L, N, d, d), "W1_ns": (L, N, f, d),
+        "W2_ns": (L, N, d, f), "g1_ns": (L, N, d), "g2_ns": (L, N, d),
+        "W_router": (L, E, d), "W1_moe": (L, E, f, d), "W2_moe": (L, E, d, f),
+        "S": (U, cfg.L0, d), "dS": (U, cfg.L0, d), "ns": (U, Cn, N, d), "dns": (U, Cn, N, d),
+        "G_ns": (U, Cn, N, d), "out_ns": (U, Cn, N, d), "G_s": (U, q_last, d), "out_s_tail": (U, q_last, d),
+    }
+
+
 def full_backward(cfg: OtConfig, weights: dict, S, ns, G_s, G_ns, *, grads=None, dS=None,
                   dns=None, out_s_tail=None, out_ns=None, ws=None, want_outputs=True,
                   want_input_grads=True, stream=None):
@@ -499,6 +525,18 @@ def full_backward(cfg: OtConfig, weights: dict, S, ns, G_s, G_ns, *, grads=None,
     U, Cn = S.shape[0], (ns.shape[1] if ns is not None else 0)
     dev = S.device
     present = [k for k in GRAD_NAMES + MOE_WEIGHT_NAMES if weights.get(k) is not None]
+    nbytes = backward_workspace_bytes(cfg, U, Cn)
+    if nbytes > 0:
+        # a configuration the library accepts (else its own status is
+        # reported below): every tensor given must have its shape and fp32
+        shapes = _backward_shapes(cfg, U, Cn)
+        for k in present:
+            _expect(weights[k], shapes[k], k)
+            if grads is not None:
+                _expect(grads.get(k), shapes[k], f"grads[{k}]")
+        for name, t in (("S", S), ("ns", ns), ("G_s", G_s), ("G_ns", G_ns), ("out_s_tail", out_s_tail),
+                        ("out_ns", out_ns), ("dS", dS), ("dns", dns)):
+            _expect(t, shapes[name], name)
     if grads is None:
         grads = {k: torch.empty_like(weights[k]) for k in present}
     if want_outputs:
@@ -511,7 +549,6 @@ def full_backward(cfg: OtConfig, weights: dict, S, ns, G_s, G_ns, *, grads=None,
             dS = torch.empty_like(S)
         if dns is None and Cn:
             dns = torch.empty_like(ns)
-    nbytes = backward_workspace_bytes(cfg, U, Cn)
     if ws is None:
         ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
     w = OtWeights(**{k: _ptr(weights.get(k)) for k in GRAD_NAMES + MOE_WEIGHT_NAMES})
