@@ -395,9 +395,10 @@ int ot_profile_read(ot_model *m, ot_launch_record *out, int max);
  *     loss = sum(s_tail * G_s) + sum(ns_out * G_ns)
  * (s_tail, ns_out: the outputs of ot_full_forward; G_s, G_ns: the upstream
  * gradients) with respect to every weight and gain and to S and ns.
- * Activation checkpointing: a forward pass keeps only each layer's input
- * rows; the backward then recomputes one layer at a time from them, top
- * layer first, and takes its gradients.  CUDA-core fp32 kernels.
+ * Activation checkpointing: a forward pass keeps each layer's input rows
+ * and its attention outputs with their softmax statistics (row max and sum);
+ * the backward then recomputes the rest of one layer at a time from them,
+ * top layer first, and takes its gradients.  CUDA-core fp32 kernels.
  * All pointers are device pointers to fp32, 16-byte aligned:
  *   w      the tensors of ot_weights, fp32, gains NOT folded: Wqkv_s ..
  *          g2_ns, and with E > 0 W_router, W1_moe, W2_moe (then W1_s / W2_s
