@@ -14,7 +14,9 @@
   and per-tensor scales) against the brute force, exact results on
   representable operands, a hand-worked row, the scale granularity and the
   calibration amax;
-* Auto-Split and embedding gather against numpy.
+* Auto-Split and embedding gather against numpy;
+* the brute force again on random tiny shapes (hypothesis, derandomized):
+  causal, full attention and the mixture of experts.
 """
 
 from __future__ import annotations
@@ -903,3 +905,97 @@ def test_backward_oracle_moe_matches_finite_differences(topk, monkeypatch):
         fd = loss(*with_(p_plus)) - loss(*with_(p_minus))
         an = 2.0 * float((grads[name] * step).sum())
         assert abs(fd - an) <= 2e-5 * max(1.0, abs(an)) + 1e-9, (name, fd, an)
+
+
+# ------------------------------------------------------------- random small shapes
+try:
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+except ImportError:  # pragma: no cover - hypothesis is in the image
+    given = None
+
+
+if given is not None:
+    @st.composite
+    def _tiny_stack(draw):
+        """A random tiny configuration: any layer count, width, head split,
+        FFN width, NS count, sequence length, monotone pyramid, users and
+        candidates the brute force finishes in milliseconds."""
+        layers = draw(st.integers(1, 3))
+        H = draw(st.sampled_from([1, 2]))
+        d = H * draw(st.sampled_from([2, 4, 6]))
+        f = draw(st.integers(1, 3)) * 4
+        N = draw(st.integers(1, 3))
+        L0 = draw(st.integers(1, 12))
+        q, prev = [], L0
+        for _ in range(layers):
+            prev = draw(st.integers(1, prev))
+            q.append(prev)
+        U = draw(st.integers(1, 2))
+        C = draw(st.integers(1, 2))
+        seed = draw(st.integers(0, 10_000))
+        return layers, d, H, f, N, L0, q, U, C, seed
+
+    @settings(max_examples=25, deadline=None, derandomize=True)
+    @given(_tiny_stack())
+    def test_brute_force_matches_oracle_random_shapes(case):
+        """The C oracle's split (encode + score) and joint forms against the
+        token-by-token brute force on random tiny shapes (one-row tails,
+        one-token sequences, heads of width 1 to 6, pyramids that keep or cut
+        every row)."""
+        layers, d, H, f, N, L0, q, U, Cn, seed = case
+        w = rand_weights(layers, d, f, N, seed=seed)
+        S, ns = rand_inputs(U, Cn, L0, N, d, seed=seed + 1)
+        cfg = cfg_of(layers, d, H, f, N, L0, q)
+        kv, s_out = O.encode_user(cfg, w, S)
+        ns_out = O.score_candidates(cfg, w, kv, ns)
+        js, _, jns = O.full_forward_joint(cfg, w, S, ns)
+        wl = to_lists(w)
+        for u in range(U):
+            for c in range(Cn):
+                bs, bns, _ = run_candidate(wl, S[u].double().tolist(), ns[u, c].double().tolist(),
+                                           q, H, 1e-6)
+                np.testing.assert_allclose(s_out[u], np.array(bs), rtol=0, atol=1e-12)
+                np.testing.assert_allclose(js[u, c], np.array(bs), rtol=0, atol=1e-12)
+                np.testing.assert_allclose(ns_out[u, c], np.array(bns), rtol=0, atol=1e-12)
+                np.testing.assert_allclose(jns[u, c], np.array(bns), rtol=0, atol=1e-12)
+
+    @settings(max_examples=15, deadline=None, derandomize=True)
+    @given(_tiny_stack())
+    def test_brute_force_matches_oracle_random_shapes_full_attention(case):
+        """Full attention (joint form) against the brute force's every-key
+        visibility on random tiny shapes."""
+        layers, d, H, f, N, L0, q, U, Cn, seed = case
+        w = rand_weights(layers, d, f, N, seed=seed + 2)
+        S, ns = rand_inputs(U, Cn, L0, N, d, seed=seed + 3)
+        cfg = cfg_of(layers, d, H, f, N, L0, q)
+        cfg.full_attn = True
+        js, _, jns = O.full_forward_joint(cfg, w, S, ns)
+        wl = to_lists(w)
+        for u in range(U):
+            for c in range(Cn):
+                bs, bns, _ = run_candidate(wl, S[u].double().tolist(), ns[u, c].double().tolist(),
+                                           q, H, 1e-6, full=True)
+                np.testing.assert_allclose(js[u, c], np.array(bs), rtol=0, atol=1e-12)
+                np.testing.assert_allclose(jns[u, c], np.array(bns), rtol=0, atol=1e-12)
+
+    @settings(max_examples=15, deadline=None, derandomize=True)
+    @given(_tiny_stack(), st.integers(1, 5), st.integers(1, 2))
+    def test_brute_force_matches_oracle_random_shapes_moe(case, experts, topk):
+        """The sparse-MoE S-side FFN against the brute force on random tiny
+        shapes, expert counts and top-k (k <= E)."""
+        layers, d, H, f, N, L0, q, U, Cn, seed = case
+        topk = min(topk, experts)
+        w = rand_weights(layers, d, f, N, seed=seed + 4, experts=experts)
+        S, ns = rand_inputs(U, Cn, L0, N, d, seed=seed + 5)
+        cfg = cfg_of(layers, d, H, f, N, L0, q)
+        cfg.moe_experts, cfg.moe_topk = experts, topk
+        kv, s_out = O.encode_user(cfg, w, S)
+        ns_out = O.score_candidates(cfg, w, kv, ns)
+        wl = to_lists(w)
+        for u in range(U):
+            for c in range(Cn):
+                bs, bns, _ = run_candidate(wl, S[u].double().tolist(), ns[u, c].double().tolist(),
+                                           q, H, 1e-6, moe_topk=topk)
+                np.testing.assert_allclose(s_out[u], np.array(bs), rtol=0, atol=1e-12)
+                np.testing.assert_allclose(ns_out[u, c], np.array(bns), rtol=0, atol=1e-12)
