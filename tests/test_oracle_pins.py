@@ -999,3 +999,48 @@ if given is not None:
                                            q, H, 1e-6, moe_topk=topk)
                 np.testing.assert_allclose(s_out[u], np.array(bs), rtol=0, atol=1e-12)
                 np.testing.assert_allclose(ns_out[u, c], np.array(bns), rtol=0, atol=1e-12)
+
+    @settings(max_examples=6, deadline=None, derandomize=True)
+    @given(_tiny_stack())
+    def test_backward_oracle_random_shapes(case):
+        """The gradient oracle on random tiny shapes: its forward equals the C
+        oracle's, and every gradient along a random direction equals the
+        central difference of the C oracle's loss (as the fixed-shape pin)."""
+        from oracle import backward as OB
+        layers, d, H, f, N, L0, q, U, Cn, seed = case
+        w = rand_weights(layers, d, f, N, seed=seed + 6, dtype=torch.float64)
+        w = {k: v.float().double() for k, v in w.items()}
+        S, ns = rand_inputs(U, Cn, L0, N, d, seed=seed + 7, dtype=torch.float64)
+        S, ns = S.float().double(), ns.float().double()
+        g = torch.Generator().manual_seed(seed + 8)
+        G_s = torch.randn(U, q[-1], d, generator=g, dtype=torch.float64)
+        G_ns = torch.randn(U, Cn, N, d, generator=g, dtype=torch.float64)
+        cfg = cfg_of(layers, d, H, f, N, L0, q)
+        s_t, ns_t = OB.forward(cfg, w, S, ns)
+        kv, s_c = O.encode_user(cfg, w, S)
+        ns_c = O.score_candidates(cfg, w, kv, ns)
+        np.testing.assert_allclose(s_t.detach().numpy(), s_c, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(ns_t.detach().numpy(), ns_c, rtol=0, atol=1e-12)
+        _, grads = OB.gradients(cfg, w, S, ns, G_s, G_ns)
+
+        def loss(w_, S_, ns_):
+            kv_, s_ = O.encode_user(cfg, w_, S_.float())
+            return float((s_ * G_s.numpy()).sum() +
+                         (O.score_candidates(cfg, w_, kv_, ns_) * G_ns.numpy()).sum())
+
+        eps = 1e-3
+        for name in ["S", "ns"] + list(OB.W_NAMES):
+            base = {"S": S, "ns": ns}.get(name, w.get(name))
+            v = torch.randn(base.shape, generator=g, dtype=torch.float64)
+            p_plus, p_minus = (base + eps * v).float().double(), (base - eps * v).float().double()
+            step = (p_plus - p_minus).double() / 2
+
+            def with_(p):
+                if name == "S":
+                    return w, p, ns
+                if name == "ns":
+                    return w, S, p
+                return dict(w, **{name: p}), S, ns
+            fd = loss(*with_(p_plus)) - loss(*with_(p_minus))
+            an = 2.0 * float((grads[name] * step).sum())
+            assert abs(fd - an) <= 2e-5 * max(1.0, abs(an)), (name, fd, an)
