@@ -16,7 +16,8 @@
   calibration amax;
 * Auto-Split and embedding gather against numpy;
 * the brute force again on random tiny shapes (hypothesis, derandomized):
-  causal, full attention and the mixture of experts.
+  causal, full attention, the mixture of experts and both FP8 rules, and
+  the gradient oracle against finite differences.
 """
 
 from __future__ import annotations
@@ -1044,3 +1045,29 @@ if given is not None:
             fd = loss(*with_(p_plus)) - loss(*with_(p_minus))
             an = 2.0 * float((grads[name] * step).sum())
             assert abs(fd - an) <= 2e-5 * max(1.0, abs(an)), (name, fd, an)
+
+    @settings(max_examples=12, deadline=None, derandomize=True)
+    @given(_tiny_stack(), st.sampled_from([O.FP8_ROW, O.FP8_TENSOR]))
+    def test_brute_force_matches_oracle_random_shapes_fp8(case, rule):
+        """Both FP8 rules against the brute force (torch's e4m3 cast) on
+        random tiny shapes: outputs and the calibration maxima."""
+        from brute_force import Fp8
+        layers, d, H, f, N, L0, q, U, Cn, seed = case
+        w = rand_weights(layers, d, f, N, seed=seed + 9)
+        S, ns = rand_inputs(U, Cn, L0, N, d, seed=seed + 10)
+        cfg = cfg_of(layers, d, H, f, N, L0, q, fp8=rule)
+        if rule == O.FP8_TENSOR:
+            cfg.act_scale = _fp8_scales(cfg, seed=seed)
+        amax = np.zeros(cfg.scale_shape())
+        kv, s_out = O.encode_user(cfg, w, S, amax=amax)
+        ns_out = O.score_candidates(cfg, w, kv, ns, amax=amax)
+        wl = to_lists(w)
+        bam = np.zeros(cfg.scale_shape()).tolist()
+        fp8 = Fp8(rule, None if cfg.act_scale is None else cfg.act_scale.tolist(), bam)
+        for u in range(U):
+            for c in range(Cn):
+                bs, bns, _ = run_candidate(wl, S[u].double().tolist(), ns[u, c].double().tolist(),
+                                           q, H, 1e-6, fp8=fp8)
+                np.testing.assert_allclose(s_out[u], np.array(bs), rtol=0, atol=1e-12)
+                np.testing.assert_allclose(ns_out[u, c], np.array(bns), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(amax, np.array(bam), rtol=0, atol=1e-12)
