@@ -16,8 +16,8 @@
   calibration amax;
 * Auto-Split and embedding gather against numpy;
 * the brute force again on random tiny shapes (hypothesis, derandomized):
-  causal, full attention, the mixture of experts and both FP8 rules, and
-  the gradient oracle against finite differences.
+  causal, full attention, the mixture of experts, both FP8 rules and the
+  sequence append, and the gradient oracle against finite differences.
 """
 
 from __future__ import annotations
@@ -1071,3 +1071,24 @@ if given is not None:
                 np.testing.assert_allclose(s_out[u], np.array(bs), rtol=0, atol=1e-12)
                 np.testing.assert_allclose(ns_out[u, c], np.array(bns), rtol=0, atol=1e-12)
         np.testing.assert_allclose(amax, np.array(bam), rtol=0, atol=1e-12)
+
+    @settings(max_examples=12, deadline=None, derandomize=True)
+    @given(_tiny_stack(), st.integers(1, 4))
+    def test_append_equals_reencode_random_shapes(case, delta):
+        """Appending delta rows to an encoded cache equals encoding the grown
+        sequence (cache and the new rows' outputs), and the new rows' outputs
+        equal the brute force's, on random tiny shapes."""
+        layers, d, H, f, N, L0, q, U, _, seed = case
+        w = rand_weights(layers, d, f, N, seed=seed + 11)
+        S_all, _ = rand_inputs(U, 1, L0 + delta, N, d, seed=seed + 12)
+        cfg0 = cfg_of(layers, d, H, f, N, L0, q)
+        kv0, _ = O.encode_user(cfg0, w, S_all[:, :L0])
+        cfg1 = cfg0.grown(delta)
+        kv1, new1 = O.encode_append(cfg1, w, kv0, S_all[:, L0:])
+        kvf, sf = O.encode_user(cfg1, w, S_all)
+        np.testing.assert_allclose(kv1, kvf, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(new1, sf[:, -delta:], rtol=0, atol=1e-12)
+        wl = to_lists(w)
+        for u in range(U):
+            bs, _, _ = run_candidate(wl, S_all[u].double().tolist(), [[0.0] * d] * N, cfg1.q, H, 1e-6)
+            np.testing.assert_allclose(new1[u], np.array(bs)[-delta:], rtol=0, atol=1e-12)
