@@ -17,7 +17,8 @@
 * Auto-Split and embedding gather against numpy;
 * the brute force again on random tiny shapes (hypothesis, derandomized):
   causal, full attention, the mixture of experts, both FP8 rules and the
-  sequence append, and the gradient oracle against finite differences.
+  sequence append; the textbook reduction on random shapes; and the
+  gradient oracle against finite differences.
 """
 
 from __future__ import annotations
@@ -1092,3 +1093,30 @@ if given is not None:
         for u in range(U):
             bs, _, _ = run_candidate(wl, S_all[u].double().tolist(), [[0.0] * d] * N, cfg1.q, H, 1e-6)
             np.testing.assert_allclose(new1[u], np.array(bs)[-delta:], rtol=0, atol=1e-12)
+
+    @settings(max_examples=16, deadline=None, derandomize=True)
+    @given(_tiny_stack(), st.booleans())
+    def test_textbook_reduction_random_shapes(case, full):
+        """With every NS parameter set equal to the S set, each block is a
+        pre-norm Transformer layer over [S; NS] from torch's library routines
+        (causal, or bidirectional for full attention), on random tiny shapes."""
+        layers, d, H, f, N, L0, q, _, Cn, seed = case
+        w = rand_weights(layers, d, f, N, seed=seed + 13, dtype=torch.float64)
+        for name in ("Wqkv", "Wo", "W1", "W2", "g1", "g2"):
+            w[name + "_ns"] = w[name + "_s"][:, None].expand(-1, N, *w[name + "_s"].shape[1:]).clone()
+        S, ns = rand_inputs(1, Cn, L0, N, d, seed=seed + 14, dtype=torch.float64)
+        w = {k: v.float().double() for k, v in w.items()}
+        S, ns = S.float().double(), ns.float().double()
+        cfg = cfg_of(layers, d, H, f, N, L0, q)
+        cfg.full_attn = full
+        js, _, jns = O.full_forward_joint(cfg, w, S, ns)
+        for c in range(Cn):
+            x = torch.cat([S[0], ns[0, c]])
+            L = L0
+            for l in range(layers):
+                y = _torch_causal_layer(x, w["Wqkv_s"][l], w["Wo_s"][l], w["W1_s"][l], w["W2_s"][l],
+                                        w["g1_s"][l], w["g2_s"][l], H, 1e-6, causal=not full)
+                x = torch.cat([y[L - q[l]:L], y[L:]])
+                L = q[l]
+            np.testing.assert_allclose(js[0, c], x[:L].numpy(), rtol=0, atol=1e-11)
+            np.testing.assert_allclose(jns[0, c], x[L:].numpy(), rtol=0, atol=1e-11)
