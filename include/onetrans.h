@@ -42,8 +42,9 @@
  * no TF32); OT_DTYPE_BF16 = bfloat16 activations, weights, cache (fp32
  * accumulation on tcgen05 tensor cores); OT_DTYPE_FP8 = bfloat16 storage with
  * every QKV / O / FFN projection run on e4m3 operands, attention and cache in
- * bf16.  FP8 rule (the V2 podcast page names "kernel fusion + FP8" without a
- * recipe; e4m3 with per-tensor fp32 scales is the library's reading): every
+ * bf16.  FP8 rule (the V2 podcast page credits kernel fusion and FP8 with
+ * its speed but gives no recipe; e4m3 with per-tensor fp32 scales is the
+ * library's reading): every
  * projection input tensor -- the input of one layer's QKV, O, W1 or W2
  * projection for one parameter set (S, or NS position n), after its RMSNorm
  * and gain where the block has one -- has one fixed fp32 scale s, set with
