@@ -43,7 +43,7 @@
  * Storage: every input is passed as float32, which holds the bf16 / fp32
  * values of the runs exactly; all arithmetic is fp64 (double).
  *
- * FP8 modes (the V2 podcast page names "kernel fusion + FP8" and nothing
+ * FP8 modes (the V2 podcast page credits kernel fusion and FP8 and says no
  * more; the workload fixes e4m3 with per-tensor fp32 scales):
  *   fp8 = 2 (per-tensor): every projection input tensor -- the input of the
  *     QKV, O, W1 or W2 projection of one layer and one parameter set (S, or
